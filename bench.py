@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""AQLM matmul throughput on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one pass of the AQLM linear layers of a workload over one batch of
+synthetic activations.  The default workload is the Llama-2-7B decoder layer
+set (q, k, v, o 4096x4096; gate, up 11008x4096; down 4096x11008), 2x8 g8
+codebooks (2 bits per weight), batch 1.
+
+Metric: effective HBM GB/s = algorithmic bytes (codes + codebooks + scales + x +
+y, each once) / device time, summed over ranks; microseconds per layer are
+reported beside it.  Inputs are resident in HBM; every step reads a different
+copy of the layer set from a rotating pool larger than 3x the L2 cache, so no
+step finds its weights in L2.  Each step is one CUDA graph replay (its seven
+kernel launches); the timed region is bracketed by a barrier and a device
+synchronise and measured with CUDA events on the launching stream; the max over
+ranks is taken.  With N > 1 GPUs each rank runs its own replica (weak scaling,
+no data-path collective).
+
+--impl reference times the CPU oracle (decode to fp16, fp64 matmul) on the
+host cores on a bounded sample of rows of every layer per step and reports the
+same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from weight_only_additive_b200 import synth, workloads  # noqa: E402
+
+METRIC = "AQLM matmul µs/layer & achieved HBM GB/s (frac. of ~8 TB/s), batch 1–256"
+DEFAULT_WORKLOAD = "llama2_7b_layer_set_2x8g8"
+L2_FALLBACK = 126 * 1024 * 1024
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100000)
+    p.add_argument("--warmup", type=int, default=1000)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.BY_NAME))
+    p.add_argument("--batch", type=int, default=None, help="override the workload's batch size")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be at least 3")
+    return a
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def workload_batch(w, override):
+    return override if override is not None else w.batches[0]
+
+
+def step_bytes(w, batch):
+    return sum(l.algorithmic_bytes(batch) for l in w.layers)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, enabled: bool = True):
+        self.gpu = gpu_index
+        self.proc = None
+        self.enabled = enabled
+
+    def __enter__(self):
+        if self.enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                time.sleep(0.3)
+            except OSError:
+                self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), max=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hw_thermal=parts[6], sw_thermal=parts[7], sw_power=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": rows[0]["max"],
+                "power_w_max": max(r["power"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on the host cores, bounded row samples
+# ---------------------------------------------------------------------------
+_HOST_LAYERS = {}
+
+
+def host_layers(w, batch):
+    """The workload's layers as host arrays (generated once per process)."""
+    key = (w.name, batch)
+    if key not in _HOST_LAYERS:
+        layers = []
+        for li, lay in enumerate(w.layers):
+            s = lay.scheme
+            ld = synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index, layer=li)
+            x = synth.make_x(batch, lay.K, seed=0, workload=w.index, layer=li)
+            layers.append((lay, ld, x))
+        _HOST_LAYERS[key] = layers
+    return _HOST_LAYERS[key]
+
+
+def oracle_sample_run(w, batch, seconds, copy=0):
+    """Times oracle.linear (decode + fp64 matmul) on row samples of every layer.
+    Returns (algorithmic bytes of the sampled fraction, seconds, rows per layer, threads)."""
+    import oracle
+
+    layers = host_layers(w, batch)
+    # probe the per-row cost on a few rows of each layer
+    t0 = time.perf_counter()
+    for lay, ld, x in layers:
+        oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=np.arange(8))
+    probe = (time.perf_counter() - t0) / 8.0  # seconds per "one row of every layer"
+    rows = max(1, int(seconds / max(probe, 1e-9)))
+    total_bytes, elapsed = 0.0, 0.0
+    rng = np.random.Generator(np.random.PCG64(copy))
+    for lay, ld, x in layers:
+        r = min(rows, lay.N)
+        sel = np.sort(rng.choice(lay.N, size=r, replace=False))
+        t0 = time.perf_counter()
+        oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=sel)
+        elapsed += time.perf_counter() - t0
+        total_bytes += lay.algorithmic_bytes(batch) * (r / lay.N)
+    return total_bytes, elapsed, rows, oracle.max_threads()
+
+
+def run_reference(a):
+    rank, world, _ = env_rank()
+    w = workloads.get(a.workload)
+    batch = workload_batch(w, a.batch)
+    if rank != 0:
+        return 0
+    # each step is a bounded sample sized so that warmup + steps fit ~2 minutes
+    per_step = max(0.002, min(5.0, 120.0 / (a.steps + a.warmup)))
+    for i in range(a.warmup):
+        oracle_sample_run(w, batch, per_step, copy=i)
+    tot_b, tot_s = 0.0, 0.0
+    rows = 0
+    for i in range(a.steps):
+        b, s, rows, threads = oracle_sample_run(w, batch, per_step, copy=i)
+        tot_b += b
+        tot_s += s
+    value = tot_b / tot_s / 1e9
+    sample = (f"{rows} sampled rows of each of the {len(w.layers)} layers per step "
+              f"(decode to fp16 + fp64 matmul), batch {batch}")
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": a.gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": tot_s * 1e3 / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "layers": len(w.layers), "batch": batch,
+                       "scheme": w.layers[0].scheme.name, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def run_ours(a):
+    import torch
+
+    from weight_only_additive_b200 import layer as L
+    from weight_only_additive_b200 import native
+    from weight_only_additive_b200.native import Path
+
+    rank, world, local = env_rank()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist = None
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = native.lib()
+
+    w = workloads.get(a.workload)
+    batch = workload_batch(w, a.batch)
+    sbytes = step_bytes(w, batch)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 0) or L2_FALLBACK
+    copy_bytes = sum(l.algorithmic_bytes(batch) for l in w.layers)
+    pool = max(2, math.ceil(3 * l2 / copy_bytes))
+    while pool > 2 and pool * copy_bytes > 60e9:
+        pool -= 1
+
+    # device-resident pool: pool copies of every layer's weights and activations
+    weights, xs = [], []
+    for c in range(pool):
+        wc, xc = [], []
+        for li, lay in enumerate(w.layers):
+            s = lay.scheme
+            ld = synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index,
+                                  layer=li, copy=c + 1000 * rank)
+            wc.append(L.AqlmWeights.from_numpy(ld, dev))
+            xc.append(torch.from_numpy(synth.make_x(batch, lay.K, seed=0, workload=w.index, layer=li,
+                                                    copy=c + 1000 * rank)).to(dev))
+        weights.append(wc)
+        xs.append(xc)
+    ys = [torch.empty((batch, lay.N), dtype=torch.float16, device=dev) for lay in w.layers]
+    paths = [native.aqlm_select_path(l.scheme.M, l.scheme.B, l.scheme.g, l.K, l.N, batch) for l in w.layers]
+
+    stream = torch.cuda.Stream(dev)
+    h = stream.cuda_stream
+    # raw argument tuples: the step is seven C-ABI calls
+    calls = []
+    for c in range(pool):
+        cc = []
+        for li, lay in enumerate(w.layers):
+            wt = weights[c][li]
+            cc.append((xs[c][li].data_ptr(), wt.codes.data_ptr(), wt.codebooks.data_ptr(),
+                       wt.scales.data_ptr(), None, ys[li].data_ptr(), wt.M, wt.B, wt.g, lay.K, lay.N,
+                       batch, h))
+        calls.append(cc)
+
+    def step(c):
+        for args in calls[c]:
+            st = lib.aqlm_matmul(*args)
+            if st != 0:
+                raise native.AqlmError(st, "aqlm_matmul")
+
+    with torch.cuda.stream(stream):
+        for c in range(pool):
+            step(c)
+    torch.cuda.synchronize(dev)
+    graphs = []
+    for c in range(pool):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(c)
+        graphs.append(g)
+    torch.cuda.synchronize(dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for i in range(a.warmup):
+            graphs[i % pool].replay()
+    torch.cuda.synchronize(dev)
+    barrier()
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, enabled=not a.no_clocks) as clocks:
+        torch.cuda.synchronize(dev)
+        barrier()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for i in range(a.steps):
+                graphs[i % pool].replay()
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    st, detail = L.check_device_status(stream=stream)
+    if st != native.Status.OK:
+        raise RuntimeError(f"device status {st.name} {detail:#x}")
+
+    launches_per_step = len(w.layers)
+    total_bytes = sbytes * a.steps * world
+    value = total_bytes / (ms / 1e3) / 1e9
+    ms_step = ms / a.steps
+    peaks = measured_peaks()
+    avg_launch_s = (ms / 1e3) / (a.steps * launches_per_step)
+    bytes_per_launch = sbytes / launches_per_step
+    achieved = bytes_per_launch / avg_launch_s / 1e9
+    kernel_names = {int(Path.GEMV): "gemv_gather_kernel", int(Path.GEMV_LUT): "gemv_lut_kernel",
+                    int(Path.TENSOR_CORE): "tc_decode_mma_kernel"}
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": kernel_names.get(paths[0], "?"),
+                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
+                if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
+
+    # ---- end to end through the public API with host buffers ----------------
+    e2e = None
+    if not a.no_e2e:
+        e2e_steps = min(a.steps, 2000)
+        hx = [torch.from_numpy(synth.make_x(batch, lay.K, seed=7, layer=li)).pin_memory()
+              for li, lay in enumerate(w.layers)]
+        hy = [torch.empty((batch, lay.N), dtype=torch.float16).pin_memory() for lay in w.layers]
+        dx = [torch.empty((batch, lay.K), dtype=torch.float16, device=dev) for lay in w.layers]
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                for li in range(len(w.layers)):
+                    dx[li].copy_(hx[li], non_blocking=True)
+                    L.matmul(dx[li], weights[i % pool][li], out=ys[li], stream=stream)
+                    hy[li].copy_(ys[li], non_blocking=True)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(e2e_steps):
+                c = i % pool
+                for li in range(len(w.layers)):
+                    dx[li].copy_(hx[li], non_blocking=True)
+                    L.matmul(dx[li], weights[c][li], out=ys[li], stream=stream)
+                    hy[li].copy_(ys[li], non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": sbytes * e2e_steps * world / (ems / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": sum(t.numel() * 2 for t in hx),
+               "d2h_bytes_per_step": sum(t.numel() * 2 for t in hy),
+               "steps": e2e_steps, "us_per_layer": ems * 1e3 / (e2e_steps * len(w.layers)),
+               "how": "per layer: pinned H2D copy of x, matmul via the public API "
+                      "(weight_only_additive_b200.layer.matmul -> aqlm_matmul), D2H copy of y; "
+                      "no CUDA graph"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        b, s, rows, threads = oracle_sample_run(w, batch, a.cpu_seconds)
+        cpu = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{rows} sampled rows of each of the {len(w.layers)} layers "
+                         f"(decode to fp16 + fp64 matmul), batch {batch}, {s:.1f} s"}
+
+    if dist is not None:
+        del graphs
+        dist.barrier()
+        dist.destroy_process_group()
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": ms_step,
+                "us_per_layer": ms_step * 1e3 / launches_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+                "data": "synthetic",
+                "config": {"workload": w.name, "layers": len(w.layers), "batch": batch,
+                           "scheme": w.layers[0].scheme.name,
+                           "algorithmic_bytes_per_step": sbytes,
+                           "l2": f"inputs larger than L2: rotating pool of {pool} copies "
+                                 f"({pool * copy_bytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
+                           "launch": "one CUDA graph replay per step",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches_per_step * a.steps,
+                "clocks": clocks.summary(), "gpu": props.name}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    a = parse_args(argv)
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_ours(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,133 @@
+/*
+ * aqlm.h -- C ABI of libaqlm.so, the B200 (sm_100a) AQLM weight-only linear layer.
+ *
+ * The layer (AQLM, "Extreme Compression of Large Language Models via Additive
+ * Quantization"; paper record, method paragraph; AQLM repo summary "What it
+ * does"; inference-research record "AQLM (additive / multi-codebook
+ * quantization)", sections "Bits", "Activation scheme", "Kernels", "notes"):
+ *
+ *     y = x . W^T . diag(s) + bias
+ *
+ * where every g-wide group of a weight row is the SUM of M fp16 codewords, one
+ * picked from each of M codebooks of 2^B entries, and the activations x stay
+ * fp16 (w2a16).  Weights never exist in HBM in dense form: the kernels decode
+ * them on chip ("fast lookup, no per-element dequantization" for token
+ * generation; "dequantize-to-FP16 then an FP16 tensor-core GEMM" for larger
+ * batches).
+ *
+ * Data layout (all row-major, C order, caller-owned DEVICE memory):
+ *   x          fp16   [batch, K]
+ *   codes      uint8  [N, K/g, M] when B == 8, uint16 [N, K/g, M] when B == 16;
+ *              unsigned, no offset, codebook index m varies fastest
+ *   codebooks  fp16   [M, 2^B, g]
+ *   scales     fp16   [N]            (one scale per output channel)
+ *   bias       fp16   [N] or NULL
+ *   y          fp16   [batch, N]
+ *   W_out      fp16   [N, K]         (aqlm_dequantize only)
+ *
+ * Supported schemes (M, B, g): (1, 16, 8) "1x16 g8", (2, 8, 8) "2x8 g8",
+ * (1, 16, 16) "1x16 g16".  Other shapes return AQLM_ERR_UNSUPPORTED.
+ * K must be a multiple of g; N >= 1; 1 <= batch <= 65535.  Every pointer must be
+ * 16-byte aligned (AQLM_ERR_MISALIGNED otherwise); bias may be NULL.
+ *
+ * Ownership and state: the library never allocates or frees device memory on
+ * a call and keeps no per-call state.  It holds one 32-bit device status word
+ * per device (a static device variable) where kernels record a bounded wait
+ * that gave up.  All compute calls are asynchronous on `stream`
+ * (NULL = the legacy default stream) and may be captured in CUDA graphs.
+ *
+ * Errors: every function returns a status and never aborts, throws or exits.
+ * Argument errors are detected on the host before any launch.  A failed
+ * launch returns AQLM_ERR_CUDA (the CUDA error is cleared and can be read with
+ * aqlm_last_cuda_error).  Device-side failures (a wait that ran out) surface
+ * through aqlm_check_device_status.
+ */
+#ifndef AQLM_H_
+#define AQLM_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL means the legacy default stream. */
+typedef struct CUstream_st* aqlm_stream_t;
+
+typedef enum {
+  AQLM_OK = 0,
+  AQLM_ERR_INVALID_ARG = 1,   /* NULL pointer, K % g != 0, non-positive size, ... */
+  AQLM_ERR_UNSUPPORTED = 2,   /* (M, B, g) or forced path not implemented        */
+  AQLM_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned               */
+  AQLM_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed     */
+  AQLM_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up              */
+} aqlm_status;
+
+/* Kernel families aqlm_matmul can route to. */
+typedef enum {
+  AQLM_PATH_AUTO = 0,         /* pick by (M, B, g, batch)                               */
+  AQLM_PATH_GEMV = 1,         /* codeword-gather GEMV, any supported scheme, batch <= 8 */
+  AQLM_PATH_GEMV_LUT = 2,     /* x.codeword lookup-table GEMV, 2x8 only, batch <= 8     */
+  AQLM_PATH_TENSOR_CORE = 3   /* on-chip decode -> tcgen05 fp16 MMA, any batch          */
+} aqlm_path;
+
+/*
+ * y = x . W^T . diag(scales) + bias, with W decoded on chip from codes and
+ * codebooks.  Accumulation is fp32 (or better); y is rounded to fp16 (RNE).
+ * Result tolerance against the fp64 reference of the decoded fp16 weights:
+ * max|y - y_ref| / max|y_ref| <= 5e-3.
+ * Returns AQLM_OK after enqueueing the work on `stream`.
+ */
+aqlm_status aqlm_matmul(const void* x, const void* codes, const void* codebooks,
+                        const void* scales, const void* bias, void* y,
+                        int M, int B, int g, int K, int N, int batch,
+                        aqlm_stream_t stream);
+
+/* aqlm_matmul with the kernel family chosen by the caller (tests, benchmarks).
+ * AQLM_ERR_UNSUPPORTED if that family cannot run this (scheme, batch). */
+aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codebooks,
+                             const void* scales, const void* bias, void* y,
+                             int M, int B, int g, int K, int N, int batch,
+                             aqlm_path path, aqlm_stream_t stream);
+
+/*
+ * W_out[n, j*g + t] = fp16_rne( fp32( C_0[c_0][t] + C_1[c_1][t] + ... ) * fp32(s_n) )
+ * with c_m = codes[n, j, m]; the codewords are added in fp32 in ascending m,
+ * starting from C_0 itself, then one fp32 multiply by the channel scale and
+ * one round-to-nearest-even to fp16.  Bit-exact by definition.
+ */
+aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void* scales,
+                            void* W_out, int M, int B, int g, int K, int N,
+                            aqlm_stream_t stream);
+
+/* The kernel family AQLM_PATH_AUTO picks for this problem, or -1 if unsupported.
+ * Pure host logic: needs no GPU. */
+int aqlm_select_path(int M, int B, int g, int K, int N, int batch);
+
+/* Validates arguments exactly as aqlm_matmul_path does, without launching
+ * anything.  Pure host logic: needs no GPU. */
+aqlm_status aqlm_validate(const void* x, const void* codes, const void* codebooks,
+                          const void* scales, const void* bias, const void* y,
+                          int M, int B, int g, int K, int N, int batch, aqlm_path path);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* aqlm_status_string(aqlm_status status);
+
+/* Synchronises `stream`, then reads and clears the current device's status
+ * word.  Returns AQLM_ERR_TIMEOUT if a kernel recorded a wait that gave up
+ * (`detail`, if not NULL, receives the recorded site code), AQLM_ERR_CUDA if the
+ * synchronisation failed, AQLM_OK otherwise. */
+aqlm_status aqlm_check_device_status(aqlm_stream_t stream, uint32_t* detail);
+
+/* The cudaError_t value of the last CUDA failure this thread saw in the library
+ * (0 if none). */
+int aqlm_last_cuda_error(void);
+
+/* ABI version of this header (incremented on any signature change). */
+int aqlm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQLM_H_ */

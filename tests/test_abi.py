@@ -1,0 +1,95 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every symbol
+include/aqlm.h declares, and its host-side validation and path selection work
+without touching the device (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from weight_only_additive_b200 import build, native
+from weight_only_additive_b200.native import Path, Status
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "aqlm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return native.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(aqlm_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(native.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.aqlm_abi_version() == native.ABI_VERSION
+    for st in Status:
+        assert native.status_string(st).startswith("AQLM_")
+    assert "unknown" in native.status_string(99)
+
+
+A = 1 << 20  # a 16-byte aligned fake address: validation never dereferences it
+
+
+@pytest.mark.parametrize("M,B,g", [(1, 16, 8), (2, 8, 8), (1, 16, 16)])
+def test_supported_schemes_validate(lib, M, B, g):
+    assert native.aqlm_validate(A, A, A, A, None, A, M, B, g, 4096, 4096, 1) == Status.OK
+    assert native.aqlm_validate(A, A, A, A, A, A, M, B, g, 4096, 11008, 256) == Status.OK
+
+
+@pytest.mark.parametrize("args,want", [
+    ((None, A, A, A, None, A, 1, 16, 8, 64, 64, 1), Status.INVALID_ARG),   # null x
+    ((A, None, A, A, None, A, 1, 16, 8, 64, 64, 1), Status.INVALID_ARG),   # null codes
+    ((A, A, A, A, None, None, 1, 16, 8, 64, 64, 1), Status.INVALID_ARG),   # null y
+    ((A, A, A, A, None, A, 1, 16, 8, 60, 64, 1), Status.INVALID_ARG),      # K % g != 0
+    ((A, A, A, A, None, A, 1, 16, 8, 64, 0, 1), Status.INVALID_ARG),       # N = 0
+    ((A, A, A, A, None, A, 1, 16, 8, 64, 64, 0), Status.INVALID_ARG),      # batch = 0
+    ((A, A, A, A, None, A, 1, 16, 8, 64, 64, 70000), Status.INVALID_ARG),  # batch too large
+    ((A, A, A, A, None, A, 3, 8, 8, 64, 64, 1), Status.UNSUPPORTED),       # 3x8 not built
+    ((A, A, A, A, None, A, 2, 16, 8, 64, 64, 1), Status.UNSUPPORTED),      # 2x16
+    ((A, A, A, A, None, A, 1, 12, 8, 64, 64, 1), Status.UNSUPPORTED),      # B = 12
+    ((A + 8, A, A, A, None, A, 1, 16, 8, 64, 64, 1), Status.MISALIGNED),
+    ((A, A + 2, A, A, None, A, 1, 16, 8, 64, 64, 1), Status.MISALIGNED),
+    ((A, A, A, A, A + 4, A, 1, 16, 8, 64, 64, 1), Status.MISALIGNED),       # bias
+])
+def test_validation_errors_need_no_gpu(lib, args, want):
+    assert native.aqlm_validate(*args) == want
+
+
+def test_compute_entry_points_reject_bad_arguments_before_any_cuda_call(lib):
+    # these return before touching the device, so they are safe without a GPU
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_matmul(None, A, A, A, None, A, 1, 16, 8, 64, 64, 1)
+    assert e.value.status == Status.INVALID_ARG
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_dequantize(A, A, A, A + 2, 1, 16, 8, 64, 64)
+    assert e.value.status == Status.MISALIGNED
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_matmul_path(A, A, A, A, None, A, 1, 16, 8, 64, 64, 16, Path.GEMV)
+    assert e.value.status == Status.UNSUPPORTED  # the GEMV family stops at batch 8
+
+
+def test_path_selection(lib):
+    sel = native.aqlm_select_path
+    for M, B, g in ((1, 16, 8), (2, 8, 8), (1, 16, 16)):
+        for batch in range(1, 9):
+            assert sel(M, B, g, 4096, 4096, batch) in (Path.GEMV, Path.GEMV_LUT)
+        for batch in (9, 16, 64, 256, 1000):
+            assert sel(M, B, g, 4096, 4096, batch) == Path.TENSOR_CORE
+    assert sel(3, 8, 8, 4096, 4096, 1) == -1
+    assert sel(1, 16, 8, 4095, 4096, 1) == -1

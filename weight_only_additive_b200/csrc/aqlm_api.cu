@@ -1,0 +1,169 @@
+// C ABI of libaqlm.so: argument validation, kernel-family dispatch and the
+// device status word.  Declarations and the contract live in include/aqlm.h.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "aqlm.h"
+#include "aqlm_internal.h"
+
+namespace {
+
+// One status word per device (the array lives in every device's copy of this
+// module).  Kernels record the site of a bounded wait that gave up here.
+__device__ uint32_t g_device_status;
+
+thread_local int t_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+uint32_t* g_status_ptr[kMaxDevices] = {};
+
+// Device address of g_device_status for the current device (nullptr on failure).
+uint32_t* device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_status_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+aqlm_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return AQLM_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  cudaGetLastError();  // clear the sticky-free error so later calls start clean
+  return AQLM_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool path_accepts(aqlm_path path, int M, int B, int g, int batch) {
+  switch (path) {
+    case AQLM_PATH_GEMV: return batch <= 8;
+    case AQLM_PATH_GEMV_LUT: return false;  // not built yet
+    case AQLM_PATH_TENSOR_CORE: return true;
+    default: return false;
+  }
+  (void)M; (void)B; (void)g;
+}
+
+aqlm_status validate_shape(int M, int B, int g, int K, int N, int batch) {
+  if (M < 1 || B < 1 || g < 1 || K < 1 || N < 1 || batch < 1) return AQLM_ERR_INVALID_ARG;
+  if (K % g != 0) return AQLM_ERR_INVALID_ARG;
+  if (batch > 65535) return AQLM_ERR_INVALID_ARG;
+  if (!aqlm::scheme_supported(M, B, g)) return AQLM_ERR_UNSUPPORTED;
+  return AQLM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int aqlm_abi_version(void) { return 1; }
+
+const char* aqlm_status_string(aqlm_status status) {
+  switch (status) {
+    case AQLM_OK: return "AQLM_OK";
+    case AQLM_ERR_INVALID_ARG: return "AQLM_ERR_INVALID_ARG: invalid argument";
+    case AQLM_ERR_UNSUPPORTED: return "AQLM_ERR_UNSUPPORTED: scheme or path not supported";
+    case AQLM_ERR_MISALIGNED: return "AQLM_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case AQLM_ERR_CUDA: return "AQLM_ERR_CUDA: CUDA call or kernel launch failed";
+    case AQLM_ERR_TIMEOUT: return "AQLM_ERR_TIMEOUT: device-side bounded wait gave up";
+  }
+  return "AQLM: unknown status";
+}
+
+int aqlm_last_cuda_error(void) { return t_last_cuda_error; }
+
+int aqlm_select_path(int M, int B, int g, int K, int N, int batch) {
+  if (validate_shape(M, B, g, K, N, batch) != AQLM_OK) return -1;
+  if (batch <= 8) return AQLM_PATH_GEMV;
+  return AQLM_PATH_TENSOR_CORE;
+}
+
+aqlm_status aqlm_validate(const void* x, const void* codes, const void* codebooks,
+                          const void* scales, const void* bias, const void* y,
+                          int M, int B, int g, int K, int N, int batch, aqlm_path path) {
+  if (!x || !codes || !codebooks || !scales || !y) return AQLM_ERR_INVALID_ARG;
+  const aqlm_status st = validate_shape(M, B, g, K, N, batch);
+  if (st != AQLM_OK) return st;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(codebooks) || !aligned16(scales) ||
+      !aligned16(y) || (bias && !aligned16(bias)))
+    return AQLM_ERR_MISALIGNED;
+  if (path != AQLM_PATH_AUTO && !path_accepts(path, M, B, g, batch)) {
+    if (path < AQLM_PATH_AUTO || path > AQLM_PATH_TENSOR_CORE) return AQLM_ERR_INVALID_ARG;
+    return AQLM_ERR_UNSUPPORTED;
+  }
+  return AQLM_OK;
+}
+
+aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codebooks,
+                             const void* scales, const void* bias, void* y,
+                             int M, int B, int g, int K, int N, int batch,
+                             aqlm_path path, aqlm_stream_t stream) {
+  const aqlm_status st = aqlm_validate(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path);
+  if (st != AQLM_OK) return st;
+  if (path == AQLM_PATH_AUTO) path = static_cast<aqlm_path>(aqlm_select_path(M, B, g, K, N, batch));
+  const aqlm::Problem p{x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (path) {
+    case AQLM_PATH_GEMV: return from_cuda(aqlm::launch_gemv(p, s));
+    case AQLM_PATH_TENSOR_CORE: {
+      uint32_t* status = device_status_ptr();
+      if (!status) return from_cuda(cudaErrorInvalidDevice);
+      return from_cuda(aqlm::launch_tc(p, status, s));
+    }
+    default: return AQLM_ERR_UNSUPPORTED;
+  }
+}
+
+aqlm_status aqlm_matmul(const void* x, const void* codes, const void* codebooks,
+                        const void* scales, const void* bias, void* y,
+                        int M, int B, int g, int K, int N, int batch, aqlm_stream_t stream) {
+  return aqlm_matmul_path(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch,
+                          AQLM_PATH_AUTO, stream);
+}
+
+aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void* scales,
+                            void* W_out, int M, int B, int g, int K, int N,
+                            aqlm_stream_t stream) {
+  if (!codes || !codebooks || !scales || !W_out) return AQLM_ERR_INVALID_ARG;
+  const aqlm_status st = validate_shape(M, B, g, K, N, 1);
+  if (st != AQLM_OK) return st;
+  if (!aligned16(codes) || !aligned16(codebooks) || !aligned16(scales) || !aligned16(W_out))
+    return AQLM_ERR_MISALIGNED;
+  return from_cuda(aqlm::launch_dequantize(codes, codebooks, scales, W_out, M, B, g, K, N,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+aqlm_status aqlm_check_device_status(aqlm_stream_t stream, uint32_t* detail) {
+  if (detail) *detail = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return from_cuda(e);
+  uint32_t* dev_status = device_status_ptr();
+  if (!dev_status) return from_cuda(cudaErrorInvalidDevice);
+  uint32_t value = 0;
+  e = cudaMemcpy(&value, dev_status, sizeof value, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (value != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpy(dev_status, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (detail) *detail = value;
+    return AQLM_ERR_TIMEOUT;
+  }
+  return AQLM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,42 @@
+// Internal interface between the C-ABI layer (aqlm_api.cu) and the kernels.
+// Host code only calls these after aqlm_validate-style checks have passed.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace aqlm {
+
+// Bounded device waits give up after this much wall time (1 s) and record a
+// site code in the library's device status word.
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
+
+// Site codes written to the device status word.
+enum : uint32_t {
+  kSiteTcMmaDone = 0x101,   // tensor-core kernel: waiting for an MMA commit
+};
+
+struct Problem {
+  const void* x;
+  const void* codes;
+  const void* codebooks;
+  const void* scales;
+  const void* bias;  // may be null
+  void* y;
+  int M, B, g, K, N, batch;
+};
+
+// Each launcher enqueues its kernel(s) on `stream` and returns the launch error.
+cudaError_t launch_dequantize(const void* codes, const void* codebooks, const void* scales,
+                              void* W_out, int M, int B, int g, int K, int N,
+                              cudaStream_t stream);
+cudaError_t launch_gemv(const Problem& p, cudaStream_t stream);
+cudaError_t launch_gemv_lut(const Problem& p, cudaStream_t stream);
+cudaError_t launch_tc(const Problem& p, uint32_t* status, cudaStream_t stream);
+
+// True if the scheme is one the kernels are instantiated for.
+inline bool scheme_supported(int M, int B, int g) {
+  return (M == 1 && B == 16 && (g == 8 || g == 16)) || (M == 2 && B == 8 && g == 8);
+}
+
+}  // namespace aqlm

@@ -1,0 +1,99 @@
+"""PyTorch-facing wrappers over the C ABI: pass `data_ptr()`s and the current
+CUDA stream to libaqlm.so.  Torch provides device memory and streams only; the
+arithmetic happens in the library's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import native
+from .native import Path
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream], device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+@dataclass
+class AqlmWeights:
+    """One AQLM linear layer resident on a CUDA device."""
+    codes: torch.Tensor       # [N, K/g, M] uint8 (B=8) or int16 holding uint16 bits (B=16)
+    codebooks: torch.Tensor   # [M, 2^B, g] float16
+    scales: torch.Tensor      # [N] float16
+    bias: Optional[torch.Tensor]
+    M: int
+    B: int
+    g: int
+
+    @property
+    def N(self) -> int:
+        return self.codes.shape[0]
+
+    @property
+    def K(self) -> int:
+        return self.codes.shape[1] * self.g
+
+    @classmethod
+    def from_numpy(cls, layer, device="cuda") -> "AqlmWeights":
+        """From a synth.LayerData (numpy host arrays)."""
+        # 16-bit codes travel as int16 (same bytes): torch has few uint16 kernels.
+        raw = layer.codes.view(np.int16) if layer.codes.dtype == np.uint16 else layer.codes
+        codes = torch.from_numpy(np.ascontiguousarray(raw))
+        return cls(codes=codes.to(device), codebooks=torch.from_numpy(layer.codebooks).to(device),
+                   scales=torch.from_numpy(layer.scales).to(device),
+                   bias=None if layer.bias is None else torch.from_numpy(layer.bias).to(device),
+                   M=layer.M, B=layer.B, g=layer.g)
+
+
+def _check_tensor(t: torch.Tensor, name: str, dtype, device):
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def matmul(x: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = None,
+           path: Path = Path.AUTO, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """y = x . W^T . diag(s) + bias for x [batch, K] fp16 on the weights' device."""
+    dev = w.codes.device
+    if dev.type != "cuda":
+        raise ValueError("AQLM weights must live on a CUDA device")
+    _check_tensor(x, "x", torch.float16, dev)
+    batch, K = x.shape
+    if K != w.K:
+        raise ValueError(f"x has K={K}, weights have K={w.K}")
+    if out is None:
+        out = torch.empty((batch, w.N), dtype=torch.float16, device=dev)
+    _check_tensor(out, "out", torch.float16, dev)
+    native.aqlm_matmul_path(x.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(),
+                            w.scales.data_ptr(), _ptr(w.bias), out.data_ptr(),
+                            w.M, w.B, w.g, K, w.N, batch, path, _stream_handle(stream, dev))
+    return out
+
+
+def dequantize(w: AqlmWeights, out: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """W [N, K] fp16, bit-exact decode of the AQLM weights."""
+    dev = w.codes.device
+    if out is None:
+        out = torch.empty((w.N, w.K), dtype=torch.float16, device=dev)
+    _check_tensor(out, "out", torch.float16, dev)
+    native.aqlm_dequantize(w.codes.data_ptr(), w.codebooks.data_ptr(), w.scales.data_ptr(),
+                           out.data_ptr(), w.M, w.B, w.g, w.K, w.N, _stream_handle(stream, dev))
+    return out
+
+
+def check_device_status(stream: Optional[torch.cuda.Stream] = None, device=None):
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return native.aqlm_check_device_status(_stream_handle(stream, dev))

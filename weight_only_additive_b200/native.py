@@ -1,0 +1,130 @@
+"""ctypes binding to libaqlm.so (include/aqlm.h), names as in the C ABI.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  There is no CPU or PyTorch fallback -- if libaqlm.so is missing or
+cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import enum
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(PKG, "libaqlm.so")
+
+# Every exported symbol of include/aqlm.h.
+EXPORTS = ("aqlm_matmul", "aqlm_matmul_path", "aqlm_dequantize", "aqlm_select_path",
+           "aqlm_validate", "aqlm_status_string", "aqlm_check_device_status",
+           "aqlm_last_cuda_error", "aqlm_abi_version")
+
+ABI_VERSION = 1
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    INVALID_ARG = 1
+    UNSUPPORTED = 2
+    MISALIGNED = 3
+    CUDA = 4
+    TIMEOUT = 5
+
+
+class Path(enum.IntEnum):
+    AUTO = 0
+    GEMV = 1
+    GEMV_LUT = 2
+    TENSOR_CORE = 3
+
+
+class AqlmError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = Status(status) if status in Status._value2member_map_ else status
+        msg = status_string(status)
+        if what:
+            msg = f"{what}: {msg}"
+        if status == Status.CUDA:
+            msg += f" (cudaError {lib().aqlm_last_cuda_error()})"
+        super().__init__(msg)
+
+
+_lib = None
+_lock = threading.Lock()
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+
+def lib() -> ctypes.CDLL:
+    """Load libaqlm.so (raises if it is missing: the product has no fallback)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIBRARY):
+                    raise ImportError(
+                        f"{LIBRARY} is missing: build it with `python -m weight_only_additive_b200.build`")
+                L = ctypes.CDLL(LIBRARY)
+                L.aqlm_matmul.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+                L.aqlm_matmul.restype = _i
+                L.aqlm_matmul_path.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+                L.aqlm_matmul_path.restype = _i
+                L.aqlm_dequantize.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+                L.aqlm_dequantize.restype = _i
+                L.aqlm_select_path.argtypes = [_i] * 6
+                L.aqlm_select_path.restype = _i
+                L.aqlm_validate.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i]
+                L.aqlm_validate.restype = _i
+                L.aqlm_status_string.argtypes = [_i]
+                L.aqlm_status_string.restype = ctypes.c_char_p
+                L.aqlm_check_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
+                L.aqlm_check_device_status.restype = _i
+                L.aqlm_last_cuda_error.restype = _i
+                L.aqlm_abi_version.restype = _i
+                if L.aqlm_abi_version() != ABI_VERSION:
+                    raise ImportError(f"libaqlm.so ABI {L.aqlm_abi_version()} != binding ABI {ABI_VERSION}")
+                _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().aqlm_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != Status.OK:
+        raise AqlmError(status, what)
+
+
+# --------------------------------------------------------------------------
+# raw-pointer entry points (same names and argument order as the C ABI)
+# --------------------------------------------------------------------------
+def aqlm_matmul(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, stream=None):
+    _check(lib().aqlm_matmul(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, stream),
+           "aqlm_matmul")
+
+
+def aqlm_matmul_path(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path, stream=None):
+    _check(lib().aqlm_matmul_path(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch,
+                                  int(path), stream), "aqlm_matmul_path")
+
+
+def aqlm_dequantize(codes, codebooks, scales, W_out, M, B, g, K, N, stream=None):
+    _check(lib().aqlm_dequantize(codes, codebooks, scales, W_out, M, B, g, K, N, stream),
+           "aqlm_dequantize")
+
+
+def aqlm_select_path(M, B, g, K, N, batch) -> int:
+    return lib().aqlm_select_path(M, B, g, K, N, batch)
+
+
+def aqlm_validate(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path=Path.AUTO) -> int:
+    return lib().aqlm_validate(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, int(path))
+
+
+def aqlm_check_device_status(stream=None):
+    """Returns (status, detail) after synchronising `stream`."""
+    detail = ctypes.c_uint32(0)
+    st = lib().aqlm_check_device_status(stream, ctypes.byref(detail))
+    return Status(st), detail.value
