@@ -82,13 +82,22 @@ def test_compute_entry_points_reject_bad_arguments_before_any_cuda_call(lib):
     with pytest.raises(native.AqlmError) as e:
         native.aqlm_matmul_path(A, A, A, A, None, A, 1, 16, 8, 64, 64, 16, Path.GEMV)
     assert e.value.status == Status.UNSUPPORTED  # the GEMV family stops at batch 8
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_matmul_path(A, A, A, A, None, A, 1, 16, 8, 64, 64, 1, Path.GEMV_LUT)
+    assert e.value.status == Status.UNSUPPORTED  # the lookup table is the 2x8 kernel
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_matmul_path(A, A, A, A, None, A, 2, 8, 8, 64, 64, 2, Path.GEMV_LUT)
+    assert e.value.status == Status.UNSUPPORTED  # batch 1 only
 
 
 def test_path_selection(lib):
     sel = native.aqlm_select_path
+    assert sel(2, 8, 8, 4096, 4096, 1) == Path.GEMV_LUT
+    assert sel(2, 8, 8, 4096 + 8, 4096, 1) == Path.GEMV      # K % 64 != 0: no lookup table
+    assert sel(1, 16, 8, 4096, 4096, 1) == Path.GEMV
     for M, B, g in ((1, 16, 8), (2, 8, 8), (1, 16, 16)):
-        for batch in range(1, 9):
-            assert sel(M, B, g, 4096, 4096, batch) in (Path.GEMV, Path.GEMV_LUT)
+        for batch in range(2, 9):
+            assert sel(M, B, g, 4096, 4096, batch) == Path.GEMV
         for batch in (9, 16, 64, 256, 1000):
             assert sel(M, B, g, 4096, 4096, batch) == Path.TENSOR_CORE
     assert sel(3, 8, 8, 4096, 4096, 1) == -1

@@ -131,13 +131,27 @@ def test_tensor_core_parity(dev, M, B, g, N, K, batch):
                  f"tc {M}x{B}g{g} N={N} K={K} b={batch}")
 
 
+@pytest.mark.parametrize("N,K", [(1, 64), (37, 128), (200, 512), (300, 4096), (129, 64 * 23),
+                                 (1000, 11008), (700, 14336), (4100, 4096)])
+def test_gemv_lut_parity(dev, N, K):
+    """Lookup-table GEMV (2x8, batch 1): ragged row counts, K from one pass to
+    several passes per CTA, cluster sizes from 1 to 16."""
+    ld = synth.make_layer(2, 8, 8, K, N, seed=17, layer=N, with_bias=(N % 2 == 1))
+    x = synth.make_x(1, K, seed=17, layer=N)
+    y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, 2, 8, 8)
+    assert_close(gpu_matmul(ld, x, dev, Path.GEMV_LUT), y_ref, f"lut N={N} K={K}")
+
+
 @pytest.mark.parametrize("M,B,g", SCHEMES)
 @pytest.mark.parametrize("path,batch", [(Path.GEMV, 1), (Path.GEMV, 4), (Path.GEMV, 8),
+                                        (Path.GEMV_LUT, 1),
                                         (Path.TENSOR_CORE, 16), (Path.TENSOR_CORE, 100)])
 def test_integer_layers_bit_exact(dev, M, B, g, path, batch):
     """Small-integer codebooks and x, scales in {1, 2}: every product and partial sum
     is an exact small integer in fp16/fp32, so any summation order gives the exact
     value and y must equal the oracle bit for bit."""
+    if path == Path.GEMV_LUT and (M, B, g) != (2, 8, 8):
+        pytest.skip("the lookup-table GEMV is the 2x8 kernel")
     N, K = 260, 512
     rng = np.random.Generator(np.random.PCG64(14))
     cb = rng.integers(-2, 3, size=(M, 1 << B, g)).astype(np.float16)
@@ -162,8 +176,9 @@ def test_zero_codebooks_give_bias(dev):
 
 
 def test_runs_are_deterministic(dev):
-    ld = synth.make_layer(1, 16, 8, 4096, 1000, seed=16)
-    for batch, path in ((1, Path.GEMV), (64, Path.TENSOR_CORE)):
+    for (M, B, g), batch, path in (((1, 16, 8), 1, Path.GEMV), ((1, 16, 8), 64, Path.TENSOR_CORE),
+                                   ((2, 8, 8), 1, Path.GEMV_LUT)):
+        ld = synth.make_layer(M, B, g, 4096, 1000, seed=16)
         x = synth.make_x(batch, 4096, seed=16)
         a = gpu_matmul(ld, x, dev, path)
         b = gpu_matmul(ld, x, dev, path)

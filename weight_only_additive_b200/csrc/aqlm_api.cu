@@ -47,14 +47,13 @@ aqlm_status from_cuda(cudaError_t e) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool path_accepts(aqlm_path path, int M, int B, int g, int batch) {
+bool path_accepts(aqlm_path path, int M, int B, int g, int K, int batch) {
   switch (path) {
     case AQLM_PATH_GEMV: return batch <= 8;
-    case AQLM_PATH_GEMV_LUT: return false;  // not built yet
+    case AQLM_PATH_GEMV_LUT: return aqlm::gemv_lut_supported(M, B, g, K, batch);
     case AQLM_PATH_TENSOR_CORE: return true;
     default: return false;
   }
-  (void)M; (void)B; (void)g;
 }
 
 aqlm_status validate_shape(int M, int B, int g, int K, int N, int batch) {
@@ -87,6 +86,7 @@ int aqlm_last_cuda_error(void) { return t_last_cuda_error; }
 
 int aqlm_select_path(int M, int B, int g, int K, int N, int batch) {
   if (validate_shape(M, B, g, K, N, batch) != AQLM_OK) return -1;
+  if (aqlm::gemv_lut_supported(M, B, g, K, batch)) return AQLM_PATH_GEMV_LUT;
   if (batch <= 8) return AQLM_PATH_GEMV;
   return AQLM_PATH_TENSOR_CORE;
 }
@@ -100,7 +100,7 @@ aqlm_status aqlm_validate(const void* x, const void* codes, const void* codebook
   if (!aligned16(x) || !aligned16(codes) || !aligned16(codebooks) || !aligned16(scales) ||
       !aligned16(y) || (bias && !aligned16(bias)))
     return AQLM_ERR_MISALIGNED;
-  if (path != AQLM_PATH_AUTO && !path_accepts(path, M, B, g, batch)) {
+  if (path != AQLM_PATH_AUTO && !path_accepts(path, M, B, g, K, batch)) {
     if (path < AQLM_PATH_AUTO || path > AQLM_PATH_TENSOR_CORE) return AQLM_ERR_INVALID_ARG;
     return AQLM_ERR_UNSUPPORTED;
   }
@@ -118,6 +118,11 @@ aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codeb
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (path) {
     case AQLM_PATH_GEMV: return from_cuda(aqlm::launch_gemv(p, s));
+    case AQLM_PATH_GEMV_LUT: {
+      uint32_t* status = device_status_ptr();
+      if (!status) return from_cuda(cudaErrorInvalidDevice);
+      return from_cuda(aqlm::launch_gemv_lut(p, status, s));
+    }
     case AQLM_PATH_TENSOR_CORE: {
       uint32_t* status = device_status_ptr();
       if (!status) return from_cuda(cudaErrorInvalidDevice);

@@ -14,6 +14,8 @@ constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
 // Site codes written to the device status word.
 enum : uint32_t {
   kSiteTcMmaDone = 0x101,   // tensor-core kernel: waiting for an MMA commit
+  kSiteLutMma = 0x201,      // lookup-table GEMV: waiting for the table-building MMA
+  kSiteLutReduce = 0x202,   // lookup-table GEMV: waiting for the cluster's partial sums
 };
 
 struct Problem {
@@ -31,7 +33,9 @@ cudaError_t launch_dequantize(const void* codes, const void* codebooks, const vo
                               void* W_out, int M, int B, int g, int K, int N,
                               cudaStream_t stream);
 cudaError_t launch_gemv(const Problem& p, cudaStream_t stream);
-cudaError_t launch_gemv_lut(const Problem& p, cudaStream_t stream);
+cudaError_t launch_gemv_lut(const Problem& p, uint32_t* status, cudaStream_t stream);
+// True if the lookup-table GEMV handles this problem (2x8 g8, batch 1, K % 64 == 0).
+bool gemv_lut_supported(int M, int B, int g, int K, int batch);
 cudaError_t launch_tc(const Problem& p, uint32_t* status, cudaStream_t stream);
 
 // True if the scheme is one the kernels are instantiated for.
