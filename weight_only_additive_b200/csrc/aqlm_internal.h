@@ -15,7 +15,7 @@ constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
 enum : uint32_t {
   kSiteTcMmaDone = 0x101,   // tensor-core kernel: waiting for an MMA commit
   kSiteLutMma = 0x201,      // lookup-table GEMV: waiting for the table-building MMA
-  kSiteLutReduce = 0x202,   // lookup-table GEMV: waiting for the cluster's partial sums
+  kSiteLutCodes = 0x202,    // lookup-table GEMV: code-tile pipeline (TMA landing / slot release)
 };
 
 struct Problem {

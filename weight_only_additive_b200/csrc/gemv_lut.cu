@@ -26,6 +26,8 @@
 // lanes of a lookup touch 32 different banks whatever the codes are.  The
 // table is written from TMEM lane rho = word column, which is conflict-free
 // too: A row rho holds group 2*(rho mod 32) + rho/32.
+#include <cuda.h>
+
 #include <algorithm>
 #include <map>
 #include <mutex>
@@ -36,18 +38,20 @@
 namespace aqlm {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kGroupsPerPass = 64;
+constexpr int kMaxPasses = 4;                      // K <= 16 CTAs x 4 passes x 64 groups x 8
+constexpr int kTileRows = 64;                      // rows per code tile (one TMA box)
 constexpr uint32_t kLutBytes = 256u * 64u * 4u;   // 64 KB
-constexpr uint32_t kAOpBytes = 128u * 32u;         // 4 KB
+constexpr uint32_t kAOpBytes = 128u * 32u;         // 4 KB per pass
 constexpr uint32_t kBOpBytes = 256u * 32u;         // 8 KB per codebook
-constexpr uint32_t kChunkBytes = 32u * 128u;       // 32 rows x 128 B of codes
+constexpr uint32_t kTileBytes = 64u * 128u;        // 64 rows x 128 B of codes (one TMA box)
 constexpr uint32_t kTmemCols = 512;                // D_0 at [0,256), D_1 at [256,512)
+constexpr uint32_t kSmemLimit = 227u * 1024u;
 
 struct LutParams {
   const __half* x;
-  const uint8_t* codes;
   const __half* codebooks;
   const __half* scales;
   const __half* bias;
@@ -57,27 +61,41 @@ struct LutParams {
   int P;      // passes of 64 groups per CTA
   int RB;     // output rows per cluster
   int RBc;    // rows each CTA reduces (multiple of 4)
-  int nchunk; // ceil(RB / 32)
+  int ntask;  // ceil(RB / 8): 8-row tasks per pass
+  int ntile;  // ceil(RB / 64): code tiles per pass
   uint32_t* status;
 };
 
 struct SmemLayout {
-  uint32_t lut, aop, bop, codebuf, part, recv, bars, total;
+  uint32_t lut, aop, bop, tiles, part, recv, bars, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int C, int RBc, int nchunk) {
+// All code tiles of the CTA's passes stay resident: P * ntile tiles of 8 KB.
+__host__ __device__ inline SmemLayout smem_layout(int C, int P, int RBc, int ntask, int ntile) {
   SmemLayout L;
-  L.lut = 0;                                   // must stay at offset 0 (see lookup addressing)
-  L.aop = L.lut + kLutBytes;                   // 1024-aligned
-  L.bop = L.aop + kAOpBytes;
-  L.codebuf = L.bop + 2 * kBOpBytes;
-  L.part = L.codebuf + kWarps * 2 * kChunkBytes;
-  const int part_count = nchunk * 32 > C * RBc ? nchunk * 32 : C * RBc;
-  const uint32_t part_floats = static_cast<uint32_t>(part_count);
-  L.recv = L.part + ((part_floats * 4 + 15) & ~15u);
+  L.lut = 0;
+  L.aop = L.lut + kLutBytes;                                        // 1024-aligned
+  L.bop = L.aop + kAOpBytes * static_cast<uint32_t>(P);
+  L.tiles = L.bop + 2 * kBOpBytes;
+  L.part = L.tiles + static_cast<uint32_t>(P * ntile) * kTileBytes;
+  const int part_count = ntask * 8 > C * RBc ? ntask * 8 : C * RBc;
+  L.recv = L.part + ((static_cast<uint32_t>(part_count) * 4u + 15u) & ~15u);
   L.bars = L.recv + static_cast<uint32_t>(C * RBc * 4);
-  L.total = L.bars + 64;
+  L.total = L.bars + 8u * static_cast<uint32_t>(P * ntile + 2);
   return L;
+}
+
+// Rows per cluster for a layer: as even a split over Q resident clusters as the
+// shared memory allows (all code tiles of a CTA resident); 0 if not even 64 fit.
+__host__ __device__ inline int rows_per_cluster(int N, int Q, int C, int P) {
+  int RB = (N + Q - 1) / Q;
+  RB = (RB + 7) & ~7;
+  while (RB >= 8) {
+    const int RBc = (((RB + C - 1) / C) + 3) & ~3;
+    if (smem_layout(C, P, RBc, (RB + 7) / 8, (RB + kTileRows - 1) / kTileRows).total <= kSmemLimit) return RB;
+    RB = RB > 64 ? RB - 64 : RB - 8;
+  }
+  return 0;
 }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -96,32 +114,10 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes, uint64_t pol) {
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;"
-               ::"r"(dst), "l"(src), "r"(src_bytes), "l"(pol) : "memory");
+__device__ __forceinline__ void cp_async_16_keep(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-
-// acc + (low or high fp16 half of w), exact conversion and one fp32 rounding.
-__device__ __forceinline__ float add_lo(float acc, uint32_t w) {
-  float r;
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, lo, %2;\n\t}" : "=f"(r) : "r"(w), "f"(acc));
-  return r;
-}
-__device__ __forceinline__ float add_hi(float acc, uint32_t w) {
-  float r;
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, hi, %2;\n\t}" : "=f"(r) : "r"(w), "f"(acc));
-  return r;
-}
-
 // Descriptor of a K-major operand in the no-swizzle canonical layout: 8-row x
 // 16-byte core matrices, the two K halves 128 bytes apart (leading byte
 // offset), consecutive 8-row groups 256 bytes apart (stride byte offset).
@@ -133,7 +129,7 @@ __device__ __forceinline__ uint64_t umma_desc_kmajor_noswizzle(uint32_t smem_byt
   d |= static_cast<uint64_t>(1u) << 46;
   return d;  // layout type 0 (no swizzle), base offset 0
 }
-__device__ __forceinline__ uint32_t kmajor_noswizzle_offset(int row, int khalf) {
+__host__ __device__ inline uint32_t kmajor_noswizzle_offset(int row, int khalf) {
   return static_cast<uint32_t>((row >> 3) * 256 + khalf * 128 + (row & 7) * 16);
 }
 
@@ -151,39 +147,34 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "memory");
 }
 
-// Issue the cp.async copies of one 32-row code chunk (rows row0.., groups
-// gbeg..gbeg+gcnt) into `buf`; bytes outside the rows or groups are zero-filled.
-__device__ __forceinline__ void load_code_chunk(const LutParams& p, uint32_t buf, int row0, int row_end,
-                                                int gbeg, int gcnt, int lane, uint64_t pol) {
-  const size_t row_bytes = static_cast<size_t>(p.G) * 2;
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int id = it * 32 + lane;
-    const int r = id >> 3;
-    const int part = id & 7;
-    const int row = row0 + r;
-    const int valid_groups = gcnt - part * 8;
-    uint32_t bytes = 0;
-    const uint8_t* src = p.codes;
-    if (row < row_end && valid_groups > 0) {
-      bytes = static_cast<uint32_t>(valid_groups >= 8 ? 16 : valid_groups * 2);
-      src = p.codes + static_cast<size_t>(row) * row_bytes + static_cast<size_t>(gbeg) * 2 + part * 16;
-    }
-    cp_async_16(buf + static_cast<uint32_t>(r * 128 + part * 16), src, bytes, pol);
-  }
-  cp_async_commit();
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const LutParams p) {
+// 2D TMA tile load (no multicast) of codes: box = 128 bytes x 8 rows at (x bytes, row y).
+// Rows past N and bytes past the row end arrive as zeros.
+__device__ __forceinline__ void tma_load_code_tile(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                   uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(pol) : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_constant__ CUtensorMap code_map,
+                                                                    const LutParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int C = p.C;
-  const SmemLayout L = smem_layout(C, p.RBc, p.nchunk);
+  const SmemLayout L = smem_layout(C, p.P, p.RBc, p.ntask, p.ntile);
   const uint32_t sbase = smem_addr(smem);
   float* part = reinterpret_cast<float*>(smem + L.part);
   float* recv = reinterpret_cast<float*>(smem + L.recv);
-  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* red_bar = mma_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 2);
+  uint64_t* tile_bar = reinterpret_cast<uint64_t*>(smem + L.bars);   // [P * ntile] tile landed
+  uint64_t* mma_bar = tile_bar + p.P * p.ntile;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -193,24 +184,69 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const LutPara
   const int rb0 = cluster * p.RB;
   const int rb1 = min(p.N, rb0 + p.RB);
   const int nrows = max(0, rb1 - rb0);
-  const int nch = (nrows + 31) >> 5;
-  const uint64_t pol = l2_policy_evict_first();
+  const int nt = (nrows + 7) >> 3;                          // 8-row tasks of this row block
+  const int ntl = (nrows + kTileRows - 1) / kTileRows;      // 64-row tiles of this row block
 
-  // ---- set-up: TMEM, barriers, B operands (both codebooks, K padded to 16) ----
-  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  // passes this CTA runs (gcnt > 0); uniform across the CTA
+  int npass = 0;
+  while (npass < p.P && (static_cast<int>(crank) * p.P + npass) * kGroupsPerPass < p.G) ++npass;
+
+  // ---- 1. barriers; one thread starts the whole code stream (a TMA box per tile) --------
   if (tid == 0) {
+    for (int i = 0; i < p.P * p.ntile; ++i) mbar_init(&tile_bar[i], 1);
     mbar_init(mma_bar, 1);
-    mbar_init(red_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int i = tid; i < 2 * 256; i += kThreads) {
-    const int m = i >> 8, idx = i & 255;
-    const uint4 v = ldg_nc_v4(p.codebooks + (static_cast<size_t>(m) * 256 + idx) * 8);
-    uint8_t* b = smem + L.bop + m * kBOpBytes;
-    *reinterpret_cast<uint4*>(b + kmajor_noswizzle_offset(idx, 0)) = v;
-    *reinterpret_cast<uint4*>(b + kmajor_noswizzle_offset(idx, 1)) = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  if (tid == 32 * (kWarps - 1)) {
+    const uint64_t pol = l2_policy_evict_first();
+    for (int ps = 0; ps < npass; ++ps) {
+      const int gbeg = (static_cast<int>(crank) * p.P + ps) * kGroupsPerPass;
+      for (int tl = 0; tl < ntl; ++tl) {
+        const int i = ps * p.ntile + tl;
+        mbar_arrive_expect_tx(&tile_bar[i], kTileBytes);
+        tma_load_code_tile(sbase + L.tiles + static_cast<uint32_t>(i) * kTileBytes, &code_map, gbeg * 2,
+                           rb0 + tl * kTileRows, &tile_bar[i], pol);
+      }
+    }
   }
-  for (int i = tid; i < p.nchunk * 32; i += kThreads) part[i] = 0.f;
+
+  // scale and bias of the rows this CTA reduces at the end (read now, used last)
+  float row_scale = 0.f, row_bias = 0.f;
+  {
+    const int row = rb0 + static_cast<int>(crank) * p.RBc + tid;
+    if (tid < p.RBc && row < rb1) {
+      row_scale = __half2float(p.scales[row]);
+      row_bias = p.bias ? __half2float(p.bias[row]) : 0.f;
+    }
+  }
+
+  // ---- 2. operands (both codebooks, x of every pass) and TMEM ------------------------------
+  {
+    for (int i = tid; i < 2 * 256; i += kThreads) {
+      const int m = i >> 8, idx = i & 255;
+      const uint32_t bo = L.bop + static_cast<uint32_t>(m) * kBOpBytes;
+      cp_async_16_keep(sbase + bo + kmajor_noswizzle_offset(idx, 0), p.codebooks + (static_cast<size_t>(m) * 256 + idx) * 8, 16);
+      *reinterpret_cast<uint4*>(smem + bo + kmajor_noswizzle_offset(idx, 1)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int i = tid; i < npass * 128; i += kThreads) {  // A row rho (and rho+64) = one group of x
+      const int ps = i >> 7, rho = i & 127;
+      const int gbeg = (static_cast<int>(crank) * p.P + ps) * kGroupsPerPass;
+      const int gg = 2 * (rho & 31) + ((rho >> 5) & 1);
+      const uint32_t ao = L.aop + static_cast<uint32_t>(ps) * kAOpBytes;
+      const bool valid = gbeg + gg < p.G;
+      cp_async_16_keep(sbase + ao + kmajor_noswizzle_offset(rho, 0),
+                       valid ? static_cast<const void*>(p.x + static_cast<size_t>(gbeg + gg) * 8)
+                             : static_cast<const void*>(p.x),
+                       valid ? 16u : 0u);
+      *reinterpret_cast<uint4*>(smem + ao + kmajor_noswizzle_offset(rho, 1)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+    for (int i = tid; i < p.ntask * 8; i += kThreads) part[i] = 0.f;
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -218,148 +254,131 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const LutPara
   const uint32_t idesc = umma_idesc_f16_f32(128, 256);
   uint32_t mma_phase = 0;
   bool ok = true;
+  const int r8 = lane >> 2;  // row of the 8-row task
+  const int q4 = lane & 3;   // quarter of the row's 32 code words
 
-  const uint32_t code_buf0 = sbase + L.codebuf + static_cast<uint32_t>(warp) * 2 * kChunkBytes;
-
-  for (int pass = 0; pass < p.P; ++pass) {
-    const int gbeg = (static_cast<int>(crank) * p.P + pass) * kGroupsPerPass;
-    const int gcnt = min(kGroupsPerPass, p.G - gbeg);
-    if (gcnt <= 0) break;  // uniform across the CTA
-
-    // prefetch this warp's first code chunk while the table is being built
-    if (warp < nch) load_code_chunk(p, code_buf0, rb0 + warp * 32, rb1, gbeg, gcnt, lane, pol);
-
-    // ---- A operand: row rho holds x of group gbeg + 2*(rho % 32) + rho / 32 ----
-    if (tid < 128) {
-      const int rho = tid;
-      const int gg = 2 * (rho & 31) + (rho >> 5);
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (rho < 64 && gg < gcnt) v = ldg_nc_v4(p.x + static_cast<size_t>(gbeg + gg) * 8);
-      *reinterpret_cast<uint4*>(smem + L.aop + kmajor_noswizzle_offset(rho, 0)) = v;
-      *reinterpret_cast<uint4*>(smem + L.aop + kmajor_noswizzle_offset(rho, 1)) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
+  for (int ps = 0; ps < npass; ++ps) {
+    // ---- 3. table of this pass: two MMAs into TMEM ---------------------------------------
     if (tid == 0 && ok) {
       tc_fence_after_sync();
-      const uint64_t adesc = umma_desc_kmajor_noswizzle(sbase + L.aop);
+      const uint64_t adesc = umma_desc_kmajor_noswizzle(sbase + L.aop + static_cast<uint32_t>(ps) * kAOpBytes);
       umma_f16_ss(tmem, adesc, umma_desc_kmajor_noswizzle(sbase + L.bop), idesc, 0u);
       umma_f16_ss(tmem + 256, adesc, umma_desc_kmajor_noswizzle(sbase + L.bop + kBOpBytes), idesc, 0u);
       umma_commit(mma_bar);
     }
-    bool done = ok ? mbar_wait_bounded(mma_bar, mma_phase, p.status, kSiteLutMma) : false;
+    const bool done = ok ? mbar_wait_bounded(mma_bar, mma_phase, p.status, kSiteLutMma) : false;
     mma_phase ^= 1u;
     ok = __syncthreads_and(done ? 1 : 0) != 0;
     tc_fence_after_sync();
 
-    // ---- table: TMEM lanes 0..63 (warps 0,1,4,5) -> fp16 pairs in shared memory ----
-    if (ok && (warp & 3) < 2) {
-      const int rho = 32 * (warp & 3) + lane;  // word column of this thread
-      const int idx0 = (warp >> 2) * 128;
+    // ---- 4. TMEM -> shared-memory table, all 16 warps (A rows rho and rho+64 agree) --------
+    if (ok) {
+      const int qd = warp & 3;
+      const int col = 32 * (qd & 1) + lane;                 // word column = rho mod 64
+      const int i0 = 32 * (2 * (warp >> 2) + (qd >> 1));    // 32 table entries per warp
+      const uint32_t lane_off = static_cast<uint32_t>(32 * qd) << 16;
       uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        const int i0 = idx0 + 32 * c;
-        uint32_t r0[32], r1[32];
-        const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-        tmem_ld_32x32b_x32(tmem + lane_off + static_cast<uint32_t>(i0), r0);
-        tmem_ld_32x32b_x32(tmem + lane_off + 256u + static_cast<uint32_t>(i0), r1);
+      uint32_t r0[32], r1[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + static_cast<uint32_t>(i0), r0);
+      tmem_ld_32x32b_x32(tmem + lane_off + 256u + static_cast<uint32_t>(i0), r1);
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          lut[(i0 + j) * 64 + rho] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
-      }
+      for (int j = 0; j < 32; ++j)
+        lut[(i0 + j) * 64 + col] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
     }
     tc_fence_before_sync();
     __syncthreads();
 
-    // ---- lookups: lane = row of a 32-row chunk, rotated code words ----
-    if (ok) {
-      int it = 0;
-      for (int ch = warp; ch < nch; ch += kWarps, ++it) {
-        const uint32_t buf = code_buf0 + static_cast<uint32_t>(it & 1) * kChunkBytes;
-        const int next = ch + kWarps;
-        if (next < nch) {
-          load_code_chunk(p, code_buf0 + static_cast<uint32_t>((it + 1) & 1) * kChunkBytes,
-                          rb0 + next * 32, rb1, gbeg, gcnt, lane, pol);
-          cp_async_wait<1>();
-        } else {
-          cp_async_wait<0>();
+    {
+      // ---- 5. lookups: a task is 8 rows; 4 lanes per row, 8 code words each -------------------
+      // Lane (r8, q4) reads code word w = 8*q4 + ((r8 + s) mod 8) at step s: the 32 lanes
+      // always touch 32 distinct words, so both the code reads and the table reads are
+      // free of bank conflicts.  Pairs of looked-up fp16 values are added as half2 and
+      // the task's 16 pair sums are accumulated in half2, then widened to fp32.
+      for (int t = warp; t < nt; t += kWarps) {
+        const int i = ps * p.ntile + t / 8;  // tile holding rows 8t .. 8t+7
+        const bool landed = mbar_wait_bounded(&tile_bar[i], 0u, p.status, kSiteLutCodes);
+        if (ok && landed) {
+          const uint32_t* cw_row = reinterpret_cast<const uint32_t*>(
+              smem + L.tiles + i * kTileBytes + ((t & 7) * 8 + r8) * 128);
+          uint32_t cw[8];
+#pragma unroll
+          for (int s8 = 0; s8 < 8; ++s8) cw[s8] = cw_row[8 * q4 + ((r8 + s8) & 7)];
+          __half2 hacc = __float2half2_rn(0.f);
+#pragma unroll
+          for (int s8 = 0; s8 < 8; ++s8) {
+            const uint32_t wv = static_cast<uint32_t>((8 * q4 + ((r8 + s8) & 7)) << 2);  // 4 * code word
+            // table byte offsets: entry * 256 + column * 4 (column w, or 32 + w at +128)
+            const uint32_t t0 = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(cw[s8], wv, 0x5504));
+            const uint32_t t1 = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(cw[s8], wv, 0x5514));
+            const uint32_t t2 = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(cw[s8], wv, 0x5524) + 128u);
+            const uint32_t t3 = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(cw[s8], wv, 0x5534) + 128u);
+            // (codebook-0 value of t0, codebook-1 value of t1) and likewise for t2, t3
+            const uint32_t p01 = __byte_perm(t0, t1, 0x7610);
+            const uint32_t p23 = __byte_perm(t2, t3, 0x7610);
+            hacc = __hadd2(hacc, __hadd2(*reinterpret_cast<const __half2*>(&p01),
+                                         *reinterpret_cast<const __half2*>(&p23)));
+          }
+          const float2 f = __half22float2(hacc);
+          float v = f.x + f.y;
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          if (q4 == 0) part[t * 8 + r8] += v;
+        } else if (!landed) {
+          ok = false;
         }
-        __syncwarp();
-        const uint32_t row_buf = buf + static_cast<uint32_t>(lane) * 128u;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-        for (int s = 0; s < 32; ++s) {
-          const uint32_t wv = static_cast<uint32_t>(((lane + s) & 31) << 2);   // 4 * code word
-          const uint32_t cw = lds32(row_buf + wv);
-          // byte offsets into the table (it starts at shared offset 0): entry * 256 + column * 4
-          const uint32_t o0 = __byte_perm(cw, wv, 0x5504);
-          const uint32_t o1 = __byte_perm(cw, wv, 0x5514);
-          const uint32_t o2 = __byte_perm(cw, wv, 0x5524);
-          const uint32_t o3 = __byte_perm(cw, wv, 0x5534);
-          a0 = add_lo(a0, lds32(sbase + o0));
-          a1 = add_hi(a1, lds32(sbase + o1));
-          a2 = add_lo(a2, lds32(sbase + o2 + 128u));
-          a3 = add_hi(a3, lds32(sbase + o3 + 128u));
-        }
-        part[ch * 32 + lane] += (a0 + a1) + (a2 + a3);
-        __syncwarp();
       }
     }
     // the next pass rebuilds the table: every warp must be done reading it
-    __syncthreads();
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
   }
 
-  cp_async_wait<0>();  // no copy may still be in flight when the CTA moves on
-
-  // ---- cluster reduction of the row partials ----------------------------------
+  // ---- 6. partials -> their owner CTA (remote shared-memory stores), one cluster barrier ----
+  // Row r of the block is reduced by CTA r / RBc; this CTA's partial of it lands in
+  // the owner's recv[crank][r mod RBc].  After the barrier every owner holds all C
+  // partials of its rows and no CTA touches another CTA's memory any more.
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
-  const uint32_t slice_bytes = static_cast<uint32_t>(p.RBc) * 4u;
-  if (tid == 0) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                 ::"r"(smem_addr(red_bar)), "r"(slice_bytes * static_cast<uint32_t>(C)) : "memory");
+  for (int v4 = tid; v4 * 4 < p.RBc * C; v4 += kThreads) {
+    const int r = v4 * 4;  // 4 consecutive rows, never split between owners (RBc % 4 == 0)
+    const uint32_t owner = static_cast<uint32_t>(r / p.RBc);
+    const float4 val = *reinterpret_cast<const float4*>(part + r);
+    const uint32_t dst = mapa_shared(sbase + L.recv + (crank * static_cast<uint32_t>(p.RBc) +
+                                                       static_cast<uint32_t>(r - static_cast<int>(owner) * p.RBc)) * 4u,
+                                     owner);
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(dst), "f"(val.x), "f"(val.y), "f"(val.z), "f"(val.w) : "memory");
   }
-  fence_proxy_async_smem();
-  cluster_sync_all();  // partials final everywhere, every receive barrier armed
-  if (tid < C) {
-    const uint32_t dst_rank = static_cast<uint32_t>(tid);
-    const uint32_t src = sbase + L.part + dst_rank * slice_bytes;
-    const uint32_t dst = mapa_shared(sbase + L.recv + crank * slice_bytes, dst_rank);
-    const uint32_t bar = mapa_shared(smem_addr(red_bar), dst_rank);
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "r"(src), "r"(slice_bytes), "r"(bar) : "memory");
-  }
-  const bool got = mbar_wait_bounded(red_bar, 0, p.status, kSiteLutReduce);
-  if (got && ok) {
+  cluster_sync_all();
+  if (ok) {
     for (int r = tid; r < p.RBc; r += kThreads) {
       const int row = rb0 + static_cast<int>(crank) * p.RBc + r;
       if (row >= rb1) break;
       float s = 0.f;
       for (int c = 0; c < C; ++c) s += recv[c * p.RBc + r];
-      const float bi = p.bias ? __half2float(p.bias[row]) : 0.f;
-      p.y[row] = __float2half_rn(s * __half2float(p.scales[row]) + bi);
+      const float sc = (r == tid) ? row_scale : __half2float(p.scales[row]);
+      const float bi = (r == tid) ? row_bias : (p.bias ? __half2float(p.bias[row]) : 0.f);
+      p.y[row] = __float2half_rn(s * sc + bi);
     }
   }
-  cluster_sync_all();  // no CTA leaves while a peer's copy may still read its memory
 }
 
 struct Plan {
-  int C, P, Q;
+  int C, P, Q, RB;
 };
 
 // The cost model picks (cluster size C, passes P) for a layer: P passes of 64
-// groups per CTA, C = ceil(G / 64P) <= 16 CTAs per cluster, Q clusters resident.
-// Cost per CTA (cycles): rows * 128P lookups at ~24 per cycle plus ~600 per pass
-// to build and store the table.
-int plan_cost(int N, int C, int P, int Q) {
-  const int rows = (N + Q - 1) / Q;
-  return rows * 128 * P / 24 + 600 * P;
+// groups per CTA, C = ceil(G / 64P) <= 16 CTAs per cluster, Q clusters resident,
+// RB rows per cluster (fewer than N / Q when the code tiles would not fit, which
+// costs extra waves).  Cycles per CTA: rows * 128P lookups at ~24 per cycle plus
+// ~600 per pass to build and store the table.
+int plan_cost(int N, int P, int Q, int RB) {
+  const int clusters = (N + RB - 1) / RB;
+  const int waves = (clusters + Q - 1) / Q;
+  return waves * (RB * 128 * P / 24 + 600 * P);
 }
 
 // Chooses (C, P, Q) for a layer on the current device; cached per (device, N, K).
@@ -378,16 +397,14 @@ cudaError_t lut_plan(int dev, int N, int G, Plan* out) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   const int cmax = (e == cudaSuccess) ? 16 : 8;
   cudaGetLastError();
-  Plan best{0, 0, 0};
+  Plan best{0, 0, 0, 0};
   int best_cost = 0;
-  for (int P = 1; P <= 64; ++P) {
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
+  if (e != cudaSuccess) return e;
+  for (int P = 1; P <= kMaxPasses; ++P) {
     const int C = (G + 64 * P - 1) / (64 * P);
     if (C > cmax) continue;
-    const int RB_guess = (N + 7) / 8;
-    const int RBc_guess = (((RB_guess + C - 1) / C) + 3) & ~3;
-    const SmemLayout Lg = smem_layout(C, RBc_guess, (RB_guess + 31) / 32);
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Lg.total));
-    if (e != cudaSuccess) return e;
+    // one CTA per SM (its TMEM and shared memory), so residency is set by cluster placement
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -396,7 +413,7 @@ cudaError_t lut_plan(int dev, int N, int G, Plan* out) {
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(static_cast<unsigned>(C), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = Lg.total;
+    cfg.dynamicSmemBytes = kSmemLimit;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int q = 0;
@@ -406,9 +423,15 @@ cudaError_t lut_plan(int dev, int N, int G, Plan* out) {
       if (C == 1) break;
       continue;
     }
-    const int cost = plan_cost(N, C, P, q);
+    q = std::min(q, std::max(1, (N + 31) / 32));
+    const int RB = rows_per_cluster(N, q, C, P);
+    if (RB == 0) {
+      if (C == 1) break;
+      continue;
+    }
+    const int cost = plan_cost(N, P, q, RB);
     if (best.C == 0 || cost < best_cost) {
-      best = Plan{C, P, q};
+      best = Plan{C, P, q, RB};
       best_cost = cost;
     }
     if (C == 1) break;
@@ -420,10 +443,28 @@ cudaError_t lut_plan(int dev, int N, int G, Plan* out) {
   return cudaSuccess;
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
 }  // namespace
 
 bool gemv_lut_supported(int M, int B, int g, int K, int batch) {
-  return M == 2 && B == 8 && g == 8 && batch == 1 && K % 64 == 0;
+  return M == 2 && B == 8 && g == 8 && batch == 1 && K % 64 == 0 && K <= 16 * kMaxPasses * kGroupsPerPass * 8;
 }
 
 cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t stream) {
@@ -436,9 +477,22 @@ cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t st
   if (e != cudaSuccess) return e;
   auto kern = gemv_lut_2x8_kernel;
 
+  // Codes as a 2D byte tensor [N rows][2G bytes]; a box is 64 rows x 128 bytes
+  // (one 64-group pass of 64 rows).  Out-of-range rows and bytes read as zero.
+  EncodeTiledFn encode = encode_tiled();
+  if (!encode) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(G) * 2, static_cast<cuuint64_t>(pr.N)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(G) * 2};
+  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kTileRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pr.codes), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
   LutParams p{};
   p.x = static_cast<const __half*>(pr.x);
-  p.codes = static_cast<const uint8_t*>(pr.codes);
   p.codebooks = static_cast<const __half*>(pr.codebooks);
   p.scales = static_cast<const __half*>(pr.scales);
   p.bias = static_cast<const __half*>(pr.bias);
@@ -448,12 +502,12 @@ cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t st
   p.G = G;
   p.C = best.C;
   p.P = best.P;
-  const int Q = std::max(1, std::min(best.Q, (pr.N + 31) / 32));
-  p.RB = (pr.N + Q - 1) / Q;
+  p.RB = best.RB;
   p.RBc = (((p.RB + p.C - 1) / p.C) + 3) & ~3;
-  p.nchunk = (p.RB + 31) / 32;
+  p.ntask = (p.RB + 7) / 8;
+  p.ntile = (p.RB + kTileRows - 1) / kTileRows;
   p.status = status;
-  const SmemLayout L = smem_layout(p.C, p.RBc, p.nchunk);
+  const SmemLayout L = smem_layout(p.C, p.P, p.RBc, p.ntask, p.ntile);
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
   if (e != cudaSuccess) return e;
   const int clusters = (pr.N + p.RB - 1) / p.RB;
@@ -470,7 +524,7 @@ cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t st
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return cudaLaunchKernelEx(&cfg, kern, map, p);
 }
 
 }  // namespace aqlm
