@@ -60,6 +60,9 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    p.add_argument("--layer", default=None, help="time only this layer of the workload (e.g. q_proj)")
+    p.add_argument("--pool", type=int, default=None,
+                   help="rotating-pool copies (default: enough to exceed 3x L2); smaller for profiler captures")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be at least 3")
@@ -83,8 +86,59 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
+KERNEL_SOURCES = {"gemv_gather_kernel": "gemv.cu", "gemv_lut_2x8_kernel": "gemv_lut.cu",
+                  "tc_decode_mma_kernel": "tc_gemm.cu"}
+
+
+def measured_traffic(workload_name, kernel):
+    """DRAM bytes per launch (read + write) of `kernel` on this workload, from the ncu
+    capture recorded in profiles/roofline_traffic.json -- or None when there is none or
+    the kernel's source changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
+        return None
+    with open(path) as fh:
+        rec = json.load(fh).get(workload_name)
+    if not rec or rec.get("kernel") != kernel:
+        return None
+    src = os.path.join(ROOT, "weight_only_additive_b200", "csrc", KERNEL_SOURCES[kernel])
+    with open(src, "rb") as fh:
+        if hashlib.sha256(fh.read()).hexdigest() != rec.get("source_sha256"):
+            return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def workload_batch(w, override):
     return override if override is not None else w.batches[0]
+
+
+def select_workload(a):
+    """The named workload, restricted to one layer when --layer is given."""
+    w = workloads.get(a.workload)
+    if a.layer is None:
+        return w
+    layers = tuple(l for l in w.layers if l.name == a.layer)
+    if not layers:
+        raise SystemExit(f"--layer {a.layer!r} is not a layer of {w.name}: {[l.name for l in w.layers]}")
+    idx = [i for i, l in enumerate(w.layers) if l.name == a.layer][0]
+    return workloads.Workload(w.index, f"{w.name}/{a.layer}", layers, w.batches, w.description,
+                              extra={"layer_offset": idx})
+
+
+def max_over_ranks(ms, dist, device):
+    """The slowest rank's time: every rank takes part, every rank gets the max."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput_gbs(bytes_per_step, steps, world, ms):
+    """Whole-job GB/s: the algorithmic bytes all ranks processed / the slowest rank's time."""
+    return bytes_per_step * steps * world / (ms / 1e3) / 1e9
 
 
 def step_bytes(w, batch):
@@ -172,7 +226,8 @@ def host_layers(w, batch):
 
 
 def oracle_sample_run(w, batch, seconds, copy=0):
-    """Times oracle.linear (decode + fp64 matmul) on row samples of every layer.
+    """Times oracle.linear (decode + fp64 matmul) on row samples of every layer, repeating
+    the sample until about `seconds` of CPU time have been spent.
     Returns (algorithmic bytes of the sampled fraction, seconds, rows per layer, threads)."""
     import oracle
 
@@ -183,21 +238,25 @@ def oracle_sample_run(w, batch, seconds, copy=0):
         oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=np.arange(8))
     probe = (time.perf_counter() - t0) / 8.0  # seconds per "one row of every layer"
     rows = max(1, int(seconds / max(probe, 1e-9)))
-    total_bytes, elapsed = 0.0, 0.0
+    total_bytes, elapsed, sampled = 0.0, 0.0, 0
     rng = np.random.Generator(np.random.PCG64(copy))
-    for lay, ld, x in layers:
-        r = min(rows, lay.N)
-        sel = np.sort(rng.choice(lay.N, size=r, replace=False))
-        t0 = time.perf_counter()
-        oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=sel)
-        elapsed += time.perf_counter() - t0
-        total_bytes += lay.algorithmic_bytes(batch) * (r / lay.N)
-    return total_bytes, elapsed, rows, oracle.max_threads()
+    while True:
+        for lay, ld, x in layers:
+            r = min(rows, lay.N)
+            sel = np.sort(rng.choice(lay.N, size=r, replace=False))
+            t0 = time.perf_counter()
+            oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=sel)
+            elapsed += time.perf_counter() - t0
+            total_bytes += lay.algorithmic_bytes(batch) * (r / lay.N)
+        sampled += rows
+        if elapsed >= 0.9 * seconds:
+            break
+    return total_bytes, elapsed, sampled, oracle.max_threads()
 
 
 def run_reference(a):
     rank, world, _ = env_rank()
-    w = workloads.get(a.workload)
+    w = select_workload(a)
     batch = workload_batch(w, a.batch)
     if rank != 0:
         return 0
@@ -249,13 +308,13 @@ def run_ours(a):
     dev = torch.device("cuda", local)
     lib = native.lib()
 
-    w = workloads.get(a.workload)
+    w = select_workload(a)
     batch = workload_batch(w, a.batch)
     sbytes = step_bytes(w, batch)
     props = torch.cuda.get_device_properties(dev)
     l2 = getattr(props, "L2_cache_size", 0) or L2_FALLBACK
     copy_bytes = sum(l.algorithmic_bytes(batch) for l in w.layers)
-    pool = max(2, math.ceil(3 * l2 / copy_bytes))
+    pool = max(2, math.ceil(3 * l2 / copy_bytes)) if a.pool is None else max(1, a.pool)
     while pool > 2 and pool * copy_bytes > 60e9:
         pool -= 1
 
@@ -266,7 +325,7 @@ def run_ours(a):
         for li, lay in enumerate(w.layers):
             s = lay.scheme
             ld = synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index,
-                                  layer=li, copy=c + 1000 * rank)
+                                  layer=li + w.extra.get("layer_offset", 0), copy=c + 1000 * rank)
             wc.append(L.AqlmWeights.from_numpy(ld, dev))
             xc.append(torch.from_numpy(synth.make_x(batch, lay.K, seed=0, workload=w.index, layer=li,
                                                     copy=c + 1000 * rank)).to(dev))
@@ -328,28 +387,24 @@ def run_ours(a):
             end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-    ms = start.elapsed_time(end)
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dist, dev)
     st, detail = L.check_device_status(stream=stream)
     if st != native.Status.OK:
         raise RuntimeError(f"device status {st.name} {detail:#x}")
 
     launches_per_step = len(w.layers)
-    total_bytes = sbytes * a.steps * world
-    value = total_bytes / (ms / 1e3) / 1e9
+    value = job_throughput_gbs(sbytes, a.steps, world, ms)
     ms_step = ms / a.steps
     peaks = measured_peaks()
     avg_launch_s = (ms / 1e3) / (a.steps * launches_per_step)
     bytes_per_launch = sbytes / launches_per_step
     achieved = bytes_per_launch / avg_launch_s / 1e9
-    kernel_names = {int(Path.GEMV): "gemv_gather_kernel", int(Path.GEMV_LUT): "gemv_lut_kernel",
+    kernel_names = {int(Path.GEMV): "gemv_gather_kernel", int(Path.GEMV_LUT): "gemv_lut_2x8_kernel",
                     int(Path.TENSOR_CORE): "tc_decode_mma_kernel"}
+    kernel = kernel_names.get(paths[0], "?")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "kernel": kernel_names.get(paths[0], "?"),
+                "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(w.name, kernel),
+                "kernel": kernel,
                 "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
                 if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
 
@@ -381,12 +436,8 @@ def run_ours(a):
                     hy[li].copy_(ys[li], non_blocking=True)
             e1.record(stream)
         torch.cuda.synchronize(dev)
-        ems = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": sbytes * e2e_steps * world / (ems / 1e3) / 1e9, "unit": "GB/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        e2e = {"value": job_throughput_gbs(sbytes, e2e_steps, world, ems), "unit": "GB/s",
                "h2d_bytes_per_step": sum(t.numel() * 2 for t in hx),
                "d2h_bytes_per_step": sum(t.numel() * 2 for t in hy),
                "steps": e2e_steps, "us_per_layer": ems * 1e3 / (e2e_steps * len(w.layers)),
@@ -398,8 +449,9 @@ def run_ours(a):
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         b, s, rows, threads = oracle_sample_run(w, batch, a.cpu_seconds)
         cpu = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"{rows} sampled rows of each of the {len(w.layers)} layers "
-                         f"(decode to fp16 + fp64 matmul), batch {batch}, {s:.1f} s"}
+               "sample": f"{rows} rows of each of the {len(w.layers)} layers (whole layers repeated "
+                         f"when the budget exceeds them; decode to fp16 + fp64 matmul), batch {batch}, "
+                         f"{s:.1f} s on the host cores"}
 
     if dist is not None:
         del graphs
