@@ -66,6 +66,22 @@ aqlm_status validate_shape(int M, int B, int g, int K, int N, int batch) {
 
 }  // namespace
 
+namespace aqlm {
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+}  // namespace aqlm
+
 extern "C" {
 
 int aqlm_abi_version(void) { return 1; }

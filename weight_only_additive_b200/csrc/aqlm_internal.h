@@ -2,6 +2,7 @@
 // Host code only calls these after aqlm_validate-style checks have passed.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,6 +17,10 @@ enum : uint32_t {
   kSiteTcMmaDone = 0x101,   // tensor-core kernel: waiting for an MMA commit
   kSiteLutMma = 0x201,      // lookup-table GEMV: waiting for the table-building MMA
   kSiteLutCodes = 0x202,    // lookup-table GEMV: code-tile pipeline (TMA landing / slot release)
+  kSitePipeFull = 0x301,    // pipelined tensor-core kernel: waiting for a decoded/loaded stage
+  kSitePipeEmpty = 0x302,   // pipelined tensor-core kernel: waiting for a stage to be released
+  kSitePipeCodes = 0x303,   // pipelined tensor-core kernel: code-tile ring
+  kSitePipeAcc = 0x304,     // pipelined tensor-core kernel: waiting for the accumulator
 };
 
 struct Problem {
@@ -37,6 +42,17 @@ cudaError_t launch_gemv_lut(const Problem& p, uint32_t* status, cudaStream_t str
 // True if the lookup-table GEMV handles this problem (2x8 g8, batch 1, K % 64 == 0).
 bool gemv_lut_supported(int M, int B, int g, int K, int batch);
 cudaError_t launch_tc(const Problem& p, uint32_t* status, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled from the driver (through the runtime's entry-point
+// query, so the library does not link libcuda); nullptr if unavailable.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled();
+
+// Pipelined decode -> tcgen05 kernel; cudaErrorNotSupported when the shape is
+// outside what it handles (the caller then uses the single-stage kernel).
+cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t stream);
 
 // True if the scheme is one the kernels are instantiated for.
 inline bool scheme_supported(int M, int B, int g) {

@@ -114,9 +114,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ void cp_async_16_keep(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 // Descriptor of a K-major operand in the no-swizzle canonical layout: 8-row x
 // 16-byte core matrices, the two K halves 128 bytes apart (leading byte
@@ -145,23 +142,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr)
       : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
-}
-
-// 2D TMA tile load (no multicast) of codes: box = 128 bytes x 8 rows at (x bytes, row y).
-// Rows past N and bytes past the row end arrive as zeros.
-__device__ __forceinline__ void tma_load_code_tile(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                                   uint64_t* bar, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;"
-      ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(pol) : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_constant__ CUtensorMap code_map,
@@ -205,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
       for (int tl = 0; tl < ntl; ++tl) {
         const int i = ps * p.ntile + tl;
         mbar_arrive_expect_tx(&tile_bar[i], kTileBytes);
-        tma_load_code_tile(sbase + L.tiles + static_cast<uint32_t>(i) * kTileBytes, &code_map, gbeg * 2,
+        tma_load_2d(sbase + L.tiles + static_cast<uint32_t>(i) * kTileBytes, &code_map, gbeg * 2,
                            rb0 + tl * kTileRows, &tile_bar[i], pol);
       }
     }
@@ -226,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
     for (int i = tid; i < 2 * 256; i += kThreads) {
       const int m = i >> 8, idx = i & 255;
       const uint32_t bo = L.bop + static_cast<uint32_t>(m) * kBOpBytes;
-      cp_async_16_keep(sbase + bo + kmajor_noswizzle_offset(idx, 0), p.codebooks + (static_cast<size_t>(m) * 256 + idx) * 8, 16);
+      cp_async_16_zfill(sbase + bo + kmajor_noswizzle_offset(idx, 0), p.codebooks + (static_cast<size_t>(m) * 256 + idx) * 8, 16);
       *reinterpret_cast<uint4*>(smem + bo + kmajor_noswizzle_offset(idx, 1)) = make_uint4(0u, 0u, 0u, 0u);
     }
     for (int i = tid; i < npass * 128; i += kThreads) {  // A row rho (and rho+64) = one group of x
@@ -235,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
       const int gg = 2 * (rho & 31) + ((rho >> 5) & 1);
       const uint32_t ao = L.aop + static_cast<uint32_t>(ps) * kAOpBytes;
       const bool valid = gbeg + gg < p.G;
-      cp_async_16_keep(sbase + ao + kmajor_noswizzle_offset(rho, 0),
+      cp_async_16_zfill(sbase + ao + kmajor_noswizzle_offset(rho, 0),
                        valid ? static_cast<const void*>(p.x + static_cast<size_t>(gbeg + gg) * 8)
                              : static_cast<const void*>(p.x),
                        valid ? 16u : 0u);
@@ -441,24 +421,6 @@ cudaError_t lut_plan(int dev, int N, int G, Plan* out) {
   cache[std::make_tuple(dev, N, G)] = best;
   *out = best;
   return cudaSuccess;
-}
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-    cudaGetLastError();
-  });
-  return fn;
 }
 
 }  // namespace

@@ -1,0 +1,489 @@
+// Pipelined batch >= 16 path: codeword decode into shared memory overlapped with
+// 5th-generation tensor-core MMAs (tcgen05.mma kind::f16, fp32 accumulator in TMEM).
+//
+// "Dequantize-to-FP16 then an FP16 tensor-core GEMM" (inference-research record
+// "AQLM (additive / multi-codebook quantization)", notes), fused so the fp16
+// weights exist only as 128 x 64 shared-memory tiles.  Swap-AB: the MMA's M is
+// 128 weight rows, its N is the batch tile (16..256), so D[n, b] lands in TMEM
+// with one weight row per lane.
+//
+// Warp roles (224 threads):
+//   warps 0-3  decoders, then epilogue.  Thread r owns weight row n0 + r.  Per
+//              64-wide K stage it reads its 8 (g = 8) or 4 (g = 16) codes from the
+//              code tile and writes the row's 128 bytes of the A stage in the
+//              128-byte-swizzled K-major layout:
+//                1x16: the codeword is the fp16 data, so each 16-byte piece is one
+//                      cp.async gather from the (L2-resident) codebook straight into
+//                      its swizzled slot, tracked by cp.async.mbarrier.arrive;
+//                2x8:  the two codewords come from the codebooks staged in shared
+//                      memory, are added in fp32, rounded once to fp16 and stored.
+//   warp 4     TMA producer of x tiles (B operand, 128-byte swizzle, zero-filled
+//              past the batch and K edges).
+//   warp 5     MMA issuer: 4 x (128 x BN x 16) per stage, commit releases the stage.
+//   warp 6     TMA producer of code tiles (128 rows x 64 bytes = 4 or 8 stages).
+// Epilogue: tcgen05.ld of 16 columns at a time, y = s_n * D + bias_n -> fp16.
+#include <cuda.h>
+
+#include <type_traits>
+
+#include "aqlm_device.cuh"
+
+namespace aqlm {
+namespace {
+
+constexpr int kRows = 128;            // MMA M: weight rows per CTA
+constexpr int kStageK = 64;           // K per stage (one 128-byte swizzle row of fp16)
+constexpr int kDecoders = 256;        // warps 0-7: two threads per weight row
+constexpr int kThreads = 352;         // + x producer, MMA issuer, code producer
+constexpr int kWarpX = 8, kWarpMma = 9, kWarpCodes = 10;
+constexpr uint32_t kABytes = kRows * 128u;   // 16 KB per A stage
+constexpr uint32_t kCodeRowBytes = 64u;      // code bytes per row per code tile
+constexpr uint32_t kCodeTileBytes = kRows * kCodeRowBytes;  // 8 KB
+constexpr int kCodeSlots = 4;
+constexpr uint32_t kSmemLimit = 227u * 1024u;
+
+struct PipeParams {
+  const __half* codebooks;
+  const __half* scales;
+  const __half* bias;
+  __half* y;
+  int K, N, batch;
+  int BN;          // batch tile (multiple of 16, <= 256)
+  int nk;          // K / 64 stages (whole K)
+  int S;           // A/B stage ring depth
+  int SK;          // CTAs splitting K (cluster size along z): 1, 2 or 4
+  int ct_per;      // code tiles per K split
+  uint32_t tmem_cols;
+  uint32_t* status;
+};
+
+struct PipeLayout {
+  uint32_t a, b, codes, cb, bars, total;
+};
+
+__host__ __device__ inline PipeLayout pipe_layout(int S, int BN, bool smem_codebook) {
+  PipeLayout L;
+  L.a = 0;                                                          // 1024-aligned stages
+  L.b = L.a + static_cast<uint32_t>(S) * kABytes;
+  L.codes = L.b + static_cast<uint32_t>(S) * static_cast<uint32_t>(BN) * 128u;
+  L.cb = L.codes + kCodeSlots * kCodeTileBytes;
+  L.bars = L.cb + (smem_codebook ? 2u * 256u * 16u : 0u);
+  // full[S], empty[S], code_full[kCodeSlots], code_empty[kCodeSlots], acc, tmem slot, abort flag
+  L.total = L.bars + 8u * static_cast<uint32_t>(2 * S + 2 * kCodeSlots + 1) + 16u;
+  return L;
+}
+
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+  __half2 r = __hadd2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ uint32_t mapa_shared_cluster(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t swz128(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// Bounded wait that also gives up at once when another role has aborted.
+__device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                          uint32_t* status, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      record_failure(status, site);
+      *abort_flag = 1u;
+      return false;
+    }
+  }
+  return true;
+}
+
+// Decode half (`hf` = 0: chunks 0-3, 1: chunks 4-7) of one 64-wide K stage of
+// weight row `r` into the swizzled A stage at shared offset `a_off`.  `cw` points
+// at this stage's codes of the row.
+template <int M, int B, int G>
+__device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase, uint32_t a_off, int r, int hf,
+                                                  bool row_valid, const uint8_t* cw,
+                                                  const __half* __restrict__ codebooks, const uint8_t* smem_cb) {
+  if constexpr (M == 1) {
+    // 1x16: each 16-byte piece of the row is (part of) one codeword: gather it.
+    const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const int chunk = 4 * hf + cc;
+      const int j = chunk / (G / 8), h = chunk % (G / 8);
+      const uint32_t code = c16[j];
+      const __half* src = codebooks + static_cast<size_t>(code) * G + 8 * h;
+      cp_async_16_zfill(sbase + a_off + swz128(r, chunk),
+                        row_valid ? static_cast<const void*>(src) : static_cast<const void*>(codebooks),
+                        row_valid ? 16u : 0u);
+    }
+  } else {
+    // 2x8: codes (c0, c1) per group; codebooks staged in shared memory as [2][256][8].
+    // The two codewords are added as half2 (one rounding of their exact sum).
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const int j = 4 * hf + cc;
+      uint4 out = make_uint4(0u, 0u, 0u, 0u);
+      if (row_valid) {
+        const uint4 q0 = *reinterpret_cast<const uint4*>(smem_cb + (static_cast<uint32_t>(cw[2 * j]) << 4));
+        const uint4 q1 = *reinterpret_cast<const uint4*>(smem_cb + 4096u + (static_cast<uint32_t>(cw[2 * j + 1]) << 4));
+        out.x = hadd2_u32(q0.x, q1.x);
+        out.y = hadd2_u32(q0.y, q1.y);
+        out.z = hadd2_u32(q0.z, q1.z);
+        out.w = hadd2_u32(q0.w, q1.w);
+      }
+      *reinterpret_cast<uint4*>(smem + a_off + swz128(r, j)) = out;
+    }
+  }
+}
+
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int M, int B, int G>
+__global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_constant__ CUtensorMap x_map,
+                                                              const __grid_constant__ CUtensorMap code_map,
+                                                              const PipeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // stages must be 1024-byte aligned for the 128-byte swizzle
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  constexpr bool kSmemCb = (M == 2);
+  constexpr int kStageCodeBytes = (kStageK / G) * M * (B <= 8 ? 1 : 2);  // 16 (g8) or 8 (g16)
+  constexpr int kStagesPerTile = static_cast<int>(kCodeRowBytes) / kStageCodeBytes;
+  const int S = p.S;
+  const PipeLayout L = pipe_layout(S, p.BN, kSmemCb);
+  const uint32_t sbase = smem_addr(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);   // stage s decoded and x landed
+  uint64_t* empty = full + S;                                     // stage s consumed by the MMAs
+  uint64_t* cfull = empty + S;                                    // code tile landed
+  uint64_t* cempty = cfull + kCodeSlots;                          // code tile read by the 8 decoder warps
+  uint64_t* acc_bar = cempty + kCodeSlots;                        // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int n0 = blockIdx.x * kRows;
+  const int b0 = blockIdx.y * p.BN;
+  const int split = blockIdx.z;  // == rank in the (1, 1, SK) cluster
+  // this CTA's K range, in whole code tiles: tiles [ct0, ct1), stages [ks0, ks1)
+  const int nct_all = (p.nk + kStagesPerTile - 1) / kStagesPerTile;
+  const int ct0 = split * p.ct_per;
+  const int ct1 = min(nct_all, ct0 + p.ct_per);
+  const int ks0 = ct0 * kStagesPerTile;
+  const int ks1 = min(p.nk, ct1 * kStagesPerTile);
+  const int nks = max(0, ks1 - ks0);  // host guarantees >= 1
+
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], kDecoders + 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < kCodeSlots; ++i) {
+      mbar_init(&cfull[i], 1);
+      mbar_init(&cempty[i], kDecoders / 32);
+    }
+    mbar_init(acc_bar, 1);
+    *abort_flag = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if constexpr (kSmemCb) {
+    for (int i = tid; i < 2 * 256; i += kThreads)
+      *reinterpret_cast<uint4*>(smem + L.cb + 16u * static_cast<uint32_t>(i)) = ldg_nc_v4(p.codebooks + 8 * i);
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, p.tmem_cols);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kWarpX) {
+    // ---- x tiles (B operand): reused by every CTA, keep them in L2 ----
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_last();
+      for (int i = 0; i < nks; ++i) {
+        const int s = i % S, u = i / S;
+        if (u > 0 && !pipe_wait(&empty[s], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeEmpty))
+          break;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.BN) * 128u);
+        tma_load_2d(sbase + L.b + static_cast<uint32_t>(s * p.BN) * 128u, &x_map, (ks0 + i) * kStageK, b0, &full[s],
+                    pol);
+      }
+    }
+  } else if (warp == kWarpCodes) {
+    // ---- code tiles: 128 rows x 64 bytes, read once ----
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      for (int t = 0; t < ct1 - ct0; ++t) {
+        const int c = t % kCodeSlots, u = t / kCodeSlots;
+        if (u > 0 && !pipe_wait(&cempty[c], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeCodes))
+          break;
+        mbar_arrive_expect_tx(&cfull[c], kCodeTileBytes);
+        tma_load_2d(sbase + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes, &code_map,
+                    (ct0 + t) * static_cast<int>(kCodeRowBytes), n0, &cfull[c], pol);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ---- one thread issues the MMAs; each stage's commit releases it ----
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16_f32(kRows, static_cast<uint32_t>(p.BN));
+      for (int i = 0; i < nks; ++i) {
+        const int s = i % S;
+        if (!pipe_wait(&full[s], static_cast<uint32_t>((i / S) & 1), abort_flag, p.status, kSitePipeFull)) break;
+        fence_proxy_async_smem();  // decoder writes (cp.async / st.shared) -> tensor-core reads
+        tc_fence_after_sync();
+        const uint64_t adesc = umma_desc_sw128_kmajor(sbase + L.a + static_cast<uint32_t>(s) * kABytes);
+        const uint64_t bdesc = umma_desc_sw128_kmajor(sbase + L.b + static_cast<uint32_t>(s * p.BN) * 128u);
+#pragma unroll
+        for (int kk = 0; kk < kStageK / 16; ++kk)
+          umma_f16_ss(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(acc_bar);
+    }
+  } else {
+    // ---- decoders: threads r and r + 128 share weight row n0 + r (chunks 0-3 / 4-7) ----
+    const int r = tid & (kRows - 1);
+    const int hf = tid >> 7;
+    const bool row_valid = n0 + r < p.N;
+    for (int i = 0; i < nks; ++i) {
+      const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
+      // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
+      bool ready = true;
+      if (within == 0)
+        ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
+                          kSitePipeCodes);
+      const int s = i % S, u = i / S;
+      if (ready && u > 0)
+        ready = pipe_wait(&empty[s], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
+      if (!__all_sync(0xffffffffu, ready)) {
+        *abort_flag = 1u;
+        break;
+      }
+      const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
+                          static_cast<uint32_t>(r) * kCodeRowBytes + static_cast<uint32_t>(within * kStageCodeBytes);
+      decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
+                                 p.codebooks, smem + L.cb);
+      if constexpr (M == 1) {
+        cp_async_arrive_noinc(&full[s]);
+      } else {
+        fence_proxy_async_smem();
+        mbar_arrive(&full[s]);
+      }
+      if (within == kStagesPerTile - 1 || i == nks - 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cempty[c]);
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  }
+
+  // ---- epilogue ----------------------------------------------------------------------
+  // Decoder warp w reads TMEM lanes 32*(w % 4).. (weight rows) and, with its twin
+  // w +- 4, alternating 16-column chunks of the batch tile.
+  const bool decoder = warp < kDecoders / 32;
+  const int q = warp & 3;        // TMEM lane quadrant
+  const int cpar = warp >> 2;    // which 16-column chunks
+  bool acc_ok = true;
+  if (decoder) {
+    acc_ok = __all_sync(0xffffffffu, pipe_wait(acc_bar, 0u, abort_flag, p.status, kSitePipeAcc) && !*abort_flag);
+    tc_fence_after_sync();
+  }
+  const int n = n0 + 32 * q + lane;
+  const bool n_valid = n < p.N;
+  if (p.SK == 1) {
+    if (decoder && acc_ok) {
+      const float sc = n_valid ? __half2float(p.scales[n]) : 0.f;
+      const float bi = (n_valid && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
+      for (int c0 = 16 * cpar; c0 < p.BN; c0 += 32) {
+        float v[16];
+        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), v);
+        if (n_valid) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int b = b0 + c0 + i;
+            if (b < p.batch) p.y[static_cast<size_t>(b) * p.N + n] = __float2half_rn(v[i] * sc + bi);
+          }
+        }
+      }
+    }
+  } else {
+    // Split K: quadrant q of every CTA's partial goes to CTA (q mod SK), which sums
+    // the SK partials in split order.  Receive buffer (over the stages, which every
+    // CTA has stopped using at the first cluster barrier): slot (split, q / SK) of 32
+    // rows x (BN + 4) floats.
+    const int SK = p.SK;
+    const int pitch = p.BN + 4;
+    const int qper = 4 / SK;
+    tc_fence_before_sync();
+    cluster_barrier();  // every CTA's MMAs are done: its stage memory may be overwritten
+    if (decoder && acc_ok) {
+      const uint32_t owner = static_cast<uint32_t>(q % SK);
+      const uint32_t slot = static_cast<uint32_t>(split * qper + q / SK);
+      const uint32_t row_off = (slot * 32u + static_cast<uint32_t>(lane)) * static_cast<uint32_t>(pitch) * 4u;
+      const uint32_t remote_base = mapa_shared_cluster(sbase + L.a + row_off, owner);
+      for (int c0 = 16 * cpar; c0 < p.BN; c0 += 32) {
+        float v[16];
+        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), v);
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+          asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(remote_base + static_cast<uint32_t>(c0 + i) * 4u), "f"(v[i]), "f"(v[i + 1]),
+                       "f"(v[i + 2]), "f"(v[i + 3]) : "memory");
+      }
+    }
+    if (!acc_ok) *abort_flag = 1u;
+    cluster_barrier();  // every partial has landed
+    if (!*abort_flag) {
+      // this CTA owns quadrants q with q mod SK == split: 32 * qper rows
+      const float* recv = reinterpret_cast<const float*>(smem + L.a);
+      const int rows_owned = 32 * qper;
+      for (int idx = tid; idx < rows_owned * p.BN; idx += kThreads) {
+        const int rl = idx % rows_owned;      // owned row (fast index: coalesced y stores)
+        const int col = idx / rows_owned;
+        const int ql = rl / 32, rr = rl % 32;
+        const int qq = ql * SK + split;       // quadrant of the tile
+        const int nn = n0 + 32 * qq + rr;
+        const int b = b0 + col;
+        if (nn >= p.N || b >= p.batch) continue;
+        float acc = 0.f;
+        for (int j = 0; j < SK; ++j) acc += recv[((j * qper + ql) * 32 + rr) * pitch + col];
+        const float bi = p.bias != nullptr ? __half2float(p.bias[nn]) : 0.f;
+        p.y[static_cast<size_t>(b) * p.N + nn] = __float2half_rn(acc * __half2float(p.scales[nn]) + bi);
+      }
+    }
+  }
+
+  if (*abort_flag) {
+    // a wait gave up: let copies already in flight land before the CTA leaves
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 50000ull) {
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+template <int M, int B, int G>
+cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream) {
+  constexpr bool kSmemCb = (M == 2);
+  const int G_count = pr.K / G;
+  const size_t row_bytes = static_cast<size_t>(G_count) * M * (B <= 8 ? 1 : 2);
+  if (pr.K % kStageK != 0 || row_bytes % 16 != 0) return cudaErrorNotSupported;
+  EncodeTiledFn encode = encode_tiled();
+  if (!encode) return cudaErrorNotSupported;
+
+  int BN = ((pr.batch + 15) / 16) * 16;
+  if (BN > 256) BN = 256;
+  int S = 0;
+  for (int s = 6; s >= 2; --s)
+    if (pipe_layout(s, BN, kSmemCb).total + 1024 <= kSmemLimit) {
+      S = s;
+      break;
+    }
+  if (S == 0) return cudaErrorNotSupported;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(BN)) cols <<= 1;
+
+  CUtensorMap x_map, code_map;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.K), static_cast<cuuint64_t>(pr.batch)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.K) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kStageK), static_cast<cuuint32_t>(BN)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(pr.x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(pr.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const cuuint32_t box[2] = {kCodeRowBytes, static_cast<cuuint32_t>(kRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&code_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pr.codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
+
+  constexpr int kStageCodeBytes = (kStageK / G) * M * (B <= 8 ? 1 : 2);
+  constexpr int kStagesPerTile = static_cast<int>(kCodeRowBytes) / kStageCodeBytes;
+  const int nk = pr.K / kStageK;
+  const int nct = (nk + kStagesPerTile - 1) / kStagesPerTile;
+  const int row_tiles = (pr.N + kRows - 1) / kRows;
+  const int batch_tiles = (pr.batch + BN - 1) / BN;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
+  // Split K over a cluster when the row tiles alone leave SMs idle: the largest SK in
+  // {4, 2} that still fits one wave, gives every split a code tile, and whose receive
+  // buffer (128 rows x (BN + 4) floats) fits in the stage memory.
+  int SK = 1;
+  const uint32_t stage_bytes = static_cast<uint32_t>(S) * (kABytes + static_cast<uint32_t>(BN) * 128u);
+  const uint32_t recv_bytes = 128u * static_cast<uint32_t>(BN + 4) * 4u;
+  for (int sk = 4; sk >= 2; sk /= 2) {
+    const int per = (nct + sk - 1) / sk;
+    if (row_tiles * batch_tiles * sk <= sms && (sk - 1) * per < nct && recv_bytes <= stage_bytes) {
+      SK = sk;
+      break;
+    }
+  }
+
+  PipeParams p{};
+  p.codebooks = static_cast<const __half*>(pr.codebooks);
+  p.scales = static_cast<const __half*>(pr.scales);
+  p.bias = static_cast<const __half*>(pr.bias);
+  p.y = static_cast<__half*>(pr.y);
+  p.K = pr.K;
+  p.N = pr.N;
+  p.batch = pr.batch;
+  p.BN = BN;
+  p.nk = nk;
+  p.S = S;
+  p.SK = SK;
+  p.ct_per = (nct + SK - 1) / SK;
+  p.tmem_cols = cols;
+  p.status = status;
+  const uint32_t smem = pipe_layout(S, BN, kSmemCb).total + 1024;
+  auto kern = tc_pipe_kernel<M, B, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(SK);
+  cfg.gridDim = dim3(static_cast<unsigned>(row_tiles), static_cast<unsigned>(batch_tiles), static_cast<unsigned>(SK));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, x_map, code_map, p);
+}
+
+}  // namespace
+
+cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t stream) {
+  if (p.M == 1 && p.B == 16 && p.g == 8) return launch_pipe<1, 16, 8>(p, status, stream);
+  if (p.M == 2 && p.B == 8 && p.g == 8) return launch_pipe<2, 8, 8>(p, status, stream);
+  if (p.M == 1 && p.B == 16 && p.g == 16) return launch_pipe<1, 16, 16>(p, status, stream);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace aqlm
