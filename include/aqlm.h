@@ -36,6 +36,13 @@
  * that gave up.  All compute calls are asynchronous on `stream`
  * (NULL = the legacy default stream) and may be captured in CUDA graphs.
  *
+ * Stream ordering: kernels are launched with programmatic dependent launch.  A
+ * call may start reading the weight buffers (codes, codebooks, scales, bias)
+ * while the kernel launched just before it on the same stream is still running;
+ * it reads x and writes y only after that kernel has completed.  Weight buffers
+ * must therefore not be written by the kernel immediately preceding a call on
+ * the same stream (they are constant during inference).
+ *
  * Errors: every function returns a status and never aborts, throws or exits.
  * Argument errors are detected on the host before any launch.  A failed
  * launch returns AQLM_ERR_CUDA (the CUDA error is cleared and can be read with

@@ -93,12 +93,19 @@ def test_compute_entry_points_reject_bad_arguments_before_any_cuda_call(lib):
 def test_path_selection(lib):
     sel = native.aqlm_select_path
     assert sel(2, 8, 8, 4096, 4096, 1) == Path.GEMV_LUT
-    assert sel(2, 8, 8, 4096 + 8, 4096, 1) == Path.GEMV      # K % 64 != 0: no lookup table
-    assert sel(1, 16, 8, 4096, 4096, 1) == Path.GEMV
+    # K % 64 == 0 (and 16-byte code rows): the pipelined tensor-core kernel from batch 1
+    assert sel(1, 16, 8, 4096, 4096, 1) == Path.TENSOR_CORE
+    assert sel(1, 16, 16, 4096, 4096, 1) == Path.TENSOR_CORE
     for M, B, g in ((1, 16, 8), (2, 8, 8), (1, 16, 16)):
-        for batch in range(2, 9):
-            assert sel(M, B, g, 4096, 4096, batch) == Path.GEMV
-        for batch in (9, 16, 64, 256, 1000):
+        for batch in (2, 3, 8, 9, 16, 64, 256, 1000):
             assert sel(M, B, g, 4096, 4096, batch) == Path.TENSOR_CORE
+    # other K: the GEMV up to batch 8, the single-stage tensor-core kernel above
+    assert sel(2, 8, 8, 4096 + 8, 4096, 1) == Path.GEMV
+    assert sel(1, 16, 16, 4096 + 64, 4096, 1) == Path.GEMV  # g = 16 code rows of 520 bytes
+    for M, B, g in ((1, 16, 8), (2, 8, 8)):
+        for batch in (1, 4, 8):
+            assert sel(M, B, g, 4096 + 8, 4096, batch) == Path.GEMV
+        for batch in (9, 16, 256):
+            assert sel(M, B, g, 4096 + 8, 4096, batch) == Path.TENSOR_CORE
     assert sel(3, 8, 8, 4096, 4096, 1) == -1
     assert sel(1, 16, 8, 4095, 4096, 1) == -1

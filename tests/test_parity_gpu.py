@@ -226,3 +226,31 @@ def test_published_layers_sampled_rows(dev, wname, li, batch):
 def test_device_status_clean_after_all(dev):
     st, detail = L.check_device_status()
     assert st == Status.OK, hex(detail)
+
+
+@pytest.mark.parametrize("M,B,g,path,batch", [(2, 8, 8, Path.GEMV_LUT, 1), (2, 8, 8, Path.GEMV, 3),
+                                              (1, 16, 8, Path.GEMV, 1), (1, 16, 16, Path.GEMV, 4),
+                                              (1, 16, 8, Path.TENSOR_CORE, 64), (2, 8, 8, Path.TENSOR_CORE, 32)])
+def test_chained_layers_read_the_previous_output(dev, M, B, g, path, batch):
+    """Kernels start their weight-only set-up while the previous kernel on the stream
+    is still running (programmatic dependent launch); x must still be read only after
+    that kernel has written it.  Layer 2 consumes layer 1's output, back to back on one
+    stream with no synchronisation in between."""
+    K = N = 1024
+    ld1 = synth.make_layer(M, B, g, K, N, seed=18, layer=1)
+    ld2 = synth.make_layer(M, B, g, K, N, seed=18, layer=2)
+    x = synth.make_x(batch, K, seed=18)
+    w1, w2 = L.AqlmWeights.from_numpy(ld1, dev), L.AqlmWeights.from_numpy(ld2, dev)
+    xt = torch.from_numpy(x).to(dev)
+    outs = []
+    for _ in range(3):  # repeat to give overlapping launches a chance to race
+        y1 = L.matmul(xt, w1, path=path)
+        y2 = L.matmul(y1, w2, path=path)
+        outs.append((y1, y2))
+    torch.cuda.synchronize()
+    st, detail = L.check_device_status()
+    assert st == Status.OK, hex(detail)
+    for y1, y2 in outs:
+        y1h = y1.cpu().numpy()
+        ref2 = oracle.linear(y1h, ld2.codes, ld2.codebooks, ld2.scales, None, M, B, g)
+        assert_close(y2.cpu().numpy(), ref2, f"chained {M}x{B}g{g} {path.name}")

@@ -103,6 +103,10 @@ int aqlm_last_cuda_error(void) { return t_last_cuda_error; }
 int aqlm_select_path(int M, int B, int g, int K, int N, int batch) {
   if (validate_shape(M, B, g, K, N, batch) != AQLM_OK) return -1;
   if (aqlm::gemv_lut_supported(M, B, g, K, batch)) return AQLM_PATH_GEMV_LUT;
+  // The pipelined tensor-core kernel decodes a weight tile once for the whole batch
+  // and gathers codewords faster than the GEMV, so it wins from batch 1 on whenever
+  // its shape test holds; the GEMV covers the remaining small-batch shapes.
+  if (aqlm::tc_pipelined_shape(M, B, g, K)) return AQLM_PATH_TENSOR_CORE;
   if (batch <= 8) return AQLM_PATH_GEMV;
   return AQLM_PATH_TENSOR_CORE;
 }

@@ -53,6 +53,11 @@ EncodeTiledFn encode_tiled();
 // Pipelined decode -> tcgen05 kernel; cudaErrorNotSupported when the shape is
 // outside what it handles (the caller then uses the single-stage kernel).
 cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t stream);
+// Shape test of the pipelined kernel: K % 64 == 0 and code rows a multiple of 16 bytes.
+inline bool tc_pipelined_shape(int M, int B, int g, int K) {
+  const long long row_bytes = static_cast<long long>(K / g) * M * (B <= 8 ? 1 : 2);
+  return K % 64 == 0 && row_bytes % 16 == 0;
+}
 
 // True if the scheme is one the kernels are instantiated for.
 inline bool scheme_supported(int M, int B, int g) {

@@ -65,9 +65,10 @@ __global__ void __launch_bounds__(128) gemv_gather_kernel(
   using code_t = typename std::conditional<(B <= 8), uint8_t, uint16_t>::type;
   constexpr int kCodeBytes = sizeof(code_t);
   constexpr int kGroupsPerVec = 16 / (M * kCodeBytes);
+  grid_dependents_launch();
   const int lane = threadIdx.x & 31;
   const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (n >= N) return;
+  if (n >= N) return;  // never the block's first warp: every block reaches the wait below
   const int groups = K / G;
   const size_t row_bytes = static_cast<size_t>(groups) * M * kCodeBytes;
   const uint8_t* row = static_cast<const uint8_t*>(codes) + static_cast<size_t>(n) * row_bytes;
@@ -76,17 +77,22 @@ __global__ void __launch_bounds__(128) gemv_gather_kernel(
   float acc[BATCH];
 #pragma unroll
   for (int b = 0; b < BATCH; ++b) acc[b] = 0.f;
+  // x may be the previous kernel's output (and y its input): wait for it
+  grid_dependency_wait();
 
   // 16-byte code vectors when every row starts 16-byte aligned.
   const int nvec = (row_bytes % 16 == 0) ? groups / kGroupsPerVec : 0;
   for (int v = lane; v < nvec; v += 32) {
     const uint4 q = ldg_stream_v4(row + static_cast<size_t>(v) * 16, stream_pol);
-    const code_t* cv = reinterpret_cast<const code_t*>(&q);
+    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int gi = 0; gi < kGroupsPerVec; ++gi) {
       uint32_t code[M];
 #pragma unroll
-      for (int m = 0; m < M; ++m) code[m] = cv[gi * M + m];
+      for (int m = 0; m < M; ++m) {
+        const int byte = (gi * M + m) * kCodeBytes;  // little-endian position in the vector
+        code[m] = (words[byte / 4] >> (8 * (byte % 4))) & ((1u << (8 * kCodeBytes)) - 1u);
+      }
       accumulate_group<M, B, G, BATCH>(x, K, v * kGroupsPerVec + gi, code, codebooks, acc);
     }
   }
@@ -115,12 +121,18 @@ __global__ void __launch_bounds__(128) gemv_gather_kernel(
 template <int M, int B, int G, int BATCH>
 cudaError_t launch_fixed(const Problem& p, cudaStream_t stream) {
   const int warps_per_block = 4;
-  const unsigned blocks = static_cast<unsigned>((p.N + warps_per_block - 1) / warps_per_block);
-  gemv_gather_kernel<M, B, G, BATCH><<<blocks, 32 * warps_per_block, 0, stream>>>(
-      static_cast<const __half*>(p.x), p.codes, static_cast<const __half*>(p.codebooks),
-      static_cast<const __half*>(p.scales), static_cast<const __half*>(p.bias),
-      static_cast<__half*>(p.y), p.K, p.N);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>((p.N + warps_per_block - 1) / warps_per_block), 1, 1);
+  cfg.blockDim = dim3(32 * warps_per_block, 1, 1);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_gather_kernel<M, B, G, BATCH>, static_cast<const __half*>(p.x), p.codes,
+                            static_cast<const __half*>(p.codebooks), static_cast<const __half*>(p.scales),
+                            static_cast<const __half*>(p.bias), static_cast<__half*>(p.y), p.K, p.N);
 }
 
 template <int M, int B, int G>

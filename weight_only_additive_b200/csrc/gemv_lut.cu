@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
   int npass = 0;
   while (npass < p.P && (static_cast<int>(crank) * p.P + npass) * kGroupsPerPass < p.G) ++npass;
 
+  // The next kernel in the stream may start its own weight-only set-up now.
+  grid_dependents_launch();
+
   // ---- 1. barriers; one thread starts the whole code stream (a TMA box per tile) --------
   if (tid == 0) {
     for (int i = 0; i < p.P * p.ntile; ++i) mbar_init(&tile_bar[i], 1);
@@ -209,6 +212,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
       cp_async_16_zfill(sbase + bo + kmajor_noswizzle_offset(idx, 0), p.codebooks + (static_cast<size_t>(m) * 256 + idx) * 8, 16);
       *reinterpret_cast<uint4*>(smem + bo + kmajor_noswizzle_offset(idx, 1)) = make_uint4(0u, 0u, 0u, 0u);
     }
+    for (int i = tid; i < p.ntask * 8; i += kThreads) part[i] = 0.f;
+    // Everything above reads only weights.  x may be the output of the kernel just
+    // before this one in the stream (programmatic dependent launch): wait for it.
+    grid_dependency_wait();
     for (int i = tid; i < npass * 128; i += kThreads) {  // A row rho (and rho+64) = one group of x
       const int ps = i >> 7, rho = i & 127;
       const int gbeg = (static_cast<int>(crank) * p.P + ps) * kGroupsPerPass;
@@ -222,7 +229,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
       *reinterpret_cast<uint4*>(smem + ao + kmajor_noswizzle_offset(rho, 1)) = make_uint4(0u, 0u, 0u, 0u);
     }
     cp_async_commit();
-    for (int i = tid; i < p.ntask * 8; i += kThreads) part[i] = 0.f;
   }
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -475,7 +481,7 @@ cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t st
   const int clusters = (pr.N + p.RB - 1) / p.RB;
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(p.C);
   attr[0].val.clusterDim.y = 1;
@@ -485,7 +491,9 @@ cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t st
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, map, p);
 }
 

@@ -1,29 +1,38 @@
-// Pipelined batch >= 16 path: codeword decode into shared memory overlapped with
-// 5th-generation tensor-core MMAs (tcgen05.mma kind::f16, fp32 accumulator in TMEM).
+// Pipelined decode -> tensor-core path (every batch size when K % 64 == 0): codeword
+// decode into shared memory overlapped with 5th-generation tensor-core MMAs
+// (tcgen05.mma kind::f16, fp32 accumulator in TMEM).
 //
 // "Dequantize-to-FP16 then an FP16 tensor-core GEMM" (inference-research record
 // "AQLM (additive / multi-codebook quantization)", notes), fused so the fp16
 // weights exist only as 128 x 64 shared-memory tiles.  Swap-AB: the MMA's M is
 // 128 weight rows, its N is the batch tile (16..256), so D[n, b] lands in TMEM
-// with one weight row per lane.
+// with one weight row per lane.  Because the weight tile is decoded once for the
+// whole batch tile, the same kernel also serves token generation (batch 1..8):
+// its decoders gather codewords faster than the GEMV's lanes do.
 //
-// Warp roles (224 threads):
-//   warps 0-3  decoders, then epilogue.  Thread r owns weight row n0 + r.  Per
-//              64-wide K stage it reads its 8 (g = 8) or 4 (g = 16) codes from the
-//              code tile and writes the row's 128 bytes of the A stage in the
-//              128-byte-swizzled K-major layout:
+// Warp roles (352 threads):
+//   warps 0-7  decoders, then epilogue.  Threads r and r + 128 own weight row
+//              n0 + r (16-byte chunks 0-3 and 4-7 of each 64-wide K stage).  Per
+//              stage a thread reads its codes from the code tile and writes its
+//              64 bytes of the A stage in the 128-byte-swizzled K-major layout:
 //                1x16: the codeword is the fp16 data, so each 16-byte piece is one
 //                      cp.async gather from the (L2-resident) codebook straight into
 //                      its swizzled slot, tracked by cp.async.mbarrier.arrive;
 //                2x8:  the two codewords come from the codebooks staged in shared
-//                      memory, are added in fp32, rounded once to fp16 and stored.
-//   warp 4     TMA producer of x tiles (B operand, 128-byte swizzle, zero-filled
+//                      memory, are added as half2 and stored.
+//   warp 8     TMA producer of x tiles (B operand, 128-byte swizzle, zero-filled
 //              past the batch and K edges).
-//   warp 5     MMA issuer: 4 x (128 x BN x 16) per stage, commit releases the stage.
-//   warp 6     TMA producer of code tiles (128 rows x 64 bytes = 4 or 8 stages).
+//   warp 9     MMA issuer: 4 x (128 x BN x 16) per stage, commit releases the stage.
+//   warp 10    TMA producer of code tiles (128 rows x 64 bytes = 4 or 8 stages).
+// Split K: SK CTAs of a (1, 1, SK) cluster take consecutive K ranges of the same
+// weight rows and exchange fp32 partials through distributed shared memory.
 // Epilogue: tcgen05.ld of 16 columns at a time, y = s_n * D + bias_n -> fp16.
 #include <cuda.h>
 
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
 #include <type_traits>
 
 #include "aqlm_device.cuh"
@@ -51,8 +60,9 @@ struct PipeParams {
   int BN;          // batch tile (multiple of 16, <= 256)
   int nk;          // K / 64 stages (whole K)
   int S;           // A/B stage ring depth
-  int SK;          // CTAs splitting K (cluster size along z): 1, 2 or 4
-  int ct_per;      // code tiles per K split
+  int SK;          // CTAs splitting K (cluster size along z): 1..16
+  int ks_per;      // K stages per split (the last split may have fewer)
+  int red_rows;    // split-K reduction: weight rows each CTA of the cluster owns
   uint32_t tmem_cols;
   uint32_t* status;
 };
@@ -175,14 +185,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
   const int n0 = blockIdx.x * kRows;
   const int b0 = blockIdx.y * p.BN;
   const int split = blockIdx.z;  // == rank in the (1, 1, SK) cluster
-  // this CTA's K range, in whole code tiles: tiles [ct0, ct1), stages [ks0, ks1)
-  const int nct_all = (p.nk + kStagesPerTile - 1) / kStagesPerTile;
-  const int ct0 = split * p.ct_per;
-  const int ct1 = min(nct_all, ct0 + p.ct_per);
-  const int ks0 = ct0 * kStagesPerTile;
-  const int ks1 = min(p.nk, ct1 * kStagesPerTile);
+  // this CTA's K range: stages [ks0, ks1), read as nct code tiles of kStagesPerTile
+  // stages starting at stage ks0 (the host keeps ks0's code offset 16-byte aligned)
+  const int ks0 = split * p.ks_per;
+  const int ks1 = min(p.nk, ks0 + p.ks_per);
   const int nks = max(0, ks1 - ks0);  // host guarantees >= 1
+  const int nct = (nks + kStagesPerTile - 1) / kStagesPerTile;
 
+  // the next kernel on the stream may start its own set-up now; x is read (and
+  // y written) only after this grid's dependency wait in the x producer below
+  grid_dependents_launch();
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], kDecoders + 1);
@@ -210,6 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     // ---- x tiles (B operand): reused by every CTA, keep them in L2 ----
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_last();
+      // x may be the previous kernel's output.  Every y store of this CTA
+      // follows the MMAs, which follow these x tiles, so it is ordered too.
+      grid_dependency_wait();
       for (int i = 0; i < nks; ++i) {
         const int s = i % S, u = i / S;
         if (u > 0 && !pipe_wait(&empty[s], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeEmpty))
@@ -223,13 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     // ---- code tiles: 128 rows x 64 bytes, read once ----
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
-      for (int t = 0; t < ct1 - ct0; ++t) {
+      for (int t = 0; t < nct; ++t) {
         const int c = t % kCodeSlots, u = t / kCodeSlots;
         if (u > 0 && !pipe_wait(&cempty[c], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeCodes))
           break;
         mbar_arrive_expect_tx(&cfull[c], kCodeTileBytes);
+        // bytes past the row end (K edge) are zero-filled; stages past ks1 are not decoded
         tma_load_2d(sbase + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes, &code_map,
-                    (ct0 + t) * static_cast<int>(kCodeRowBytes), n0, &cfull[c], pol);
+                    (ks0 + t * kStagesPerTile) * kStageCodeBytes, n0, &cfull[c], pol);
       }
     }
   } else if (warp == kWarpMma) {
@@ -317,20 +333,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
       }
     }
   } else {
-    // Split K: quadrant q of every CTA's partial goes to CTA (q mod SK), which sums
-    // the SK partials in split order.  Receive buffer (over the stages, which every
-    // CTA has stopped using at the first cluster barrier): slot (split, q / SK) of 32
-    // rows x (BN + 4) floats.
+    // Split K: the CTA of rank k owns weight rows [k R, (k + 1) R) of the tile
+    // (R = red_rows).  Every CTA stores its fp32 partial of row r into slot
+    // (split, r - k R) of the owner's receive buffer (over the stages, which every
+    // CTA has stopped using at the first cluster barrier; pitch BN + 4 floats); the
+    // owner then sums the SK partials in split order.
     const int SK = p.SK;
+    const int R = p.red_rows;
     const int pitch = p.BN + 4;
-    const int qper = 4 / SK;
     tc_fence_before_sync();
     cluster_barrier();  // every CTA's MMAs are done: its stage memory may be overwritten
     if (decoder && acc_ok) {
-      const uint32_t owner = static_cast<uint32_t>(q % SK);
-      const uint32_t slot = static_cast<uint32_t>(split * qper + q / SK);
-      const uint32_t row_off = (slot * 32u + static_cast<uint32_t>(lane)) * static_cast<uint32_t>(pitch) * 4u;
-      const uint32_t remote_base = mapa_shared_cluster(sbase + L.a + row_off, owner);
+      const int r = 32 * q + lane;
+      const uint32_t owner = static_cast<uint32_t>(r / R);
+      const uint32_t slot_row = static_cast<uint32_t>(split * R + (r - static_cast<int>(owner) * R));
+      const uint32_t remote_base =
+          mapa_shared_cluster(sbase + L.a + slot_row * static_cast<uint32_t>(pitch) * 4u, owner);
       for (int c0 = 16 * cpar; c0 < p.BN; c0 += 32) {
         float v[16];
         tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), v);
@@ -344,19 +362,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     if (!acc_ok) *abort_flag = 1u;
     cluster_barrier();  // every partial has landed
     if (!*abort_flag) {
-      // this CTA owns quadrants q with q mod SK == split: 32 * qper rows
       const float* recv = reinterpret_cast<const float*>(smem + L.a);
-      const int rows_owned = 32 * qper;
+      const int r_begin = split * R;
+      const int rows_owned = max(0, min(kRows, r_begin + R) - r_begin);
       for (int idx = tid; idx < rows_owned * p.BN; idx += kThreads) {
-        const int rl = idx % rows_owned;      // owned row (fast index: coalesced y stores)
+        const int rl = idx % rows_owned;  // owned row (fast index: coalesced y stores)
         const int col = idx / rows_owned;
-        const int ql = rl / 32, rr = rl % 32;
-        const int qq = ql * SK + split;       // quadrant of the tile
-        const int nn = n0 + 32 * qq + rr;
+        const int nn = n0 + r_begin + rl;
         const int b = b0 + col;
         if (nn >= p.N || b >= p.batch) continue;
         float acc = 0.f;
-        for (int j = 0; j < SK; ++j) acc += recv[((j * qper + ql) * 32 + rr) * pitch + col];
+        for (int j = 0; j < SK; ++j) acc += recv[(j * R + rl) * pitch + col];
         const float bi = p.bias != nullptr ? __half2float(p.bias[nn]) : 0.f;
         p.y[static_cast<size_t>(b) * p.N + nn] = __float2half_rn(acc * __half2float(p.scales[nn]) + bi);
       }
@@ -377,24 +393,105 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
   }
 }
 
+// Launch plan: ring depth S and the K split SK (cluster size).  The kernel is bound by
+// the decode rate of the SMs it occupies, so the plan spreads row tiles x K splits
+// over the SMs: estimated time = waves x (stages per CTA + fixed cost per CTA) + the
+// split-K exchange, with the number of co-resident clusters taken from the occupancy
+// calculator.  A CTA that allocates tensor memory runs alone on its SM (the
+// calculator reports one CTA per SM for such kernels whatever their shared memory),
+// so the deepest ring that fits is taken.  The exchange moves 128 x BN fp32 partials
+// per CTA through distributed shared memory; measured on B200 it costs about two
+// stage times per 16 batch columns, which makes SK = 1 the choice for wide batches.
+struct TcPlan {
+  int S = 0, SK = 1, ks_per = 0, red_rows = 128;
+};
+
+constexpr int kPlanFixedStages = 3;     // set-up, pipeline fill and epilogue, in stage times
+constexpr int kPlanExchangePer16 = 2;   // split-K exchange, stage times per 16 batch columns
+constexpr int kMaxSplit = 16;
+
+inline uint32_t pipe_smem_bytes(int S, int BN, bool smem_cb) { return pipe_layout(S, BN, smem_cb).total + 1024; }
+
 template <int M, int B, int G>
-cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream) {
+cudaError_t plan_pipe(int dev, const Problem& pr, int BN, TcPlan* out) {
   constexpr bool kSmemCb = (M == 2);
-  const int G_count = pr.K / G;
-  const size_t row_bytes = static_cast<size_t>(G_count) * M * (B <= 8 ? 1 : 2);
-  if (pr.K % kStageK != 0 || row_bytes % 16 != 0) return cudaErrorNotSupported;
+  constexpr int kStageCodeBytes = (kStageK / G) * M * (B <= 8 ? 1 : 2);
+  constexpr int kSplitAlign = 16 / kStageCodeBytes;  // split starts keep 16-byte code offsets
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int>, TcPlan> cache;
+  const auto key = std::make_tuple(dev, pr.N, pr.K, pr.batch);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *out = it->second;
+      return cudaSuccess;
+    }
+  }
+  auto kern = tc_pipe_kernel<M, B, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
+  if (e != cudaSuccess) return e;
+  const int cmax = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess
+                       ? kMaxSplit : 8;
+  cudaGetLastError();
+
+  const int nk = pr.K / kStageK;
+  const int row_tiles = (pr.N + kRows - 1) / kRows;
+  const int batch_tiles = (pr.batch + BN - 1) / BN;
+  const long long clusters = static_cast<long long>(row_tiles) * batch_tiles;
+  TcPlan best;
+  long long best_cost = -1;
+  for (int S = 6; S >= 2; --S) {
+    const uint32_t smem = pipe_smem_bytes(S, BN, kSmemCb);
+    if (smem > kSmemLimit) continue;
+    const uint32_t stage_bytes = static_cast<uint32_t>(S) * (kABytes + static_cast<uint32_t>(BN) * 128u);
+    for (int SK = 1; SK <= cmax; ++SK) {
+      int per = (nk + SK - 1) / SK;
+      per = (per + kSplitAlign - 1) / kSplitAlign * kSplitAlign;
+      if (static_cast<long long>(SK - 1) * per >= nk) continue;  // a split would be empty
+      const int R = (kRows + SK - 1) / SK;
+      if (SK > 1 && static_cast<uint32_t>(SK * R * (BN + 4)) * 4u > stage_bytes) continue;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 1;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = static_cast<unsigned>(SK);
+      cfg.gridDim = dim3(1, 1, static_cast<unsigned>(SK));
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int active = 0;
+      if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
+        cudaGetLastError();
+        continue;
+      }
+      const long long waves = (clusters + active - 1) / active;
+      const long long exchange = SK > 1 ? 16 * (1 + kPlanExchangePer16 * (BN / 16)) + SK : 0;
+      const long long cost = waves * 16 * (per + kPlanFixedStages) + exchange;
+      if (best_cost < 0 || cost < best_cost) {
+        best_cost = cost;
+        best.S = S;
+        best.SK = SK;
+        best.ks_per = per;
+        best.red_rows = R;
+      }
+    }
+  }
+  if (best_cost < 0) return cudaErrorNotSupported;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = best;
+  *out = best;
+  return cudaSuccess;
+}
+
+template <int M, int B, int G>
+cudaError_t launch_pipe_plan(const Problem& pr, uint32_t* status, cudaStream_t stream, int BN, const TcPlan& plan) {
+  constexpr bool kSmemCb = (M == 2);
+  const size_t row_bytes = static_cast<size_t>(pr.K / G) * M * (B <= 8 ? 1 : 2);
   EncodeTiledFn encode = encode_tiled();
   if (!encode) return cudaErrorNotSupported;
-
-  int BN = ((pr.batch + 15) / 16) * 16;
-  if (BN > 256) BN = 256;
-  int S = 0;
-  for (int s = 6; s >= 2; --s)
-    if (pipe_layout(s, BN, kSmemCb).total + 1024 <= kSmemLimit) {
-      S = s;
-      break;
-    }
-  if (S == 0) return cudaErrorNotSupported;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(BN)) cols <<= 1;
 
@@ -420,29 +517,6 @@ cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream
       return cudaErrorNotSupported;
   }
 
-  constexpr int kStageCodeBytes = (kStageK / G) * M * (B <= 8 ? 1 : 2);
-  constexpr int kStagesPerTile = static_cast<int>(kCodeRowBytes) / kStageCodeBytes;
-  const int nk = pr.K / kStageK;
-  const int nct = (nk + kStagesPerTile - 1) / kStagesPerTile;
-  const int row_tiles = (pr.N + kRows - 1) / kRows;
-  const int batch_tiles = (pr.batch + BN - 1) / BN;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaGetLastError();
-  // Split K over a cluster when the row tiles alone leave SMs idle: the largest SK in
-  // {4, 2} that still fits one wave, gives every split a code tile, and whose receive
-  // buffer (128 rows x (BN + 4) floats) fits in the stage memory.
-  int SK = 1;
-  const uint32_t stage_bytes = static_cast<uint32_t>(S) * (kABytes + static_cast<uint32_t>(BN) * 128u);
-  const uint32_t recv_bytes = 128u * static_cast<uint32_t>(BN + 4) * 4u;
-  for (int sk = 4; sk >= 2; sk /= 2) {
-    const int per = (nct + sk - 1) / sk;
-    if (row_tiles * batch_tiles * sk <= sms && (sk - 1) * per < nct && recv_bytes <= stage_bytes) {
-      SK = sk;
-      break;
-    }
-  }
-
   PipeParams p{};
   p.codebooks = static_cast<const __half*>(pr.codebooks);
   p.scales = static_cast<const __half*>(pr.scales);
@@ -452,29 +526,56 @@ cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream
   p.N = pr.N;
   p.batch = pr.batch;
   p.BN = BN;
-  p.nk = nk;
-  p.S = S;
-  p.SK = SK;
-  p.ct_per = (nct + SK - 1) / SK;
+  p.nk = pr.K / kStageK;
+  p.S = plan.S;
+  p.SK = plan.SK;
+  p.ks_per = plan.ks_per;
+  p.red_rows = plan.red_rows;
   p.tmem_cols = cols;
   p.status = status;
-  const uint32_t smem = pipe_layout(S, BN, kSmemCb).total + 1024;
+  const uint32_t smem = pipe_smem_bytes(plan.S, BN, kSmemCb);
   auto kern = tc_pipe_kernel<M, B, G>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
   if (e != cudaSuccess) return e;
+  if (plan.SK > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  const int row_tiles = (pr.N + kRows - 1) / kRows;
+  const int batch_tiles = (pr.batch + BN - 1) / BN;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = static_cast<unsigned>(SK);
-  cfg.gridDim = dim3(static_cast<unsigned>(row_tiles), static_cast<unsigned>(batch_tiles), static_cast<unsigned>(SK));
+  attr[0].val.clusterDim.z = static_cast<unsigned>(plan.SK);
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(row_tiles), static_cast<unsigned>(batch_tiles),
+                     static_cast<unsigned>(plan.SK));
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, x_map, code_map, p);
+}
+
+// Batch tile: the batch rounded up to a multiple of 16, at most 256 (the MMA's N).
+inline int pipe_batch_tile(int batch) { return std::min(256, (batch + 15) / 16 * 16); }
+
+template <int M, int B, int G>
+cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream) {
+  if (!tc_pipelined_shape(M, B, G, pr.K)) return cudaErrorNotSupported;
+  if (!encode_tiled()) return cudaErrorNotSupported;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int BN = pipe_batch_tile(pr.batch);
+  TcPlan plan;
+  e = plan_pipe<M, B, G>(dev, pr, BN, &plan);
+  if (e != cudaSuccess) return e;
+  return launch_pipe_plan<M, B, G>(pr, status, stream, BN, plan);
 }
 
 }  // namespace
