@@ -52,6 +52,7 @@
 #ifndef AQLM_H_
 #define AQLM_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -106,6 +107,51 @@ aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codeb
 aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void* scales,
                             void* W_out, int M, int B, int g, int K, int N,
                             aqlm_stream_t stream);
+
+/* One layer of a group call: the arguments of aqlm_matmul, same meaning and
+ * layout. */
+typedef struct {
+  const void* x;
+  const void* codes;
+  const void* codebooks;
+  const void* scales;
+  const void* bias;   /* may be NULL */
+  void* y;
+  int M, B, g, K, N, batch;
+} aqlm_problem;
+
+/*
+ * Grouped launch of independent layers (a decoder block's linears, or a set of
+ * experts).  The AQLM pages give no such call; it serves the token-generation case
+ * where one layer is too small to fill the GPU (inference-research record "AQLM
+ * (additive / multi-codebook quantization)": batch-1 decoding is dominated by
+ * per-layer overheads, which CUDA graphs and fused launches remove).
+ *
+ * Computes y_i for every problems[i] exactly as aqlm_matmul would (same
+ * definition and tolerance).  The problems must be independent: no y_i may
+ * overlap another problem's x, y, codes, codebooks, scales or bias (overlapping
+ * outputs and inputs are rejected with AQLM_ERR_INVALID_ARG as far as the
+ * pointer ranges show).  2x8 g8 batch-1 problems with K % 64 == 0 are computed
+ * together, up to 16 per launch pair (a partial-sum kernel and a reduction); the
+ * others are launched one after another as by aqlm_matmul.  Both kernels of a
+ * pair keep the stream-ordering contract above.
+ *
+ * workspace: caller-owned DEVICE memory of at least
+ * aqlm_group_workspace_size(problems, count) bytes, 256-byte aligned (NULL
+ * allowed when that size is 0).  It holds fp32 partial sums between the two
+ * kernels of a pair and needs no initialisation; calls that may run
+ * concurrently (different streams) must not share a workspace.
+ * count == 0 is a no-op; count < 0 or problems == NULL (with count > 0) is
+ * AQLM_ERR_INVALID_ARG.  Every problem is validated as aqlm_validate does before
+ * anything is launched.
+ */
+aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* workspace,
+                              size_t workspace_bytes, aqlm_stream_t stream);
+
+/* Workspace bytes aqlm_matmul_group needs for these problems: for every run of
+ * up to 16 grouped problems, the sum over them of ceil(K / 512) * N * 4 bytes
+ * rounded up to 256; the maximum over runs.  Pure host logic. */
+size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count);
 
 /* The kernel family AQLM_PATH_AUTO picks for this problem, or -1 if unsupported.
  * Pure host logic: needs no GPU. */

@@ -109,3 +109,57 @@ def test_path_selection(lib):
             assert sel(M, B, g, 4096 + 8, 4096, batch) == Path.TENSOR_CORE
     assert sel(3, 8, 8, 4096, 4096, 1) == -1
     assert sel(1, 16, 8, 4095, 4096, 1) == -1
+
+
+# ---------------------------------------------------------------------------
+# group call: host-side sizing and validation (returns before any CUDA call)
+# ---------------------------------------------------------------------------
+def _prob(base, M=2, B=8, g=8, K=4096, N=4096, batch=1, bias=False):
+    """Disjoint fake buffers for one problem, laid out from `base` (never dereferenced)."""
+    step = 1 << 26
+    return (base, base + step, base + 2 * step, base + 3 * step, base + 4 * step if bias else None,
+            base + 5 * step, M, B, g, K, N, batch)
+
+
+def _ws_bytes(K, N):
+    return ((K // 8 + 63) // 64 * N * 4 + 255) // 256 * 256
+
+
+def test_group_workspace_size(lib):
+    P = [_prob(1 << 32), _prob(1 << 33, K=11008, N=200), _prob(1 << 34, M=1, B=16)]
+    assert native.aqlm_group_workspace_size(P) == _ws_bytes(4096, 4096) + _ws_bytes(11008, 200)
+    assert native.aqlm_group_workspace_size([]) == 0
+    assert native.aqlm_group_workspace_size([_prob(1 << 32, M=1, B=16)]) == 0       # nothing grouped
+    assert native.aqlm_group_workspace_size([_prob(1 << 32, batch=2)]) == 0         # batch 2: not grouped
+    assert native.aqlm_group_workspace_size([_prob(1 << 32, K=4104)]) == 0          # K % 64 != 0
+    assert native.aqlm_group_workspace_size([_prob(1 << 32, K=4095)]) == 0          # invalid shape
+    # 20 grouped problems: two runs of 16 and 4; the workspace is the larger run
+    many = [_prob((i + 1) << 32, K=64 * (i + 1), N=100) for i in range(20)]
+    run1 = sum(_ws_bytes(64 * (i + 1), 100) for i in range(16))
+    run2 = sum(_ws_bytes(64 * (i + 1), 100) for i in range(16, 20))
+    assert native.aqlm_group_workspace_size(many) == max(run1, run2)
+
+
+def test_group_validation_needs_no_gpu(lib):
+    L_ = native.lib()
+    P = [_prob(1 << 32), _prob(1 << 33, K=11008, N=200)]
+    need = native.aqlm_group_workspace_size(P)
+    arr = native.problem_array(P)
+    assert L_.aqlm_matmul_group(arr, 0, None, 0, None) == Status.OK              # no-op
+    assert L_.aqlm_matmul_group(arr, -1, None, 0, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_group(None, 2, None, 0, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_group(arr, 2, None, need, None) == Status.INVALID_ARG  # no workspace
+    assert L_.aqlm_matmul_group(arr, 2, 1 << 40, need - 4, None) == Status.INVALID_ARG  # too small
+    assert L_.aqlm_matmul_group(arr, 2, (1 << 40) + 16, need, None) == Status.MISALIGNED
+    bad = native.problem_array([P[0], _prob(1 << 35, M=3)])
+    assert L_.aqlm_matmul_group(bad, 2, 1 << 40, need, None) == Status.UNSUPPORTED
+    bad = native.problem_array([P[0], _prob(1 << 35, N=0)])
+    assert L_.aqlm_matmul_group(bad, 2, 1 << 40, need, None) == Status.INVALID_ARG
+    # y of problem 1 overlaps x of problem 0 / y of problem 0: not independent
+    q = list(_prob(1 << 33))
+    q[5] = P[0][0] + 4096
+    assert L_.aqlm_matmul_group(native.problem_array([P[0], tuple(q)]), 2, 1 << 40, need, None) == \
+        Status.INVALID_ARG
+    q[5] = P[0][5]
+    assert L_.aqlm_matmul_group(native.problem_array([P[0], tuple(q)]), 2, 1 << 40, need, None) == \
+        Status.INVALID_ARG

@@ -1,0 +1,175 @@
+"""aqlm_matmul_group (grouped lookup-table kernel + reduction) vs the CPU oracle,
+through the C ABI.
+
+Every layer of a group must meet the aqlm_matmul bar: max|y - y_ref| / max|y_ref|
+<= 5e-3 against the oracle's fp64 reference of the decoded weights, no NaN/Inf;
+bit for bit on integer-valued layers; run-to-run bitwise identical; correct when
+the workspace is reused by back-to-back calls; and correct for groups that mix
+grouped and non-grouped problems or exceed one launch's 16 layers.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_only_additive_b200 import layer as L
+from weight_only_additive_b200 import native, synth, workloads
+from weight_only_additive_b200.native import Status
+
+pytestmark = pytest.mark.gpu
+
+TOL = 5e-3
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    native.lib()
+    torch.cuda.set_device(0)
+    return torch.device("cuda", 0)
+
+
+def rel_err(y_gpu, y_ref):
+    return float(np.abs(y_gpu.astype(np.float64) - y_ref).max() / max(np.abs(y_ref).max(), 1e-30))
+
+
+def assert_close(y_gpu, y_ref, what):
+    assert np.isfinite(y_gpu.astype(np.float32)).all(), f"{what}: non-finite output"
+    err = rel_err(y_gpu, y_ref)
+    assert err <= TOL, f"{what}: rel err {err:.3e} > {TOL}"
+
+
+def build_group(specs, dev, seed):
+    """specs: (M, B, g, K, N, batch, with_bias) per layer -> (LayerGroup, layer data, x, out)."""
+    lds, xs, items = [], [], []
+    for i, (M, B, g, K, N, batch, bias) in enumerate(specs):
+        ld = synth.make_layer(M, B, g, K, N, seed=seed, layer=i, with_bias=bias)
+        x = synth.make_x(batch, K, seed=seed, layer=i)
+        w = L.AqlmWeights.from_numpy(ld, dev)
+        xt = torch.from_numpy(x).to(dev)
+        out = torch.full((batch, N), float("nan"), dtype=torch.float16, device=dev)
+        lds.append(ld)
+        xs.append(x)
+        items.append((w, xt, out))
+    return L.LayerGroup(items), lds, xs, [it[2] for it in items]
+
+
+def check_status():
+    torch.cuda.synchronize()
+    st, detail = L.check_device_status()
+    assert st == Status.OK, (st, hex(detail))
+
+
+MIXED = [
+    (2, 8, 8, 4096, 4096, 1, False),   # q_proj-sized
+    (2, 8, 8, 11008, 200, 1, True),    # G = 1376: a half-filled last 64-group slice; ragged rows
+    (2, 8, 8, 64, 1, 1, True),         # one slice, one row
+    (2, 8, 8, 512, 1000, 1, False),    # ragged last 64-row tile
+    (1, 16, 8, 1024, 300, 1, True),    # not grouped: tensor-core path
+    (2, 8, 8, 1024, 130, 4, False),    # not grouped: batch 4
+    (2, 8, 8, 1032, 77, 1, False),     # not grouped: K % 64 != 0
+    (2, 8, 8, 2048, 129, 1, True),
+]
+
+
+def test_group_mixed_layers_match_oracle(dev):
+    grp, lds, xs, outs = build_group(MIXED, dev, seed=40)
+    assert grp.workspace_bytes == native.aqlm_group_workspace_size(grp.problems, grp.count) > 0
+    grp.run()
+    check_status()
+    for (M, B, g, K, N, batch, _), ld, x, out in zip(MIXED, lds, xs, outs):
+        y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+        assert_close(out.cpu().numpy(), y_ref, f"group layer {M}x{B}g{g} K={K} N={N} b={batch}")
+
+
+def test_group_is_deterministic_and_reuses_its_workspace(dev):
+    """Two calls back to back on one stream, no synchronisation between them: the
+    second call's partial-sum kernel must not overwrite the workspace before the
+    first call's reduction has read it.  Different x per call, same weights."""
+    specs = [(2, 8, 8, 4096, 1024, 1, False), (2, 8, 8, 11008, 512, 1, True), (2, 8, 8, 1024, 4096, 1, False)]
+    grp, lds, xs, outs = build_group(specs, dev, seed=41)
+    first = []
+    for rep in range(3):
+        for (w, xt, out), x in zip(grp._keep, xs):
+            xt.copy_(torch.from_numpy(x if rep % 2 == 0 else -x))
+        grp.run()
+        first.append([o.clone() for o in outs])
+    check_status()
+    for rep, ys in enumerate(first):
+        sign = 1 if rep % 2 == 0 else -1
+        for (M, B, g, K, N, batch, _), ld, x, y in zip(specs, lds, xs, ys):
+            y_ref = oracle.linear((sign * x.astype(np.float32)).astype(np.float16), ld.codes, ld.codebooks,
+                                  ld.scales, ld.bias, M, B, g)
+            assert_close(y.cpu().numpy(), y_ref, f"rep {rep} K={K} N={N}")
+    for a, b in zip(first[0], first[2]):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), "grouped runs differ"
+
+
+def test_group_larger_than_one_launch(dev):
+    """20 grouped layers: two launch pairs sharing one workspace."""
+    specs = [(2, 8, 8, 64 * (1 + i % 5), 50 + 37 * i, 1, i % 3 == 0) for i in range(20)]
+    grp, lds, xs, outs = build_group(specs, dev, seed=42)
+    grp.run()
+    check_status()
+    for (M, B, g, K, N, batch, _), ld, x, out in zip(specs, lds, xs, outs):
+        y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+        assert_close(out.cpu().numpy(), y_ref, f"K={K} N={N}")
+
+
+def test_group_integer_layers_bit_exact(dev):
+    """Small-integer codebooks and x: every lookup, half2 pair sum and fp32 partial
+    is an exact integer, so y must equal the oracle bit for bit."""
+    rng = np.random.Generator(np.random.PCG64(43))
+    items, refs = [], []
+    for N, K in ((260, 512), (70, 1024), (129, 64)):
+        cb = rng.integers(-2, 3, size=(2, 256, 8)).astype(np.float16)
+        codes = rng.integers(0, 256, size=(N, K // 8, 2)).astype(np.uint8)
+        sc = rng.choice(np.array([1.0, 2.0]), size=N).astype(np.float16)
+        bias = rng.integers(-3, 4, size=N).astype(np.float16)
+        x = rng.integers(-1, 2, size=(1, K)).astype(np.float16)
+        y_ref = oracle.linear(x, codes, cb, sc, bias, 2, 8, 8)
+        assert np.abs(y_ref).max() <= 2048 and np.array_equal(y_ref, np.round(y_ref))
+        w = L.AqlmWeights.from_numpy(synth.LayerData(2, 8, 8, K, N, codes, cb, sc, bias), dev)
+        items.append((w, torch.from_numpy(x).to(dev), torch.empty((1, N), dtype=torch.float16, device=dev)))
+        refs.append(y_ref)
+    L.LayerGroup(items).run()
+    check_status()
+    for (_, _, out), y_ref in zip(items, refs):
+        y = out.cpu().numpy().astype(np.float64)
+        assert np.array_equal(y, y_ref), int((y != y_ref).sum())
+
+
+def test_group_zero_codebooks_give_bias(dev):
+    ld = synth.make_layer(2, 8, 8, 1024, 300, seed=44, with_bias=True)
+    ld.codebooks[:] = 0
+    w = L.AqlmWeights.from_numpy(ld, dev)
+    x = torch.from_numpy(synth.make_x(1, 1024, seed=44)).to(dev)
+    out = torch.empty((1, 300), dtype=torch.float16, device=dev)
+    L.LayerGroup([(w, x, out)]).run()
+    check_status()
+    assert np.array_equal(out.cpu().numpy()[0], ld.bias)
+
+
+@pytest.mark.parametrize("wname", ["llama2_7b_layer_set_2x8g8", "mixtral_8x7b_experts_2x8g8"])
+def test_group_published_layer_sets_sampled_rows(dev, wname):
+    """A published layer set as one group call; the oracle computes sampled rows."""
+    w = workloads.get(wname)
+    items, lds, xs = [], [], []
+    for li, lay in enumerate(w.layers):
+        s = lay.scheme
+        ld = synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index, layer=li)
+        x = synth.make_x(1, lay.K, seed=0, workload=w.index, layer=li)
+        items.append((L.AqlmWeights.from_numpy(ld, dev), torch.from_numpy(x).to(dev),
+                      torch.empty((1, lay.N), dtype=torch.float16, device=dev)))
+        lds.append(ld)
+        xs.append(x)
+    L.LayerGroup(items).run()
+    check_status()
+    rng = np.random.Generator(np.random.PCG64(45))
+    for li, (lay, ld, x, item) in enumerate(zip(w.layers, lds, xs, items)):
+        rows = np.unique(np.concatenate([rng.choice(lay.N, size=24, replace=False), [0, lay.N - 1, 63, 64]]))
+        s = lay.scheme
+        y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, s.M, s.B, s.g, rows=rows)
+        y = item[2].cpu().numpy()
+        assert np.isfinite(y.astype(np.float32)).all()
+        assert_close(y[:, rows], y_ref, f"{wname}/{lay.name}")

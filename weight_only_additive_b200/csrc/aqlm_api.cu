@@ -84,7 +84,7 @@ EncodeTiledFn encode_tiled() {
 
 extern "C" {
 
-int aqlm_abi_version(void) { return 1; }
+int aqlm_abi_version(void) { return 2; }
 
 const char* aqlm_status_string(aqlm_status status) {
   switch (status) {
@@ -157,6 +157,121 @@ aqlm_status aqlm_matmul(const void* x, const void* codes, const void* codebooks,
                         int M, int B, int g, int K, int N, int batch, aqlm_stream_t stream) {
   return aqlm_matmul_path(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch,
                           AQLM_PATH_AUTO, stream);
+}
+
+namespace {
+
+struct ByteRange {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+ByteRange range_of(const void* p, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return ByteRange{a, a + bytes};
+}
+
+bool overlaps(ByteRange a, ByteRange b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi; }
+
+// Every buffer of a (validated) problem, y last.
+int problem_ranges(const aqlm_problem& q, ByteRange (&r)[6]) {
+  const size_t code_bytes = static_cast<size_t>(q.N) * (q.K / q.g) * q.M * (q.B <= 8 ? 1 : 2);
+  r[0] = range_of(q.x, static_cast<size_t>(q.batch) * q.K * 2);
+  r[1] = range_of(q.codes, code_bytes);
+  r[2] = range_of(q.codebooks, static_cast<size_t>(q.M) * (size_t{1} << q.B) * q.g * 2);
+  r[3] = range_of(q.scales, static_cast<size_t>(q.N) * 2);
+  r[4] = range_of(q.bias, q.bias ? static_cast<size_t>(q.N) * 2 : 0);
+  r[5] = range_of(q.y, static_cast<size_t>(q.batch) * q.N * 2);
+  return 6;
+}
+
+aqlm::Problem to_problem(const aqlm_problem& q) {
+  return aqlm::Problem{q.x, q.codes, q.codebooks, q.scales, q.bias, q.y, q.M, q.B, q.g, q.K, q.N, q.batch};
+}
+
+// Workspace of the grouped runs: the largest run of up to kMaxGroupLayers
+// grouped problems (in call order).
+size_t group_workspace(const aqlm_problem* problems, int count) {
+  size_t best = 0, cur = 0;
+  int in_run = 0;
+  for (int i = 0; i < count; ++i) {
+    const aqlm::Problem p = to_problem(problems[i]);
+    if (!aqlm::lut_group_supported(p)) continue;
+    if (in_run == aqlm::kMaxGroupLayers) {
+      cur = 0;
+      in_run = 0;
+    }
+    cur += aqlm::lut_group_workspace_bytes(&p, 1);
+    ++in_run;
+    if (cur > best) best = cur;
+  }
+  return best;
+}
+
+}  // namespace
+
+size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count) {
+  if (!problems || count <= 0) return 0;
+  for (int i = 0; i < count; ++i) {
+    const aqlm_problem& q = problems[i];
+    if (validate_shape(q.M, q.B, q.g, q.K, q.N, q.batch) != AQLM_OK) return 0;
+  }
+  return group_workspace(problems, count);
+}
+
+aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* workspace,
+                              size_t workspace_bytes, aqlm_stream_t stream) {
+  if (count == 0) return AQLM_OK;
+  if (count < 0 || !problems) return AQLM_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const aqlm_problem& q = problems[i];
+    const aqlm_status st = aqlm_validate(q.x, q.codes, q.codebooks, q.scales, q.bias, q.y, q.M, q.B, q.g, q.K,
+                                         q.N, q.batch, AQLM_PATH_AUTO);
+    if (st != AQLM_OK) return st;
+  }
+  // independence: no output may overlap another problem's buffers
+  for (int i = 0; i < count; ++i) {
+    ByteRange ri[6];
+    problem_ranges(problems[i], ri);
+    for (int j = 0; j < count; ++j) {
+      if (j == i) continue;
+      ByteRange rj[6];
+      problem_ranges(problems[j], rj);
+      for (int k = 0; k < 6; ++k)
+        if (overlaps(ri[5], rj[k])) return AQLM_ERR_INVALID_ARG;
+    }
+  }
+  const size_t need = group_workspace(problems, count);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return AQLM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return AQLM_ERR_MISALIGNED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  aqlm::Problem run[aqlm::kMaxGroupLayers];
+  int n_run = 0;
+  uint32_t* status = nullptr;
+  if (need > 0) {
+    status = device_status_ptr();
+    if (!status) return from_cuda(cudaErrorInvalidDevice);
+  }
+  for (int i = 0; i <= count; ++i) {
+    const bool flush = (i == count) || n_run == aqlm::kMaxGroupLayers;
+    if (flush && n_run > 0) {
+      const aqlm_status st = from_cuda(aqlm::launch_lut_group(run, n_run, workspace, status, s));
+      if (st != AQLM_OK) return st;
+      n_run = 0;
+    }
+    if (i == count) break;
+    const aqlm::Problem p = to_problem(problems[i]);
+    if (aqlm::lut_group_supported(p)) {
+      run[n_run++] = p;
+    } else {
+      const aqlm_problem& q = problems[i];
+      const aqlm_status st = aqlm_matmul_path(q.x, q.codes, q.codebooks, q.scales, q.bias, q.y, q.M, q.B, q.g, q.K,
+                                              q.N, q.batch, AQLM_PATH_AUTO, stream);
+      if (st != AQLM_OK) return st;
+    }
+  }
+  return AQLM_OK;
 }
 
 aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void* scales,

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 namespace aqlm {
@@ -21,6 +22,8 @@ enum : uint32_t {
   kSitePipeEmpty = 0x302,   // pipelined tensor-core kernel: waiting for a stage to be released
   kSitePipeCodes = 0x303,   // pipelined tensor-core kernel: code-tile ring
   kSitePipeAcc = 0x304,     // pipelined tensor-core kernel: waiting for the accumulator
+  kSiteGroupRing = 0x401,   // grouped lookup-table kernel: code-tile ring (landing / slot release)
+  kSiteGroupMma = 0x402,    // grouped lookup-table kernel: waiting for the table-building MMA
 };
 
 struct Problem {
@@ -58,6 +61,16 @@ inline bool tc_pipelined_shape(int M, int B, int g, int K) {
   const long long row_bytes = static_cast<long long>(K / g) * M * (B <= 8 ? 1 : 2);
   return K % 64 == 0 && row_bytes % 16 == 0;
 }
+
+// Grouped lookup-table GEMV over independent 2x8 g8 batch-1 layers (one launch
+// of the partial-sum kernel, one of the reduction), at most kMaxGroupLayers per
+// launch.  The workspace holds every layer's fp32 partials, [ceil(G/64)][N] each,
+// 256-byte aligned.
+constexpr int kMaxGroupLayers = 16;
+bool lut_group_supported(const Problem& p);
+size_t lut_group_workspace_bytes(const Problem* probs, int count);
+cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, uint32_t* status,
+                             cudaStream_t stream);
 
 // True if the scheme is one the kernels are instantiated for.
 inline bool scheme_supported(int M, int B, int g) {

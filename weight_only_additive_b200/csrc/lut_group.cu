@@ -1,0 +1,535 @@
+// Grouped lookup-table GEMV: one launch computes a set of independent 2x8 g8,
+// batch-1 layers (a decoder block's linears), the "fast lookup, no per-element
+// dequantization" path of the inference-research record "AQLM (additive /
+// multi-codebook quantization)", section "Kernels", applied to a whole layer set
+// so that no layer pays its own launch, set-up and tail.
+//
+//   T_m[j][i] = sum_t x[8j + t] * C_m[i][t]                 (group j, codebook m, entry i)
+//   part[s][n] = sum_{j in slice s} (T_0[j][codes[n,j,0]] + T_1[j][codes[n,j,1]])
+//   y[n]       = s_n * sum_s part[s][n] + bias_n             (second kernel, s ascending)
+//
+// Work items.  Item (p, s, t) is layer p's 64-group K slice s on its 64-row tile
+// t; a layer has ceil(G / 64) x ceil(N / 64) items.  Items are numbered layer by
+// layer, slice-major, and every CTA (one per SM, persistent) takes a contiguous
+// range of them, so consecutive items mostly share (p, s) and therefore the
+// lookup table: a CTA rebuilds it only when (p, s) changes.
+//
+// Per CTA:
+//   warp 16     TMA producer: streams the code tile (64 rows x 128 bytes) of every
+//               item of the range into a ring of shared-memory slots, running as
+//               far ahead as the ring allows; codes are read exactly once.
+//   warps 0-15  table builders and lookup workers.  On a new (p, s) they wait for
+//               the prefetched operands (x slice, both codebooks), issue two
+//               tcgen05.mma (M = 128 rows of x groups, N = 256 entries, K = 16 with
+//               the upper 8 zero) into TMEM and move the table to shared memory as
+//               fp16 pairs (T_0, T_1) per (entry, group).  Then warps 4j..4j+3 take
+//               the tiles k = j (mod 4), two interleaved 8-row tasks per warp, and
+//               write each row's fp32 partial to the workspace.
+// The partials of a row are summed over the slices in ascending order by a second
+// small kernel (programmatic dependent launch), which applies the channel scale
+// and bias: the result does not depend on which CTA ran which item.
+//
+// Bank-conflict-free lookups: as in the single-layer lookup-table kernel, lane
+// (r8, q4) reads code word 8 q4 + ((r8 + s) mod 8) at step s, and the table keeps
+// group 2w in word column w and group 2w + 1 in column 32 + w of each entry's
+// 64-word row, so the 32 lanes of every table read hit 32 different banks.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "aqlm_device.cuh"
+
+namespace aqlm {
+namespace {
+
+constexpr int kWorkers = 512;                      // warps 0-15
+constexpr int kThreads = kWorkers + 32;            // + TMA producer warp
+constexpr int kProducerWarp = kWorkers / 32;
+constexpr int kTileRows = 64;
+constexpr uint32_t kTileBytes = 64u * 128u;        // 64 rows x 64 groups x 2 codes
+constexpr uint32_t kLutBytes = 256u * 64u * 4u;    // 64 KB
+constexpr uint32_t kAOpBytes = 128u * 32u;         // 4 KB
+constexpr uint32_t kBOpBytes = 256u * 32u;         // 8 KB per codebook
+constexpr int kSlots = 14;                         // 112 KB of code tiles in flight
+constexpr int kTileGroups = 4;                     // warps 4j..4j+3 take tiles k = j (mod 4)
+constexpr uint32_t kTmemCols = 512;                // D_0 at [0, 256), D_1 at [256, 512)
+
+constexpr uint32_t kOffLut = 0;
+constexpr uint32_t kOffA = kOffLut + kLutBytes;                 // 2 buffers
+constexpr uint32_t kOffB = kOffA + 2 * kAOpBytes;               // 2 buffers x 2 codebooks
+constexpr uint32_t kOffRing = kOffB + 4 * kBOpBytes;            // 1024-aligned
+constexpr uint32_t kOffBars = kOffRing + kSlots * kTileBytes;
+constexpr uint32_t kSmemBytes = kOffBars + 8u * (2 * kSlots + 1) + 16u;
+static_assert(kOffRing % 1024 == 0, "ring slots must stay 1024-byte aligned");
+static_assert(kSmemBytes <= 227u * 1024u, "shared memory budget");
+
+struct GroupLayerDev {
+  const __half* x;
+  const __half* codebooks;
+  const __half* scales;
+  const __half* bias;
+  __half* y;
+  float* part;   // [S][N] fp32 partials in the workspace
+  int N, G, S, T;  // rows, groups, 64-group slices, 64-row tiles
+  long long item0; // first item of this layer
+  long long row0;  // first output row of this layer in the reduction grid
+};
+
+struct GroupParams {
+  GroupLayerDev layer[kMaxGroupLayers];
+  int count;
+  long long items;
+  long long rows;
+  uint32_t* status;
+};
+
+struct GroupMaps {
+  CUtensorMap map[kMaxGroupLayers];
+};
+
+__device__ __forceinline__ uint32_t tmem_lane_base(int warp) { return static_cast<uint32_t>(32 * (warp & 3)) << 16; }
+
+// Named barrier over the 16 worker warps that also ANDs a flag across them.
+__device__ __forceinline__ bool workers_sync_and(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(v ? 1u : 0u), "n"(kWorkers)
+      : "memory");
+  return out != 0;
+}
+
+// Bounded wait that gives up at once when another role has aborted.
+__device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                           uint32_t* status, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      record_failure(status, site);
+      *abort_flag = 1u;
+      return false;
+    }
+  }
+  return true;
+}
+
+// Layer of a global item index (layers are few; a linear scan is cheapest).
+__device__ __forceinline__ int layer_of(const GroupParams& p, long long item) {
+  int l = 0;
+  while (l + 1 < p.count && p.layer[l + 1].item0 <= item) ++l;
+  return l;
+}
+
+// Position of an item as (layer, slice, tile); advanced one item at a time so the
+// loops need no division (items are numbered layer by layer, slice-major).
+struct ItemCursor {
+  int l, s, t;
+  __device__ __forceinline__ void seek(const GroupParams& p, long long item) {
+    l = layer_of(p, item);
+    const long long local = item - p.layer[l].item0;
+    s = static_cast<int>(local / p.layer[l].T);
+    t = static_cast<int>(local - static_cast<long long>(s) * p.layer[l].T);
+  }
+  __device__ __forceinline__ void next(const GroupParams& p) {
+    if (++t == p.layer[l].T) {
+      t = 0;
+      if (++s == p.layer[l].S) {
+        s = 0;
+        ++l;
+      }
+    }
+  }
+};
+
+// No-swizzle K-major operand layout: 8-row x 16-byte core matrices, the two
+// K halves 128 bytes apart, consecutive 8-row groups 256 bytes apart.
+__host__ __device__ inline uint32_t kmajor_offset(int row, int khalf) {
+  return static_cast<uint32_t>((row >> 3) * 256 + khalf * 128 + (row & 7) * 16);
+}
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t smem_byte_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;
+  d |= static_cast<uint64_t>(256u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Operands of slice s of layer l into buffer `buf` (cp.async, caller commits):
+// A row rho holds x group 2 (rho mod 32) + (rho / 32 mod 2) of the slice (rows
+// 64-127 repeat rows 0-63), zero past the layer's last group; B holds the two
+// codebooks, one 16-byte codeword per row.  The zero upper K halves are written
+// once at start-up.
+__device__ __forceinline__ void load_operands(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
+  const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * kAOpBytes;
+  const uint32_t bo = kOffB + static_cast<uint32_t>(buf) * 2u * kBOpBytes;
+  for (int i = wtid; i < 128 + 512; i += kWorkers) {
+    if (i < 128) {
+      const int rho = i;
+      const int gg = s * 64 + 2 * (rho & 31) + ((rho >> 5) & 1);
+      const bool valid = gg < L.G;
+      cp_async_16_zfill(sbase + ao + kmajor_offset(rho, 0),
+                        valid ? static_cast<const void*>(L.x + static_cast<size_t>(gg) * 8)
+                              : static_cast<const void*>(L.x),
+                        valid ? 16u : 0u);
+    } else {
+      const int e = i - 128;  // codebook m = e / 256, entry e % 256
+      cp_async_16_zfill(sbase + bo + static_cast<uint32_t>(e >> 8) * kBOpBytes + kmajor_offset(e & 255, 0),
+                        L.codebooks + static_cast<size_t>(e) * 8, 16u);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_constant__ GroupMaps maps,
+                                                                const __grid_constant__ GroupParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // the ring slots are TMA destinations: keep the layout 1024-byte aligned
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_addr(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBars);  // tile landed
+  uint64_t* empty = full + kSlots;                                  // tile read by its 8 warps
+  uint64_t* mma_bar = empty + kSlots;                               // table MMAs done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const long long it0 = p.items * blockIdx.x / gridDim.x;
+  const long long it1 = p.items * (blockIdx.x + 1) / gridDim.x;
+
+  // The next kernel in the stream (the reduction) may be scheduled now; it waits
+  // for this grid to complete before it reads the partials.
+  grid_dependents_launch();
+  if (tid == 0) {
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kWorkers / 32 / kTileGroups);
+    }
+    mbar_init(mma_bar, 1);
+    *abort_flag = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // zero upper K halves of both operand buffers (never written again)
+  for (int i = tid; i < 2 * (128 + 512); i += kThreads) {
+    const int buf = i / 640, j = i % 640;
+    const uint32_t off = j < 128 ? kOffA + static_cast<uint32_t>(buf) * kAOpBytes + kmajor_offset(j, 1)
+                                 : kOffB + static_cast<uint32_t>(buf) * 2u * kBOpBytes +
+                                       static_cast<uint32_t>((j - 128) >> 8) * kBOpBytes + kmajor_offset((j - 128) & 255, 1);
+    *reinterpret_cast<uint4*>(smem + off) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    // ---- code tiles of every item of the range, in order (weights: no dependency wait) ----
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      ItemCursor c;
+      c.seek(p, it0);
+      int slot = 0;
+      uint32_t use = 0;
+      for (long long it = it0; it < it1; ++it, c.next(p)) {
+        if (use > 0 && !group_wait(&empty[slot], (use - 1u) & 1u, abort_flag, p.status, kSiteGroupRing)) break;
+        mbar_arrive_expect_tx(&full[slot], kTileBytes);
+        // bytes past the row end and rows past N are zero-filled
+        tma_load_2d(sbase + kOffRing + static_cast<uint32_t>(slot) * kTileBytes, &maps.map[c.l], c.s * 128,
+                    c.t * kTileRows, &full[slot], pol);
+        if (++slot == kSlots) {
+          slot = 0;
+          ++use;
+        }
+      }
+    }
+  } else {
+    // ---- workers ------------------------------------------------------------------------
+    // x is read (table operands) and the workspace written only after the previous
+    // kernel in the stream has completed.
+    grid_dependency_wait();
+    const int wtid = tid;
+    const int wg = warp >> 2;    // tiles k = wg (mod 4) are this warp's
+    const int task = warp & 3;   // its two 8-row tasks of such a tile: task and task + 4
+    const int r8 = lane >> 2;    // row of the task
+    const int q4 = lane & 3;     // quarter of the row's 32 code words
+    const uint32_t idesc = umma_idesc_f16_f32(128, 256);
+    // byte offset (4 x word column) of the code word lane (r8, q4) reads at step s8
+    uint32_t wv[8];
+#pragma unroll
+    for (int s8 = 0; s8 < 8; ++s8) wv[s8] = static_cast<uint32_t>((8 * q4 + ((r8 + s8) & 7)) << 2);
+    uint32_t mma_phase = 0;
+    bool ok = true;
+    int cur_l = -1, cur_s = -1, run = 0;
+    if (it0 < it1) {
+      const int l = layer_of(p, it0);
+      load_operands(p.layer[l], static_cast<int>((it0 - p.layer[l].item0) / p.layer[l].T), sbase, 0, wtid);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+
+    ItemCursor c;
+    c.seek(p, it0);
+    int slot = 0;        // ring slot of item k
+    uint32_t ph = 0;     // its phase
+    for (long long k = 0; it0 + k < it1; ++k, c.next(p)) {
+      const int l = c.l, s = c.s, t = c.t;
+      const GroupLayerDev& L = p.layer[l];
+      const int my_slot = slot;
+      const uint32_t my_ph = ph;
+      if (++slot == kSlots) {
+        slot = 0;
+        ph ^= 1u;
+      }
+      if (l != cur_l || s != cur_s) {
+        // ---- new (layer, slice): table from the prefetched operands in buffer run & 1 ----
+        const int buf = run & 1;
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        ok = workers_sync_and(ok);  // old table no longer read; operands in place
+        tc_fence_after_sync();
+        if (ok && wtid == 0) {
+          const uint64_t adesc = kmajor_desc(sbase + kOffA + static_cast<uint32_t>(buf) * kAOpBytes);
+          const uint32_t bo = sbase + kOffB + static_cast<uint32_t>(buf) * 2u * kBOpBytes;
+          umma_f16_ss(tmem, adesc, kmajor_desc(bo), idesc, 0u);
+          umma_f16_ss(tmem + 256u, adesc, kmajor_desc(bo + kBOpBytes), idesc, 0u);
+          umma_commit(mma_bar);
+        }
+        // prefetch the operands of the range's next (layer, slice) into the other buffer,
+        // whose MMAs completed before the previous table was stored
+        const long long run_end = std::min(it1, L.item0 + static_cast<long long>(s + 1) * L.T);
+        if (ok && run_end < it1) {
+          // the next (layer, slice) in item order
+          const int nl = (s + 1 < L.S) ? l : l + 1;
+          load_operands(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        const bool done = ok && group_wait(mma_bar, mma_phase, abort_flag, p.status, kSiteGroupMma);
+        mma_phase ^= 1u;
+        ok = workers_sync_and(done);
+        tc_fence_after_sync();
+        if (ok) {
+          // TMEM -> shared-memory table; A rows rho and rho + 64 hold the same group, so
+          // all 16 warps take part: warp w reads lane quadrant w mod 4
+          const int qd = warp & 3;
+          const int col = 32 * (qd & 1) + lane;               // word column = rho mod 64
+          const int i0 = 32 * (2 * (warp >> 2) + (qd >> 1));  // 32 table entries per warp
+          uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kOffLut);
+          uint32_t r0[32], r1[32];
+          tmem_ld_x32(tmem + tmem_lane_base(warp) + static_cast<uint32_t>(i0), r0);
+          tmem_ld_x32(tmem + tmem_lane_base(warp) + 256u + static_cast<uint32_t>(i0), r1);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            lut[(i0 + j) * 64 + col] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
+        }
+        tc_fence_before_sync();
+        ok = workers_sync_and(ok);  // table complete
+        cur_l = l;
+        cur_s = s;
+        ++run;
+      }
+      if ((k & (kTileGroups - 1)) != wg) continue;
+      // ---- lookups of this item's tile: rows 8 task + r8 and 32 + 8 task + r8 ----
+      const bool landed =
+          __all_sync(0xffffffffu, ok && group_wait(&full[my_slot], my_ph, abort_flag, p.status, kSiteGroupRing));
+      if (landed) {
+        const uint32_t* rowA = reinterpret_cast<const uint32_t*>(
+            smem + kOffRing + static_cast<uint32_t>(my_slot) * kTileBytes + static_cast<uint32_t>(task * 8 + r8) * 128u);
+        const uint32_t* rowB = rowA + 32 * 32;  // 32 rows further
+        uint32_t cwA[8], cwB[8];
+#pragma unroll
+        for (int s8 = 0; s8 < 8; ++s8) {
+          cwA[s8] = rowA[wv[s8] >> 2];
+          cwB[s8] = rowB[wv[s8] >> 2];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[my_slot]);  // the tile's codes are in registers
+        __half2 haccA = __float2half2_rn(0.f), haccB = haccA;
+        const uint8_t* lut = smem + kOffLut;
+#pragma unroll
+        for (int s8 = 0; s8 < 8; ++s8) {
+          // table byte offsets: entry * 256 + column * 4 (column w, or 32 + w at +128);
+          // (codebook-0 half of one word, codebook-1 half of the other) per group
+          const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5504));
+          const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5514));
+          const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5524) + 128u);
+          const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5534) + 128u);
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5504));
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5514));
+          const uint32_t b2 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5524) + 128u);
+          const uint32_t b3 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5534) + 128u);
+          const uint32_t pa01 = __byte_perm(a0, a1, 0x7610), pa23 = __byte_perm(a2, a3, 0x7610);
+          const uint32_t pb01 = __byte_perm(b0, b1, 0x7610), pb23 = __byte_perm(b2, b3, 0x7610);
+          haccA = __hadd2(haccA, __hadd2(*reinterpret_cast<const __half2*>(&pa01), *reinterpret_cast<const __half2*>(&pa23)));
+          haccB = __hadd2(haccB, __hadd2(*reinterpret_cast<const __half2*>(&pb01), *reinterpret_cast<const __half2*>(&pb23)));
+        }
+        const float2 fa = __half22float2(haccA), fb = __half22float2(haccB);
+        float va = fa.x + fa.y, vb = fb.x + fb.y;
+        va += __shfl_xor_sync(0xffffffffu, va, 1);
+        vb += __shfl_xor_sync(0xffffffffu, vb, 1);
+        va += __shfl_xor_sync(0xffffffffu, va, 2);
+        vb += __shfl_xor_sync(0xffffffffu, vb, 2);
+        if (q4 == 0) {
+          const int row = t * kTileRows + task * 8 + r8;
+          float* dst = L.part + static_cast<size_t>(s) * L.N;
+          if (row < L.N) dst[row] = va;
+          if (row + 32 < L.N) dst[row + 32] = vb;
+        }
+      } else {
+        ok = false;
+        if (lane == 0) mbar_arrive(&empty[my_slot]);
+      }
+    }
+  }
+
+  if (*abort_flag) {
+    // a wait gave up: let copies already in flight land before the CTA leaves
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 50000ull) {
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// y[n] = fp16(s_n * sum_s part[s][n] + bias_n), slices in ascending order.
+__global__ void __launch_bounds__(256) lut_group_reduce_kernel(const __grid_constant__ GroupParams p) {
+  grid_dependents_launch();
+  const long long row = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  if (row >= p.rows) return;
+  int l = 0;
+  while (l + 1 < p.count && p.layer[l + 1].row0 <= row) ++l;
+  const GroupLayerDev& L = p.layer[l];
+  const int n = static_cast<int>(row - L.row0);
+  const float sc = __half2float(L.scales[n]);
+  const float bi = L.bias ? __half2float(L.bias[n]) : 0.f;
+  // the partials are the previous kernel's output
+  grid_dependency_wait();
+  float acc = 0.f;
+  for (int s = 0; s < L.S; ++s) acc += L.part[static_cast<size_t>(s) * L.N + n];
+  L.y[n] = __float2half_rn(acc * sc + bi);
+}
+
+}  // namespace
+}  // namespace aqlm
+
+namespace aqlm {
+
+bool lut_group_supported(const Problem& p) {
+  return p.M == 2 && p.B == 8 && p.g == 8 && p.batch == 1 && p.K % 64 == 0;
+}
+
+namespace {
+inline size_t part_bytes(const Problem& p) {
+  const size_t slices = static_cast<size_t>((p.K / 8 + 63) / 64);
+  return (slices * static_cast<size_t>(p.N) * sizeof(float) + 255u) & ~static_cast<size_t>(255u);
+}
+}  // namespace
+
+size_t lut_group_workspace_bytes(const Problem* probs, int count) {
+  size_t bytes = 0;
+  for (int i = 0; i < count; ++i)
+    if (lut_group_supported(probs[i])) bytes += part_bytes(probs[i]);
+  return bytes;
+}
+
+// All problems must satisfy lut_group_supported; count <= kMaxGroupLayers; the
+// workspace holds lut_group_workspace_bytes(probs, count) bytes, 256-byte aligned.
+cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, uint32_t* status,
+                             cudaStream_t stream) {
+  if (count <= 0 || count > kMaxGroupLayers) return cudaErrorInvalidValue;
+  EncodeTiledFn encode = encode_tiled();
+  if (!encode) return cudaErrorNotSupported;
+  GroupParams p{};
+  GroupMaps maps{};
+  long long items = 0, rows = 0;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  for (int i = 0; i < count; ++i) {
+    const Problem& pr = probs[i];
+    if (!lut_group_supported(pr)) return cudaErrorInvalidValue;
+    GroupLayerDev& L = p.layer[i];
+    L.x = static_cast<const __half*>(pr.x);
+    L.codebooks = static_cast<const __half*>(pr.codebooks);
+    L.scales = static_cast<const __half*>(pr.scales);
+    L.bias = static_cast<const __half*>(pr.bias);
+    L.y = static_cast<__half*>(pr.y);
+    L.part = reinterpret_cast<float*>(ws);
+    ws += part_bytes(pr);
+    L.N = pr.N;
+    L.G = pr.K / 8;
+    L.S = (L.G + 63) / 64;
+    L.T = (pr.N + kTileRows - 1) / kTileRows;
+    L.item0 = items;
+    L.row0 = rows;
+    items += static_cast<long long>(L.S) * L.T;
+    rows += pr.N;
+    // codes as a 2D byte tensor [N rows][2G bytes]; a box is 64 rows x 128 bytes
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(L.G) * 2, static_cast<cuuint64_t>(pr.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(L.G) * 2};
+    const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kTileRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&maps.map[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pr.codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  p.count = count;
+  p.items = items;
+  p.rows = rows;
+  p.status = status;
+
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
+  const uint32_t smem = kSmemBytes + 1024u;
+  auto kern = lut_group_kernel;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min<long long>(items, sms)), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, maps, p);
+  if (e != cudaSuccess) return e;
+
+  cudaLaunchConfig_t rcfg = {};
+  rcfg.gridDim = dim3(static_cast<unsigned>((rows + 255) / 256), 1, 1);
+  rcfg.blockDim = dim3(256, 1, 1);
+  rcfg.stream = stream;
+  rcfg.attrs = attr;
+  rcfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&rcfg, lut_group_reduce_kernel, p);
+}
+
+}  // namespace aqlm

@@ -97,3 +97,39 @@ def dequantize(w: AqlmWeights, out: Optional[torch.Tensor] = None,
 def check_device_status(stream: Optional[torch.cuda.Stream] = None, device=None):
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     return native.aqlm_check_device_status(_stream_handle(stream, dev))
+
+
+class LayerGroup:
+    """A set of independent layers computed by one aqlm_matmul_group call.
+
+    `items` is a sequence of (weights, x, out) with x [batch, K] and out [batch, N]
+    fp16 tensors on the weights' device.  The problem table and the workspace are
+    built once; run() enqueues the whole set on a stream (and may be captured in
+    a CUDA graph).
+    """
+
+    def __init__(self, items, device=None):
+        if not items:
+            raise ValueError("a layer group needs at least one layer")
+        dev = items[0][0].codes.device if device is None else torch.device(device)
+        probs = []
+        self._keep = []
+        for w, x, out in items:
+            _check_tensor(x, "x", torch.float16, dev)
+            _check_tensor(out, "out", torch.float16, dev)
+            batch, K = x.shape
+            if K != w.K or tuple(out.shape) != (batch, w.N):
+                raise ValueError(f"shapes: x {tuple(x.shape)}, out {tuple(out.shape)}, weights N={w.N} K={w.K}")
+            probs.append((x.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(), w.scales.data_ptr(),
+                          _ptr(w.bias), out.data_ptr(), w.M, w.B, w.g, K, w.N, batch))
+            self._keep.append((w, x, out))
+        self.device = dev
+        self.problems = native.problem_array(probs)
+        self.count = len(probs)
+        self.workspace_bytes = native.aqlm_group_workspace_size(self.problems, self.count)
+        # 256-byte aligned: torch's caching allocator hands out 512-byte aligned blocks
+        self.workspace = torch.empty((max(self.workspace_bytes, 1),), dtype=torch.uint8, device=dev)
+
+    def run(self, stream: Optional[torch.cuda.Stream] = None):
+        native.aqlm_matmul_group(self.problems, self.workspace.data_ptr(), self.workspace_bytes,
+                                 _stream_handle(stream, self.device), count=self.count)

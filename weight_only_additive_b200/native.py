@@ -17,9 +17,10 @@ LIBRARY = os.path.join(PKG, "libaqlm.so")
 # Every exported symbol of include/aqlm.h.
 EXPORTS = ("aqlm_matmul", "aqlm_matmul_path", "aqlm_dequantize", "aqlm_select_path",
            "aqlm_validate", "aqlm_status_string", "aqlm_check_device_status",
-           "aqlm_last_cuda_error", "aqlm_abi_version")
+           "aqlm_last_cuda_error", "aqlm_abi_version", "aqlm_matmul_group",
+           "aqlm_group_workspace_size")
 
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 
 class Status(enum.IntEnum):
@@ -36,6 +37,14 @@ class Path(enum.IntEnum):
     GEMV = 1
     GEMV_LUT = 2
     TENSOR_CORE = 3
+
+
+class AqlmProblem(ctypes.Structure):
+    """aqlm_problem: one layer of a group call (raw device pointers and sizes)."""
+    _fields_ = [("x", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("codebooks", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("M", ctypes.c_int), ("B", ctypes.c_int), ("g", ctypes.c_int), ("K", ctypes.c_int),
+                ("N", ctypes.c_int), ("batch", ctypes.c_int)]
 
 
 class AqlmError(RuntimeError):
@@ -82,6 +91,10 @@ def lib() -> ctypes.CDLL:
                 L.aqlm_check_device_status.restype = _i
                 L.aqlm_last_cuda_error.restype = _i
                 L.aqlm_abi_version.restype = _i
+                L.aqlm_matmul_group.argtypes = [ctypes.POINTER(AqlmProblem), _i, _vp, ctypes.c_size_t, _vp]
+                L.aqlm_matmul_group.restype = _i
+                L.aqlm_group_workspace_size.argtypes = [ctypes.POINTER(AqlmProblem), _i]
+                L.aqlm_group_workspace_size.restype = ctypes.c_size_t
                 if L.aqlm_abi_version() != ABI_VERSION:
                     raise ImportError(f"libaqlm.so ABI {L.aqlm_abi_version()} != binding ABI {ABI_VERSION}")
                 _lib = L
@@ -128,3 +141,24 @@ def aqlm_check_device_status(stream=None):
     detail = ctypes.c_uint32(0)
     st = lib().aqlm_check_device_status(stream, ctypes.byref(detail))
     return Status(st), detail.value
+
+
+def problem_array(problems) -> ctypes.Array:
+    """An aqlm_problem[] from AqlmProblem instances or 12-tuples in C argument order."""
+    arr = (AqlmProblem * max(1, len(problems)))()
+    for i, q in enumerate(problems):
+        arr[i] = q if isinstance(q, AqlmProblem) else AqlmProblem(*q)
+    return arr
+
+
+def aqlm_matmul_group(problems, workspace, workspace_bytes, stream=None, count=None):
+    """`problems`: a ctypes aqlm_problem array (see problem_array) or a sequence."""
+    arr = problems if isinstance(problems, ctypes.Array) else problem_array(problems)
+    n = len(problems) if count is None else count
+    _check(lib().aqlm_matmul_group(arr, n, workspace, workspace_bytes, stream), "aqlm_matmul_group")
+
+
+def aqlm_group_workspace_size(problems, count=None) -> int:
+    arr = problems if isinstance(problems, ctypes.Array) else problem_array(problems)
+    n = len(problems) if count is None else count
+    return lib().aqlm_group_workspace_size(arr, n)
