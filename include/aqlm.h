@@ -148,6 +148,23 @@ typedef struct {
 aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* workspace,
                               size_t workspace_bytes, aqlm_stream_t stream);
 
+/*
+ * aqlm_matmul_group without a caller workspace, for callers that cannot
+ * allocate device memory.  The AQLM pages have no counterpart: this is a library
+ * convenience.  The partial sums live in a static device buffer of
+ * AQLM_STATIC_GROUP_SCRATCH_BYTES inside the library (one per device, its address
+ * taken with cudaGetSymbolAddress); the call allocates nothing.  Problems whose
+ * aqlm_group_workspace_size exceeds that size are rejected with
+ * AQLM_ERR_INVALID_ARG before anything is launched (8 MiB covers, for example,
+ * a Llama-2-7B decoder layer set or 16 Mixtral-8x7B expert linears).  The buffer
+ * needs no clearing: the reduction reads only partials written by the same call.
+ * Calls that overlap in time (different streams or host threads on one device)
+ * share the buffer and RACE: the caller must serialise them.  Calls on one
+ * stream are ordered and safe.  Otherwise identical to aqlm_matmul_group.
+ */
+#define AQLM_STATIC_GROUP_SCRATCH_BYTES (8u << 20)
+aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aqlm_stream_t stream);
+
 /* Workspace bytes aqlm_matmul_group needs for these problems: for every run of
  * up to 16 grouped problems, the sum over them of ceil(K / 512) * N * 4 bytes
  * rounded up to 256; the maximum over runs.  Pure host logic. */

@@ -163,3 +163,19 @@ def test_group_validation_needs_no_gpu(lib):
     q[5] = P[0][5]
     assert L_.aqlm_matmul_group(native.problem_array([P[0], tuple(q)]), 2, 1 << 40, need, None) == \
         Status.INVALID_ARG
+
+
+def test_group_static_validation_needs_no_gpu(lib):
+    L_ = native.lib()
+    assert L_.aqlm_matmul_group_static(native.problem_array([_prob(1 << 32)]), 0, None) == Status.OK
+    assert L_.aqlm_matmul_group_static(None, 1, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_group_static(native.problem_array([_prob(1 << 32)]), -3, None) == Status.INVALID_ARG
+    # 5 grouped 28672 x 8192 layers need 5 x 16 x 28672 x 4 bytes > 8 MiB
+    big = [_prob((i + 1) << 34, K=8192, N=28672) for i in range(5)]
+    assert native.aqlm_group_workspace_size(big) == 5 * _ws_bytes(8192, 28672) > native.STATIC_GROUP_SCRATCH_BYTES
+    assert L_.aqlm_matmul_group_static(native.problem_array(big), 5, None) == Status.INVALID_ARG
+    # 16 Mixtral-8x7B expert linears (4096 x 14336) fit
+    assert native.aqlm_group_workspace_size([_prob((i + 1) << 34, K=14336, N=4096) for i in range(16)]) == \
+        16 * _ws_bytes(14336, 4096) <= native.STATIC_GROUP_SCRATCH_BYTES
+    bad = [_prob(1 << 32, M=3)]
+    assert L_.aqlm_matmul_group_static(native.problem_array(bad), 1, None) == Status.UNSUPPORTED

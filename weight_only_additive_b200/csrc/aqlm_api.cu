@@ -13,6 +13,10 @@ namespace {
 // module).  Kernels record the site of a bounded wait that gave up here.
 __device__ uint32_t g_device_status;
 
+// Scratch of aqlm_matmul_group_static: fp32 partial sums between its two
+// kernels, one buffer per device (every device's copy of this module has one).
+__device__ __align__(256) uint8_t g_group_scratch[AQLM_STATIC_GROUP_SCRATCH_BYTES];
+
 thread_local int t_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
@@ -36,6 +40,28 @@ uint32_t* device_status_ptr() {
     g_status_ptr[dev] = static_cast<uint32_t*>(p);
   }
   return g_status_ptr[dev];
+}
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_group_scratch for the current device (nullptr on failure).
+void* static_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_group_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
 }
 
 aqlm_status from_cuda(cudaError_t e) {
@@ -84,7 +110,7 @@ EncodeTiledFn encode_tiled() {
 
 extern "C" {
 
-int aqlm_abi_version(void) { return 2; }
+int aqlm_abi_version(void) { return 3; }
 
 const char* aqlm_status_string(aqlm_status status) {
   switch (status) {
@@ -272,6 +298,26 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
     }
   }
   return AQLM_OK;
+}
+
+aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aqlm_stream_t stream) {
+  if (count == 0) return AQLM_OK;
+  if (count < 0 || !problems) return AQLM_ERR_INVALID_ARG;
+  const size_t need = aqlm_group_workspace_size(problems, count);
+  if (need > AQLM_STATIC_GROUP_SCRATCH_BYTES) return AQLM_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if (need > 0) {
+    // validate before touching the device, as every entry point does
+    for (int i = 0; i < count; ++i) {
+      const aqlm_problem& q = problems[i];
+      const aqlm_status st = aqlm_validate(q.x, q.codes, q.codebooks, q.scales, q.bias, q.y, q.M, q.B, q.g, q.K,
+                                           q.N, q.batch, AQLM_PATH_AUTO);
+      if (st != AQLM_OK) return st;
+    }
+    scratch = static_scratch_ptr();
+    if (!scratch) return from_cuda(cudaErrorInvalidDevice);
+  }
+  return aqlm_matmul_group(problems, count, scratch, AQLM_STATIC_GROUP_SCRATCH_BYTES, stream);
 }
 
 aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void* scales,

@@ -18,9 +18,12 @@ LIBRARY = os.path.join(PKG, "libaqlm.so")
 EXPORTS = ("aqlm_matmul", "aqlm_matmul_path", "aqlm_dequantize", "aqlm_select_path",
            "aqlm_validate", "aqlm_status_string", "aqlm_check_device_status",
            "aqlm_last_cuda_error", "aqlm_abi_version", "aqlm_matmul_group",
-           "aqlm_group_workspace_size")
+           "aqlm_group_workspace_size", "aqlm_matmul_group_static")
 
-ABI_VERSION = 2
+ABI_VERSION = 3
+
+# Size of the library's static scratch buffer behind aqlm_matmul_group_static.
+STATIC_GROUP_SCRATCH_BYTES = 8 << 20
 
 
 class Status(enum.IntEnum):
@@ -95,6 +98,8 @@ def lib() -> ctypes.CDLL:
                 L.aqlm_matmul_group.restype = _i
                 L.aqlm_group_workspace_size.argtypes = [ctypes.POINTER(AqlmProblem), _i]
                 L.aqlm_group_workspace_size.restype = ctypes.c_size_t
+                L.aqlm_matmul_group_static.argtypes = [ctypes.POINTER(AqlmProblem), _i, _vp]
+                L.aqlm_matmul_group_static.restype = _i
                 if L.aqlm_abi_version() != ABI_VERSION:
                     raise ImportError(f"libaqlm.so ABI {L.aqlm_abi_version()} != binding ABI {ABI_VERSION}")
                 _lib = L
@@ -162,3 +167,11 @@ def aqlm_group_workspace_size(problems, count=None) -> int:
     arr = problems if isinstance(problems, ctypes.Array) else problem_array(problems)
     n = len(problems) if count is None else count
     return lib().aqlm_group_workspace_size(arr, n)
+
+
+def aqlm_matmul_group_static(problems, stream=None, count=None):
+    """Group call on the library's static scratch buffer (allocates nothing; calls
+    that overlap in time race on that buffer)."""
+    arr = problems if isinstance(problems, ctypes.Array) else problem_array(problems)
+    n = len(problems) if count is None else count
+    _check(lib().aqlm_matmul_group_static(arr, n, stream), "aqlm_matmul_group_static")
