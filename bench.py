@@ -7,14 +7,18 @@
 A step is one pass of the AQLM linear layers of a workload over one batch of
 synthetic activations.  The default workload is the Llama-2-7B decoder layer
 set (q, k, v, o 4096x4096; gate, up 11008x4096; down 4096x11008), 2x8 g8
-codebooks (2 bits per weight), batch 1.
+codebooks (2 bits per weight), batch 1.  By default (--launch group) a step is
+one aqlm_matmul_group call over the set (the grouped lookup-table kernel and its
+reduction, two launches); --launch per-layer makes it one aqlm_matmul call per
+layer.  The group run also times the per-layer launches and reports them beside
+the headline.
 
 Metric: effective HBM GB/s = algorithmic bytes (codes + codebooks + scales + x +
 y, each once) / device time, summed over ranks; microseconds per layer are
 reported beside it.  Inputs are resident in HBM; every step reads a different
 copy of the layer set from a rotating pool larger than 3x the L2 cache, so no
-step finds its weights in L2.  Each step is one CUDA graph replay (its seven
-kernel launches); the timed region is bracketed by a barrier and a device
+step finds its weights in L2.  Each step is one CUDA graph replay of its
+launches; the timed region is bracketed by a barrier and a device
 synchronise and measured with CUDA events on the launching stream; the max over
 ranks is taken.  With N > 1 GPUs each rank runs its own replica (weak scaling,
 no data-path collective).
@@ -61,6 +65,10 @@ def parse_args(argv=None):
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     p.add_argument("--layer", default=None, help="time only this layer of the workload (e.g. q_proj)")
+    p.add_argument("--no-other-launch", action="store_true",
+                   help="skip the extra per-layer timing that the group mode reports beside its headline")
+    p.add_argument("--launch", choices=("group", "per-layer"), default="group",
+                   help="one aqlm_matmul_group call per step (default) or one aqlm_matmul call per layer")
     p.add_argument("--pool", type=int, default=None,
                    help="rotating-pool copies (default: enough to exceed 3x L2); smaller for profiler captures")
     a = p.parse_args(argv)
@@ -87,7 +95,8 @@ def measured_peaks():
 
 
 KERNEL_SOURCES = {"gemv_gather_kernel": "gemv.cu", "gemv_lut_2x8_kernel": "gemv_lut.cu",
-                  "tc_decode_mma_kernel": "tc_gemm.cu"}
+                  "tc_decode_mma_kernel": "tc_gemm.cu", "tc_pipe_kernel": "tc_pipe.cu",
+                  "lut_group_kernel": "lut_group.cu"}
 
 
 def measured_traffic(workload_name, kernel):
@@ -336,7 +345,7 @@ def run_ours(a):
 
     stream = torch.cuda.Stream(dev)
     h = stream.cuda_stream
-    # raw argument tuples: the step is seven C-ABI calls
+    # per-layer mode: raw argument tuples, one C-ABI call per layer
     calls = []
     for c in range(pool):
         cc = []
@@ -346,65 +355,101 @@ def run_ours(a):
                        wt.scales.data_ptr(), None, ys[li].data_ptr(), wt.M, wt.B, wt.g, lay.K, lay.N,
                        batch, h))
         calls.append(cc)
+    # group mode: one aqlm_matmul_group call per step (problem table + workspace per copy)
+    groups = [L.LayerGroup([(weights[c][li], xs[c][li], ys[li]) for li in range(len(w.layers))])
+              for c in range(pool)]
 
-    def step(c):
+    def step_per_layer(c):
         for args in calls[c]:
             st = lib.aqlm_matmul(*args)
             if st != 0:
                 raise native.AqlmError(st, "aqlm_matmul")
 
-    with torch.cuda.stream(stream):
-        for c in range(pool):
-            step(c)
-    torch.cuda.synchronize(dev)
-    graphs = []
-    for c in range(pool):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            step(c)
-        graphs.append(g)
-    torch.cuda.synchronize(dev)
+    def step_group(c):
+        groups[c].run(stream=stream)
+
+    def launches(mode):
+        """Kernel launches of one step: the grouped layers take two (partial sums and
+        reduction) per run of up to 16; every other layer one."""
+        if mode == "per-layer":
+            return len(w.layers)
+        grouped = sum(1 for l in w.layers if l.scheme.M == 2 and l.scheme.B == 8 and l.scheme.g == 8
+                      and batch == 1 and l.K % 64 == 0)
+        return 2 * ((grouped + 15) // 16) + (len(w.layers) - grouped)
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
-    with torch.cuda.stream(stream):
-        for i in range(a.warmup):
-            graphs[i % pool].replay()
-    torch.cuda.synchronize(dev)
-    barrier()
-
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local, enabled=not a.no_clocks) as clocks:
-        torch.cuda.synchronize(dev)
-        barrier()
+    def timed(step, steps, warmup, sample_clocks):
         with torch.cuda.stream(stream):
-            start.record(stream)
-            for i in range(a.steps):
+            for c in range(pool):
+                step(c)
+        torch.cuda.synchronize(dev)
+        graphs = []
+        for c in range(pool):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(c)
+            graphs.append(g)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            for i in range(warmup):
                 graphs[i % pool].replay()
-            end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-    ms = max_over_ranks(start.elapsed_time(end), dist, dev)
-    st, detail = L.check_device_status(stream=stream)
-    if st != native.Status.OK:
-        raise RuntimeError(f"device status {st.name} {detail:#x}")
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local, enabled=sample_clocks) as clocks:
+            torch.cuda.synchronize(dev)
+            barrier()
+            with torch.cuda.stream(stream):
+                start.record(stream)
+                for i in range(steps):
+                    graphs[i % pool].replay()
+                end.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier()
+        ms = max_over_ranks(start.elapsed_time(end), dist, dev)
+        st, detail = L.check_device_status(stream=stream)
+        if st != native.Status.OK:
+            raise RuntimeError(f"device status {st.name} {detail:#x}")
+        del graphs
+        return ms, clocks.summary()
 
-    launches_per_step = len(w.layers)
+    mode = a.launch
+    ms, clock_summary = timed(step_group if mode == "group" else step_per_layer, a.steps, a.warmup,
+                              not a.no_clocks)
+    launches_per_step = launches(mode)
     value = job_throughput_gbs(sbytes, a.steps, world, ms)
     ms_step = ms / a.steps
+    other = None
+    if mode == "group" and not a.no_other_launch:
+        # the same workload with one aqlm_matmul launch per layer, for comparison
+        o_steps = min(a.steps, 20000)
+        o_ms, _ = timed(step_per_layer, o_steps, max(3, min(a.warmup, 200)), False)
+        other = {"launch": "per-layer", "value": job_throughput_gbs(sbytes, o_steps, world, o_ms),
+                 "unit": "GB/s", "us_per_layer": o_ms * 1e3 / (o_steps * len(w.layers)), "steps": o_steps}
+
     peaks = measured_peaks()
-    avg_launch_s = (ms / 1e3) / (a.steps * launches_per_step)
-    bytes_per_launch = sbytes / launches_per_step
-    achieved = bytes_per_launch / avg_launch_s / 1e9
     kernel_names = {int(Path.GEMV): "gemv_gather_kernel", int(Path.GEMV_LUT): "gemv_lut_2x8_kernel",
-                    int(Path.TENSOR_CORE): "tc_decode_mma_kernel"}
-    kernel = kernel_names.get(paths[0], "?")
+                    int(Path.TENSOR_CORE): "tc_pipe_kernel"}
+    if mode == "group" and launches_per_step == 2 * ((len(w.layers) + 15) // 16):
+        # every layer grouped: the timed launches are the partial-sum kernel and its
+        # reduction, measured together (one step = one group call); the rate below is
+        # therefore a lower bound on the partial-sum kernel's own
+        kernel = "lut_group_kernel"
+        timed_as = "step: lut_group_kernel + lut_group_reduce_kernel"
+        achieved = sbytes / (ms_step / 1e3) / 1e9
+    else:
+        kernel = kernel_names.get(paths[0], "?")
+        timed_as = "average launch of the step"
+        avg_launch_s = (ms / 1e3) / (a.steps * launches_per_step)
+        achieved = sbytes / launches_per_step / avg_launch_s / 1e9
+    traffic = measured_traffic(w.name, kernel)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(w.name, kernel),
-                "kernel": kernel,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": kernel, "timed": timed_as,
+                "algorithmic_bytes": sbytes if kernel == "lut_group_kernel" else sbytes / launches_per_step,
                 "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
                 if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
 
@@ -412,16 +457,34 @@ def run_ours(a):
     e2e = None
     if not a.no_e2e:
         e2e_steps = min(a.steps, 2000)
-        hx = [torch.from_numpy(synth.make_x(batch, lay.K, seed=7, layer=li)).pin_memory()
-              for li, lay in enumerate(w.layers)]
-        hy = [torch.empty((batch, lay.N), dtype=torch.float16).pin_memory() for lay in w.layers]
-        dx = [torch.empty((batch, lay.K), dtype=torch.float16, device=dev) for lay in w.layers]
+        # every layer's x (and y) packed in one pinned host buffer and one device buffer:
+        # one H2D and one D2H copy per step (offsets stay 16-byte aligned: K, N % 8 == 0)
+        koff = np.cumsum([0] + [batch * lay.K for lay in w.layers])
+        noff = np.cumsum([0] + [batch * lay.N for lay in w.layers])
+        hx_flat = torch.empty((int(koff[-1]),), dtype=torch.float16).pin_memory()
+        for li, lay in enumerate(w.layers):
+            hx_flat[koff[li]:koff[li + 1]] = torch.from_numpy(
+                synth.make_x(batch, lay.K, seed=7, layer=li)).reshape(-1)
+        hy_flat = torch.empty((int(noff[-1]),), dtype=torch.float16).pin_memory()
+        dx_flat = torch.empty_like(hx_flat, device=dev)
+        dy_flat = torch.empty_like(hy_flat, device=dev)
+        dx = [dx_flat[koff[li]:koff[li + 1]].view(batch, lay.K) for li, lay in enumerate(w.layers)]
+        dy = [dy_flat[noff[li]:noff[li + 1]].view(batch, lay.N) for li, lay in enumerate(w.layers)]
+        e2e_groups = [L.LayerGroup([(weights[c][li], dx[li], dy[li]) for li in range(len(w.layers))])
+                      for c in range(pool)]
+
+        def e2e_step(c):
+            dx_flat.copy_(hx_flat, non_blocking=True)
+            if mode == "group":
+                e2e_groups[c].run(stream=stream)
+            else:
+                for li in range(len(w.layers)):
+                    L.matmul(dx[li], weights[c][li], out=dy[li], stream=stream)
+            hy_flat.copy_(dy_flat, non_blocking=True)
+
         with torch.cuda.stream(stream):
             for i in range(3):
-                for li in range(len(w.layers)):
-                    dx[li].copy_(hx[li], non_blocking=True)
-                    L.matmul(dx[li], weights[i % pool][li], out=ys[li], stream=stream)
-                    hy[li].copy_(ys[li], non_blocking=True)
+                e2e_step(i % pool)
         torch.cuda.synchronize(dev)
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
@@ -429,21 +492,18 @@ def run_ours(a):
         with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(e2e_steps):
-                c = i % pool
-                for li in range(len(w.layers)):
-                    dx[li].copy_(hx[li], non_blocking=True)
-                    L.matmul(dx[li], weights[c][li], out=ys[li], stream=stream)
-                    hy[li].copy_(ys[li], non_blocking=True)
+                e2e_step(i % pool)
             e1.record(stream)
         torch.cuda.synchronize(dev)
         ems = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        api = ("weight_only_additive_b200.layer.LayerGroup.run -> aqlm_matmul_group" if mode == "group"
+               else "weight_only_additive_b200.layer.matmul -> aqlm_matmul, per layer")
         e2e = {"value": job_throughput_gbs(sbytes, e2e_steps, world, ems), "unit": "GB/s",
-               "h2d_bytes_per_step": sum(t.numel() * 2 for t in hx),
-               "d2h_bytes_per_step": sum(t.numel() * 2 for t in hy),
+               "h2d_bytes_per_step": hx_flat.numel() * 2,
+               "d2h_bytes_per_step": hy_flat.numel() * 2,
                "steps": e2e_steps, "us_per_layer": ems * 1e3 / (e2e_steps * len(w.layers)),
-               "how": "per layer: pinned H2D copy of x, matmul via the public API "
-                      "(weight_only_additive_b200.layer.matmul -> aqlm_matmul), D2H copy of y; "
-                      "no CUDA graph"}
+               "how": f"per step: one pinned H2D copy of every layer's x (packed), {api}, one D2H copy "
+                      f"of every y (packed); no CUDA graph"}
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -454,14 +514,13 @@ def run_ours(a):
                          f"{s:.1f} s on the host cores"}
 
     if dist is not None:
-        del graphs
         dist.barrier()
         dist.destroy_process_group()
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
                 "warmup": a.warmup, "ms_per_step": ms_step,
-                "us_per_layer": ms_step * 1e3 / launches_per_step,
+                "us_per_layer": ms_step * 1e3 / len(w.layers),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
                 "data": "synthetic",
                 "config": {"workload": w.name, "layers": len(w.layers), "batch": batch,
@@ -469,11 +528,14 @@ def run_ours(a):
                            "algorithmic_bytes_per_step": sbytes,
                            "l2": f"inputs larger than L2: rotating pool of {pool} copies "
                                  f"({pool * copy_bytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
-                           "launch": "one CUDA graph replay per step",
+                           "launch": ("one aqlm_matmul_group call per step (grouped lookup-table kernel + "
+                                      "reduction), one CUDA graph replay per step" if mode == "group" else
+                                      "one aqlm_matmul call per layer, one CUDA graph replay per step"),
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "other_launch": other,
                 "gpu_launches": launches_per_step * a.steps,
-                "clocks": clocks.summary(), "gpu": props.name}
+                "clocks": clock_summary, "gpu": props.name}
         print(json.dumps(line), flush=True)
     return 0
 

@@ -315,7 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
         }
         // prefetch the operands of the range's next (layer, slice) into the other buffer,
         // whose MMAs completed before the previous table was stored
-        const long long run_end = std::min(it1, L.item0 + static_cast<long long>(s + 1) * L.T);
+        const long long slice_end = L.item0 + static_cast<long long>(s + 1) * L.T;
+        const long long run_end = slice_end < it1 ? slice_end : it1;
         if (ok && run_end < it1) {
           // the next (layer, slice) in item order
           const int nl = (s + 1 < L.S) ? l : l + 1;

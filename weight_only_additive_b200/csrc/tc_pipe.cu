@@ -98,6 +98,13 @@ __device__ __forceinline__ uint32_t swz128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Byte `off` (< 64) of row `row` of a code tile loaded with the 64-byte TMA swizzle:
+// the 16-byte chunk index is XORed with bits 7-8 of the byte offset (row / 2 mod 4),
+// so the 32 rows a warp reads at one chunk spread over all banks instead of two.
+__device__ __forceinline__ uint32_t code_tile_offset(int row, int off) {
+  return static_cast<uint32_t>(row * 64 + ((((off >> 4) ^ (row >> 1)) & 3) << 4) + (off & 15));
+}
+
 // Bounded wait that also gives up at once when another role has aborted.
 __device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
                                           uint32_t* status, uint32_t site) {
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
         break;
       }
       const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
-                          static_cast<uint32_t>(r) * kCodeRowBytes + static_cast<uint32_t>(within * kStageCodeBytes);
+                          code_tile_offset(r, within * kStageCodeBytes);
       decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
                                  p.codebooks, smem + L.cb);
       if constexpr (M == 1) {
@@ -511,8 +518,9 @@ cudaError_t launch_pipe_plan(const Problem& pr, uint32_t* status, cudaStream_t s
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
     const cuuint32_t box[2] = {kCodeRowBytes, static_cast<cuuint32_t>(kRows)};
     const cuuint32_t estr[2] = {1, 1};
+    // 64-byte swizzle: the decoders read one chunk of 32 consecutive rows at a time
     if (encode(&code_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pr.codes), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorNotSupported;
   }
