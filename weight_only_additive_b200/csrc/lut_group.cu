@@ -278,27 +278,24 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
     for (int s8 = 0; s8 < 8; ++s8) wv[s8] = static_cast<uint32_t>((8 * q4 + ((r8 + s8) & 7)) << 2);
     uint32_t mma_phase = 0;
     bool ok = true;
-    int cur_l = -1, cur_s = -1, run = 0;
     if (it0 < it1) {
       const int l = layer_of(p, it0);
       load_operands(p.layer[l], static_cast<int>((it0 - p.layer[l].item0) / p.layer[l].T), sbase, 0, wtid);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 
+    // Items come in runs of equal (layer, slice): the table is rebuilt at the start of
+    // every run, then each warp visits only its own tiles of the run (item index
+    // k = wg mod kTileGroups), so no warp walks the items of other warps.
     ItemCursor c;
     c.seek(p, it0);
-    int slot = 0;        // ring slot of item k
-    uint32_t ph = 0;     // its phase
-    for (long long k = 0; it0 + k < it1; ++k, c.next(p)) {
-      const int l = c.l, s = c.s, t = c.t;
+    const int nitems = static_cast<int>(it1 - it0);  // < 2^31 items per CTA
+    int run = 0;
+    for (int kbase = 0; kbase < nitems;) {
+      const int l = c.l, s = c.s, t0 = c.t;
       const GroupLayerDev& L = p.layer[l];
-      const int my_slot = slot;
-      const uint32_t my_ph = ph;
-      if (++slot == kSlots) {
-        slot = 0;
-        ph ^= 1u;
-      }
-      if (l != cur_l || s != cur_s) {
+      const int run_len = (nitems - kbase < L.T - t0) ? nitems - kbase : L.T - t0;
+      {
         // ---- new (layer, slice): table from the prefetched operands in buffer run & 1 ----
         const int buf = run & 1;
         asm volatile("cp.async.wait_all;" ::: "memory");
@@ -315,10 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
         }
         // prefetch the operands of the range's next (layer, slice) into the other buffer,
         // whose MMAs completed before the previous table was stored
-        const long long slice_end = L.item0 + static_cast<long long>(s + 1) * L.T;
-        const long long run_end = slice_end < it1 ? slice_end : it1;
-        if (ok && run_end < it1) {
-          // the next (layer, slice) in item order
+        if (ok && kbase + run_len < nitems) {
           const int nl = (s + 1 < L.S) ? l : l + 1;
           load_operands(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
         }
@@ -343,60 +337,69 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
         }
         tc_fence_before_sync();
         ok = workers_sync_and(ok);  // table complete
-        cur_l = l;
-        cur_s = s;
         ++run;
       }
-      if ((k & (kTileGroups - 1)) != wg) continue;
-      // ---- lookups of this item's tile: rows 8 task + r8 and 32 + 8 task + r8 ----
-      const bool landed =
-          __all_sync(0xffffffffu, ok && group_wait(&full[my_slot], my_ph, abort_flag, p.status, kSiteGroupRing));
-      if (landed) {
-        const uint32_t* rowA = reinterpret_cast<const uint32_t*>(
-            smem + kOffRing + static_cast<uint32_t>(my_slot) * kTileBytes + static_cast<uint32_t>(task * 8 + r8) * 128u);
-        const uint32_t* rowB = rowA + 32 * 32;  // 32 rows further
-        uint32_t cwA[8], cwB[8];
+      for (int i = (wg - kbase) & (kTileGroups - 1); i < run_len; i += kTileGroups) {
+        const int k = kbase + i;
+        const int my_slot = k % kSlots;
+        const uint32_t my_ph = static_cast<uint32_t>((k / kSlots) & 1);
+        const int t = t0 + i;
+        // ---- lookups of this item's tile: rows 8 task + r8 and 32 + 8 task + r8 ----
+        const bool landed =
+            __all_sync(0xffffffffu, ok && group_wait(&full[my_slot], my_ph, abort_flag, p.status, kSiteGroupRing));
+        if (landed) {
+          const uint32_t* rowA = reinterpret_cast<const uint32_t*>(
+              smem + kOffRing + static_cast<uint32_t>(my_slot) * kTileBytes + static_cast<uint32_t>(task * 8 + r8) * 128u);
+          const uint32_t* rowB = rowA + 32 * 32;  // 32 rows further
+          uint32_t cwA[8], cwB[8];
 #pragma unroll
-        for (int s8 = 0; s8 < 8; ++s8) {
-          cwA[s8] = rowA[wv[s8] >> 2];
-          cwB[s8] = rowB[wv[s8] >> 2];
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[my_slot]);  // the tile's codes are in registers
-        __half2 haccA = __float2half2_rn(0.f), haccB = haccA;
-        const uint8_t* lut = smem + kOffLut;
+          for (int s8 = 0; s8 < 8; ++s8) {
+            cwA[s8] = rowA[wv[s8] >> 2];
+            cwB[s8] = rowB[wv[s8] >> 2];
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[my_slot]);  // the tile's codes are in registers
+          __half2 haccA = __float2half2_rn(0.f), haccB = haccA;
+          const uint8_t* lut = smem + kOffLut;
 #pragma unroll
-        for (int s8 = 0; s8 < 8; ++s8) {
-          // table byte offsets: entry * 256 + column * 4 (column w, or 32 + w at +128);
-          // (codebook-0 half of one word, codebook-1 half of the other) per group
-          const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5504));
-          const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5514));
-          const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5524) + 128u);
-          const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5534) + 128u);
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5504));
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5514));
-          const uint32_t b2 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5524) + 128u);
-          const uint32_t b3 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5534) + 128u);
-          const uint32_t pa01 = __byte_perm(a0, a1, 0x7610), pa23 = __byte_perm(a2, a3, 0x7610);
-          const uint32_t pb01 = __byte_perm(b0, b1, 0x7610), pb23 = __byte_perm(b2, b3, 0x7610);
-          haccA = __hadd2(haccA, __hadd2(*reinterpret_cast<const __half2*>(&pa01), *reinterpret_cast<const __half2*>(&pa23)));
-          haccB = __hadd2(haccB, __hadd2(*reinterpret_cast<const __half2*>(&pb01), *reinterpret_cast<const __half2*>(&pb23)));
+          for (int s8 = 0; s8 < 8; ++s8) {
+            // table byte offsets: entry * 256 + column * 4 (column w, or 32 + w at +128);
+            // (codebook-0 half of one word, codebook-1 half of the other) per group
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5504));
+            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5514));
+            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5524) + 128u);
+            const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5534) + 128u);
+            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5504));
+            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5514));
+            const uint32_t b2 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5524) + 128u);
+            const uint32_t b3 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5534) + 128u);
+            const uint32_t pa01 = __byte_perm(a0, a1, 0x7610), pa23 = __byte_perm(a2, a3, 0x7610);
+            const uint32_t pb01 = __byte_perm(b0, b1, 0x7610), pb23 = __byte_perm(b2, b3, 0x7610);
+            haccA = __hadd2(haccA, __hadd2(*reinterpret_cast<const __half2*>(&pa01), *reinterpret_cast<const __half2*>(&pa23)));
+            haccB = __hadd2(haccB, __hadd2(*reinterpret_cast<const __half2*>(&pb01), *reinterpret_cast<const __half2*>(&pb23)));
+          }
+          const float2 fa = __half22float2(haccA), fb = __half22float2(haccB);
+          float va = fa.x + fa.y, vb = fb.x + fb.y;
+          va += __shfl_xor_sync(0xffffffffu, va, 1);
+          vb += __shfl_xor_sync(0xffffffffu, vb, 1);
+          va += __shfl_xor_sync(0xffffffffu, va, 2);
+          vb += __shfl_xor_sync(0xffffffffu, vb, 2);
+          if (q4 == 0) {
+            const int row = t * kTileRows + task * 8 + r8;
+            float* dst = L.part + static_cast<size_t>(s) * L.N;
+            if (row < L.N) dst[row] = va;
+            if (row + 32 < L.N) dst[row + 32] = vb;
+          }
+        } else {
+          ok = false;
+          if (lane == 0) mbar_arrive(&empty[my_slot]);
         }
-        const float2 fa = __half22float2(haccA), fb = __half22float2(haccB);
-        float va = fa.x + fa.y, vb = fb.x + fb.y;
-        va += __shfl_xor_sync(0xffffffffu, va, 1);
-        vb += __shfl_xor_sync(0xffffffffu, vb, 1);
-        va += __shfl_xor_sync(0xffffffffu, va, 2);
-        vb += __shfl_xor_sync(0xffffffffu, vb, 2);
-        if (q4 == 0) {
-          const int row = t * kTileRows + task * 8 + r8;
-          float* dst = L.part + static_cast<size_t>(s) * L.N;
-          if (row < L.N) dst[row] = va;
-          if (row + 32 < L.N) dst[row + 32] = vb;
-        }
-      } else {
-        ok = false;
-        if (lane == 0) mbar_arrive(&empty[my_slot]);
+      }
+      kbase += run_len;
+      c.t = 0;  // the next run starts the next slice (or the next layer's first)
+      if (++c.s == L.S) {
+        c.s = 0;
+        ++c.l;
       }
     }
   }
