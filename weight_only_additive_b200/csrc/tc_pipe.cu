@@ -129,7 +129,9 @@ __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase,
                                                   bool row_valid, const uint8_t* cw,
                                                   const __half* __restrict__ codebooks, const uint8_t* smem_cb) {
   if constexpr (M == 1) {
-    // 1x16: each 16-byte piece of the row is (part of) one codeword: gather it.
+    // 1x16: each 16-byte piece of the row is (part of) one codeword: gather it.  Codes
+    // are read one by one (measured faster here than one wide load: each gather can
+    // issue as soon as its own code has arrived).
     const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
@@ -143,14 +145,19 @@ __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase,
     }
   } else {
     // 2x8: codes (c0, c1) per group; codebooks staged in shared memory as [2][256][8].
-    // The two codewords are added as half2 (one rounding of their exact sum).
+    // The two codewords are added as half2 (one rounding of their exact sum).  The
+    // thread's 8 code bytes of this stage come in one load.
+    const uint2 q = *reinterpret_cast<const uint2*>(cw + 8 * hf);
+    const uint32_t cwords[2] = {q.x, q.y};
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       const int j = 4 * hf + cc;
       uint4 out = make_uint4(0u, 0u, 0u, 0u);
       if (row_valid) {
-        const uint4 q0 = *reinterpret_cast<const uint4*>(smem_cb + (static_cast<uint32_t>(cw[2 * j]) << 4));
-        const uint4 q1 = *reinterpret_cast<const uint4*>(smem_cb + 4096u + (static_cast<uint32_t>(cw[2 * j + 1]) << 4));
+        const uint32_t c0 = (cwords[cc >> 1] >> (16 * (cc & 1))) & 0xFFu;
+        const uint32_t c1 = (cwords[cc >> 1] >> (16 * (cc & 1) + 8)) & 0xFFu;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(smem_cb + (c0 << 4));
+        const uint4 q1 = *reinterpret_cast<const uint4*>(smem_cb + 4096u + (c1 << 4));
         out.x = hadd2_u32(q0.x, q1.x);
         out.y = hadd2_u32(q0.y, q1.y);
         out.z = hadd2_u32(q0.z, q1.z);
