@@ -108,7 +108,7 @@ def measured_traffic(workload_name, kernel):
     if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
         return None
     with open(path) as fh:
-        rec = json.load(fh).get(workload_name)
+        rec = json.load(fh).get(f"{workload_name}/{kernel}")
     if not rec or rec.get("kernel") != kernel:
         return None
     src = os.path.join(ROOT, "weight_only_additive_b200", "csrc", KERNEL_SOURCES[kernel])
