@@ -189,6 +189,16 @@ const char* aqlm_status_string(aqlm_status status);
  * synchronisation failed, AQLM_OK otherwise. */
 aqlm_status aqlm_check_device_status(aqlm_stream_t stream, uint32_t* detail);
 
+/* Exercises the device-side failure path without faulting the GPU: launches a
+ * one-thread kernel that waits, through the same bounded wait the matmul kernels
+ * use, on an mbarrier nothing arrives on.  The wait gives up after timeout_us
+ * microseconds (1..1000000, else AQLM_ERR_INVALID_ARG) and records site code
+ * AQLM_SITE_SELFTEST in the status word; the kernel returns normally.  A following
+ * aqlm_check_device_status reports AQLM_ERR_TIMEOUT with that detail.  For tests;
+ * the pages have no counterpart. */
+#define AQLM_SITE_SELFTEST 0x501u
+aqlm_status aqlm_selftest_bounded_wait(unsigned timeout_us, aqlm_stream_t stream);
+
 /* The cudaError_t value of the last CUDA failure this thread saw in the library
  * (0 if none). */
 int aqlm_last_cuda_error(void);

@@ -179,3 +179,8 @@ def test_group_static_validation_needs_no_gpu(lib):
         16 * _ws_bytes(14336, 4096) <= native.STATIC_GROUP_SCRATCH_BYTES
     bad = [_prob(1 << 32, M=3)]
     assert L_.aqlm_matmul_group_static(native.problem_array(bad), 1, None) == Status.UNSUPPORTED
+
+
+def test_selftest_rejects_bad_limits_without_a_gpu(lib):
+    assert native.lib().aqlm_selftest_bounded_wait(0, None) == Status.INVALID_ARG
+    assert native.lib().aqlm_selftest_bounded_wait(1000001, None) == Status.INVALID_ARG

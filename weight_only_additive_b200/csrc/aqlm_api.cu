@@ -110,7 +110,7 @@ EncodeTiledFn encode_tiled() {
 
 extern "C" {
 
-int aqlm_abi_version(void) { return 3; }
+int aqlm_abi_version(void) { return 4; }
 
 const char* aqlm_status_string(aqlm_status status) {
   switch (status) {
@@ -318,6 +318,14 @@ aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aq
     if (!scratch) return from_cuda(cudaErrorInvalidDevice);
   }
   return aqlm_matmul_group(problems, count, scratch, AQLM_STATIC_GROUP_SCRATCH_BYTES, stream);
+}
+
+aqlm_status aqlm_selftest_bounded_wait(unsigned timeout_us, aqlm_stream_t stream) {
+  if (timeout_us == 0 || timeout_us > 1000000u) return AQLM_ERR_INVALID_ARG;
+  uint32_t* status = device_status_ptr();
+  if (!status) return from_cuda(cudaErrorInvalidDevice);
+  return from_cuda(aqlm::launch_selftest_wait(status, static_cast<uint64_t>(timeout_us) * 1000u,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void* scales,

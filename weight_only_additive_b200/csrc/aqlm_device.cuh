@@ -113,11 +113,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for phase `parity` of `bar` to complete, giving up after
 // kWaitTimeoutNs of wall time.  Returns false (and records `site`) on timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  uint32_t* status, uint32_t site) {
+                                                  uint32_t* status, uint32_t site,
+                                                  uint64_t timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > timeout_ns) {
       record_failure(status, site);
       return false;
     }

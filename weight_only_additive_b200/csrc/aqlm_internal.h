@@ -24,7 +24,12 @@ enum : uint32_t {
   kSitePipeAcc = 0x304,     // pipelined tensor-core kernel: waiting for the accumulator
   kSiteGroupRing = 0x401,   // grouped lookup-table kernel: code-tile ring (landing / slot release)
   kSiteGroupMma = 0x402,    // grouped lookup-table kernel: waiting for the table-building MMA
+  kSiteSelftest = 0x501,    // aqlm_selftest_bounded_wait: the wait that nothing completes
 };
+
+// Self-test of the bounded-wait path: one thread waits on an mbarrier that nothing
+// arrives on, gives up after timeout_ns and records kSiteSelftest.
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t stream);
 
 struct Problem {
   const void* x;

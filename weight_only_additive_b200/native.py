@@ -18,9 +18,12 @@ LIBRARY = os.path.join(PKG, "libaqlm.so")
 EXPORTS = ("aqlm_matmul", "aqlm_matmul_path", "aqlm_dequantize", "aqlm_select_path",
            "aqlm_validate", "aqlm_status_string", "aqlm_check_device_status",
            "aqlm_last_cuda_error", "aqlm_abi_version", "aqlm_matmul_group",
-           "aqlm_group_workspace_size", "aqlm_matmul_group_static")
+           "aqlm_group_workspace_size", "aqlm_matmul_group_static", "aqlm_selftest_bounded_wait")
 
-ABI_VERSION = 3
+ABI_VERSION = 4
+
+# Site code aqlm_selftest_bounded_wait records in the device status word.
+SITE_SELFTEST = 0x501
 
 # Size of the library's static scratch buffer behind aqlm_matmul_group_static.
 STATIC_GROUP_SCRATCH_BYTES = 8 << 20
@@ -100,6 +103,8 @@ def lib() -> ctypes.CDLL:
                 L.aqlm_group_workspace_size.restype = ctypes.c_size_t
                 L.aqlm_matmul_group_static.argtypes = [ctypes.POINTER(AqlmProblem), _i, _vp]
                 L.aqlm_matmul_group_static.restype = _i
+                L.aqlm_selftest_bounded_wait.argtypes = [ctypes.c_uint, _vp]
+                L.aqlm_selftest_bounded_wait.restype = _i
                 if L.aqlm_abi_version() != ABI_VERSION:
                     raise ImportError(f"libaqlm.so ABI {L.aqlm_abi_version()} != binding ABI {ABI_VERSION}")
                 _lib = L
@@ -175,3 +180,8 @@ def aqlm_matmul_group_static(problems, stream=None, count=None):
     arr = problems if isinstance(problems, ctypes.Array) else problem_array(problems)
     n = len(problems) if count is None else count
     _check(lib().aqlm_matmul_group_static(arr, n, stream), "aqlm_matmul_group_static")
+
+
+def aqlm_selftest_bounded_wait(timeout_us: int, stream=None):
+    """Launch the bounded-wait self-test kernel (see include/aqlm.h)."""
+    _check(lib().aqlm_selftest_bounded_wait(int(timeout_us), stream), "aqlm_selftest_bounded_wait")
