@@ -418,22 +418,50 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
   }
 }
 
-// y[n] = fp16(s_n * sum_s part[s][n] + bias_n), slices in ascending order.
-__global__ void __launch_bounds__(256) lut_group_reduce_kernel(const __grid_constant__ GroupParams p) {
+// y[n] = fp16(s_n * sum_s part[s][n] + bias_n).  A block takes 64 rows; thread
+// (row r, lane j) adds slices j, j + 4, j + 8, ... of row r (loads coalesced across
+// the 64 rows, and the thread's loads issued together, eight at a time), and the
+// four lane sums of a row are added in the order j = 0..3.  The order is fixed, so
+// the result does not depend on timing or on which CTA produced which partial.
+constexpr int kReduceRows = 64;
+constexpr int kReduceLanes = 4;
+__global__ void __launch_bounds__(kReduceRows* kReduceLanes) lut_group_reduce_kernel(
+    const __grid_constant__ GroupParams p) {
+  __shared__ float sums[kReduceLanes][kReduceRows];
   grid_dependents_launch();
-  const long long row = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-  if (row >= p.rows) return;
+  const int r = threadIdx.x % kReduceRows;
+  const int j = threadIdx.x / kReduceRows;
+  const long long row = static_cast<long long>(blockIdx.x) * kReduceRows + r;
+  const bool valid = row < p.rows;
   int l = 0;
   while (l + 1 < p.count && p.layer[l + 1].row0 <= row) ++l;
   const GroupLayerDev& L = p.layer[l];
   const int n = static_cast<int>(row - L.row0);
-  const float sc = __half2float(L.scales[n]);
-  const float bi = L.bias ? __half2float(L.bias[n]) : 0.f;
   // the partials are the previous kernel's output
   grid_dependency_wait();
   float acc = 0.f;
-  for (int s = 0; s < L.S; ++s) acc += L.part[static_cast<size_t>(s) * L.N + n];
-  L.y[n] = __float2half_rn(acc * sc + bi);
+  if (valid) {
+    const float* col = L.part + n;
+    for (int s0 = j; s0 < L.S; s0 += 8 * kReduceLanes) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u * kReduceLanes;
+        v[u] = s < L.S ? col[static_cast<size_t>(s) * L.N] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc += v[u];
+    }
+  }
+  sums[j][r] = acc;
+  __syncthreads();
+  if (j == 0 && valid) {
+    float t = sums[0][r];
+#pragma unroll
+    for (int q = 1; q < kReduceLanes; ++q) t += sums[q][r];
+    const float bi = L.bias ? __half2float(L.bias[n]) : 0.f;
+    L.y[n] = __float2half_rn(t * __half2float(L.scales[n]) + bi);
+  }
 }
 
 }  // namespace
@@ -528,8 +556,8 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
   if (e != cudaSuccess) return e;
 
   cudaLaunchConfig_t rcfg = {};
-  rcfg.gridDim = dim3(static_cast<unsigned>((rows + 255) / 256), 1, 1);
-  rcfg.blockDim = dim3(256, 1, 1);
+  rcfg.gridDim = dim3(static_cast<unsigned>((rows + kReduceRows - 1) / kReduceRows), 1, 1);
+  rcfg.blockDim = dim3(kReduceRows * kReduceLanes, 1, 1);
   rcfg.stream = stream;
   rcfg.attrs = attr;
   rcfg.numAttrs = 1;
