@@ -22,9 +22,10 @@
 //               the prefetched operands (x slice, both codebooks), issue two
 //               tcgen05.mma (M = 128 rows of x groups, N = 256 entries, K = 16 with
 //               the upper 8 zero) into TMEM and move the table to shared memory as
-//               fp16 pairs (T_0, T_1) per (entry, group).  Then warps 4j..4j+3 take
-//               the tiles k = j (mod 4), two interleaved 8-row tasks per warp, and
-//               write each row's fp32 partial to the workspace.
+//               fp16 pairs (T_0, T_1) per (entry, group).  Then the warps of tile
+//               group j take the tiles k = j (mod kTileGroups), kTasks interleaved
+//               8-row tasks per warp, and write each row's fp32 partial to the
+//               workspace.
 // The partials of a row are summed over the slices in ascending order by a second
 // small kernel (programmatic dependent launch), which applies the channel scale
 // and bias: the result does not depend on which CTA ran which item.
@@ -50,14 +51,20 @@ constexpr uint32_t kTileBytes = 64u * 128u;        // 64 rows x 64 groups x 2 co
 constexpr uint32_t kLutBytes = 256u * 64u * 4u;    // 64 KB
 constexpr uint32_t kAOpBytes = 128u * 32u;         // 4 KB
 constexpr uint32_t kBOpBytes = 256u * 32u;         // 8 KB per codebook
-constexpr int kSlots = 14;                         // 112 KB of code tiles in flight
-constexpr int kTileGroups = 4;                     // warps 4j..4j+3 take tiles k = j (mod 4)
+constexpr int kSlots = 16;                         // 128 KB of code tiles in flight
+#ifndef AQLM_GROUP_TASKS
+#define AQLM_GROUP_TASKS 2
+#endif
+constexpr int kTasks = AQLM_GROUP_TASKS;           // 8-row tasks per warp and tile (interleaved)
+constexpr int kWarpsPerTile = 8 / kTasks;          // a 64-row tile is 8 tasks
+constexpr int kTileGroups = 16 / kWarpsPerTile;    // warps of group j take tiles k = j (mod kTileGroups)
+static_assert(kTasks * kWarpsPerTile == 8 && (kTileGroups & (kTileGroups - 1)) == 0, "tile split");
 constexpr uint32_t kTmemCols = 512;                // D_0 at [0, 256), D_1 at [256, 512)
 
 constexpr uint32_t kOffLut = 0;
 constexpr uint32_t kOffA = kOffLut + kLutBytes;                 // 2 buffers
-constexpr uint32_t kOffB = kOffA + 2 * kAOpBytes;               // 2 buffers x 2 codebooks
-constexpr uint32_t kOffRing = kOffB + 4 * kBOpBytes;            // 1024-aligned
+constexpr uint32_t kOffB = kOffA + 2 * kAOpBytes;               // 1 buffer x 2 codebooks
+constexpr uint32_t kOffRing = kOffB + 2 * kBOpBytes;            // 1024-aligned
 constexpr uint32_t kOffBars = kOffRing + kSlots * kTileBytes;
 constexpr uint32_t kSmemBytes = kOffBars + 8u * (2 * kSlots + 1) + 16u;
 static_assert(kOffRing % 1024 == 0, "ring slots must stay 1024-byte aligned");
@@ -172,29 +179,25 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
-// Operands of slice s of layer l into buffer `buf` (cp.async, caller commits):
-// A row rho holds x group 2 (rho mod 32) + (rho / 32 mod 2) of the slice (rows
-// 64-127 repeat rows 0-63), zero past the layer's last group; B holds the two
-// codebooks, one 16-byte codeword per row.  The zero upper K halves are written
-// once at start-up.
-__device__ __forceinline__ void load_operands(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
+// Table operands (cp.async, caller commits).  A (two buffers): row rho holds x
+// group 2 (rho mod 32) + (rho / 32 mod 2) of slice s (rows 64-127 repeat rows 0-63),
+// zero past the layer's last group.  B (one buffer, reloaded only when the layer
+// changes): the two codebooks, one 16-byte codeword per row.  The zero upper K
+// halves are written once at start-up.
+__device__ __forceinline__ void load_x_slice(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
   const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * kAOpBytes;
-  const uint32_t bo = kOffB + static_cast<uint32_t>(buf) * 2u * kBOpBytes;
-  for (int i = wtid; i < 128 + 512; i += kWorkers) {
-    if (i < 128) {
-      const int rho = i;
-      const int gg = s * 64 + 2 * (rho & 31) + ((rho >> 5) & 1);
-      const bool valid = gg < L.G;
-      cp_async_16_zfill(sbase + ao + kmajor_offset(rho, 0),
-                        valid ? static_cast<const void*>(L.x + static_cast<size_t>(gg) * 8)
-                              : static_cast<const void*>(L.x),
-                        valid ? 16u : 0u);
-    } else {
-      const int e = i - 128;  // codebook m = e / 256, entry e % 256
-      cp_async_16_zfill(sbase + bo + static_cast<uint32_t>(e >> 8) * kBOpBytes + kmajor_offset(e & 255, 0),
-                        L.codebooks + static_cast<size_t>(e) * 8, 16u);
-    }
+  for (int rho = wtid; rho < 128; rho += kWorkers) {
+    const int gg = s * 64 + 2 * (rho & 31) + ((rho >> 5) & 1);
+    const bool valid = gg < L.G;
+    cp_async_16_zfill(sbase + ao + kmajor_offset(rho, 0),
+                      valid ? static_cast<const void*>(L.x + static_cast<size_t>(gg) * 8) : static_cast<const void*>(L.x),
+                      valid ? 16u : 0u);
   }
+}
+__device__ __forceinline__ void load_codebooks(const GroupLayerDev& L, uint32_t sbase, int wtid) {
+  for (int e = wtid; e < 512; e += kWorkers)  // codebook m = e / 256, entry e % 256
+    cp_async_16_zfill(sbase + kOffB + static_cast<uint32_t>(e >> 8) * kBOpBytes + kmajor_offset(e & 255, 0),
+                      L.codebooks + static_cast<size_t>(e) * 8, 16u);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_constant__ GroupMaps maps,
@@ -221,18 +224,17 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
   if (tid == 0) {
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kWorkers / 32 / kTileGroups);
+      mbar_init(&empty[i], kWarpsPerTile);
     }
     mbar_init(mma_bar, 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // zero upper K halves of both operand buffers (never written again)
-  for (int i = tid; i < 2 * (128 + 512); i += kThreads) {
-    const int buf = i / 640, j = i % 640;
-    const uint32_t off = j < 128 ? kOffA + static_cast<uint32_t>(buf) * kAOpBytes + kmajor_offset(j, 1)
-                                 : kOffB + static_cast<uint32_t>(buf) * 2u * kBOpBytes +
-                                       static_cast<uint32_t>((j - 128) >> 8) * kBOpBytes + kmajor_offset((j - 128) & 255, 1);
+  // zero upper K halves of the operand buffers (never written again)
+  for (int i = tid; i < 2 * 128 + 512; i += kThreads) {
+    const uint32_t off = i < 256 ? kOffA + static_cast<uint32_t>(i >> 7) * kAOpBytes + kmajor_offset(i & 127, 1)
+                                 : kOffB + static_cast<uint32_t>((i - 256) >> 8) * kBOpBytes +
+                                       kmajor_offset((i - 256) & 255, 1);
     *reinterpret_cast<uint4*>(smem + off) = make_uint4(0u, 0u, 0u, 0u);
   }
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
@@ -267,8 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
     // kernel in the stream has completed.
     grid_dependency_wait();
     const int wtid = tid;
-    const int wg = warp >> 2;    // tiles k = wg (mod 4) are this warp's
-    const int task = warp & 3;   // its two 8-row tasks of such a tile: task and task + 4
+    const int wg = warp / kWarpsPerTile;    // tiles k = wg (mod kTileGroups) are this warp's
+    const int task = warp % kWarpsPerTile;  // its tasks of such a tile: task + kWarpsPerTile * u
     const int r8 = lane >> 2;    // row of the task
     const int q4 = lane & 3;     // quarter of the row's 32 code words
     const uint32_t idesc = umma_idesc_f16_f32(128, 256);
@@ -280,7 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
     bool ok = true;
     if (it0 < it1) {
       const int l = layer_of(p, it0);
-      load_operands(p.layer[l], static_cast<int>((it0 - p.layer[l].item0) / p.layer[l].T), sbase, 0, wtid);
+      load_codebooks(p.layer[l], sbase, wtid);
+      load_x_slice(p.layer[l], static_cast<int>((it0 - p.layer[l].item0) / p.layer[l].T), sbase, 0, wtid);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 
@@ -305,20 +308,21 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
         tc_fence_after_sync();
         if (ok && wtid == 0) {
           const uint64_t adesc = kmajor_desc(sbase + kOffA + static_cast<uint32_t>(buf) * kAOpBytes);
-          const uint32_t bo = sbase + kOffB + static_cast<uint32_t>(buf) * 2u * kBOpBytes;
+          const uint32_t bo = sbase + kOffB;
           umma_f16_ss(tmem, adesc, kmajor_desc(bo), idesc, 0u);
           umma_f16_ss(tmem + 256u, adesc, kmajor_desc(bo + kBOpBytes), idesc, 0u);
           umma_commit(mma_bar);
         }
-        // prefetch the operands of the range's next (layer, slice) into the other buffer,
-        // whose MMAs completed before the previous table was stored
-        if (ok && kbase + run_len < nitems) {
-          const int nl = (s + 1 < L.S) ? l : l + 1;
-          load_operands(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
+        // prefetch the x slice of the range's next (layer, slice) into the other A
+        // buffer, whose MMAs completed before the previous table was stored
+        const bool more = kbase + run_len < nitems;
+        const int nl = (s + 1 < L.S) ? l : l + 1;
+        if (ok && more) load_x_slice(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
         const bool done = ok && group_wait(mma_bar, mma_phase, abort_flag, p.status, kSiteGroupMma);
         mma_phase ^= 1u;
+        // the MMAs have read B: a new layer's codebooks may replace it now
+        if (done && more && nl != l) load_codebooks(p.layer[nl], sbase, wtid);
+        asm volatile("cp.async.commit_group;" ::: "memory");
         ok = workers_sync_and(done);
         tc_fence_after_sync();
         if (ok) {
@@ -344,51 +348,57 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
         const int my_slot = k % kSlots;
         const uint32_t my_ph = static_cast<uint32_t>((k / kSlots) & 1);
         const int t = t0 + i;
-        // ---- lookups of this item's tile: rows 8 task + r8 and 32 + 8 task + r8 ----
+        // ---- lookups of this item's tile: rows 8 (task + kWarpsPerTile u) + r8 ----
         const bool landed =
             __all_sync(0xffffffffu, ok && group_wait(&full[my_slot], my_ph, abort_flag, p.status, kSiteGroupRing));
         if (landed) {
-          const uint32_t* rowA = reinterpret_cast<const uint32_t*>(
+          const uint32_t* row0 = reinterpret_cast<const uint32_t*>(
               smem + kOffRing + static_cast<uint32_t>(my_slot) * kTileBytes + static_cast<uint32_t>(task * 8 + r8) * 128u);
-          const uint32_t* rowB = rowA + 32 * 32;  // 32 rows further
-          uint32_t cwA[8], cwB[8];
+          uint32_t cw[kTasks][8];
 #pragma unroll
-          for (int s8 = 0; s8 < 8; ++s8) {
-            cwA[s8] = rowA[wv[s8] >> 2];
-            cwB[s8] = rowB[wv[s8] >> 2];
-          }
+          for (int u = 0; u < kTasks; ++u)
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) cw[u][s8] = row0[u * kWarpsPerTile * 8 * 32 + (wv[s8] >> 2)];
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[my_slot]);  // the tile's codes are in registers
-          __half2 haccA = __float2half2_rn(0.f), haccB = haccA;
+          __half2 hacc[kTasks];
+#pragma unroll
+          for (int u = 0; u < kTasks; ++u) hacc[u] = __float2half2_rn(0.f);
           const uint8_t* lut = smem + kOffLut;
 #pragma unroll
           for (int s8 = 0; s8 < 8; ++s8) {
-            // table byte offsets: entry * 256 + column * 4 (column w, or 32 + w at +128);
-            // (codebook-0 half of one word, codebook-1 half of the other) per group
-            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5504));
-            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5514));
-            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5524) + 128u);
-            const uint32_t a3 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwA[s8], wv[s8], 0x5534) + 128u);
-            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5504));
-            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5514));
-            const uint32_t b2 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5524) + 128u);
-            const uint32_t b3 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cwB[s8], wv[s8], 0x5534) + 128u);
-            const uint32_t pa01 = __byte_perm(a0, a1, 0x7610), pa23 = __byte_perm(a2, a3, 0x7610);
-            const uint32_t pb01 = __byte_perm(b0, b1, 0x7610), pb23 = __byte_perm(b2, b3, 0x7610);
-            haccA = __hadd2(haccA, __hadd2(*reinterpret_cast<const __half2*>(&pa01), *reinterpret_cast<const __half2*>(&pa23)));
-            haccB = __hadd2(haccB, __hadd2(*reinterpret_cast<const __half2*>(&pb01), *reinterpret_cast<const __half2*>(&pb23)));
+#pragma unroll
+            for (int u = 0; u < kTasks; ++u) {
+              // table byte offsets: entry * 256 + column * 4 (column w, or 32 + w at +128);
+              // (codebook-0 half of one word, codebook-1 half of the other) per group
+              const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cw[u][s8], wv[s8], 0x5504));
+              const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cw[u][s8], wv[s8], 0x5514));
+              const uint32_t a2 =
+                  *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cw[u][s8], wv[s8], 0x5524) + 128u);
+              const uint32_t a3 =
+                  *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cw[u][s8], wv[s8], 0x5534) + 128u);
+              const uint32_t p01 = __byte_perm(a0, a1, 0x7610), p23 = __byte_perm(a2, a3, 0x7610);
+              hacc[u] = __hadd2(hacc[u],
+                                __hadd2(*reinterpret_cast<const __half2*>(&p01), *reinterpret_cast<const __half2*>(&p23)));
+            }
           }
-          const float2 fa = __half22float2(haccA), fb = __half22float2(haccB);
-          float va = fa.x + fa.y, vb = fb.x + fb.y;
-          va += __shfl_xor_sync(0xffffffffu, va, 1);
-          vb += __shfl_xor_sync(0xffffffffu, vb, 1);
-          va += __shfl_xor_sync(0xffffffffu, va, 2);
-          vb += __shfl_xor_sync(0xffffffffu, vb, 2);
+          float v[kTasks];
+#pragma unroll
+          for (int u = 0; u < kTasks; ++u) {
+            const float2 f = __half22float2(hacc[u]);
+            v[u] = f.x + f.y;
+          }
+#pragma unroll
+          for (int u = 0; u < kTasks; ++u) v[u] += __shfl_xor_sync(0xffffffffu, v[u], 1);
+#pragma unroll
+          for (int u = 0; u < kTasks; ++u) v[u] += __shfl_xor_sync(0xffffffffu, v[u], 2);
           if (q4 == 0) {
-            const int row = t * kTileRows + task * 8 + r8;
             float* dst = L.part + static_cast<size_t>(s) * L.N;
-            if (row < L.N) dst[row] = va;
-            if (row + 32 < L.N) dst[row + 32] = vb;
+#pragma unroll
+            for (int u = 0; u < kTasks; ++u) {
+              const int row = t * kTileRows + (task + kWarpsPerTile * u) * 8 + r8;
+              if (row < L.N) dst[row] = v[u];
+            }
           }
         } else {
           ok = false;
