@@ -64,6 +64,7 @@ struct PipeParams {
   int ks_per;      // K stages per split (the last split may have fewer)
   int red_rows;    // split-K reduction: weight rows each CTA of the cluster owns
   uint32_t tmem_cols;
+  int cb32;        // codebooks 32-byte aligned: g = 16 codewords in one 256-bit load
   uint32_t* status;
 };
 
@@ -119,6 +120,27 @@ __device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, volati
     }
   }
   return true;
+}
+
+// 1x16 g16 with register staging: the thread's 4 16-byte pieces of one stage
+// (chunks 4 hf .. 4 hf + 3 = its two 32-byte codewords), gathered from the
+// L2-resident codebook into registers: one 256-bit load per codeword when the
+// codebook is 32-byte aligned, else two 128-bit loads.
+__device__ __forceinline__ void gather_stage_g16(uint4 (&v)[4], const uint8_t* cw, int hf, bool row_valid,
+                                                 const __half* __restrict__ codebooks, bool cb32) {
+  const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
+  if (!row_valid) {
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) v[cc] = make_uint4(0u, 0u, 0u, 0u);
+  } else if (cb32) {
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc)
+      ldg_nc_v8(codebooks + static_cast<size_t>(c16[2 * hf + cc]) * 16, v[2 * cc], v[2 * cc + 1]);
+  } else {
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc)
+      v[cc] = ldg_nc_v4(codebooks + static_cast<size_t>(c16[2 * hf + (cc >> 1)]) * 16 + 8 * (cc & 1));
+  }
 }
 
 // Decode half (`hf` = 0: chunks 0-3, 1: chunks 4-7) of one 64-wide K stage of
@@ -285,6 +307,55 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     const int r = tid & (kRows - 1);
     const int hf = tid >> 7;
     const bool row_valid = n0 + r < p.N;
+    if constexpr (M == 1 && G == 16) {
+      // 1x16 g16: register-staged gathers, kLook stages ahead.  At step i the thread
+      // issues the gathers of stage i (one 256-bit load per 32-byte codeword: one L1TEX
+      // request instead of two cp.async) and stores stage i - kLook, gathered kLook
+      // steps earlier, into its A slot.  Measured faster than cp.async for g = 16 and
+      // slower for g = 8 (16-byte codewords), which keeps the cp.async path below.
+      constexpr int kLook = 3;
+      uint4 st[kLook + 1][4];
+      bool alive = true;
+      for (int base = 0; alive && base < nks + kLook; base += kLook + 1) {
+#pragma unroll
+        for (int u = 0; u <= kLook; ++u) {
+          const int i = base + u;      // stage gathered now
+          const int j = i - kLook;     // stage stored now
+          const bool issue = i < nks, store = j >= 0 && j < nks;
+          const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
+          const int sj = j >= 0 ? j % S : 0, uj = j >= 0 ? j / S : 0;
+          // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
+          bool ready = true;
+          if (issue && within == 0)
+            ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
+                              kSitePipeCodes);
+          if (ready && store && uj > 0)
+            ready = pipe_wait(&empty[sj], static_cast<uint32_t>((uj - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
+          if (!__all_sync(0xffffffffu, ready)) {
+            *abort_flag = 1u;
+            alive = false;
+            break;
+          }
+          if (issue) {
+            const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
+                                code_tile_offset(r, within * kStageCodeBytes);
+            gather_stage_g16(st[u], cw, hf, row_valid, p.codebooks, p.cb32 != 0);
+            if (within == kStagesPerTile - 1 || i == nks - 1) {
+              __syncwarp();  // every lane has read its codes of this tile
+              if (lane == 0) mbar_arrive(&cempty[c]);
+            }
+          }
+          if (store) {
+            const uint32_t a_off = L.a + static_cast<uint32_t>(sj) * kABytes;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = st[(u + 1) % (kLook + 1)][cc];
+            fence_proxy_async_smem();
+            mbar_arrive(&full[sj]);
+          }
+        }
+      }
+    } else {
     for (int i = 0; i < nks; ++i) {
       const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
       // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
@@ -313,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
         __syncwarp();
         if (lane == 0) mbar_arrive(&cempty[c]);
       }
+    }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   }
@@ -547,6 +619,7 @@ cudaError_t launch_pipe_plan(const Problem& pr, uint32_t* status, cudaStream_t s
   p.ks_per = plan.ks_per;
   p.red_rows = plan.red_rows;
   p.tmem_cols = cols;
+  p.cb32 = (reinterpret_cast<uintptr_t>(pr.codebooks) & 31u) == 0 ? 1 : 0;
   p.status = status;
   const uint32_t smem = pipe_smem_bytes(plan.S, BN, kSmemCb);
   auto kern = tc_pipe_kernel<M, B, G>;
