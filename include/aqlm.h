@@ -25,8 +25,10 @@
  *   y          fp16   [batch, N]
  *   W_out      fp16   [N, K]         (aqlm_dequantize only)
  *
- * Supported schemes (M, B, g): (1, 16, 8) "1x16 g8", (2, 8, 8) "2x8 g8",
- * (1, 16, 16) "1x16 g16".  Other shapes return AQLM_ERR_UNSUPPORTED.
+ * Supported schemes (M, B, g): B = 8 (256-entry codebooks) with M = 1..4, and
+ * B = 16 (65536-entry codebooks) with M = 1..2, each with g = 8 or 16 -- among them
+ * the published (1, 16, 8) "1x16 g8", (2, 8, 8) "2x8 g8", (1, 16, 16) "1x16 g16" and
+ * the 4-bit (2, 16, 8) and (4, 8, 8).  Other shapes return AQLM_ERR_UNSUPPORTED.
  * K must be a multiple of g; N >= 1; 1 <= batch <= 65535.  Every pointer must be
  * 16-byte aligned (AQLM_ERR_MISALIGNED otherwise); bias may be NULL.
  *

@@ -46,7 +46,10 @@ def test_abi_version_and_status_strings(lib):
 A = 1 << 20  # a 16-byte aligned fake address: validation never dereferences it
 
 
-@pytest.mark.parametrize("M,B,g", [(1, 16, 8), (2, 8, 8), (1, 16, 16)])
+SUPPORTED = [(m, 8, g) for m in (1, 2, 3, 4) for g in (8, 16)] + [(m, 16, g) for m in (1, 2) for g in (8, 16)]
+
+
+@pytest.mark.parametrize("M,B,g", SUPPORTED)
 def test_supported_schemes_validate(lib, M, B, g):
     assert native.aqlm_validate(A, A, A, A, None, A, M, B, g, 4096, 4096, 1) == Status.OK
     assert native.aqlm_validate(A, A, A, A, A, A, M, B, g, 4096, 11008, 256) == Status.OK
@@ -60,9 +63,10 @@ def test_supported_schemes_validate(lib, M, B, g):
     ((A, A, A, A, None, A, 1, 16, 8, 64, 0, 1), Status.INVALID_ARG),       # N = 0
     ((A, A, A, A, None, A, 1, 16, 8, 64, 64, 0), Status.INVALID_ARG),      # batch = 0
     ((A, A, A, A, None, A, 1, 16, 8, 64, 64, 70000), Status.INVALID_ARG),  # batch too large
-    ((A, A, A, A, None, A, 3, 8, 8, 64, 64, 1), Status.UNSUPPORTED),       # 3x8 not built
-    ((A, A, A, A, None, A, 2, 16, 8, 64, 64, 1), Status.UNSUPPORTED),      # 2x16
+    ((A, A, A, A, None, A, 5, 8, 8, 64, 64, 1), Status.UNSUPPORTED),       # 5x8 not built
+    ((A, A, A, A, None, A, 3, 16, 8, 64, 64, 1), Status.UNSUPPORTED),      # 3x16
     ((A, A, A, A, None, A, 1, 12, 8, 64, 64, 1), Status.UNSUPPORTED),      # B = 12
+    ((A, A, A, A, None, A, 1, 8, 4, 64, 64, 1), Status.UNSUPPORTED),       # g = 4
     ((A + 8, A, A, A, None, A, 1, 16, 8, 64, 64, 1), Status.MISALIGNED),
     ((A, A + 2, A, A, None, A, 1, 16, 8, 64, 64, 1), Status.MISALIGNED),
     ((A, A, A, A, A + 4, A, 1, 16, 8, 64, 64, 1), Status.MISALIGNED),       # bias
@@ -107,7 +111,8 @@ def test_path_selection(lib):
             assert sel(M, B, g, 4096 + 8, 4096, batch) == Path.GEMV
         for batch in (9, 16, 256):
             assert sel(M, B, g, 4096 + 8, 4096, batch) == Path.TENSOR_CORE
-    assert sel(3, 8, 8, 4096, 4096, 1) == -1
+    assert sel(5, 8, 8, 4096, 4096, 1) == -1
+    assert sel(3, 8, 8, 4096, 4096, 1) == Path.TENSOR_CORE  # f2 schemes: tensor core from batch 1
     assert sel(1, 16, 8, 4095, 4096, 1) == -1
 
 
@@ -151,7 +156,7 @@ def test_group_validation_needs_no_gpu(lib):
     assert L_.aqlm_matmul_group(arr, 2, None, need, None) == Status.INVALID_ARG  # no workspace
     assert L_.aqlm_matmul_group(arr, 2, 1 << 40, need - 4, None) == Status.INVALID_ARG  # too small
     assert L_.aqlm_matmul_group(arr, 2, (1 << 40) + 16, need, None) == Status.MISALIGNED
-    bad = native.problem_array([P[0], _prob(1 << 35, M=3)])
+    bad = native.problem_array([P[0], _prob(1 << 35, M=5)])
     assert L_.aqlm_matmul_group(bad, 2, 1 << 40, need, None) == Status.UNSUPPORTED
     bad = native.problem_array([P[0], _prob(1 << 35, N=0)])
     assert L_.aqlm_matmul_group(bad, 2, 1 << 40, need, None) == Status.INVALID_ARG
@@ -177,7 +182,7 @@ def test_group_static_validation_needs_no_gpu(lib):
     # 16 Mixtral-8x7B expert linears (4096 x 14336) fit
     assert native.aqlm_group_workspace_size([_prob((i + 1) << 34, K=14336, N=4096) for i in range(16)]) == \
         16 * _ws_bytes(14336, 4096) <= native.STATIC_GROUP_SCRATCH_BYTES
-    bad = [_prob(1 << 32, M=3)]
+    bad = [_prob(1 << 32, M=5)]
     assert L_.aqlm_matmul_group_static(native.problem_array(bad), 1, None) == Status.UNSUPPORTED
 
 

@@ -77,9 +77,27 @@ size_t lut_group_workspace_bytes(const Problem* probs, int count);
 cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, uint32_t* status,
                              cudaStream_t stream);
 
-// True if the scheme is one the kernels are instantiated for.
+// True if the scheme is one the kernels are instantiated for: B = 8 codebooks
+// (256 entries) with M = 1..4, B = 16 codebooks (65536 entries) with M = 1..2, each
+// with codewords of g = 8 or 16 weights.
 inline bool scheme_supported(int M, int B, int g) {
-  return (M == 1 && B == 16 && (g == 8 || g == 16)) || (M == 2 && B == 8 && g == 8);
+  if (g != 8 && g != 16) return false;
+  if (B == 8) return M >= 1 && M <= 4;
+  if (B == 16) return M == 1 || M == 2;
+  return false;
+}
+
+// Calls F::template run<M, B, G>(args...) for the supported scheme (M, B, g), or
+// returns `fallback`.  Every launcher instantiates its kernels through this list.
+template <typename F, typename R, typename... Args>
+inline R dispatch_scheme(int M, int B, int g, R fallback, Args&&... args) {
+#define AQLM_SCHEME(m, b, gg) \
+  if (M == m && B == b && g == gg) return F::template run<m, b, gg>(args...);
+  AQLM_SCHEME(1, 8, 8) AQLM_SCHEME(2, 8, 8) AQLM_SCHEME(3, 8, 8) AQLM_SCHEME(4, 8, 8)
+  AQLM_SCHEME(1, 8, 16) AQLM_SCHEME(2, 8, 16) AQLM_SCHEME(3, 8, 16) AQLM_SCHEME(4, 8, 16)
+  AQLM_SCHEME(1, 16, 8) AQLM_SCHEME(2, 16, 8) AQLM_SCHEME(1, 16, 16) AQLM_SCHEME(2, 16, 16)
+#undef AQLM_SCHEME
+  return fallback;
 }
 
 }  // namespace aqlm

@@ -81,13 +81,21 @@ cudaError_t launch(const void* codes, const void* codebooks, const void* scales,
 
 }  // namespace
 
+namespace {
+struct DequantLauncher {
+  template <int M, int B, int G>
+  static cudaError_t run(const void* codes, const void* codebooks, const void* scales, void* W_out, int K, int N,
+                         cudaStream_t stream) {
+    return launch<M, B, G>(codes, codebooks, scales, W_out, K, N, stream);
+  }
+};
+}  // namespace
+
 cudaError_t launch_dequantize(const void* codes, const void* codebooks, const void* scales,
                               void* W_out, int M, int B, int g, int K, int N,
                               cudaStream_t stream) {
-  if (M == 1 && B == 16 && g == 8) return launch<1, 16, 8>(codes, codebooks, scales, W_out, K, N, stream);
-  if (M == 2 && B == 8 && g == 8) return launch<2, 8, 8>(codes, codebooks, scales, W_out, K, N, stream);
-  if (M == 1 && B == 16 && g == 16) return launch<1, 16, 16>(codes, codebooks, scales, W_out, K, N, stream);
-  return cudaErrorInvalidValue;
+  return dispatch_scheme<DequantLauncher>(M, B, g, cudaErrorInvalidValue, codes, codebooks, scales, W_out, K, N,
+                                          stream);
 }
 
 }  // namespace aqlm

@@ -81,7 +81,10 @@ __global__ void __launch_bounds__(128) gemv_gather_kernel(
   grid_dependency_wait();
 
   // 16-byte code vectors when every row starts 16-byte aligned.
-  const int nvec = (row_bytes % 16 == 0) ? groups / kGroupsPerVec : 0;
+  // (when M codes of a group do not tile 16 bytes, e.g. M = 3, every group takes the
+  // scalar path below)
+  constexpr bool kVecOk = (16 % (M * kCodeBytes)) == 0;
+  const int nvec = (kVecOk && row_bytes % 16 == 0) ? groups / kGroupsPerVec : 0;
   for (int v = lane; v < nvec; v += 32) {
     const uint4 q = ldg_stream_v4(row + static_cast<size_t>(v) * 16, stream_pol);
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
@@ -152,11 +155,17 @@ cudaError_t launch_scheme(const Problem& p, cudaStream_t stream) {
 
 }  // namespace
 
+namespace {
+struct GemvLauncher {
+  template <int M, int B, int G>
+  static cudaError_t run(const Problem& p, cudaStream_t stream) {
+    return launch_scheme<M, B, G>(p, stream);
+  }
+};
+}  // namespace
+
 cudaError_t launch_gemv(const Problem& p, cudaStream_t stream) {
-  if (p.M == 1 && p.B == 16 && p.g == 8) return launch_scheme<1, 16, 8>(p, stream);
-  if (p.M == 2 && p.B == 8 && p.g == 8) return launch_scheme<2, 8, 8>(p, stream);
-  if (p.M == 1 && p.B == 16 && p.g == 16) return launch_scheme<1, 16, 16>(p, stream);
-  return cudaErrorInvalidValue;
+  return dispatch_scheme<GemvLauncher>(p.M, p.B, p.g, cudaErrorInvalidValue, p, stream);
 }
 
 }  // namespace aqlm

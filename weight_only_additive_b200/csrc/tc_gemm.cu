@@ -187,14 +187,20 @@ cudaError_t launch_scheme(const Problem& p, uint32_t* status, cudaStream_t strea
 
 }  // namespace
 
+namespace {
+struct TcLauncher {
+  template <int M, int B, int G>
+  static cudaError_t run(const Problem& p, uint32_t* status, cudaStream_t stream) {
+    return launch_scheme<M, B, G>(p, status, stream);
+  }
+};
+}  // namespace
+
 cudaError_t launch_tc(const Problem& p, uint32_t* status, cudaStream_t stream) {
   // the pipelined kernel takes every shape with K % 64 == 0 and 16-byte code rows
   const cudaError_t e = launch_tc_pipelined(p, status, stream);
   if (e != cudaErrorNotSupported) return e;
-  if (p.M == 1 && p.B == 16 && p.g == 8) return launch_scheme<1, 16, 8>(p, status, stream);
-  if (p.M == 2 && p.B == 8 && p.g == 8) return launch_scheme<2, 8, 8>(p, status, stream);
-  if (p.M == 1 && p.B == 16 && p.g == 16) return launch_scheme<1, 16, 16>(p, status, stream);
-  return cudaErrorInvalidValue;
+  return dispatch_scheme<TcLauncher>(p.M, p.B, p.g, cudaErrorInvalidValue, p, status, stream);
 }
 
 }  // namespace aqlm
