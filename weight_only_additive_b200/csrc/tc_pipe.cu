@@ -46,8 +46,6 @@ constexpr int kDecoders = 256;        // warps 0-7: two threads per weight row
 constexpr int kThreads = 352;         // + x producer, MMA issuer, code producer
 constexpr int kWarpX = 8, kWarpMma = 9, kWarpCodes = 10;
 constexpr uint32_t kABytes = kRows * 128u;   // 16 KB per A stage
-constexpr uint32_t kCodeRowBytes = 64u;      // code bytes per row per code tile
-constexpr uint32_t kCodeTileBytes = kRows * kCodeRowBytes;  // 8 KB
 constexpr int kCodeSlots = 4;
 constexpr uint32_t kSmemLimit = 227u * 1024u;
 
@@ -68,17 +66,38 @@ struct PipeParams {
   uint32_t* status;
 };
 
+// Per-scheme constants.  A stage is 64 weights of a row: kStageCodeBytes of codes.
+// Code tiles are TMA boxes of 128 rows x kTileRowBytes (64 bytes when stages tile 64
+// bytes, loaded with the 64-byte swizzle; 48 bytes for M = 3, unswizzled).  B = 8
+// codebooks live in shared memory; B = 16 codebooks (1-2 MiB) are gathered from L2.
+constexpr int gcd_int(int a, int b) { return b == 0 ? a : gcd_int(b, a % b); }
+template <int M, int B, int G>
+struct PipeScheme {
+  static constexpr int kCodeBytes = B <= 8 ? 1 : 2;
+  static constexpr int kStageCodeBytes = (kStageK / G) * M * kCodeBytes;
+  static constexpr int kTileRowBytes = (64 % kStageCodeBytes == 0) ? 64 : 48;
+  static constexpr int kStagesPerTile = kTileRowBytes / kStageCodeBytes;
+  static constexpr uint32_t kCodeTileBytes = static_cast<uint32_t>(kRows * kTileRowBytes);
+  static constexpr bool kSwizzle64 = kTileRowBytes == 64;
+  static constexpr bool kSmemCb = B == 8;
+  static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;
+  static constexpr int kSplitAlign = 16 / gcd_int(16, kStageCodeBytes);  // split starts: 16-byte code offsets
+  static_assert(kTileRowBytes % kStageCodeBytes == 0 && kTileRowBytes % 16 == 0, "code tile rows");
+  // a decoder thread reads half a stage of codes: inside one 16-byte chunk when swizzled
+  static_assert(kStageCodeBytes % 2 == 0 && (!kSwizzle64 || 16 % (kStageCodeBytes / 2) == 0), "code halves");
+};
+
 struct PipeLayout {
   uint32_t a, b, codes, cb, bars, total;
 };
 
-__host__ __device__ inline PipeLayout pipe_layout(int S, int BN, bool smem_codebook) {
+__host__ __device__ inline PipeLayout pipe_layout(int S, int BN, uint32_t code_tile_bytes, uint32_t cb_bytes) {
   PipeLayout L;
   L.a = 0;                                                          // 1024-aligned stages
   L.b = L.a + static_cast<uint32_t>(S) * kABytes;
   L.codes = L.b + static_cast<uint32_t>(S) * static_cast<uint32_t>(BN) * 128u;
-  L.cb = L.codes + kCodeSlots * kCodeTileBytes;
-  L.bars = L.cb + (smem_codebook ? 2u * 256u * 16u : 0u);
+  L.cb = L.codes + kCodeSlots * code_tile_bytes;
+  L.bars = L.cb + cb_bytes;
   // full[S], empty[S], code_full[kCodeSlots], code_empty[kCodeSlots], acc, tmem slot, abort flag
   L.total = L.bars + 8u * static_cast<uint32_t>(2 * S + 2 * kCodeSlots + 1) + 16u;
   return L;
@@ -99,11 +118,15 @@ __device__ __forceinline__ uint32_t swz128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// Byte `off` (< 64) of row `row` of a code tile loaded with the 64-byte TMA swizzle:
-// the 16-byte chunk index is XORed with bits 7-8 of the byte offset (row / 2 mod 4),
-// so the 32 rows a warp reads at one chunk spread over all banks instead of two.
+// Byte `off` of row `row` of a code tile.  With the 64-byte TMA swizzle the 16-byte
+// chunk index is XORed with bits 7-8 of the byte offset (row / 2 mod 4), so the 32
+// rows a warp reads at one chunk spread over all banks instead of two.
+template <int kTileRowBytes, bool kSwizzle64>
 __device__ __forceinline__ uint32_t code_tile_offset(int row, int off) {
-  return static_cast<uint32_t>(row * 64 + ((((off >> 4) ^ (row >> 1)) & 3) << 4) + (off & 15));
+  if constexpr (kSwizzle64)
+    return static_cast<uint32_t>(row * 64 + ((((off >> 4) ^ (row >> 1)) & 3) << 4) + (off & 15));
+  else
+    return static_cast<uint32_t>(row * kTileRowBytes + off);
 }
 
 // Bounded wait that also gives up at once when another role has aborted.
@@ -122,70 +145,125 @@ __device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, volati
   return true;
 }
 
-// 1x16 g16 with register staging: the thread's 4 16-byte pieces of one stage
-// (chunks 4 hf .. 4 hf + 3 = its two 32-byte codewords), gathered from the
-// L2-resident codebook into registers: one 256-bit load per codeword when the
-// codebook is 32-byte aligned, else two 128-bit loads.
-__device__ __forceinline__ void gather_stage_g16(uint4 (&v)[4], const uint8_t* cw, int hf, bool row_valid,
+// B = 16 with register staging: the 16-byte pieces of the thread's 4 chunks of one
+// stage (chunks 4 hf .. 4 hf + 3), for each of the M codebooks, gathered from the
+// L2-resident codebooks into registers.  g = 16: one 256-bit load per 32-byte
+// codeword (two chunks) when the codebooks are 32-byte aligned, else two 128-bit
+// loads; g = 8: one 128-bit load per codeword.  `cw` points at the codes of the
+// thread's half of the stage ([group][m], 2 bytes each).
+template <int M, int G>
+__device__ __forceinline__ void gather_stage_b16(uint4 (&v)[M][4], const uint8_t* cw, bool row_valid,
                                                  const __half* __restrict__ codebooks, bool cb32) {
   const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
   if (!row_valid) {
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) v[cc] = make_uint4(0u, 0u, 0u, 0u);
-  } else if (cb32) {
+    for (int m = 0; m < M; ++m)
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc)
-      ldg_nc_v8(codebooks + static_cast<size_t>(c16[2 * hf + cc]) * 16, v[2 * cc], v[2 * cc + 1]);
+      for (int cc = 0; cc < 4; ++cc) v[m][cc] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const __half* cb = codebooks + static_cast<size_t>(m) * 65536u * G;
+    if constexpr (G == 8) {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) v[m][cc] = ldg_nc_v4(cb + static_cast<size_t>(c16[cc * M + m]) * 8);
+    } else if (cb32) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        ldg_nc_v8(cb + static_cast<size_t>(c16[q * M + m]) * 16, v[m][2 * q], v[m][2 * q + 1]);
+    } else {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        v[m][cc] = ldg_nc_v4(cb + static_cast<size_t>(c16[(cc >> 1) * M + m]) * 16 + 8 * (cc & 1));
+    }
+  }
+}
+
+// fp32 sum of the M 16-byte pieces (8 fp16 each) in codebook order, one rounding.
+template <int M>
+__device__ __forceinline__ uint4 sum_pieces(const uint4 (&q)[M]) {
+  if constexpr (M == 1) {
+    return q[0];
+  } else if constexpr (M == 2) {
+    // two fp16 values: their half2 sum is their exact sum rounded once
+    return make_uint4(hadd2_u32(q[0].x, q[1].x), hadd2_u32(q[0].y, q[1].y), hadd2_u32(q[0].z, q[1].z),
+                      hadd2_u32(q[0].w, q[1].w));
   } else {
+    float f[8];
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc)
-      v[cc] = ldg_nc_v4(codebooks + static_cast<size_t>(c16[2 * hf + (cc >> 1)]) * 16 + 8 * (cc & 1));
+    for (int m = 0; m < M; ++m) {
+      const uint32_t w[4] = {q[m].x, q[m].y, q[m].z, q[m].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 t = h2_to_f2(w[h]);
+        f[2 * h] = (m == 0) ? t.x : f[2 * h] + t.x;
+        f[2 * h + 1] = (m == 0) ? t.y : f[2 * h + 1] + t.y;
+      }
+    }
+    return make_uint4(f2_to_h2_rn(f[0], f[1]), f2_to_h2_rn(f[2], f[3]), f2_to_h2_rn(f[4], f[5]),
+                      f2_to_h2_rn(f[6], f[7]));
   }
 }
 
 // Decode half (`hf` = 0: chunks 0-3, 1: chunks 4-7) of one 64-wide K stage of
-// weight row `r` into the swizzled A stage at shared offset `a_off`.  `cw` points
-// at this stage's codes of the row.
+// weight row `r` into the swizzled A stage at shared offset `a_off`.  `cw` points at
+// the codes of this half of the stage (half the stage's code bytes, never crossing a
+// 16-byte chunk of a swizzled code tile).
+//   B = 16, M = 1, g = 8: each 16-byte chunk is one codeword, copied from the
+//     L2-resident codebook straight into its slot by cp.async (one 2-byte code load
+//     per gather, so each gather issues as soon as its own code has arrived).
+//   B = 8: the codebooks are staged in shared memory ([M][256][G]); a chunk is the
+//     sum of the matching 16-byte pieces of the group's M codewords.
 template <int M, int B, int G>
 __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase, uint32_t a_off, int r, int hf,
                                                   bool row_valid, const uint8_t* cw,
                                                   const __half* __restrict__ codebooks, const uint8_t* smem_cb) {
-  if constexpr (M == 1) {
-    // 1x16: each 16-byte piece of the row is (part of) one codeword: gather it.  Codes
-    // are read one by one (measured faster here than one wide load: each gather can
-    // issue as soon as its own code has arrived).
+  if constexpr (B == 16) {
+    static_assert(M == 1 && G == 8, "other B = 16 shapes use the register-staged decoder");
     const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       const int chunk = 4 * hf + cc;
-      const int j = chunk / (G / 8), h = chunk % (G / 8);
-      const uint32_t code = c16[j];
-      const __half* src = codebooks + static_cast<size_t>(code) * G + 8 * h;
+      const uint32_t code = c16[cc];
+      const __half* src = codebooks + static_cast<size_t>(code) * 8;
       cp_async_16_zfill(sbase + a_off + swz128(r, chunk),
                         row_valid ? static_cast<const void*>(src) : static_cast<const void*>(codebooks),
                         row_valid ? 16u : 0u);
     }
-  } else {
-    // 2x8: codes (c0, c1) per group; codebooks staged in shared memory as [2][256][8].
-    // The two codewords are added as half2 (one rounding of their exact sum).  The
-    // thread's 8 code bytes of this stage come in one load.
-    const uint2 q = *reinterpret_cast<const uint2*>(cw + 8 * hf);
+  } else if constexpr (M == 2 && G == 8) {
+    // 2x8: the thread's 8 code bytes (c0, c1 per group) of this stage in one load
+    const uint2 q = *reinterpret_cast<const uint2*>(cw);
     const uint32_t cwords[2] = {q.x, q.y};
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      const int j = 4 * hf + cc;
       uint4 out = make_uint4(0u, 0u, 0u, 0u);
       if (row_valid) {
         const uint32_t c0 = (cwords[cc >> 1] >> (16 * (cc & 1))) & 0xFFu;
         const uint32_t c1 = (cwords[cc >> 1] >> (16 * (cc & 1) + 8)) & 0xFFu;
-        const uint4 q0 = *reinterpret_cast<const uint4*>(smem_cb + (c0 << 4));
-        const uint4 q1 = *reinterpret_cast<const uint4*>(smem_cb + 4096u + (c1 << 4));
-        out.x = hadd2_u32(q0.x, q1.x);
-        out.y = hadd2_u32(q0.y, q1.y);
-        out.z = hadd2_u32(q0.z, q1.z);
-        out.w = hadd2_u32(q0.w, q1.w);
+        const uint4 pieces[2] = {*reinterpret_cast<const uint4*>(smem_cb + (c0 << 4)),
+                                 *reinterpret_cast<const uint4*>(smem_cb + 4096u + (c1 << 4))};
+        out = sum_pieces<2>(pieces);
       }
-      *reinterpret_cast<uint4*>(smem + a_off + swz128(r, j)) = out;
+      *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = out;
+    }
+  } else {
+    constexpr uint32_t kCbStride = 256u * G * 2u;  // bytes per codebook
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const int chunk = 4 * hf + cc;
+      const int j = cc / (G / 8), h = cc % (G / 8);  // group within the half, 16-byte piece
+      uint4 out = make_uint4(0u, 0u, 0u, 0u);
+      if (row_valid) {
+        uint4 pieces[M];
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+          pieces[m] = *reinterpret_cast<const uint4*>(smem_cb + static_cast<uint32_t>(m) * kCbStride +
+                                                      static_cast<uint32_t>(cw[j * M + m]) * (G * 2u) +
+                                                      16u * static_cast<uint32_t>(h));
+        out = sum_pieces<M>(pieces);
+      }
+      *reinterpret_cast<uint4*>(smem + a_off + swz128(r, chunk)) = out;
     }
   }
 }
@@ -201,11 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
   extern __shared__ uint8_t smem_raw[];
   // stages must be 1024-byte aligned for the 128-byte swizzle
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-  constexpr bool kSmemCb = (M == 2);
-  constexpr int kStageCodeBytes = (kStageK / G) * M * (B <= 8 ? 1 : 2);  // 16 (g8) or 8 (g16)
-  constexpr int kStagesPerTile = static_cast<int>(kCodeRowBytes) / kStageCodeBytes;
+  using SC = PipeScheme<M, B, G>;
+  constexpr int kStageCodeBytes = SC::kStageCodeBytes;
+  constexpr int kStagesPerTile = SC::kStagesPerTile;
+  constexpr uint32_t kCodeTileBytes = SC::kCodeTileBytes;
   const int S = p.S;
-  const PipeLayout L = pipe_layout(S, p.BN, kSmemCb);
+  const PipeLayout L = pipe_layout(S, p.BN, kCodeTileBytes, SC::kCbBytes);
   const uint32_t sbase = smem_addr(smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);   // stage s decoded and x landed
   uint64_t* empty = full + S;                                     // stage s consumed by the MMAs
@@ -244,8 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if constexpr (kSmemCb) {
-    for (int i = tid; i < 2 * 256; i += kThreads)
+  if constexpr (SC::kSmemCb) {
+    // the M codebooks, [M][256][G] fp16, copied as they are
+    for (int i = tid; i < static_cast<int>(SC::kCbBytes / 16u); i += kThreads)
       *reinterpret_cast<uint4*>(smem + L.cb + 16u * static_cast<uint32_t>(i)) = ldg_nc_v4(p.codebooks + 8 * i);
   }
   if (warp == 0) tmem_alloc(tmem_slot, p.tmem_cols);
@@ -307,14 +387,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     const int r = tid & (kRows - 1);
     const int hf = tid >> 7;
     const bool row_valid = n0 + r < p.N;
-    if constexpr (M == 1 && G == 16) {
-      // 1x16 g16: register-staged gathers, kLook stages ahead.  At step i the thread
-      // issues the gathers of stage i (one 256-bit load per 32-byte codeword: one L1TEX
-      // request instead of two cp.async) and stores stage i - kLook, gathered kLook
-      // steps earlier, into its A slot.  Measured faster than cp.async for g = 16 and
-      // slower for g = 8 (16-byte codewords), which keeps the cp.async path below.
-      constexpr int kLook = 3;
-      uint4 st[kLook + 1][4];
+    if constexpr (B == 16 && !(M == 1 && G == 8)) {
+      // B = 16 except 1x16 g8: register-staged gathers, kLook stages ahead.  At step i
+      // the thread issues the gathers of stage i (g = 16: one 256-bit load per 32-byte
+      // codeword, one L1TEX request instead of two cp.async) and stores stage i - kLook,
+      // gathered kLook steps earlier and summed over the M codebooks, into its A slot.
+      // Measured faster than cp.async for g = 16 and slower for 1x16 g8, which keeps
+      // the cp.async path below.
+      constexpr int kLook = (M == 1) ? 3 : 1;
+      uint4 st[kLook + 1][M][4];
       bool alive = true;
       for (int base = 0; alive && base < nks + kLook; base += kLook + 1) {
 #pragma unroll
@@ -338,8 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
           }
           if (issue) {
             const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
-                                code_tile_offset(r, within * kStageCodeBytes);
-            gather_stage_g16(st[u], cw, hf, row_valid, p.codebooks, p.cb32 != 0);
+                                code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
+                                    r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
+            gather_stage_b16<M, G>(st[u], cw, row_valid, p.codebooks, p.cb32 != 0);
             if (within == kStagesPerTile - 1 || i == nks - 1) {
               __syncwarp();  // every lane has read its codes of this tile
               if (lane == 0) mbar_arrive(&cempty[c]);
@@ -348,8 +430,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
           if (store) {
             const uint32_t a_off = L.a + static_cast<uint32_t>(sj) * kABytes;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-              *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = st[(u + 1) % (kLook + 1)][cc];
+            for (int cc = 0; cc < 4; ++cc) {
+              uint4 pieces[M];
+#pragma unroll
+              for (int m = 0; m < M; ++m) pieces[m] = st[(u + 1) % (kLook + 1)][m][cc];
+              *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = sum_pieces<M>(pieces);
+            }
             fence_proxy_async_smem();
             mbar_arrive(&full[sj]);
           }
@@ -371,11 +457,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
         break;
       }
       const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
-                          code_tile_offset(r, within * kStageCodeBytes);
+                          code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
+                              r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
       decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
                                  p.codebooks, smem + L.cb);
-      if constexpr (M == 1) {
-        cp_async_arrive_noinc(&full[s]);
+      if constexpr (B == 16) {
+        cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
       } else {
         fence_proxy_async_smem();
         mbar_arrive(&full[s]);
@@ -496,13 +583,15 @@ constexpr int kPlanFixedStages = 3;     // set-up, pipeline fill and epilogue, i
 constexpr int kPlanExchangePer16 = 2;   // split-K exchange, stage times per 16 batch columns
 constexpr int kMaxSplit = 16;
 
-inline uint32_t pipe_smem_bytes(int S, int BN, bool smem_cb) { return pipe_layout(S, BN, smem_cb).total + 1024; }
+template <int M, int B, int G>
+inline uint32_t pipe_smem_bytes(int S, int BN) {
+  using SC = PipeScheme<M, B, G>;
+  return pipe_layout(S, BN, SC::kCodeTileBytes, SC::kCbBytes).total + 1024;
+}
 
 template <int M, int B, int G>
 cudaError_t plan_pipe(int dev, const Problem& pr, int BN, TcPlan* out) {
-  constexpr bool kSmemCb = (M == 2);
-  constexpr int kStageCodeBytes = (kStageK / G) * M * (B <= 8 ? 1 : 2);
-  constexpr int kSplitAlign = 16 / kStageCodeBytes;  // split starts keep 16-byte code offsets
+  constexpr int kSplitAlign = PipeScheme<M, B, G>::kSplitAlign;  // split starts keep 16-byte code offsets
   static std::mutex mu;
   static std::map<std::tuple<int, int, int, int>, TcPlan> cache;
   const auto key = std::make_tuple(dev, pr.N, pr.K, pr.batch);
@@ -528,7 +617,7 @@ cudaError_t plan_pipe(int dev, const Problem& pr, int BN, TcPlan* out) {
   TcPlan best;
   long long best_cost = -1;
   for (int S = 6; S >= 2; --S) {
-    const uint32_t smem = pipe_smem_bytes(S, BN, kSmemCb);
+    const uint32_t smem = pipe_smem_bytes<M, B, G>(S, BN);
     if (smem > kSmemLimit) continue;
     const uint32_t stage_bytes = static_cast<uint32_t>(S) * (kABytes + static_cast<uint32_t>(BN) * 128u);
     for (int SK = 1; SK <= cmax; ++SK) {
@@ -574,7 +663,7 @@ cudaError_t plan_pipe(int dev, const Problem& pr, int BN, TcPlan* out) {
 
 template <int M, int B, int G>
 cudaError_t launch_pipe_plan(const Problem& pr, uint32_t* status, cudaStream_t stream, int BN, const TcPlan& plan) {
-  constexpr bool kSmemCb = (M == 2);
+  using SC = PipeScheme<M, B, G>;
   const size_t row_bytes = static_cast<size_t>(pr.K / G) * M * (B <= 8 ? 1 : 2);
   EncodeTiledFn encode = encode_tiled();
   if (!encode) return cudaErrorNotSupported;
@@ -595,11 +684,13 @@ cudaError_t launch_pipe_plan(const Problem& pr, uint32_t* status, cudaStream_t s
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(pr.N)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-    const cuuint32_t box[2] = {kCodeRowBytes, static_cast<cuuint32_t>(kRows)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(SC::kTileRowBytes), static_cast<cuuint32_t>(kRows)};
     const cuuint32_t estr[2] = {1, 1};
-    // 64-byte swizzle: the decoders read one chunk of 32 consecutive rows at a time
+    // 64-byte swizzle on 64-byte tile rows: the decoders read one chunk of 32
+    // consecutive rows at a time (48-byte rows, M = 3, are not swizzled)
     if (encode(&code_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pr.codes), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, SC::kSwizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorNotSupported;
   }
@@ -621,7 +712,7 @@ cudaError_t launch_pipe_plan(const Problem& pr, uint32_t* status, cudaStream_t s
   p.tmem_cols = cols;
   p.cb32 = (reinterpret_cast<uintptr_t>(pr.codebooks) & 31u) == 0 ? 1 : 0;
   p.status = status;
-  const uint32_t smem = pipe_smem_bytes(plan.S, BN, kSmemCb);
+  const uint32_t smem = pipe_smem_bytes<M, B, G>(plan.S, BN);
   auto kern = tc_pipe_kernel<M, B, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
   if (e != cudaSuccess) return e;
@@ -668,11 +759,17 @@ cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream
 
 }  // namespace
 
+namespace {
+struct PipeLauncher {
+  template <int M, int B, int G>
+  static cudaError_t run(const Problem& p, uint32_t* status, cudaStream_t stream) {
+    return launch_pipe<M, B, G>(p, status, stream);
+  }
+};
+}  // namespace
+
 cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t stream) {
-  if (p.M == 1 && p.B == 16 && p.g == 8) return launch_pipe<1, 16, 8>(p, status, stream);
-  if (p.M == 2 && p.B == 8 && p.g == 8) return launch_pipe<2, 8, 8>(p, status, stream);
-  if (p.M == 1 && p.B == 16 && p.g == 16) return launch_pipe<1, 16, 16>(p, status, stream);
-  return cudaErrorNotSupported;
+  return dispatch_scheme<PipeLauncher>(p.M, p.B, p.g, cudaErrorNotSupported, p, status, stream);
 }
 
 }  // namespace aqlm
