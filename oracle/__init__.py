@@ -14,11 +14,15 @@ Every function follows the definition stated at the top of
 * ``linear_lut``    -- the lookup-table route: per group and codebook a table of
                        x . codeword for every entry, then y = s . sum of looked-up
                        values + bias (fp64);
+* ``input_grad``    -- dx = dy . W16 in fp64 (n ascending): the gradient of the
+                       layer with respect to its input, for fine-tuning through a
+                       fixed quantised layer;
 * ``half_to_float`` / ``float_to_half`` -- IEEE-754 binary16 conversions written
                        from the format's definition (round to nearest, ties to even).
 
 Sources: the AQLM pages -- repo summary "What it does" (weights as sums of
-codebook vectors), inference-research record "Bits" / "Activation scheme" /
+codebook vectors; PV-Tuning fine-tuning after quantisation), "Key highlights"
+(PEFT fine-tuning), inference-research record "Bits" / "Activation scheme" /
 "Kernels" / "notes" (fp16 activations, lookup route, dequantise-then-GEMM
 route, no group-shared scale), paper record method paragraph.
 """
@@ -62,6 +66,9 @@ def _bind(path: str):
     lib.oracle_linear_rows.argtypes = [_u16p, _vp, _u16p, _u16p, _u16p, _f64p,
                                        _i, _i, _i, _i, _i, _i, _i64p, _i64, _i]
     lib.oracle_linear_rows.restype = _i
+    lib.oracle_input_grad_cols.argtypes = [_u16p, _vp, _u16p, _u16p, _f64p,
+                                           _i, _i, _i, _i, _i, _i, _i64p, _i64, _i]
+    lib.oracle_input_grad_cols.restype = _i
     for name in ("oracle_linear_exact", "oracle_linear_lut"):
         fn = getattr(lib, name)
         fn.argtypes = [_u16p, _vp, _u16p, _u16p, _u16p, _f64p, _i, _i, _i, _i, _i, _i, _i]
@@ -219,6 +226,25 @@ def linear_exact(x, codes, codebooks, scales, bias, M: int, B: int, g: int, nthr
 
 def linear_lut(x, codes, codebooks, scales, bias, M: int, B: int, g: int, nthreads: int = 0):
     return _linear_variant("oracle_linear_lut", x, codes, codebooks, scales, bias, M, B, g, nthreads)
+
+
+def input_grad(dy, codes, codebooks, scales, M: int, B: int, g: int,
+               cols=None, nthreads: int = 0) -> np.ndarray:
+    """Reference dx [batch, K] (or [batch, len(cols)]) in fp64: dx = dy . W16, where
+    W16 is dequantize()'s fp16 weight and n is summed in ascending order."""
+    codes = _codes(codes, B)
+    dy, cb, sc = _bits16(dy), _bits16(codebooks), _bits16(scales)
+    N, K = _shape(codes, cb, M, B, g)
+    batch = dy.shape[0]
+    if dy.shape[1] != N:
+        raise ValueError("dy must be [batch, N]")
+    c = None if cols is None else np.ascontiguousarray(np.asarray(cols, dtype=np.int64))
+    ncols = K if c is None else c.size
+    dx = np.empty((batch, ncols), np.float64)
+    _check(_load().oracle_input_grad_cols(_p(dy, _u16p), codes.ctypes.data, _p(cb, _u16p),
+                                          _p(sc, _u16p), _p(dx, _f64p), M, B, g, K, N, batch,
+                                          _p(c, _i64p), ncols, nthreads))
+    return dx
 
 
 def library_path() -> str:

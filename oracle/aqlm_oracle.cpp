@@ -23,7 +23,11 @@
 //     a group, so the only scale is per output row;
 //   * large batches dequantise to fp16 and run a dense fp16 GEMM ("notes"),
 //     small batches use lookups instead of per-element dequantisation
-//     ("Kernels") -- the LUT form below states that second route.
+//     ("Kernels") -- the LUT form below states that second route;
+//   * fine-tuning through a quantised layer (PEFT fine-tuning, repo summary
+//     "Key highlights"; PV-Tuning after quantisation, "What it does") keeps W
+//     fixed and needs the gradient with respect to the layer input,
+//     dx = dy . W16, the transpose of the same product (input-gradient form).
 //
 // Readings where the pages are silent (each also listed in the design notes):
 //   * codes layout [N, K/g, M] (m fastest), unsigned, no offset; uint8 when
@@ -322,6 +326,41 @@ int oracle_linear_lut(const uint16_t* x, const void* codes, const uint16_t* code
       double out = static_cast<double>(half_bits_to_float(scales[n])) * acc;
       if (bias) out += static_cast<double>(half_bits_to_float(bias[n]));
       y[b * N + n] = out;
+    }
+  }
+  return 0;
+}
+
+// Input gradient of y = x . W16^T + bias with respect to x:
+//   dx[b, k] = sum_{n ascending} f64(dy[b, n]) * f64(W16[n, k])     (fp64)
+// W16 is the dequantised weight of oracle_dequantize (scale included, rounded
+// to fp16), so this is exactly the transpose of the product that
+// oracle_linear_rows computes.  cols == NULL means all K columns in order; dx
+// is [batch, ncols].
+int oracle_input_grad_cols(const uint16_t* dy, const void* codes, const uint16_t* codebooks,
+                           const uint16_t* scales, double* dx, int M, int B, int g, int K, int N,
+                           int batch, const int64_t* cols, int64_t ncols, int nthreads) {
+  Shape s;
+  if (!make_shape(M, B, g, K, N, &s) || !dy || !codes || !codebooks || !scales || !dx || batch < 1)
+    return 1;
+  if (!cols) ncols = K;
+  for (int64_t r = 0; cols && r < ncols; ++r)
+    if (cols[r] < 0 || cols[r] >= K) return 1;
+  if (!codes_in_range(codes, s)) return 2;
+  const int nt = pick_threads(nthreads);
+  std::vector<uint16_t> W(static_cast<size_t>(N) * static_cast<size_t>(K));
+#pragma omp parallel for schedule(static) num_threads(nt)
+  for (int64_t n = 0; n < N; ++n) decode_row(codes, codebooks, scales, s, n, W.data() + n * K);
+#pragma omp parallel for schedule(static) num_threads(nt)
+  for (int64_t r = 0; r < ncols; ++r) {
+    const int64_t k = cols ? cols[r] : r;
+    for (int64_t b = 0; b < batch; ++b) {
+      double acc = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        acc += static_cast<double>(half_bits_to_float(dy[b * N + n])) *
+               static_cast<double>(half_bits_to_float(W[n * K + k]));
+      }
+      dx[b * ncols + r] = acc;
     }
   }
   return 0;

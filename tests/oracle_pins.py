@@ -124,6 +124,10 @@ def pin_integer_layer_exact(seed=2, M=2, B=8, g=8, K=256, N=96, batch=3):
     for fn in (oracle.linear, oracle.linear_exact, oracle.linear_lut):
         y = fn(x, codes, cb, sc, bias, M, B, g)
         assert np.array_equal(y * 2, y2.astype(np.float64)), fn.__name__
+    # the input gradient of the same layer: dy . W, exact in int64 (times 2)
+    dy = np.random.Generator(np.random.PCG64(seed + 100)).integers(-2, 3, size=(batch, N)).astype(np.float16)
+    dx2 = dy.astype(np.int64) @ W2
+    assert np.array_equal(oracle.input_grad(dy, codes, cb, sc, M, B, g) * 2, dx2.astype(np.float64))
 
 
 def pin_brute_force_tiny():
@@ -273,6 +277,59 @@ ALL_PINS = [pin_golden_decode, pin_identity_codebook_reproduces_w, pin_integer_l
 # ---------------------------------------------------------------------------
 # binary16 conversions (fast subset; tests/test_oracle_fp16.py is exhaustive)
 # ---------------------------------------------------------------------------
+# ---------------------------------------------------------------------------
+# input gradient dx = dy . W16 (fine-tuning through a fixed quantised layer)
+# ---------------------------------------------------------------------------
+def pin_golden_input_grad():
+    """Hand-derived worked example, tests/golden/input_grad_worked_example.json."""
+    with open(os.path.join(GOLDEN, "input_grad_worked_example.json")) as fh:
+        cases = json.load(fh)["cases"]
+    for c in cases:
+        M, B, g, cb, codes, sc = _case_arrays(c)
+        W = oracle.dequantize(codes, cb, sc, M, B, g)
+        assert np.array_equal(W, _f16(c["W"]).view(np.uint16)), c["name"]
+        dx = oracle.input_grad(_f16(c["dy"]), codes, cb, sc, M, B, g)
+        assert np.array_equal(dx, np.asarray(c["dx"], dtype=np.float64)), (c["name"], dx)
+        cols = [3, 0]
+        dx_cols = oracle.input_grad(_f16(c["dy"]), codes, cb, sc, M, B, g, cols=cols)
+        assert np.array_equal(dx_cols, np.asarray(c["dx"], dtype=np.float64)[:, cols]), c["name"]
+
+
+def pin_input_grad_matches_numpy(seed=11, M=3, B=8, g=16, K=320, N=72, batch=4):
+    """input_grad() = numpy fp64 dy @ W16 (an independent BLAS), W16 from dequantize()."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    cb = rng.normal(0, 0.05, size=(M, 1 << B, g)).astype(np.float16)
+    codes = rng.integers(0, 1 << B, size=(N, K // g, M)).astype(np.uint8)
+    sc = rng.uniform(0.5, 1.5, size=N).astype(np.float16)
+    dy = rng.normal(0, 1, size=(batch, N)).astype(np.float16)
+    W = oracle.dequantize(codes, cb, sc, M, B, g).view(np.float16).astype(np.float64)
+    want = dy.astype(np.float64) @ W
+    got = oracle.input_grad(dy, codes, cb, sc, M, B, g)
+    assert np.allclose(got, want, rtol=0, atol=1e-13 * np.abs(want).max())
+    cols = rng.choice(K, size=17, replace=False)
+    assert np.array_equal(oracle.input_grad(dy, codes, cb, sc, M, B, g, cols=cols), got[:, cols])
+
+
+def pin_input_grad_is_the_adjoint_of_linear(seed=12, K=256, N=96, batch=3):
+    """<dx, x> = <dy, y - bias> for every x: input_grad() is the transpose of the very
+    operator linear() applies (same W16, same scale, same index layout), checked on
+    schemes with one and two byte codes."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    for M, B, g in ((2, 8, 8), (1, 16, 8), (2, 16, 16)):
+        cb = rng.normal(0, 0.05, size=(M, 1 << B, g)).astype(np.float16)
+        codes = rng.integers(0, 1 << B, size=(N, K // g, M)).astype(np.uint8 if B <= 8 else np.uint16)
+        sc = rng.uniform(0.5, 1.5, size=N).astype(np.float16)
+        bias = rng.normal(0, 1, size=N).astype(np.float16)
+        x = rng.normal(0, 1, size=(batch, K)).astype(np.float16)
+        dy = rng.normal(0, 1, size=(batch, N)).astype(np.float16)
+        y = oracle.linear(x, codes, cb, sc, bias, M, B, g)
+        dx = oracle.input_grad(dy, codes, cb, sc, M, B, g)
+        lhs = (dx * x.astype(np.float64)).sum(axis=1)
+        rhs = (dy.astype(np.float64) * (y - bias.astype(np.float64))).sum(axis=1)
+        scale = np.abs(dx).sum() * np.abs(x.astype(np.float64)).max()
+        assert np.allclose(lhs, rhs, rtol=0, atol=1e-12 * scale), (M, B, g, lhs, rhs)
+
+
 def pin_fp16_conversions():
     import math
     import warnings
@@ -298,4 +355,5 @@ def pin_fp16_conversions():
     assert np.array_equal(oracle.float_to_half(u.view(np.float32)), ref16)
 
 
-ALL_PINS.append(pin_fp16_conversions)
+ALL_PINS += [pin_fp16_conversions, pin_golden_input_grad, pin_input_grad_matches_numpy,
+             pin_input_grad_is_the_adjoint_of_linear]

@@ -53,6 +53,18 @@ MUTANTS = {
         "acc += T[(j * M + m) * s.entries + code_at(codes, s, n, j, 0)];"),
     "lut_sign_flip": (
         "T[(j * M + m) * s.entries + i] = dot;", "T[(j * M + m) * s.entries + i] = -dot;"),
+    "input_grad_reads_dy_transposed": (
+        "acc += static_cast<double>(half_bits_to_float(dy[b * N + n])) *",
+        "acc += static_cast<double>(half_bits_to_float(dy[n * batch + b])) *"),
+    "input_grad_shifts_weight_column": (
+        "static_cast<double>(half_bits_to_float(W[n * K + k]));",
+        "static_cast<double>(half_bits_to_float(W[n * K + (k + 1) % K]));"),
+    "input_grad_skips_first_row": (
+        "for (int64_t n = 0; n < N; ++n) {\n        acc += static_cast<double>(half_bits_to_float(dy[",
+        "for (int64_t n = 1; n < N; ++n) {\n        acc += static_cast<double>(half_bits_to_float(dy["),
+    "input_grad_uses_row_as_column": (
+        "static_cast<double>(half_bits_to_float(W[n * K + k]));",
+        "static_cast<double>(half_bits_to_float(W[(k % N) * K + (n % K)]));"),
     "half_to_float_subnormal_scale": (
         "mag = std::ldexp(static_cast<float>(f), -24);", "mag = std::ldexp(static_cast<float>(f), -25);"),
     "half_to_float_drops_sign": ("return sign ? -mag : mag;", "return mag;"),
