@@ -110,6 +110,36 @@ aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void
                             void* W_out, int M, int B, int g, int K, int N,
                             aqlm_stream_t stream);
 
+/*
+ * Input gradient of the layer, for fine-tuning through a fixed quantised layer
+ * (AQLM repo summary "Additive quantization that actually survives one-bit
+ * weights": PV-Tuning after quantisation, section "What it does"; PEFT
+ * fine-tuning, section "Key highlights").  The weights do not change, so the
+ * backward pass of y = x . W^T . diag(s) + bias needs only
+ *
+ *   dx[b, k] = sum_n dy[b, n] * W16[n, k]        (dx = dy . diag(s) . W)
+ *
+ * with W16 exactly what aqlm_dequantize writes (the channel scale inside).
+ *   dy   fp16 [batch, N]   row-major, read
+ *   dx   fp16 [batch, K]   row-major, written; must not overlap dy or the weights
+ * codes, codebooks, scales: as for aqlm_matmul.  Accumulation is fp32; dx is
+ * rounded to fp16 (RNE).  Tolerance against the fp64 reference dy . W16:
+ * max|dx - dx_ref| / max|dx_ref| <= 5e-3.
+ * Supported: every scheme above, with N % 8 == 0 and code rows (K/g * M * B/8
+ * bytes) a multiple of 16 bytes; other shapes return AQLM_ERR_UNSUPPORTED.
+ * Alignment, ownership, stream ordering (dy plays x's part, dx y's) and errors
+ * as for aqlm_matmul; overlapping dx and inputs is AQLM_ERR_INVALID_ARG.
+ */
+aqlm_status aqlm_input_grad(const void* dy, const void* codes, const void* codebooks,
+                            const void* scales, void* dx, int M, int B, int g, int K, int N,
+                            int batch, aqlm_stream_t stream);
+
+/* Validates aqlm_input_grad's arguments exactly as it does, without launching
+ * anything.  Pure host logic: needs no GPU. */
+aqlm_status aqlm_validate_input_grad(const void* dy, const void* codes, const void* codebooks,
+                                     const void* scales, const void* dx, int M, int B, int g,
+                                     int K, int N, int batch);
+
 /* One layer of a group call: the arguments of aqlm_matmul, same meaning and
  * layout. */
 typedef struct {

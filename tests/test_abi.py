@@ -189,3 +189,37 @@ def test_group_static_validation_needs_no_gpu(lib):
 def test_selftest_rejects_bad_limits_without_a_gpu(lib):
     assert native.lib().aqlm_selftest_bounded_wait(0, None) == Status.INVALID_ARG
     assert native.lib().aqlm_selftest_bounded_wait(1000001, None) == Status.INVALID_ARG
+
+
+@pytest.mark.parametrize("M,B,g", SUPPORTED)
+def test_input_grad_supported_schemes_validate(lib, M, B, g):
+    v = native.aqlm_validate_input_grad
+    dx = 1 << 34  # far from every input range
+    assert v(A, A, A, A, dx, M, B, g, 4096, 4096, 1) == Status.OK
+    assert v(A, A, A, A, dx, M, B, g, 4096, 11008, 512) == Status.OK
+
+
+@pytest.mark.parametrize("args,want", [
+    ((None, A, A, A, 1 << 34, 2, 8, 8, 1024, 64, 1), Status.INVALID_ARG),      # null dy
+    ((A, A, A, A, None, 2, 8, 8, 1024, 64, 1), Status.INVALID_ARG),            # null dx
+    ((A, A, A, A, 1 << 34, 2, 8, 8, 1020, 64, 1), Status.INVALID_ARG),         # K % g != 0
+    ((A, A, A, A, 1 << 34, 2, 8, 8, 1024, 64, 0), Status.INVALID_ARG),         # batch = 0
+    ((A, A, A, A, 1 << 34, 5, 8, 8, 1024, 64, 1), Status.UNSUPPORTED),         # 5x8
+    ((A, A, A, A, 1 << 34, 2, 8, 8, 1024, 60, 1), Status.UNSUPPORTED),         # N % 8 != 0
+    ((A, A, A, A, 1 << 34, 1, 8, 16, 1088, 64, 1), Status.UNSUPPORTED),        # 68-byte code rows
+    ((A, A, A, A + 8, 1 << 34, 2, 8, 8, 1024, 64, 1), Status.MISALIGNED),      # scales
+    ((A, A, A, A, (1 << 34) + 2, 2, 8, 8, 1024, 64, 1), Status.MISALIGNED),    # dx
+    ((A, A, 1 << 30, A, A + 64, 2, 8, 8, 1024, 64, 1), Status.INVALID_ARG),     # dx overlaps dy
+    ((A, 1 << 30, A, A, (1 << 30) + 4096, 2, 8, 8, 1024, 64, 1), Status.INVALID_ARG),  # dx inside codes
+])
+def test_input_grad_validation_needs_no_gpu(lib, args, want):
+    assert native.aqlm_validate_input_grad(*args) == want
+
+
+def test_input_grad_rejects_bad_arguments_before_any_cuda_call(lib):
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_input_grad(A, A, A, A, 1 << 34, 2, 8, 8, 1024, 60, 1)
+    assert e.value.status == Status.UNSUPPORTED
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_input_grad(None, A, A, A, 1 << 34, 2, 8, 8, 1024, 64, 1)
+    assert e.value.status == Status.INVALID_ARG

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <utility>
 
 #include "aqlm.h"
 #include "aqlm_internal.h"
@@ -110,7 +111,7 @@ EncodeTiledFn encode_tiled() {
 
 extern "C" {
 
-int aqlm_abi_version(void) { return 4; }
+int aqlm_abi_version(void) { return 5; }
 
 const char* aqlm_status_string(aqlm_status status) {
   switch (status) {
@@ -183,6 +184,41 @@ aqlm_status aqlm_matmul(const void* x, const void* codes, const void* codebooks,
                         int M, int B, int g, int K, int N, int batch, aqlm_stream_t stream) {
   return aqlm_matmul_path(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch,
                           AQLM_PATH_AUTO, stream);
+}
+
+aqlm_status aqlm_validate_input_grad(const void* dy, const void* codes, const void* codebooks,
+                                     const void* scales, const void* dx, int M, int B, int g,
+                                     int K, int N, int batch) {
+  if (!dy || !codes || !codebooks || !scales || !dx) return AQLM_ERR_INVALID_ARG;
+  const aqlm_status st = validate_shape(M, B, g, K, N, batch);
+  if (st != AQLM_OK) return st;
+  if (!aligned16(dy) || !aligned16(codes) || !aligned16(codebooks) || !aligned16(scales) || !aligned16(dx))
+    return AQLM_ERR_MISALIGNED;
+  if (!aqlm::grad_shape_supported(M, B, g, K, N)) return AQLM_ERR_UNSUPPORTED;
+  // dx is written while dy and the weights are read
+  const auto at = [](const void* p, size_t n) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return std::make_pair(a, a + n);
+  };
+  const auto dxr = at(dx, static_cast<size_t>(batch) * K * 2);
+  const size_t code_bytes = static_cast<size_t>(N) * (K / g) * M * (B <= 8 ? 1 : 2);
+  const std::pair<uintptr_t, uintptr_t> inputs[4] = {
+      at(dy, static_cast<size_t>(batch) * N * 2), at(codes, code_bytes),
+      at(codebooks, static_cast<size_t>(M) * (size_t(1) << B) * g * 2), at(scales, static_cast<size_t>(N) * 2)};
+  for (const auto& r : inputs)
+    if (dxr.first < r.second && r.first < dxr.second) return AQLM_ERR_INVALID_ARG;
+  return AQLM_OK;
+}
+
+aqlm_status aqlm_input_grad(const void* dy, const void* codes, const void* codebooks,
+                            const void* scales, void* dx, int M, int B, int g, int K, int N,
+                            int batch, aqlm_stream_t stream) {
+  const aqlm_status st = aqlm_validate_input_grad(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch);
+  if (st != AQLM_OK) return st;
+  uint32_t* status = device_status_ptr();
+  if (!status) return from_cuda(cudaErrorInvalidDevice);
+  const aqlm::GradProblem p{dy, codes, codebooks, scales, dx, M, B, g, K, N, batch};
+  return from_cuda(aqlm::launch_input_grad(p, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 namespace {

@@ -67,6 +67,24 @@ inline bool tc_pipelined_shape(int M, int B, int g, int K) {
   return K % 64 == 0 && row_bytes % 16 == 0;
 }
 
+// Input gradient dx = dy . W16 (W16 the dequantised weight, scale included) on the
+// pipelined tensor-core kernel run transposed: dy [batch, N], dx [batch, K].
+struct GradProblem {
+  const void* dy;
+  const void* codes;
+  const void* codebooks;
+  const void* scales;
+  void* dx;
+  int M, B, g, K, N, batch;
+};
+cudaError_t launch_input_grad(const GradProblem& p, uint32_t* status, cudaStream_t stream);
+// Shape test of the gradient kernel: dy rows and code rows are TMA tensors, so
+// N % 8 == 0 (16-byte dy rows) and code rows a multiple of 16 bytes.
+inline bool grad_shape_supported(int M, int B, int g, int K, int N) {
+  const long long row_bytes = static_cast<long long>(K / g) * M * (B <= 8 ? 1 : 2);
+  return N % 8 == 0 && row_bytes % 16 == 0;
+}
+
 // Grouped lookup-table GEMV over independent 2x8 g8 batch-1 layers (one launch
 // of the partial-sum kernel, one of the reduction), at most kMaxGroupLayers per
 // launch.  The workspace holds every layer's fp32 partials, [ceil(G/64)][N] each,

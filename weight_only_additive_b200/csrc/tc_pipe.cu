@@ -53,8 +53,9 @@ struct PipeParams {
   const __half* codebooks;
   const __half* scales;
   const __half* bias;
-  __half* y;
+  __half* y;       // [batch, rows]
   int K, N, batch;
+  int rows;        // output rows = the MMA's M extent: N (layer) or K (input gradient)
   int BN;          // batch tile (multiple of 16, <= 256)
   int nk;          // K / 64 stages (whole K)
   int S;           // A/B stage ring depth
@@ -87,6 +88,30 @@ struct PipeScheme {
   static_assert(kStageCodeBytes % 2 == 0 && (!kSwizzle64 || 16 % (kStageCodeBytes / 2) == 0), "code halves");
 };
 
+// Input gradient dx = dy . W16 (kGrad kernels).  The MMA's M is 128 input features
+// k, its K is the reduction over output rows n, 64 per stage.  The A stage holds
+// W16[n][k] for 64 rows n x 128 features k in the MN-major 128-byte-swizzled
+// layout (k contiguous), which is the order a decoded codeword comes in.  A code
+// tile is one stage: 64 rows x the (128 / g) groups of the CTA's 128 features,
+// loaded as a TMA box of kBoxBytes (rounded up to 16 bytes, starting at the
+// 16-byte boundary at or below the tile's first code byte).
+template <int M, int B, int G>
+struct GradScheme {
+  static constexpr int kCodeBytes = B <= 8 ? 1 : 2;
+  static constexpr int kTileCodeBytes = (kRows / G) * M * kCodeBytes;   // codes of 128 features
+  static constexpr int kBoxBytes = kTileCodeBytes % 16 == 0 ? kTileCodeBytes : (kTileCodeBytes + 8 + 15) / 16 * 16;
+  static constexpr int kStagesPerTile = 1;
+  static constexpr int kStageCodeBytes = kTileCodeBytes;   // one code tile per stage
+  static constexpr int kTileRowBytes = kBoxBytes;
+  static constexpr bool kSwizzle64 = false;
+  static constexpr uint32_t kCodeTileBytes = static_cast<uint32_t>(kStageK * kBoxBytes);
+  static constexpr bool kSmemCb = B == 8;
+  static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;
+  static constexpr int kSplitAlign = 1;
+  // a decoder thread reads the codes of a quarter of the tile's features
+  static_assert(kTileCodeBytes % 8 == 0 && kBoxBytes <= 64, "gradient code tiles");
+};
+
 struct PipeLayout {
   uint32_t a, b, codes, cb, bars, total;
 };
@@ -116,6 +141,31 @@ __device__ __forceinline__ uint32_t mapa_shared_cluster(uint32_t addr, uint32_t 
 
 __device__ __forceinline__ uint32_t swz128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// MN-major 128-byte-swizzled A stage of the input-gradient kernel: feature k
+// (0..127) is the contiguous (MN) index, row n (0..63) the reduction (K) index.
+// Swizzle atoms are 8 rows x 64 features (1 KB, rows 128 bytes apart); atoms along
+// n are kGradSbo apart, the two 64-feature halves kGradLbo apart.  Offset of the
+// 16-byte chunk holding features 8 kc .. 8 kc + 7 of row n.
+constexpr uint32_t kGradSbo = 1024u;
+constexpr uint32_t kGradLbo = 8192u;
+__device__ __forceinline__ uint32_t grad_a_offset(int n, int kc) {
+  return static_cast<uint32_t>(kc >> 3) * kGradLbo + static_cast<uint32_t>(n >> 3) * kGradSbo +
+         static_cast<uint32_t>((n & 7) * 128 + (((kc & 7) ^ (n & 7)) << 4));
+}
+
+// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
+// leading byte offset = stride between swizzle atoms along M/N, stride byte
+// offset = stride between 8-row groups along K.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mnmajor(uint32_t smem_byte_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
 }
 
 // Byte `off` of row `row` of a code tile.  With the 64-byte TMA swizzle the 16-byte
@@ -206,6 +256,67 @@ __device__ __forceinline__ uint4 sum_pieces(const uint4 (&q)[M]) {
   }
 }
 
+// W16 for 8 features of one row from the M 16-byte codeword pieces: the pieces
+// summed in fp32 in codebook order, times the row's scale, rounded once to fp16 --
+// the dequantisation definition, so the gradient kernel's A operand is W16 bit for
+// bit.  For M = 1 a half2 multiply gives the same bits: the product of two fp16
+// values is exact in fp32, so both round the exact product once.
+template <int M>
+__device__ __forceinline__ uint4 scaled_sum_pieces(const uint4 (&q)[M], float s) {
+  if constexpr (M == 1) {
+    const __half2 s2 = __float2half2_rn(s);
+    const uint32_t w[4] = {q[0].x, q[0].y, q[0].z, q[0].w};
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&w[h]), s2);
+      o[h] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  } else {
+    float f[8];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const uint32_t w[4] = {q[m].x, q[m].y, q[m].z, q[m].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 t = h2_to_f2(w[h]);
+        f[2 * h] = (m == 0) ? t.x : f[2 * h] + t.x;
+        f[2 * h + 1] = (m == 0) ? t.y : f[2 * h + 1] + t.y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = f[e] * s;
+    return make_uint4(f2_to_h2_rn(f[0], f[1]), f2_to_h2_rn(f[2], f[3]), f2_to_h2_rn(f[4], f[5]),
+                      f2_to_h2_rn(f[6], f[7]));
+  }
+}
+
+// Input gradient, B = 8: decode the 4 chunks (32 features) of row `n` that thread
+// quarter `qq` owns into the MN-major A stage at shared offset `a_off`.  `cw`
+// points at the quarter's codes ([group][m], 1 byte each); `smem_cb` holds the M
+// codebooks [M][256][G].
+template <int M, int G>
+__device__ __forceinline__ void decode_grad_b8(uint8_t* smem, uint32_t a_off, int n, int qq, bool row_valid,
+                                               const uint8_t* cw, const uint8_t* smem_cb, float s) {
+  constexpr uint32_t kCbStride = 256u * G * 2u;
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int j = cc / (G / 8), h = cc % (G / 8);  // group within the quarter, 16-byte piece
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    if (row_valid) {
+      uint4 pieces[M];
+#pragma unroll
+      for (int m = 0; m < M; ++m)
+        pieces[m] = *reinterpret_cast<const uint4*>(smem_cb + static_cast<uint32_t>(m) * kCbStride +
+                                                    static_cast<uint32_t>(cw[j * M + m]) * (G * 2u) +
+                                                    16u * static_cast<uint32_t>(h));
+      out = scaled_sum_pieces<M>(pieces, s);
+    }
+    *reinterpret_cast<uint4*>(smem + a_off + grad_a_offset(n, 4 * qq + cc)) = out;
+  }
+}
+
 // Decode half (`hf` = 0: chunks 0-3, 1: chunks 4-7) of one 64-wide K stage of
 // weight row `r` into the swizzled A stage at shared offset `a_off`.  `cw` points at
 // the codes of this half of the stage (half the stage's code bytes, never crossing a
@@ -272,14 +383,17 @@ __device__ __forceinline__ void cluster_barrier() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int M, int B, int G>
+// kGrad = false: y = x . W16^T . diag(s) + bias (rows = N, reduction over K).
+// kGrad = true:  dx = dy . W16 (rows = K input features, reduction over the N
+//                output rows; x_map then describes dy [batch, N]).
+template <int M, int B, int G, bool kGrad>
 __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_constant__ CUtensorMap x_map,
                                                               const __grid_constant__ CUtensorMap code_map,
                                                               const PipeParams p) {
   extern __shared__ uint8_t smem_raw[];
   // stages must be 1024-byte aligned for the 128-byte swizzle
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-  using SC = PipeScheme<M, B, G>;
+  using SC = std::conditional_t<kGrad, GradScheme<M, B, G>, PipeScheme<M, B, G>>;
   constexpr int kStageCodeBytes = SC::kStageCodeBytes;
   constexpr int kStagesPerTile = SC::kStagesPerTile;
   constexpr uint32_t kCodeTileBytes = SC::kCodeTileBytes;
@@ -359,30 +473,128 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
         if (u > 0 && !pipe_wait(&cempty[c], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeCodes))
           break;
         mbar_arrive_expect_tx(&cfull[c], kCodeTileBytes);
-        // bytes past the row end (K edge) are zero-filled; stages past ks1 are not decoded
-        tma_load_2d(sbase + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes, &code_map,
-                    (ks0 + t * kStagesPerTile) * kStageCodeBytes, n0, &cfull[c], pol);
+        if constexpr (kGrad) {
+          // rows (ks0 + t) 64 .. + 63 of the CTA's feature columns; rows past N and
+          // bytes past the row end are zero-filled
+          tma_load_2d(sbase + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes, &code_map,
+                      (n0 * SC::kTileCodeBytes / kRows) & ~15, (ks0 + t) * kStageK, &cfull[c], pol);
+        } else {
+          // bytes past the row end (K edge) are zero-filled; stages past ks1 are not decoded
+          tma_load_2d(sbase + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes, &code_map,
+                      (ks0 + t * kStagesPerTile) * kStageCodeBytes, n0, &cfull[c], pol);
+        }
       }
     }
   } else if (warp == kWarpMma) {
     // ---- one thread issues the MMAs; each stage's commit releases it ----
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_f16_f32(kRows, static_cast<uint32_t>(p.BN));
+      // the gradient's A stage is MN-major (bit 15 of the instruction descriptor)
+      const uint32_t idesc = umma_idesc_f16_f32(kRows, static_cast<uint32_t>(p.BN)) | (kGrad ? (1u << 15) : 0u);
       for (int i = 0; i < nks; ++i) {
         const int s = i % S;
         if (!pipe_wait(&full[s], static_cast<uint32_t>((i / S) & 1), abort_flag, p.status, kSitePipeFull)) break;
         fence_proxy_async_smem();  // decoder writes (cp.async / st.shared) -> tensor-core reads
         tc_fence_after_sync();
-        const uint64_t adesc = umma_desc_sw128_kmajor(sbase + L.a + static_cast<uint32_t>(s) * kABytes);
+        const uint32_t a_addr = sbase + L.a + static_cast<uint32_t>(s) * kABytes;
         const uint64_t bdesc = umma_desc_sw128_kmajor(sbase + L.b + static_cast<uint32_t>(s * p.BN) * 128u);
 #pragma unroll
-        for (int kk = 0; kk < kStageK / 16; ++kk)
-          umma_f16_ss(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kStageK / 16; ++kk) {
+          // K = 16 per MMA: 32 bytes along a K-major row, or two 8-row atoms (2 x SBO) MN-major
+          const uint64_t adesc = kGrad ? umma_desc_sw128_mnmajor(a_addr + 2u * kGradSbo * kk, kGradLbo, kGradSbo)
+                                       : umma_desc_sw128_kmajor(a_addr) + 2 * kk;
+          umma_f16_ss(tmem, adesc, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
         umma_commit(&empty[s]);
       }
       umma_commit(acc_bar);
     }
   } else {
+    if constexpr (kGrad) {
+    // ---- decoders (input gradient): thread (row nl = 8 w + lane / 4, quarter qq =
+    // lane % 4) decodes features 32 qq .. 32 qq + 31 of row (ks0 + i) 64 + nl at
+    // stage i, scaled by that row's s_n.  A warp reads 8 rows x 4 quarters of codes
+    // (contiguous bytes) and its 32 chunk stores cover every bank group 4 times.
+    const int nl = 8 * warp + (lane >> 2);
+    const int qq = lane & 3;
+    const uint32_t code_off = static_cast<uint32_t>(nl * SC::kBoxBytes + ((n0 * SC::kTileCodeBytes / kRows) & 15) +
+                                                    qq * (SC::kTileCodeBytes / 4));
+    if constexpr (B == 16) {
+      // codewords gathered from L2 into registers kLook stages ahead, as in the layer kernel
+      constexpr int kLook = (M == 1) ? 3 : 1;
+      uint4 st[kLook + 1][M][4];
+      float sv[kLook + 1];
+      bool alive = true;
+      for (int base = 0; alive && base < nks + kLook; base += kLook + 1) {
+#pragma unroll
+        for (int u = 0; u <= kLook; ++u) {
+          const int i = base + u;      // stage gathered now
+          const int j = i - kLook;     // stage stored now
+          const bool issue = i < nks, store = j >= 0 && j < nks;
+          const int c = i % kCodeSlots;
+          const int sj = j >= 0 ? j % S : 0, uj = j >= 0 ? j / S : 0;
+          bool ready = true;
+          if (issue)
+            ready = pipe_wait(&cfull[c], static_cast<uint32_t>((i / kCodeSlots) & 1), abort_flag, p.status,
+                              kSitePipeCodes);
+          if (ready && store && uj > 0)
+            ready = pipe_wait(&empty[sj], static_cast<uint32_t>((uj - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
+          if (!__all_sync(0xffffffffu, ready)) {
+            *abort_flag = 1u;
+            alive = false;
+            break;
+          }
+          if (issue) {
+            const int n = (ks0 + i) * kStageK + nl;
+            const bool valid = n < p.N;
+            sv[u] = valid ? __half2float(p.scales[n]) : 0.f;
+            gather_stage_b16<M, G>(st[u], smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, valid,
+                                   p.codebooks, p.cb32 != 0);
+            __syncwarp();  // every lane has read its codes of this tile
+            if (lane == 0) mbar_arrive(&cempty[c]);
+          }
+          if (store) {
+            const int slot = (u + 1) % (kLook + 1);
+            const bool valid = (ks0 + j) * kStageK + nl < p.N;
+            const uint32_t a_off = L.a + static_cast<uint32_t>(sj) * kABytes;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              uint4 pieces[M];
+#pragma unroll
+              for (int m = 0; m < M; ++m) pieces[m] = st[slot][m][cc];
+              const uint4 out = valid ? scaled_sum_pieces<M>(pieces, sv[slot]) : make_uint4(0u, 0u, 0u, 0u);
+              *reinterpret_cast<uint4*>(smem + a_off + grad_a_offset(nl, 4 * qq + cc)) = out;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&full[sj]);
+          }
+        }
+      }
+    } else {
+      // B = 8: codebooks in shared memory; the next stage's scale is loaded one stage ahead
+      float s_next = (nks > 0 && ks0 * kStageK + nl < p.N) ? __half2float(p.scales[ks0 * kStageK + nl]) : 0.f;
+      for (int i = 0; i < nks; ++i) {
+        const int c = i % kCodeSlots;
+        bool ready = pipe_wait(&cfull[c], static_cast<uint32_t>((i / kCodeSlots) & 1), abort_flag, p.status,
+                               kSitePipeCodes);
+        const int s = i % S, u = i / S;
+        if (ready && u > 0)
+          ready = pipe_wait(&empty[s], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
+        if (!__all_sync(0xffffffffu, ready)) {
+          *abort_flag = 1u;
+          break;
+        }
+        const int n = (ks0 + i) * kStageK + nl;
+        const float sc = s_next;
+        if (i + 1 < nks) s_next = n + kStageK < p.N ? __half2float(p.scales[n + kStageK]) : 0.f;
+        decode_grad_b8<M, G>(smem, L.a + static_cast<uint32_t>(s) * kABytes, nl, qq, n < p.N,
+                             smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, smem + L.cb, sc);
+        fence_proxy_async_smem();
+        mbar_arrive(&full[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cempty[c]);
+      }
+    }
+    } else {
     // ---- decoders: threads r and r + 128 share weight row n0 + r (chunks 0-3 / 4-7) ----
     const int r = tid & (kRows - 1);
     const int hf = tid >> 7;
@@ -473,6 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
       }
     }
     }
+    }  // kGrad
     asm volatile("cp.async.wait_all;" ::: "memory");
   }
 
@@ -487,12 +700,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     acc_ok = __all_sync(0xffffffffu, pipe_wait(acc_bar, 0u, abort_flag, p.status, kSitePipeAcc) && !*abort_flag);
     tc_fence_after_sync();
   }
-  const int n = n0 + 32 * q + lane;
-  const bool n_valid = n < p.N;
+  const int n = n0 + 32 * q + lane;   // output row (input feature k for the gradient)
+  const bool n_valid = n < p.rows;
   if (p.SK == 1) {
     if (decoder && acc_ok) {
-      const float sc = n_valid ? __half2float(p.scales[n]) : 0.f;
-      const float bi = (n_valid && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
+      // the gradient's scale is inside its A operand and it has no bias
+      const float sc = kGrad ? 1.f : (n_valid ? __half2float(p.scales[n]) : 0.f);
+      const float bi = (!kGrad && n_valid && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
       for (int c0 = 16 * cpar; c0 < p.BN; c0 += 32) {
         float v[16];
         tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), v);
@@ -500,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int b = b0 + c0 + i;
-            if (b < p.batch) p.y[static_cast<size_t>(b) * p.N + n] = __float2half_rn(v[i] * sc + bi);
+            if (b < p.batch) p.y[static_cast<size_t>(b) * p.rows + n] = __float2half_rn(v[i] * sc + bi);
           }
         }
       }
@@ -543,11 +757,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
         const int col = idx / rows_owned;
         const int nn = n0 + r_begin + rl;
         const int b = b0 + col;
-        if (nn >= p.N || b >= p.batch) continue;
+        if (nn >= p.rows || b >= p.batch) continue;
         float acc = 0.f;
         for (int j = 0; j < SK; ++j) acc += recv[(j * R + rl) * pitch + col];
-        const float bi = p.bias != nullptr ? __half2float(p.bias[nn]) : 0.f;
-        p.y[static_cast<size_t>(b) * p.N + nn] = __float2half_rn(acc * __half2float(p.scales[nn]) + bi);
+        if constexpr (kGrad) {
+          p.y[static_cast<size_t>(b) * p.rows + nn] = __float2half_rn(acc);
+        } else {
+          const float bi = p.bias != nullptr ? __half2float(p.bias[nn]) : 0.f;
+          p.y[static_cast<size_t>(b) * p.rows + nn] = __float2half_rn(acc * __half2float(p.scales[nn]) + bi);
+        }
       }
     }
   }
@@ -583,18 +801,22 @@ constexpr int kPlanFixedStages = 3;     // set-up, pipeline fill and epilogue, i
 constexpr int kPlanExchangePer16 = 2;   // split-K exchange, stage times per 16 batch columns
 constexpr int kMaxSplit = 16;
 
-template <int M, int B, int G>
+template <int M, int B, int G, bool kGrad>
+using PipeSchemeOf = std::conditional_t<kGrad, GradScheme<M, B, G>, PipeScheme<M, B, G>>;
+
+template <int M, int B, int G, bool kGrad>
 inline uint32_t pipe_smem_bytes(int S, int BN) {
-  using SC = PipeScheme<M, B, G>;
+  using SC = PipeSchemeOf<M, B, G, kGrad>;
   return pipe_layout(S, BN, SC::kCodeTileBytes, SC::kCbBytes).total + 1024;
 }
 
-template <int M, int B, int G>
-cudaError_t plan_pipe(int dev, const Problem& pr, int BN, TcPlan* out) {
-  constexpr int kSplitAlign = PipeScheme<M, B, G>::kSplitAlign;  // split starts keep 16-byte code offsets
+// rows: output rows (the MMA's M extent); nk: 64-wide reduction stages.
+template <int M, int B, int G, bool kGrad>
+cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, TcPlan* out) {
+  constexpr int kSplitAlign = PipeSchemeOf<M, B, G, kGrad>::kSplitAlign;  // split starts keep 16-byte code offsets
   static std::mutex mu;
   static std::map<std::tuple<int, int, int, int>, TcPlan> cache;
-  const auto key = std::make_tuple(dev, pr.N, pr.K, pr.batch);
+  const auto key = std::make_tuple(dev, rows, nk, batch);
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -603,21 +825,20 @@ cudaError_t plan_pipe(int dev, const Problem& pr, int BN, TcPlan* out) {
       return cudaSuccess;
     }
   }
-  auto kern = tc_pipe_kernel<M, B, G>;
+  auto kern = tc_pipe_kernel<M, B, G, kGrad>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
   if (e != cudaSuccess) return e;
   const int cmax = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess
                        ? kMaxSplit : 8;
   cudaGetLastError();
 
-  const int nk = pr.K / kStageK;
-  const int row_tiles = (pr.N + kRows - 1) / kRows;
-  const int batch_tiles = (pr.batch + BN - 1) / BN;
+  const int row_tiles = (rows + kRows - 1) / kRows;
+  const int batch_tiles = (batch + BN - 1) / BN;
   const long long clusters = static_cast<long long>(row_tiles) * batch_tiles;
   TcPlan best;
   long long best_cost = -1;
   for (int S = 6; S >= 2; --S) {
-    const uint32_t smem = pipe_smem_bytes<M, B, G>(S, BN);
+    const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(S, BN);
     if (smem > kSmemLimit) continue;
     const uint32_t stage_bytes = static_cast<uint32_t>(S) * (kABytes + static_cast<uint32_t>(BN) * 128u);
     for (int SK = 1; SK <= cmax; ++SK) {
@@ -661,67 +882,58 @@ cudaError_t plan_pipe(int dev, const Problem& pr, int BN, TcPlan* out) {
   return cudaSuccess;
 }
 
-template <int M, int B, int G>
-cudaError_t launch_pipe_plan(const Problem& pr, uint32_t* status, cudaStream_t stream, int BN, const TcPlan& plan) {
-  using SC = PipeScheme<M, B, G>;
-  const size_t row_bytes = static_cast<size_t>(pr.K / G) * M * (B <= 8 ? 1 : 2);
+// Encodes the two tensor maps and launches one (row tile, batch tile, split) grid.
+//   x_src  [batch, red] fp16: x (layer, red = K) or dy (gradient, red = N)
+//   codes  [N, row_bytes] bytes; box {box_x, box_rows}
+template <int M, int B, int G, bool kGrad>
+cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, size_t row_bytes, int N,
+                               uint32_t box_x, uint32_t box_rows, PipeParams p, const TcPlan& plan,
+                               cudaStream_t stream) {
   EncodeTiledFn encode = encode_tiled();
   if (!encode) return cudaErrorNotSupported;
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(BN)) cols <<= 1;
-
   CUtensorMap x_map, code_map;
   {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.K), static_cast<cuuint64_t>(pr.batch)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.K) * 2};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kStageK), static_cast<cuuint32_t>(BN)};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(red), static_cast<cuuint64_t>(p.batch)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(red) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kStageK), static_cast<cuuint32_t>(p.BN)};
     const cuuint32_t estr[2] = {1, 1};
-    if (encode(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(pr.x), dims, strides, box, estr,
+    if (encode(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(x_src), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorNotSupported;
   }
   {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(pr.N)};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(N)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(SC::kTileRowBytes), static_cast<cuuint32_t>(kRows)};
+    const cuuint32_t box[2] = {box_x, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    // 64-byte swizzle on 64-byte tile rows: the decoders read one chunk of 32
-    // consecutive rows at a time (48-byte rows, M = 3, are not swizzled)
-    if (encode(&code_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pr.codes), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, SC::kSwizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    // layer kernel: the 64-byte swizzle on 64-byte tile rows, so the decoders' reads
+    // of one chunk of 32 consecutive rows spread over the banks (48-byte rows, M = 3,
+    // are not swizzled).  Gradient kernel: unswizzled (a warp reads contiguous bytes).
+    const bool swz = !kGrad && box_x == 64;
+    if (encode(&code_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swz ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorNotSupported;
   }
-
-  PipeParams p{};
-  p.codebooks = static_cast<const __half*>(pr.codebooks);
-  p.scales = static_cast<const __half*>(pr.scales);
-  p.bias = static_cast<const __half*>(pr.bias);
-  p.y = static_cast<__half*>(pr.y);
-  p.K = pr.K;
-  p.N = pr.N;
-  p.batch = pr.batch;
-  p.BN = BN;
-  p.nk = pr.K / kStageK;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(p.BN)) cols <<= 1;
+  p.tmem_cols = cols;
   p.S = plan.S;
   p.SK = plan.SK;
   p.ks_per = plan.ks_per;
   p.red_rows = plan.red_rows;
-  p.tmem_cols = cols;
-  p.cb32 = (reinterpret_cast<uintptr_t>(pr.codebooks) & 31u) == 0 ? 1 : 0;
-  p.status = status;
-  const uint32_t smem = pipe_smem_bytes<M, B, G>(plan.S, BN);
-  auto kern = tc_pipe_kernel<M, B, G>;
+  p.cb32 = (reinterpret_cast<uintptr_t>(p.codebooks) & 31u) == 0 ? 1 : 0;
+  const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(plan.S, p.BN);
+  auto kern = tc_pipe_kernel<M, B, G, kGrad>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
   if (e != cudaSuccess) return e;
   if (plan.SK > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  const int row_tiles = (pr.N + kRows - 1) / kRows;
-  const int batch_tiles = (pr.batch + BN - 1) / BN;
+  const int row_tiles = (p.rows + kRows - 1) / kRows;
+  const int batch_tiles = (p.batch + p.BN - 1) / p.BN;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -745,6 +957,7 @@ inline int pipe_batch_tile(int batch) { return std::min(256, (batch + 15) / 16 *
 
 template <int M, int B, int G>
 cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream) {
+  using SC = PipeScheme<M, B, G>;
   if (!tc_pipelined_shape(M, B, G, pr.K)) return cudaErrorNotSupported;
   if (!encode_tiled()) return cudaErrorNotSupported;
   int dev = 0;
@@ -752,24 +965,79 @@ cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream
   if (e != cudaSuccess) return e;
   const int BN = pipe_batch_tile(pr.batch);
   TcPlan plan;
-  e = plan_pipe<M, B, G>(dev, pr, BN, &plan);
+  e = plan_pipe<M, B, G, false>(dev, pr.N, pr.K / kStageK, pr.batch, BN, &plan);
   if (e != cudaSuccess) return e;
-  return launch_pipe_plan<M, B, G>(pr, status, stream, BN, plan);
+  PipeParams p{};
+  p.codebooks = static_cast<const __half*>(pr.codebooks);
+  p.scales = static_cast<const __half*>(pr.scales);
+  p.bias = static_cast<const __half*>(pr.bias);
+  p.y = static_cast<__half*>(pr.y);
+  p.K = pr.K;
+  p.N = pr.N;
+  p.batch = pr.batch;
+  p.rows = pr.N;
+  p.BN = BN;
+  p.nk = pr.K / kStageK;
+  p.status = status;
+  const size_t row_bytes = static_cast<size_t>(pr.K / G) * M * SC::kCodeBytes;
+  return launch_pipe_kernel<M, B, G, false>(pr.x, pr.K, pr.codes, row_bytes, pr.N,
+                                            static_cast<uint32_t>(SC::kTileRowBytes), static_cast<uint32_t>(kRows), p,
+                                            plan, stream);
 }
 
-}  // namespace
+template <int M, int B, int G>
+cudaError_t launch_grad(const GradProblem& pr, uint32_t* status, cudaStream_t stream) {
+  using SC = GradScheme<M, B, G>;
+  if (!grad_shape_supported(M, B, G, pr.K, pr.N)) return cudaErrorNotSupported;
+  if (!encode_tiled()) return cudaErrorNotSupported;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int BN = pipe_batch_tile(pr.batch);
+  const int nk = (pr.N + kStageK - 1) / kStageK;
+  TcPlan plan;
+  e = plan_pipe<M, B, G, true>(dev, pr.K, nk, pr.batch, BN, &plan);
+  if (e != cudaSuccess) return e;
+  PipeParams p{};
+  p.codebooks = static_cast<const __half*>(pr.codebooks);
+  p.scales = static_cast<const __half*>(pr.scales);
+  p.bias = nullptr;
+  p.y = static_cast<__half*>(pr.dx);
+  p.K = pr.K;
+  p.N = pr.N;
+  p.batch = pr.batch;
+  p.rows = pr.K;
+  p.BN = BN;
+  p.nk = nk;
+  p.status = status;
+  const size_t row_bytes = static_cast<size_t>(pr.K / G) * M * SC::kCodeBytes;
+  return launch_pipe_kernel<M, B, G, true>(pr.dy, pr.N, pr.codes, row_bytes, pr.N,
+                                           static_cast<uint32_t>(SC::kBoxBytes), static_cast<uint32_t>(kStageK), p,
+                                           plan, stream);
+}
 
-namespace {
 struct PipeLauncher {
   template <int M, int B, int G>
   static cudaError_t run(const Problem& p, uint32_t* status, cudaStream_t stream) {
     return launch_pipe<M, B, G>(p, status, stream);
   }
 };
+
+struct GradLauncher {
+  template <int M, int B, int G>
+  static cudaError_t run(const GradProblem& p, uint32_t* status, cudaStream_t stream) {
+    return launch_grad<M, B, G>(p, status, stream);
+  }
+};
+
 }  // namespace
 
 cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t stream) {
   return dispatch_scheme<PipeLauncher>(p.M, p.B, p.g, cudaErrorNotSupported, p, status, stream);
+}
+
+cudaError_t launch_input_grad(const GradProblem& p, uint32_t* status, cudaStream_t stream) {
+  return dispatch_scheme<GradLauncher>(p.M, p.B, p.g, cudaErrorNotSupported, p, status, stream);
 }
 
 }  // namespace aqlm

@@ -82,6 +82,25 @@ def matmul(x: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = None,
     return out
 
 
+def input_grad(dy: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """dx = dy . diag(s) . W [batch, K] for dy [batch, N] fp16: the gradient of
+    matmul() with respect to its input (the weights are fixed)."""
+    dev = w.codes.device
+    if dev.type != "cuda":
+        raise ValueError("AQLM weights must live on a CUDA device")
+    _check_tensor(dy, "dy", torch.float16, dev)
+    batch, N = dy.shape
+    if N != w.N:
+        raise ValueError(f"dy has N={N}, weights have N={w.N}")
+    if out is None:
+        out = torch.empty((batch, w.K), dtype=torch.float16, device=dev)
+    _check_tensor(out, "out", torch.float16, dev)
+    native.aqlm_input_grad(dy.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(), w.scales.data_ptr(),
+                           out.data_ptr(), w.M, w.B, w.g, w.K, N, batch, _stream_handle(stream, dev))
+    return out
+
+
 def dequantize(w: AqlmWeights, out: Optional[torch.Tensor] = None,
                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """W [N, K] fp16, bit-exact decode of the AQLM weights."""

@@ -18,9 +18,10 @@ LIBRARY = os.path.join(PKG, "libaqlm.so")
 EXPORTS = ("aqlm_matmul", "aqlm_matmul_path", "aqlm_dequantize", "aqlm_select_path",
            "aqlm_validate", "aqlm_status_string", "aqlm_check_device_status",
            "aqlm_last_cuda_error", "aqlm_abi_version", "aqlm_matmul_group",
-           "aqlm_group_workspace_size", "aqlm_matmul_group_static", "aqlm_selftest_bounded_wait")
+           "aqlm_group_workspace_size", "aqlm_matmul_group_static", "aqlm_selftest_bounded_wait",
+           "aqlm_input_grad", "aqlm_validate_input_grad")
 
-ABI_VERSION = 4
+ABI_VERSION = 5
 
 # Site code aqlm_selftest_bounded_wait records in the device status word.
 SITE_SELFTEST = 0x501
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
                 L.aqlm_select_path.restype = _i
                 L.aqlm_validate.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i]
                 L.aqlm_validate.restype = _i
+                L.aqlm_input_grad.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+                L.aqlm_input_grad.restype = _i
+                L.aqlm_validate_input_grad.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i]
+                L.aqlm_validate_input_grad.restype = _i
                 L.aqlm_status_string.argtypes = [_i]
                 L.aqlm_status_string.restype = ctypes.c_char_p
                 L.aqlm_check_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -144,6 +149,15 @@ def aqlm_select_path(M, B, g, K, N, batch) -> int:
 
 def aqlm_validate(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path=Path.AUTO) -> int:
     return lib().aqlm_validate(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, int(path))
+
+
+def aqlm_input_grad(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch, stream=None):
+    _check(lib().aqlm_input_grad(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch, stream),
+           "aqlm_input_grad")
+
+
+def aqlm_validate_input_grad(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch) -> int:
+    return lib().aqlm_validate_input_grad(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch)
 
 
 def aqlm_check_device_status(stream=None):
