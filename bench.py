@@ -27,6 +27,11 @@ no data-path collective).
 --impl reference times the CPU oracle (decode to fp16, fp64 matmul) on the
 host cores on a bounded sample of rows of every layer per step and reports the
 same metric.
+
+--op input-grad times the layer's input gradient instead (dx = dy . diag(s) . W,
+one aqlm_input_grad call per layer, default batch 1024 rows of dy, a fine-tuning
+micro-batch): metric TFLOP/s (2 . batch . N . K per layer), roofline against
+the tensor-core peak when the flops bound it.
 """
 from __future__ import annotations
 
@@ -56,7 +61,8 @@ L2_FALLBACK = 126 * 1024 * 1024
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=100000)
+    p.add_argument("--steps", type=int, default=None,
+                   help="timed steps (default 100000; 1000 with --op input-grad)")
     p.add_argument("--warmup", type=int, default=1000)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.BY_NAME))
@@ -70,9 +76,13 @@ def parse_args(argv=None):
                    help="skip the extra per-layer timing that the group mode reports beside its headline")
     p.add_argument("--launch", choices=("group", "per-layer"), default="group",
                    help="one aqlm_matmul_group call per step (default) or one aqlm_matmul call per layer")
+    p.add_argument("--op", choices=("matmul", "input-grad"), default="matmul",
+                   help="the layer (default) or its input gradient dx = dy . diag(s) . W")
     p.add_argument("--pool", type=int, default=None,
                    help="rotating-pool copies (default: enough to exceed 3x L2); smaller for profiler captures")
     a = p.parse_args(argv)
+    if a.steps is None:
+        a.steps = 1000 if a.op == "input-grad" else 100000
     if a.warmup < 3:
         p.error("--warmup must be at least 3")
     return a
@@ -91,8 +101,9 @@ def measured_peaks():
     if os.path.exists(path):
         with open(path) as fh:
             d = json.load(fh)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "source": "fallback"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured",
+                "tc_tflops_sustained": float(d.get("bf16_tflops_sustained", 1400.0))}
+    return {"hbm_gbs": 6650.0, "source": "fallback", "tc_tflops_sustained": 1400.0}
 
 
 KERNEL_SOURCES = {"gemv_gather_kernel": "gemv.cu", "gemv_lut_2x8_kernel": "gemv_lut.cu",
@@ -556,10 +567,226 @@ def run_ours(a):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# input gradient dx = dy . diag(s) . W
+# ---------------------------------------------------------------------------
+GRAD_METRIC = "AQLM input gradient dx = dy·diag(s)·W: TFLOP/s (2·batch·N·K per layer) & µs/layer"
+GRAD_DEFAULT_BATCH = 1024
+
+
+def grad_step_bytes(w, batch):
+    """Algorithmic bytes of one pass: codes + codebooks + scales + dy + dx per layer."""
+    out = 0
+    for l in w.layers:
+        s = l.scheme
+        out += (l.N * l.G * s.M * s.code_bytes + s.M * (1 << s.B) * s.g * 2 + 2 * l.N
+                + 2 * batch * l.N + 2 * batch * l.K)
+    return out
+
+
+def oracle_grad_sample_run(w, batch, seconds):
+    """Times oracle.input_grad (decode to fp16 + fp64 dy . W16) on column samples of
+    every layer until about `seconds` have been spent.  Returns (flops credited, seconds,
+    columns per layer, threads)."""
+    import oracle
+
+    rng = np.random.Generator(np.random.PCG64(5))
+    flops, elapsed, cols = 0.0, 0.0, 16
+    host = []
+    for li, lay in enumerate(w.layers):
+        s = lay.scheme
+        host.append((synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index, layer=li),
+                     synth.make_x(batch, lay.N, seed=1, workload=w.index, layer=li)))
+    while elapsed < 0.9 * seconds:
+        for lay, (ld, dy) in zip(w.layers, host):
+            s = lay.scheme
+            sel = np.sort(rng.choice(lay.K, size=cols, replace=False))
+            t0 = time.perf_counter()
+            oracle.input_grad(dy, ld.codes, ld.codebooks, ld.scales, s.M, s.B, s.g, cols=sel)
+            elapsed += time.perf_counter() - t0
+            flops += 2.0 * batch * lay.N * cols
+            if elapsed >= 0.9 * seconds:
+                break
+    return flops, elapsed, cols, oracle.max_threads()
+
+
+def run_input_grad(a):
+    import torch
+
+    from weight_only_additive_b200 import layer as L
+    from weight_only_additive_b200 import native
+
+    rank, world, local = env_rank()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist = None
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = native.lib()
+    w = select_workload(a)
+    batch = a.batch if a.batch is not None else GRAD_DEFAULT_BATCH
+    sbytes = grad_step_bytes(w, batch)
+    sflops = sum(2.0 * batch * l.N * l.K for l in w.layers)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 0) or L2_FALLBACK
+    pool = max(2, math.ceil(3 * l2 / sbytes)) if a.pool is None else max(1, a.pool)
+
+    weights, dys = [], []
+    for c in range(pool):
+        wc, dc = [], []
+        for li, lay in enumerate(w.layers):
+            s = lay.scheme
+            ld = synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index,
+                                  layer=li + w.extra.get("layer_offset", 0), copy=c + 1000 * rank)
+            wc.append(L.AqlmWeights.from_numpy(ld, dev))
+            dc.append(torch.from_numpy(synth.make_x(batch, lay.N, seed=1, workload=w.index, layer=li,
+                                                    copy=c + 1000 * rank)).to(dev))
+        weights.append(wc)
+        dys.append(dc)
+    dxs = [torch.empty((batch, lay.K), dtype=torch.float16, device=dev) for lay in w.layers]
+    stream = torch.cuda.Stream(dev)
+    h = stream.cuda_stream
+    calls = [[(dys[c][li].data_ptr(), weights[c][li].codes.data_ptr(), weights[c][li].codebooks.data_ptr(),
+               weights[c][li].scales.data_ptr(), dxs[li].data_ptr(), lay.scheme.M, lay.scheme.B, lay.scheme.g,
+               lay.K, lay.N, batch, h) for li, lay in enumerate(w.layers)] for c in range(pool)]
+
+    def step(c):
+        for args in calls[c]:
+            st = lib.aqlm_input_grad(*args)
+            if st != 0:
+                raise native.AqlmError(st, "aqlm_input_grad")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for c in range(pool):
+            step(c)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for c in range(pool):
+            step(c)
+    passes = max(1, a.steps // pool)
+    steps = passes * pool
+    with torch.cuda.stream(stream):
+        for _ in range(-(-a.warmup // pool)):  # at least `warmup` steps
+            graph.replay()
+    torch.cuda.synchronize(dev)
+    barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, enabled=not a.no_clocks) as clocks:
+        torch.cuda.synchronize(dev)
+        barrier()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(passes):
+                graph.replay()
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    ms = max_over_ranks(start.elapsed_time(end), dist, dev)
+    st, detail = L.check_device_status(stream=stream)
+    if st != native.Status.OK:
+        raise RuntimeError(f"device status {st.name} {detail:#x}")
+    del graph
+    ms_step = ms / steps
+    value = sflops * steps * world / (ms / 1e3) / 1e12
+    peaks = measured_peaks()
+    launch_s = (ms / 1e3) / (steps * len(w.layers))
+    t_tc = sflops / len(w.layers) / (peaks["tc_tflops_sustained"] * 1e12)
+    t_hbm = sbytes / len(w.layers) / (peaks["hbm_gbs"] * 1e9)
+    if t_tc >= t_hbm:
+        roofline = {"bound": "tensor", "achieved": sflops / len(w.layers) / launch_s / 1e12,
+                    "peak": peaks["tc_tflops_sustained"], "unit": "TFLOP/s"}
+    else:
+        roofline = {"bound": "hbm", "achieved": sbytes / len(w.layers) / launch_s / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roofline.update({"frac": roofline["achieved"] / roofline["peak"], "traffic": None,
+                     "kernel": "tc_pipe_kernel (input gradient)", "timed": "average launch of the step",
+                     "peak_source": ("measured (MEASURED_PEAKS.json bf16_tflops_sustained; fp16 has the same "
+                                     "nominal tensor rate)" if roofline["bound"] == "tensor"
+                                     else "measured (MEASURED_PEAKS.json hbm_gbs)")
+                     if peaks["source"] == "measured" else "fallback"})
+
+    e2e = None
+    if not a.no_e2e:
+        e2e_steps = max(3, min(steps, 200))
+        noff = np.cumsum([0] + [batch * lay.N for lay in w.layers])
+        koff = np.cumsum([0] + [batch * lay.K for lay in w.layers])
+        hdy = torch.empty((int(noff[-1]),), dtype=torch.float16).pin_memory()
+        for li, lay in enumerate(w.layers):
+            hdy[noff[li]:noff[li + 1]] = torch.from_numpy(synth.make_x(batch, lay.N, seed=7, layer=li)).reshape(-1)
+        hdx = torch.empty((int(koff[-1]),), dtype=torch.float16).pin_memory()
+        ddy, ddx = torch.empty_like(hdy, device=dev), torch.empty_like(hdx, device=dev)
+        vdy = [ddy[noff[li]:noff[li + 1]].view(batch, lay.N) for li, lay in enumerate(w.layers)]
+        vdx = [ddx[koff[li]:koff[li + 1]].view(batch, lay.K) for li, lay in enumerate(w.layers)]
+
+        def e2e_step(c):
+            ddy.copy_(hdy, non_blocking=True)
+            for li in range(len(w.layers)):
+                L.input_grad(vdy[li], weights[c][li], out=vdx[li], stream=stream)
+            hdx.copy_(ddx, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                e2e_step(i % pool)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(e2e_steps):
+                e2e_step(i % pool)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        e2e = {"value": sflops * e2e_steps * world / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": hdy.numel() * 2, "d2h_bytes_per_step": hdx.numel() * 2,
+               "steps": e2e_steps, "us_per_layer": ems * 1e3 / (e2e_steps * len(w.layers)),
+               "how": "per step: one pinned H2D copy of every layer's dy (packed), "
+                      "weight_only_additive_b200.layer.input_grad -> aqlm_input_grad per layer, one D2H copy "
+                      "of every dx (packed); no CUDA graph"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        f, s, cols, threads = oracle_grad_sample_run(w, batch, a.cpu_seconds)
+        cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{cols} sampled columns of dx per layer (the oracle decodes the whole W16 each call, "
+                         f"then fp64 dy . W16 for those columns), batch {batch}, {s:.1f} s on the host cores"}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        line = {"metric": GRAD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+                "warmup": a.warmup, "ms_per_step": ms_step, "us_per_layer": ms_step * 1e3 / len(w.layers),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+                "data": "synthetic",
+                "config": {"workload": w.name, "op": "input-grad", "layers": len(w.layers), "batch": batch,
+                           "scheme": w.layers[0].scheme.name, "algorithmic_bytes_per_step": sbytes,
+                           "flops_per_step": sflops,
+                           "l2": f"inputs larger than L2: rotating pool of {pool} copies "
+                                 f"({pool * sbytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
+                           "launch": f"one aqlm_input_grad call per layer; CUDA graphs of {pool} steps",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": len(w.layers) * steps, "clocks": clocks.summary(), "gpu": props.name}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     a = parse_args(argv)
     if a.impl == "reference":
         return run_reference(a)
+    if a.op == "input-grad":
+        return run_input_grad(a)
     return run_ours(a)
 
 

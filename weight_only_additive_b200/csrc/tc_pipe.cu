@@ -200,10 +200,11 @@ __device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, volati
 // L2-resident codebooks into registers.  g = 16: one 256-bit load per 32-byte
 // codeword (two chunks) when the codebooks are 32-byte aligned, else two 128-bit
 // loads; g = 8: one 128-bit load per codeword.  `cw` points at the codes of the
-// thread's half of the stage ([group][m], 2 bytes each).
+// thread's half of the stage ([group][m], 2 bytes each).  v[m][i] receives chunk
+// (i + rot) mod 4 (rot = 0 or 2).
 template <int M, int G>
 __device__ __forceinline__ void gather_stage_b16(uint4 (&v)[M][4], const uint8_t* cw, bool row_valid,
-                                                 const __half* __restrict__ codebooks, bool cb32) {
+                                                 const __half* __restrict__ codebooks, bool cb32, int rot = 0) {
   const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
   if (!row_valid) {
 #pragma unroll
@@ -217,15 +218,17 @@ __device__ __forceinline__ void gather_stage_b16(uint4 (&v)[M][4], const uint8_t
     const __half* cb = codebooks + static_cast<size_t>(m) * 65536u * G;
     if constexpr (G == 8) {
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) v[m][cc] = ldg_nc_v4(cb + static_cast<size_t>(c16[cc * M + m]) * 8);
+      for (int cc = 0; cc < 4; ++cc) v[m][cc] = ldg_nc_v4(cb + static_cast<size_t>(c16[((cc + rot) & 3) * M + m]) * 8);
     } else if (cb32) {
 #pragma unroll
       for (int q = 0; q < 2; ++q)
-        ldg_nc_v8(cb + static_cast<size_t>(c16[q * M + m]) * 16, v[m][2 * q], v[m][2 * q + 1]);
+        ldg_nc_v8(cb + static_cast<size_t>(c16[(q ^ (rot >> 1)) * M + m]) * 16, v[m][2 * q], v[m][2 * q + 1]);
     } else {
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
-        v[m][cc] = ldg_nc_v4(cb + static_cast<size_t>(c16[(cc >> 1) * M + m]) * 16 + 8 * (cc & 1));
+      for (int cc = 0; cc < 4; ++cc) {
+        const int ch = (cc + rot) & 3;
+        v[m][cc] = ldg_nc_v4(cb + static_cast<size_t>(c16[(ch >> 1) * M + m]) * 16 + 8 * (ch & 1));
+      }
     }
   }
 }
@@ -292,6 +295,12 @@ __device__ __forceinline__ uint4 scaled_sum_pieces(const uint4 (&q)[M], float s)
   }
 }
 
+// The chunk (of the thread's 4) that quarter `qq` stores at step `step`.  The 8
+// lanes of a quarter-warp (2 rows x 4 quarters) then write 8 different 16-byte bank
+// groups of the MN-major stage: quarters 0 and 2 (and 1 and 3) differ only in the
+// 64-feature half, which the swizzle does not separate, so they start 2 chunks apart.
+__device__ __forceinline__ int grad_chunk_at(int step, int qq) { return (step + 2 * (qq >> 1)) & 3; }
+
 // Input gradient, B = 8: decode the 4 chunks (32 features) of row `n` that thread
 // quarter `qq` owns into the MN-major A stage at shared offset `a_off`.  `cw`
 // points at the quarter's codes ([group][m], 1 byte each); `smem_cb` holds the M
@@ -301,7 +310,8 @@ __device__ __forceinline__ void decode_grad_b8(uint8_t* smem, uint32_t a_off, in
                                                const uint8_t* cw, const uint8_t* smem_cb, float s) {
   constexpr uint32_t kCbStride = 256u * G * 2u;
 #pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {
+  for (int step = 0; step < 4; ++step) {
+    const int cc = grad_chunk_at(step, qq);
     const int j = cc / (G / 8), h = cc % (G / 8);  // group within the quarter, 16-byte piece
     uint4 out = make_uint4(0u, 0u, 0u, 0u);
     if (row_valid) {
@@ -548,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
             const bool valid = n < p.N;
             sv[u] = valid ? __half2float(p.scales[n]) : 0.f;
             gather_stage_b16<M, G>(st[u], smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, valid,
-                                   p.codebooks, p.cb32 != 0);
+                                   p.codebooks, p.cb32 != 0, 2 * (qq >> 1));
             __syncwarp();  // every lane has read its codes of this tile
             if (lane == 0) mbar_arrive(&cempty[c]);
           }
@@ -557,12 +567,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
             const bool valid = (ks0 + j) * kStageK + nl < p.N;
             const uint32_t a_off = L.a + static_cast<uint32_t>(sj) * kABytes;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int step = 0; step < 4; ++step) {
+              // register slot `step` holds chunk grad_chunk_at(step, qq) (gathered rotated)
               uint4 pieces[M];
 #pragma unroll
-              for (int m = 0; m < M; ++m) pieces[m] = st[slot][m][cc];
+              for (int m = 0; m < M; ++m) pieces[m] = st[slot][m][step];
               const uint4 out = valid ? scaled_sum_pieces<M>(pieces, sv[slot]) : make_uint4(0u, 0u, 0u, 0u);
-              *reinterpret_cast<uint4*>(smem + a_off + grad_a_offset(nl, 4 * qq + cc)) = out;
+              *reinterpret_cast<uint4*>(smem + a_off + grad_a_offset(nl, 4 * qq + grad_chunk_at(step, qq))) = out;
             }
             fence_proxy_async_smem();
             mbar_arrive(&full[sj]);
