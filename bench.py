@@ -275,6 +275,33 @@ def oracle_sample_run(w, batch, seconds, copy=0):
     return total_bytes, elapsed, sampled, oracle.max_threads()
 
 
+def cpu_kernel_run(w, batch, seconds):
+    """Times libaqlm_cpu.so (the multithreaded lookup-table / decode+dot CPU kernel)
+    on whole layers of the workload, repeating the set for about `seconds`.  Not the
+    oracle: reported beside cpu_baseline as the fast CPU implementation."""
+    from weight_only_additive_b200 import cpu as cpu_lib
+
+    layers = host_layers(w, batch)
+    cpu_lib.matmul(layers[0][2], layers[0][1].codes, layers[0][1].codebooks, layers[0][1].scales, None,
+                   layers[0][1].M, layers[0][1].B, layers[0][1].g)  # warm-up (thread pool, pages)
+    passes, elapsed = 0, 0.0
+    while elapsed < seconds or passes < 2:
+        t0 = time.perf_counter()
+        for lay, ld, x in layers:
+            cpu_lib.matmul(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g)
+        elapsed += time.perf_counter() - t0
+        passes += 1
+    sbytes = step_bytes(w, batch)
+    method = ("lookup tables per 16-group K slice" if w.layers[0].scheme.B == 8 and batch <= 8
+              else "decode to fp32 + dot products")
+    return {"value": sbytes * passes / elapsed / 1e9, "unit": "GB/s",
+            "ms_per_step": elapsed * 1e3 / passes, "cores": os.cpu_count(),
+            "simd": "avx2+fma+f16c" if cpu_lib.simd_level() == 1 else "scalar",
+            "kind": "libaqlm_cpu.so (aqlm_cpu_matmul)",
+            "sample": f"{passes} passes over all {len(w.layers)} whole layers, batch {batch}, {method}, "
+                      f"{elapsed:.1f} s"}
+
+
 def run_reference(a):
     rank, world, _ = env_rank()
     w = select_workload(a)
@@ -533,12 +560,14 @@ def run_ours(a):
                       f"of every y (packed); no CUDA graph"}
 
     cpu = None
+    cpu_kernel = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         b, s, rows, threads = oracle_sample_run(w, batch, a.cpu_seconds)
         cpu = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": f"{rows} rows of each of the {len(w.layers)} layers (whole layers repeated "
                          f"when the budget exceeds them; decode to fp16 + fp64 matmul), batch {batch}, "
                          f"{s:.1f} s on the host cores"}
+        cpu_kernel = cpu_kernel_run(w, batch, min(a.cpu_seconds, 5.0))
 
     if dist is not None:
         dist.barrier()
@@ -559,7 +588,7 @@ def run_ours(a):
                                       "reduction)" if mode == "group" else "one aqlm_matmul call per layer")
                                      + f"; CUDA graphs of {pool} consecutive steps (one pass over the pool)",
                            "parallelism": f"replicas x{world}"},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "cpu_baseline": cpu, "cpu_kernel": cpu_kernel, "e2e": e2e,
                 "other_launch": other,
                 "gpu_launches": launches_per_step * a.steps,
                 "clocks": clock_summary, "gpu": props.name}

@@ -1,0 +1,135 @@
+"""libaqlm_cpu.so (the multithreaded host-CPU kernel) against the CPU oracle.
+
+The same bar as the GPU path: max|y - y_ref| / max|y_ref| <= 5e-3 against the
+oracle's fp64 reference of the decoded fp16 weights, no NaN/Inf, for every
+supported scheme on both methods (lookup tables for B = 8 at batch <= 8, decode +
+dot otherwise); integer-valued layers bit for bit; the same bits run to run for a
+given thread count; argument errors before any work.  No GPU is involved.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from weight_only_additive_b200 import build as lib_build
+from weight_only_additive_b200 import cpu, synth
+from weight_only_additive_b200.native import Status
+
+TOL = 5e-3
+SCHEMES = [(m, 8, g) for m in (1, 2, 3, 4) for g in (8, 16)] + [(m, 16, g) for m in (1, 2) for g in (8, 16)]
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "aqlm_cpu.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    lib_build.build_cpu()
+    cpu.lib()
+
+
+def close(y, ref, what):
+    assert np.isfinite(y.astype(np.float32)).all(), what
+    err = float(np.abs(y.astype(np.float64) - ref).max() / max(np.abs(ref).max(), 1e-30))
+    assert err <= TOL, f"{what}: rel err {err:.3e}"
+
+
+def test_header_declares_the_binding_exports():
+    text = open(HEADER).read()
+    declared = sorted(set(re.findall(r"\b(aqlm_cpu_\w+)\s*\(", text)))
+    assert declared == sorted(cpu.EXPORTS)
+    for name in cpu.EXPORTS:
+        assert isinstance(getattr(cpu.lib(), name), ctypes._CFuncPtr)
+    assert cpu.simd_level() in (0, 1)
+
+
+@pytest.mark.parametrize("M,B,g", SCHEMES)
+@pytest.mark.parametrize("batch", [1, 3, 8, 9])
+def test_cpu_matmul_matches_oracle(M, B, g, batch):
+    N, K = 150, 16 * 37  # several table slices and a partial one; ragged rows
+    ld = synth.make_layer(M, B, g, K, N, seed=80, layer=batch, with_bias=batch % 2 == 1)
+    x = synth.make_x(batch, K, seed=81, layer=M)
+    ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+    for nt in (1, 4):
+        close(cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g, nthreads=nt), ref,
+              f"{M}x{B} g{g} b={batch} threads={nt}")
+
+
+@pytest.mark.parametrize("M,B,g", SCHEMES)
+@pytest.mark.parametrize("batch", [1, 20])
+def test_cpu_matmul_integer_layers_bit_exact(M, B, g, batch):
+    N, K = 70, 512
+    rng = np.random.Generator(np.random.PCG64(82 + M + g + B))
+    cb = rng.integers(-2, 3, size=(M, 1 << B, g)).astype(np.float16)
+    codes = rng.integers(0, 1 << B, size=(N, K // g, M)).astype(np.uint8 if B <= 8 else np.uint16)
+    sc = rng.choice(np.array([1.0, 2.0]), size=N).astype(np.float16)
+    bias = rng.integers(-3, 4, size=N).astype(np.float16)
+    x = rng.integers(-1, 2, size=(batch, K)).astype(np.float16)
+    ref = oracle.linear(x, codes, cb, sc, bias, M, B, g)
+    assert np.abs(ref).max() <= 2048
+    for nt in (1, 3):
+        y = cpu.matmul(x, codes, cb, sc, bias, M, B, g, nthreads=nt).astype(np.float64)
+        assert np.array_equal(y, ref), (nt, int((y != ref).sum()))
+
+
+def test_cpu_matmul_full_size_layer_sampled_rows():
+    """A Llama-2-7B down_proj-shaped layer (4096 x 11008), 2x8 g8, batch 1."""
+    ld = synth.make_layer(2, 8, 8, 11008, 4096, seed=83)
+    x = synth.make_x(1, 11008, seed=83)
+    y = cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, None, 2, 8, 8)
+    rows = np.random.Generator(np.random.PCG64(84)).choice(4096, size=64, replace=False)
+    ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, 2, 8, 8, rows=rows)
+    close(y[:, rows], ref, "4096x11008 2x8 g8")
+
+
+def test_cpu_matmul_deterministic_for_a_thread_count():
+    ld = synth.make_layer(2, 8, 8, 4096, 512, seed=85)
+    x = synth.make_x(2, 4096, seed=85)
+    a = cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, None, 2, 8, 8, nthreads=4)
+    b = cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, None, 2, 8, 8, nthreads=4)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+def test_cpu_matmul_special_values():
+    """fp16 rounding of the output: zero codebooks leave the bias (a +0 sum plus a
+    -0 bias is +0, as in the oracle's fp64 sum), subnormal and large values pass
+    through, and an overflowing sum becomes +inf."""
+    M, B, g, K, N = 1, 8, 8, 64, 8
+    cb = np.zeros((M, 256, g), np.float16)
+    codes = np.zeros((N, K // g, M), np.uint8)
+    sc = np.ones(N, np.float16)
+    bias = np.array([-0.0, 0.0, 6e-8, -6e-8, 1e-5, 60000, -60000, 1], np.float16)
+    x = np.ones((1, K), np.float16)
+    y = cpu.matmul(x, codes, cb, sc, bias, M, B, g)
+    ref = oracle.linear(x, codes, cb, sc, bias, M, B, g).astype(np.float16)
+    assert np.array_equal(y.view(np.uint16), ref.view(np.uint16))
+    assert y[0, 0].view(np.uint16) == 0  # +0
+    cb[0, 0, :] = 60000
+    y = cpu.matmul(np.ones((1, K), np.float16), codes, cb, sc, None, M, B, g)
+    assert np.isinf(y).all() and (y > 0).all()
+
+
+@pytest.mark.parametrize("kwargs,want", [
+    (dict(M=5), Status.UNSUPPORTED),
+    (dict(g=4), Status.UNSUPPORTED),
+    (dict(nthreads=-1), Status.INVALID_ARG),
+])
+def test_cpu_matmul_argument_errors(kwargs, want):
+    M, B, g = kwargs.get("M", 2), 8, kwargs.get("g", 8)
+    lib = cpu.lib()
+    x = np.zeros((1, 64), np.float16)
+    codes = np.zeros((4, 64 // 8, 2), np.uint8)
+    cb = np.zeros((2, 256, 8), np.float16)
+    sc = np.ones(4, np.float16)
+    y = np.zeros((1, 4), np.float16)
+    st = lib.aqlm_cpu_matmul(x.ctypes.data, codes.ctypes.data, cb.ctypes.data, sc.ctypes.data, None,
+                             y.ctypes.data, M, B, g, 64, 4, 1, kwargs.get("nthreads", 0))
+    assert st == want
+    # output overlapping an input, misaligned fp16 pointer, NULL input
+    assert lib.aqlm_cpu_matmul(x.ctypes.data, codes.ctypes.data, cb.ctypes.data, sc.ctypes.data, None,
+                               x.ctypes.data, 2, 8, 8, 64, 4, 1, 0) == Status.INVALID_ARG
+    assert lib.aqlm_cpu_matmul(x.ctypes.data + 1, codes.ctypes.data, cb.ctypes.data, sc.ctypes.data, None,
+                               y.ctypes.data, 2, 8, 8, 64, 4, 1, 0) == Status.MISALIGNED
+    assert lib.aqlm_cpu_matmul(None, codes.ctypes.data, cb.ctypes.data, sc.ctypes.data, None,
+                               y.ctypes.data, 2, 8, 8, 64, 4, 1, 0) == Status.INVALID_ARG
