@@ -42,9 +42,21 @@ namespace {
 
 constexpr int kRows = 128;            // MMA M: weight rows per CTA
 constexpr int kStageK = 64;           // K per stage (one 128-byte swizzle row of fp16)
-constexpr int kDecoders = 256;        // warps 0-7: two threads per weight row
-constexpr int kThreads = 352;         // + x producer, MMA issuer, code producer
-constexpr int kWarpX = 8, kWarpMma = 9, kWarpCodes = 10;
+constexpr int kGroupThreads = 256;    // a decoder group: 8 warps, two threads per weight row of a stage
+constexpr int kMaxDecoderGroups = 2;
+
+// Decoder groups per CTA.  With two, group g decodes the stages i = g mod 2 of the
+// CTA's range, so two stages are decoded at once (latency hiding: measured 1.1-1.2x
+// on the B = 8 layer kernels and 1.55x on the input gradient at large batch).  The
+// codeword-gather decoders of the B = 16 layer kernels already keep L1TEX busy with
+// one group (a second made them 2-7 % slower), and 4x8 g8 ran faster with one.
+// Block: the decoder warps, then the x producer, the MMA issuer and the code producer.
+template <int M, int B, int G, bool kGrad>
+struct PipeShape {
+  static constexpr int kGroups = (!kGrad && (B == 16 || (M == 4 && G == 8))) ? 1 : kMaxDecoderGroups;
+  static constexpr int kDecoders = kGroups * kGroupThreads;
+  static constexpr int kThreads = kDecoders + 96;
+};
 constexpr uint32_t kABytes = kRows * 128u;   // 16 KB per A stage
 constexpr int kCodeSlots = 4;
 constexpr uint32_t kSmemLimit = 227u * 1024u;
@@ -84,6 +96,8 @@ struct PipeScheme {
   static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;
   static constexpr int kSplitAlign = 16 / gcd_int(16, kStageCodeBytes);  // split starts: 16-byte code offsets
   static_assert(kTileRowBytes % kStageCodeBytes == 0 && kTileRowBytes % 16 == 0, "code tile rows");
+  // every full code tile holds stages of both decoder groups
+  static_assert(kStagesPerTile % kMaxDecoderGroups == 0, "stages per code tile");
   // a decoder thread reads half a stage of codes: inside one 16-byte chunk when swizzled
   static_assert(kStageCodeBytes % 2 == 0 && (!kSwizzle64 || 16 % (kStageCodeBytes / 2) == 0), "code halves");
 };
@@ -397,9 +411,13 @@ __device__ __forceinline__ void cluster_barrier() {
 // kGrad = true:  dx = dy . W16 (rows = K input features, reduction over the N
 //                output rows; x_map then describes dy [batch, N]).
 template <int M, int B, int G, bool kGrad>
-__global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_constant__ CUtensorMap x_map,
-                                                              const __grid_constant__ CUtensorMap code_map,
-                                                              const PipeParams p) {
+__global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
+    tc_pipe_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap code_map,
+                   const PipeParams p) {
+  constexpr int kDecoderGroups = PipeShape<M, B, G, kGrad>::kGroups;
+  constexpr int kDecoders = PipeShape<M, B, G, kGrad>::kDecoders;
+  constexpr int kThreads = PipeShape<M, B, G, kGrad>::kThreads;
+  constexpr int kWarpX = kDecoders / 32, kWarpMma = kWarpX + 1, kWarpCodes = kWarpX + 2;
   extern __shared__ uint8_t smem_raw[];
   // stages must be 1024-byte aligned for the 128-byte swizzle
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -436,12 +454,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
   grid_dependents_launch();
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], kDecoders + 1);
+      mbar_init(&full[i], kGroupThreads + 1);  // the group that decodes the stage + the x tile
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < kCodeSlots; ++i) {
       mbar_init(&cfull[i], 1);
-      mbar_init(&cempty[i], kDecoders / 32);
+      // every decoder warp that reads the tile: both groups when a tile holds several
+      // stages (the final, partial tile may see one group only: its slot is not reused)
+      mbar_init(&cempty[i], (kStagesPerTile >= kDecoderGroups ? kDecoders : kGroupThreads) / 32);
     }
     mbar_init(acc_bar, 1);
     *abort_flag = 0u;
@@ -524,7 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     // lane % 4) decodes features 32 qq .. 32 qq + 31 of row (ks0 + i) 64 + nl at
     // stage i, scaled by that row's s_n.  A warp reads 8 rows x 4 quarters of codes
     // (contiguous bytes) and its 32 chunk stores cover every bank group 4 times.
-    const int nl = 8 * warp + (lane >> 2);
+    const int grp = warp / (kGroupThreads / 32);
+    const int nl = 8 * (warp % (kGroupThreads / 32)) + (lane >> 2);
     const int qq = lane & 3;
     const uint32_t code_off = static_cast<uint32_t>(nl * SC::kBoxBytes + ((n0 * SC::kTileCodeBytes / kRows) & 15) +
                                                     qq * (SC::kTileCodeBytes / 4));
@@ -534,12 +555,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
       uint4 st[kLook + 1][M][4];
       float sv[kLook + 1];
       bool alive = true;
-      for (int base = 0; alive && base < nks + kLook; base += kLook + 1) {
+      const int nmine = (nks - grp + kDecoderGroups - 1) / kDecoderGroups;  // this group's stages
+      for (int base = 0; alive && base < nmine + kLook; base += kLook + 1) {
 #pragma unroll
         for (int u = 0; u <= kLook; ++u) {
-          const int i = base + u;      // stage gathered now
-          const int j = i - kLook;     // stage stored now
-          const bool issue = i < nks, store = j >= 0 && j < nks;
+          const int ki = base + u, kj = ki - kLook;   // this group's stage numbers
+          const int i = grp + kDecoderGroups * ki;    // stage gathered now
+          const int j = grp + kDecoderGroups * kj;    // stage stored now
+          const bool issue = ki < nmine, store = kj >= 0 && kj < nmine;
           const int c = i % kCodeSlots;
           const int sj = j >= 0 ? j % S : 0, uj = j >= 0 ? j / S : 0;
           bool ready = true;
@@ -582,8 +605,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
       }
     } else {
       // B = 8: codebooks in shared memory; the next stage's scale is loaded one stage ahead
-      float s_next = (nks > 0 && ks0 * kStageK + nl < p.N) ? __half2float(p.scales[ks0 * kStageK + nl]) : 0.f;
-      for (int i = 0; i < nks; ++i) {
+      const int n_first = (ks0 + grp) * kStageK + nl;
+      float s_next = (grp < nks && n_first < p.N) ? __half2float(p.scales[n_first]) : 0.f;
+      for (int i = grp; i < nks; i += kDecoderGroups) {
         const int c = i % kCodeSlots;
         bool ready = pipe_wait(&cfull[c], static_cast<uint32_t>((i / kCodeSlots) & 1), abort_flag, p.status,
                                kSitePipeCodes);
@@ -596,7 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
         }
         const int n = (ks0 + i) * kStageK + nl;
         const float sc = s_next;
-        if (i + 1 < nks) s_next = n + kStageK < p.N ? __half2float(p.scales[n + kStageK]) : 0.f;
+        const int n_next = n + kDecoderGroups * kStageK;
+        if (i + kDecoderGroups < nks) s_next = n_next < p.N ? __half2float(p.scales[n_next]) : 0.f;
         decode_grad_b8<M, G>(smem, L.a + static_cast<uint32_t>(s) * kABytes, nl, qq, n < p.N,
                              smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, smem + L.cb, sc);
         fence_proxy_async_smem();
@@ -608,7 +633,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
     } else {
     // ---- decoders: threads r and r + 128 share weight row n0 + r (chunks 0-3 / 4-7) ----
     const int r = tid & (kRows - 1);
-    const int hf = tid >> 7;
+    const int hf = kDecoderGroups == 1 ? tid >> 7 : (tid >> 7) & 1;
+    const int grp = kDecoderGroups == 1 ? 0 : tid / kGroupThreads;
     const bool row_valid = n0 + r < p.N;
     if constexpr (B == 16 && !(M == 1 && G == 8)) {
       // B = 16 except 1x16 g8: register-staged gathers, kLook stages ahead.  At step i
@@ -620,17 +646,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
       constexpr int kLook = (M == 1) ? 3 : 1;
       uint4 st[kLook + 1][M][4];
       bool alive = true;
-      for (int base = 0; alive && base < nks + kLook; base += kLook + 1) {
+      const int nmine = (nks - grp + kDecoderGroups - 1) / kDecoderGroups;  // this group's stages
+      for (int base = 0; alive && base < nmine + kLook; base += kLook + 1) {
 #pragma unroll
         for (int u = 0; u <= kLook; ++u) {
-          const int i = base + u;      // stage gathered now
-          const int j = i - kLook;     // stage stored now
-          const bool issue = i < nks, store = j >= 0 && j < nks;
+          const int ki = base + u, kj = ki - kLook;   // this group's stage numbers
+          const int i = grp + kDecoderGroups * ki;    // stage gathered now
+          const int j = grp + kDecoderGroups * kj;    // stage stored now
+          const bool issue = ki < nmine, store = kj >= 0 && kj < nmine;
           const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
           const int sj = j >= 0 ? j % S : 0, uj = j >= 0 ? j / S : 0;
           // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
           bool ready = true;
-          if (issue && within == 0)
+          if (issue && within < kDecoderGroups)  // this group's first stage of the tile
             ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
                               kSitePipeCodes);
           if (ready && store && uj > 0)
@@ -645,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
                                 code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                     r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
             gather_stage_b16<M, G>(st[u], cw, row_valid, p.codebooks, p.cb32 != 0);
-            if (within == kStagesPerTile - 1 || i == nks - 1) {
+            if (within + kDecoderGroups >= kStagesPerTile || i + kDecoderGroups >= nks) {  // its last one
               __syncwarp();  // every lane has read its codes of this tile
               if (lane == 0) mbar_arrive(&cempty[c]);
             }
@@ -665,34 +693,69 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
         }
       }
     } else {
-    for (int i = 0; i < nks; ++i) {
-      const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
-      // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
-      bool ready = true;
-      if (within == 0)
-        ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
-                          kSitePipeCodes);
-      const int s = i % S, u = i / S;
-      if (ready && u > 0)
-        ready = pipe_wait(&empty[s], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
-      if (!__all_sync(0xffffffffu, ready)) {
-        *abort_flag = 1u;
-        break;
+    if constexpr (kDecoderGroups == 1) {
+      // one group: every stage in order (written without the group arithmetic:
+      // the compiler schedules this form measurably better for 4x8 g8)
+      for (int i = 0; i < nks; ++i) {
+        const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
+        // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
+        bool ready = true;
+        if (within == 0)
+          ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
+                            kSitePipeCodes);
+        const int s = i % S, u = i / S;
+        if (ready && u > 0)
+          ready = pipe_wait(&empty[s], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
+        if (!__all_sync(0xffffffffu, ready)) {
+          *abort_flag = 1u;
+          break;
+        }
+        const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
+                            code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
+                                r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
+        decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
+                                   p.codebooks, smem + L.cb);
+        if constexpr (B == 16) {
+          cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
+        } else {
+          fence_proxy_async_smem();
+          mbar_arrive(&full[s]);
+        }
+        if (within == kStagesPerTile - 1 || i == nks - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&cempty[c]);
+        }
       }
-      const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
-                          code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
-                              r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
-      decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
-                                 p.codebooks, smem + L.cb);
-      if constexpr (B == 16) {
-        cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
-      } else {
-        fence_proxy_async_smem();
-        mbar_arrive(&full[s]);
-      }
-      if (within == kStagesPerTile - 1 || i == nks - 1) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&cempty[c]);
+    } else {
+      for (int i = grp; i < nks; i += kDecoderGroups) {
+        const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
+        // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
+        bool ready = true;
+        if (within < kDecoderGroups)  // this group's first stage of the tile
+          ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
+                            kSitePipeCodes);
+        const int s = i % S, u = i / S;
+        if (ready && u > 0)
+          ready = pipe_wait(&empty[s], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
+        if (!__all_sync(0xffffffffu, ready)) {
+          *abort_flag = 1u;
+          break;
+        }
+        const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
+                            code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
+                                r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
+        decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
+                                   p.codebooks, smem + L.cb);
+        if constexpr (B == 16) {
+          cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
+        } else {
+          fence_proxy_async_smem();
+          mbar_arrive(&full[s]);
+        }
+        if (within + kDecoderGroups >= kStagesPerTile || i + kDecoderGroups >= nks) {  // its last one
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&cempty[c]);
+        }
       }
     }
     }
@@ -701,8 +764,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
   }
 
   // ---- epilogue ----------------------------------------------------------------------
-  // Decoder warp w reads TMEM lanes 32*(w % 4).. (weight rows) and, with its twin
-  // w +- 4, alternating 16-column chunks of the batch tile.
+  // Decoder warp w reads TMEM lanes 32*(w % 4).. (weight rows) and, with the other
+  // warps of its lane quadrant, every (kDecoders / 128)-th 16-column chunk of the batch tile.
   const bool decoder = warp < kDecoders / 32;
   const int q = warp & 3;        // TMEM lane quadrant
   const int cpar = warp >> 2;    // which 16-column chunks
@@ -718,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
       // the gradient's scale is inside its A operand and it has no bias
       const float sc = kGrad ? 1.f : (n_valid ? __half2float(p.scales[n]) : 0.f);
       const float bi = (!kGrad && n_valid && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
-      for (int c0 = 16 * cpar; c0 < p.BN; c0 += 32) {
+      for (int c0 = 16 * cpar; c0 < p.BN; c0 += 16 * (kDecoders / 128)) {
         float v[16];
         tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), v);
         if (n_valid) {
@@ -747,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pipe_kernel(const __grid_const
       const uint32_t slot_row = static_cast<uint32_t>(split * R + (r - static_cast<int>(owner) * R));
       const uint32_t remote_base =
           mapa_shared_cluster(sbase + L.a + slot_row * static_cast<uint32_t>(pitch) * 4u, owner);
-      for (int c0 = 16 * cpar; c0 < p.BN; c0 += 32) {
+      for (int c0 = 16 * cpar; c0 < p.BN; c0 += 16 * (kDecoders / 128)) {
         float v[16];
         tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), v);
 #pragma unroll
@@ -865,7 +928,7 @@ cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, TcPlan* out)
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = static_cast<unsigned>(SK);
       cfg.gridDim = dim3(1, 1, static_cast<unsigned>(SK));
-      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.blockDim = dim3(PipeShape<M, B, G, kGrad>::kThreads, 1, 1);
       cfg.dynamicSmemBytes = smem;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
@@ -955,7 +1018,7 @@ cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, si
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(row_tiles), static_cast<unsigned>(batch_tiles),
                      static_cast<unsigned>(plan.SK));
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(PipeShape<M, B, G, kGrad>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
