@@ -528,13 +528,14 @@ def run_ours(a):
                       for c in range(pool)]
 
         def e2e_step(c):
-            dx_flat.copy_(hx_flat, non_blocking=True)
             if mode == "group":
-                e2e_groups[c].run(stream=stream)
+                # one C-ABI call: H2D of every x, the group, D2H of every y
+                e2e_groups[c].run_host(hx_flat, hy_flat, stream=stream)
             else:
+                dx_flat.copy_(hx_flat, non_blocking=True)
                 for li in range(len(w.layers)):
                     L.matmul(dx[li], weights[c][li], out=dy[li], stream=stream)
-            hy_flat.copy_(dy_flat, non_blocking=True)
+                hy_flat.copy_(dy_flat, non_blocking=True)
 
         with torch.cuda.stream(stream):
             for i in range(3):
@@ -550,7 +551,8 @@ def run_ours(a):
             e1.record(stream)
         torch.cuda.synchronize(dev)
         ems = max_over_ranks(e0.elapsed_time(e1), dist, dev)
-        api = ("weight_only_additive_b200.layer.LayerGroup.run -> aqlm_matmul_group" if mode == "group"
+        api = ("weight_only_additive_b200.layer.LayerGroup.run_host -> aqlm_matmul_group_host (the copies "
+               "inside the call)" if mode == "group"
                else "weight_only_additive_b200.layer.matmul -> aqlm_matmul, per layer")
         e2e = {"value": job_throughput_gbs(sbytes, e2e_steps, world, ems), "unit": "GB/s",
                "h2d_bytes_per_step": hx_flat.numel() * 2,

@@ -197,6 +197,25 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
 #define AQLM_STATIC_GROUP_SCRATCH_BYTES (8u << 20)
 aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aqlm_stream_t stream);
 
+/*
+ * aqlm_matmul_group with the activations in HOST memory: on `stream`, copies
+ * x_host into the problems' device x buffers, runs the group, and copies every
+ * problem's y back into y_host.
+ *   x_host  fp16, the problems' x one after another in problem order
+ *           (problem i: batch_i * K_i values), read
+ *   y_host  fp16, the problems' y one after another (batch_i * N_i values), written
+ * When the device buffers of consecutive problems are contiguous (problem i + 1's x
+ * starts where problem i's ends, likewise y), one copy moves all of them; otherwise
+ * there is one copy per problem (cudaMemcpyAsync; pinned host buffers make the
+ * copies asynchronous).  The call returns after enqueueing: y_host is valid, and
+ * x_host may be modified, once `stream` has passed the call (synchronise before).  The pages have
+ * no counterpart: this is the token-generation step of a serving loop, from host
+ * activations to host outputs.  Validation, workspace and errors as for
+ * aqlm_matmul_group; NULL x_host or y_host (with count > 0) is AQLM_ERR_INVALID_ARG.
+ */
+aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, const void* x_host, void* y_host,
+                                   void* workspace, size_t workspace_bytes, aqlm_stream_t stream);
+
 /* Workspace bytes aqlm_matmul_group needs for these problems: for every run of
  * up to 16 grouped problems, the sum over them of ceil(K / 512) * N * 4 bytes
  * rounded up to 256; the maximum over runs.  Pure host logic. */

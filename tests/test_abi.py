@@ -223,3 +223,11 @@ def test_input_grad_rejects_bad_arguments_before_any_cuda_call(lib):
     with pytest.raises(native.AqlmError) as e:
         native.aqlm_input_grad(None, A, A, A, 1 << 34, 2, 8, 8, 1024, 64, 1)
     assert e.value.status == Status.INVALID_ARG
+
+
+def test_group_host_rejects_missing_host_buffers_without_a_gpu(lib):
+    L_ = native.lib()
+    probs = native.problem_array([_prob(1 << 32)])
+    assert L_.aqlm_matmul_group_host(probs, 1, None, A, A, 1 << 20, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_group_host(probs, 1, A, None, A, 1 << 20, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_group_host(probs, 0, None, None, None, 0, None) == Status.OK

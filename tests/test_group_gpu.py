@@ -173,3 +173,45 @@ def test_group_published_layer_sets_sampled_rows(dev, wname):
         y = item[2].cpu().numpy()
         assert np.isfinite(y.astype(np.float32)).all()
         assert_close(y[:, rows], y_ref, f"{wname}/{lay.name}")
+
+
+@pytest.mark.parametrize("packed,pinned", [(True, True), (False, True), (True, False)])
+def test_group_from_host_buffers(dev, packed, pinned):
+    """aqlm_matmul_group_host: x copied from one packed host buffer, y copied back into
+    one; with packed device buffers (one copy each way) and with separate ones (one
+    copy per problem); page-locked and pageable host buffers."""
+    # packed offsets stay 16-byte aligned: every batch * K and batch * N is a multiple of 8
+    specs = [(2, 8, 8, 4096, 1024, 1, False), (2, 8, 8, 11008, 512, 1, True), (1, 16, 8, 1024, 304, 1, False),
+             (2, 8, 8, 1024, 130, 4, False)]
+    lds, xs = [], []
+    for i, (M, B, g, K, N, batch, bias) in enumerate(specs):
+        lds.append(synth.make_layer(M, B, g, K, N, seed=46, layer=i, with_bias=bias))
+        xs.append(synth.make_x(batch, K, seed=46, layer=i))
+    nx = sum(x.size for x in xs)
+    ny = sum(batch * N for (_, _, _, _, N, batch, _) in specs)
+    if packed:
+        dxf = torch.empty(nx, dtype=torch.float16, device=dev)
+        dyf = torch.full((ny,), float("nan"), dtype=torch.float16, device=dev)
+        xo = np.cumsum([0] + [x.size for x in xs])
+        yo = np.cumsum([0] + [batch * N for (_, _, _, _, N, batch, _) in specs])
+        dx = [dxf[xo[i]:xo[i + 1]].view(xs[i].shape) for i in range(len(specs))]
+        dy = [dyf[yo[i]:yo[i + 1]].view(specs[i][5], specs[i][4]) for i in range(len(specs))]
+    else:
+        dx = [torch.empty(x.shape, dtype=torch.float16, device=dev) for x in xs]
+        dy = [torch.full((s[5], s[4]), float("nan"), dtype=torch.float16, device=dev) for s in specs]
+    items = [(L.AqlmWeights.from_numpy(ld, dev), dx[i], dy[i]) for i, ld in enumerate(lds)]
+    grp = L.LayerGroup(items)
+    hx = torch.from_numpy(np.concatenate([x.reshape(-1) for x in xs]))
+    hy = torch.full((ny,), float("nan"), dtype=torch.float16)
+    if pinned:
+        hx, hy = hx.pin_memory(), hy.pin_memory()
+    s = torch.cuda.Stream(dev)
+    for rep in range(3):  # back to back on one stream
+        grp.run_host(hx, hy, stream=s)
+    s.synchronize()
+    check_status()
+    off = 0
+    for (M, B, g, K, N, batch, _), ld, x in zip(specs, lds, xs):
+        y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+        assert_close(hy[off:off + batch * N].numpy().reshape(batch, N), y_ref, f"host group K={K} N={N} b={batch}")
+        off += batch * N

@@ -111,7 +111,7 @@ EncodeTiledFn encode_tiled() {
 
 extern "C" {
 
-int aqlm_abi_version(void) { return 5; }
+int aqlm_abi_version(void) { return 6; }
 
 const char* aqlm_status_string(aqlm_status status) {
   switch (status) {
@@ -334,6 +334,49 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
     }
   }
   return AQLM_OK;
+}
+
+aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, const void* x_host, void* y_host,
+                                   void* workspace, size_t workspace_bytes, aqlm_stream_t stream) {
+  if (count == 0) return AQLM_OK;
+  if (count < 0 || !problems || !x_host || !y_host) return AQLM_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const aqlm_problem& q = problems[i];
+    const aqlm_status st = aqlm_validate(q.x, q.codes, q.codebooks, q.scales, q.bias, q.y, q.M, q.B, q.g, q.K,
+                                         q.N, q.batch, AQLM_PATH_AUTO);
+    if (st != AQLM_OK) return st;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const auto xbytes = [&](int i) { return static_cast<size_t>(problems[i].batch) * problems[i].K * 2; };
+  const auto ybytes = [&](int i) { return static_cast<size_t>(problems[i].batch) * problems[i].N * 2; };
+  // one copy per maximal run of problems whose device buffers are contiguous
+  const auto copy_runs = [&](bool in) -> aqlm_status {
+    size_t off = 0;
+    for (int i = 0; i < count;) {
+      const auto bytes = [&](int k) { return in ? xbytes(k) : ybytes(k); };
+      const auto dptr = [&](int k) {
+        return in ? static_cast<uint8_t*>(const_cast<void*>(problems[k].x)) : static_cast<uint8_t*>(problems[k].y);
+      };
+      int j = i;
+      size_t run = bytes(i);
+      while (j + 1 < count && dptr(j + 1) == dptr(i) + run) {
+        ++j;
+        run += bytes(j);
+      }
+      const aqlm_status st = from_cuda(
+          in ? cudaMemcpyAsync(dptr(i), static_cast<const uint8_t*>(x_host) + off, run, cudaMemcpyHostToDevice, s)
+             : cudaMemcpyAsync(static_cast<uint8_t*>(y_host) + off, dptr(i), run, cudaMemcpyDeviceToHost, s));
+      if (st != AQLM_OK) return st;
+      off += run;
+      i = j + 1;
+    }
+    return AQLM_OK;
+  };
+  aqlm_status st = copy_runs(true);
+  if (st != AQLM_OK) return st;
+  st = aqlm_matmul_group(problems, count, workspace, workspace_bytes, stream);
+  if (st != AQLM_OK) return st;
+  return copy_runs(false);
 }
 
 aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aqlm_stream_t stream) {

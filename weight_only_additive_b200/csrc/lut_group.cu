@@ -37,6 +37,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "aqlm_device.cuh"
 
@@ -497,15 +498,56 @@ size_t lut_group_workspace_bytes(const Problem* probs, int count) {
   return bytes;
 }
 
-// All problems must satisfy lut_group_supported; count <= kMaxGroupLayers; the
-// workspace holds lut_group_workspace_bytes(probs, count) bytes, 256-byte aligned.
-cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, uint32_t* status,
-                             cudaStream_t stream) {
-  if (count <= 0 || count > kMaxGroupLayers) return cudaErrorInvalidValue;
+namespace {
+
+// Everything a launch pair needs besides the stream: built once per distinct call
+// (problem list, workspace, status word, device) and kept in a small cache, so a
+// call repeated every token (the usual case: the same layer set with new x and y
+// contents) skips the tensor-map encoding and the per-layer bookkeeping.
+struct GroupLaunch {
+  GroupParams p;
+  GroupMaps maps;
+  unsigned grid = 0, rgrid = 0;
+};
+
+struct GroupKey {
+  int dev = -1, count = 0;
+  const void* workspace = nullptr;
+  const uint32_t* status = nullptr;
+  Problem probs[kMaxGroupLayers];
+};
+
+bool same_problem(const Problem& a, const Problem& b) {
+  return a.x == b.x && a.codes == b.codes && a.codebooks == b.codebooks && a.scales == b.scales &&
+         a.bias == b.bias && a.y == b.y && a.M == b.M && a.B == b.B && a.g == b.g && a.K == b.K && a.N == b.N &&
+         a.batch == b.batch;
+}
+
+bool same_key(const GroupKey& k, int dev, const Problem* probs, int count, const void* ws, const uint32_t* status) {
+  if (k.dev != dev || k.count != count || k.workspace != ws || k.status != status) return false;
+  for (int i = 0; i < count; ++i)
+    if (!same_problem(k.probs[i], probs[i])) return false;
+  return true;
+}
+
+constexpr int kLaunchCacheEntries = 8;
+constexpr int kMaxDevices = 64;
+std::mutex g_launch_mu;
+GroupKey g_launch_key[kLaunchCacheEntries];
+GroupLaunch g_launch_val[kLaunchCacheEntries];
+int g_launch_next = 0;
+int g_sms[kMaxDevices] = {};  // 0 = not queried yet (also means "attribute not set")
+
+// Tensor maps and parameters of one launch pair (host work only, no CUDA calls but
+// the driver's tensor-map encoder).
+cudaError_t build_group_launch(const Problem* probs, int count, void* workspace, uint32_t* status, int sms,
+                               GroupLaunch* out) {
   EncodeTiledFn encode = encode_tiled();
   if (!encode) return cudaErrorNotSupported;
-  GroupParams p{};
-  GroupMaps maps{};
+  GroupParams& p = out->p;
+  GroupMaps& maps = out->maps;
+  p = GroupParams{};
+  maps = GroupMaps{};
   long long items = 0, rows = 0;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   for (int i = 0; i < count; ++i) {
@@ -541,37 +583,74 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
   p.items = items;
   p.rows = rows;
   p.status = status;
+  out->grid = static_cast<unsigned>(std::min<long long>(items, sms));
+  out->rgrid = static_cast<unsigned>((rows + kReduceRows - 1) / kReduceRows);
+  return cudaSuccess;
+}
 
-  int dev = 0, sms = 148;
+}  // namespace
+
+// All problems must satisfy lut_group_supported; count <= kMaxGroupLayers; the
+// workspace holds lut_group_workspace_bytes(probs, count) bytes, 256-byte aligned.
+cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, uint32_t* status,
+                             cudaStream_t stream) {
+  if (count <= 0 || count > kMaxGroupLayers) return cudaErrorInvalidValue;
+  int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaGetLastError();
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   const uint32_t smem = kSmemBytes + 1024u;
-  auto kern = lut_group_kernel;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  GroupLaunch launch;
+  {
+    std::lock_guard<std::mutex> lock(g_launch_mu);
+    if (g_sms[dev] == 0) {
+      // once per device: the SM count and the kernel's shared-memory limit
+      int sms = 0;
+      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(lut_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      g_sms[dev] = std::max(1, sms);
+    }
+    int hit = -1;
+    for (int c = 0; c < kLaunchCacheEntries && hit < 0; ++c)
+      if (same_key(g_launch_key[c], dev, probs, count, workspace, status)) hit = c;
+    if (hit < 0) {
+      hit = g_launch_next;
+      g_launch_next = (g_launch_next + 1) % kLaunchCacheEntries;
+      g_launch_key[hit].dev = -1;  // invalid until built
+      e = build_group_launch(probs, count, workspace, status, g_sms[dev], &g_launch_val[hit]);
+      if (e != cudaSuccess) return e;
+      GroupKey& k = g_launch_key[hit];
+      k.dev = dev;
+      k.count = count;
+      k.workspace = workspace;
+      k.status = status;
+      for (int i = 0; i < count; ++i) k.probs[i] = probs[i];
+    }
+    launch = g_launch_val[hit];
+  }
 
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(std::min<long long>(items, sms)), 1, 1);
+  cfg.gridDim = dim3(launch.grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, maps, p);
+  e = cudaLaunchKernelEx(&cfg, lut_group_kernel, launch.maps, launch.p);
   if (e != cudaSuccess) return e;
 
   cudaLaunchConfig_t rcfg = {};
-  rcfg.gridDim = dim3(static_cast<unsigned>((rows + kReduceRows - 1) / kReduceRows), 1, 1);
+  rcfg.gridDim = dim3(launch.rgrid, 1, 1);
   rcfg.blockDim = dim3(kReduceRows * kReduceLanes, 1, 1);
   rcfg.stream = stream;
   rcfg.attrs = attr;
   rcfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&rcfg, lut_group_reduce_kernel, p);
+  return cudaLaunchKernelEx(&rcfg, lut_group_reduce_kernel, launch.p);
 }
 
 }  // namespace aqlm

@@ -152,3 +152,16 @@ class LayerGroup:
     def run(self, stream: Optional[torch.cuda.Stream] = None):
         native.aqlm_matmul_group(self.problems, self.workspace.data_ptr(), self.workspace_bytes,
                                  _stream_handle(stream, self.device), count=self.count)
+
+    def run_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
+        """One step from host activations to host outputs: x_host holds every layer's x
+        one after another (fp16, CPU, ideally pinned), y_host receives every y; the
+        copies and the group run on `stream` (aqlm_matmul_group_host).  Synchronise the
+        stream before reading y_host."""
+        nx = sum(int(x.numel()) for _, x, _ in self._keep)
+        ny = sum(int(o.numel()) for _, _, o in self._keep)
+        for t, n, name in ((x_host, nx, "x_host"), (y_host, ny, "y_host")):
+            if t.device.type != "cpu" or t.dtype != torch.float16 or not t.is_contiguous() or t.numel() != n:
+                raise ValueError(f"{name} must be a contiguous CPU fp16 tensor of {n} values")
+        native.aqlm_matmul_group_host(self.problems, x_host.data_ptr(), y_host.data_ptr(), self.workspace.data_ptr(),
+                                      self.workspace_bytes, _stream_handle(stream, self.device), count=self.count)

@@ -19,9 +19,9 @@ EXPORTS = ("aqlm_matmul", "aqlm_matmul_path", "aqlm_dequantize", "aqlm_select_pa
            "aqlm_validate", "aqlm_status_string", "aqlm_check_device_status",
            "aqlm_last_cuda_error", "aqlm_abi_version", "aqlm_matmul_group",
            "aqlm_group_workspace_size", "aqlm_matmul_group_static", "aqlm_selftest_bounded_wait",
-           "aqlm_input_grad", "aqlm_validate_input_grad")
+           "aqlm_input_grad", "aqlm_validate_input_grad", "aqlm_matmul_group_host")
 
-ABI_VERSION = 5
+ABI_VERSION = 6
 
 # Site code aqlm_selftest_bounded_wait records in the device status word.
 SITE_SELFTEST = 0x501
@@ -107,6 +107,9 @@ def lib() -> ctypes.CDLL:
                 L.aqlm_group_workspace_size.argtypes = [ctypes.POINTER(AqlmProblem), _i]
                 L.aqlm_group_workspace_size.restype = ctypes.c_size_t
                 L.aqlm_matmul_group_static.argtypes = [ctypes.POINTER(AqlmProblem), _i, _vp]
+                L.aqlm_matmul_group_host.argtypes = [ctypes.POINTER(AqlmProblem), _i, _vp, _vp, _vp,
+                                                     ctypes.c_size_t, _vp]
+                L.aqlm_matmul_group_host.restype = _i
                 L.aqlm_matmul_group_static.restype = _i
                 L.aqlm_selftest_bounded_wait.argtypes = [ctypes.c_uint, _vp]
                 L.aqlm_selftest_bounded_wait.restype = _i
@@ -194,6 +197,14 @@ def aqlm_matmul_group_static(problems, stream=None, count=None):
     arr = problems if isinstance(problems, ctypes.Array) else problem_array(problems)
     n = len(problems) if count is None else count
     _check(lib().aqlm_matmul_group_static(arr, n, stream), "aqlm_matmul_group_static")
+
+
+def aqlm_matmul_group_host(problems, x_host, y_host, workspace, workspace_bytes, stream=None, count=None):
+    """Group call from packed host x to packed host y (pointers; pinned for async copies)."""
+    arr = problems if isinstance(problems, ctypes.Array) else problem_array(problems)
+    n = len(problems) if count is None else count
+    _check(lib().aqlm_matmul_group_host(arr, n, x_host, y_host, workspace, workspace_bytes, stream),
+           "aqlm_matmul_group_host")
 
 
 def aqlm_selftest_bounded_wait(timeout_us: int, stream=None):
