@@ -76,6 +76,8 @@ def parse_args(argv=None):
                    help="skip the extra per-layer timing that the group mode reports beside its headline")
     p.add_argument("--launch", choices=("group", "per-layer"), default="group",
                    help="one aqlm_matmul_group call per step (default) or one aqlm_matmul call per layer")
+    p.add_argument("--scheme", default=None,
+                   help="replace every layer's codebook scheme (MxBgG, e.g. 4x8g8): the generic shapes")
     p.add_argument("--op", choices=("matmul", "input-grad"), default="matmul",
                    help="the layer (default) or its input gradient dx = dy . diag(s) . W")
     p.add_argument("--pool", type=int, default=None,
@@ -134,9 +136,23 @@ def workload_batch(w, override):
     return override if override is not None else w.batches[0]
 
 
+def parse_scheme(text):
+    """'MxBgG' (e.g. 4x8g8, 2x16g16) -> workloads.Scheme."""
+    import re
+    m = re.fullmatch(r"(\d+)x(\d+)g(\d+)", text or "")
+    if not m:
+        raise SystemExit(f"--scheme {text!r}: expected MxBgG, e.g. 4x8g8")
+    return workloads.Scheme(int(m.group(1)), int(m.group(2)), int(m.group(3)))
+
+
 def select_workload(a):
-    """The named workload, restricted to one layer when --layer is given."""
+    """The named workload, restricted to one layer when --layer is given, with every
+    layer's codebook scheme replaced when --scheme is given."""
     w = workloads.get(a.workload)
+    if getattr(a, "scheme", None):
+        sch = parse_scheme(a.scheme)
+        layers = tuple(workloads.Layer(l.name, l.N, l.K, sch) for l in w.layers)
+        w = workloads.Workload(w.index, f"{w.name}@{sch.name}", layers, w.batches, w.description)
     if a.layer is None:
         return w
     layers = tuple(l for l in w.layers if l.name == a.layer)
