@@ -428,8 +428,8 @@ def run_ours(a):
         reduction) per run of up to 16; every other layer one."""
         if mode == "per-layer":
             return len(w.layers)
-        grouped = sum(1 for l in w.layers if l.scheme.M == 2 and l.scheme.B == 8 and l.scheme.g == 8
-                      and batch == 1 and l.K % 64 == 0)
+        grouped = sum(1 for l in w.layers if l.scheme.B == 8 and batch == 1 and l.K % l.scheme.g == 0
+                      and (l.K // l.scheme.g * l.scheme.M) % 16 == 0)
         return 2 * ((grouped + 15) // 16) + (len(w.layers) - grouped)
 
     def barrier():

@@ -163,9 +163,10 @@ typedef struct {
  * definition and tolerance).  The problems must be independent: no y_i may
  * overlap another problem's x, y, codes, codebooks, scales or bias (overlapping
  * outputs and inputs are rejected with AQLM_ERR_INVALID_ARG as far as the
- * pointer ranges show).  2x8 g8 batch-1 problems with K % 64 == 0 are computed
- * together, up to 16 per launch pair (a partial-sum kernel and a reduction); the
- * others are launched one after another as by aqlm_matmul.  Both kernels of a
+ * pointer ranges show).  Batch-1 problems with 256-entry codebooks (B = 8, any M
+ * and g above) whose code rows (K / g * M bytes) are whole 16-byte units are
+ * computed together, up to 16 per launch pair (a partial-sum kernel and a
+ * reduction); the others are launched one after another as by aqlm_matmul.  Both kernels of a
  * pair keep the stream-ordering contract above.
  *
  * workspace: caller-owned DEVICE memory of at least
@@ -217,8 +218,9 @@ aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, cons
                                    void* workspace, size_t workspace_bytes, aqlm_stream_t stream);
 
 /* Workspace bytes aqlm_matmul_group needs for these problems: for every run of
- * up to 16 grouped problems, the sum over them of ceil(K / 512) * N * 4 bytes
- * rounded up to 256; the maximum over runs.  Pure host logic. */
+ * up to 16 grouped problems, the sum over them of ceil(K / g * M / 128) * N * 4
+ * bytes (one fp32 partial per row and 128 code bytes) rounded up to 256; the
+ * maximum over runs.  Pure host logic. */
 size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count);
 
 /* The kernel family AQLM_PATH_AUTO picks for this problem, or -1 if unsupported.

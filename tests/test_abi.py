@@ -231,3 +231,13 @@ def test_group_host_rejects_missing_host_buffers_without_a_gpu(lib):
     assert L_.aqlm_matmul_group_host(probs, 1, None, A, A, 1 << 20, None) == Status.INVALID_ARG
     assert L_.aqlm_matmul_group_host(probs, 1, A, None, A, 1 << 20, None) == Status.INVALID_ARG
     assert L_.aqlm_matmul_group_host(probs, 0, None, None, None, 0, None) == Status.OK
+
+
+@pytest.mark.parametrize("M,g,K", [(1, 8, 4096), (3, 8, 1024), (4, 16, 4096), (1, 16, 4096)])
+def test_group_workspace_size_generic_schemes(lib, M, g, K):
+    """Grouped B = 8 layers of any scheme: one fp32 partial per row and 128-code-byte
+    slice, rounded up to 256 bytes."""
+    N = 300
+    probs = native.problem_array([_prob(1 << 32, M=M, B=8, g=g, K=K, N=N)])
+    slices = (K // g * M + 127) // 128
+    assert native.aqlm_group_workspace_size(probs, 1) == (slices * N * 4 + 255) // 256 * 256

@@ -215,3 +215,84 @@ def test_group_from_host_buffers(dev, packed, pinned):
         y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
         assert_close(hy[off:off + batch * N].numpy().reshape(batch, N), y_ref, f"host group K={K} N={N} b={batch}")
         off += batch * N
+
+
+GENERIC = [
+    (1, 8, 8, 4096, 1000, 1, False),    # 1 bit: 512-byte code rows, 4 slices
+    (1, 8, 16, 4096, 520, 1, True),     # 0.5 bit: 256-byte rows, 2 slices
+    (2, 8, 16, 2048, 300, 1, False),    # 1 bit
+    (3, 8, 8, 1024, 257, 1, True),      # 3 bit: groups straddle the 128-byte slices
+    (3, 8, 16, 2048, 130, 1, False),    # 1.5 bit
+    (4, 8, 8, 1024, 64, 1, True),       # 4 bit: two MMA rounds per table
+    (4, 8, 16, 4096, 200, 1, False),
+    (2, 8, 8, 1024, 129, 1, True),      # the tuned 2x8 g8 path in the same launch
+]
+
+
+def test_group_generic_schemes_match_oracle(dev):
+    """Every B = 8 scheme as grouped lookup-table layers, several in one launch (with
+    four-codebook layers present the launch uses the four-codebook layout)."""
+    grp, lds, xs, outs = build_group(GENERIC, dev, seed=47)
+    grp.run()
+    check_status()
+    for (M, B, g, K, N, batch, _), ld, x, out in zip(GENERIC, lds, xs, outs):
+        y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+        assert_close(out.cpu().numpy(), y_ref, f"group {M}x{B}g{g} K={K} N={N}")
+
+
+@pytest.mark.parametrize("M,g", [(1, 8), (1, 16), (2, 16), (3, 8), (3, 16), (4, 8), (4, 16)])
+def test_group_generic_scheme_alone(dev, M, g):
+    """One scheme per launch (the two-codebook layout for M <= 2), ragged rows."""
+    spec = [(M, 8, g, 2048, 333, 1, True), (M, 8, g, 1024, 64, 1, False)]
+    grp, lds, xs, outs = build_group(spec, dev, seed=48 + M + g)
+    grp.run()
+    check_status()
+    for (M_, B, g_, K, N, batch, _), ld, x, out in zip(spec, lds, xs, outs):
+        y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M_, B, g_)
+        assert_close(out.cpu().numpy(), y_ref, f"{M_}x{B}g{g_} K={K} N={N}")
+
+
+@pytest.mark.parametrize("M,g", [(1, 8), (3, 8), (4, 16)])
+def test_group_generic_integer_layers_bit_exact(dev, M, g):
+    """Small-integer codebooks and x: every table entry, half2 sum and fp32 partial is
+    an exact integer, so y equals the oracle bit for bit."""
+    rng = np.random.Generator(np.random.PCG64(49 + M + g))
+    items, refs = [], []
+    for N, K in ((260, 1024), (70, 2048)):
+        cb = rng.integers(-2, 3, size=(M, 256, g)).astype(np.float16)
+        codes = rng.integers(0, 256, size=(N, K // g, M)).astype(np.uint8)
+        sc = rng.choice(np.array([1.0, 2.0]), size=N).astype(np.float16)
+        bias = rng.integers(-3, 4, size=N).astype(np.float16)
+        x = rng.integers(-1, 2, size=(1, K)).astype(np.float16)
+        y_ref = oracle.linear(x, codes, cb, sc, bias, M, 8, g)
+        assert np.abs(y_ref).max() <= 2048 and np.array_equal(y_ref, np.round(y_ref))
+        w = L.AqlmWeights.from_numpy(synth.LayerData(M, 8, g, K, N, codes, cb, sc, bias), dev)
+        items.append((w, torch.from_numpy(x).to(dev), torch.empty((1, N), dtype=torch.float16, device=dev)))
+        refs.append(y_ref)
+    L.LayerGroup(items).run()
+    check_status()
+    for (_, _, out), y_ref in zip(items, refs):
+        y = out.cpu().numpy().astype(np.float64)
+        assert np.array_equal(y, y_ref), int((y != y_ref).sum())
+
+
+@pytest.mark.parametrize("scheme", ["4x8g8", "1x8g16", "3x8g8"])
+def test_group_llama_set_other_schemes_sampled_rows(dev, scheme):
+    """The Llama-2-7B layer set with another B = 8 scheme, one group call, sampled rows."""
+    M, g = int(scheme[0]), int(scheme.split("g")[1])
+    w = workloads.get("llama2_7b_layer_set_2x8g8")
+    items, lds, xs = [], [], []
+    for li, lay in enumerate(w.layers):
+        ld = synth.make_layer(M, 8, g, lay.K, lay.N, seed=3, layer=li)
+        x = synth.make_x(1, lay.K, seed=3, layer=li)
+        items.append((L.AqlmWeights.from_numpy(ld, dev), torch.from_numpy(x).to(dev),
+                      torch.empty((1, lay.N), dtype=torch.float16, device=dev)))
+        lds.append(ld)
+        xs.append(x)
+    L.LayerGroup(items).run()
+    check_status()
+    rng = np.random.Generator(np.random.PCG64(50))
+    for lay, ld, x, item in zip(w.layers, lds, xs, items):
+        rows = np.unique(np.concatenate([rng.choice(lay.N, size=24, replace=False), [0, lay.N - 1]]))
+        y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, M, 8, g, rows=rows)
+        assert_close(item[2].cpu().numpy()[:, rows], y_ref, f"{scheme}/{lay.name}")

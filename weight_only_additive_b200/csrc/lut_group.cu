@@ -52,7 +52,6 @@ constexpr uint32_t kTileBytes = 64u * 128u;        // 64 rows x 64 groups x 2 co
 constexpr uint32_t kLutBytes = 256u * 64u * 4u;    // 64 KB
 constexpr uint32_t kAOpBytes = 128u * 32u;         // 4 KB
 constexpr uint32_t kBOpBytes = 256u * 32u;         // 8 KB per codebook
-constexpr int kSlots = 16;                         // 128 KB of code tiles in flight
 #ifndef AQLM_GROUP_TASKS
 #define AQLM_GROUP_TASKS 2
 #endif
@@ -64,12 +63,20 @@ constexpr uint32_t kTmemCols = 512;                // D_0 at [0, 256), D_1 at [2
 
 constexpr uint32_t kOffLut = 0;
 constexpr uint32_t kOffA = kOffLut + kLutBytes;                 // 2 buffers
-constexpr uint32_t kOffB = kOffA + 2 * kAOpBytes;               // 1 buffer x 2 codebooks
-constexpr uint32_t kOffRing = kOffB + 2 * kBOpBytes;            // 1024-aligned
-constexpr uint32_t kOffBars = kOffRing + kSlots * kTileBytes;
-constexpr uint32_t kSmemBytes = kOffBars + 8u * (2 * kSlots + 1) + 16u;
-static_assert(kOffRing % 1024 == 0, "ring slots must stay 1024-byte aligned");
-static_assert(kSmemBytes <= 227u * 1024u, "shared memory budget");
+constexpr uint32_t kOffB = kOffA + 2 * kAOpBytes;               // 1 buffer x up to kMaxM codebooks
+
+// Shared-memory layout of the instantiation for launches whose layers have at most
+// kMaxM codebooks: the B operand holds kMaxM codebooks, and the code-tile ring takes
+// what is left (16 slots = 128 KB in flight for kMaxM = 2, 14 for kMaxM = 4).
+template <int kMaxM>
+struct GroupLayout {
+  static constexpr int kSlots = kMaxM <= 2 ? 16 : 14;
+  static constexpr uint32_t kOffRing = kOffB + kMaxM * kBOpBytes;   // 1024-aligned
+  static constexpr uint32_t kOffBars = kOffRing + kSlots * kTileBytes;
+  static constexpr uint32_t kSmemBytes = kOffBars + 8u * (2 * kSlots + 1) + 16u;
+  static_assert(kOffRing % 1024 == 0, "ring slots must stay 1024-byte aligned");
+  static_assert(kSmemBytes + 1024u <= 227u * 1024u, "shared memory budget");
+};
 
 struct GroupLayerDev {
   const __half* x;
@@ -78,7 +85,8 @@ struct GroupLayerDev {
   const __half* bias;
   __half* y;
   float* part;   // [S][N] fp32 partials in the workspace
-  int N, G, S, T;  // rows, groups, 64-group slices, 64-row tiles
+  int N, G, S, T;  // rows, groups (K / g), 128-code-byte slices, 64-row tiles
+  int M, g;        // codebooks per group, group width
   long long item0; // first item of this layer
   long long row0;  // first output row of this layer in the reduction grid
 };
@@ -180,12 +188,50 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
-// Table operands (cp.async, caller commits).  A (two buffers): row rho holds x
-// group 2 (rho mod 32) + (rho / 32 mod 2) of slice s (rows 64-127 repeat rows 0-63),
-// zero past the layer's last group.  B (one buffer, reloaded only when the layer
-// changes): the two codebooks, one 16-byte codeword per row.  The zero upper K
-// halves are written once at start-up.
+// Table operands (cp.async, caller commits).  Both K halves of every row are written
+// (zeros where g = 8), since layers with g = 16 may share the launch.
+//
+// 2x8 g8 (the tuned path): A row rho holds x group 2 (rho mod 32) + (rho / 32 mod 2)
+// of slice s (rows 64-127 repeat rows 0-63), zero past the layer's last group, so
+// that every TMEM lane quadrant holds the groups its conversion warps pack.
+__device__ __forceinline__ void load_x_slice_2x8(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
+  const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * kAOpBytes;
+  for (int idx = wtid; idx < 256; idx += kWorkers) {
+    const int rho = idx >> 1, h = idx & 1;
+    const int gg = s * 64 + 2 * (rho & 31) + ((rho >> 5) & 1);
+    const bool valid = h == 0 && gg < L.G;
+    cp_async_16_zfill(sbase + ao + kmajor_offset(rho, h),
+                      valid ? static_cast<const void*>(L.x + static_cast<size_t>(gg) * 8) : static_cast<const void*>(L.x),
+                      valid ? 16u : 0u);
+  }
+}
+// Other schemes: a slice is 128 code bytes b0 .. b0 + 127 (b0 = 128 s), byte b being
+// code m = b mod M of group j = b / M.  A row rho holds group j_lo + rho (j_lo = b0 / M),
+// for every group with a code byte in the slice (at most 128 / M + 1 groups).
+__device__ __forceinline__ void load_x_slice_generic(const GroupLayerDev& L, int s, uint32_t sbase, int buf,
+                                                     int wtid) {
+  const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * kAOpBytes;
+  const int b0 = s * 128;
+  const int j_lo = b0 / L.M;
+  for (int idx = wtid; idx < 256; idx += kWorkers) {
+    const int rho = idx >> 1, h = idx & 1;
+    const int j = j_lo + rho;
+    const bool valid = j < L.G && j * L.M < b0 + 128 && (h == 0 || L.g == 16);
+    cp_async_16_zfill(sbase + ao + kmajor_offset(rho, h),
+                      valid ? static_cast<const void*>(L.x + static_cast<size_t>(j) * L.g + 8 * h)
+                            : static_cast<const void*>(L.x),
+                      valid ? 16u : 0u);
+  }
+}
 __device__ __forceinline__ void load_x_slice(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
+  if (L.M == 2 && L.g == 8)
+    load_x_slice_2x8(L, s, sbase, buf, wtid);
+  else
+    load_x_slice_generic(L, s, sbase, buf, wtid);
+}
+// Launches of 2x8 g8 layers only (the tuned instantiation): the upper K halves are
+// zeroed once at start-up and the loaders write only the lower halves.
+__device__ __forceinline__ void load_x_slice_tuned(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
   const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * kAOpBytes;
   for (int rho = wtid; rho < 128; rho += kWorkers) {
     const int gg = s * 64 + 2 * (rho & 31) + ((rho >> 5) & 1);
@@ -195,14 +241,69 @@ __device__ __forceinline__ void load_x_slice(const GroupLayerDev& L, int s, uint
                       valid ? 16u : 0u);
   }
 }
-__device__ __forceinline__ void load_codebooks(const GroupLayerDev& L, uint32_t sbase, int wtid) {
+__device__ __forceinline__ void load_codebooks_tuned(const GroupLayerDev& L, uint32_t sbase, int wtid) {
   for (int e = wtid; e < 512; e += kWorkers)  // codebook m = e / 256, entry e % 256
     cp_async_16_zfill(sbase + kOffB + static_cast<uint32_t>(e >> 8) * kBOpBytes + kmajor_offset(e & 255, 0),
                       L.codebooks + static_cast<size_t>(e) * 8, 16u);
 }
+// B (one buffer, reloaded only when the layer changes): codebook m in rows of entry e,
+// both K halves (zeros for g = 8).
+__device__ __forceinline__ void load_codebooks(const GroupLayerDev& L, uint32_t sbase, int wtid) {
+  for (int idx = wtid; idx < L.M * 512; idx += kWorkers) {
+    const int m = idx >> 9, e = (idx >> 1) & 255, h = idx & 1;
+    const bool valid = h == 0 || L.g == 16;
+    cp_async_16_zfill(sbase + kOffB + static_cast<uint32_t>(m) * kBOpBytes + kmajor_offset(e, h),
+                      valid ? static_cast<const void*>(L.codebooks + (static_cast<size_t>(m) * 256 + e) * L.g + 8 * h)
+                            : static_cast<const void*>(L.codebooks),
+                      valid ? 16u : 0u);
+  }
+}
 
+// TMEM -> shared-memory table for round r of a scheme other than 2x8 g8 (codebooks
+// 2r and 2r + 1 of slice s; kept out of line so its registers do not weigh on the
+// lookup loop).  TMEM lane rho = group j_lo + rho; its codebook-m result is the table
+// of code byte b = (j_lo + rho) M + m - b0 when that byte lies in the slice.  Byte b
+// goes to half b mod 2 of the word of pair p = b / 2, in word column p / 2 (p even)
+// or 32 + p / 2 (p odd) of each entry's 64-word row, the layout the lookups read.
+// The warps of lane quadrant q = w mod 4 take entries 64 (w / 4) .. + 63.
+__device__ __noinline__ void generic_table_round(const GroupLayerDev& L, int s, int r, uint32_t tmem, int warp,
+                                                 int lane, uint8_t* lut_base) {
+  const int qd = warp & 3, sub = warp >> 2;
+  const int b0 = s * 128;
+  const int jj = b0 / L.M + 32 * qd + lane;
+  uint16_t* lut16 = reinterpret_cast<uint16_t*>(lut_base);
+  for (int mm = 0; mm < 2 && 2 * r + mm < L.M; ++mm) {
+    const int b = jj * L.M + 2 * r + mm - b0;
+    // every byte of the slice gets its entries, also the zero-filled bytes past the row
+    // end: their groups' A rows are zero, so their table entries are zero (a skipped
+    // entry would keep the previous run's value)
+    const bool keep = b >= 0 && b < 128;
+    const int pr = b >> 1;
+    const int col = ((pr & 1) ? 32 : 0) + (pr >> 1);
+#pragma unroll 1
+    for (int h = 0; h < 4; ++h) {
+      float v[16];
+      tmem_ld_32x32b_x16(tmem + tmem_lane_base(warp) + 256u * mm + static_cast<uint32_t>(64 * sub + 16 * h), v);
+      if (keep) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i = 64 * sub + 16 * h + e;
+          lut16[(i * 64 + col) * 2 + (b & 1)] = __half_as_ushort(__float2half_rn(v[e]));
+        }
+      }
+    }
+  }
+}
+
+// kGeneric = false: every layer of the launch is 2x8 g8 (the tuned code);
+// kGeneric = true: any B = 8 scheme, at most kMaxM codebooks.
+template <int kMaxM, bool kGeneric>
 __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_constant__ GroupMaps maps,
                                                                 const __grid_constant__ GroupParams p) {
+  static_assert(kGeneric || kMaxM == 2, "the tuned instantiation holds two codebooks");
+  using LY = GroupLayout<kMaxM>;
+  constexpr int kSlots = LY::kSlots;
+  constexpr uint32_t kOffRing = LY::kOffRing, kOffBars = LY::kOffBars;
   extern __shared__ uint8_t smem_raw[];
   // the ring slots are TMA destinations: keep the layout 1024-byte aligned
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -231,12 +332,14 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // zero upper K halves of the operand buffers (never written again)
-  for (int i = tid; i < 2 * 128 + 512; i += kThreads) {
-    const uint32_t off = i < 256 ? kOffA + static_cast<uint32_t>(i >> 7) * kAOpBytes + kmajor_offset(i & 127, 1)
-                                 : kOffB + static_cast<uint32_t>((i - 256) >> 8) * kBOpBytes +
-                                       kmajor_offset((i - 256) & 255, 1);
-    *reinterpret_cast<uint4*>(smem + off) = make_uint4(0u, 0u, 0u, 0u);
+  if constexpr (!kGeneric) {
+    // zero upper K halves of the operand buffers (never written again)
+    for (int i = tid; i < 2 * 128 + 512; i += kThreads) {
+      const uint32_t off = i < 256 ? kOffA + static_cast<uint32_t>(i >> 7) * kAOpBytes + kmajor_offset(i & 127, 1)
+                                   : kOffB + static_cast<uint32_t>((i - 256) >> 8) * kBOpBytes +
+                                         kmajor_offset((i - 256) & 255, 1);
+      *reinterpret_cast<uint4*>(smem + off) = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before_sync();
@@ -283,8 +386,14 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
     bool ok = true;
     if (it0 < it1) {
       const int l = layer_of(p, it0);
-      load_codebooks(p.layer[l], sbase, wtid);
-      load_x_slice(p.layer[l], static_cast<int>((it0 - p.layer[l].item0) / p.layer[l].T), sbase, 0, wtid);
+      const int s0 = static_cast<int>((it0 - p.layer[l].item0) / p.layer[l].T);
+      if constexpr (kGeneric) {
+        load_codebooks(p.layer[l], sbase, wtid);
+        load_x_slice(p.layer[l], s0, sbase, 0, wtid);
+      } else {
+        load_codebooks_tuned(p.layer[l], sbase, wtid);
+        load_x_slice_tuned(p.layer[l], s0, sbase, 0, wtid);
+      }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 
@@ -307,41 +416,95 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
         tc_fence_before_sync();
         ok = workers_sync_and(ok);  // old table no longer read; operands in place
         tc_fence_after_sync();
-        if (ok && wtid == 0) {
+        if constexpr (!kGeneric) {
+          if (ok && wtid == 0) {
+            const uint64_t adesc = kmajor_desc(sbase + kOffA + static_cast<uint32_t>(buf) * kAOpBytes);
+            const uint32_t bo = sbase + kOffB;
+            umma_f16_ss(tmem, adesc, kmajor_desc(bo), idesc, 0u);
+            umma_f16_ss(tmem + 256u, adesc, kmajor_desc(bo + kBOpBytes), idesc, 0u);
+            umma_commit(mma_bar);
+          }
+          // prefetch the x slice of the range's next (layer, slice) into the other A
+          // buffer, whose MMAs completed before the previous table was stored
+          const bool more = kbase + run_len < nitems;
+          const int nl = (s + 1 < L.S) ? l : l + 1;
+          if (ok && more) load_x_slice_tuned(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
+          const bool done = ok && group_wait(mma_bar, mma_phase, abort_flag, p.status, kSiteGroupMma);
+          mma_phase ^= 1u;
+          // the MMAs have read B: a new layer's codebooks may replace it now
+          if (done && more && nl != l) load_codebooks_tuned(p.layer[nl], sbase, wtid);
+          asm volatile("cp.async.commit_group;" ::: "memory");
+          ok = workers_sync_and(done);
+          tc_fence_after_sync();
+          if (ok) {
+            // TMEM -> shared-memory table; A rows rho and rho + 64 hold the same group, so
+            // all 16 warps take part: warp w reads lane quadrant w mod 4
+            const int qd = warp & 3;
+            const int col = 32 * (qd & 1) + lane;               // word column = rho mod 64
+            const int i0 = 32 * (2 * (warp >> 2) + (qd >> 1));  // 32 table entries per warp
+            uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kOffLut);
+            uint32_t r0[32], r1[32];
+            tmem_ld_x32(tmem + tmem_lane_base(warp) + static_cast<uint32_t>(i0), r0);
+            tmem_ld_x32(tmem + tmem_lane_base(warp) + 256u + static_cast<uint32_t>(i0), r1);
+  #pragma unroll
+            for (int j = 0; j < 32; ++j)
+              lut[(i0 + j) * 64 + col] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
+          }
+          tc_fence_before_sync();
+          ok = workers_sync_and(ok);  // table complete
+        } else {
+          // 2x8 g8 packs both codebooks' tables from one TMEM lane per word (the tuned
+          // path); every other scheme runs its M codebooks through the MMA two at a time
+          // (TMEM holds two 256-column results) and stores 16-bit table entries.
+          const bool tuned = L.M == 2 && L.g == 8;
+          const int rounds = tuned ? 1 : (L.M + 1) / 2;
           const uint64_t adesc = kmajor_desc(sbase + kOffA + static_cast<uint32_t>(buf) * kAOpBytes);
           const uint32_t bo = sbase + kOffB;
-          umma_f16_ss(tmem, adesc, kmajor_desc(bo), idesc, 0u);
-          umma_f16_ss(tmem + 256u, adesc, kmajor_desc(bo + kBOpBytes), idesc, 0u);
-          umma_commit(mma_bar);
+          if (ok && wtid == 0) {
+            umma_f16_ss(tmem, adesc, kmajor_desc(bo), idesc, 0u);
+            if (L.M >= 2) umma_f16_ss(tmem + 256u, adesc, kmajor_desc(bo + kBOpBytes), idesc, 0u);
+            umma_commit(mma_bar);
+          }
+          // prefetch the x slice of the range's next (layer, slice) into the other A
+          // buffer, whose MMAs completed before the previous table was stored
+          const bool more = kbase + run_len < nitems;
+          const int nl = (s + 1 < L.S) ? l : l + 1;
+          if (ok && more) load_x_slice(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
+          for (int r = 0; r < rounds; ++r) {
+            if (r > 0 && ok && wtid == 0) {
+              tc_fence_after_sync();
+              for (int mm = 0; mm < 2 && 2 * r + mm < L.M; ++mm)
+                umma_f16_ss(tmem + 256u * mm, adesc, kmajor_desc(bo + static_cast<uint32_t>(2 * r + mm) * kBOpBytes),
+                            idesc, 0u);
+              umma_commit(mma_bar);
+            }
+            const bool done = ok && group_wait(mma_bar, mma_phase, abort_flag, p.status, kSiteGroupMma);
+            mma_phase ^= 1u;
+            // the MMAs have read B: a new layer's codebooks may replace it now
+            if (r == rounds - 1 && done && more && nl != l) load_codebooks(p.layer[nl], sbase, wtid);
+            ok = workers_sync_and(done);
+            tc_fence_after_sync();
+            if (ok && tuned) {
+              // TMEM -> shared-memory table; A rows rho and rho + 64 hold the same group, so
+              // all 16 warps take part: warp w reads lane quadrant w mod 4
+              const int qd = warp & 3;
+              const int col = 32 * (qd & 1) + lane;               // word column = rho mod 64
+              const int i0 = 32 * (2 * (warp >> 2) + (qd >> 1));  // 32 table entries per warp
+              uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kOffLut);
+              uint32_t r0[32], r1[32];
+              tmem_ld_x32(tmem + tmem_lane_base(warp) + static_cast<uint32_t>(i0), r0);
+              tmem_ld_x32(tmem + tmem_lane_base(warp) + 256u + static_cast<uint32_t>(i0), r1);
+  #pragma unroll
+              for (int j = 0; j < 32; ++j)
+                lut[(i0 + j) * 64 + col] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
+            } else if (ok) {
+              generic_table_round(L, s, r, tmem, warp, lane, smem + kOffLut);
+            }
+            tc_fence_before_sync();
+            ok = workers_sync_and(ok);  // this round's table entries stored
+          }
+          asm volatile("cp.async.commit_group;" ::: "memory");
         }
-        // prefetch the x slice of the range's next (layer, slice) into the other A
-        // buffer, whose MMAs completed before the previous table was stored
-        const bool more = kbase + run_len < nitems;
-        const int nl = (s + 1 < L.S) ? l : l + 1;
-        if (ok && more) load_x_slice(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
-        const bool done = ok && group_wait(mma_bar, mma_phase, abort_flag, p.status, kSiteGroupMma);
-        mma_phase ^= 1u;
-        // the MMAs have read B: a new layer's codebooks may replace it now
-        if (done && more && nl != l) load_codebooks(p.layer[nl], sbase, wtid);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        ok = workers_sync_and(done);
-        tc_fence_after_sync();
-        if (ok) {
-          // TMEM -> shared-memory table; A rows rho and rho + 64 hold the same group, so
-          // all 16 warps take part: warp w reads lane quadrant w mod 4
-          const int qd = warp & 3;
-          const int col = 32 * (qd & 1) + lane;               // word column = rho mod 64
-          const int i0 = 32 * (2 * (warp >> 2) + (qd >> 1));  // 32 table entries per warp
-          uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kOffLut);
-          uint32_t r0[32], r1[32];
-          tmem_ld_x32(tmem + tmem_lane_base(warp) + static_cast<uint32_t>(i0), r0);
-          tmem_ld_x32(tmem + tmem_lane_base(warp) + 256u + static_cast<uint32_t>(i0), r1);
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            lut[(i0 + j) * 64 + col] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
-        }
-        tc_fence_before_sync();
-        ok = workers_sync_and(ok);  // table complete
         ++run;
       }
       for (int i = (wg - kbase) & (kTileGroups - 1); i < run_len; i += kTileGroups) {
@@ -480,13 +643,19 @@ __global__ void __launch_bounds__(kReduceRows* kReduceLanes) lut_group_reduce_ke
 
 namespace aqlm {
 
+// Batch-1 layers with 256-entry codebooks (B = 8), M = 1..4, g = 8 or 16, whose code
+// rows are whole 16-byte units (the TMA tensor's row stride).
 bool lut_group_supported(const Problem& p) {
-  return p.M == 2 && p.B == 8 && p.g == 8 && p.batch == 1 && p.K % 64 == 0;
+  if (p.B != 8 || p.batch != 1 || p.M < 1 || p.M > 4 || (p.g != 8 && p.g != 16) || p.K % p.g != 0) return false;
+  const long long row_bytes = static_cast<long long>(p.K / p.g) * p.M;
+  return row_bytes % 16 == 0;
 }
 
 namespace {
+// One fp32 partial per row and 128-code-byte slice.
 inline size_t part_bytes(const Problem& p) {
-  const size_t slices = static_cast<size_t>((p.K / 8 + 63) / 64);
+  const size_t row_bytes = static_cast<size_t>(p.K / p.g) * p.M;
+  const size_t slices = (row_bytes + 127) / 128;
   return (slices * static_cast<size_t>(p.N) * sizeof(float) + 255u) & ~static_cast<size_t>(255u);
 }
 }  // namespace
@@ -508,6 +677,8 @@ struct GroupLaunch {
   GroupParams p;
   GroupMaps maps;
   unsigned grid = 0, rgrid = 0;
+  int max_m = 0;          // the largest M of the run: selects the kernel instantiation
+  bool generic = false;   // some layer is not 2x8 g8
 };
 
 struct GroupKey {
@@ -548,6 +719,8 @@ cudaError_t build_group_launch(const Problem* probs, int count, void* workspace,
   GroupMaps& maps = out->maps;
   p = GroupParams{};
   maps = GroupMaps{};
+  out->max_m = 0;
+  out->generic = false;
   long long items = 0, rows = 0;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   for (int i = 0; i < count; ++i) {
@@ -562,16 +735,21 @@ cudaError_t build_group_launch(const Problem* probs, int count, void* workspace,
     L.part = reinterpret_cast<float*>(ws);
     ws += part_bytes(pr);
     L.N = pr.N;
-    L.G = pr.K / 8;
-    L.S = (L.G + 63) / 64;
+    L.M = pr.M;
+    L.g = pr.g;
+    L.G = pr.K / pr.g;
+    const int row_bytes = L.G * pr.M;
+    L.S = (row_bytes + 127) / 128;
     L.T = (pr.N + kTileRows - 1) / kTileRows;
+    out->max_m = std::max(out->max_m, pr.M);
+    if (pr.M != 2 || pr.g != 8) out->generic = true;
     L.item0 = items;
     L.row0 = rows;
     items += static_cast<long long>(L.S) * L.T;
     rows += pr.N;
-    // codes as a 2D byte tensor [N rows][2G bytes]; a box is 64 rows x 128 bytes
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(L.G) * 2, static_cast<cuuint64_t>(pr.N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(L.G) * 2};
+    // codes as a 2D byte tensor [N rows][G M bytes]; a box is 64 rows x 128 bytes
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(pr.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
     const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kTileRows)};
     const cuuint32_t estr[2] = {1, 1};
     if (encode(&maps.map[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pr.codes), dims, strides, box, estr,
@@ -599,16 +777,22 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  const uint32_t smem = kSmemBytes + 1024u;
   GroupLaunch launch;
   {
     std::lock_guard<std::mutex> lock(g_launch_mu);
     if (g_sms[dev] == 0) {
-      // once per device: the SM count and the kernel's shared-memory limit
+      // once per device: the SM count and the kernels' shared-memory limits
       int sms = 0;
       e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
       if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(lut_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      e = cudaFuncSetAttribute(lut_group_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(GroupLayout<2>::kSmemBytes + 1024u));
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(lut_group_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(GroupLayout<2>::kSmemBytes + 1024u));
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(lut_group_kernel<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(GroupLayout<4>::kSmemBytes + 1024u));
       if (e != cudaSuccess) return e;
       g_sms[dev] = std::max(1, sms);
     }
@@ -634,14 +818,20 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const bool wide = launch.max_m > 2;  // up to four codebooks: the kMaxM = 4 layout
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(launch.grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = (wide ? GroupLayout<4>::kSmemBytes : GroupLayout<2>::kSmemBytes) + 1024u;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, lut_group_kernel, launch.maps, launch.p);
+  if (wide)
+    e = cudaLaunchKernelEx(&cfg, lut_group_kernel<4, true>, launch.maps, launch.p);
+  else if (launch.generic)
+    e = cudaLaunchKernelEx(&cfg, lut_group_kernel<2, true>, launch.maps, launch.p);
+  else
+    e = cudaLaunchKernelEx(&cfg, lut_group_kernel<2, false>, launch.maps, launch.p);
   if (e != cudaSuccess) return e;
 
   cudaLaunchConfig_t rcfg = {};
