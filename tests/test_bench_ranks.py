@@ -45,3 +45,15 @@ def test_single_rank_and_throughput():
     assert bench.max_over_ranks(3.5, None, None) == 3.5
     # 2 ranks x 100 steps x 1e9 bytes in 50 ms -> 4000 GB/s
     assert bench.job_throughput_gbs(1e9, 100, 2, 50.0) == pytest.approx(4000.0)
+
+
+def test_bench_scheme_override_parses():
+    import bench
+    from weight_only_additive_b200 import workloads
+    a = bench.parse_args(["--workload", "llama2_7b_layer_set_2x8g8", "--scheme", "3x8g16"])
+    w = bench.select_workload(a)
+    assert all(l.scheme == workloads.Scheme(3, 8, 16) for l in w.layers)
+    assert w.name.endswith("@3x8g16")
+    import pytest
+    with pytest.raises(SystemExit):
+        bench.parse_scheme("3x8")
