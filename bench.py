@@ -108,16 +108,29 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "source": "fallback", "tc_tflops_sustained": 1400.0}
 
 
-KERNEL_SOURCES = {"gemv_gather_kernel": "gemv.cu", "gemv_lut_2x8_kernel": "gemv_lut.cu",
-                  "tc_decode_mma_kernel": "tc_gemm.cu", "tc_pipe_kernel": "tc_pipe.cu",
-                  "lut_group_kernel": "lut_group.cu"}
+# the files under csrc/ each kernel is compiled from (its .cu first, then the headers
+# that hold its device code): a traffic record is valid only while they are unchanged
+KERNEL_SOURCES = {"gemv_gather_kernel": ("gemv.cu", "aqlm_device.cuh"),
+                  "gemv_lut_kernel": ("gemv_lut.cu", "lut_table.cuh", "aqlm_device.cuh"),
+                  "tc_decode_mma_kernel": ("tc_gemm.cu", "aqlm_device.cuh"),
+                  "tc_pipe_kernel": ("tc_pipe.cu", "aqlm_device.cuh"),
+                  "lut_group_kernel": ("lut_group.cu", "lut_table.cuh", "aqlm_device.cuh")}
+
+
+def kernel_source_sha256(kernel):
+    """sha256 over the kernel's source files, concatenated in KERNEL_SOURCES order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "weight_only_additive_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
 def measured_traffic(workload_name, kernel):
     """DRAM bytes per launch (read + write) of `kernel` on this workload, from the ncu
     capture recorded in profiles/roofline_traffic.json -- or None when there is none or
     the kernel's source changed since it was taken."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
     if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
         return None
@@ -125,10 +138,8 @@ def measured_traffic(workload_name, kernel):
         rec = json.load(fh).get(f"{workload_name}/{kernel}")
     if not rec or rec.get("kernel") != kernel:
         return None
-    src = os.path.join(ROOT, "weight_only_additive_b200", "csrc", KERNEL_SOURCES[kernel])
-    with open(src, "rb") as fh:
-        if hashlib.sha256(fh.read()).hexdigest() != rec.get("source_sha256"):
-            return None
+    if kernel_source_sha256(kernel) != rec.get("source_sha256"):
+        return None
     return rec.get("dram_bytes_per_launch")
 
 
@@ -502,7 +513,7 @@ def run_ours(a):
                  "unit": "GB/s", "us_per_layer": o_ms * 1e3 / (o_steps * len(w.layers)), "steps": o_steps}
 
     peaks = measured_peaks()
-    kernel_names = {int(Path.GEMV): "gemv_gather_kernel", int(Path.GEMV_LUT): "gemv_lut_2x8_kernel",
+    kernel_names = {int(Path.GEMV): "gemv_gather_kernel", int(Path.GEMV_LUT): "gemv_lut_kernel",
                     int(Path.TENSOR_CORE): "tc_pipe_kernel"}
     if mode == "group" and launches_per_step == 2 * ((len(w.layers) + 15) // 16):
         # every layer grouped: the timed launches are the partial-sum kernel and its

@@ -77,7 +77,8 @@ typedef enum {
 typedef enum {
   AQLM_PATH_AUTO = 0,         /* pick by (M, B, g, batch)                               */
   AQLM_PATH_GEMV = 1,         /* codeword-gather GEMV, any supported scheme, batch <= 8 */
-  AQLM_PATH_GEMV_LUT = 2,     /* x.codeword lookup-table GEMV, 2x8 only, batch <= 8     */
+  AQLM_PATH_GEMV_LUT = 2,     /* x.codeword lookup-table GEMV, B = 8, batch 1; code     *
+                               * rows (K/g * M bytes) a multiple of 16 and <= 8192       */
   AQLM_PATH_TENSOR_CORE = 3   /* on-chip decode -> tcgen05 fp16 MMA, any batch          */
 } aqlm_path;
 

@@ -88,7 +88,13 @@ def test_compute_entry_points_reject_bad_arguments_before_any_cuda_call(lib):
     assert e.value.status == Status.UNSUPPORTED  # the GEMV family stops at batch 8
     with pytest.raises(native.AqlmError) as e:
         native.aqlm_matmul_path(A, A, A, A, None, A, 1, 16, 8, 64, 64, 1, Path.GEMV_LUT)
-    assert e.value.status == Status.UNSUPPORTED  # the lookup table is the 2x8 kernel
+    assert e.value.status == Status.UNSUPPORTED  # the lookup table needs 256-entry codebooks
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_matmul_path(A, A, A, A, None, A, 3, 8, 8, 64, 64, 1, Path.GEMV_LUT)
+    assert e.value.status == Status.UNSUPPORTED  # code rows of 24 bytes: not whole 16-byte units
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_matmul_path(A, A, A, A, None, A, 1, 8, 8, 8 * 8200, 64, 1, Path.GEMV_LUT)
+    assert e.value.status == Status.UNSUPPORTED  # code rows above 16 x 4 x 128 bytes
     with pytest.raises(native.AqlmError) as e:
         native.aqlm_matmul_path(A, A, A, A, None, A, 2, 8, 8, 64, 64, 2, Path.GEMV_LUT)
     assert e.value.status == Status.UNSUPPORTED  # batch 1 only
@@ -112,7 +118,16 @@ def test_path_selection(lib):
         for batch in (9, 16, 256):
             assert sel(M, B, g, 4096 + 8, 4096, batch) == Path.TENSOR_CORE
     assert sel(5, 8, 8, 4096, 4096, 1) == -1
-    assert sel(3, 8, 8, 4096, 4096, 1) == Path.TENSOR_CORE  # f2 schemes: tensor core from batch 1
+    # f2 schemes with B = 8: the lookup table at batch 1 (16-byte code rows of at most
+    # 8 KB), the tensor-core kernel above
+    for M in (1, 2, 3, 4):
+        for g in (8, 16):
+            assert sel(M, 8, g, 4096, 4096, 1) == Path.GEMV_LUT, (M, g)
+            assert sel(M, 8, g, 4096, 4096, 2) == Path.TENSOR_CORE, (M, g)
+    assert sel(1, 8, 8, 8 * 8192, 4096, 1) == Path.GEMV_LUT  # 8192-byte rows: the longest
+    assert sel(1, 8, 8, 8 * 8208, 4096, 1) != Path.GEMV_LUT
+    assert sel(3, 8, 16, 16 * 1000, 4096, 1) != Path.GEMV_LUT  # 3000-byte rows
+    assert sel(4, 8, 16, 16 * 1000, 4096, 1) == Path.GEMV_LUT  # 4000-byte rows
     assert sel(1, 16, 8, 4095, 4096, 1) == -1
 
 

@@ -150,8 +150,8 @@ def test_integer_layers_bit_exact(dev, M, B, g, path, batch):
     """Small-integer codebooks and x, scales in {1, 2}: every product and partial sum
     is an exact small integer in fp16/fp32, so any summation order gives the exact
     value and y must equal the oracle bit for bit."""
-    if path == Path.GEMV_LUT and (M, B, g) != (2, 8, 8):
-        pytest.skip("the lookup-table GEMV is the 2x8 kernel")
+    if path == Path.GEMV_LUT and B != 8:
+        pytest.skip("the lookup-table GEMV needs 256-entry codebooks")
     N, K = 260, 512
     rng = np.random.Generator(np.random.PCG64(14))
     cb = rng.integers(-2, 3, size=(M, 1 << B, g)).astype(np.float16)

@@ -1,31 +1,39 @@
-// Lookup-table GEMV for 2x8 codebooks (two codebooks of 256 fp16 codewords of
-// 8 weights), batch 1: "fast lookup, no per-element dequantization"
-// (inference-research record "AQLM (additive / multi-codebook quantization)",
-// section "Kernels").
+// Lookup-table GEMV for codebooks of 256 entries (B = 8), batch 1: "fast lookup,
+// no per-element dequantization" (inference-research record "AQLM (additive /
+// multi-codebook quantization)", section "Kernels").
 //
-//   T_m[j][i] = sum_t x[8j + t] * C_m[i][t]            (per group j, codebook m, entry i)
-//   y[n]      = s_n * sum_j (T_0[j][codes[n,j,0]] + T_1[j][codes[n,j,1]]) + bias_n
+//   T_m[j][i] = sum_t x[g j + t] * C_m[i][t]            (per group j, codebook m, entry i)
+//   y[n]      = s_n * sum_j sum_m T_m[j][codes[n,j,m]] + bias_n
+//
+// A code row is G M bytes (byte b = code of codebook b mod M in group b / M), cut
+// into slices of 128 bytes; the table of a slice holds the 128 x 256 entries of
+// its bytes, and a row's partial over the slice is the sum of its 128 lookups.
 //
 // Work split.  A cluster of C CTAs owns a block of output rows; CTA c of the
-// cluster owns a K slice of P passes x 64 groups.  Per pass the CTA
-//   1. builds the lookup table of its 64 groups with two tcgen05.mma
-//      (M = 128 rows of x groups, N = 256 codebook entries, K = 16 with the
-//      upper 8 zero), accumulator in TMEM;
-//   2. moves it TMEM -> registers -> shared memory as fp16 pairs
-//      (T_0, T_1) per (entry, group): 256 entries x 64 groups x 4 B = 64 KB;
-//   3. streams the codes of its rows (cp.async, double-buffered, 32 rows x
-//      128 B per warp chunk) and sums lookups.
-// The row partials of the C CTAs are exchanged with bulk shared-memory copies
-// inside the cluster and summed in a fixed order (deterministic), then the
-// channel scale and bias are applied.
+// cluster owns P consecutive slices (passes).  Per pass the CTA
+//   1. builds the slice's table with tcgen05.mma (M = 128 rows, N = 256 codebook
+//      entries, K = 16 per step), accumulator in TMEM;
+//   2. moves it TMEM -> registers -> shared memory as fp16 entries,
+//      256 entries x 128 bytes x 2 B = 64 KB;
+//   3. sums the lookups of its rows from code tiles (64 rows x 128 bytes, one TMA
+//      box each).  The CTA's tiles are issued at the start into R shared-memory
+//      slots; when they do not all fit (long rows), a slot is reloaded with a later
+//      pass's tile as soon as the pass that read it ends.
+// The row partials of the C CTAs are exchanged through distributed shared memory
+// inside the cluster and summed in a fixed order (deterministic), then the channel
+// scale and bias are applied.
 //
-// Bank-conflict-free lookups.  Lane l of a warp owns row l of a 32-row chunk.
-// At step s it reads code word w = (l + s) mod 32 of its row (4 codes: groups
-// 2w and 2w+1, codebooks 0 and 1).  The table stores group 2w in word column
-// w and group 2w+1 in column 32 + w of each entry's 64-word row, so the 32
-// lanes of a lookup touch 32 different banks whatever the codes are.  The
-// table is written from TMEM lane rho = word column, which is conflict-free
-// too: A row rho holds group 2*(rho mod 32) + rho/32.
+// 2x8 g8 (two codebooks of 8-wide codewords, a slice = 64 groups) has its own tuned
+// instantiation: one MMA per codebook, whose two results pack into one word per
+// (entry, group).  Every other scheme uses the stacked build of lut_table.cuh (the
+// M codebooks side by side along K, one TMEM lane per code byte), with its x slices
+// double-buffered.
+//
+// Bank-conflict-free lookups.  A task is 8 rows, 4 lanes per row; lane (r8, q4)
+// reads code word w = 8 q4 + ((r8 + s) mod 8) of its row at step s (4 code bytes,
+// pairs 2w and 2w + 1).  The table stores pair 2w in word column w and pair 2w + 1
+// in column 32 + w of each entry's 64-word row, so the 32 lanes of a lookup touch 32
+// different banks whatever the codes are.
 #include <cuda.h>
 
 #include <algorithm>
@@ -34,18 +42,18 @@
 #include <tuple>
 
 #include "aqlm_device.cuh"
+#include "lut_table.cuh"
 
 namespace aqlm {
 namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kGroupsPerPass = 64;
-constexpr int kMaxPasses = 4;                      // K <= 16 CTAs x 4 passes x 64 groups x 8
+constexpr int kMaxPasses = 4;                      // code rows <= 16 CTAs x 4 passes x 128 bytes
 constexpr int kTileRows = 64;                      // rows per code tile (one TMA box)
-constexpr uint32_t kLutBytes = 256u * 64u * 4u;   // 64 KB
-constexpr uint32_t kAOpBytes = 128u * 32u;         // 4 KB per pass
-constexpr uint32_t kBOpBytes = 256u * 32u;         // 8 KB per codebook
+constexpr uint32_t kLutBytes = lut::kTableBytes;   // 64 KB
+constexpr uint32_t kAOpBytes = lut::kAOpBytes;     // 4 KB per pass
+constexpr uint32_t kBOpBytes = lut::kBOpBytes;     // 8 KB per codebook
 constexpr uint32_t kTileBytes = 64u * 128u;        // 64 rows x 128 B of codes (one TMA box)
 constexpr uint32_t kTmemCols = 512;                // D_0 at [0,256), D_1 at [256,512)
 constexpr uint32_t kSmemLimit = 227u * 1024u;
@@ -56,13 +64,15 @@ struct LutParams {
   const __half* scales;
   const __half* bias;
   __half* y;
-  int K, N, G;
-  int C;      // CTAs per cluster (K slices)
-  int P;      // passes of 64 groups per CTA
+  int N, G, M, g;
+  int S;      // 128-byte slices of a code row
+  int C;      // CTAs per cluster
+  int P;      // passes (slices) per CTA
   int RB;     // output rows per cluster
   int RBc;    // rows each CTA reduces (multiple of 4)
   int ntask;  // ceil(RB / 8): 8-row tasks per pass
   int ntile;  // ceil(RB / 64): code tiles per pass
+  int R;      // code-tile slots, >= ntile: tile i = ps ntile + tl of the CTA goes to slot i mod R
   uint32_t* status;
 };
 
@@ -70,14 +80,27 @@ struct SmemLayout {
   uint32_t lut, aop, bop, tiles, part, recv, bars, total;
 };
 
-// All code tiles of the CTA's passes stay resident: P * ntile tiles of 8 KB.
-__host__ __device__ inline SmemLayout smem_layout(int C, int P, int RBc, int ntask, int ntile) {
+// Table operands: the tuned build keeps the A operands of all P passes (one K step
+// each) and two one-step codebooks; the stacked build has ks K steps
+// (lut::stacked_ksteps) and two A buffers that take the passes in turn.
+struct OperandBytes {
+  uint32_t a, b;
+};
+__host__ __device__ inline OperandBytes operand_bytes(bool generic, int P, int M, int g) {
+  if (!generic) return OperandBytes{kAOpBytes * static_cast<uint32_t>(P), 2u * kBOpBytes};
+  const uint32_t ks = static_cast<uint32_t>(lut::stacked_ksteps(M, g));
+  return OperandBytes{kAOpBytes * ks * static_cast<uint32_t>(P < 2 ? P : 2), kBOpBytes * ks};
+}
+
+// R code-tile slots of 8 KB (all P * ntile tiles of the CTA when they fit, else at
+// least one pass's ntile, reused pass after pass); one mbarrier per tile.
+__host__ __device__ inline SmemLayout smem_layout(int C, int P, int RBc, int ntask, int ntile, int R, OperandBytes ob) {
   SmemLayout L;
   L.lut = 0;
   L.aop = L.lut + kLutBytes;                                        // 1024-aligned
-  L.bop = L.aop + kAOpBytes * static_cast<uint32_t>(P);
-  L.tiles = L.bop + 2 * kBOpBytes;
-  L.part = L.tiles + static_cast<uint32_t>(P * ntile) * kTileBytes;
+  L.bop = L.aop + ob.a;
+  L.tiles = L.bop + ob.b;
+  L.part = L.tiles + static_cast<uint32_t>(R) * kTileBytes;
   const int part_count = ntask * 8 > C * RBc ? ntask * 8 : C * RBc;
   L.recv = L.part + ((static_cast<uint32_t>(part_count) * 4u + 15u) & ~15u);
   L.bars = L.recv + static_cast<uint32_t>(C * RBc * 4);
@@ -85,17 +108,26 @@ __host__ __device__ inline SmemLayout smem_layout(int C, int P, int RBc, int nta
   return L;
 }
 
-// Rows per cluster for a layer: as even a split over Q resident clusters as the
-// shared memory allows (all code tiles of a CTA resident); 0 if not even 64 fit.
-__host__ __device__ inline int rows_per_cluster(int N, int Q, int C, int P) {
+// Rows per cluster RB and code-tile slots R for a layer: as even a split over Q
+// resident clusters as the shared memory allows.  R = P ntile (every tile of the CTA
+// resident) when that fits, else the slots that fit, as long as one pass's ntile tiles
+// do; {0, 0} if not even 8 rows fit.
+struct RowSplit {
+  int RB, R;
+};
+inline RowSplit rows_per_cluster(int N, int Q, int C, int P, OperandBytes ob) {
   int RB = (N + Q - 1) / Q;
   RB = (RB + 7) & ~7;
   while (RB >= 8) {
     const int RBc = (((RB + C - 1) / C) + 3) & ~3;
-    if (smem_layout(C, P, RBc, (RB + 7) / 8, (RB + kTileRows - 1) / kTileRows).total <= kSmemLimit) return RB;
+    const int ntile = (RB + kTileRows - 1) / kTileRows;
+    const SmemLayout full = smem_layout(C, P, RBc, (RB + 7) / 8, ntile, P * ntile, ob);
+    if (full.total <= kSmemLimit) return RowSplit{RB, P * ntile};
+    const int drop = static_cast<int>((full.total - kSmemLimit + kTileBytes - 1) / kTileBytes);
+    if (P * ntile - drop >= ntile) return RowSplit{RB, P * ntile - drop};
     RB = RB > 64 ? RB - 64 : RB - 8;
   }
-  return 0;
+  return RowSplit{0, 0};
 }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -115,40 +147,38 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Descriptor of a K-major operand in the no-swizzle canonical layout: 8-row x
-// 16-byte core matrices, the two K halves 128 bytes apart (leading byte
-// offset), consecutive 8-row groups 256 bytes apart (stride byte offset).
-__device__ __forceinline__ uint64_t umma_desc_kmajor_noswizzle(uint32_t smem_byte_addr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(128u >> 4) << 16;
-  d |= static_cast<uint64_t>(256u >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  return d;  // layout type 0 (no swizzle), base offset 0
-}
-__host__ __device__ inline uint32_t kmajor_noswizzle_offset(int row, int khalf) {
-  return static_cast<uint32_t>((row >> 3) * 256 + khalf * 128 + (row & 7) * 16);
+using lut::kmajor_desc;
+using lut::kmajor_offset;
+
+// Issues the CTA's code tiles i_begin .. i_end - 1 (one thread): tile i is row tile
+// i mod ntile (skipped from ntl on, past this cluster's rows) of pass i / ntile, a
+// 64-row x 128-byte TMA box into slot i mod R.  Out of line: it runs a few times per
+// launch and its registers would otherwise weigh on the lookup loop.
+__device__ __noinline__ void issue_code_tiles(const CUtensorMap* map, uint32_t tiles, uint64_t* tile_bar, int i_begin,
+                                              int i_end, int ntile, int ntl, int R, int slice0, int rb0) {
+  const uint64_t pol = l2_policy_evict_first();
+  for (int i = i_begin; i < i_end; ++i) {
+    const int ps = i / ntile, tl = i - ps * ntile;
+    if (tl >= ntl) continue;
+    mbar_arrive_expect_tx(&tile_bar[i], kTileBytes);
+    // bytes past the row end and rows past N are zero-filled
+    tma_load_2d(tiles + static_cast<uint32_t>(i % R) * kTileBytes, map, (slice0 + ps) * 128, rb0 + tl * kTileRows,
+                &tile_bar[i], pol);
+  }
 }
 
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-
-__global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_constant__ CUtensorMap code_map,
-                                                                    const LutParams p) {
+// kGeneric = false: 2x8 g8 (the tuned table build); true: any B = 8 scheme.
+// kRecycle = false: all P ntile code tiles of a CTA are resident (R = P ntile);
+// true: fewer slots, reloaded pass after pass.  Separate instantiations, since the
+// reload bookkeeping costs the resident case ~5 % (its lookup loop's code changes).
+template <bool kGeneric, bool kRecycle>
+__global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const __grid_constant__ CUtensorMap code_map,
+                                                                const LutParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int C = p.C;
-  const SmemLayout L = smem_layout(C, p.P, p.RBc, p.ntask, p.ntile);
+  const SmemLayout L = smem_layout(C, p.P, p.RBc, p.ntask, p.ntile, p.R, operand_bytes(kGeneric, p.P, p.M, p.g));
+  const int ks = lut::stacked_ksteps(p.M, p.g);                      // stacked build only
+  const uint32_t abuf = kAOpBytes * static_cast<uint32_t>(ks);       // one A buffer of it
   const uint32_t sbase = smem_addr(smem);
   float* part = reinterpret_cast<float*>(smem + L.part);
   float* recv = reinterpret_cast<float*>(smem + L.recv);
@@ -167,9 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
   const int nt = (nrows + 7) >> 3;                          // 8-row tasks of this row block
   const int ntl = (nrows + kTileRows - 1) / kTileRows;      // 64-row tiles of this row block
 
-  // passes this CTA runs (gcnt > 0); uniform across the CTA
-  int npass = 0;
-  while (npass < p.P && (static_cast<int>(crank) * p.P + npass) * kGroupsPerPass < p.G) ++npass;
+  // passes this CTA runs (slices crank P .. crank P + npass - 1 of the row); uniform
+  const int slice0 = static_cast<int>(crank) * p.P;
+  const int npass = max(0, min(p.P, p.S - slice0));
 
   // The next kernel in the stream may start its own weight-only set-up now.
   grid_dependents_launch();
@@ -181,15 +211,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  if (tid == 32 * (kWarps - 1)) {
-    const uint64_t pol = l2_policy_evict_first();
-    for (int ps = 0; ps < npass; ++ps) {
-      const int gbeg = (static_cast<int>(crank) * p.P + ps) * kGroupsPerPass;
-      for (int tl = 0; tl < ntl; ++tl) {
-        const int i = ps * p.ntile + tl;
-        mbar_arrive_expect_tx(&tile_bar[i], kTileBytes);
-        tma_load_2d(sbase + L.tiles + static_cast<uint32_t>(i) * kTileBytes, &code_map, gbeg * 2,
-                           rb0 + tl * kTileRows, &tile_bar[i], pol);
+  // Tile i = ps ntile + tl (pass ps, rows rb0 + 64 tl ..) lands in slot i mod R.  The
+  // tiles i < R start now; tile i >= R starts at the end of the pass that consumed
+  // tile i - R (an earlier pass, since R >= ntile).
+  const bool issuer = tid == 32 * (kWarps - 1);
+  if constexpr (kRecycle) {
+    if (issuer)
+      issue_code_tiles(&code_map, sbase + L.tiles, tile_bar, 0, min(npass * p.ntile, p.R), p.ntile, ntl, p.R, slice0,
+                       rb0);
+  } else {
+    if (issuer) {
+      const uint64_t pol = l2_policy_evict_first();
+      for (int ps = 0; ps < npass; ++ps) {
+        for (int tl = 0; tl < ntl; ++tl) {
+          const int i = ps * p.ntile + tl;
+          mbar_arrive_expect_tx(&tile_bar[i], kTileBytes);
+          // bytes past the row end and rows past N are zero-filled
+          tma_load_2d(sbase + L.tiles + static_cast<uint32_t>(i) * kTileBytes, &code_map, (slice0 + ps) * 128,
+                      rb0 + tl * kTileRows, &tile_bar[i], pol);
+        }
       }
     }
   }
@@ -204,29 +244,40 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
     }
   }
 
-  // ---- 2. operands (both codebooks, x of every pass) and TMEM ------------------------------
+  // ---- 2. operands (the codebooks, x of every pass) and TMEM -------------------------------
   {
-    for (int i = tid; i < 2 * 256; i += kThreads) {
-      const int m = i >> 8, idx = i & 255;
-      const uint32_t bo = L.bop + static_cast<uint32_t>(m) * kBOpBytes;
-      cp_async_16_zfill(sbase + bo + kmajor_noswizzle_offset(idx, 0), p.codebooks + (static_cast<size_t>(m) * 256 + idx) * 8, 16);
-      *reinterpret_cast<uint4*>(smem + bo + kmajor_noswizzle_offset(idx, 1)) = make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (kGeneric) {
+      lut::load_codebooks_stacked<kThreads>(p.codebooks, p.M, p.g, sbase + L.bop, tid);
+    } else {
+      for (int i = tid; i < 2 * 256; i += kThreads) {
+        const int m = i >> 8, idx = i & 255;
+        const uint32_t bo = L.bop + static_cast<uint32_t>(m) * kBOpBytes;
+        cp_async_16_zfill(sbase + bo + kmajor_offset(idx, 0), p.codebooks + (static_cast<size_t>(m) * 256 + idx) * 8, 16);
+        *reinterpret_cast<uint4*>(smem + bo + kmajor_offset(idx, 1)) = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
     for (int i = tid; i < p.ntask * 8; i += kThreads) part[i] = 0.f;
     // Everything above reads only weights.  x may be the output of the kernel just
     // before this one in the stream (programmatic dependent launch): wait for it.
     grid_dependency_wait();
-    for (int i = tid; i < npass * 128; i += kThreads) {  // A row rho (and rho+64) = one group of x
-      const int ps = i >> 7, rho = i & 127;
-      const int gbeg = (static_cast<int>(crank) * p.P + ps) * kGroupsPerPass;
-      const int gg = 2 * (rho & 31) + ((rho >> 5) & 1);
-      const uint32_t ao = L.aop + static_cast<uint32_t>(ps) * kAOpBytes;
-      const bool valid = gbeg + gg < p.G;
-      cp_async_16_zfill(sbase + ao + kmajor_noswizzle_offset(rho, 0),
-                       valid ? static_cast<const void*>(p.x + static_cast<size_t>(gbeg + gg) * 8)
-                             : static_cast<const void*>(p.x),
-                       valid ? 16u : 0u);
-      *reinterpret_cast<uint4*>(smem + ao + kmajor_noswizzle_offset(rho, 1)) = make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (kGeneric) {
+      // passes 0 and 1; pass ps + 2 follows once the MMAs of pass ps have read its buffer
+      for (int ps = 0; ps < npass && ps < 2; ++ps)
+        lut::load_x_stacked<kThreads>(p.x, p.G, p.M, p.g, slice0 + ps, sbase + L.aop + static_cast<uint32_t>(ps) * abuf,
+                                      tid);
+    } else {
+      for (int i = tid; i < npass * 128; i += kThreads) {  // A row rho (and rho+64) = one group of x
+        const int ps = i >> 7, rho = i & 127;
+        const int gbeg = (slice0 + ps) * 64;
+        const int gg = 2 * (rho & 31) + ((rho >> 5) & 1);
+        const uint32_t ao = L.aop + static_cast<uint32_t>(ps) * kAOpBytes;
+        const bool valid = gbeg + gg < p.G;
+        cp_async_16_zfill(sbase + ao + kmajor_offset(rho, 0),
+                          valid ? static_cast<const void*>(p.x + static_cast<size_t>(gbeg + gg) * 8)
+                                : static_cast<const void*>(p.x),
+                          valid ? 16u : 0u);
+        *reinterpret_cast<uint4*>(smem + ao + kmajor_offset(rho, 1)) = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
     cp_async_commit();
   }
@@ -244,35 +295,43 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
   const int q4 = lane & 3;   // quarter of the row's 32 code words
 
   for (int ps = 0; ps < npass; ++ps) {
-    // ---- 3. table of this pass: two MMAs into TMEM ---------------------------------------
-    if (tid == 0 && ok) {
+    // ---- 3.-4. table of this pass: MMAs into TMEM, then TMEM -> shared memory --------------
+    const uint64_t adesc = kmajor_desc(sbase + L.aop + static_cast<uint32_t>(ps) * kAOpBytes);
+    if constexpr (!kGeneric) {
+      if (tid == 0 && ok) {
+        tc_fence_after_sync();
+        umma_f16_ss(tmem, adesc, kmajor_desc(sbase + L.bop), idesc, 0u);
+        umma_f16_ss(tmem + 256, adesc, kmajor_desc(sbase + L.bop + kBOpBytes), idesc, 0u);
+        umma_commit(mma_bar);
+      }
+      const bool done = ok ? mbar_wait_bounded(mma_bar, mma_phase, p.status, kSiteLutMma) : false;
+      mma_phase ^= 1u;
+      ok = __syncthreads_and(done ? 1 : 0) != 0;
       tc_fence_after_sync();
-      const uint64_t adesc = umma_desc_kmajor_noswizzle(sbase + L.aop + static_cast<uint32_t>(ps) * kAOpBytes);
-      umma_f16_ss(tmem, adesc, umma_desc_kmajor_noswizzle(sbase + L.bop), idesc, 0u);
-      umma_f16_ss(tmem + 256, adesc, umma_desc_kmajor_noswizzle(sbase + L.bop + kBOpBytes), idesc, 0u);
-      umma_commit(mma_bar);
+      // all 16 warps: A rows rho and rho + 64 hold the same group
+      if (ok) lut::store_table_2x8(tmem, warp, lane, smem + L.lut);
+      tc_fence_before_sync();
+      __syncthreads();
+    } else {
+      // the stacked build: one MMA chain, one TMEM lane per code byte of the slice
+      if (tid == 0 && ok) {
+        tc_fence_after_sync();
+        lut::mma_stacked(tmem, sbase + L.aop + static_cast<uint32_t>(ps & 1) * abuf, sbase + L.bop, ks, idesc);
+        umma_commit(mma_bar);
+      }
+      const bool done = ok ? mbar_wait_bounded(mma_bar, mma_phase, p.status, kSiteLutMma) : false;
+      mma_phase ^= 1u;
+      // A buffer ps mod 2 has been read: start the x slice of pass ps + 2 there
+      if (done && ps + 2 < npass)
+        lut::load_x_stacked<kThreads>(p.x, p.G, p.M, p.g, slice0 + ps + 2,
+                                      sbase + L.aop + static_cast<uint32_t>(ps & 1) * abuf, tid);
+      cp_async_commit();
+      ok = __syncthreads_and(done ? 1 : 0) != 0;
+      tc_fence_after_sync();
+      if (ok) lut::store_table_stacked(tmem, warp, lane, smem + L.lut);
+      tc_fence_before_sync();
+      __syncthreads();
     }
-    const bool done = ok ? mbar_wait_bounded(mma_bar, mma_phase, p.status, kSiteLutMma) : false;
-    mma_phase ^= 1u;
-    ok = __syncthreads_and(done ? 1 : 0) != 0;
-    tc_fence_after_sync();
-
-    // ---- 4. TMEM -> shared-memory table, all 16 warps (A rows rho and rho+64 agree) --------
-    if (ok) {
-      const int qd = warp & 3;
-      const int col = 32 * (qd & 1) + lane;                 // word column = rho mod 64
-      const int i0 = 32 * (2 * (warp >> 2) + (qd >> 1));    // 32 table entries per warp
-      const uint32_t lane_off = static_cast<uint32_t>(32 * qd) << 16;
-      uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
-      uint32_t r0[32], r1[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + static_cast<uint32_t>(i0), r0);
-      tmem_ld_32x32b_x32(tmem + lane_off + 256u + static_cast<uint32_t>(i0), r1);
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        lut[(i0 + j) * 64 + col] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
-    }
-    tc_fence_before_sync();
-    __syncthreads();
 
     {
       // ---- 5. lookups: a task is 8 rows; 4 lanes per row, 8 code words each -------------------
@@ -280,12 +339,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
       // always touch 32 distinct words, so both the code reads and the table reads are
       // free of bank conflicts.  Pairs of looked-up fp16 values are added as half2 and
       // the task's 16 pair sums are accumulated in half2, then widened to fp32.
+      const int slot0 = kRecycle ? (ps * p.ntile) % p.R : 0;  // slot of the pass's first tile
       for (int t = warp; t < nt; t += kWarps) {
         const int i = ps * p.ntile + t / 8;  // tile holding rows 8t .. 8t+7
+        int slot = i;                        // its slot, i mod R
+        if constexpr (kRecycle) {
+          slot = slot0 + t / 8;
+          if (slot >= p.R) slot -= p.R;
+        }
         const bool landed = mbar_wait_bounded(&tile_bar[i], 0u, p.status, kSiteLutCodes);
         if (ok && landed) {
           const uint32_t* cw_row = reinterpret_cast<const uint32_t*>(
-              smem + L.tiles + i * kTileBytes + ((t & 7) * 8 + r8) * 128);
+              smem + L.tiles + slot * kTileBytes + ((t & 7) * 8 + r8) * 128);
           uint32_t cw[8];
 #pragma unroll
           for (int s8 = 0; s8 < 8; ++s8) cw[s8] = cw_row[8 * q4 + ((r8 + s8) & 7)];
@@ -314,9 +379,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
         }
       }
     }
+    if constexpr (kGeneric) {
+      // the next pass's A operand (committed one group before the newest) has landed
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+      fence_proxy_async_smem();
+    }
     // the next pass rebuilds the table: every warp must be done reading it
     ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    // the slots of pass ps are free: start the tiles R + ps ntile .. that take them
+    if (kRecycle && issuer && ok && p.R + ps * p.ntile < npass * p.ntile)
+      issue_code_tiles(&code_map, sbase + L.tiles, tile_bar, p.R + ps * p.ntile,
+                       min(npass * p.ntile, p.R + (ps + 1) * p.ntile), p.ntile, ntl, p.R, slice0, rb0);
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
 
   // ---- 6. partials -> their owner CTA (remote shared-memory stores), one cluster barrier ----
   // Row r of the block is reduced by CTA r / RBc; this CTA's partial of it lands in
@@ -353,42 +428,58 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_2x8_kernel(const __grid_
 }
 
 struct Plan {
-  int C, P, Q, RB;
+  int C, P, Q, RB, R;
 };
 
-// The cost model picks (cluster size C, passes P) for a layer: P passes of 64
-// groups per CTA, C = ceil(G / 64P) <= 16 CTAs per cluster, Q clusters resident,
-// RB rows per cluster (fewer than N / Q when the code tiles would not fit, which
-// costs extra waves).  Cycles per CTA: rows * 128P lookups at ~24 per cycle plus
-// ~600 per pass to build and store the table.
-int plan_cost(int N, int P, int Q, int RB) {
+// The cost model picks (cluster size C, passes P) for a layer: P slices of 128 code
+// bytes per CTA, C = ceil(S / P) <= 16 CTAs per cluster, Q clusters resident, RB
+// rows per cluster (fewer than N / Q when not even one pass of code tiles fits,
+// which costs extra waves).  Cycles per CTA: rows * 128P lookups at ~24 per cycle,
+// ~600 per pass to build and store the table, and ~800 per pass whose tiles wait for
+// recycled slots (their loads start only when the previous pass ends).
+int plan_cost(int N, int P, int Q, int RB, int R) {
   const int clusters = (N + RB - 1) / RB;
   const int waves = (clusters + Q - 1) / Q;
-  return waves * (RB * 128 * P / 24 + 600 * P);
+  const int ntile = (RB + kTileRows - 1) / kTileRows;
+  const int late_passes = (P * ntile - R + ntile - 1) / ntile;
+  return waves * (RB * 128 * P / 24 + 600 * P + 800 * late_passes);
 }
 
-// Chooses (C, P, Q) for a layer on the current device; cached per (device, N, K).
-cudaError_t lut_plan(int dev, int N, int G, Plan* out) {
+// Chooses (C, P, Q) for a layer on the current device; cached per (device, N, S, M,
+// g, instantiation).
+template <bool kGeneric>
+cudaError_t lut_plan(int dev, int N, int S, int M, int g, Plan* out) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int>, Plan> cache;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(std::make_tuple(dev, N, G));
-    if (it != cache.end()) {
-      *out = it->second;
-      return cudaSuccess;
-    }
+  static std::map<std::tuple<int, int, int, int, int>, Plan> cache;
+  static bool wide_clusters[64] = {};
+  static bool attrs_set[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(std::make_tuple(dev, N, S, M, g));
+  if (it != cache.end()) {
+    *out = it->second;
+    return cudaSuccess;
   }
-  auto kern = gemv_lut_2x8_kernel;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  const int cmax = (e == cudaSuccess) ? 16 : 8;
-  cudaGetLastError();
-  Plan best{0, 0, 0, 0};
+  if (!attrs_set[dev]) {
+    // clusters of up to 16 CTAs where the device allows them, else the portable 8
+    wide_clusters[dev] = cudaFuncSetAttribute(gemv_lut_kernel<kGeneric, false>,
+                                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+                         cudaFuncSetAttribute(gemv_lut_kernel<kGeneric, true>,
+                                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    cudaGetLastError();
+    cudaError_t e = cudaFuncSetAttribute(gemv_lut_kernel<kGeneric, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemLimit));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemv_lut_kernel<kGeneric, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSmemLimit));
+    if (e != cudaSuccess) return e;
+    attrs_set[dev] = true;
+  }
+  const int cmax = wide_clusters[dev] ? 16 : 8;
+  Plan best{0, 0, 0, 0, 0};
   int best_cost = 0;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
-  if (e != cudaSuccess) return e;
   for (int P = 1; P <= kMaxPasses; ++P) {
-    const int C = (G + 64 * P - 1) / (64 * P);
+    const int C = (S + P - 1) / P;
     if (C > cmax) continue;
     // one CTA per SM (its TMEM and shared memory), so residency is set by cluster placement
     cudaLaunchConfig_t cfg = {};
@@ -403,55 +494,52 @@ cudaError_t lut_plan(int dev, int N, int G, Plan* out) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int q = 0;
-    e = cudaOccupancyMaxActiveClusters(&q, kern, &cfg);
+    // both instantiations: one CTA per SM, the same shared memory and TMEM
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&q, gemv_lut_kernel<kGeneric, false>, &cfg);
     if (e != cudaSuccess || q <= 0) {
       cudaGetLastError();
       if (C == 1) break;
       continue;
     }
     q = std::min(q, std::max(1, (N + 31) / 32));
-    const int RB = rows_per_cluster(N, q, C, P);
+    const RowSplit split = rows_per_cluster(N, q, C, P, operand_bytes(kGeneric, P, M, g));
+    const int RB = split.RB;
     if (RB == 0) {
       if (C == 1) break;
       continue;
     }
-    const int cost = plan_cost(N, P, q, RB);
+    const int cost = plan_cost(N, P, q, RB, split.R);
     if (best.C == 0 || cost < best_cost) {
-      best = Plan{C, P, q, RB};
+      best = Plan{C, P, q, RB, split.R};
       best_cost = cost;
     }
     if (C == 1) break;
   }
   if (best.C == 0) return cudaErrorInvalidConfiguration;
-  std::lock_guard<std::mutex> lock(mu);
-  cache[std::make_tuple(dev, N, G)] = best;
+  cache[std::make_tuple(dev, N, S, M, g)] = best;
   *out = best;
   return cudaSuccess;
 }
 
-}  // namespace
-
-bool gemv_lut_supported(int M, int B, int g, int K, int batch) {
-  return M == 2 && B == 8 && g == 8 && batch == 1 && K % 64 == 0 && K <= 16 * kMaxPasses * kGroupsPerPass * 8;
-}
-
-cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t stream) {
-  const int G = pr.K / 8;
+template <bool kGeneric>
+cudaError_t launch_lut(const Problem& pr, uint32_t* status, cudaStream_t stream) {
+  const int G = pr.K / pr.g;
+  const int row_bytes = G * pr.M;
+  const int S = (row_bytes + 127) / 128;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   Plan best;
-  e = lut_plan(dev, pr.N, G, &best);
+  e = lut_plan<kGeneric>(dev, pr.N, S, pr.M, pr.g, &best);
   if (e != cudaSuccess) return e;
-  auto kern = gemv_lut_2x8_kernel;
 
-  // Codes as a 2D byte tensor [N rows][2G bytes]; a box is 64 rows x 128 bytes
-  // (one 64-group pass of 64 rows).  Out-of-range rows and bytes read as zero.
+  // Codes as a 2D byte tensor [N rows][G M bytes]; a box is 64 rows x 128 bytes
+  // (one slice of 64 rows).  Out-of-range rows and bytes read as zero.
   EncodeTiledFn encode = encode_tiled();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap map;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(G) * 2, static_cast<cuuint64_t>(pr.N)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(G) * 2};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(pr.N)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
   const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kTileRows)};
   const cuuint32_t estr[2] = {1, 1};
   if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pr.codes), dims, strides, box, estr,
@@ -465,19 +553,20 @@ cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t st
   p.scales = static_cast<const __half*>(pr.scales);
   p.bias = static_cast<const __half*>(pr.bias);
   p.y = static_cast<__half*>(pr.y);
-  p.K = pr.K;
   p.N = pr.N;
   p.G = G;
+  p.M = pr.M;
+  p.g = pr.g;
+  p.S = S;
   p.C = best.C;
   p.P = best.P;
   p.RB = best.RB;
   p.RBc = (((p.RB + p.C - 1) / p.C) + 3) & ~3;
   p.ntask = (p.RB + 7) / 8;
   p.ntile = (p.RB + kTileRows - 1) / kTileRows;
+  p.R = best.R;
   p.status = status;
-  const SmemLayout L = smem_layout(p.C, p.P, p.RBc, p.ntask, p.ntile);
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
-  if (e != cudaSuccess) return e;
+  const SmemLayout L = smem_layout(p.C, p.P, p.RBc, p.ntask, p.ntile, p.R, operand_bytes(kGeneric, p.P, p.M, p.g));
   const int clusters = (pr.N + p.RB - 1) / p.RB;
 
   cudaLaunchConfig_t cfg = {};
@@ -494,7 +583,24 @@ cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t st
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, map, p);
+  if (p.R < p.P * p.ntile) return cudaLaunchKernelEx(&cfg, gemv_lut_kernel<kGeneric, true>, map, p);
+  return cudaLaunchKernelEx(&cfg, gemv_lut_kernel<kGeneric, false>, map, p);
+}
+
+}  // namespace
+
+// Batch-1 layers with 256-entry codebooks (B = 8), M = 1..4, g = 8 or 16, whose code
+// rows are whole 16-byte units (the TMA tensor's row stride) and at most 16 CTAs x 4
+// passes x 128 bytes long.
+bool gemv_lut_supported(int M, int B, int g, int K, int batch) {
+  if (B != 8 || batch != 1 || M < 1 || M > 4 || (g != 8 && g != 16) || K <= 0 || K % g != 0) return false;
+  const long long row_bytes = static_cast<long long>(K / g) * M;
+  return row_bytes % 16 == 0 && row_bytes <= 16LL * kMaxPasses * 128;
+}
+
+cudaError_t launch_gemv_lut(const Problem& pr, uint32_t* status, cudaStream_t stream) {
+  if (pr.M == 2 && pr.g == 8) return launch_lut<false>(pr, status, stream);
+  return launch_lut<true>(pr, status, stream);
 }
 
 }  // namespace aqlm

@@ -1,5 +1,5 @@
-// Grouped lookup-table GEMV: one launch computes a set of independent 2x8 g8,
-// batch-1 layers (a decoder block's linears), the "fast lookup, no per-element
+// Grouped lookup-table GEMV: one launch computes a set of independent batch-1 layers
+// with 256-entry codebooks (a decoder block's linears), the "fast lookup, no per-element
 // dequantization" path of the inference-research record "AQLM (additive /
 // multi-codebook quantization)", section "Kernels", applied to a whole layer set
 // so that no layer pays its own launch, set-up and tail.
@@ -7,9 +7,11 @@
 //   T_m[j][i] = sum_t x[8j + t] * C_m[i][t]                 (group j, codebook m, entry i)
 //   part[s][n] = sum_{j in slice s} (T_0[j][codes[n,j,0]] + T_1[j][codes[n,j,1]])
 //   y[n]       = s_n * sum_s part[s][n] + bias_n             (second kernel, s ascending)
+// (written for 2x8 g8, where a slice of 128 code bytes is 64 groups; for any M, g a
+// slice is 128 code bytes and part sums the table entries of its bytes).
 //
-// Work items.  Item (p, s, t) is layer p's 64-group K slice s on its 64-row tile
-// t; a layer has ceil(G / 64) x ceil(N / 64) items.  Items are numbered layer by
+// Work items.  Item (p, s, t) is layer p's 128-code-byte slice s on its 64-row tile
+// t; a layer has ceil(G M / 128) x ceil(N / 64) items.  Items are numbered layer by
 // layer, slice-major, and every CTA (one per SM, persistent) takes a contiguous
 // range of them, so consecutive items mostly share (p, s) and therefore the
 // lookup table: a CTA rebuilds it only when (p, s) changes.
@@ -26,6 +28,10 @@
 //               group j take the tiles k = j (mod kTileGroups), kTasks interleaved
 //               8-row tasks per warp, and write each row's fp32 partial to the
 //               workspace.
+// Generic instantiations (any B = 8 scheme) build each slice's table with the stacked
+// build of lut_table.cuh (the M codebooks side by side along K, one TMEM lane per code
+// byte); launches of 2x8 g8 layers only keep the tuned build described above.
+//
 // The partials of a row are summed over the slices in ascending order by a second
 // small kernel (programmatic dependent launch), which applies the channel scale
 // and bias: the result does not depend on which CTA ran which item.
@@ -40,6 +46,7 @@
 #include <mutex>
 
 #include "aqlm_device.cuh"
+#include "lut_table.cuh"
 
 namespace aqlm {
 namespace {
@@ -49,9 +56,9 @@ constexpr int kThreads = kWorkers + 32;            // + TMA producer warp
 constexpr int kProducerWarp = kWorkers / 32;
 constexpr int kTileRows = 64;
 constexpr uint32_t kTileBytes = 64u * 128u;        // 64 rows x 64 groups x 2 codes
-constexpr uint32_t kLutBytes = 256u * 64u * 4u;    // 64 KB
-constexpr uint32_t kAOpBytes = 128u * 32u;         // 4 KB
-constexpr uint32_t kBOpBytes = 256u * 32u;         // 8 KB per codebook
+constexpr uint32_t kLutBytes = lut::kTableBytes;   // 64 KB
+constexpr uint32_t kAOpBytes = lut::kAOpBytes;     // 4 KB
+constexpr uint32_t kBOpBytes = lut::kBOpBytes;     // 8 KB per codebook
 #ifndef AQLM_GROUP_TASKS
 #define AQLM_GROUP_TASKS 2
 #endif
@@ -62,21 +69,25 @@ static_assert(kTasks * kWarpsPerTile == 8 && (kTileGroups & (kTileGroups - 1)) =
 constexpr uint32_t kTmemCols = 512;                // D_0 at [0, 256), D_1 at [256, 512)
 
 constexpr uint32_t kOffLut = 0;
-constexpr uint32_t kOffA = kOffLut + kLutBytes;                 // 2 buffers
-constexpr uint32_t kOffB = kOffA + 2 * kAOpBytes;               // 1 buffer x up to kMaxM codebooks
+constexpr uint32_t kOffA = kOffLut + kLutBytes;    // 2 A buffers
 
-// Shared-memory layout of the instantiation for launches whose layers have at most
-// kMaxM codebooks: the B operand holds kMaxM codebooks, and the code-tile ring takes
-// what is left (16 slots = 128 KB in flight for kMaxM = 2, 14 for kMaxM = 4).
-template <int kMaxM>
+// Shared-memory layout of an instantiation.  The tuned one (2x8 g8 layers only) has
+// A buffers of one K step and B = two codebooks of one K step each (kBSteps = 2); the
+// generic ones (stacked build) have A buffers and a B operand of kBSteps K steps,
+// enough for layers whose M g is at most 16 kBSteps.  The code-tile ring takes what is
+// left: 16 slots (128 KB in flight) for kBSteps = 2, 12 for kBSteps = 4.
+template <int kBSteps, bool kGeneric>
 struct GroupLayout {
-  static constexpr int kSlots = kMaxM <= 2 ? 16 : 14;
-  static constexpr uint32_t kOffRing = kOffB + kMaxM * kBOpBytes;   // 1024-aligned
+  static constexpr uint32_t kABytes = (kGeneric ? kBSteps : 1) * kAOpBytes;
+  static constexpr uint32_t kOffB = kOffA + 2 * kABytes;
+  static constexpr uint32_t kOffRing = kOffB + kBSteps * kBOpBytes;   // 1024-aligned
+  static constexpr int kSlots = kBSteps <= 2 ? 16 : 12;
   static constexpr uint32_t kOffBars = kOffRing + kSlots * kTileBytes;
   static constexpr uint32_t kSmemBytes = kOffBars + 8u * (2 * kSlots + 1) + 16u;
   static_assert(kOffRing % 1024 == 0, "ring slots must stay 1024-byte aligned");
   static_assert(kSmemBytes + 1024u <= 227u * 1024u, "shared memory budget");
 };
+using TunedLayout = GroupLayout<2, false>;
 
 struct GroupLayerDev {
   const __half* x;
@@ -102,8 +113,6 @@ struct GroupParams {
 struct GroupMaps {
   CUtensorMap map[kMaxGroupLayers];
 };
-
-__device__ __forceinline__ uint32_t tmem_lane_base(int warp) { return static_cast<uint32_t>(32 * (warp & 3)) << 16; }
 
 // Named barrier over the 16 worker warps that also ANDs a flag across them.
 __device__ __forceinline__ bool workers_sync_and(bool v) {
@@ -160,79 +169,16 @@ struct ItemCursor {
   }
 };
 
-// No-swizzle K-major operand layout: 8-row x 16-byte core matrices, the two
-// K halves 128 bytes apart, consecutive 8-row groups 256 bytes apart.
-__host__ __device__ inline uint32_t kmajor_offset(int row, int khalf) {
-  return static_cast<uint32_t>((row >> 3) * 256 + khalf * 128 + (row & 7) * 16);
-}
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t smem_byte_addr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(128u >> 4) << 16;
-  d |= static_cast<uint64_t>(256u >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  return d;
-}
+using lut::kmajor_offset;
+using lut::kmajor_desc;
 
-__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-
-// Table operands (cp.async, caller commits).  Both K halves of every row are written
-// (zeros where g = 8), since layers with g = 16 may share the launch.
-//
-// 2x8 g8 (the tuned path): A row rho holds x group 2 (rho mod 32) + (rho / 32 mod 2)
-// of slice s (rows 64-127 repeat rows 0-63), zero past the layer's last group, so
-// that every TMEM lane quadrant holds the groups its conversion warps pack.
-__device__ __forceinline__ void load_x_slice_2x8(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
-  const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * kAOpBytes;
-  for (int idx = wtid; idx < 256; idx += kWorkers) {
-    const int rho = idx >> 1, h = idx & 1;
-    const int gg = s * 64 + 2 * (rho & 31) + ((rho >> 5) & 1);
-    const bool valid = h == 0 && gg < L.G;
-    cp_async_16_zfill(sbase + ao + kmajor_offset(rho, h),
-                      valid ? static_cast<const void*>(L.x + static_cast<size_t>(gg) * 8) : static_cast<const void*>(L.x),
-                      valid ? 16u : 0u);
-  }
-}
-// Other schemes: a slice is 128 code bytes b0 .. b0 + 127 (b0 = 128 s), byte b being
-// code m = b mod M of group j = b / M.  A row rho holds group j_lo + rho (j_lo = b0 / M),
-// for every group with a code byte in the slice (at most 128 / M + 1 groups).
-__device__ __forceinline__ void load_x_slice_generic(const GroupLayerDev& L, int s, uint32_t sbase, int buf,
-                                                     int wtid) {
-  const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * kAOpBytes;
-  const int b0 = s * 128;
-  const int j_lo = b0 / L.M;
-  for (int idx = wtid; idx < 256; idx += kWorkers) {
-    const int rho = idx >> 1, h = idx & 1;
-    const int j = j_lo + rho;
-    const bool valid = j < L.G && j * L.M < b0 + 128 && (h == 0 || L.g == 16);
-    cp_async_16_zfill(sbase + ao + kmajor_offset(rho, h),
-                      valid ? static_cast<const void*>(L.x + static_cast<size_t>(j) * L.g + 8 * h)
-                            : static_cast<const void*>(L.x),
-                      valid ? 16u : 0u);
-  }
-}
-__device__ __forceinline__ void load_x_slice(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
-  if (L.M == 2 && L.g == 8)
-    load_x_slice_2x8(L, s, sbase, buf, wtid);
-  else
-    load_x_slice_generic(L, s, sbase, buf, wtid);
-}
-// Launches of 2x8 g8 layers only (the tuned instantiation): the upper K halves are
-// zeroed once at start-up and the loaders write only the lower halves.
+// Table operands of the tuned instantiation (cp.async, caller commits): A row rho holds
+// x group 2 (rho mod 32) + (rho / 32 mod 2) of slice s (rows 64-127 repeat rows 0-63),
+// zero past the layer's last group, so that every TMEM lane quadrant holds the groups
+// its conversion warps pack; B holds the two codebooks.  The upper K halves are zeroed
+// once at start-up and the loaders write only the lower halves.
 __device__ __forceinline__ void load_x_slice_tuned(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
-  const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * kAOpBytes;
+  const uint32_t ao = kOffA + static_cast<uint32_t>(buf) * TunedLayout::kABytes;
   for (int rho = wtid; rho < 128; rho += kWorkers) {
     const int gg = s * 64 + 2 * (rho & 31) + ((rho >> 5) & 1);
     const bool valid = gg < L.G;
@@ -243,65 +189,28 @@ __device__ __forceinline__ void load_x_slice_tuned(const GroupLayerDev& L, int s
 }
 __device__ __forceinline__ void load_codebooks_tuned(const GroupLayerDev& L, uint32_t sbase, int wtid) {
   for (int e = wtid; e < 512; e += kWorkers)  // codebook m = e / 256, entry e % 256
-    cp_async_16_zfill(sbase + kOffB + static_cast<uint32_t>(e >> 8) * kBOpBytes + kmajor_offset(e & 255, 0),
+    cp_async_16_zfill(sbase + TunedLayout::kOffB + static_cast<uint32_t>(e >> 8) * kBOpBytes + kmajor_offset(e & 255, 0),
                       L.codebooks + static_cast<size_t>(e) * 8, 16u);
 }
-// B (one buffer, reloaded only when the layer changes): codebook m in rows of entry e,
-// both K halves (zeros for g = 8).
-__device__ __forceinline__ void load_codebooks(const GroupLayerDev& L, uint32_t sbase, int wtid) {
-  for (int idx = wtid; idx < L.M * 512; idx += kWorkers) {
-    const int m = idx >> 9, e = (idx >> 1) & 255, h = idx & 1;
-    const bool valid = h == 0 || L.g == 16;
-    cp_async_16_zfill(sbase + kOffB + static_cast<uint32_t>(m) * kBOpBytes + kmajor_offset(e, h),
-                      valid ? static_cast<const void*>(L.codebooks + (static_cast<size_t>(m) * 256 + e) * L.g + 8 * h)
-                            : static_cast<const void*>(L.codebooks),
-                      valid ? 16u : 0u);
-  }
+// Generic instantiations: the stacked build's operands (A buffer buf of slice s; B, one
+// buffer, reloaded only when the layer changes).
+template <int kBSteps>
+__device__ __forceinline__ void load_x_slice_stacked(const GroupLayerDev& L, int s, uint32_t sbase, int buf, int wtid) {
+  using LY = GroupLayout<kBSteps, true>;
+  lut::load_x_stacked<kWorkers>(L.x, L.G, L.M, L.g, s, sbase + kOffA + static_cast<uint32_t>(buf) * LY::kABytes, wtid);
 }
-
-// TMEM -> shared-memory table for round r of a scheme other than 2x8 g8 (codebooks
-// 2r and 2r + 1 of slice s; kept out of line so its registers do not weigh on the
-// lookup loop).  TMEM lane rho = group j_lo + rho; its codebook-m result is the table
-// of code byte b = (j_lo + rho) M + m - b0 when that byte lies in the slice.  Byte b
-// goes to half b mod 2 of the word of pair p = b / 2, in word column p / 2 (p even)
-// or 32 + p / 2 (p odd) of each entry's 64-word row, the layout the lookups read.
-// The warps of lane quadrant q = w mod 4 take entries 64 (w / 4) .. + 63.
-__device__ __noinline__ void generic_table_round(const GroupLayerDev& L, int s, int r, uint32_t tmem, int warp,
-                                                 int lane, uint8_t* lut_base) {
-  const int qd = warp & 3, sub = warp >> 2;
-  const int b0 = s * 128;
-  const int jj = b0 / L.M + 32 * qd + lane;
-  uint16_t* lut16 = reinterpret_cast<uint16_t*>(lut_base);
-  for (int mm = 0; mm < 2 && 2 * r + mm < L.M; ++mm) {
-    const int b = jj * L.M + 2 * r + mm - b0;
-    // every byte of the slice gets its entries, also the zero-filled bytes past the row
-    // end: their groups' A rows are zero, so their table entries are zero (a skipped
-    // entry would keep the previous run's value)
-    const bool keep = b >= 0 && b < 128;
-    const int pr = b >> 1;
-    const int col = ((pr & 1) ? 32 : 0) + (pr >> 1);
-#pragma unroll 1
-    for (int h = 0; h < 4; ++h) {
-      float v[16];
-      tmem_ld_32x32b_x16(tmem + tmem_lane_base(warp) + 256u * mm + static_cast<uint32_t>(64 * sub + 16 * h), v);
-      if (keep) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i = 64 * sub + 16 * h + e;
-          lut16[(i * 64 + col) * 2 + (b & 1)] = __half_as_ushort(__float2half_rn(v[e]));
-        }
-      }
-    }
-  }
+template <int kBSteps>
+__device__ __forceinline__ void load_codebooks_stacked(const GroupLayerDev& L, uint32_t sbase, int wtid) {
+  lut::load_codebooks_stacked<kWorkers>(L.codebooks, L.M, L.g, sbase + GroupLayout<kBSteps, true>::kOffB, wtid);
 }
 
 // kGeneric = false: every layer of the launch is 2x8 g8 (the tuned code);
-// kGeneric = true: any B = 8 scheme, at most kMaxM codebooks.
-template <int kMaxM, bool kGeneric>
+// kGeneric = true: any B = 8 scheme with M g <= 16 kBSteps (the stacked build).
+template <int kBSteps, bool kGeneric>
 __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_constant__ GroupMaps maps,
                                                                 const __grid_constant__ GroupParams p) {
-  static_assert(kGeneric || kMaxM == 2, "the tuned instantiation holds two codebooks");
-  using LY = GroupLayout<kMaxM>;
+  static_assert(kGeneric || kBSteps == 2, "the tuned instantiation holds two one-step codebooks");
+  using LY = GroupLayout<kBSteps, kGeneric>;
   constexpr int kSlots = LY::kSlots;
   constexpr uint32_t kOffRing = LY::kOffRing, kOffBars = LY::kOffBars;
   extern __shared__ uint8_t smem_raw[];
@@ -335,8 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
   if constexpr (!kGeneric) {
     // zero upper K halves of the operand buffers (never written again)
     for (int i = tid; i < 2 * 128 + 512; i += kThreads) {
-      const uint32_t off = i < 256 ? kOffA + static_cast<uint32_t>(i >> 7) * kAOpBytes + kmajor_offset(i & 127, 1)
-                                   : kOffB + static_cast<uint32_t>((i - 256) >> 8) * kBOpBytes +
+      const uint32_t off = i < 256 ? kOffA + static_cast<uint32_t>(i >> 7) * LY::kABytes + kmajor_offset(i & 127, 1)
+                                   : LY::kOffB + static_cast<uint32_t>((i - 256) >> 8) * kBOpBytes +
                                          kmajor_offset((i - 256) & 255, 1);
       *reinterpret_cast<uint4*>(smem + off) = make_uint4(0u, 0u, 0u, 0u);
     }
@@ -388,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
       const int l = layer_of(p, it0);
       const int s0 = static_cast<int>((it0 - p.layer[l].item0) / p.layer[l].T);
       if constexpr (kGeneric) {
-        load_codebooks(p.layer[l], sbase, wtid);
-        load_x_slice(p.layer[l], s0, sbase, 0, wtid);
+        load_codebooks_stacked<kBSteps>(p.layer[l], sbase, wtid);
+        load_x_slice_stacked<kBSteps>(p.layer[l], s0, sbase, 0, wtid);
       } else {
         load_codebooks_tuned(p.layer[l], sbase, wtid);
         load_x_slice_tuned(p.layer[l], s0, sbase, 0, wtid);
@@ -418,8 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
         tc_fence_after_sync();
         if constexpr (!kGeneric) {
           if (ok && wtid == 0) {
-            const uint64_t adesc = kmajor_desc(sbase + kOffA + static_cast<uint32_t>(buf) * kAOpBytes);
-            const uint32_t bo = sbase + kOffB;
+            const uint64_t adesc = kmajor_desc(sbase + kOffA + static_cast<uint32_t>(buf) * LY::kABytes);
+            const uint32_t bo = sbase + LY::kOffB;
             umma_f16_ss(tmem, adesc, kmajor_desc(bo), idesc, 0u);
             umma_f16_ss(tmem + 256u, adesc, kmajor_desc(bo + kBOpBytes), idesc, 0u);
             umma_commit(mma_bar);
@@ -436,74 +345,32 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
           asm volatile("cp.async.commit_group;" ::: "memory");
           ok = workers_sync_and(done);
           tc_fence_after_sync();
-          if (ok) {
-            // TMEM -> shared-memory table; A rows rho and rho + 64 hold the same group, so
-            // all 16 warps take part: warp w reads lane quadrant w mod 4
-            const int qd = warp & 3;
-            const int col = 32 * (qd & 1) + lane;               // word column = rho mod 64
-            const int i0 = 32 * (2 * (warp >> 2) + (qd >> 1));  // 32 table entries per warp
-            uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kOffLut);
-            uint32_t r0[32], r1[32];
-            tmem_ld_x32(tmem + tmem_lane_base(warp) + static_cast<uint32_t>(i0), r0);
-            tmem_ld_x32(tmem + tmem_lane_base(warp) + 256u + static_cast<uint32_t>(i0), r1);
-  #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              lut[(i0 + j) * 64 + col] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
-          }
+          if (ok) lut::store_table_2x8(tmem, warp, lane, smem + kOffLut);
           tc_fence_before_sync();
           ok = workers_sync_and(ok);  // table complete
         } else {
-          // 2x8 g8 packs both codebooks' tables from one TMEM lane per word (the tuned
-          // path); every other scheme runs its M codebooks through the MMA two at a time
-          // (TMEM holds two 256-column results) and stores 16-bit table entries.
-          const bool tuned = L.M == 2 && L.g == 8;
-          const int rounds = tuned ? 1 : (L.M + 1) / 2;
-          const uint64_t adesc = kmajor_desc(sbase + kOffA + static_cast<uint32_t>(buf) * kAOpBytes);
-          const uint32_t bo = sbase + kOffB;
+          // the stacked build: one MMA chain gives the whole slice's table, one TMEM
+          // lane per code byte
           if (ok && wtid == 0) {
-            umma_f16_ss(tmem, adesc, kmajor_desc(bo), idesc, 0u);
-            if (L.M >= 2) umma_f16_ss(tmem + 256u, adesc, kmajor_desc(bo + kBOpBytes), idesc, 0u);
+            lut::mma_stacked(tmem, sbase + kOffA + static_cast<uint32_t>(buf) * LY::kABytes, sbase + LY::kOffB,
+                             lut::stacked_ksteps(L.M, L.g), idesc);
             umma_commit(mma_bar);
           }
           // prefetch the x slice of the range's next (layer, slice) into the other A
           // buffer, whose MMAs completed before the previous table was stored
           const bool more = kbase + run_len < nitems;
           const int nl = (s + 1 < L.S) ? l : l + 1;
-          if (ok && more) load_x_slice(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
-          for (int r = 0; r < rounds; ++r) {
-            if (r > 0 && ok && wtid == 0) {
-              tc_fence_after_sync();
-              for (int mm = 0; mm < 2 && 2 * r + mm < L.M; ++mm)
-                umma_f16_ss(tmem + 256u * mm, adesc, kmajor_desc(bo + static_cast<uint32_t>(2 * r + mm) * kBOpBytes),
-                            idesc, 0u);
-              umma_commit(mma_bar);
-            }
-            const bool done = ok && group_wait(mma_bar, mma_phase, abort_flag, p.status, kSiteGroupMma);
-            mma_phase ^= 1u;
-            // the MMAs have read B: a new layer's codebooks may replace it now
-            if (r == rounds - 1 && done && more && nl != l) load_codebooks(p.layer[nl], sbase, wtid);
-            ok = workers_sync_and(done);
-            tc_fence_after_sync();
-            if (ok && tuned) {
-              // TMEM -> shared-memory table; A rows rho and rho + 64 hold the same group, so
-              // all 16 warps take part: warp w reads lane quadrant w mod 4
-              const int qd = warp & 3;
-              const int col = 32 * (qd & 1) + lane;               // word column = rho mod 64
-              const int i0 = 32 * (2 * (warp >> 2) + (qd >> 1));  // 32 table entries per warp
-              uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kOffLut);
-              uint32_t r0[32], r1[32];
-              tmem_ld_x32(tmem + tmem_lane_base(warp) + static_cast<uint32_t>(i0), r0);
-              tmem_ld_x32(tmem + tmem_lane_base(warp) + 256u + static_cast<uint32_t>(i0), r1);
-  #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                lut[(i0 + j) * 64 + col] = f2_to_h2_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
-            } else if (ok) {
-              generic_table_round(L, s, r, tmem, warp, lane, smem + kOffLut);
-            }
-            tc_fence_before_sync();
-            ok = workers_sync_and(ok);  // this round's table entries stored
-          }
+          if (ok && more) load_x_slice_stacked<kBSteps>(p.layer[nl], (s + 1 < L.S) ? s + 1 : 0, sbase, buf ^ 1, wtid);
+          const bool done = ok && group_wait(mma_bar, mma_phase, abort_flag, p.status, kSiteGroupMma);
+          mma_phase ^= 1u;
+          // the MMAs have read B: a new layer's codebooks may replace it now
+          if (done && more && nl != l) load_codebooks_stacked<kBSteps>(p.layer[nl], sbase, wtid);
           asm volatile("cp.async.commit_group;" ::: "memory");
+          ok = workers_sync_and(done);
+          tc_fence_after_sync();
+          if (ok) lut::store_table_stacked(tmem, warp, lane, smem + kOffLut);
+          tc_fence_before_sync();
+          ok = workers_sync_and(ok);  // table complete
         }
         ++run;
       }
@@ -677,7 +544,7 @@ struct GroupLaunch {
   GroupParams p;
   GroupMaps maps;
   unsigned grid = 0, rgrid = 0;
-  int max_m = 0;          // the largest M of the run: selects the kernel instantiation
+  int max_ksteps = 0;     // the most stacked-build K steps of a layer: selects the instantiation
   bool generic = false;   // some layer is not 2x8 g8
 };
 
@@ -719,7 +586,7 @@ cudaError_t build_group_launch(const Problem* probs, int count, void* workspace,
   GroupMaps& maps = out->maps;
   p = GroupParams{};
   maps = GroupMaps{};
-  out->max_m = 0;
+  out->max_ksteps = 0;
   out->generic = false;
   long long items = 0, rows = 0;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -741,7 +608,7 @@ cudaError_t build_group_launch(const Problem* probs, int count, void* workspace,
     const int row_bytes = L.G * pr.M;
     L.S = (row_bytes + 127) / 128;
     L.T = (pr.N + kTileRows - 1) / kTileRows;
-    out->max_m = std::max(out->max_m, pr.M);
+    out->max_ksteps = std::max(out->max_ksteps, lut::stacked_ksteps(pr.M, pr.g));
     if (pr.M != 2 || pr.g != 8) out->generic = true;
     L.item0 = items;
     L.row0 = rows;
@@ -786,13 +653,13 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
       e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
       if (e != cudaSuccess) return e;
       e = cudaFuncSetAttribute(lut_group_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(GroupLayout<2>::kSmemBytes + 1024u));
+                               static_cast<int>(GroupLayout<2, false>::kSmemBytes + 1024u));
       if (e != cudaSuccess) return e;
       e = cudaFuncSetAttribute(lut_group_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(GroupLayout<2>::kSmemBytes + 1024u));
+                               static_cast<int>(GroupLayout<2, true>::kSmemBytes + 1024u));
       if (e != cudaSuccess) return e;
       e = cudaFuncSetAttribute(lut_group_kernel<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(GroupLayout<4>::kSmemBytes + 1024u));
+                               static_cast<int>(GroupLayout<4, true>::kSmemBytes + 1024u));
       if (e != cudaSuccess) return e;
       g_sms[dev] = std::max(1, sms);
     }
@@ -818,11 +685,14 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  const bool wide = launch.max_m > 2;  // up to four codebooks: the kMaxM = 4 layout
+  const bool wide = launch.max_ksteps > 2;  // M g above 32: the kBSteps = 4 layout
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(launch.grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = (wide ? GroupLayout<4>::kSmemBytes : GroupLayout<2>::kSmemBytes) + 1024u;
+  cfg.dynamicSmemBytes = (wide ? GroupLayout<4, true>::kSmemBytes
+                               : launch.generic ? GroupLayout<2, true>::kSmemBytes
+                                                : GroupLayout<2, false>::kSmemBytes) +
+                         1024u;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
