@@ -73,7 +73,8 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     p.add_argument("--layer", default=None, help="time only this layer of the workload (e.g. q_proj)")
     p.add_argument("--no-other-launch", action="store_true",
-                   help="skip the extra per-layer timing that the group mode reports beside its headline")
+                   help="skip the comparison timings beside the headline: per-layer launches (group mode), "
+                        "launches without CUDA graphs, and aqlm_dequantize + cuBLAS (the context line)")
     p.add_argument("--launch", choices=("group", "per-layer"), default="group",
                    help="one aqlm_matmul_group call per step (default) or one aqlm_matmul call per layer")
     p.add_argument("--scheme", default=None,
@@ -512,6 +513,45 @@ def run_ours(a):
         other = {"launch": "per-layer", "value": job_throughput_gbs(sbytes, o_steps, world, o_ms),
                  "unit": "GB/s", "us_per_layer": o_ms * 1e3 / (o_steps * len(w.layers)), "steps": o_steps}
 
+    direct = context = None
+    if not a.no_other_launch:
+        # launch overhead included: the same steps issued one by one from the host, no graph
+        d_steps = min(a.steps, 2000)
+        step = step_group if mode == "group" else step_per_layer
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                step(i % pool)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(d_steps):
+                step(i % pool)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        d_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        direct = {"launch": mode, "value": job_throughput_gbs(sbytes, d_steps, world, d_ms), "unit": "GB/s",
+                  "us_per_layer": d_ms * 1e3 / (d_steps * len(w.layers)), "steps": d_steps,
+                  "how": "the timed step launched from Python once per step, no CUDA graph"}
+        # context: the dequantise-then-GEMM route on the same layers (W written to HBM by
+        # aqlm_dequantize, then cuBLAS through torch.matmul); not this library's path
+        wbuf = [torch.empty((lay.N, lay.K), dtype=torch.float16, device=dev) for lay in w.layers]
+
+        def step_context(c):
+            for li in range(len(w.layers)):
+                L.dequantize(weights[c][li], out=wbuf[li], stream=stream)
+                torch.matmul(xs[c][li], wbuf[li].t(), out=ys[li])
+
+        c_steps = min(a.steps, 2000)
+        c_ms, _ = timed(step_context, c_steps, 3, False)
+        context = {"what": "aqlm_dequantize + torch.matmul (cuBLAS fp16) per layer", "unit": "GB/s",
+                   "value": job_throughput_gbs(sbytes, c_steps, world, c_ms),
+                   "us_per_layer": c_ms * 1e3 / (c_steps * len(w.layers)), "steps": c_steps,
+                   "how": "algorithmic bytes of the step / time; W itself crosses HBM twice more"}
+        del wbuf
+
     peaks = measured_peaks()
     kernel_names = {int(Path.GEMV): "gemv_gather_kernel", int(Path.GEMV_LUT): "gemv_lut_kernel",
                     int(Path.TENSOR_CORE): "tc_pipe_kernel"}
@@ -618,7 +658,7 @@ def run_ours(a):
                                      + f"; CUDA graphs of {pool} consecutive steps (one pass over the pool)",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu, "cpu_kernel": cpu_kernel, "e2e": e2e,
-                "other_launch": other,
+                "other_launch": other, "no_graph": direct, "context": context,
                 "gpu_launches": launches_per_step * a.steps,
                 "clocks": clock_summary, "gpu": props.name}
         print(json.dumps(line), flush=True)
