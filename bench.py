@@ -274,9 +274,10 @@ def host_layers(w, batch):
     return _HOST_LAYERS[key]
 
 
-def oracle_sample_run(w, batch, seconds, copy=0):
+def oracle_sample_run(w, batch, seconds, copy=0, nthreads=0):
     """Times oracle.linear (decode + fp64 matmul) on row samples of every layer, repeating
-    the sample until about `seconds` of CPU time have been spent.
+    the sample until about `seconds` of CPU time have been spent; nthreads = 0 uses every
+    host core (OpenMP), else that many threads.
     Returns (algorithmic bytes of the sampled fraction, seconds, rows per layer, threads)."""
     import oracle
 
@@ -284,7 +285,8 @@ def oracle_sample_run(w, batch, seconds, copy=0):
     # probe the per-row cost on a few rows of each layer
     t0 = time.perf_counter()
     for lay, ld, x in layers:
-        oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=np.arange(8))
+        oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=np.arange(8),
+                      nthreads=nthreads)
     probe = (time.perf_counter() - t0) / 8.0  # seconds per "one row of every layer"
     rows = max(1, int(seconds / max(probe, 1e-9)))
     total_bytes, elapsed, sampled = 0.0, 0.0, 0
@@ -294,13 +296,26 @@ def oracle_sample_run(w, batch, seconds, copy=0):
             r = min(rows, lay.N)
             sel = np.sort(rng.choice(lay.N, size=r, replace=False))
             t0 = time.perf_counter()
-            oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=sel)
+            oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, ld.M, ld.B, ld.g, rows=sel,
+                          nthreads=nthreads)
             elapsed += time.perf_counter() - t0
             total_bytes += lay.algorithmic_bytes(batch) * (r / lay.N)
         sampled += rows
         if elapsed >= 0.9 * seconds:
             break
-    return total_bytes, elapsed, sampled, oracle.max_threads()
+    return total_bytes, elapsed, sampled, nthreads if nthreads > 0 else oracle.max_threads()
+
+
+def host_cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def cpu_kernel_run(w, batch, seconds):
@@ -636,6 +651,11 @@ def run_ours(a):
                "sample": f"{rows} rows of each of the {len(w.layers)} layers (whole layers repeated "
                          f"when the budget exceeds them; decode to fp16 + fp64 matmul), batch {batch}, "
                          f"{s:.1f} s on the host cores"}
+        cpu["cpu_model"] = host_cpu_model()
+        # the same oracle on one thread, a shorter sample
+        b1, s1, rows1, _ = oracle_sample_run(w, batch, min(3.0, a.cpu_seconds / 4), copy=1, nthreads=1)
+        cpu["single_thread"] = {"value": b1 / s1 / 1e9, "unit": "GB/s", "cores": 1,
+                                "sample": f"{rows1} rows of each layer, {s1:.1f} s on one thread"}
         cpu_kernel = cpu_kernel_run(w, batch, min(a.cpu_seconds, 5.0))
 
     if dist is not None:
