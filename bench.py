@@ -339,7 +339,7 @@ def cpu_kernel_run(w, batch, seconds):
               else "decode to fp32 + dot products")
     return {"value": sbytes * passes / elapsed / 1e9, "unit": "GB/s",
             "ms_per_step": elapsed * 1e3 / passes, "cores": os.cpu_count(),
-            "simd": "avx2+fma+f16c" if cpu_lib.simd_level() == 1 else "scalar",
+            "simd": cpu_lib.SIMD_NAMES.get(cpu_lib.simd_level(), "?"),
             "kind": "libaqlm_cpu.so (aqlm_cpu_matmul)",
             "sample": f"{passes} passes over all {len(w.layers)} whole layers, batch {batch}, {method}, "
                       f"{elapsed:.1f} s"}

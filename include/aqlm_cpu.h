@@ -32,7 +32,7 @@
  * groups and read for every output row (threads take slices and keep per-thread
  * partial sums, added in thread order at the end); otherwise each thread decodes its
  * output rows to fp32 one at a time and takes dot products with every batch row.
- * The result is deterministic for a given nthreads.
+ * The result is deterministic for a given nthreads and SIMD level.
  *
  * nthreads: 0 = the OpenMP default, else that many threads.  The call allocates
  * host scratch (tables, partial sums; released before it returns).
@@ -57,8 +57,14 @@ aqlm_status aqlm_cpu_matmul(const void* x, const void* codes, const void* codebo
                             int M, int B, int g, int K, int N, int batch, int nthreads);
 
 /* SIMD level the kernels run with on this CPU: 0 = portable scalar code,
- * 1 = AVX2 + FMA + F16C. */
+ * 1 = AVX2 + FMA + F16C.  At most the cap set below. */
 int aqlm_cpu_simd_level(void);
+
+/* Caps the SIMD level (clamped to 0..1) for every later call in the process, so
+ * that the scalar code can be run and tested on an AVX2 CPU; the default cap is 1.
+ * Returns the previous cap.  Not meant to be changed while another thread is inside
+ * aqlm_cpu_matmul. */
+int aqlm_cpu_set_max_simd_level(int level);
 
 /* ABI version of this header. */
 int aqlm_cpu_abi_version(void);

@@ -4,7 +4,9 @@ The same bar as the GPU path: max|y - y_ref| / max|y_ref| <= 5e-3 against the
 oracle's fp64 reference of the decoded fp16 weights, no NaN/Inf, for every
 supported scheme on both methods (lookup tables for B = 8 at batch <= 8, decode +
 dot otherwise); integer-valued layers bit for bit; the same bits run to run for a
-given thread count; argument errors before any work.  No GPU is involved.
+given thread count; argument errors before any work.  The numeric tests run at every
+SIMD level this CPU has (scalar, AVX2), selected with the library's process-wide
+cap.  No GPU is involved.
 """
 import ctypes
 import os
@@ -29,6 +31,19 @@ def built():
     cpu.lib()
 
 
+@pytest.fixture(params=[0, 1], ids=["scalar", "avx2"])
+def simd(request):
+    """Runs the test with the SIMD level capped at the parameter (skipped where the CPU
+    lacks it); the previous cap is restored afterwards."""
+    prev = cpu.set_max_simd_level(request.param)
+    try:
+        if cpu.simd_level() != request.param:
+            pytest.skip(f"this CPU has no SIMD level {request.param}")
+        yield request.param
+    finally:
+        cpu.set_max_simd_level(prev)
+
+
 def close(y, ref, what):
     assert np.isfinite(y.astype(np.float32)).all(), what
     err = float(np.abs(y.astype(np.float64) - ref).max() / max(np.abs(ref).max(), 1e-30))
@@ -46,19 +61,19 @@ def test_header_declares_the_binding_exports():
 
 @pytest.mark.parametrize("M,B,g", SCHEMES)
 @pytest.mark.parametrize("batch", [1, 3, 8, 9])
-def test_cpu_matmul_matches_oracle(M, B, g, batch):
+def test_cpu_matmul_matches_oracle(M, B, g, batch, simd):
     N, K = 150, 16 * 37  # several table slices and a partial one; ragged rows
     ld = synth.make_layer(M, B, g, K, N, seed=80, layer=batch, with_bias=batch % 2 == 1)
     x = synth.make_x(batch, K, seed=81, layer=M)
     ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
     for nt in (1, 4):
         close(cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g, nthreads=nt), ref,
-              f"{M}x{B} g{g} b={batch} threads={nt}")
+              f"{M}x{B} g{g} b={batch} threads={nt} simd={simd}")
 
 
 @pytest.mark.parametrize("M,B,g", SCHEMES)
 @pytest.mark.parametrize("batch", [1, 20])
-def test_cpu_matmul_integer_layers_bit_exact(M, B, g, batch):
+def test_cpu_matmul_integer_layers_bit_exact(M, B, g, batch, simd):
     N, K = 70, 512
     rng = np.random.Generator(np.random.PCG64(82 + M + g + B))
     cb = rng.integers(-2, 3, size=(M, 1 << B, g)).astype(np.float16)
@@ -73,7 +88,7 @@ def test_cpu_matmul_integer_layers_bit_exact(M, B, g, batch):
         assert np.array_equal(y, ref), (nt, int((y != ref).sum()))
 
 
-def test_cpu_matmul_full_size_layer_sampled_rows():
+def test_cpu_matmul_full_size_layer_sampled_rows(simd):
     """A Llama-2-7B down_proj-shaped layer (4096 x 11008), 2x8 g8, batch 1."""
     ld = synth.make_layer(2, 8, 8, 11008, 4096, seed=83)
     x = synth.make_x(1, 11008, seed=83)
@@ -83,7 +98,7 @@ def test_cpu_matmul_full_size_layer_sampled_rows():
     close(y[:, rows], ref, "4096x11008 2x8 g8")
 
 
-def test_cpu_matmul_deterministic_for_a_thread_count():
+def test_cpu_matmul_deterministic_for_a_thread_count(simd):
     ld = synth.make_layer(2, 8, 8, 4096, 512, seed=85)
     x = synth.make_x(2, 4096, seed=85)
     a = cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, None, 2, 8, 8, nthreads=4)

@@ -22,8 +22,8 @@ class AqlmCpuError(RuntimeError):
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIBRARY = os.path.join(PKG, "libaqlm_cpu.so")
 
-EXPORTS = ("aqlm_cpu_matmul", "aqlm_cpu_simd_level", "aqlm_cpu_abi_version")
-ABI_VERSION = 1
+EXPORTS = ("aqlm_cpu_matmul", "aqlm_cpu_simd_level", "aqlm_cpu_set_max_simd_level", "aqlm_cpu_abi_version")
+ABI_VERSION = 2
 
 _lib = None
 _lock = threading.Lock()
@@ -42,6 +42,8 @@ def lib() -> ctypes.CDLL:
                 L.aqlm_cpu_matmul.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i]
                 L.aqlm_cpu_matmul.restype = _i
                 L.aqlm_cpu_simd_level.restype = _i
+                L.aqlm_cpu_set_max_simd_level.argtypes = [_i]
+                L.aqlm_cpu_set_max_simd_level.restype = _i
                 L.aqlm_cpu_abi_version.restype = _i
                 if L.aqlm_cpu_abi_version() != ABI_VERSION:
                     raise ImportError(f"libaqlm_cpu.so ABI {L.aqlm_cpu_abi_version()} != binding ABI {ABI_VERSION}")
@@ -50,7 +52,17 @@ def lib() -> ctypes.CDLL:
 
 
 def simd_level() -> int:
+    """0 = scalar, 1 = AVX2 + FMA + F16C."""
     return lib().aqlm_cpu_simd_level()
+
+
+def set_max_simd_level(level: int) -> int:
+    """Caps the SIMD level for the whole process (tests, comparisons); returns the
+    previous cap."""
+    return lib().aqlm_cpu_set_max_simd_level(int(level))
+
+
+SIMD_NAMES = {0: "scalar", 1: "avx2+fma+f16c"}
 
 
 def _arr(a, dtype):

@@ -17,11 +17,14 @@
 // fp32 accumulation everywhere; y = fp16_rne(s_n * acc + bias_n).
 //
 // The AVX2 functions carry target attributes and run only when the CPU reports
-// AVX2, FMA and F16C; otherwise portable scalar versions of the same loops run.
+// AVX2, FMA and F16C; otherwise portable scalar versions of the same loops run.  A
+// process-wide cap (aqlm_cpu_set_max_simd_level) selects the scalar code on such a
+// CPU too, for tests and comparisons.
 #include <immintrin.h>
 #include <omp.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <vector>
@@ -90,6 +93,15 @@ bool cpu_has_avx2() {
   static const bool ok = __builtin_cpu_supports("avx2") && __builtin_cpu_supports("fma") &&
                          __builtin_cpu_supports("f16c");
   return ok;
+}
+
+std::atomic<int> g_max_simd{1};
+
+// 0 = scalar, 1 = AVX2 + FMA + F16C: what the CPU has, capped by
+// aqlm_cpu_set_max_simd_level.
+int simd_level() {
+  const int hw = cpu_has_avx2() ? 1 : 0;
+  return std::min(hw, g_max_simd.load());
 }
 
 struct Layer {
@@ -186,7 +198,7 @@ void run_lut(const Layer& L, const float* xf, int nt) {
   const int S = (L.G + kSlice - 1) / kSlice;
   nt = std::max(1, std::min(nt, S));
   std::vector<std::vector<float>> partial(static_cast<size_t>(nt));
-  const bool avx2 = cpu_has_avx2();
+  const int level = simd_level();
 #pragma omp parallel num_threads(nt)
   {
     const int tid = omp_get_thread_num();
@@ -196,7 +208,7 @@ void run_lut(const Layer& L, const float* xf, int nt) {
     for (int s = 0; s < S; ++s) {
       if (part.empty()) part.assign(static_cast<size_t>(L.batch) * L.N, 0.f);
       const int j0 = s * kSlice, nj = std::min(kSlice, L.G - j0);
-      if (avx2)
+      if (level == 1)
         build_tables_avx2(L, xf, ct.data(), j0, nj, T.data());
       else
         build_tables_scalar(L, xf, ct.data(), j0, nj, T.data());
@@ -275,7 +287,7 @@ void dots_scalar(const float* xb, const float* w, int rows, int K, float* dots) 
 }
 
 void run_decode_dot(const Layer& L, const float* xf, int nt) {
-  const bool avx2 = cpu_has_avx2();
+  const bool avx2 = simd_level() >= 1;
   const int64_t blocks = (L.N + kRowBlock - 1) / kRowBlock;
 #pragma omp parallel num_threads(nt)
   {
@@ -323,9 +335,13 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 extern "C" {
 
-int aqlm_cpu_abi_version(void) { return 1; }
+int aqlm_cpu_abi_version(void) { return 2; }
 
-int aqlm_cpu_simd_level(void) { return cpu_has_avx2() ? 1 : 0; }
+int aqlm_cpu_simd_level(void) { return simd_level(); }
+
+int aqlm_cpu_set_max_simd_level(int level) {
+  return g_max_simd.exchange(std::max(0, std::min(1, level)));
+}
 
 aqlm_status aqlm_cpu_matmul(const void* x, const void* codes, const void* codebooks,
                             const void* scales, const void* bias, void* y,
