@@ -223,7 +223,7 @@ GENERIC = [
     (2, 8, 16, 2048, 300, 1, False),    # 1 bit
     (3, 8, 8, 1024, 257, 1, True),      # 3 bit: groups straddle the 128-byte slices
     (3, 8, 16, 2048, 130, 1, False),    # 1.5 bit
-    (4, 8, 8, 1024, 64, 1, True),       # 4 bit: two MMA rounds per table
+    (4, 8, 8, 1024, 64, 1, True),       # 4 bit: two K steps in the stacked table build
     (4, 8, 16, 4096, 200, 1, False),
     (2, 8, 8, 1024, 129, 1, True),      # the tuned 2x8 g8 path in the same launch
 ]
@@ -231,7 +231,7 @@ GENERIC = [
 
 def test_group_generic_schemes_match_oracle(dev):
     """Every B = 8 scheme as grouped lookup-table layers, several in one launch (with
-    four-codebook layers present the launch uses the four-codebook layout)."""
+    layers of M g > 32 present the launch uses the four-K-step layout)."""
     grp, lds, xs, outs = build_group(GENERIC, dev, seed=47)
     grp.run()
     check_status()
@@ -242,7 +242,8 @@ def test_group_generic_schemes_match_oracle(dev):
 
 @pytest.mark.parametrize("M,g", [(1, 8), (1, 16), (2, 16), (3, 8), (3, 16), (4, 8), (4, 16)])
 def test_group_generic_scheme_alone(dev, M, g):
-    """One scheme per launch (the two-codebook layout for M <= 2), ragged rows."""
+    """One scheme per launch (the two-K-step layout for M g <= 32, else four), ragged
+    rows."""
     spec = [(M, 8, g, 2048, 333, 1, True), (M, 8, g, 1024, 64, 1, False)]
     grp, lds, xs, outs = build_group(spec, dev, seed=48 + M + g)
     grp.run()
@@ -250,6 +251,19 @@ def test_group_generic_scheme_alone(dev, M, g):
     for (M_, B, g_, K, N, batch, _), ld, x, out in zip(spec, lds, xs, outs):
         y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M_, B, g_)
         assert_close(out.cpu().numpy(), y_ref, f"{M_}x{B}g{g_} K={K} N={N}")
+
+
+def test_group_two_step_layout_mixed_schemes(dev):
+    """Schemes of one and two K steps (M g <= 32) sharing the two-K-step layout, the
+    codebooks reloaded with a different step count at every layer change."""
+    spec = [(4, 8, 8, 2048, 300, 1, True), (1, 8, 16, 4096, 130, 1, False), (3, 8, 8, 1024, 200, 1, False),
+            (2, 8, 16, 2048, 64, 1, True), (2, 8, 8, 1024, 100, 1, False), (4, 8, 8, 1024, 70, 1, False)]
+    grp, lds, xs, outs = build_group(spec, dev, seed=46)
+    grp.run()
+    check_status()
+    for (M, B, g, K, N, batch, _), ld, x, out in zip(spec, lds, xs, outs):
+        y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+        assert_close(out.cpu().numpy(), y_ref, f"group {M}x{B}g{g} K={K} N={N}")
 
 
 @pytest.mark.parametrize("M,g", [(1, 8), (3, 8), (4, 16)])
