@@ -52,8 +52,8 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxPasses = 4;                      // code rows <= 16 CTAs x 4 passes x 128 bytes
 constexpr int kTileRows = 64;                      // rows per code tile (one TMA box)
 constexpr uint32_t kLutBytes = lut::kTableBytes;   // 64 KB
-constexpr uint32_t kAOpBytes = lut::kAOpBytes;     // 4 KB per pass
-constexpr uint32_t kBOpBytes = lut::kBOpBytes;     // 8 KB per codebook
+constexpr uint32_t kAOpBytes = lut::kAOpBytes;     // 4 KB per pass and K step
+constexpr uint32_t kBOpBytes = lut::kBOpBytes;     // 8 KB per codebook (tuned) or K step (stacked)
 constexpr uint32_t kTileBytes = 64u * 128u;        // 64 rows x 128 B of codes (one TMA box)
 constexpr uint32_t kTmemCols = 512;                // D_0 at [0,256), D_1 at [256,512)
 constexpr uint32_t kSmemLimit = 227u * 1024u;
@@ -170,7 +170,8 @@ __device__ __noinline__ void issue_code_tiles(const CUtensorMap* map, uint32_t t
 // kGeneric = false: 2x8 g8 (the tuned table build); true: any B = 8 scheme.
 // kRecycle = false: all P ntile code tiles of a CTA are resident (R = P ntile);
 // true: fewer slots, reloaded pass after pass.  Separate instantiations, since the
-// reload bookkeeping costs the resident case ~5 % (its lookup loop's code changes).
+// reload bookkeeping cost the resident case 3-20 % when it was one kernel (its lookup
+// loop's code changes).
 template <bool kGeneric, bool kRecycle>
 __global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const __grid_constant__ CUtensorMap code_map,
                                                                 const LutParams p) {
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const __grid_cons
   // The next kernel in the stream may start its own weight-only set-up now.
   grid_dependents_launch();
 
-  // ---- 1. barriers; one thread starts the whole code stream (a TMA box per tile) --------
+  // ---- 1. barriers; one thread starts the code stream (a TMA box per tile) ---------------
   if (tid == 0) {
     for (int i = 0; i < p.P * p.ntile; ++i) mbar_init(&tile_bar[i], 1);
     mbar_init(mma_bar, 1);
