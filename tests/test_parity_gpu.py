@@ -132,10 +132,11 @@ def test_tensor_core_parity(dev, M, B, g, N, K, batch):
 
 
 @pytest.mark.parametrize("N,K", [(1, 64), (37, 128), (200, 512), (300, 4096), (129, 64 * 23),
-                                 (1000, 11008), (700, 14336), (4100, 4096)])
+                                 (1000, 11008), (700, 14336), (4100, 4096), (2048, 32768)])
 def test_gemv_lut_parity(dev, N, K):
     """Lookup-table GEMV (2x8, batch 1): ragged row counts, K from one pass to
-    several passes per CTA, cluster sizes from 1 to 16."""
+    several passes per CTA, cluster sizes from 1 to 16; 2048 x 32768 (the longest rows,
+    four passes per CTA) does not keep every code tile resident and recycles slots."""
     ld = synth.make_layer(2, 8, 8, K, N, seed=17, layer=N, with_bias=(N % 2 == 1))
     x = synth.make_x(1, K, seed=17, layer=N)
     y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, 2, 8, 8)
