@@ -231,7 +231,8 @@ def test_device_status_clean_after_all(dev):
 
 @pytest.mark.parametrize("M,B,g,path,batch", [(2, 8, 8, Path.GEMV_LUT, 1), (2, 8, 8, Path.GEMV, 3),
                                               (1, 16, 8, Path.GEMV, 1), (1, 16, 16, Path.GEMV, 4),
-                                              (1, 16, 8, Path.TENSOR_CORE, 64), (2, 8, 8, Path.TENSOR_CORE, 32)])
+                                              (1, 16, 8, Path.TENSOR_CORE, 64), (2, 8, 8, Path.TENSOR_CORE, 32),
+                                              (3, 8, 16, Path.GEMV_LUT, 1), (4, 8, 8, Path.GEMV_LUT, 1)])
 def test_chained_layers_read_the_previous_output(dev, M, B, g, path, batch):
     """Kernels start their weight-only set-up while the previous kernel on the stream
     is still running (programmatic dependent launch); x must still be read only after
