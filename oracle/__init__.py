@@ -61,8 +61,6 @@ def _bind(path: str):
     lib.oracle_float_bits_to_half_range.argtypes = [ctypes.c_uint32, _i64, _u16p]
     lib.oracle_dequantize.argtypes = [_vp, _u16p, _u16p, _u16p, _i, _i, _i, _i, _i, _i]
     lib.oracle_dequantize.restype = _i
-    lib.oracle_matmul_dense.argtypes = [_u16p, _u16p, _u16p, _f64p, _i, _i, _i, _i]
-    lib.oracle_matmul_dense.restype = _i
     lib.oracle_linear_rows.argtypes = [_u16p, _vp, _u16p, _u16p, _u16p, _f64p,
                                        _i, _i, _i, _i, _i, _i, _i64p, _i64, _i]
     lib.oracle_linear_rows.restype = _i
@@ -176,17 +174,6 @@ def dequantize(codes, codebooks, scales, M: int, B: int, g: int, nthreads: int =
     _check(_load().oracle_dequantize(codes.ctypes.data, _p(cb, _u16p), _p(sc, _u16p),
                                      _p(out, _u16p), M, B, g, K, N, nthreads))
     return out
-
-
-def matmul_dense(x, W16, bias=None, nthreads: int = 0) -> np.ndarray:
-    x, W = _bits16(x), _bits16(W16)
-    batch, K = x.shape
-    N = W.shape[0]
-    bi = _bits16(bias) if bias is not None else None
-    y = np.empty((batch, N), np.float64)
-    _check(_load().oracle_matmul_dense(_p(x, _u16p), _p(W, _u16p), _p(bi, _u16p),
-                                       _p(y, _f64p), K, N, batch, nthreads))
-    return y
 
 
 def linear(x, codes, codebooks, scales, bias, M: int, B: int, g: int,

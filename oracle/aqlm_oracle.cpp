@@ -206,26 +206,6 @@ int oracle_dequantize(const void* codes, const uint16_t* codebooks, const uint16
   return 0;
 }
 
-// y[b, n] = sum_{k ascending} f64(x[b,k]) * f64(W16[n,k]) + f64(bias[n])  (fp64).
-int oracle_matmul_dense(const uint16_t* x, const uint16_t* W16, const uint16_t* bias,
-                        double* y, int K, int N, int batch, int nthreads) {
-  if (!x || !W16 || !y || K < 1 || N < 1 || batch < 1) return 1;
-  const int nt = pick_threads(nthreads);
-#pragma omp parallel for schedule(static) num_threads(nt)
-  for (int64_t n = 0; n < N; ++n) {
-    for (int64_t b = 0; b < batch; ++b) {
-      double acc = 0.0;
-      for (int64_t k = 0; k < K; ++k) {
-        acc += static_cast<double>(half_bits_to_float(x[b * K + k])) *
-               static_cast<double>(half_bits_to_float(W16[n * K + k]));
-      }
-      if (bias) acc += static_cast<double>(half_bits_to_float(bias[n]));
-      y[b * N + n] = acc;
-    }
-  }
-  return 0;
-}
-
 // Reference output: decode each requested row to fp16 (the dequantisation
 // definition), then the fp64 dot product with every batch row.
 // rows == NULL means all N rows in order; y is [batch, nrows].
