@@ -5,13 +5,23 @@
                     [--workload NAME]
 
 A step is one pass of the AQLM linear layers of a workload over one batch of
-synthetic activations.  The default workload is the Llama-2-7B decoder layer
-set (q, k, v, o 4096x4096; gate, up 11008x4096; down 4096x11008), 2x8 g8
-codebooks (2 bits per weight), batch 1.  By default (--launch group) a step is
-one aqlm_matmul_group call over the set (the grouped lookup-table kernel and its
-reduction, two launches); --launch per-layer makes it one aqlm_matmul call per
-layer.  The group run also times the per-layer launches and reports them beside
-the headline.
+synthetic activations.  The default workload (the headline) is the largest of the
+published configurations: the Mixtral-8x7B expert FFNs of one layer, 8 experts x
+(w1, w3 14336x4096; w2 4096x14336), 2x8 g8 codebooks (2 bits per weight), batch 1
+per expert, 354 MB of codes per step.  By default (--launch group) a step is one
+aqlm_matmul_group call over the set (the grouped lookup-table kernel and its
+reduction); --launch per-layer makes it one aqlm_matmul call per layer.  The group
+run also times the per-layer launches and reports them beside the headline.
+
+After the headline (N = 1, default workload) the other published configurations
+are measured the same way, one record each under "per_config": the 4096x4096 1x16
+g8 layer, the Llama-2-7B 2x8 g8 set, the Llama-2-70B 1x16 g8 shapes at batch 1 and
+4, the batch sweep 1..256 on 11008x4096 and 4096x11008 per scheme, and the
+Mixtral-8x7B experts in 1x16 g16.  Every record carries its roofline against the
+binding roof, the one with the longest ideal time for the step: HBM (algorithmic
+bytes / measured copy bandwidth), tensor (2 batch N K flops / measured bf16 rate)
+or, for the 65536-entry codebooks, the L1TEX gather rate (one random codeword
+request per SM and clock); every roof's fraction is listed beside it.
 
 Metric: effective HBM GB/s = algorithmic bytes (codes + codebooks + scales + x +
 y, each once) / device time, summed over ranks; microseconds per layer are
@@ -19,7 +29,8 @@ reported beside it.  Inputs are resident in HBM; every step reads a different
 copy of the layer set from a rotating pool larger than 3x the L2 cache, so no
 step finds its weights in L2.  The steps run as replays of CUDA graphs that
 each hold one pass over the pool (launches inside a graph overlap through
-programmatic dependent launch); the timed region is bracketed by a barrier and a device
+programmatic dependent launch); every graph the timed region uses is replayed
+once before it.  The timed region is bracketed by a barrier and a device
 synchronise and measured with CUDA events on the launching stream; the max over
 ranks is taken.  With N > 1 GPUs each rank runs its own replica (weak scaling,
 no data-path collective).
@@ -54,7 +65,7 @@ if ROOT not in sys.path:
 from weight_only_additive_b200 import synth, workloads  # noqa: E402
 
 METRIC = "AQLM matmul µs/layer & achieved HBM GB/s (frac. of ~8 TB/s), batch 1–256"
-DEFAULT_WORKLOAD = "llama2_7b_layer_set_2x8g8"
+DEFAULT_WORKLOAD = "mixtral_8x7b_experts_2x8g8"
 L2_FALLBACK = 126 * 1024 * 1024
 
 
@@ -62,7 +73,7 @@ def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=None,
-                   help="timed steps (default 100000; 1000 with --op input-grad)")
+                   help="timed steps (default 20000; 1000 with --op input-grad)")
     p.add_argument("--warmup", type=int, default=1000)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.BY_NAME))
@@ -70,6 +81,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="skip the records of the other published configurations after the headline")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     p.add_argument("--layer", default=None, help="time only this layer of the workload (e.g. q_proj)")
     p.add_argument("--no-other-launch", action="store_true",
@@ -85,7 +98,7 @@ def parse_args(argv=None):
                    help="rotating-pool copies (default: enough to exceed 3x L2); smaller for profiler captures")
     a = p.parse_args(argv)
     if a.steps is None:
-        a.steps = 1000 if a.op == "input-grad" else 100000
+        a.steps = 1000 if a.op == "input-grad" else 20000
     if a.warmup < 3:
         p.error("--warmup must be at least 3")
     return a
@@ -100,13 +113,18 @@ def env_rank():
 
 
 def measured_peaks():
+    """Roofline denominators: MEASURED_PEAKS.json (the machine's measured copy bandwidth and
+    cuBLAS bf16 rates; fp16 has the same nominal tensor rate), else the fallback figures."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as fh:
             d = json.load(fh)
         return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured",
-                "tc_tflops_sustained": float(d.get("bf16_tflops_sustained", 1400.0))}
-    return {"hbm_gbs": 6650.0, "source": "fallback", "tc_tflops_sustained": 1400.0}
+                "tc_tflops": float(d.get("bf16_tflops", 1590.0)),
+                "tc_tflops_sustained": float(d.get("bf16_tflops_sustained", 1400.0)),
+                "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0))}
+    return {"hbm_gbs": 6650.0, "source": "fallback", "tc_tflops": 1590.0, "tc_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0}
 
 
 # the files under csrc/ each kernel is compiled from (its .cu first, then the headers
@@ -380,151 +398,321 @@ def run_reference(a):
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
-def run_ours(a):
-    import torch
+# One L1TEX request per SM and clock: the rate at which an SM serves gathers of
+# random 16-byte (or, with a 256-bit load, 32-byte) codewords from the L2-resident
+# 65536-entry codebooks.  Derived from the unit count (one L1TEX unit per SM) and
+# the SM clock; probes of random 16-byte gathers on this GPU measured 0.73-1.0.
+GATHERS_PER_SM_CLOCK = 1.0
 
-    from weight_only_additive_b200 import layer as L
-    from weight_only_additive_b200 import native
-    from weight_only_additive_b200.native import Path
+# The published configurations measured after the headline at N = 1, each as
+# (workload, scheme filter or None, batch).  The batch sweep holds two schemes and is
+# measured per scheme, so every record has one binding roof.
+PER_CONFIG = (("single_4096x4096_1x16g8", None, 1),
+              ("llama2_7b_layer_set_2x8g8", None, 1),
+              ("llama2_70b_layers_1x16g8", None, 1),
+              ("llama2_70b_layers_1x16g8", None, 4),
+              *(("batch_sweep_11008x4096", "1x16g8", b) for b in (1, 4, 16, 64, 256)),
+              *(("batch_sweep_11008x4096", "2x8g8", b) for b in (1, 4, 16, 64, 256)),
+              ("mixtral_8x7b_experts_1x16g16", None, 1),
+              ("mixtral_8x7b_experts_2x8g8", None, 1))
 
-    rank, world, local = env_rank()
-    if world > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        dist = None
-        torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    lib = native.lib()
 
-    w = select_workload(a)
-    batch = workload_batch(w, a.batch)
-    sbytes = step_bytes(w, batch)
-    props = torch.cuda.get_device_properties(dev)
-    l2 = getattr(props, "L2_cache_size", 0) or L2_FALLBACK
-    copy_bytes = sum(l.algorithmic_bytes(batch) for l in w.layers)
-    pool = max(2, math.ceil(3 * l2 / copy_bytes)) if a.pool is None else max(1, a.pool)
-    while pool > 2 and pool * copy_bytes > 60e9:
-        pool -= 1
+def scheme_subset(w, scheme_name):
+    """The workload restricted to the layers of one codebook scheme."""
+    layers = tuple(l for l in w.layers if l.scheme.name == scheme_name)
+    if not layers:
+        raise SystemExit(f"{w.name} has no {scheme_name} layer")
+    return workloads.Workload(w.index, f"{w.name}[{scheme_name}]", layers, w.batches, w.description)
 
-    # device-resident pool: pool copies of every layer's weights and activations
-    weights, xs = [], []
-    for c in range(pool):
-        wc, xc = [], []
-        for li, lay in enumerate(w.layers):
-            s = lay.scheme
-            ld = synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index,
-                                  layer=li + w.extra.get("layer_offset", 0), copy=c + 1000 * rank)
-            wc.append(L.AqlmWeights.from_numpy(ld, dev))
-            xc.append(torch.from_numpy(synth.make_x(batch, lay.K, seed=0, workload=w.index, layer=li,
-                                                    copy=c + 1000 * rank)).to(dev))
-        weights.append(wc)
-        xs.append(xc)
-    ys = [torch.empty((batch, lay.N), dtype=torch.float16, device=dev) for lay in w.layers]
-    paths = [native.aqlm_select_path(l.scheme.M, l.scheme.B, l.scheme.g, l.K, l.N, batch) for l in w.layers]
 
-    stream = torch.cuda.Stream(dev)
-    h = stream.cuda_stream
-    # per-layer mode: raw argument tuples, one C-ABI call per layer
-    calls = []
-    for c in range(pool):
-        cc = []
-        for li, lay in enumerate(w.layers):
-            wt = weights[c][li]
-            cc.append((xs[c][li].data_ptr(), wt.codes.data_ptr(), wt.codebooks.data_ptr(),
-                       wt.scales.data_ptr(), None, ys[li].data_ptr(), wt.M, wt.B, wt.g, lay.K, lay.N,
-                       batch, h))
-        calls.append(cc)
-    # group mode: one aqlm_matmul_group call per step (problem table + workspace per copy)
-    groups = [L.LayerGroup([(weights[c][li], xs[c][li], ys[li]) for li in range(len(w.layers))])
-              for c in range(pool)]
+def step_roofs(w, batch, peaks, sms, sm_mhz):
+    """The three roofs of one step, each as (time in s, quantity, peak rate, unit):
+    HBM (algorithmic bytes), tensor (2 batch N K flops at the measured burst bf16 rate;
+    fp16 has the same nominal rate) and the codeword gathers of the B = 16 schemes (one
+    request per codeword per code, GATHERS_PER_SM_CLOCK per SM and clock)."""
+    nbytes = step_bytes(w, batch)
+    flops = sum(l.flops(batch) for l in w.layers)
+    gathers = sum(l.N * l.G * l.scheme.M for l in w.layers if l.scheme.B == 16)
+    gather_rate = GATHERS_PER_SM_CLOCK * sms * sm_mhz * 1e6
+    return {"hbm": (nbytes / (peaks["hbm_gbs"] * 1e9), nbytes / 1e9, peaks["hbm_gbs"], "GB/s"),
+            "tensor": (flops / (peaks["tc_tflops"] * 1e12), flops / 1e12, peaks["tc_tflops"], "TFLOP/s"),
+            "l1tex_gather": (gathers / gather_rate, gathers / 1e9, gather_rate / 1e9, "Greq/s")}
 
-    def step_per_layer(c):
-        for args in calls[c]:
-            st = lib.aqlm_matmul(*args)
+
+def roofline_record(w, batch, step_s, peaks, sms, sm_mhz):
+    """`roofline` of a step: the binding roof (the one with the longest ideal time),
+    achieved = its quantity per step / the measured step time, against its peak; and
+    every roof's fraction beside it."""
+    roofs = step_roofs(w, batch, peaks, sms, sm_mhz)
+    bound = max(roofs, key=lambda k: roofs[k][0])
+    out = {}
+    for name, (t, qty, peak, unit) in roofs.items():
+        if qty == 0:
+            continue
+        achieved = qty / step_s
+        out[name] = {"achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                     "ideal_us": t * 1e6}
+    rec = {"bound": bound, **{k: out[bound][k] for k in ("achieved", "peak", "unit", "frac")},
+           "roofs": out}
+    src = "measured (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"
+    rec["peak_source"] = {"hbm": f"{src} hbm_gbs", "tensor": f"{src} bf16_tflops (burst)",
+                          "l1tex_gather": f"{GATHERS_PER_SM_CLOCK:g} request per SM per clock x {sms} SMs x "
+                                          f"{sm_mhz:.0f} MHz"}[bound]
+    return rec
+
+
+class Bench:
+    """The device, stream and library shared by every measurement of one run."""
+
+    def __init__(self, a):
+        import torch
+
+        from weight_only_additive_b200 import layer as L
+        from weight_only_additive_b200 import native
+
+        self.torch, self.L, self.native = torch, L, native
+        self.rank, self.world, self.local = env_rank()
+        if self.world > 1:
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.dist = dist
+        else:
+            self.dist = None
+            torch.cuda.set_device(self.local)
+        self.dev = torch.device("cuda", self.local)
+        self.lib = native.lib()
+        self.props = torch.cuda.get_device_properties(self.dev)
+        self.l2 = getattr(self.props, "L2_cache_size", 0) or L2_FALLBACK
+        self.sms = self.props.multi_processor_count
+        self.stream = torch.cuda.Stream(self.dev)
+        self.peaks = measured_peaks()
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+
+class Pool:
+    """A rotating pool of seeded copies of a workload's layers, resident in HBM and
+    larger than 3x L2, with one aqlm_matmul_group problem table (and workspace) per copy."""
+
+    def __init__(self, b, w, batch, copies=None):
+        torch, L = b.torch, b.L
+        self.w, self.batch = w, batch
+        copy_bytes = step_bytes(w, batch)
+        pool = max(2, math.ceil(3 * b.l2 / copy_bytes)) if copies is None else max(1, copies)
+        while pool > 2 and pool * copy_bytes > 60e9:
+            pool -= 1
+        self.size, self.copy_bytes = pool, copy_bytes
+        self.weights, self.xs = [], []
+        off = w.extra.get("layer_offset", 0)
+        for c in range(pool):
+            wc, xc = [], []
+            for li, lay in enumerate(w.layers):
+                s = lay.scheme
+                ld = synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index,
+                                      layer=li + off, copy=c + 1000 * b.rank)
+                wc.append(L.AqlmWeights.from_numpy(ld, b.dev))
+                xc.append(torch.from_numpy(synth.make_x(batch, lay.K, seed=0, workload=w.index, layer=li,
+                                                        copy=c + 1000 * b.rank)).to(b.dev))
+            self.weights.append(wc)
+            self.xs.append(xc)
+        self.ys = [torch.empty((batch, lay.N), dtype=torch.float16, device=b.dev) for lay in w.layers]
+        self.groups = [L.LayerGroup([(self.weights[c][li], self.xs[c][li], self.ys[li])
+                                     for li in range(len(w.layers))]) for c in range(pool)]
+        h = b.stream.cuda_stream
+        self.calls = [[(self.xs[c][li].data_ptr(), wt.codes.data_ptr(), wt.codebooks.data_ptr(), wt.scales.data_ptr(),
+                        None, self.ys[li].data_ptr(), wt.M, wt.B, wt.g, lay.K, lay.N, batch, h)
+                       for li, (lay, wt) in enumerate(zip(w.layers, self.weights[c]))] for c in range(pool)]
+        self.b = b
+
+    def step_group(self, c):
+        self.groups[c].run(stream=self.b.stream)
+
+    def step_per_layer(self, c):
+        for args in self.calls[c]:
+            st = self.b.lib.aqlm_matmul(*args)
             if st != 0:
-                raise native.AqlmError(st, "aqlm_matmul")
+                raise self.b.native.AqlmError(st, "aqlm_matmul")
 
-    def step_group(c):
-        groups[c].run(stream=stream)
+    def grouped_layers(self):
+        return sum(1 for l in self.w.layers if l.scheme.B == 8 and self.batch == 1 and l.K % l.scheme.g == 0
+                   and (l.K // l.scheme.g * l.scheme.M) % 16 == 0)
 
-    def launches(mode):
+    def launches(self, mode):
         """Kernel launches of one step: the grouped layers take two (partial sums and
-        reduction) per run of up to 16; every other layer one."""
+        reduction) per run of up to MAX_GROUP_LAYERS; every other layer one."""
+        n = len(self.w.layers)
         if mode == "per-layer":
-            return len(w.layers)
-        grouped = sum(1 for l in w.layers if l.scheme.B == 8 and batch == 1 and l.K % l.scheme.g == 0
-                      and (l.K // l.scheme.g * l.scheme.M) % 16 == 0)
-        return 2 * ((grouped + 15) // 16) + (len(w.layers) - grouped)
+            return n
+        grouped = self.grouped_layers()
+        runs = (grouped + self.b.native.MAX_GROUP_LAYERS - 1) // self.b.native.MAX_GROUP_LAYERS
+        return 2 * runs + (n - grouped)
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
+    def kernel(self, mode):
+        if mode == "group" and self.grouped_layers() == len(self.w.layers):
+            return "lut_group_kernel"
+        lay = self.w.layers[0]
+        path = self.b.native.aqlm_select_path(lay.scheme.M, lay.scheme.B, lay.scheme.g, lay.K, lay.N, self.batch)
+        P = self.b.native.Path
+        return {int(P.GEMV): "gemv_gather_kernel", int(P.GEMV_LUT): "gemv_lut_kernel",
+                int(P.TENSOR_CORE): "tc_pipe_kernel"}.get(int(path), "?")
 
-    def timed(step, steps, warmup, sample_clocks):
-        """K steps as replays of CUDA graphs that each hold one pass over the pool
-        (pool consecutive steps, copy c at step c), plus one graph for the remainder;
-        launches inside a graph overlap through programmatic dependent launch."""
-        with torch.cuda.stream(stream):
+    def timed(self, step, steps, warmup, sample_clocks=False):
+        """`steps` steps as replays of CUDA graphs that each hold one pass over the pool
+        (copy c at step c), plus one graph for the remainder; launches inside a graph
+        overlap through programmatic dependent launch.  Every graph the timed region
+        replays is captured and replayed at least once before it, whatever `warmup` is,
+        so no first-replay cost lands in the timed region."""
+        b, torch, pool = self.b, self.b.torch, self.size
+        with torch.cuda.stream(b.stream):
             for c in range(pool):
                 step(c)
-        torch.cuda.synchronize(dev)
+        torch.cuda.synchronize(b.dev)
 
         def capture(n):
             g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
+            with torch.cuda.graph(g, stream=b.stream):
                 for c in range(n):
                     step(c)
             return g
 
         full = capture(pool)
         rest = {}
+        for n in (steps % pool, warmup % pool):
+            if n and n not in rest:
+                rest[n] = capture(n)
 
         def run(n):
             for _ in range(n // pool):
                 full.replay()
             if n % pool:
-                if n % pool not in rest:
-                    rest[n % pool] = capture(n % pool)
                 rest[n % pool].replay()
 
-        with torch.cuda.stream(stream):
+        with torch.cuda.stream(b.stream):
+            full.replay()
+            for g in rest.values():
+                g.replay()
             run(warmup)
-        torch.cuda.synchronize(dev)
-        if steps % pool and steps % pool not in rest:
-            rest[steps % pool] = capture(steps % pool)
-        barrier()
+        torch.cuda.synchronize(b.dev)
+        b.barrier()
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
-        with ClockSampler(local, enabled=sample_clocks) as clocks:
-            torch.cuda.synchronize(dev)
-            barrier()
-            with torch.cuda.stream(stream):
-                start.record(stream)
+        with ClockSampler(b.local, enabled=sample_clocks) as clocks:
+            torch.cuda.synchronize(b.dev)
+            b.barrier()
+            with torch.cuda.stream(b.stream):
+                start.record(b.stream)
                 run(steps)
-                end.record(stream)
-            torch.cuda.synchronize(dev)
-            barrier()
-        ms = max_over_ranks(start.elapsed_time(end), dist, dev)
-        st, detail = L.check_device_status(stream=stream)
-        if st != native.Status.OK:
+                end.record(b.stream)
+            torch.cuda.synchronize(b.dev)
+            b.barrier()
+        ms = max_over_ranks(start.elapsed_time(end), b.dist, b.dev)
+        st, detail = b.L.check_device_status(stream=b.stream)
+        if st != b.native.Status.OK:
             raise RuntimeError(f"device status {st.name} {detail:#x}")
         del full, rest
         return ms, clocks.summary()
 
+    def e2e(self, mode, steps):
+        """The same metric through the public API with host buffers: per step one pinned
+        H2D copy of every layer's x (packed), the group call (aqlm_matmul_group_host, the
+        copies inside the call) or one aqlm_matmul per layer, one D2H copy of every y."""
+        b, torch, w, batch = self.b, self.b.torch, self.w, self.batch
+        L = b.L
+        koff = np.cumsum([0] + [batch * lay.K for lay in w.layers])
+        noff = np.cumsum([0] + [batch * lay.N for lay in w.layers])
+        hx_flat = torch.empty((int(koff[-1]),), dtype=torch.float16).pin_memory()
+        for li, lay in enumerate(w.layers):
+            hx_flat[koff[li]:koff[li + 1]] = torch.from_numpy(
+                synth.make_x(batch, lay.K, seed=7, layer=li)).reshape(-1)
+        hy_flat = torch.empty((int(noff[-1]),), dtype=torch.float16).pin_memory()
+        dx_flat = torch.empty_like(hx_flat, device=b.dev)
+        dy_flat = torch.empty_like(hy_flat, device=b.dev)
+        dx = [dx_flat[koff[li]:koff[li + 1]].view(batch, lay.K) for li, lay in enumerate(w.layers)]
+        dy = [dy_flat[noff[li]:noff[li + 1]].view(batch, lay.N) for li, lay in enumerate(w.layers)]
+        groups = [L.LayerGroup([(self.weights[c][li], dx[li], dy[li]) for li in range(len(w.layers))])
+                  for c in range(self.size)]
+
+        def e2e_step(c):
+            if mode == "group":
+                groups[c].run_host(hx_flat, hy_flat, stream=b.stream)
+            else:
+                dx_flat.copy_(hx_flat, non_blocking=True)
+                for li in range(len(w.layers)):
+                    L.matmul(dx[li], self.weights[c][li], out=dy[li], stream=b.stream)
+                hy_flat.copy_(dy_flat, non_blocking=True)
+
+        with torch.cuda.stream(b.stream):
+            for i in range(3):
+                e2e_step(i % self.size)
+        torch.cuda.synchronize(b.dev)
+        b.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(b.stream):
+            e0.record(b.stream)
+            for i in range(steps):
+                e2e_step(i % self.size)
+            e1.record(b.stream)
+        torch.cuda.synchronize(b.dev)
+        ems = max_over_ranks(e0.elapsed_time(e1), b.dist, b.dev)
+        api = ("weight_only_additive_b200.layer.LayerGroup.run_host -> aqlm_matmul_group_host (the copies "
+               "inside the call)" if mode == "group"
+               else "weight_only_additive_b200.layer.matmul -> aqlm_matmul, per layer")
+        return {"value": job_throughput_gbs(self.copy_bytes, steps, b.world, ems), "unit": "GB/s",
+                "h2d_bytes_per_step": hx_flat.numel() * 2, "d2h_bytes_per_step": hy_flat.numel() * 2,
+                "steps": steps, "us_per_layer": ems * 1e3 / (steps * len(w.layers)),
+                "how": f"per step: one pinned H2D copy of every layer's x (packed), {api}, one D2H copy "
+                       f"of every y (packed); no CUDA graph"}
+
+
+def measure_config(b, w, batch, steps, warmup, with_e2e=True):
+    """One per-config record: the group call of every layer per step (graphs over the
+    pool), its binding roofline, and the end-to-end number through host buffers."""
+    pool = Pool(b, w, batch)
+    ms, _ = pool.timed(pool.step_group, steps, warmup)
+    step_s = ms / 1e3 / steps
+    sm_mhz = b.peaks["sm_max_mhz"]
+    rec = {"workload": w.name, "batch": batch, "scheme": w.layers[0].scheme.name, "layers": len(w.layers),
+           "value": job_throughput_gbs(pool.copy_bytes, steps, b.world, ms), "unit": "GB/s",
+           "us_per_layer": step_s * 1e6 / len(w.layers), "us_per_step": step_s * 1e6, "steps": steps,
+           "kernel": pool.kernel("group"), "gpu_launches_per_step": pool.launches("group"),
+           "roofline": roofline_record(w, batch, step_s, b.peaks, b.sms, sm_mhz),
+           "pool": f"{pool.size} copies ({pool.size * pool.copy_bytes / 1e6:.0f} MB)"}
+    if with_e2e:
+        rec["e2e"] = pool.e2e("group", steps)
+    del pool
+    b.torch.cuda.empty_cache()
+    return rec
+
+
+def run_ours(a):
+    b = Bench(a)
+    torch, L, native = b.torch, b.L, b.native
+    rank, world, dev = b.rank, b.world, b.dev
+    w = select_workload(a)
+    batch = workload_batch(w, a.batch)
+    sbytes = step_bytes(w, batch)
+    pool = Pool(b, w, batch, a.pool)
     mode = a.launch
-    ms, clock_summary = timed(step_group if mode == "group" else step_per_layer, a.steps, a.warmup,
-                              not a.no_clocks)
-    launches_per_step = launches(mode)
+    ms, clock_summary = pool.timed(pool.step_group if mode == "group" else pool.step_per_layer, a.steps, a.warmup,
+                                   not a.no_clocks)
+    launches_per_step = pool.launches(mode)
     value = job_throughput_gbs(sbytes, a.steps, world, ms)
     ms_step = ms / a.steps
     other = None
     if mode == "group" and not a.no_other_launch:
         # the same workload with one aqlm_matmul launch per layer, for comparison
         o_steps = min(a.steps, 20000)
-        o_ms, _ = timed(step_per_layer, o_steps, max(3, min(a.warmup, 200)), False)
+        o_ms, _ = pool.timed(pool.step_per_layer, o_steps, max(3, min(a.warmup, 200)))
         other = {"launch": "per-layer", "value": job_throughput_gbs(sbytes, o_steps, world, o_ms),
                  "unit": "GB/s", "us_per_layer": o_ms * 1e3 / (o_steps * len(w.layers)), "steps": o_steps}
 
@@ -532,21 +720,21 @@ def run_ours(a):
     if not a.no_other_launch:
         # launch overhead included: the same steps issued one by one from the host, no graph
         d_steps = min(a.steps, 2000)
-        step = step_group if mode == "group" else step_per_layer
-        with torch.cuda.stream(stream):
+        step = pool.step_group if mode == "group" else pool.step_per_layer
+        with torch.cuda.stream(b.stream):
             for i in range(3):
-                step(i % pool)
+                step(i % pool.size)
         torch.cuda.synchronize(dev)
-        barrier()
+        b.barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
+        with torch.cuda.stream(b.stream):
+            e0.record(b.stream)
             for i in range(d_steps):
-                step(i % pool)
-            e1.record(stream)
+                step(i % pool.size)
+            e1.record(b.stream)
         torch.cuda.synchronize(dev)
-        d_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        d_ms = max_over_ranks(e0.elapsed_time(e1), b.dist, dev)
         direct = {"launch": mode, "value": job_throughput_gbs(sbytes, d_steps, world, d_ms), "unit": "GB/s",
                   "us_per_layer": d_ms * 1e3 / (d_steps * len(w.layers)), "steps": d_steps,
                   "how": "the timed step launched from Python once per step, no CUDA graph"}
@@ -556,98 +744,38 @@ def run_ours(a):
 
         def step_context(c):
             for li in range(len(w.layers)):
-                L.dequantize(weights[c][li], out=wbuf[li], stream=stream)
-                torch.matmul(xs[c][li], wbuf[li].t(), out=ys[li])
+                L.dequantize(pool.weights[c][li], out=wbuf[li], stream=b.stream)
+                torch.matmul(pool.xs[c][li], wbuf[li].t(), out=pool.ys[li])
 
         c_steps = min(a.steps, 2000)
-        c_ms, _ = timed(step_context, c_steps, 3, False)
+        c_ms, _ = pool.timed(step_context, c_steps, 3)
         context = {"what": "aqlm_dequantize + torch.matmul (cuBLAS fp16) per layer", "unit": "GB/s",
                    "value": job_throughput_gbs(sbytes, c_steps, world, c_ms),
                    "us_per_layer": c_ms * 1e3 / (c_steps * len(w.layers)), "steps": c_steps,
                    "how": "algorithmic bytes of the step / time; W itself crosses HBM twice more"}
         del wbuf
 
-    peaks = measured_peaks()
-    kernel_names = {int(Path.GEMV): "gemv_gather_kernel", int(Path.GEMV_LUT): "gemv_lut_kernel",
-                    int(Path.TENSOR_CORE): "tc_pipe_kernel"}
-    if mode == "group" and launches_per_step == 2 * ((len(w.layers) + 15) // 16):
+    peaks = b.peaks
+    kernel = pool.kernel(mode)
+    sm_mhz = clock_summary.get("sm_mhz") or peaks["sm_max_mhz"]
+    if kernel == "lut_group_kernel":
         # every layer grouped: the timed launches are the partial-sum kernel and its
         # reduction, measured together (one step = one group call); the rate below is
         # therefore a lower bound on the partial-sum kernel's own
-        kernel = "lut_group_kernel"
         timed_as = "step: lut_group_kernel + lut_group_reduce_kernel"
-        achieved = sbytes / (ms_step / 1e3) / 1e9
     else:
-        kernel = kernel_names.get(paths[0], "?")
-        timed_as = "average launch of the step"
-        avg_launch_s = (ms / 1e3) / (a.steps * launches_per_step)
-        achieved = sbytes / launches_per_step / avg_launch_s / 1e9
-    traffic = measured_traffic(w.name, kernel)
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": kernel, "timed": timed_as,
-                "algorithmic_bytes": sbytes if kernel == "lut_group_kernel" else sbytes / launches_per_step,
-                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
-                if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
+        timed_as = "step: every launch of the step (one family of kernels)"
+    roofline = roofline_record(w, batch, ms_step / 1e3, peaks, b.sms, sm_mhz)
+    roofline.update({"traffic": measured_traffic(w.name, kernel) if roofline["bound"] == "hbm" else None,
+                     "kernel": kernel, "timed": timed_as, "algorithmic_bytes": sbytes})
 
-    # ---- end to end through the public API with host buffers ----------------
-    e2e = None
-    if not a.no_e2e:
-        e2e_steps = min(a.steps, 2000)
-        # every layer's x (and y) packed in one pinned host buffer and one device buffer:
-        # one H2D and one D2H copy per step (offsets stay 16-byte aligned: K, N % 8 == 0)
-        koff = np.cumsum([0] + [batch * lay.K for lay in w.layers])
-        noff = np.cumsum([0] + [batch * lay.N for lay in w.layers])
-        hx_flat = torch.empty((int(koff[-1]),), dtype=torch.float16).pin_memory()
-        for li, lay in enumerate(w.layers):
-            hx_flat[koff[li]:koff[li + 1]] = torch.from_numpy(
-                synth.make_x(batch, lay.K, seed=7, layer=li)).reshape(-1)
-        hy_flat = torch.empty((int(noff[-1]),), dtype=torch.float16).pin_memory()
-        dx_flat = torch.empty_like(hx_flat, device=dev)
-        dy_flat = torch.empty_like(hy_flat, device=dev)
-        dx = [dx_flat[koff[li]:koff[li + 1]].view(batch, lay.K) for li, lay in enumerate(w.layers)]
-        dy = [dy_flat[noff[li]:noff[li + 1]].view(batch, lay.N) for li, lay in enumerate(w.layers)]
-        e2e_groups = [L.LayerGroup([(weights[c][li], dx[li], dy[li]) for li in range(len(w.layers))])
-                      for c in range(pool)]
-
-        def e2e_step(c):
-            if mode == "group":
-                # one C-ABI call: H2D of every x, the group, D2H of every y
-                e2e_groups[c].run_host(hx_flat, hy_flat, stream=stream)
-            else:
-                dx_flat.copy_(hx_flat, non_blocking=True)
-                for li in range(len(w.layers)):
-                    L.matmul(dx[li], weights[c][li], out=dy[li], stream=stream)
-                hy_flat.copy_(dy_flat, non_blocking=True)
-
-        with torch.cuda.stream(stream):
-            for i in range(3):
-                e2e_step(i % pool)
-        torch.cuda.synchronize(dev)
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for i in range(e2e_steps):
-                e2e_step(i % pool)
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ems = max_over_ranks(e0.elapsed_time(e1), dist, dev)
-        api = ("weight_only_additive_b200.layer.LayerGroup.run_host -> aqlm_matmul_group_host (the copies "
-               "inside the call)" if mode == "group"
-               else "weight_only_additive_b200.layer.matmul -> aqlm_matmul, per layer")
-        e2e = {"value": job_throughput_gbs(sbytes, e2e_steps, world, ems), "unit": "GB/s",
-               "h2d_bytes_per_step": hx_flat.numel() * 2,
-               "d2h_bytes_per_step": hy_flat.numel() * 2,
-               "steps": e2e_steps, "us_per_layer": ems * 1e3 / (e2e_steps * len(w.layers)),
-               "how": f"per step: one pinned H2D copy of every layer's x (packed), {api}, one D2H copy "
-                      f"of every y (packed); no CUDA graph"}
+    e2e = pool.e2e(mode, min(a.steps, 2000)) if not a.no_e2e else None
 
     cpu = None
     cpu_kernel = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        b, s, rows, threads = oracle_sample_run(w, batch, a.cpu_seconds)
-        cpu = {"value": b / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+        bb, s, rows, threads = oracle_sample_run(w, batch, a.cpu_seconds)
+        cpu = {"value": bb / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": f"{rows} rows of each of the {len(w.layers)} layers (whole layers repeated "
                          f"when the budget exceeds them; decode to fp16 + fp64 matmul), batch {batch}, "
                          f"{s:.1f} s on the host cores"}
@@ -657,10 +785,27 @@ def run_ours(a):
         cpu["single_thread"] = {"value": b1 / s1 / 1e9, "unit": "GB/s", "cores": 1,
                                 "sample": f"{rows1} rows of each layer, {s1:.1f} s on one thread"}
         cpu_kernel = cpu_kernel_run(w, batch, min(a.cpu_seconds, 5.0))
+    pool_desc = (f"inputs larger than L2: rotating pool of {pool.size} copies "
+                 f"({pool.size * pool.copy_bytes / 1e6:.0f} MB > {b.l2 / 1e6:.0f} MB L2)")
+    pool_size = pool.size
+    del pool
+    torch.cuda.empty_cache()
 
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    per_config = None
+    if world == 1 and not a.no_per_config and a.workload == DEFAULT_WORKLOAD and a.scheme is None \
+            and a.layer is None and a.batch is None:
+        per_config = []
+        sub_steps = min(max(a.steps, 20), 2000)
+        for name, scheme, bt in PER_CONFIG:
+            sw = workloads.get(name)
+            if scheme is not None:
+                sw = scheme_subset(sw, scheme)
+            if sw.name == w.name and bt == batch:
+                continue  # the headline itself
+            per_config.append(measure_config(b, sw, bt, sub_steps, max(3, min(a.warmup, 50)),
+                                             with_e2e=not a.no_e2e))
+
+    b.close()
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": a.steps,
@@ -671,16 +816,16 @@ def run_ours(a):
                 "config": {"workload": w.name, "layers": len(w.layers), "batch": batch,
                            "scheme": w.layers[0].scheme.name,
                            "algorithmic_bytes_per_step": sbytes,
-                           "l2": f"inputs larger than L2: rotating pool of {pool} copies "
-                                 f"({pool * copy_bytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
+                           "l2": pool_desc,
                            "launch": ("one aqlm_matmul_group call per step (grouped lookup-table kernel + "
                                       "reduction)" if mode == "group" else "one aqlm_matmul call per layer")
-                                     + f"; CUDA graphs of {pool} consecutive steps (one pass over the pool)",
+                                     + f"; CUDA graphs of {pool_size} consecutive steps (one pass over the pool)",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu, "cpu_kernel": cpu_kernel, "e2e": e2e,
                 "other_launch": other, "no_graph": direct, "context": context,
+                "per_config": per_config,
                 "gpu_launches": launches_per_step * a.steps,
-                "clocks": clock_summary, "gpu": props.name}
+                "clocks": clock_summary, "gpu": b.props.name}
         print(json.dumps(line), flush=True)
     return 0
 

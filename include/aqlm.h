@@ -35,7 +35,7 @@
  * Ownership and state: the library never allocates or frees device memory on
  * a call and keeps no per-call state.  It holds one 32-bit device status word
  * per device (a static device variable) where kernels record a bounded wait
- * that gave up.  All compute calls are asynchronous on `stream`
+ * that gave up, and the static scratch of aqlm_matmul_group_static.  All compute calls are asynchronous on `stream`
  * (NULL = the legacy default stream) and may be captured in CUDA graphs.
  *
  * Stream ordering: kernels are launched with programmatic dependent launch.  A
@@ -84,10 +84,25 @@ typedef enum {
 
 /*
  * y = x . W^T . diag(scales) + bias, with W decoded on chip from codes and
- * codebooks.  Accumulation is fp32 (or better); y is rounded to fp16 (RNE).
- * Result tolerance against the fp64 reference of the decoded fp16 weights:
- * max|y - y_ref| / max|y_ref| <= 5e-3.
- * Returns AQLM_OK after enqueueing the work on `stream`.
+ * codebooks.  Defined by the AQLM pages as follows.  A weight group is the sum of
+ * the codewords its codes pick: repo summary "Additive quantization that actually
+ * survives one-bit weights", section "What it does"; paper record "Extreme
+ * Compression of Large Language Models via Additive Quantization", method
+ * paragraph.  Activations stay fp16 (w2a16): inference-research record "AQLM
+ * (additive / multi-codebook quantization)", sections "Bits" and "Activation
+ * scheme".  One scale per output channel, none shared over a group: the same
+ * record, "notes".  Token generation looks the products up ("Kernels"); larger
+ * batches decode to fp16 and run an fp16 tensor-core GEMM ("notes").
+ *   x          fp16 [batch, K], read          codes      [N, K/g, M] u8/u16, read
+ *   codebooks  fp16 [M, 2^B, g], read         scales     fp16 [N], read
+ *   bias       fp16 [N] or NULL, read         y          fp16 [batch, N], written
+ * All are caller-owned device memory (layout, alignment and ownership as in the file
+ * header); y must not overlap an input.  Accumulation is fp32 (or better); y is
+ * rounded to fp16 (RNE).  Result tolerance against the fp64 reference of the
+ * decoded fp16 weights: max|y - y_ref| / max|y_ref| <= 5e-3.
+ * Returns AQLM_OK after enqueueing the work on `stream`; AQLM_ERR_INVALID_ARG,
+ * AQLM_ERR_UNSUPPORTED or AQLM_ERR_MISALIGNED (nothing launched) for bad arguments;
+ * AQLM_ERR_CUDA if the launch failed.
  */
 aqlm_status aqlm_matmul(const void* x, const void* codes, const void* codebooks,
                         const void* scales, const void* bias, void* y,
@@ -102,10 +117,20 @@ aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codeb
                              aqlm_path path, aqlm_stream_t stream);
 
 /*
- * W_out[n, j*g + t] = fp16_rne( fp32( C_0[c_0][t] + C_1[c_1][t] + ... ) * fp32(s_n) )
+ * The dense fp16 weight of the layer, the first half of the large-batch route
+ * "dequantize-to-FP16 then an FP16 tensor-core GEMM" (inference-research record
+ * "AQLM (additive / multi-codebook quantization)", notes), each group the sum of
+ * the codewords its codes pick (repo summary "Additive quantization that actually
+ * survives one-bit weights", section "What it does"):
+ *
+ *   W_out[n, j*g + t] = fp16_rne( fp32( C_0[c_0][t] + C_1[c_1][t] + ... ) * fp32(s_n) )
+ *
  * with c_m = codes[n, j, m]; the codewords are added in fp32 in ascending m,
  * starting from C_0 itself, then one fp32 multiply by the channel scale and
  * one round-to-nearest-even to fp16.  Bit-exact by definition.
+ *   codes, codebooks, scales  as for aqlm_matmul, read
+ *   W_out                     fp16 [N, K], caller-owned device memory, written
+ * Errors as for aqlm_matmul (no bias, no batch); returns after enqueueing.
  */
 aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void* scales,
                             void* W_out, int M, int B, int g, int K, int N,
@@ -166,7 +191,7 @@ typedef struct {
  * outputs and inputs are rejected with AQLM_ERR_INVALID_ARG as far as the
  * pointer ranges show).  Batch-1 problems with 256-entry codebooks (B = 8, any M
  * and g above) whose code rows (K / g * M bytes) are whole 16-byte units are
- * computed together, up to 16 per launch pair (a partial-sum kernel and a
+ * computed together, up to 32 per launch pair (a partial-sum kernel and a
  * reduction); the others are launched one after another as by aqlm_matmul.  Both kernels of a
  * pair keep the stream-ordering contract above.
  *
@@ -186,17 +211,22 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
  * aqlm_matmul_group without a caller workspace, for callers that cannot
  * allocate device memory.  The AQLM pages have no counterpart: this is a library
  * convenience.  The partial sums live in a static device buffer of
- * AQLM_STATIC_GROUP_SCRATCH_BYTES inside the library (one per device, its address
- * taken with cudaGetSymbolAddress); the call allocates nothing.  Problems whose
- * aqlm_group_workspace_size exceeds that size are rejected with
- * AQLM_ERR_INVALID_ARG before anything is launched (8 MiB covers, for example,
- * a Llama-2-7B decoder layer set or 16 Mixtral-8x7B expert linears).  The buffer
- * needs no clearing: the reduction reads only partials written by the same call.
+ * AQLM_STATIC_GROUP_SCRATCH_BYTES inside the library (one per device; the address
+ * is taken with cudaGetSymbolAddress on a device's first call and again whenever
+ * the device's CUDA context has changed, e.g. after cudaDeviceReset); the call
+ * allocates nothing.  Problems whose aqlm_group_workspace_size exceeds that size
+ * are rejected with AQLM_ERR_INVALID_ARG before anything is launched (16 MiB
+ * covers, for example, a Llama-2-7B decoder layer set, 1.6 MB, or the 24
+ * Mixtral-8x7B expert linears of one layer, 11 MB).  The buffer needs no
+ * clearing: the reduction reads only partials written by the same call.
  * Calls that overlap in time (different streams or host threads on one device)
  * share the buffer and RACE: the caller must serialise them.  Calls on one
  * stream are ordered and safe.  Otherwise identical to aqlm_matmul_group.
  */
-#define AQLM_STATIC_GROUP_SCRATCH_BYTES (8u << 20)
+#define AQLM_STATIC_GROUP_SCRATCH_BYTES (16u << 20)
+/* The library's value of AQLM_STATIC_GROUP_SCRATCH_BYTES (a caller compiled
+ * against another header can read the real limit here).  Pure host logic. */
+size_t aqlm_static_group_scratch_bytes(void);
 aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aqlm_stream_t stream);
 
 /*
@@ -219,7 +249,7 @@ aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, cons
                                    void* workspace, size_t workspace_bytes, aqlm_stream_t stream);
 
 /* Workspace bytes aqlm_matmul_group needs for these problems: for every run of
- * up to 16 grouped problems, the sum over them of ceil(K / g * M / 128) * N * 4
+ * up to 32 grouped problems, the sum over them of ceil(K / g * M / 128) * N * 4
  * bytes (one fp32 partial per row and 128 code bytes) rounded up to 256; the
  * maximum over runs.  Pure host logic. */
 size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count);

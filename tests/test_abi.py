@@ -153,11 +153,12 @@ def test_group_workspace_size(lib):
     assert native.aqlm_group_workspace_size([_prob(1 << 32, batch=2)]) == 0         # batch 2: not grouped
     assert native.aqlm_group_workspace_size([_prob(1 << 32, K=4104)]) == 0          # K % 64 != 0
     assert native.aqlm_group_workspace_size([_prob(1 << 32, K=4095)]) == 0          # invalid shape
-    # 20 grouped problems: two runs of 16 and 4; the workspace is the larger run
-    many = [_prob((i + 1) << 32, K=64 * (i + 1), N=100) for i in range(20)]
-    run1 = sum(_ws_bytes(64 * (i + 1), 100) for i in range(16))
-    run2 = sum(_ws_bytes(64 * (i + 1), 100) for i in range(16, 20))
-    assert native.aqlm_group_workspace_size(many) == max(run1, run2)
+    # 40 grouped problems: runs of 32 and 8; the workspace is the larger run
+    R = native.MAX_GROUP_LAYERS
+    many = [_prob((i + 1) << 32, K=64 * (i + 1), N=100) for i in range(R + 8)]
+    run1 = sum(_ws_bytes(64 * (i + 1), 100) for i in range(R))
+    run2 = sum(_ws_bytes(64 * (i + 1), 100) for i in range(R, R + 8))
+    assert native.aqlm_group_workspace_size(many) == max(run1, run2) == run1
 
 
 def test_group_validation_needs_no_gpu(lib):
@@ -190,15 +191,29 @@ def test_group_static_validation_needs_no_gpu(lib):
     assert L_.aqlm_matmul_group_static(native.problem_array([_prob(1 << 32)]), 0, None) == Status.OK
     assert L_.aqlm_matmul_group_static(None, 1, None) == Status.INVALID_ARG
     assert L_.aqlm_matmul_group_static(native.problem_array([_prob(1 << 32)]), -3, None) == Status.INVALID_ARG
-    # 5 grouped 28672 x 8192 layers need 5 x 16 x 28672 x 4 bytes > 8 MiB
-    big = [_prob((i + 1) << 34, K=8192, N=28672) for i in range(5)]
-    assert native.aqlm_group_workspace_size(big) == 5 * _ws_bytes(8192, 28672) > native.STATIC_GROUP_SCRATCH_BYTES
-    assert L_.aqlm_matmul_group_static(native.problem_array(big), 5, None) == Status.INVALID_ARG
-    # 16 Mixtral-8x7B expert linears (4096 x 14336) fit
-    assert native.aqlm_group_workspace_size([_prob((i + 1) << 34, K=14336, N=4096) for i in range(16)]) == \
-        16 * _ws_bytes(14336, 4096) <= native.STATIC_GROUP_SCRATCH_BYTES
+    # 10 grouped 28672 x 8192 layers need 10 x 16 x 28672 x 4 bytes > 16 MiB
+    big = [_prob((i + 1) << 34, K=8192, N=28672) for i in range(10)]
+    assert native.aqlm_group_workspace_size(big) == 10 * _ws_bytes(8192, 28672) > native.STATIC_GROUP_SCRATCH_BYTES
+    assert L_.aqlm_matmul_group_static(native.problem_array(big), 10, None) == Status.INVALID_ARG
+    # the 24 Mixtral-8x7B expert linears of a layer (w1, w3 14336 x 4096, w2 4096 x 14336) fit
+    mixtral = [_prob((i + 1) << 34, K=14336, N=4096) if i % 3 == 2 else _prob((i + 1) << 34, K=4096, N=14336)
+               for i in range(24)]
+    assert native.aqlm_group_workspace_size(mixtral) == \
+        8 * (_ws_bytes(14336, 4096) + 2 * _ws_bytes(4096, 14336)) <= native.STATIC_GROUP_SCRATCH_BYTES
     bad = [_prob(1 << 32, M=5)]
     assert L_.aqlm_matmul_group_static(native.problem_array(bad), 1, None) == Status.UNSUPPORTED
+
+
+def test_static_scratch_size_agrees_everywhere(lib):
+    """The #define in include/aqlm.h, the library's own report and the binding's
+    constant are one number."""
+    import os
+    import re
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "aqlm.h")).read()
+    m = re.search(r"#define AQLM_STATIC_GROUP_SCRATCH_BYTES \((\d+)u << (\d+)\)", hdr)
+    assert m, "AQLM_STATIC_GROUP_SCRATCH_BYTES not found in include/aqlm.h"
+    from_header = int(m.group(1)) << int(m.group(2))
+    assert from_header == native.lib().aqlm_static_group_scratch_bytes() == native.STATIC_GROUP_SCRATCH_BYTES
 
 
 def test_selftest_rejects_bad_limits_without_a_gpu(lib):

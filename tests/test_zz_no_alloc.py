@@ -82,12 +82,13 @@ def test_static_scratch_matches_caller_workspace_on_two_calls_in_a_row(dev):
 
 
 def test_static_scratch_rejects_groups_over_its_size(dev):
-    """5 grouped 28672 x 8192 layers need 5 x 1835008 bytes of partials > 8 MiB:
+    """10 grouped 28672 x 8192 layers need 10 x 1835008 bytes of partials > 16 MiB:
     rejected before anything is launched (the fake pointers are never touched)."""
     A = 1 << 40
     step = 1 << 32
     probs = [(A + i * step, A + i * step + (1 << 28), A + i * step + (2 << 28), A + i * step + (3 << 28), None,
-              A + i * step + (4 << 28), 2, 8, 8, 8192, 28672, 1) for i in range(5)]
+              A + i * step + (4 << 28), 2, 8, 8, 8192, 28672, 1) for i in range(10)]
     arr = native.problem_array(probs)
-    assert native.aqlm_group_workspace_size(arr, 5) > native.STATIC_GROUP_SCRATCH_BYTES
-    assert native.lib().aqlm_matmul_group_static(arr, 5, None) == Status.INVALID_ARG
+    assert native.aqlm_group_workspace_size(arr, 10) > native.STATIC_GROUP_SCRATCH_BYTES
+    assert native.lib().aqlm_static_group_scratch_bytes() == native.STATIC_GROUP_SCRATCH_BYTES
+    assert native.lib().aqlm_matmul_group_static(arr, 10, None) == Status.INVALID_ARG

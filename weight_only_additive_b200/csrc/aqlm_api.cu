@@ -21,48 +21,48 @@ __device__ __align__(256) uint8_t g_group_scratch[AQLM_STATIC_GROUP_SCRATCH_BYTE
 thread_local int t_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
-std::mutex g_status_mu;
-uint32_t* g_status_ptr[kMaxDevices] = {};
+
+// Device address of a file-scope __device__ variable on the current device, looked up
+// with cudaGetSymbolAddress once per device and context: a cudaDeviceReset ends the
+// context and the next one may place the module's variables elsewhere, so an address
+// is reused only while the context that it came from is still current.
+struct SymbolCache {
+  std::mutex mu;
+  uint64_t ctx[kMaxDevices] = {};
+  void* ptr[kMaxDevices] = {};
+};
+
+void* symbol_address(const void* symbol, SymbolCache& cache) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(cache.mu);
+  const uint64_t ctx = aqlm::current_context_id();
+  if (cache.ptr[dev] && ctx != 0 && cache.ctx[dev] == ctx) return cache.ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  cache.ptr[dev] = p;
+  // read after the lookup, which creates the device's context when there is none yet
+  cache.ctx[dev] = aqlm::current_context_id();
+  return p;
+}
+
+SymbolCache g_status_cache;
+SymbolCache g_scratch_cache;
 
 // Device address of g_device_status for the current device (nullptr on failure).
 uint32_t* device_status_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  std::lock_guard<std::mutex> lock(g_status_mu);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
-      cudaGetLastError();
-      return nullptr;
-    }
-    g_status_ptr[dev] = static_cast<uint32_t*>(p);
-  }
-  return g_status_ptr[dev];
+  return static_cast<uint32_t*>(symbol_address(reinterpret_cast<const void*>(&g_device_status), g_status_cache));
 }
-
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_group_scratch for the current device (nullptr on failure).
 void* static_scratch_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_group_scratch) != cudaSuccess) {
-      cudaGetLastError();
-      return nullptr;
-    }
-    g_scratch_ptr[dev] = p;
-  }
-  return g_scratch_ptr[dev];
+  return symbol_address(reinterpret_cast<const void*>(&g_group_scratch), g_scratch_cache);
 }
 
 aqlm_status from_cuda(cudaError_t e) {
@@ -94,6 +94,32 @@ aqlm_status validate_shape(int M, int B, int g, int K, int N, int batch) {
 }  // namespace
 
 namespace aqlm {
+uint64_t current_context_id() {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(f);
+    cudaGetLastError();
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return static_cast<uint64_t>(id) + 1u;  // 0 stays "unknown"
+}
+
 EncodeTiledFn encode_tiled() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
@@ -111,7 +137,7 @@ EncodeTiledFn encode_tiled() {
 
 extern "C" {
 
-int aqlm_abi_version(void) { return 6; }
+int aqlm_abi_version(void) { return 7; }
 
 const char* aqlm_status_string(aqlm_status status) {
   switch (status) {
@@ -378,6 +404,8 @@ aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, cons
   if (st != AQLM_OK) return st;
   return copy_runs(false);
 }
+
+size_t aqlm_static_group_scratch_bytes(void) { return AQLM_STATIC_GROUP_SCRATCH_BYTES; }
 
 aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aqlm_stream_t stream) {
   if (count == 0) return AQLM_OK;

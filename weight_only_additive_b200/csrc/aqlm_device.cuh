@@ -81,6 +81,20 @@ __device__ __forceinline__ uint4 ldg_nc_v4_hint(const void* p, uint64_t pol) {
   return v;
 }
 
+// acc + (the fp16 value in the low / high half of w), one fp32 add rounded to
+// nearest: the mixed-precision add of sm_100 widens the fp16 operand exactly, so
+// this equals acc + float(half) with no intermediate fp16 rounding.
+__device__ __forceinline__ float add_f32_lo_f16(uint32_t w, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, lo, %2;\n\t}" : "=f"(r) : "r"(w), "f"(acc));
+  return r;
+}
+__device__ __forceinline__ float add_f32_hi_f16(uint32_t w, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, hi, %2;\n\t}" : "=f"(r) : "r"(w), "f"(acc));
+  return r;
+}
+
 __device__ __forceinline__ float2 h2_to_f2(uint32_t v) {
   __half2 h = *reinterpret_cast<__half2*>(&v);
   return __half22float2(h);

@@ -58,6 +58,12 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn encode_tiled();
 
+// A process-unique id (never 0) of the calling thread's current CUDA context, or 0 when
+// there is none or the driver cannot say.  Per-device host caches of things that live
+// in a context (symbol addresses, kernel attributes) compare it to notice a context
+// created after cudaDeviceReset.
+uint64_t current_context_id();
+
 // Pipelined decode -> tcgen05 kernel; cudaErrorNotSupported when the shape is
 // outside what it handles (the caller then uses the single-stage kernel).
 cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t stream);
@@ -89,7 +95,7 @@ inline bool grad_shape_supported(int M, int B, int g, int K, int N) {
 // of the partial-sum kernel, one of the reduction), at most kMaxGroupLayers per
 // launch.  The workspace holds every layer's fp32 partials, [ceil(G/64)][N] each,
 // 256-byte aligned.
-constexpr int kMaxGroupLayers = 16;
+constexpr int kMaxGroupLayers = 32;
 bool lut_group_supported(const Problem& p);
 size_t lut_group_workspace_bytes(const Problem* probs, int count);
 cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, uint32_t* status,

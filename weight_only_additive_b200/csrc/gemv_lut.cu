@@ -338,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const __grid_cons
       // ---- 5. lookups: a task is 8 rows; 4 lanes per row, 8 code words each -------------------
       // Lane (r8, q4) reads code word w = 8*q4 + ((r8 + s) mod 8) at step s: the 32 lanes
       // always touch 32 distinct words, so both the code reads and the table reads are
-      // free of bank conflicts.  Pairs of looked-up fp16 values are added as half2 and
-      // the task's 16 pair sums are accumulated in half2, then widened to fp32.
+      // free of bank conflicts.  Every looked-up fp16 value is added to an fp32
+      // accumulator (two per lane, one per half of the table word).
       const int slot0 = kRecycle ? (ps * p.ntile) % p.R : 0;  // slot of the pass's first tile
       for (int t = warp; t < nt; t += kWarps) {
         const int i = ps * p.ntile + t / 8;  // tile holding rows 8t .. 8t+7
@@ -355,7 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const __grid_cons
           uint32_t cw[8];
 #pragma unroll
           for (int s8 = 0; s8 < 8; ++s8) cw[s8] = cw_row[8 * q4 + ((r8 + s8) & 7)];
-          __half2 hacc = __float2half2_rn(0.f);
+          // fp32 accumulators: even code bytes (low halves of their table words) and odd
+          // code bytes (high halves)
+          float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
           for (int s8 = 0; s8 < 8; ++s8) {
             const uint32_t wv = static_cast<uint32_t>((8 * q4 + ((r8 + s8) & 7)) << 2);  // 4 * code word
@@ -364,14 +366,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(const __grid_cons
             const uint32_t t1 = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(cw[s8], wv, 0x5514));
             const uint32_t t2 = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(cw[s8], wv, 0x5524) + 128u);
             const uint32_t t3 = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(cw[s8], wv, 0x5534) + 128u);
-            // (codebook-0 value of t0, codebook-1 value of t1) and likewise for t2, t3
-            const uint32_t p01 = __byte_perm(t0, t1, 0x7610);
-            const uint32_t p23 = __byte_perm(t2, t3, 0x7610);
-            hacc = __hadd2(hacc, __hadd2(*reinterpret_cast<const __half2*>(&p01),
-                                         *reinterpret_cast<const __half2*>(&p23)));
+            acc0 = add_f32_lo_f16(t0, acc0);
+            acc1 = add_f32_hi_f16(t1, acc1);
+            acc0 = add_f32_lo_f16(t2, acc0);
+            acc1 = add_f32_hi_f16(t3, acc1);
           }
-          const float2 f = __half22float2(hacc);
-          float v = f.x + f.y;
+          float v = acc0 + acc1;
           v += __shfl_xor_sync(0xffffffffu, v, 1);
           v += __shfl_xor_sync(0xffffffffu, v, 2);
           if (q4 == 0) part[t * 8 + r8] += v;
@@ -453,7 +453,7 @@ cudaError_t lut_plan(int dev, int N, int S, int M, int g, Plan* out) {
   static std::mutex mu;
   static std::map<std::tuple<int, int, int, int, int>, Plan> cache;
   static bool wide_clusters[64] = {};
-  static bool attrs_set[64] = {};
+  static uint64_t attrs_ctx[64] = {};  // context the kernels' attributes were set in (0: not yet)
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   auto it = cache.find(std::make_tuple(dev, N, S, M, g));
@@ -461,7 +461,8 @@ cudaError_t lut_plan(int dev, int N, int S, int M, int g, Plan* out) {
     *out = it->second;
     return cudaSuccess;
   }
-  if (!attrs_set[dev]) {
+  const uint64_t ctx = current_context_id();
+  if (ctx == 0 || attrs_ctx[dev] != ctx) {
     // clusters of up to 16 CTAs where the device allows them, else the portable 8
     wide_clusters[dev] = cudaFuncSetAttribute(gemv_lut_kernel<kGeneric, false>,
                                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
@@ -474,7 +475,7 @@ cudaError_t lut_plan(int dev, int N, int S, int M, int g, Plan* out) {
       e = cudaFuncSetAttribute(gemv_lut_kernel<kGeneric, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kSmemLimit));
     if (e != cudaSuccess) return e;
-    attrs_set[dev] = true;
+    attrs_ctx[dev] = ctx;
   }
   const int cmax = wide_clusters[dev] ? 16 : 8;
   Plan best{0, 0, 0, 0, 0};

@@ -392,33 +392,33 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
             for (int s8 = 0; s8 < 8; ++s8) cw[u][s8] = row0[u * kWarpsPerTile * 8 * 32 + (wv[s8] >> 2)];
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[my_slot]);  // the tile's codes are in registers
-          __half2 hacc[kTasks];
+          // fp32 accumulators: even code bytes (the low halves of their words) into
+          // acc0, odd code bytes (high halves) into acc1
+          float acc0[kTasks], acc1[kTasks];
 #pragma unroll
-          for (int u = 0; u < kTasks; ++u) hacc[u] = __float2half2_rn(0.f);
+          for (int u = 0; u < kTasks; ++u) acc0[u] = acc1[u] = 0.f;
           const uint8_t* lut = smem + kOffLut;
 #pragma unroll
           for (int s8 = 0; s8 < 8; ++s8) {
 #pragma unroll
             for (int u = 0; u < kTasks; ++u) {
               // table byte offsets: entry * 256 + column * 4 (column w, or 32 + w at +128);
-              // (codebook-0 half of one word, codebook-1 half of the other) per group
+              // a byte's value is half (byte mod 2) of the word its pair reads
               const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cw[u][s8], wv[s8], 0x5504));
               const uint32_t a1 = *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cw[u][s8], wv[s8], 0x5514));
               const uint32_t a2 =
                   *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cw[u][s8], wv[s8], 0x5524) + 128u);
               const uint32_t a3 =
                   *reinterpret_cast<const uint32_t*>(lut + __byte_perm(cw[u][s8], wv[s8], 0x5534) + 128u);
-              const uint32_t p01 = __byte_perm(a0, a1, 0x7610), p23 = __byte_perm(a2, a3, 0x7610);
-              hacc[u] = __hadd2(hacc[u],
-                                __hadd2(*reinterpret_cast<const __half2*>(&p01), *reinterpret_cast<const __half2*>(&p23)));
+              acc0[u] = add_f32_lo_f16(a0, acc0[u]);
+              acc1[u] = add_f32_hi_f16(a1, acc1[u]);
+              acc0[u] = add_f32_lo_f16(a2, acc0[u]);
+              acc1[u] = add_f32_hi_f16(a3, acc1[u]);
             }
           }
           float v[kTasks];
 #pragma unroll
-          for (int u = 0; u < kTasks; ++u) {
-            const float2 f = __half22float2(hacc[u]);
-            v[u] = f.x + f.y;
-          }
+          for (int u = 0; u < kTasks; ++u) v[u] = acc0[u] + acc1[u];
 #pragma unroll
           for (int u = 0; u < kTasks; ++u) v[u] += __shfl_xor_sync(0xffffffffu, v[u], 1);
 #pragma unroll
@@ -575,6 +575,7 @@ GroupKey g_launch_key[kLaunchCacheEntries];
 GroupLaunch g_launch_val[kLaunchCacheEntries];
 int g_launch_next = 0;
 int g_sms[kMaxDevices] = {};  // 0 = not queried yet (also means "attribute not set")
+uint64_t g_attr_ctx[kMaxDevices] = {};  // context the kernels' attributes were set in
 
 // Tensor maps and parameters of one launch pair (host work only, no CUDA calls but
 // the driver's tensor-map encoder).
@@ -647,8 +648,9 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
   GroupLaunch launch;
   {
     std::lock_guard<std::mutex> lock(g_launch_mu);
-    if (g_sms[dev] == 0) {
-      // once per device: the SM count and the kernels' shared-memory limits
+    const uint64_t ctx = current_context_id();
+    if (g_sms[dev] == 0 || ctx == 0 || g_attr_ctx[dev] != ctx) {
+      // once per device and context: the SM count and the kernels' shared-memory limits
       int sms = 0;
       e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
       if (e != cudaSuccess) return e;
@@ -662,6 +664,7 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
                                static_cast<int>(GroupLayout<4, true>::kSmemBytes + 1024u));
       if (e != cudaSuccess) return e;
       g_sms[dev] = std::max(1, sms);
+      g_attr_ctx[dev] = ctx;
     }
     int hit = -1;
     for (int c = 0; c < kLaunchCacheEntries && hit < 0; ++c)

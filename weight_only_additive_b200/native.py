@@ -19,15 +19,21 @@ EXPORTS = ("aqlm_matmul", "aqlm_matmul_path", "aqlm_dequantize", "aqlm_select_pa
            "aqlm_validate", "aqlm_status_string", "aqlm_check_device_status",
            "aqlm_last_cuda_error", "aqlm_abi_version", "aqlm_matmul_group",
            "aqlm_group_workspace_size", "aqlm_matmul_group_static", "aqlm_selftest_bounded_wait",
-           "aqlm_input_grad", "aqlm_validate_input_grad", "aqlm_matmul_group_host")
+           "aqlm_input_grad", "aqlm_validate_input_grad", "aqlm_matmul_group_host",
+           "aqlm_static_group_scratch_bytes")
 
-ABI_VERSION = 6
+ABI_VERSION = 7
 
 # Site code aqlm_selftest_bounded_wait records in the device status word.
 SITE_SELFTEST = 0x501
 
-# Size of the library's static scratch buffer behind aqlm_matmul_group_static.
-STATIC_GROUP_SCRATCH_BYTES = 8 << 20
+# Size of the library's static scratch buffer behind aqlm_matmul_group_static
+# (AQLM_STATIC_GROUP_SCRATCH_BYTES; the library reports its own value through
+# aqlm_static_group_scratch_bytes, which a CPU test compares with this one).
+STATIC_GROUP_SCRATCH_BYTES = 16 << 20
+
+# Grouped problems one launch pair of aqlm_matmul_group computes together.
+MAX_GROUP_LAYERS = 32
 
 
 class Status(enum.IntEnum):
@@ -111,6 +117,8 @@ def lib() -> ctypes.CDLL:
                                                      ctypes.c_size_t, _vp]
                 L.aqlm_matmul_group_host.restype = _i
                 L.aqlm_matmul_group_static.restype = _i
+                L.aqlm_static_group_scratch_bytes.argtypes = []
+                L.aqlm_static_group_scratch_bytes.restype = ctypes.c_size_t
                 L.aqlm_selftest_bounded_wait.argtypes = [ctypes.c_uint, _vp]
                 L.aqlm_selftest_bounded_wait.restype = _i
                 if L.aqlm_abi_version() != ABI_VERSION:

@@ -11,6 +11,7 @@ Recipe (one generator per tensor, so tensors never share a stream):
     tensor 2  scales     uniform(0.5, 1.5) -> fp16           [N]
     tensor 3  x          normal(0, 1) -> fp16                [batch, K]
     tensor 4  bias       normal(0, 1) -> fp16                [N] (only when asked)
+    tensor 5  outliers   make_x_outliers: the outlier channels and their values
 Uniform codes are the worst case for codebook locality; the pages give no code
 statistics of trained checkpoints.
 """
@@ -21,7 +22,7 @@ from typing import Optional
 
 import numpy as np
 
-CODES, CODEBOOKS, SCALES, X, BIAS = range(5)
+CODES, CODEBOOKS, SCALES, X, BIAS, OUTLIERS = range(6)
 
 
 def rng(seed: int, workload: int, layer: int, tensor: int, copy: int = 0) -> np.random.Generator:
@@ -66,3 +67,20 @@ def make_x(batch: int, K: int, *, seed: int = 0, workload: int = 0, layer: int =
            copy: int = 0) -> np.ndarray:
     return rng(seed, workload, layer, X, copy).normal(0.0, 1.0, size=(batch, K)).astype(
         np.float32).astype(np.float16)
+
+
+def make_x_outliers(batch: int, K: int, *, sigma: float, n_outliers: int, lo: float = 500.0,
+                    hi: float = 2000.0, seed: int = 0, workload: int = 0, layer: int = 0,
+                    copy: int = 0) -> np.ndarray:
+    """Activations with the spread of a real fp16 layer input: x ~ normal(0, sigma), and
+    n_outliers channels (the same K indices in every batch row, drawn without replacement)
+    whose values are uniform in [lo, hi] in magnitude with a random sign per element,
+    all rounded to fp16."""
+    x = rng(seed, workload, layer, X, copy).normal(0.0, sigma, size=(batch, K))
+    if n_outliers:
+        r = rng(seed, workload, layer, OUTLIERS, copy)
+        cols = r.choice(K, size=n_outliers, replace=False)
+        mag = r.uniform(lo, hi, size=(batch, n_outliers))
+        sign = np.where(r.integers(0, 2, size=(batch, n_outliers)) == 1, 1.0, -1.0)
+        x[:, cols] = sign * mag
+    return x.astype(np.float32).astype(np.float16)
