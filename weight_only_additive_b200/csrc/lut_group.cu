@@ -14,7 +14,8 @@
 // t; a layer has ceil(G M / 128) x ceil(N / 64) items.  Items are numbered layer by
 // layer, slice-major, and every CTA (one per SM, persistent) takes a contiguous
 // range of them, so consecutive items mostly share (p, s) and therefore the
-// lookup table: a CTA rebuilds it only when (p, s) changes.
+// lookup table: a CTA rebuilds it only when (p, s) changes.  The ranges have equal
+// estimated cost (items plus the table builds they start), not equal item counts.
 //
 // Per CTA:
 //   warp 16     TMA producer: streams the code tile (64 rows x 128 bytes) of every
@@ -33,8 +34,9 @@
 // byte); launches of 2x8 g8 layers only keep the tuned build described above.
 //
 // The partials of a row are summed over the slices in ascending order by a second
-// small kernel (programmatic dependent launch), which applies the channel scale
-// and bias: the result does not depend on which CTA ran which item.
+// small kernel (programmatic dependent launch; one thread per row, its loads issued
+// eight slices at a time), which applies the channel scale and bias: the result does
+// not depend on which CTA ran which item.
 //
 // Bank-conflict-free lookups: as in the single-layer lookup-table kernel, lane
 // (r8, q4) reads code word 8 q4 + ((r8 + s) mod 8) at step s, and the table keeps
@@ -51,7 +53,11 @@
 namespace aqlm {
 namespace {
 
-constexpr int kWorkers = 512;                      // warps 0-15
+#ifndef AQLM_GROUP_WORKER_WARPS
+#define AQLM_GROUP_WORKER_WARPS 16
+#endif
+constexpr int kWorkerWarps = AQLM_GROUP_WORKER_WARPS;  // table builders (the first 16) and lookup workers
+constexpr int kWorkers = 32 * kWorkerWarps;
 constexpr int kThreads = kWorkers + 32;            // + TMA producer warp
 constexpr int kProducerWarp = kWorkers / 32;
 constexpr int kTileRows = 64;
@@ -64,8 +70,9 @@ constexpr uint32_t kBOpBytes = lut::kBOpBytes;     // 8 KB per codebook
 #endif
 constexpr int kTasks = AQLM_GROUP_TASKS;           // 8-row tasks per warp and tile (interleaved)
 constexpr int kWarpsPerTile = 8 / kTasks;          // a 64-row tile is 8 tasks
-constexpr int kTileGroups = 16 / kWarpsPerTile;    // warps of group j take tiles k = j (mod kTileGroups)
-static_assert(kTasks * kWarpsPerTile == 8 && (kTileGroups & (kTileGroups - 1)) == 0, "tile split");
+constexpr int kTileGroups = kWorkerWarps / kWarpsPerTile;  // warps of group j take tiles k = j (mod kTileGroups)
+static_assert(kTasks * kWarpsPerTile == 8 && kTileGroups * kWarpsPerTile == kWorkerWarps && kWorkerWarps >= 16,
+              "tile split");
 constexpr uint32_t kTmemCols = 512;                // D_0 at [0, 256), D_1 at [256, 512)
 
 constexpr uint32_t kOffLut = 0;
@@ -102,19 +109,25 @@ struct GroupLayerDev {
   long long row0;  // first output row of this layer in the reduction grid
 };
 
+// CTAs of one launch: one per SM (the host clamps the grid to this).
+constexpr int kMaxGroupCtas = 160;
+
 struct GroupParams {
   GroupLayerDev layer[kMaxGroupLayers];
   int count;
   long long items;
   long long rows;
   uint32_t* status;
+  // CTA c takes items [cta_item0[c], cta_item0[c + 1]): contiguous ranges of equal
+  // estimated cost (items plus the table builds they start, see build_group_launch)
+  long long cta_item0[kMaxGroupCtas + 1];
 };
 
 struct GroupMaps {
   CUtensorMap map[kMaxGroupLayers];
 };
 
-// Named barrier over the 16 worker warps that also ANDs a flag across them.
+// Named barrier over the worker warps that also ANDs a flag across them.
 __device__ __forceinline__ bool workers_sync_and(bool v) {
   uint32_t out;
   asm volatile(
@@ -226,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const long long it0 = p.items * blockIdx.x / gridDim.x;
-  const long long it1 = p.items * (blockIdx.x + 1) / gridDim.x;
+  const long long it0 = p.cta_item0[blockIdx.x];
+  const long long it1 = p.cta_item0[blockIdx.x + 1];
 
   // The next kernel in the stream (the reduction) may be scheduled now; it waits
   // for this grid to complete before it reads the partials.
@@ -345,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
           asm volatile("cp.async.commit_group;" ::: "memory");
           ok = workers_sync_and(done);
           tc_fence_after_sync();
-          if (ok) lut::store_table_2x8(tmem, warp, lane, smem + kOffLut);
+          if (ok && warp < 16) lut::store_table_2x8(tmem, warp, lane, smem + kOffLut);
           tc_fence_before_sync();
           ok = workers_sync_and(ok);  // table complete
         } else {
@@ -368,13 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
           asm volatile("cp.async.commit_group;" ::: "memory");
           ok = workers_sync_and(done);
           tc_fence_after_sync();
-          if (ok) lut::store_table_stacked(tmem, warp, lane, smem + kOffLut);
+          if (ok && warp < 16) lut::store_table_stacked(tmem, warp, lane, smem + kOffLut);
           tc_fence_before_sync();
           ok = workers_sync_and(ok);  // table complete
         }
         ++run;
       }
-      for (int i = (wg - kbase) & (kTileGroups - 1); i < run_len; i += kTileGroups) {
+      for (int i = ((wg - kbase) % kTileGroups + kTileGroups) % kTileGroups; i < run_len; i += kTileGroups) {
         const int k = kbase + i;
         const int my_slot = k % kSlots;
         const uint32_t my_ph = static_cast<uint32_t>((k / kSlots) & 1);
@@ -459,49 +472,69 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
   }
 }
 
-// y[n] = fp16(s_n * sum_s part[s][n] + bias_n).  A block takes 64 rows; thread
-// (row r, lane j) adds slices j, j + 4, j + 8, ... of row r (loads coalesced across
-// the 64 rows, and the thread's loads issued together, eight at a time), and the
-// four lane sums of a row are added in the order j = 0..3.  The order is fixed, so
-// the result does not depend on timing or on which CTA produced which partial.
-constexpr int kReduceRows = 64;
-constexpr int kReduceLanes = 4;
-__global__ void __launch_bounds__(kReduceRows* kReduceLanes) lut_group_reduce_kernel(
+// y[n] = fp16(s_n * sum_s part[s][n] + bias_n).  A block takes kReduceRows consecutive
+// rows of the launch's concatenated row space; thread t owns rows t, t + kReduceThreads,
+// ... of it (consecutive threads read consecutive rows of a slice: coalesced), issues
+// its loads eight slices at a time for all its rows and adds every row's slices in
+// ascending order.  The order is fixed, so the result does not depend on
+// timing or on which CTA produced which partial.
+#ifndef AQLM_REDUCE_THREADS
+#define AQLM_REDUCE_THREADS 128
+#endif
+#ifndef AQLM_REDUCE_ROWS_PER_THREAD
+#define AQLM_REDUCE_ROWS_PER_THREAD 1
+#endif
+constexpr int kReduceThreads = AQLM_REDUCE_THREADS;
+constexpr int kReduceRowsPerThread = AQLM_REDUCE_ROWS_PER_THREAD;
+constexpr int kReduceRows = kReduceThreads * kReduceRowsPerThread;
+// At most 48 registers a thread: a block then fits beside a partial-sum CTA (17 warps
+// of 96 registers), so the reduction's blocks are resident and waiting when that grid
+// completes, and the next call's CTAs are not held back by them.
+constexpr int kReduceMinBlocks = 65536 / (kReduceThreads * 48);
+__global__ void __launch_bounds__(kReduceThreads, kReduceMinBlocks) lut_group_reduce_kernel(
     const __grid_constant__ GroupParams p) {
-  __shared__ float sums[kReduceLanes][kReduceRows];
   grid_dependents_launch();
-  const int r = threadIdx.x % kReduceRows;
-  const int j = threadIdx.x / kReduceRows;
-  const long long row = static_cast<long long>(blockIdx.x) * kReduceRows + r;
-  const bool valid = row < p.rows;
+  const float* col[kReduceRowsPerThread];
+  int S[kReduceRowsPerThread], N[kReduceRowsPerThread], lay[kReduceRowsPerThread], nn[kReduceRowsPerThread];
+  int smax = 0;
   int l = 0;
-  while (l + 1 < p.count && p.layer[l + 1].row0 <= row) ++l;
-  const GroupLayerDev& L = p.layer[l];
-  const int n = static_cast<int>(row - L.row0);
+#pragma unroll
+  for (int k = 0; k < kReduceRowsPerThread; ++k) {
+    const long long row = static_cast<long long>(blockIdx.x) * kReduceRows + k * kReduceThreads + threadIdx.x;
+    while (l + 1 < p.count && p.layer[l + 1].row0 <= row) ++l;
+    const GroupLayerDev& L = p.layer[l];
+    const bool valid = row < p.rows;
+    lay[k] = l;
+    nn[k] = static_cast<int>(row - L.row0);
+    N[k] = L.N;
+    S[k] = valid ? L.S : 0;
+    col[k] = L.part + (valid ? nn[k] : 0);
+    smax = max(smax, S[k]);
+  }
   // the partials are the previous kernel's output
   grid_dependency_wait();
-  float acc = 0.f;
-  if (valid) {
-    const float* col = L.part + n;
-    for (int s0 = j; s0 < L.S; s0 += 8 * kReduceLanes) {
-      float v[8];
+  float acc[kReduceRowsPerThread];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int s = s0 + u * kReduceLanes;
-        v[u] = s < L.S ? col[static_cast<size_t>(s) * L.N] : 0.f;
-      }
+  for (int k = 0; k < kReduceRowsPerThread; ++k) acc[k] = 0.f;
+  for (int s0 = 0; s0 < smax; s0 += 8) {
+    float v[kReduceRowsPerThread][8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) acc += v[u];
-    }
+    for (int k = 0; k < kReduceRowsPerThread; ++k)
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[k][u] = s0 + u < S[k] ? col[k][static_cast<size_t>(s0 + u) * N[k]] : 0.f;
+#pragma unroll
+    for (int k = 0; k < kReduceRowsPerThread; ++k)
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc[k] += v[k][u];
   }
-  sums[j][r] = acc;
-  __syncthreads();
-  if (j == 0 && valid) {
-    float t = sums[0][r];
 #pragma unroll
-    for (int q = 1; q < kReduceLanes; ++q) t += sums[q][r];
+  for (int k = 0; k < kReduceRowsPerThread; ++k) {
+    if (S[k] == 0) continue;
+    const GroupLayerDev& L = p.layer[lay[k]];
+    const int n = nn[k];
     const float bi = L.bias ? __half2float(L.bias[n]) : 0.f;
-    L.y[n] = __float2half_rn(t * __half2float(L.scales[n]) + bi);
+    L.y[n] = __float2half_rn(acc[k] * __half2float(L.scales[n]) + bi);
   }
 }
 
@@ -629,7 +662,39 @@ cudaError_t build_group_launch(const Problem* probs, int count, void* workspace,
   p.items = items;
   p.rows = rows;
   p.status = status;
-  out->grid = static_cast<unsigned>(std::min<long long>(items, sms));
+  const int grid = static_cast<int>(std::min<long long>(std::min(items, static_cast<long long>(sms)), kMaxGroupCtas));
+  out->grid = static_cast<unsigned>(grid);
+  // Contiguous item ranges of equal estimated cost: an item (one 64-row code tile)
+  // costs 1, and every run of equal (layer, slice) costs kTableCost more for its
+  // lookup-table build (a build stalls a CTA's lookups for a few tile times; 3 timed
+  // best on B200 among 3, 5 and 8).  Layers with few rows have short runs, so a CTA
+  // whose range falls on them takes fewer items.
+#ifndef AQLM_GROUP_TABLE_COST
+#define AQLM_GROUP_TABLE_COST 3
+#endif
+  constexpr long long kTableCost = AQLM_GROUP_TABLE_COST;
+  long long total = 0;
+  for (int i = 0; i < count; ++i) total += static_cast<long long>(p.layer[i].S) * (p.layer[i].T + kTableCost);
+  p.cta_item0[0] = 0;
+  int next = 1;
+  long long cost = 0;  // cost of the items before the current run
+  for (int i = 0; i < count && next < grid; ++i) {
+    const GroupLayerDev& L = p.layer[i];
+    for (int sl = 0; sl < L.S && next < grid; ++sl) {
+      const long long run0 = L.item0 + static_cast<long long>(sl) * L.T;
+      const long long run_cost = L.T + kTableCost;
+      // boundaries whose target cost falls inside this run: target = next * total / grid
+      while (next < grid && static_cast<long long>(next) * total < (cost + run_cost) * grid) {
+        const long long target = (static_cast<long long>(next) * total + grid - 1) / grid;  // ceil
+        long long off = target - cost - kTableCost;  // items of the run before the boundary
+        off = std::max(0LL, std::min(off, static_cast<long long>(L.T)));
+        p.cta_item0[next] = std::max(p.cta_item0[next - 1], run0 + off);
+        ++next;
+      }
+      cost += run_cost;
+    }
+  }
+  for (; next <= grid; ++next) p.cta_item0[next] = items;
   out->rgrid = static_cast<unsigned>((rows + kReduceRows - 1) / kReduceRows);
   return cudaSuccess;
 }
@@ -709,7 +774,7 @@ cudaError_t launch_lut_group(const Problem* probs, int count, void* workspace, u
 
   cudaLaunchConfig_t rcfg = {};
   rcfg.gridDim = dim3(launch.rgrid, 1, 1);
-  rcfg.blockDim = dim3(kReduceRows * kReduceLanes, 1, 1);
+  rcfg.blockDim = dim3(kReduceThreads, 1, 1);
   rcfg.stream = stream;
   rcfg.attrs = attr;
   rcfg.numAttrs = 1;
