@@ -95,6 +95,13 @@ __device__ __forceinline__ float add_f32_hi_f16(uint32_t w, float acc) {
   return r;
 }
 
+// 32-byte read-only load with an L2 policy (g = 16 codeword gathers: evict_last).
+__device__ __forceinline__ void ldg_nc_v8_hint(const void* p, uint4& lo, uint4& hi, uint64_t pol) {
+  asm volatile("ld.global.nc.L2::cache_hint.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+               : "l"(p), "l"(pol));
+}
+
 __device__ __forceinline__ float2 h2_to_f2(uint32_t v) {
   __half2 h = *reinterpret_cast<__half2*>(&v);
   return __half22float2(h);
@@ -283,6 +290,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 // 16-byte cp.async (L2 only); `src_bytes` < 16 zero-fills the rest (0: all zeros).
 __device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// cp_async_16_zfill with an L2 cache policy (codebook gathers: evict_last).
+__device__ __forceinline__ void cp_async_16_zfill_hint(uint32_t dst, const void* src, uint32_t src_bytes,
+                                                       uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
+               "r"(src_bytes), "l"(pol) : "memory");
 }
 
 // Arrive on `bar` once every cp.async this thread issued so far has landed

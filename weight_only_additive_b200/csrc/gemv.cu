@@ -20,7 +20,7 @@ namespace {
 template <int M, int B, int G, int BATCH>
 __device__ __forceinline__ void accumulate_group(const __half* __restrict__ x, int K, int j,
                                                  const uint32_t (&code)[M],
-                                                 const __half* __restrict__ codebooks,
+                                                 const __half* __restrict__ codebooks, uint64_t cb_pol,
                                                  float (&acc)[BATCH]) {
   constexpr int kVec = G / 8;
   float w[G];
@@ -29,7 +29,7 @@ __device__ __forceinline__ void accumulate_group(const __half* __restrict__ x, i
     const __half* cw = codebooks + (static_cast<size_t>(m) * (1u << B) + code[m]) * G;
 #pragma unroll
     for (int v = 0; v < kVec; ++v) {
-      const uint4 q = ldg_nc_v4(cw + 8 * v);
+      const uint4 q = ldg_nc_v4_hint(cw + 8 * v, cb_pol);
       const uint32_t h[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(128) gemv_gather_kernel(
   const uint8_t* row = static_cast<const uint8_t*>(codes) + static_cast<size_t>(n) * row_bytes;
 
   const uint64_t stream_pol = l2_policy_evict_first();
+  // codebook lines are gathered all kernel long: keep them in L2
+  const uint64_t cb_pol = l2_policy_evict_last();
   float acc[BATCH];
 #pragma unroll
   for (int b = 0; b < BATCH; ++b) acc[b] = 0.f;
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(128) gemv_gather_kernel(
         const int byte = (gi * M + m) * kCodeBytes;  // little-endian position in the vector
         code[m] = (words[byte / 4] >> (8 * (byte % 4))) & ((1u << (8 * kCodeBytes)) - 1u);
       }
-      accumulate_group<M, B, G, BATCH>(x, K, v * kGroupsPerVec + gi, code, codebooks, acc);
+      accumulate_group<M, B, G, BATCH>(x, K, v * kGroupsPerVec + gi, code, codebooks, cb_pol, acc);
     }
   }
   // Remaining groups (ragged tail, or rows that are not 16-byte aligned).
@@ -105,7 +107,7 @@ __global__ void __launch_bounds__(128) gemv_gather_kernel(
     uint32_t code[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) code[m] = rc[static_cast<size_t>(j) * M + m];
-    accumulate_group<M, B, G, BATCH>(x, K, j, code, codebooks, acc);
+    accumulate_group<M, B, G, BATCH>(x, K, j, code, codebooks, cb_pol, acc);
   }
 
 #pragma unroll

@@ -270,23 +270,26 @@ __global__ void __launch_bounds__(kThreads, 1) lut_group_kernel(const __grid_con
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kProducerWarp) {
-    // ---- code tiles of every item of the range, in order (weights: no dependency wait) ----
-    if (lane == 0) {
+    // ---- code tiles of every item of the range (weights: no dependency wait) ----
+    // Tile k of the range goes to slot k mod kSlots and is read by warp group
+    // k mod kTileGroups, so each group owns every kTileGroups-th slot.  Producer lane j
+    // streams group j's tiles in order, waiting only for that group's slots: a group
+    // that falls behind holds back its own loads, not every group's.
+    static_assert(kSlots % kTileGroups == 0 && kTileGroups <= 32, "slots per warp group");
+    if (lane < kTileGroups) {
       const uint64_t pol = l2_policy_evict_first();
       ItemCursor c;
-      c.seek(p, it0);
-      int slot = 0;
-      uint32_t use = 0;
-      for (long long it = it0; it < it1; ++it, c.next(p)) {
+      c.seek(p, it0 + lane);
+      for (long long k = lane; it0 + k < it1; k += kTileGroups) {
+        const int slot = static_cast<int>(k % kSlots);
+        const uint32_t use = static_cast<uint32_t>(k / kSlots);
         if (use > 0 && !group_wait(&empty[slot], (use - 1u) & 1u, abort_flag, p.status, kSiteGroupRing)) break;
         mbar_arrive_expect_tx(&full[slot], kTileBytes);
         // bytes past the row end and rows past N are zero-filled
         tma_load_2d(sbase + kOffRing + static_cast<uint32_t>(slot) * kTileBytes, &maps.map[c.l], c.s * 128,
                     c.t * kTileRows, &full[slot], pol);
-        if (++slot == kSlots) {
-          slot = 0;
-          ++use;
-        }
+        if (it0 + k + kTileGroups < it1)
+          for (int i = 0; i < kTileGroups; ++i) c.next(p);
       }
     }
   } else {

@@ -218,7 +218,8 @@ __device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, volati
 // (i + rot) mod 4 (rot = 0 or 2).
 template <int M, int G>
 __device__ __forceinline__ void gather_stage_b16(uint4 (&v)[M][4], const uint8_t* cw, bool row_valid,
-                                                 const __half* __restrict__ codebooks, bool cb32, int rot = 0) {
+                                                 const __half* __restrict__ codebooks, bool cb32, uint64_t cb_pol,
+                                                 int rot = 0) {
   const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
   if (!row_valid) {
 #pragma unroll
@@ -232,16 +233,18 @@ __device__ __forceinline__ void gather_stage_b16(uint4 (&v)[M][4], const uint8_t
     const __half* cb = codebooks + static_cast<size_t>(m) * 65536u * G;
     if constexpr (G == 8) {
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) v[m][cc] = ldg_nc_v4(cb + static_cast<size_t>(c16[((cc + rot) & 3) * M + m]) * 8);
+      for (int cc = 0; cc < 4; ++cc)
+        v[m][cc] = ldg_nc_v4_hint(cb + static_cast<size_t>(c16[((cc + rot) & 3) * M + m]) * 8, cb_pol);
     } else if (cb32) {
 #pragma unroll
       for (int q = 0; q < 2; ++q)
-        ldg_nc_v8(cb + static_cast<size_t>(c16[(q ^ (rot >> 1)) * M + m]) * 16, v[m][2 * q], v[m][2 * q + 1]);
+        ldg_nc_v8_hint(cb + static_cast<size_t>(c16[(q ^ (rot >> 1)) * M + m]) * 16, v[m][2 * q], v[m][2 * q + 1],
+                       cb_pol);
     } else {
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int ch = (cc + rot) & 3;
-        v[m][cc] = ldg_nc_v4(cb + static_cast<size_t>(c16[(ch >> 1) * M + m]) * 16 + 8 * (ch & 1));
+        v[m][cc] = ldg_nc_v4_hint(cb + static_cast<size_t>(c16[(ch >> 1) * M + m]) * 16 + 8 * (ch & 1), cb_pol);
       }
     }
   }
@@ -353,7 +356,8 @@ __device__ __forceinline__ void decode_grad_b8(uint8_t* smem, uint32_t a_off, in
 template <int M, int B, int G>
 __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase, uint32_t a_off, int r, int hf,
                                                   bool row_valid, const uint8_t* cw,
-                                                  const __half* __restrict__ codebooks, const uint8_t* smem_cb) {
+                                                  const __half* __restrict__ codebooks, const uint8_t* smem_cb,
+                                                  uint64_t cb_pol) {
   if constexpr (B == 16) {
     static_assert(M == 1 && G == 8, "other B = 16 shapes use the register-staged decoder");
     const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
@@ -362,9 +366,9 @@ __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase,
       const int chunk = 4 * hf + cc;
       const uint32_t code = c16[cc];
       const __half* src = codebooks + static_cast<size_t>(code) * 8;
-      cp_async_16_zfill(sbase + a_off + swz128(r, chunk),
-                        row_valid ? static_cast<const void*>(src) : static_cast<const void*>(codebooks),
-                        row_valid ? 16u : 0u);
+      cp_async_16_zfill_hint(sbase + a_off + swz128(r, chunk),
+                             row_valid ? static_cast<const void*>(src) : static_cast<const void*>(codebooks),
+                             row_valid ? 16u : 0u, cb_pol);
     }
   } else if constexpr (M == 2 && G == 8) {
     // 2x8: the thread's 8 code bytes (c0, c1 per group) of this stage in one load
@@ -539,6 +543,9 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
       umma_commit(acc_bar);
     }
   } else {
+    // the 65536-entry codebooks of the B = 16 schemes are gathered from L2 all kernel
+    // long: keep their lines there while the code stream (evict_first) passes by
+    const uint64_t cb_pol = l2_policy_evict_last();
     if constexpr (kGrad) {
     // ---- decoders (input gradient): thread (row nl = 8 w + lane / 4, quarter qq =
     // lane % 4) decodes features 32 qq .. 32 qq + 31 of row (ks0 + i) 64 + nl at
@@ -581,7 +588,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
             const bool valid = n < p.N;
             sv[u] = valid ? __half2float(p.scales[n]) : 0.f;
             gather_stage_b16<M, G>(st[u], smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, valid,
-                                   p.codebooks, p.cb32 != 0, 2 * (qq >> 1));
+                                   p.codebooks, p.cb32 != 0, cb_pol, 2 * (qq >> 1));
             __syncwarp();  // every lane has read its codes of this tile
             if (lane == 0) mbar_arrive(&cempty[c]);
           }
@@ -672,7 +679,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
             const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
                                 code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                     r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
-            gather_stage_b16<M, G>(st[u], cw, row_valid, p.codebooks, p.cb32 != 0);
+            gather_stage_b16<M, G>(st[u], cw, row_valid, p.codebooks, p.cb32 != 0, cb_pol);
             if (within + kDecoderGroups >= kStagesPerTile || i + kDecoderGroups >= nks) {  // its last one
               __syncwarp();  // every lane has read its codes of this tile
               if (lane == 0) mbar_arrive(&cempty[c]);
@@ -714,7 +721,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
                             code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                 r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
         decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
-                                   p.codebooks, smem + L.cb);
+                                   p.codebooks, smem + L.cb, cb_pol);
         if constexpr (B == 16) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
         } else {
@@ -745,7 +752,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
                             code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                 r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
         decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
-                                   p.codebooks, smem + L.cb);
+                                   p.codebooks, smem + L.cb, cb_pol);
         if constexpr (B == 16) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
         } else {
