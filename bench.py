@@ -507,7 +507,10 @@ class Pool:
         torch, L = b.torch, b.L
         self.w, self.batch = w, batch
         copy_bytes = step_bytes(w, batch)
-        pool = max(2, math.ceil(3 * b.l2 / copy_bytes)) if copies is None else max(1, copies)
+        # at least 3x L2 so no step finds its weights in L2, and at least 8 copies so a
+        # CUDA graph holds 8 steps: consecutive launches overlap through programmatic
+        # dependent launch inside a graph, not across graph launches
+        pool = max(8, math.ceil(3 * b.l2 / copy_bytes)) if copies is None else max(1, copies)
         while pool > 2 and pool * copy_bytes > 60e9:
             pool -= 1
         self.size, self.copy_bytes = pool, copy_bytes
