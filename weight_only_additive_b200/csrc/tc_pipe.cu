@@ -76,6 +76,7 @@ struct PipeParams {
   int red_rows;    // split-K reduction: weight rows each CTA of the cluster owns
   uint32_t tmem_cols;
   int cb32;        // codebooks 32-byte aligned: g = 16 codewords in one 256-bit load
+  int cb_sh;       // 2x8 g8 codebook copies in shared memory: 8 >> cb_sh of them (cb_layout_offset)
   uint32_t* status;
 };
 
@@ -93,7 +94,11 @@ struct PipeScheme {
   static constexpr uint32_t kCodeTileBytes = static_cast<uint32_t>(kRows * kTileRowBytes);
   static constexpr bool kSwizzle64 = kTileRowBytes == 64;
   static constexpr bool kSmemCb = B == 8;
-  static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;
+  // 2x8 g8: up to eight copies of each codebook in shared memory (cb_layout_offset), so
+  // that the eight lanes of a quarter-warp phase read random codewords with few or no
+  // bank conflicts; the host picks the count that still leaves room for three stages
+  static constexpr int kCbMaxReplicas = (B == 8 && M == 2 && G == 8) ? 8 : 1;
+  static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;  // one copy
   static constexpr int kSplitAlign = 16 / gcd_int(16, kStageCodeBytes);  // split starts: 16-byte code offsets
   static_assert(kTileRowBytes % kStageCodeBytes == 0 && kTileRowBytes % 16 == 0, "code tile rows");
   // every full code tile holds stages of both decoder groups
@@ -120,6 +125,7 @@ struct GradScheme {
   static constexpr bool kSwizzle64 = false;
   static constexpr uint32_t kCodeTileBytes = static_cast<uint32_t>(kStageK * kBoxBytes);
   static constexpr bool kSmemCb = B == 8;
+  static constexpr int kCbMaxReplicas = 1;
   static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;
   static constexpr int kSplitAlign = 1;
   // a decoder thread reads the codes of a quarter of the tile's features
@@ -155,6 +161,17 @@ __device__ __forceinline__ uint32_t mapa_shared_cluster(uint32_t addr, uint32_t 
 
 __device__ __forceinline__ uint32_t swz128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// Shared-memory offset, within one codebook's region, of 16-byte codeword e in copy j
+// of R = 8 >> sh copies.  A codebook region is 256 / (8 / R) rows of 128 bytes; copy j
+// owns the 16-byte columns j (8 / R) .. j (8 / R) + 8 / R - 1 of every row, and entry e
+// sits in row e / (8 / R), column j (8 / R) + e mod (8 / R).  Lane l of a warp reads
+// copy l mod R, so the eight lanes of a quarter-warp phase share each column group
+// with 8 / R - 1 others only (R = 8: none, conflict-free; R = 1: the plain [256][16 B]
+// layout, which this formula reduces to).
+__device__ __forceinline__ uint32_t cb_layout_offset(uint32_t e, uint32_t j, int sh) {
+  return ((e >> sh) << 7) | (((j << sh) | (e & ((1u << sh) - 1u))) << 4);
 }
 
 // MN-major 128-byte-swizzled A stage of the input-gradient kernel: feature k
@@ -357,7 +374,7 @@ template <int M, int B, int G>
 __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase, uint32_t a_off, int r, int hf,
                                                   bool row_valid, const uint8_t* cw,
                                                   const __half* __restrict__ codebooks, const uint8_t* smem_cb,
-                                                  uint64_t cb_pol) {
+                                                  uint64_t cb_pol, int cb_sh) {
   if constexpr (B == 16) {
     static_assert(M == 1 && G == 8, "other B = 16 shapes use the register-staged decoder");
     const uint16_t* c16 = reinterpret_cast<const uint16_t*>(cw);
@@ -380,8 +397,12 @@ __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase,
       if (row_valid) {
         const uint32_t c0 = (cwords[cc >> 1] >> (16 * (cc & 1))) & 0xFFu;
         const uint32_t c1 = (cwords[cc >> 1] >> (16 * (cc & 1) + 8)) & 0xFFu;
-        const uint4 pieces[2] = {*reinterpret_cast<const uint4*>(smem_cb + (c0 << 4)),
-                                 *reinterpret_cast<const uint4*>(smem_cb + 4096u + (c1 << 4))};
+        // the thread reads copy r mod R of each codebook (r mod 32 is its lane); the
+        // second codebook's region follows the first's (4 KB per copy)
+        const uint32_t j = static_cast<uint32_t>(r) & ((8u >> cb_sh) - 1u);
+        const uint4 pieces[2] = {
+            *reinterpret_cast<const uint4*>(smem_cb + cb_layout_offset(c0, j, cb_sh)),
+            *reinterpret_cast<const uint4*>(smem_cb + (32768u >> cb_sh) + cb_layout_offset(c1, j, cb_sh))};
         out = sum_pieces<2>(pieces);
       }
       *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = out;
@@ -430,7 +451,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
   constexpr int kStagesPerTile = SC::kStagesPerTile;
   constexpr uint32_t kCodeTileBytes = SC::kCodeTileBytes;
   const int S = p.S;
-  const PipeLayout L = pipe_layout(S, p.BN, kCodeTileBytes, SC::kCbBytes);
+  const PipeLayout L = pipe_layout(S, p.BN, kCodeTileBytes, SC::kCbBytes * (8u >> p.cb_sh));
   const uint32_t sbase = smem_addr(smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);   // stage s decoded and x landed
   uint64_t* empty = full + S;                                     // stage s consumed by the MMAs
@@ -472,9 +493,20 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if constexpr (SC::kSmemCb) {
-    // the M codebooks, [M][256][G] fp16, copied as they are
-    for (int i = tid; i < static_cast<int>(SC::kCbBytes / 16u); i += kThreads)
-      *reinterpret_cast<uint4*>(smem + L.cb + 16u * static_cast<uint32_t>(i)) = ldg_nc_v4(p.codebooks + 8 * i);
+    if constexpr (SC::kCbMaxReplicas == 1) {
+      // the M codebooks, [M][256][G] fp16, copied as they are
+      for (int i = tid; i < static_cast<int>(SC::kCbBytes / 16u); i += kThreads)
+        *reinterpret_cast<uint4*>(smem + L.cb + 16u * static_cast<uint32_t>(i)) = ldg_nc_v4(p.codebooks + 8 * i);
+    } else {
+      // 2x8 g8: every copy of codeword e of codebook m (cb_layout_offset)
+      const int reps = 8 >> p.cb_sh;
+      for (int i = tid; i < M * 256 * reps; i += kThreads) {
+        const int j = i % reps, me = i / reps;  // copy, codeword m * 256 + e
+        const uint32_t m = static_cast<uint32_t>(me >> 8), e = static_cast<uint32_t>(me & 255);
+        *reinterpret_cast<uint4*>(smem + L.cb + m * (32768u >> p.cb_sh) +
+                                  cb_layout_offset(e, static_cast<uint32_t>(j), p.cb_sh)) = ldg_nc_v4(p.codebooks + 8 * me);
+      }
+    }
   }
   if (warp == 0) tmem_alloc(tmem_slot, p.tmem_cols);
   tc_fence_before_sync();
@@ -721,7 +753,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
                             code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                 r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
         decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
-                                   p.codebooks, smem + L.cb, cb_pol);
+                                   p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
         if constexpr (B == 16) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
         } else {
@@ -752,7 +784,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
                             code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                 r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
         decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
-                                   p.codebooks, smem + L.cb, cb_pol);
+                                   p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
         if constexpr (B == 16) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
         } else {
@@ -875,7 +907,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
 // per CTA through distributed shared memory; measured on B200 it costs about two
 // stage times per 16 batch columns, which makes SK = 1 the choice for wide batches.
 struct TcPlan {
-  int S = 0, SK = 1, ks_per = 0, red_rows = 128;
+  int S = 0, SK = 1, ks_per = 0, red_rows = 128, cb_sh = 3;
 };
 
 constexpr int kPlanFixedStages = 3;     // set-up, pipeline fill and epilogue, in stage times
@@ -886,9 +918,9 @@ template <int M, int B, int G, bool kGrad>
 using PipeSchemeOf = std::conditional_t<kGrad, GradScheme<M, B, G>, PipeScheme<M, B, G>>;
 
 template <int M, int B, int G, bool kGrad>
-inline uint32_t pipe_smem_bytes(int S, int BN) {
+inline uint32_t pipe_smem_bytes(int S, int BN, int cb_sh) {
   using SC = PipeSchemeOf<M, B, G, kGrad>;
-  return pipe_layout(S, BN, SC::kCodeTileBytes, SC::kCbBytes).total + 1024;
+  return pipe_layout(S, BN, SC::kCodeTileBytes, SC::kCbBytes * (8u >> cb_sh)).total + 1024;
 }
 
 // rows: output rows (the MMA's M extent); nk: 64-wide reduction stages.
@@ -916,10 +948,22 @@ cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, TcPlan* out)
   const int row_tiles = (rows + kRows - 1) / kRows;
   const int batch_tiles = (batch + BN - 1) / BN;
   const long long clusters = static_cast<long long>(row_tiles) * batch_tiles;
+  // codebook copies (2x8 g8): the most that still leave room for three stages.
+  // Measured on 11008 x 4096: 8 copies made batch 4-64 11 % faster, but at batch 256
+  // they left room for two stages only and the kernel ran 1.8x slower.
+  int cb_sh = 3;
+  if constexpr (PipeSchemeOf<M, B, G, kGrad>::kCbMaxReplicas > 1) {
+    for (int sh = 0; sh < 3; ++sh)
+      if (pipe_smem_bytes<M, B, G, kGrad>(3, BN, sh) <= kSmemLimit) {
+        cb_sh = sh;
+        break;
+      }
+  }
   TcPlan best;
+  best.cb_sh = cb_sh;
   long long best_cost = -1;
   for (int S = 6; S >= 2; --S) {
-    const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(S, BN);
+    const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(S, BN, cb_sh);
     if (smem > kSmemLimit) continue;
     const uint32_t stage_bytes = static_cast<uint32_t>(S) * (kABytes + static_cast<uint32_t>(BN) * 128u);
     for (int SK = 1; SK <= cmax; ++SK) {
@@ -1004,8 +1048,9 @@ cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, si
   p.SK = plan.SK;
   p.ks_per = plan.ks_per;
   p.red_rows = plan.red_rows;
+  p.cb_sh = plan.cb_sh;
   p.cb32 = (reinterpret_cast<uintptr_t>(p.codebooks) & 31u) == 0 ? 1 : 0;
-  const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(plan.S, p.BN);
+  const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(plan.S, p.BN, plan.cb_sh);
   auto kern = tc_pipe_kernel<M, B, G, kGrad>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
   if (e != cudaSuccess) return e;
