@@ -125,8 +125,9 @@ struct GradScheme {
   static constexpr bool kSwizzle64 = false;
   static constexpr uint32_t kCodeTileBytes = static_cast<uint32_t>(kStageK * kBoxBytes);
   static constexpr bool kSmemCb = B == 8;
-  static constexpr int kCbMaxReplicas = 1;
-  static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;
+  // 2x8 g8: codebook copies as in the layer kernel (decode_grad_b8)
+  static constexpr int kCbMaxReplicas = (B == 8 && M == 2 && G == 8) ? 8 : 1;
+  static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;  // one copy
   static constexpr int kSplitAlign = 1;
   // a decoder thread reads the codes of a quarter of the tile's features
   static_assert(kTileCodeBytes % 8 == 0 && kBoxBytes <= 64, "gradient code tiles");
@@ -338,10 +339,12 @@ __device__ __forceinline__ int grad_chunk_at(int step, int qq) { return (step + 
 // Input gradient, B = 8: decode the 4 chunks (32 features) of row `n` that thread
 // quarter `qq` owns into the MN-major A stage at shared offset `a_off`.  `cw`
 // points at the quarter's codes ([group][m], 1 byte each); `smem_cb` holds the M
-// codebooks [M][256][G].
+// codebooks [M][256][G], or for 2x8 g8 the 8 >> cb_sh copies of cb_layout_offset (the
+// thread reads copy `lane` mod R).
 template <int M, int G>
 __device__ __forceinline__ void decode_grad_b8(uint8_t* smem, uint32_t a_off, int n, int qq, bool row_valid,
-                                               const uint8_t* cw, const uint8_t* smem_cb, float s) {
+                                               const uint8_t* cw, const uint8_t* smem_cb, float s, int cb_sh,
+                                               int lane) {
   constexpr uint32_t kCbStride = 256u * G * 2u;
 #pragma unroll
   for (int step = 0; step < 4; ++step) {
@@ -350,11 +353,19 @@ __device__ __forceinline__ void decode_grad_b8(uint8_t* smem, uint32_t a_off, in
     uint4 out = make_uint4(0u, 0u, 0u, 0u);
     if (row_valid) {
       uint4 pieces[M];
+      if constexpr (M == 2 && G == 8) {
+        const uint32_t cj = static_cast<uint32_t>(lane) & ((8u >> cb_sh) - 1u);
 #pragma unroll
-      for (int m = 0; m < M; ++m)
-        pieces[m] = *reinterpret_cast<const uint4*>(smem_cb + static_cast<uint32_t>(m) * kCbStride +
-                                                    static_cast<uint32_t>(cw[j * M + m]) * (G * 2u) +
-                                                    16u * static_cast<uint32_t>(h));
+        for (int m = 0; m < M; ++m)
+          pieces[m] = *reinterpret_cast<const uint4*>(smem_cb + static_cast<uint32_t>(m) * (32768u >> cb_sh) +
+                                                      cb_layout_offset(cw[j * M + m], cj, cb_sh));
+      } else {
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+          pieces[m] = *reinterpret_cast<const uint4*>(smem_cb + static_cast<uint32_t>(m) * kCbStride +
+                                                      static_cast<uint32_t>(cw[j * M + m]) * (G * 2u) +
+                                                      16u * static_cast<uint32_t>(h));
+      }
       out = scaled_sum_pieces<M>(pieces, s);
     }
     *reinterpret_cast<uint4*>(smem + a_off + grad_a_offset(n, 4 * qq + cc)) = out;
@@ -662,7 +673,8 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         const int n_next = n + kDecoderGroups * kStageK;
         if (i + kDecoderGroups < nks) s_next = n_next < p.N ? __half2float(p.scales[n_next]) : 0.f;
         decode_grad_b8<M, G>(smem, L.a + static_cast<uint32_t>(s) * kABytes, nl, qq, n < p.N,
-                             smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, smem + L.cb, sc);
+                             smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, smem + L.cb, sc,
+                             p.cb_sh, lane);
         fence_proxy_async_smem();
         mbar_arrive(&full[s]);
         __syncwarp();
