@@ -92,3 +92,40 @@ def test_static_scratch_rejects_groups_over_its_size(dev):
     assert native.aqlm_group_workspace_size(arr, 10) > native.STATIC_GROUP_SCRATCH_BYTES
     assert native.lib().aqlm_static_group_scratch_bytes() == native.STATIC_GROUP_SCRATCH_BYTES
     assert native.lib().aqlm_matmul_group_static(arr, 10, None) == Status.INVALID_ARG
+
+
+def test_static_scratch_holds_the_mixtral_expert_set(dev):
+    """The 24 expert linears of a Mixtral-8x7B layer (2x8 g8, batch 1) need 11 MB of
+    partials: one launch on the static buffer, bitwise equal to the caller-workspace
+    call and within tolerance of the oracle on sampled rows."""
+    w = workloads.get("mixtral_8x7b_experts_2x8g8")
+    layers, xs = [], []
+    for i, lay in enumerate(w.layers):
+        s = lay.scheme
+        ld = synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=52, layer=i)
+        layers.append((ld, L.AqlmWeights.from_numpy(ld, dev)))
+        xs.append(synth.make_x(1, lay.K, seed=52, layer=i))
+    xts = [torch.from_numpy(x).to(dev) for x in xs]
+    outs_static = [torch.empty((1, lay.N), dtype=torch.float16, device=dev) for lay in w.layers]
+    outs_ws = [torch.empty((1, lay.N), dtype=torch.float16, device=dev) for lay in w.layers]
+    n = len(layers)
+    probs_static = _problems(layers, xts, outs_static)
+    probs_ws = _problems(layers, xts, outs_ws)
+    need = native.aqlm_group_workspace_size(probs_ws, n)
+    assert 8 << 20 < need <= native.STATIC_GROUP_SCRATCH_BYTES
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    native.aqlm_matmul_group_static(probs_static, stream, count=n)
+    ws = torch.empty((need,), dtype=torch.uint8, device=dev)
+    native.aqlm_matmul_group(probs_ws, ws.data_ptr(), need, stream, count=n)
+    torch.cuda.synchronize()
+    st, detail = L.check_device_status()
+    assert st == Status.OK, hex(detail)
+    rng = np.random.Generator(np.random.PCG64(53))
+    for i, ((ld, wt), x, a, b) in enumerate(zip(layers, xs, outs_static, outs_ws)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"layer {i}"
+        if i % 3 == 0 or i % 3 == 2:  # a w1 and the w2 of every expert
+            rows = np.unique(np.concatenate([rng.choice(wt.N, size=12, replace=False), [0, wt.N - 1]]))
+            y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, wt.M, wt.B, wt.g, rows=rows)
+            got = a.cpu().numpy()[:, rows].astype(np.float64)
+            err = np.abs(got - y_ref).max() / max(np.abs(y_ref).max(), 1e-30)
+            assert np.isfinite(got).all() and err <= TOL, (i, err)

@@ -57,8 +57,12 @@ struct PipeShape {
   static constexpr int kDecoders = kGroups * kGroupThreads;
   static constexpr int kThreads = kDecoders + 96;
 };
-constexpr uint32_t kABytes = kRows * 128u;   // 16 KB per A stage
-constexpr int kCodeSlots = 4;
+constexpr uint32_t kABytes = kRows * 128u;   // 16 KB per A stage (in shared memory)
+// A stages kept in tensor memory: the accumulator takes columns [0, 256) of a 512-column
+// allocation and A stage s columns [kATmemCol + 32 s, + 32) (128 rows x 64 fp16).
+constexpr uint32_t kATmemCol = 256;
+constexpr int kMaxATmemStages = 8;
+constexpr int kCodeSlots = 4;          // code-tile slots at most (the plan may use 2: PipeParams::cs_log)
 constexpr uint32_t kSmemLimit = 227u * 1024u;
 
 struct PipeParams {
@@ -77,6 +81,7 @@ struct PipeParams {
   uint32_t tmem_cols;
   int cb32;        // codebooks 32-byte aligned: g = 16 codewords in one 256-bit load
   int cb_sh;       // 2x8 g8 codebook copies in shared memory: 8 >> cb_sh of them (cb_layout_offset)
+  int cs_log;      // code-tile ring of 1 << cs_log slots (2 or 4)
   uint32_t* status;
 };
 
@@ -94,6 +99,11 @@ struct PipeScheme {
   static constexpr uint32_t kCodeTileBytes = static_cast<uint32_t>(kRows * kTileRowBytes);
   static constexpr bool kSwizzle64 = kTileRowBytes == 64;
   static constexpr bool kSmemCb = B == 8;
+  // Decoded A stages may live in tensor memory (tcgen05.st, the MMA reading A from TMEM)
+  // for every scheme decoded through registers; 1x16 g8 copies codewords into shared
+  // memory by cp.async, so its A stages stay there.  The host picks the kATmem
+  // instantiation per launch (pipe_kernel).
+  static constexpr bool kATmemOk = !(B == 16 && M == 1 && G == 8);
   // 2x8 g8: up to eight copies of each codebook in shared memory (cb_layout_offset), so
   // that the eight lanes of a quarter-warp phase read random codewords with few or no
   // bank conflicts; the host picks the count that still leaves room for three stages
@@ -125,6 +135,7 @@ struct GradScheme {
   static constexpr bool kSwizzle64 = false;
   static constexpr uint32_t kCodeTileBytes = static_cast<uint32_t>(kStageK * kBoxBytes);
   static constexpr bool kSmemCb = B == 8;
+  static constexpr bool kATmemOk = false;  // the MN-major A stage stays in shared memory
   // 2x8 g8: codebook copies as in the layer kernel (decode_grad_b8)
   static constexpr int kCbMaxReplicas = (B == 8 && M == 2 && G == 8) ? 8 : 1;
   static constexpr uint32_t kCbBytes = kSmemCb ? static_cast<uint32_t>(M * 256 * G * 2) : 0u;  // one copy
@@ -137,12 +148,14 @@ struct PipeLayout {
   uint32_t a, b, codes, cb, bars, total;
 };
 
-__host__ __device__ inline PipeLayout pipe_layout(int S, int BN, uint32_t code_tile_bytes, uint32_t cb_bytes) {
+// a_stage_bytes: kABytes, or 0 when the A stages live in tensor memory.
+__host__ __device__ inline PipeLayout pipe_layout(int S, int BN, uint32_t code_tile_bytes, uint32_t cb_bytes,
+                                                  int code_slots, uint32_t a_stage_bytes) {
   PipeLayout L;
   L.a = 0;                                                          // 1024-aligned stages
-  L.b = L.a + static_cast<uint32_t>(S) * kABytes;
+  L.b = L.a + static_cast<uint32_t>(S) * a_stage_bytes;
   L.codes = L.b + static_cast<uint32_t>(S) * static_cast<uint32_t>(BN) * 128u;
-  L.cb = L.codes + kCodeSlots * code_tile_bytes;
+  L.cb = L.codes + static_cast<uint32_t>(code_slots) * code_tile_bytes;
   L.bars = L.cb + cb_bytes;
   // full[S], empty[S], code_full[kCodeSlots], code_empty[kCodeSlots], acc, tmem slot, abort flag
   L.total = L.bars + 8u * static_cast<uint32_t>(2 * S + 2 * kCodeSlots + 1) + 16u;
@@ -372,6 +385,28 @@ __device__ __forceinline__ void decode_grad_b8(uint8_t* smem, uint32_t a_off, in
   }
 }
 
+// The thread's 4 decoded 16-byte chunks of weight row r (chunks 4 hf .. 4 hf + 3 of a
+// 64-wide stage) into the A stage: shared memory (128-byte swizzled K-major layout at
+// a_off), or tensor memory (to_tmem: lane r, columns 16 hf .. 16 hf + 15 of the stage at
+// a_tmem, which carries the warp's lane quadrant; warp-collective, waits for the stores).
+__device__ __forceinline__ void store_a_half(bool to_tmem, uint8_t* smem, uint32_t a_off, uint32_t a_tmem, int r,
+                                             int hf, const uint4 (&out)[4]) {
+  if (to_tmem) {
+    uint32_t v[16];
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      v[4 * cc] = out[cc].x;
+      v[4 * cc + 1] = out[cc].y;
+      v[4 * cc + 2] = out[cc].z;
+      v[4 * cc + 3] = out[cc].w;
+    }
+    tmem_st_32x32b_x16_wait(a_tmem + 16u * static_cast<uint32_t>(hf), v);
+  } else {
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = out[cc];
+  }
+}
+
 // Decode half (`hf` = 0: chunks 0-3, 1: chunks 4-7) of one 64-wide K stage of
 // weight row `r` into the swizzled A stage at shared offset `a_off`.  `cw` points at
 // the codes of this half of the stage (half the stage's code bytes, never crossing a
@@ -382,8 +417,8 @@ __device__ __forceinline__ void decode_grad_b8(uint8_t* smem, uint32_t a_off, in
 //   B = 8: the codebooks are staged in shared memory ([M][256][G]); a chunk is the
 //     sum of the matching 16-byte pieces of the group's M codewords.
 template <int M, int B, int G>
-__device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase, uint32_t a_off, int r, int hf,
-                                                  bool row_valid, const uint8_t* cw,
+__device__ __forceinline__ void decode_half_stage(bool to_tmem, uint8_t* smem, uint32_t sbase, uint32_t a_off,
+                                                  uint32_t a_tmem, int r, int hf, bool row_valid, const uint8_t* cw,
                                                   const __half* __restrict__ codebooks, const uint8_t* smem_cb,
                                                   uint64_t cb_pol, int cb_sh) {
   if constexpr (B == 16) {
@@ -402,9 +437,10 @@ __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase,
     // 2x8: the thread's 8 code bytes (c0, c1 per group) of this stage in one load
     const uint2 q = *reinterpret_cast<const uint2*>(cw);
     const uint32_t cwords[2] = {q.x, q.y};
+    uint4 out[4];
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      uint4 out = make_uint4(0u, 0u, 0u, 0u);
+      out[cc] = make_uint4(0u, 0u, 0u, 0u);
       if (row_valid) {
         const uint32_t c0 = (cwords[cc >> 1] >> (16 * (cc & 1))) & 0xFFu;
         const uint32_t c1 = (cwords[cc >> 1] >> (16 * (cc & 1) + 8)) & 0xFFu;
@@ -414,17 +450,20 @@ __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase,
         const uint4 pieces[2] = {
             *reinterpret_cast<const uint4*>(smem_cb + cb_layout_offset(c0, j, cb_sh)),
             *reinterpret_cast<const uint4*>(smem_cb + (32768u >> cb_sh) + cb_layout_offset(c1, j, cb_sh))};
-        out = sum_pieces<2>(pieces);
+        out[cc] = sum_pieces<2>(pieces);
       }
-      *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = out;
+      // shared-memory A: each chunk stored as soon as it is decoded (measured faster than
+      // one store burst at the end)
+      if (!to_tmem) *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = out[cc];
     }
+    if (to_tmem) store_a_half(true, smem, a_off, a_tmem, r, hf, out);
   } else {
     constexpr uint32_t kCbStride = 256u * G * 2u;  // bytes per codebook
+    uint4 out[4];
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      const int chunk = 4 * hf + cc;
       const int j = cc / (G / 8), h = cc % (G / 8);  // group within the half, 16-byte piece
-      uint4 out = make_uint4(0u, 0u, 0u, 0u);
+      out[cc] = make_uint4(0u, 0u, 0u, 0u);
       if (row_valid) {
         uint4 pieces[M];
 #pragma unroll
@@ -432,10 +471,11 @@ __device__ __forceinline__ void decode_half_stage(uint8_t* smem, uint32_t sbase,
           pieces[m] = *reinterpret_cast<const uint4*>(smem_cb + static_cast<uint32_t>(m) * kCbStride +
                                                       static_cast<uint32_t>(cw[j * M + m]) * (G * 2u) +
                                                       16u * static_cast<uint32_t>(h));
-        out = sum_pieces<M>(pieces);
+        out[cc] = sum_pieces<M>(pieces);
       }
-      *reinterpret_cast<uint4*>(smem + a_off + swz128(r, chunk)) = out;
+      if (!to_tmem) *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = out[cc];
     }
+    if (to_tmem) store_a_half(true, smem, a_off, a_tmem, r, hf, out);
   }
 }
 
@@ -446,7 +486,9 @@ __device__ __forceinline__ void cluster_barrier() {
 // kGrad = false: y = x . W16^T . diag(s) + bias (rows = N, reduction over K).
 // kGrad = true:  dx = dy . W16 (rows = K input features, reduction over the N
 //                output rows; x_map then describes dy [batch, N]).
-template <int M, int B, int G, bool kGrad>
+// kATmem: the decoded A stages live in tensor memory (schemes with kATmemOk); a separate
+// instantiation, since the same loops with a runtime switch compiled measurably slower.
+template <int M, int B, int G, bool kGrad, bool kATmem>
 __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     tc_pipe_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap code_map,
                    const PipeParams p) {
@@ -462,7 +504,12 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
   constexpr int kStagesPerTile = SC::kStagesPerTile;
   constexpr uint32_t kCodeTileBytes = SC::kCodeTileBytes;
   const int S = p.S;
-  const PipeLayout L = pipe_layout(S, p.BN, kCodeTileBytes, SC::kCbBytes * (8u >> p.cb_sh));
+  static_assert(!kATmem || SC::kATmemOk, "A in tensor memory needs a register-decoded scheme");
+  constexpr bool a_in_tmem = kATmem;
+  const PipeLayout L =
+      pipe_layout(S, p.BN, kCodeTileBytes, SC::kCbBytes * (8u >> p.cb_sh), 1 << p.cs_log, a_in_tmem ? 0u : kABytes);
+  const int cs_log = p.cs_log;          // code-tile slots: 1 << cs_log
+  const int cs_mask = (1 << cs_log) - 1;
   const uint32_t sbase = smem_addr(smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);   // stage s decoded and x landed
   uint64_t* empty = full + S;                                     // stage s consumed by the MMAs
@@ -546,7 +593,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
       for (int t = 0; t < nct; ++t) {
-        const int c = t % kCodeSlots, u = t / kCodeSlots;
+        const int c = t & cs_mask, u = t >> cs_log;
         if (u > 0 && !pipe_wait(&cempty[c], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeCodes))
           break;
         mbar_arrive_expect_tx(&cfull[c], kCodeTileBytes);
@@ -572,14 +619,22 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         if (!pipe_wait(&full[s], static_cast<uint32_t>((i / S) & 1), abort_flag, p.status, kSitePipeFull)) break;
         fence_proxy_async_smem();  // decoder writes (cp.async / st.shared) -> tensor-core reads
         tc_fence_after_sync();
-        const uint32_t a_addr = sbase + L.a + static_cast<uint32_t>(s) * kABytes;
         const uint64_t bdesc = umma_desc_sw128_kmajor(sbase + L.b + static_cast<uint32_t>(s * p.BN) * 128u);
+        if (a_in_tmem) {
+          // A stage s at TMEM columns kATmemCol + 32 s: 8 columns (16 fp16) per K = 16 step
+          const uint32_t a_tmem = tmem + kATmemCol + 32u * static_cast<uint32_t>(s);
 #pragma unroll
-        for (int kk = 0; kk < kStageK / 16; ++kk) {
-          // K = 16 per MMA: 32 bytes along a K-major row, or two 8-row atoms (2 x SBO) MN-major
-          const uint64_t adesc = kGrad ? umma_desc_sw128_mnmajor(a_addr + 2u * kGradSbo * kk, kGradLbo, kGradSbo)
-                                       : umma_desc_sw128_kmajor(a_addr) + 2 * kk;
-          umma_f16_ss(tmem, adesc, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kStageK / 16; ++kk)
+            umma_f16_ts(tmem, a_tmem + 8u * kk, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        } else {
+          const uint32_t a_addr = sbase + L.a + static_cast<uint32_t>(s) * kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kStageK / 16; ++kk) {
+            // K = 16 per MMA: 32 bytes along a K-major row, or two 8-row atoms (2 x SBO) MN-major
+            const uint64_t adesc = kGrad ? umma_desc_sw128_mnmajor(a_addr + 2u * kGradSbo * kk, kGradLbo, kGradSbo)
+                                         : umma_desc_sw128_kmajor(a_addr) + 2 * kk;
+            umma_f16_ss(tmem, adesc, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&empty[s]);
       }
@@ -613,11 +668,11 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
           const int i = grp + kDecoderGroups * ki;    // stage gathered now
           const int j = grp + kDecoderGroups * kj;    // stage stored now
           const bool issue = ki < nmine, store = kj >= 0 && kj < nmine;
-          const int c = i % kCodeSlots;
+          const int c = i & cs_mask;
           const int sj = j >= 0 ? j % S : 0, uj = j >= 0 ? j / S : 0;
           bool ready = true;
           if (issue)
-            ready = pipe_wait(&cfull[c], static_cast<uint32_t>((i / kCodeSlots) & 1), abort_flag, p.status,
+            ready = pipe_wait(&cfull[c], static_cast<uint32_t>((i >> cs_log) & 1), abort_flag, p.status,
                               kSitePipeCodes);
           if (ready && store && uj > 0)
             ready = pipe_wait(&empty[sj], static_cast<uint32_t>((uj - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
@@ -658,8 +713,8 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
       const int n_first = (ks0 + grp) * kStageK + nl;
       float s_next = (grp < nks && n_first < p.N) ? __half2float(p.scales[n_first]) : 0.f;
       for (int i = grp; i < nks; i += kDecoderGroups) {
-        const int c = i % kCodeSlots;
-        bool ready = pipe_wait(&cfull[c], static_cast<uint32_t>((i / kCodeSlots) & 1), abort_flag, p.status,
+        const int c = i & cs_mask;
+        bool ready = pipe_wait(&cfull[c], static_cast<uint32_t>((i >> cs_log) & 1), abort_flag, p.status,
                                kSitePipeCodes);
         const int s = i % S, u = i / S;
         if (ready && u > 0)
@@ -684,6 +739,9 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     } else {
     // ---- decoders: threads r and r + 128 share weight row n0 + r (chunks 0-3 / 4-7) ----
     const int r = tid & (kRows - 1);
+    // A stages in tensor memory: the warp's lane quadrant (rows 32 (warp mod 4) ..) at
+    // the A columns (stage s adds 32 s)
+    const uint32_t a_tmem_q = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kATmemCol;
     const int hf = kDecoderGroups == 1 ? tid >> 7 : (tid >> 7) & 1;
     const int grp = kDecoderGroups == 1 ? 0 : tid / kGroupThreads;
     const bool row_valid = n0 + r < p.N;
@@ -705,12 +763,12 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
           const int i = grp + kDecoderGroups * ki;    // stage gathered now
           const int j = grp + kDecoderGroups * kj;    // stage stored now
           const bool issue = ki < nmine, store = kj >= 0 && kj < nmine;
-          const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
+          const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t & cs_mask;
           const int sj = j >= 0 ? j % S : 0, uj = j >= 0 ? j / S : 0;
           // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
           bool ready = true;
           if (issue && within < kDecoderGroups)  // this group's first stage of the tile
-            ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
+            ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t >> cs_log) & 1), abort_flag, p.status,
                               kSitePipeCodes);
           if (ready && store && uj > 0)
             ready = pipe_wait(&empty[sj], static_cast<uint32_t>((uj - 1) & 1), abort_flag, p.status, kSitePipeEmpty);
@@ -730,15 +788,22 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
             }
           }
           if (store) {
-            const uint32_t a_off = L.a + static_cast<uint32_t>(sj) * kABytes;
+            uint4 out[4];
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
               uint4 pieces[M];
 #pragma unroll
               for (int m = 0; m < M; ++m) pieces[m] = st[(u + 1) % (kLook + 1)][m][cc];
-              *reinterpret_cast<uint4*>(smem + a_off + swz128(r, 4 * hf + cc)) = sum_pieces<M>(pieces);
+              out[cc] = sum_pieces<M>(pieces);
             }
-            fence_proxy_async_smem();
+            if (a_in_tmem) tc_fence_after_sync();  // the stage's release (MMA commit) -> these tcgen05.st
+            store_a_half(a_in_tmem, smem, L.a + static_cast<uint32_t>(sj) * (a_in_tmem ? 0u : kABytes),
+                                 a_tmem_q + 32u * static_cast<uint32_t>(sj), r, hf, out);
+            if (a_in_tmem) {
+              tc_fence_before_sync();  // tcgen05.st -> the MMA issuer's reads, through the barrier
+            } else {
+              fence_proxy_async_smem();
+            }
             mbar_arrive(&full[sj]);
           }
         }
@@ -748,11 +813,11 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
       // one group: every stage in order (written without the group arithmetic:
       // the compiler schedules this form measurably better for 4x8 g8)
       for (int i = 0; i < nks; ++i) {
-        const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
+        const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t & cs_mask;
         // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
         bool ready = true;
         if (within == 0)
-          ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
+          ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t >> cs_log) & 1), abort_flag, p.status,
                             kSitePipeCodes);
         const int s = i % S, u = i / S;
         if (ready && u > 0)
@@ -764,10 +829,15 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
                             code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                 r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
-        decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
-                                   p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
-        if constexpr (B == 16) {
+        if (a_in_tmem) tc_fence_after_sync();  // the stage's release (MMA commit) -> these tcgen05.st
+        decode_half_stage<M, B, G>(a_in_tmem, smem, sbase, L.a + static_cast<uint32_t>(s) * (a_in_tmem ? 0u : kABytes),
+                                           a_tmem_q + 32u * static_cast<uint32_t>(s), r, hf, row_valid, cw,
+                                           p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
+        if constexpr (B == 16 && M == 1 && G == 8) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
+        } else if (a_in_tmem) {
+          tc_fence_before_sync();  // tcgen05.st -> the MMA issuer's reads, through the barrier
+          mbar_arrive(&full[s]);
         } else {
           fence_proxy_async_smem();
           mbar_arrive(&full[s]);
@@ -779,11 +849,11 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
       }
     } else {
       for (int i = grp; i < nks; i += kDecoderGroups) {
-        const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t % kCodeSlots;
+        const int t = i / kStagesPerTile, within = i % kStagesPerTile, c = t & cs_mask;
         // wait decisions are made warp-uniform: a warp either goes on or leaves as a whole
         bool ready = true;
         if (within < kDecoderGroups)  // this group's first stage of the tile
-          ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t / kCodeSlots) & 1), abort_flag, p.status,
+          ready = pipe_wait(&cfull[c], static_cast<uint32_t>((t >> cs_log) & 1), abort_flag, p.status,
                             kSitePipeCodes);
         const int s = i % S, u = i / S;
         if (ready && u > 0)
@@ -795,10 +865,15 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
                             code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                 r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
-        decode_half_stage<M, B, G>(smem, sbase, L.a + static_cast<uint32_t>(s) * kABytes, r, hf, row_valid, cw,
-                                   p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
-        if constexpr (B == 16) {
+        if (a_in_tmem) tc_fence_after_sync();  // the stage's release (MMA commit) -> these tcgen05.st
+        decode_half_stage<M, B, G>(a_in_tmem, smem, sbase, L.a + static_cast<uint32_t>(s) * (a_in_tmem ? 0u : kABytes),
+                                           a_tmem_q + 32u * static_cast<uint32_t>(s), r, hf, row_valid, cw,
+                                           p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
+        if constexpr (B == 16 && M == 1 && G == 8) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
+        } else if (a_in_tmem) {
+          tc_fence_before_sync();  // tcgen05.st -> the MMA issuer's reads, through the barrier
+          mbar_arrive(&full[s]);
         } else {
           fence_proxy_async_smem();
           mbar_arrive(&full[s]);
@@ -919,7 +994,8 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
 // per CTA through distributed shared memory; measured on B200 it costs about two
 // stage times per 16 batch columns, which makes SK = 1 the choice for wide batches.
 struct TcPlan {
-  int S = 0, SK = 1, ks_per = 0, red_rows = 128, cb_sh = 3;
+  int S = 0, SK = 1, ks_per = 0, red_rows = 128, cb_sh = 3, cs_log = 2;
+  bool a_tmem = false;
 };
 
 constexpr int kPlanFixedStages = 3;     // set-up, pipeline fill and epilogue, in stage times
@@ -930,9 +1006,27 @@ template <int M, int B, int G, bool kGrad>
 using PipeSchemeOf = std::conditional_t<kGrad, GradScheme<M, B, G>, PipeScheme<M, B, G>>;
 
 template <int M, int B, int G, bool kGrad>
-inline uint32_t pipe_smem_bytes(int S, int BN, int cb_sh) {
+inline uint32_t pipe_smem_bytes(int S, int BN, int cb_sh, int cs_log, bool a_tmem) {
   using SC = PipeSchemeOf<M, B, G, kGrad>;
-  return pipe_layout(S, BN, SC::kCodeTileBytes, SC::kCbBytes * (8u >> cb_sh)).total + 1024;
+  const uint32_t bytes =
+      pipe_layout(S, BN, SC::kCodeTileBytes, SC::kCbBytes * (8u >> cb_sh), 1 << cs_log, a_tmem ? 0u : kABytes).total +
+      1024;
+  // With A in tensor memory a CTA allocates all 512 columns.  Two such CTAs on one SM
+  // (from consecutive launches, or if the layout were small enough) would make the
+  // second one's tcgen05.alloc wait for the first, and with split-K clusters two
+  // clusters could then wait on each other.  Asking for more than half an SM's shared
+  // memory keeps every such CTA alone on its SM.
+  return a_tmem ? std::max(bytes, kSmemLimit / 2 + 1024u) : bytes;
+}
+
+// The instantiation a launch runs: A stages in tensor memory or in shared memory.
+using PipeKernelFn = void (*)(CUtensorMap, CUtensorMap, PipeParams);
+template <int M, int B, int G, bool kGrad>
+PipeKernelFn pipe_kernel(bool a_tmem) {
+  if constexpr (PipeSchemeOf<M, B, G, kGrad>::kATmemOk) {
+    if (a_tmem) return tc_pipe_kernel<M, B, G, kGrad, true>;
+  }
+  return tc_pipe_kernel<M, B, G, kGrad, false>;
 }
 
 // rows: output rows (the MMA's M extent); nk: 64-wide reduction stages.
@@ -950,7 +1044,11 @@ cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, TcPlan* out)
       return cudaSuccess;
     }
   }
-  auto kern = tc_pipe_kernel<M, B, G, kGrad>;
+  // A stages in tensor memory up to batch tile 128.  At 256 the decoders' tcgen05.st
+  // competed with the 256-column accumulator (2x8 11008 x 4096 at batch 256: 36.9 ->
+  // 58.7 us); below it they save the shared-memory A stores and the MMA's A reads.
+  const bool a_tmem = PipeSchemeOf<M, B, G, kGrad>::kATmemOk && BN <= 128;
+  auto kern = pipe_kernel<M, B, G, kGrad>(a_tmem);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
   if (e != cudaSuccess) return e;
   const int cmax = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess
@@ -960,24 +1058,35 @@ cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, TcPlan* out)
   const int row_tiles = (rows + kRows - 1) / kRows;
   const int batch_tiles = (batch + BN - 1) / BN;
   const long long clusters = static_cast<long long>(row_tiles) * batch_tiles;
-  // codebook copies (2x8 g8): the most that still leave room for three stages.
-  // Measured on 11008 x 4096: 8 copies made batch 4-64 11 % faster, but at batch 256
-  // they left room for two stages only and the kernel ran 1.8x slower.
-  int cb_sh = 3;
+  // codebook copies (2x8 g8) and code-tile slots: the most copies that still leave
+  // room for three stages, with four code slots if they fit, else two (a code tile
+  // holds four 2x8 stages, so two slots still keep the decoders fed).  Measured on
+  // 11008 x 4096: 8 copies made batch 4-64 11 % faster, but at batch 256 with four
+  // code slots they left room for two stages only and the kernel ran 1.8x slower.
+  int cb_sh = 3, cs_log = 2;
   if constexpr (PipeSchemeOf<M, B, G, kGrad>::kCbMaxReplicas > 1) {
-    for (int sh = 0; sh < 3; ++sh)
-      if (pipe_smem_bytes<M, B, G, kGrad>(3, BN, sh) <= kSmemLimit) {
-        cb_sh = sh;
-        break;
-      }
+    bool found = false;
+    for (int sh = 0; sh < 3 && !found; ++sh)
+      for (int cs = 2; cs >= 1 && !found; --cs)
+        if (pipe_smem_bytes<M, B, G, kGrad>(3, BN, sh, cs, a_tmem) <= kSmemLimit) {
+          cb_sh = sh;
+          cs_log = cs;
+          found = true;
+        }
   }
   TcPlan best;
   best.cb_sh = cb_sh;
+  best.cs_log = cs_log;
+  best.a_tmem = a_tmem;
   long long best_cost = -1;
   for (int S = 6; S >= 2; --S) {
-    const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(S, BN, cb_sh);
+    static_assert(6 <= kMaxATmemStages, "A stages in tensor memory");
+    const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(S, BN, cb_sh, cs_log, a_tmem);
     if (smem > kSmemLimit) continue;
-    const uint32_t stage_bytes = static_cast<uint32_t>(S) * (kABytes + static_cast<uint32_t>(BN) * 128u);
+    // shared stage memory (the split-K exchange reuses it): B tiles, plus A when A is in
+    // shared memory
+    const uint32_t kAStage = a_tmem ? 0u : kABytes;
+    const uint32_t stage_bytes = static_cast<uint32_t>(S) * (kAStage + static_cast<uint32_t>(BN) * 128u);
     for (int SK = 1; SK <= cmax; ++SK) {
       int per = (nk + SK - 1) / SK;
       per = (per + kSplitAlign - 1) / kSplitAlign * kSplitAlign;
@@ -1055,15 +1164,18 @@ cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, si
   }
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(p.BN)) cols <<= 1;
+  // A stages in tensor memory: the accumulator's 256 columns, then 32 a stage
+  if (plan.a_tmem) cols = 512;
   p.tmem_cols = cols;
   p.S = plan.S;
   p.SK = plan.SK;
   p.ks_per = plan.ks_per;
   p.red_rows = plan.red_rows;
   p.cb_sh = plan.cb_sh;
+  p.cs_log = plan.cs_log;
   p.cb32 = (reinterpret_cast<uintptr_t>(p.codebooks) & 31u) == 0 ? 1 : 0;
-  const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(plan.S, p.BN, plan.cb_sh);
-  auto kern = tc_pipe_kernel<M, B, G, kGrad>;
+  const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(plan.S, p.BN, plan.cb_sh, plan.cs_log, plan.a_tmem);
+  auto kern = pipe_kernel<M, B, G, kGrad>(plan.a_tmem);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
   if (e != cudaSuccess) return e;
   if (plan.SK > 8) {
