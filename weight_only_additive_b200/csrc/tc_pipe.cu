@@ -103,7 +103,12 @@ struct PipeScheme {
   // for every scheme decoded through registers; 1x16 g8 copies codewords into shared
   // memory by cp.async, so its A stages stay there.  The host picks the kATmem
   // instantiation per launch (pipe_kernel).
-  static constexpr bool kATmemOk = !(B == 16 && M == 1 && G == 8);
+  // 1x16 g8 decodes by cp.async copies of codewords into the A stage; measured faster
+  // than the register-staged gathers for this scheme, with A in shared memory or in
+  // tensor memory (4096 x 4096 batch 1: 14.5 against 15.5 us; 11008 x 4096 batch 256:
+  // 51.5 against 74.1 us)
+  static constexpr bool kCpAsyncDecode = B == 16 && M == 1 && G == 8;
+  static constexpr bool kATmemOk = !kCpAsyncDecode;
   // 2x8 g8: up to eight copies of each codebook in shared memory (cb_layout_offset), so
   // that the eight lanes of a quarter-warp phase read random codewords with few or no
   // bank conflicts; the host picks the count that still leaves room for three stages
@@ -745,7 +750,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     const int hf = kDecoderGroups == 1 ? tid >> 7 : (tid >> 7) & 1;
     const int grp = kDecoderGroups == 1 ? 0 : tid / kGroupThreads;
     const bool row_valid = n0 + r < p.N;
-    if constexpr (B == 16 && !(M == 1 && G == 8)) {
+    if constexpr (B == 16 && !PipeScheme<M, B, G>::kCpAsyncDecode) {
       // B = 16 except 1x16 g8: register-staged gathers, kLook stages ahead.  At step i
       // the thread issues the gathers of stage i (g = 16: one 256-bit load per 32-byte
       // codeword, one L1TEX request instead of two cp.async) and stores stage i - kLook,
@@ -833,7 +838,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         decode_half_stage<M, B, G>(a_in_tmem, smem, sbase, L.a + static_cast<uint32_t>(s) * (a_in_tmem ? 0u : kABytes),
                                            a_tmem_q + 32u * static_cast<uint32_t>(s), r, hf, row_valid, cw,
                                            p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
-        if constexpr (B == 16 && M == 1 && G == 8) {
+        if constexpr (B == 16) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
         } else if (a_in_tmem) {
           tc_fence_before_sync();  // tcgen05.st -> the MMA issuer's reads, through the barrier
@@ -869,7 +874,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         decode_half_stage<M, B, G>(a_in_tmem, smem, sbase, L.a + static_cast<uint32_t>(s) * (a_in_tmem ? 0u : kABytes),
                                            a_tmem_q + 32u * static_cast<uint32_t>(s), r, hf, row_valid, cw,
                                            p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
-        if constexpr (B == 16 && M == 1 && G == 8) {
+        if constexpr (B == 16) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
         } else if (a_in_tmem) {
           tc_fence_before_sync();  // tcgen05.st -> the MMA issuer's reads, through the barrier
