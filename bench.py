@@ -531,8 +531,15 @@ class Pool:
         self.groups = [L.LayerGroup([(self.weights[c][li], self.xs[c][li], self.ys[li])
                                      for li in range(len(w.layers))]) for c in range(pool)]
         h = b.stream.cuda_stream
+        # one zero-filled workspace for the per-layer calls (they run in turn on one stream)
+        ws_bytes = max(b.native.aqlm_matmul_workspace_size(l.scheme.M, l.scheme.B, l.scheme.g, l.K, l.N, batch)
+                       for l in w.layers)
+        self.ws = torch.zeros((max(ws_bytes, 1),), dtype=torch.uint8, device=b.dev)
+        ws = (self.ws.data_ptr(), ws_bytes) if ws_bytes else (None, 0)
         self.calls = [[(self.xs[c][li].data_ptr(), wt.codes.data_ptr(), wt.codebooks.data_ptr(), wt.scales.data_ptr(),
-                        None, self.ys[li].data_ptr(), wt.M, wt.B, wt.g, lay.K, lay.N, batch, h)
+                        None, self.ys[li].data_ptr(), wt.M, wt.B, wt.g, lay.K, lay.N, batch, int(b.native.Path.AUTO),
+                        int(b.native.Schedule.AUTO), ws[0] if b.native.aqlm_matmul_workspace_size(wt.M, wt.B, wt.g, lay.K, lay.N, batch) else None,
+                        ws[1] if b.native.aqlm_matmul_workspace_size(wt.M, wt.B, wt.g, lay.K, lay.N, batch) else 0, h)
                        for li, (lay, wt) in enumerate(zip(w.layers, self.weights[c]))] for c in range(pool)]
         self.b = b
 
@@ -541,9 +548,9 @@ class Pool:
 
     def step_per_layer(self, c):
         for args in self.calls[c]:
-            st = self.b.lib.aqlm_matmul(*args)
+            st = self.b.lib.aqlm_matmul_ws(*args)
             if st != 0:
-                raise self.b.native.AqlmError(st, "aqlm_matmul")
+                raise self.b.native.AqlmError(st, "aqlm_matmul_ws")
 
     def grouped_layers(self):
         return sum(1 for l in self.w.layers if l.scheme.B == 8 and self.batch == 1 and l.K % l.scheme.g == 0
@@ -916,15 +923,21 @@ def run_input_grad(a):
     dxs = [torch.empty((batch, lay.K), dtype=torch.float16, device=dev) for lay in w.layers]
     stream = torch.cuda.Stream(dev)
     h = stream.cuda_stream
+    # one zero-filled workspace for the stream-K schedule, shared by the calls in turn
+    ws_need = [native.aqlm_input_grad_workspace_size(l.scheme.M, l.scheme.B, l.scheme.g, l.K, l.N, batch)
+               for l in w.layers]
+    ws = torch.zeros((max(max(ws_need), 1),), dtype=torch.uint8, device=dev)
     calls = [[(dys[c][li].data_ptr(), weights[c][li].codes.data_ptr(), weights[c][li].codebooks.data_ptr(),
                weights[c][li].scales.data_ptr(), dxs[li].data_ptr(), lay.scheme.M, lay.scheme.B, lay.scheme.g,
-               lay.K, lay.N, batch, h) for li, lay in enumerate(w.layers)] for c in range(pool)]
+               lay.K, lay.N, batch, int(native.Schedule.AUTO), ws.data_ptr() if ws_need[li] else None,
+               ws.numel() if ws_need[li] else 0, h)
+              for li, lay in enumerate(w.layers)] for c in range(pool)]
 
     def step(c):
         for args in calls[c]:
-            st = lib.aqlm_input_grad(*args)
+            st = lib.aqlm_input_grad_ws(*args)
             if st != 0:
-                raise native.AqlmError(st, "aqlm_input_grad")
+                raise native.AqlmError(st, "aqlm_input_grad_ws")
 
     def barrier():
         if dist is not None:

@@ -73,6 +73,15 @@ typedef enum {
   AQLM_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up              */
 } aqlm_status;
 
+/* Work schedule of the tensor-core kernel (aqlm_matmul_ws, aqlm_input_grad_ws). */
+typedef enum {
+  AQLM_SCHEDULE_AUTO = 0,     /* the plan's cost model picks                              */
+  AQLM_SCHEDULE_TILES = 1,    /* one CTA per (row tile, batch tile, K split): no workspace */
+  AQLM_SCHEDULE_STREAMK = 2   /* stream-K over the SMs; needs the workspace, and a shape   *
+                               * with a nonzero workspace size (else                       *
+                               * AQLM_ERR_UNSUPPORTED)                                     */
+} aqlm_schedule;
+
 /* Kernel families aqlm_matmul can route to. */
 typedef enum {
   AQLM_PATH_AUTO = 0,         /* pick by (M, B, g, batch)                               */
@@ -115,6 +124,51 @@ aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codeb
                              const void* scales, const void* bias, void* y,
                              int M, int B, int g, int K, int N, int batch,
                              aqlm_path path, aqlm_stream_t stream);
+
+/*
+ * Bytes of workspace with which aqlm_matmul_ws may run the tensor-core kernel on a
+ * stream-K schedule: every SM takes an equal share of the (weight-row tile, batch
+ * tile, 64-wide K stage) space, and a tile cut between SMs is finished by the piece
+ * that ends last, from fp32 partials in the workspace, summed in K order (so results
+ * do not depend on timing).  The same y = x . W^T . diag(s) + bias as aqlm_matmul.
+ * 0 when the shape never uses it (the schedule needs the decoded weight stages in
+ * shared memory, i.e. a batch tile above 128 for schemes other than 1x16 g8, and K
+ * a whole number of code tiles), or for invalid arguments.  Pure host logic, the
+ * same for every device: needs no GPU.
+ */
+size_t aqlm_matmul_workspace_size(int M, int B, int g, int K, int N, int batch);
+
+/* A workspace that can carry the stream-K schedule starts with this many bytes of
+ * counters (one uint32 per CTA and TMEM lane quadrant, at most 160 CTAs), the same
+ * for every shape; fp32 partial slots follow. */
+#define AQLM_WORKSPACE_COUNTER_BYTES 2560u
+
+/*
+ * aqlm_matmul_path with a caller workspace and a schedule for the tensor-core kernel
+ * (other paths ignore both).  For this call AUTO is the tile plan: on B200 the stream-K
+ * schedule measured slower for every layer shape tried (it pays a fix-up, a four-warp
+ * final epilogue and a slower stage loop), so it runs only when asked for
+ * (AQLM_SCHEDULE_STREAMK).  aqlm_input_grad_ws's AUTO takes it where its cost model
+ * estimates it faster (a tile plan that would leave a nearly empty last wave of CTAs).
+ * workspace: NULL with workspace_bytes 0
+ * (then exactly aqlm_matmul_path), or caller-owned DEVICE memory, 256-byte aligned,
+ * of at least aqlm_matmul_workspace_size(...) bytes (else AQLM_ERR_MISALIGNED /
+ * AQLM_ERR_INVALID_ARG), overlapping none of the call's arrays (AQLM_ERR_INVALID_ARG).
+ * Its first AQLM_WORKSPACE_COUNTER_BYTES are counters that must be zero when the
+ * workspace is first used; every call whose kernels finish leaves them zero again,
+ * so a workspace allocated zero-filled can be reused call after call, by any shape
+ * (the counters sit at the same place for all).  After AQLM_ERR_TIMEOUT from
+ * aqlm_check_device_status, zero them again.  Calls that may run concurrently
+ * (different streams) must not share a workspace; calls on one stream may.
+ * The library may also ignore the workspace (another path, or a faster plan).
+ * AQLM_SCHEDULE_STREAMK without a workspace is AQLM_ERR_INVALID_ARG; an unknown
+ * schedule is AQLM_ERR_INVALID_ARG.
+ */
+aqlm_status aqlm_matmul_ws(const void* x, const void* codes, const void* codebooks,
+                           const void* scales, const void* bias, void* y,
+                           int M, int B, int g, int K, int N, int batch, aqlm_path path,
+                           aqlm_schedule schedule, void* workspace, size_t workspace_bytes,
+                           aqlm_stream_t stream);
 
 /*
  * The dense fp16 weight of the layer, the first half of the large-batch route
@@ -160,6 +214,19 @@ aqlm_status aqlm_input_grad(const void* dy, const void* codes, const void* codeb
                             const void* scales, void* dx, int M, int B, int g, int K, int N,
                             int batch, aqlm_stream_t stream);
 
+/* Workspace bytes with which aqlm_input_grad_ws may use the stream-K schedule
+ * (as for aqlm_matmul_workspace_size; the gradient kernel's rows are the K input
+ * features).  0 when unused (B = 16 schemes) or for invalid arguments; needs no GPU. */
+size_t aqlm_input_grad_workspace_size(int M, int B, int g, int K, int N, int batch);
+
+/* aqlm_input_grad with a schedule and a caller workspace: the same result;
+ * schedule and workspace as for aqlm_matmul_ws (it must not overlap dy, dx or the
+ * weights). */
+aqlm_status aqlm_input_grad_ws(const void* dy, const void* codes, const void* codebooks,
+                               const void* scales, void* dx, int M, int B, int g, int K, int N,
+                               int batch, aqlm_schedule schedule, void* workspace,
+                               size_t workspace_bytes, aqlm_stream_t stream);
+
 /* Validates aqlm_input_grad's arguments exactly as it does, without launching
  * anything.  Pure host logic: needs no GPU. */
 aqlm_status aqlm_validate_input_grad(const void* dy, const void* codes, const void* codebooks,
@@ -195,11 +262,16 @@ typedef struct {
  * reduction); the others are launched one after another as by aqlm_matmul.  Both kernels of a
  * pair keep the stream-ordering contract above.
  *
- * workspace: caller-owned DEVICE memory of at least
- * aqlm_group_workspace_size(problems, count) bytes, 256-byte aligned (NULL
- * allowed when that size is 0).  It holds fp32 partial sums between the two
- * kernels of a pair and needs no initialisation; calls that may run
- * concurrently (different streams) must not share a workspace.
+ * workspace: caller-owned DEVICE memory of aqlm_group_workspace_size(problems,
+ * count) bytes, 256-byte aligned (NULL allowed when that size is 0), zero-filled
+ * before its first use.  Layout: the AQLM_WORKSPACE_COUNTER_BYTES of stream-K
+ * counters (as for aqlm_matmul_ws), then the fp32 partial sums between the two
+ * kernels of a pair (required when any problem is grouped, else
+ * AQLM_ERR_INVALID_ARG), then, after those rounded up to 256 bytes, the stream-K
+ * partial slots that the problems launched one by one share (used only when the
+ * whole size is given).  Every call whose kernels finish leaves it reusable, as for
+ * aqlm_matmul_ws; calls that may run concurrently (different streams) must not
+ * share a workspace.
  * count == 0 is a no-op; count < 0 or problems == NULL (with count > 0) is
  * AQLM_ERR_INVALID_ARG.  Every problem is validated as aqlm_validate does before
  * anything is launched.
@@ -214,11 +286,14 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
  * AQLM_STATIC_GROUP_SCRATCH_BYTES inside the library (one per device; the address
  * is taken with cudaGetSymbolAddress on a device's first call and again whenever
  * the device's CUDA context has changed, e.g. after cudaDeviceReset); the call
- * allocates nothing.  Problems whose aqlm_group_workspace_size exceeds that size
- * are rejected with AQLM_ERR_INVALID_ARG before anything is launched (16 MiB
- * covers, for example, a Llama-2-7B decoder layer set, 1.6 MB, or the 24
- * Mixtral-8x7B expert linears of one layer, 11 MB).  The buffer needs no
- * clearing: the reduction reads only partials written by the same call.
+ * allocates nothing.  Problems whose grouped part (the counters plus the grouped
+ * partial sums of aqlm_group_workspace_size) exceeds that size are rejected with
+ * AQLM_ERR_INVALID_ARG before anything is launched (16 MiB covers, for example, a
+ * Llama-2-7B decoder layer set, 1.6 MB, or the 24 Mixtral-8x7B expert linears of
+ * one layer, 11 MB).  The buffer needs no clearing: the reduction reads only
+ * partials written by the same call.  Problems launched one by one use its
+ * stream-K layout when the whole aqlm_group_workspace_size fits (the buffer starts
+ * zero-filled and every call leaves the counters so).
  * Calls that overlap in time (different streams or host threads on one device)
  * share the buffer and RACE: the caller must serialise them.  Calls on one
  * stream are ordered and safe.  Otherwise identical to aqlm_matmul_group.
@@ -248,10 +323,13 @@ aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aq
 aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, const void* x_host, void* y_host,
                                    void* workspace, size_t workspace_bytes, aqlm_stream_t stream);
 
-/* Workspace bytes aqlm_matmul_group needs for these problems: for every run of
- * up to 32 grouped problems, the sum over them of ceil(K / g * M / 128) * N * 4
- * bytes (one fp32 partial per row and 128 code bytes) rounded up to 256; the
- * maximum over runs.  Pure host logic. */
+/* Workspace bytes aqlm_matmul_group takes for these problems: 0 if no problem is
+ * grouped and none launched one by one has a nonzero aqlm_matmul_workspace_size;
+ * else AQLM_WORKSPACE_COUNTER_BYTES, plus the grouped part (for every run of up to
+ * 32 grouped problems, the sum over them of ceil(K / g * M / 128) * N * 4 bytes, one
+ * fp32 partial per row and 128 code bytes, rounded up to 256; the maximum over
+ * runs), plus the largest stream-K partial-slot size (aqlm_matmul_workspace_size
+ * minus the counters) of the problems launched one by one.  Pure host logic. */
 size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count);
 
 /* The kernel family AQLM_PATH_AUTO picks for this problem, or -1 if unsupported.

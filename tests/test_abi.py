@@ -8,7 +8,7 @@ import re
 import pytest
 
 from weight_only_additive_b200 import build, native
-from weight_only_additive_b200.native import Path, Status
+from weight_only_additive_b200.native import Path, Schedule, Status
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "aqlm.h")
@@ -146,10 +146,18 @@ def _ws_bytes(K, N):
 
 
 def test_group_workspace_size(lib):
+    # layout: counters, grouped partial sums, the stream-K slots of the 1x16 layer
+    # launched on its own
     P = [_prob(1 << 32), _prob(1 << 33, K=11008, N=200), _prob(1 << 34, M=1, B=16)]
-    assert native.aqlm_group_workspace_size(P) == _ws_bytes(4096, 4096) + _ws_bytes(11008, 200)
+    grouped = _ws_bytes(4096, 4096) + _ws_bytes(11008, 200)
+    assert native.aqlm_group_workspace_size(P) == COUNTERS + grouped + _streamk_parts(32 * 16, 16)
+    assert native.aqlm_group_workspace_size(P[:2]) == COUNTERS + grouped
     assert native.aqlm_group_workspace_size([]) == 0
-    assert native.aqlm_group_workspace_size([_prob(1 << 32, M=1, B=16)]) == 0       # nothing grouped
+    assert native.aqlm_group_workspace_size([_prob(1 << 32, M=1, B=16)]) == _streamk_bytes(32, 32 * 16, 16)
+    assert native.aqlm_group_workspace_size([_prob(1 << 32, M=1, B=16, K=4104)]) == 0  # nothing grouped, no stream-K
+    # batch 256: the largest stream-K slots of the layers launched one by one
+    big = [_prob(1 << 32, batch=256, N=11008), _prob(1 << 33, batch=256, N=1000, K=2048)]
+    assert native.aqlm_group_workspace_size(big) == _streamk_bytes(86, 86 * 16, 256)
     assert native.aqlm_group_workspace_size([_prob(1 << 32, batch=2)]) == 0         # batch 2: not grouped
     assert native.aqlm_group_workspace_size([_prob(1 << 32, K=4104)]) == 0          # K % 64 != 0
     assert native.aqlm_group_workspace_size([_prob(1 << 32, K=4095)]) == 0          # invalid shape
@@ -158,7 +166,7 @@ def test_group_workspace_size(lib):
     many = [_prob((i + 1) << 32, K=64 * (i + 1), N=100) for i in range(R + 8)]
     run1 = sum(_ws_bytes(64 * (i + 1), 100) for i in range(R))
     run2 = sum(_ws_bytes(64 * (i + 1), 100) for i in range(R, R + 8))
-    assert native.aqlm_group_workspace_size(many) == max(run1, run2) == run1
+    assert native.aqlm_group_workspace_size(many) == COUNTERS + max(run1, run2) == COUNTERS + run1
 
 
 def test_group_validation_needs_no_gpu(lib):
@@ -193,13 +201,14 @@ def test_group_static_validation_needs_no_gpu(lib):
     assert L_.aqlm_matmul_group_static(native.problem_array([_prob(1 << 32)]), -3, None) == Status.INVALID_ARG
     # 10 grouped 28672 x 8192 layers need 10 x 16 x 28672 x 4 bytes > 16 MiB
     big = [_prob((i + 1) << 34, K=8192, N=28672) for i in range(10)]
-    assert native.aqlm_group_workspace_size(big) == 10 * _ws_bytes(8192, 28672) > native.STATIC_GROUP_SCRATCH_BYTES
+    assert native.aqlm_group_workspace_size(big) == COUNTERS + 10 * _ws_bytes(8192, 28672) > \
+        native.STATIC_GROUP_SCRATCH_BYTES
     assert L_.aqlm_matmul_group_static(native.problem_array(big), 10, None) == Status.INVALID_ARG
     # the 24 Mixtral-8x7B expert linears of a layer (w1, w3 14336 x 4096, w2 4096 x 14336) fit
     mixtral = [_prob((i + 1) << 34, K=14336, N=4096) if i % 3 == 2 else _prob((i + 1) << 34, K=4096, N=14336)
                for i in range(24)]
     assert native.aqlm_group_workspace_size(mixtral) == \
-        8 * (_ws_bytes(14336, 4096) + 2 * _ws_bytes(4096, 14336)) <= native.STATIC_GROUP_SCRATCH_BYTES
+        COUNTERS + 8 * (_ws_bytes(14336, 4096) + 2 * _ws_bytes(4096, 14336)) <= native.STATIC_GROUP_SCRATCH_BYTES
     bad = [_prob(1 << 32, M=5)]
     assert L_.aqlm_matmul_group_static(native.problem_array(bad), 1, None) == Status.UNSUPPORTED
 
@@ -270,4 +279,90 @@ def test_group_workspace_size_generic_schemes(lib, M, g, K):
     N = 300
     probs = native.problem_array([_prob(1 << 32, M=M, B=8, g=g, K=K, N=N)])
     slices = (K // g * M + 127) // 128
-    assert native.aqlm_group_workspace_size(probs, 1) == (slices * N * 4 + 255) // 256 * 256
+    assert native.aqlm_group_workspace_size(probs, 1) == COUNTERS + (slices * N * 4 + 255) // 256 * 256
+
+
+# ---------------------------------------------------------------------------
+# workspace of the tensor-core kernel's stream-K schedule (pure host logic)
+# ---------------------------------------------------------------------------
+COUNTERS = 2560  # AQLM_WORKSPACE_COUNTER_BYTES: a uint32 per (CTA, lane quadrant), 160 CTAs
+
+
+def _streamk_parts(units, BN):
+    """Stream-K partial slots: 2 of 128 x BN fp32 per CTA, at most 160 CTAs."""
+    return 2 * min(units, 160) * 128 * BN * 4
+
+
+def _streamk_bytes(tiles, units, BN):
+    """The size the header documents: the fixed counters, then the partial slots
+    (the tile count does not enter)."""
+    return COUNTERS + _streamk_parts(units, BN)
+
+
+def test_workspace_counter_bytes_agree_everywhere(lib):
+    text = open(HEADER).read()
+    m = re.search(r"#define AQLM_WORKSPACE_COUNTER_BYTES (\d+)u", text)
+    assert m and int(m.group(1)) == COUNTERS == native.WORKSPACE_COUNTER_BYTES == 160 * 4 * 4
+
+
+def test_matmul_workspace_size(lib):
+    # 2x8 g8 11008 x 4096 at batch 256: 86 row tiles, units of 4 stages (one code tile)
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 4096, 11008, 256) == _streamk_bytes(86, 86 * 16, 256)
+    # batch 300: two batch tiles of 256
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 4096, 1000, 300) == _streamk_bytes(16, 16 * 16, 256)
+    # 1x16 g8 keeps its A stages in shared memory at every batch: batch 1, tile 16
+    assert native.aqlm_matmul_workspace_size(1, 16, 8, 4096, 4096, 1) == _streamk_bytes(32, 32 * 16, 16)
+    # a few units only: as many CTAs as units
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 256, 128, 200) == _streamk_bytes(1, 1, 208)
+    # A in tensor memory (batch tile <= 128), K not a whole number of code tiles, or
+    # no pipelined kernel: no workspace
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 4096, 11008, 16) == 0
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 4096 + 64, 11008, 256) == 0
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 2064, 300, 256) == 0
+    # invalid arguments
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 4100, 11008, 256) == 0
+    assert native.aqlm_matmul_workspace_size(5, 8, 8, 4096, 11008, 256) == 0
+
+
+def test_input_grad_workspace_size(lib):
+    # Mixtral expert down-projection at batch 1024: 32 feature tiles x 4 batch tiles,
+    # 224 single-stage units each
+    assert native.aqlm_input_grad_workspace_size(2, 8, 8, 4096, 14336, 1024) == _streamk_bytes(128, 128 * 224, 256)
+    assert native.aqlm_input_grad_workspace_size(2, 8, 8, 1088, 1000, 16) == _streamk_bytes(9, 9 * 16, 16)
+    # B = 16 gradient kernels have no stream-K schedule
+    assert native.aqlm_input_grad_workspace_size(1, 16, 8, 4096, 4096, 1024) == 0
+    assert native.aqlm_input_grad_workspace_size(2, 8, 8, 4100, 4096, 1024) == 0
+
+
+def test_workspace_validation_needs_no_gpu(lib):
+    ws_need = native.aqlm_matmul_workspace_size(2, 8, 8, 4096, 11008, 256)
+    x, y, W = 1 << 32, 1 << 34, 1 << 40  # disjoint fake buffers, never dereferenced
+    args = (x, x + (1 << 30), x + (1 << 31), x + (1 << 31) + (1 << 20), None, y, 2, 8, 8, 4096, 11008, 256,
+            Path.TENSOR_CORE, Schedule.AUTO)
+    L_ = native.lib()
+    # misaligned, too small, bytes without a pointer, overlapping y
+    assert L_.aqlm_matmul_ws(*args, W + 128, ws_need, None) == Status.MISALIGNED
+    assert L_.aqlm_matmul_ws(*args, W, ws_need - 256, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_ws(*args, None, 256, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_ws(*args, y - 256, ws_need, None) == Status.INVALID_ARG
+    # argument errors come first, as for aqlm_matmul_path
+    bad = (None,) + args[1:]
+    assert L_.aqlm_matmul_ws(*bad, W, ws_need, None) == Status.INVALID_ARG
+    # schedules: unknown; stream-K without a workspace, on a shape without one, on
+    # another kernel family
+    assert L_.aqlm_matmul_ws(*args[:-1], 7, W, ws_need, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_ws(*args[:-1], Schedule.STREAMK, None, 0, None) == Status.INVALID_ARG
+    small = args[:6] + (2, 8, 8, 4096, 11008, 16, Path.TENSOR_CORE, Schedule.STREAMK)
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 4096, 11008, 16) == 0
+    assert L_.aqlm_matmul_ws(*small, W, 1 << 20, None) == Status.UNSUPPORTED
+    gemv = args[:6] + (1, 16, 8, 4096, 4096, 1, Path.GEMV, Schedule.STREAMK)
+    assert L_.aqlm_matmul_ws(*gemv, W, 1 << 24, None) == Status.UNSUPPORTED
+    gneed = native.aqlm_input_grad_workspace_size(2, 8, 8, 4096, 14336, 1024)
+    gargs = (x, x + (1 << 31), x + (1 << 31) + (1 << 28), x + (1 << 31) + (1 << 29), y, 2, 8, 8, 4096, 14336, 1024,
+             Schedule.AUTO)
+    assert L_.aqlm_input_grad_ws(*gargs, W + 16, gneed, None) == Status.MISALIGNED
+    assert L_.aqlm_input_grad_ws(*gargs, W, gneed - 1, None) == Status.INVALID_ARG
+    assert L_.aqlm_input_grad_ws(*gargs, x, gneed, None) == Status.INVALID_ARG  # overlaps dy
+    assert L_.aqlm_input_grad_ws(*gargs[:-1], Schedule.STREAMK, None, 0, None) == Status.INVALID_ARG
+    g16 = gargs[:5] + (1, 16, 8, 4096, 4096, 1024, Schedule.STREAMK)  # B = 16 gradient: no stream-K
+    assert L_.aqlm_input_grad_ws(*g16, W, 1 << 24, None) == Status.UNSUPPORTED

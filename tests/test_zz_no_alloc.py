@@ -60,7 +60,7 @@ def test_static_scratch_matches_caller_workspace_on_two_calls_in_a_row(dev):
     # two calls in a row on the static buffer, no synchronisation in between
     native.aqlm_matmul_group_static(probs_static[0], stream, count=n)
     native.aqlm_matmul_group_static(probs_static[1], stream, count=n)
-    ws = torch.empty((need,), dtype=torch.uint8, device=dev)
+    ws = torch.zeros((need,), dtype=torch.uint8, device=dev)
     for c in range(2):
         native.aqlm_matmul_group(probs_ws[c], ws.data_ptr(), need, stream, count=n)
     torch.cuda.synchronize()
@@ -115,7 +115,7 @@ def test_static_scratch_holds_the_mixtral_expert_set(dev):
     assert 8 << 20 < need <= native.STATIC_GROUP_SCRATCH_BYTES
     stream = torch.cuda.current_stream(dev).cuda_stream
     native.aqlm_matmul_group_static(probs_static, stream, count=n)
-    ws = torch.empty((need,), dtype=torch.uint8, device=dev)
+    ws = torch.zeros((need,), dtype=torch.uint8, device=dev)
     native.aqlm_matmul_group(probs_ws, ws.data_ptr(), need, stream, count=n)
     torch.cuda.synchronize()
     st, detail = L.check_device_status()

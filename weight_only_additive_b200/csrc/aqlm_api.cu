@@ -2,6 +2,7 @@
 // device status word.  Declarations and the contract live in include/aqlm.h.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 #include <utility>
 
@@ -83,11 +84,38 @@ bool path_accepts(aqlm_path path, int M, int B, int g, int K, int batch) {
   }
 }
 
+aqlm_status launch_matmul(const aqlm::Problem& p, aqlm_path path, cudaStream_t s);
+
+// A schedule request against the shape's workspace need (`need` 0: no stream-K).
+aqlm_status check_schedule(aqlm_schedule schedule, const void* workspace, size_t need) {
+  if (schedule < AQLM_SCHEDULE_AUTO || schedule > AQLM_SCHEDULE_STREAMK) return AQLM_ERR_INVALID_ARG;
+  if (schedule != AQLM_SCHEDULE_STREAMK) return AQLM_OK;
+  if (need == 0) return AQLM_ERR_UNSUPPORTED;
+  return workspace ? AQLM_OK : AQLM_ERR_INVALID_ARG;
+}
+
 aqlm_status validate_shape(int M, int B, int g, int K, int N, int batch) {
   if (M < 1 || B < 1 || g < 1 || K < 1 || N < 1 || batch < 1) return AQLM_ERR_INVALID_ARG;
   if (K % g != 0) return AQLM_ERR_INVALID_ARG;
   if (batch > 65535) return AQLM_ERR_INVALID_ARG;
   if (!aqlm::scheme_supported(M, B, g)) return AQLM_ERR_UNSUPPORTED;
+  return AQLM_OK;
+}
+
+// Checks a caller workspace of aqlm_matmul_ws / aqlm_input_grad_ws: NULL with 0 bytes
+// means none; otherwise 256-byte aligned, at least `need` bytes, and no overlap with
+// the call's arrays (ptrs[i], sizes[i]; NULL entries skipped).
+aqlm_status check_workspace(const void* ws, size_t ws_bytes, size_t need, const void* const* ptrs,
+                            const size_t* sizes, int count) {
+  if (ws == nullptr) return ws_bytes == 0 ? AQLM_OK : AQLM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return AQLM_ERR_MISALIGNED;
+  if (ws_bytes < need || ws_bytes == 0) return AQLM_ERR_INVALID_ARG;
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(ws), hi = lo + ws_bytes;
+  for (int i = 0; i < count; ++i) {
+    if (!ptrs[i]) continue;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(ptrs[i]);
+    if (a < hi && lo < a + sizes[i]) return AQLM_ERR_INVALID_ARG;
+  }
   return AQLM_OK;
 }
 
@@ -137,7 +165,7 @@ EncodeTiledFn encode_tiled() {
 
 extern "C" {
 
-int aqlm_abi_version(void) { return 7; }
+int aqlm_abi_version(void) { return 8; }
 
 const char* aqlm_status_string(aqlm_status status) {
   switch (status) {
@@ -180,15 +208,50 @@ aqlm_status aqlm_validate(const void* x, const void* codes, const void* codebook
   return AQLM_OK;
 }
 
-aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codebooks,
-                             const void* scales, const void* bias, void* y,
-                             int M, int B, int g, int K, int N, int batch,
-                             aqlm_path path, aqlm_stream_t stream) {
-  const aqlm_status st = aqlm_validate(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path);
+size_t aqlm_matmul_workspace_size(int M, int B, int g, int K, int N, int batch) {
+  if (validate_shape(M, B, g, K, N, batch) != AQLM_OK) return 0;
+  const size_t part = aqlm::tc_pipe_partial_bytes(M, B, g, K, N, batch);
+  return part > 0 ? AQLM_WORKSPACE_COUNTER_BYTES + part : 0;
+}
+
+aqlm_status aqlm_matmul_ws(const void* x, const void* codes, const void* codebooks,
+                           const void* scales, const void* bias, void* y,
+                           int M, int B, int g, int K, int N, int batch, aqlm_path path,
+                           aqlm_schedule schedule, void* workspace, size_t workspace_bytes,
+                           aqlm_stream_t stream) {
+  aqlm_status st = aqlm_validate(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path);
   if (st != AQLM_OK) return st;
-  if (path == AQLM_PATH_AUTO) path = static_cast<aqlm_path>(aqlm_select_path(M, B, g, K, N, batch));
-  const aqlm::Problem p{x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch};
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = check_schedule(schedule, workspace, aqlm_matmul_workspace_size(M, B, g, K, N, batch));
+  if (st != AQLM_OK) return st;
+  if (schedule == AQLM_SCHEDULE_STREAMK) {
+    // a forced stream-K schedule is the tensor-core kernel's
+    if (path != AQLM_PATH_AUTO && path != AQLM_PATH_TENSOR_CORE) return AQLM_ERR_UNSUPPORTED;
+    path = AQLM_PATH_TENSOR_CORE;
+  }
+  const size_t code_bytes = static_cast<size_t>(N) * (K / g) * M * (B <= 8 ? 1 : 2);
+  const void* ptrs[6] = {x, codes, codebooks, scales, bias, y};
+  const size_t sizes[6] = {static_cast<size_t>(batch) * K * 2, code_bytes,
+                           static_cast<size_t>(M) * (size_t(1) << B) * g * 2, static_cast<size_t>(N) * 2,
+                           static_cast<size_t>(N) * 2, static_cast<size_t>(batch) * N * 2};
+  st = check_workspace(workspace, workspace_bytes, aqlm_matmul_workspace_size(M, B, g, K, N, batch), ptrs, sizes, 6);
+  if (st != AQLM_OK) return st;
+  aqlm::Problem p{x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch};
+  if (workspace) {  // [counters][partial slots]
+    p.sk_count = static_cast<uint32_t*>(workspace);
+    p.sk_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + AQLM_WORKSPACE_COUNTER_BYTES);
+    p.sk_part_bytes = workspace_bytes - AQLM_WORKSPACE_COUNTER_BYTES;
+  }
+  p.schedule = static_cast<int>(schedule);
+  return launch_matmul(p, path, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Launches one validated problem on `path` (AUTO resolved here).
+aqlm_status launch_matmul(const aqlm::Problem& p, aqlm_path path, cudaStream_t s) {
+  if (path == AQLM_PATH_AUTO) path = static_cast<aqlm_path>(aqlm_select_path(p.M, p.B, p.g, p.K, p.N, p.batch));
   switch (path) {
     case AQLM_PATH_GEMV: return from_cuda(aqlm::launch_gemv(p, s));
     case AQLM_PATH_GEMV_LUT: {
@@ -203,6 +266,18 @@ aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codeb
     }
     default: return AQLM_ERR_UNSUPPORTED;
   }
+}
+
+}  // namespace
+
+extern "C" {
+
+aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codebooks,
+                             const void* scales, const void* bias, void* y,
+                             int M, int B, int g, int K, int N, int batch,
+                             aqlm_path path, aqlm_stream_t stream) {
+  return aqlm_matmul_ws(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path, AQLM_SCHEDULE_AUTO, nullptr,
+                        0, stream);
 }
 
 aqlm_status aqlm_matmul(const void* x, const void* codes, const void* codebooks,
@@ -236,15 +311,45 @@ aqlm_status aqlm_validate_input_grad(const void* dy, const void* codes, const vo
   return AQLM_OK;
 }
 
-aqlm_status aqlm_input_grad(const void* dy, const void* codes, const void* codebooks,
-                            const void* scales, void* dx, int M, int B, int g, int K, int N,
-                            int batch, aqlm_stream_t stream) {
-  const aqlm_status st = aqlm_validate_input_grad(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch);
+size_t aqlm_input_grad_workspace_size(int M, int B, int g, int K, int N, int batch) {
+  if (validate_shape(M, B, g, K, N, batch) != AQLM_OK) return 0;
+  const size_t part = aqlm::input_grad_partial_bytes(M, B, g, K, N, batch);
+  return part > 0 ? AQLM_WORKSPACE_COUNTER_BYTES + part : 0;
+}
+
+aqlm_status aqlm_input_grad_ws(const void* dy, const void* codes, const void* codebooks,
+                               const void* scales, void* dx, int M, int B, int g, int K, int N,
+                               int batch, aqlm_schedule schedule, void* workspace, size_t workspace_bytes,
+                               aqlm_stream_t stream) {
+  aqlm_status st = aqlm_validate_input_grad(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch);
+  if (st != AQLM_OK) return st;
+  st = check_schedule(schedule, workspace, aqlm_input_grad_workspace_size(M, B, g, K, N, batch));
+  if (st != AQLM_OK) return st;
+  const size_t code_bytes = static_cast<size_t>(N) * (K / g) * M * (B <= 8 ? 1 : 2);
+  const void* ptrs[5] = {dy, codes, codebooks, scales, dx};
+  const size_t sizes[5] = {static_cast<size_t>(batch) * N * 2, code_bytes,
+                           static_cast<size_t>(M) * (size_t(1) << B) * g * 2, static_cast<size_t>(N) * 2,
+                           static_cast<size_t>(batch) * K * 2};
+  st = check_workspace(workspace, workspace_bytes, aqlm_input_grad_workspace_size(M, B, g, K, N, batch), ptrs,
+                       sizes, 5);
   if (st != AQLM_OK) return st;
   uint32_t* status = device_status_ptr();
   if (!status) return from_cuda(cudaErrorInvalidDevice);
-  const aqlm::GradProblem p{dy, codes, codebooks, scales, dx, M, B, g, K, N, batch};
+  aqlm::GradProblem p{dy, codes, codebooks, scales, dx, M, B, g, K, N, batch};
+  if (workspace) {  // [counters][partial slots]
+    p.sk_count = static_cast<uint32_t*>(workspace);
+    p.sk_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + AQLM_WORKSPACE_COUNTER_BYTES);
+    p.sk_part_bytes = workspace_bytes - AQLM_WORKSPACE_COUNTER_BYTES;
+  }
+  p.schedule = static_cast<int>(schedule);
   return from_cuda(aqlm::launch_input_grad(p, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+aqlm_status aqlm_input_grad(const void* dy, const void* codes, const void* codebooks,
+                            const void* scales, void* dx, int M, int B, int g, int K, int N,
+                            int batch, aqlm_stream_t stream) {
+  return aqlm_input_grad_ws(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch, AQLM_SCHEDULE_AUTO, nullptr, 0,
+                            stream);
 }
 
 namespace {
@@ -295,6 +400,39 @@ size_t group_workspace(const aqlm_problem* problems, int count) {
   return best;
 }
 
+// Stream-K partial slots of a group workspace: the largest need of the problems
+// launched one by one (they run in turn on the call's stream and share them).
+size_t group_streamk_partials(const aqlm_problem* problems, int count) {
+  size_t best = 0;
+  for (int i = 0; i < count; ++i) {
+    const aqlm_problem& q = problems[i];
+    if (aqlm::lut_group_supported(to_problem(q))) continue;
+    best = std::max(best, aqlm::tc_pipe_partial_bytes(q.M, q.B, q.g, q.K, q.N, q.batch));
+  }
+  return best;
+}
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// Layout of a group workspace: [stream-K counters][grouped partial sums][stream-K
+// partial slots].  The counters come first in every workspace, so calls with other
+// problem sets (the static scratch serves them all) never write partials over them.
+struct GroupLayout {
+  size_t grouped = 0;   // bytes of grouped partial sums
+  size_t sk_part = 0;   // bytes of stream-K partial slots
+  size_t required() const { return grouped > 0 ? AQLM_WORKSPACE_COUNTER_BYTES + grouped : 0; }
+  size_t full() const {
+    return (grouped > 0 || sk_part > 0) ? AQLM_WORKSPACE_COUNTER_BYTES + round256(grouped) + sk_part : 0;
+  }
+};
+
+GroupLayout group_layout(const aqlm_problem* problems, int count) {
+  GroupLayout g;
+  g.grouped = group_workspace(problems, count);
+  g.sk_part = group_streamk_partials(problems, count);
+  return g;
+}
+
 }  // namespace
 
 size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count) {
@@ -303,7 +441,7 @@ size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count) {
     const aqlm_problem& q = problems[i];
     if (validate_shape(q.M, q.B, q.g, q.K, q.N, q.batch) != AQLM_OK) return 0;
   }
-  return group_workspace(problems, count);
+  return group_layout(problems, count).full();
 }
 
 aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* workspace,
@@ -328,11 +466,17 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
         if (overlaps(ri[5], rj[k])) return AQLM_ERR_INVALID_ARG;
     }
   }
-  const size_t need = group_workspace(problems, count);
+  const GroupLayout lay = group_layout(problems, count);
+  const size_t need = lay.required();
   if (need > 0) {
     if (!workspace || workspace_bytes < need) return AQLM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return AQLM_ERR_MISALIGNED;
   }
+  uint8_t* const ws = static_cast<uint8_t*>(workspace);
+  // the problems launched one by one run the tensor-core kernel's stream-K schedule
+  // when the workspace has room for its partial slots too
+  const bool sk_ok = lay.sk_part > 0 && ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 &&
+                     workspace_bytes >= lay.full();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   aqlm::Problem run[aqlm::kMaxGroupLayers];
   int n_run = 0;
@@ -344,7 +488,8 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
   for (int i = 0; i <= count; ++i) {
     const bool flush = (i == count) || n_run == aqlm::kMaxGroupLayers;
     if (flush && n_run > 0) {
-      const aqlm_status st = from_cuda(aqlm::launch_lut_group(run, n_run, workspace, status, s));
+      const aqlm_status st =
+          from_cuda(aqlm::launch_lut_group(run, n_run, ws + AQLM_WORKSPACE_COUNTER_BYTES, status, s));
       if (st != AQLM_OK) return st;
       n_run = 0;
     }
@@ -353,9 +498,13 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
     if (aqlm::lut_group_supported(p)) {
       run[n_run++] = p;
     } else {
-      const aqlm_problem& q = problems[i];
-      const aqlm_status st = aqlm_matmul_path(q.x, q.codes, q.codebooks, q.scales, q.bias, q.y, q.M, q.B, q.g, q.K,
-                                              q.N, q.batch, AQLM_PATH_AUTO, stream);
+      aqlm::Problem one = p;
+      if (sk_ok) {
+        one.sk_count = reinterpret_cast<uint32_t*>(ws);
+        one.sk_part = reinterpret_cast<float*>(ws + AQLM_WORKSPACE_COUNTER_BYTES + round256(lay.grouped));
+        one.sk_part_bytes = lay.sk_part;
+      }
+      const aqlm_status st = launch_matmul(one, AQLM_PATH_AUTO, s);
       if (st != AQLM_OK) return st;
     }
   }
@@ -410,10 +559,20 @@ size_t aqlm_static_group_scratch_bytes(void) { return AQLM_STATIC_GROUP_SCRATCH_
 aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aqlm_stream_t stream) {
   if (count == 0) return AQLM_OK;
   if (count < 0 || !problems) return AQLM_ERR_INVALID_ARG;
-  const size_t need = aqlm_group_workspace_size(problems, count);
+  bool shapes_ok = true;
+  for (int i = 0; i < count; ++i) {
+    const aqlm_problem& q = problems[i];
+    shapes_ok = shapes_ok && validate_shape(q.M, q.B, q.g, q.K, q.N, q.batch) == AQLM_OK;
+  }
+  // the grouped partial sums must fit; the stream-K slots of the others are used when
+  // they fit too (the buffer starts zero-filled and every call leaves its counters zero)
+  GroupLayout lay;
+  if (shapes_ok) lay = group_layout(problems, count);
+  const size_t need = lay.required();
   if (need > AQLM_STATIC_GROUP_SCRATCH_BYTES) return AQLM_ERR_INVALID_ARG;
+  const bool use_sk = lay.sk_part > 0 && lay.full() <= AQLM_STATIC_GROUP_SCRATCH_BYTES;
   void* scratch = nullptr;
-  if (need > 0) {
+  if (need > 0 || use_sk) {
     // validate before touching the device, as every entry point does
     for (int i = 0; i < count; ++i) {
       const aqlm_problem& q = problems[i];
@@ -424,7 +583,7 @@ aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aq
     scratch = static_scratch_ptr();
     if (!scratch) return from_cuda(cudaErrorInvalidDevice);
   }
-  return aqlm_matmul_group(problems, count, scratch, AQLM_STATIC_GROUP_SCRATCH_BYTES, stream);
+  return aqlm_matmul_group(problems, count, scratch, scratch ? AQLM_STATIC_GROUP_SCRATCH_BYTES : 0, stream);
 }
 
 aqlm_status aqlm_selftest_bounded_wait(unsigned timeout_us, aqlm_stream_t stream) {

@@ -156,6 +156,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Order this thread's earlier generic-proxy view of global memory (data acquired from
+// other CTAs) before its later async-proxy reads of it (bulk copies).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before_sync() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -236,6 +242,14 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Acquire load at GPU scope: later loads see what the writers released before the
+// value was stored (their writes, a fence, then the counter update).
+__device__ __forceinline__ uint32_t ld_acquire_gpu_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Load 16 consecutive fp32 columns of this warp's 32 TMEM lanes (one lane per thread).
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
@@ -310,6 +324,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1, {%2, %3}], [%4], %5;"
       ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(pol) : "memory");
+}
+
+// Bulk copy (no tensor map, never with multicast) of `bytes` (a multiple of 16) from
+// this GPU's global memory at `src` (16-byte aligned) into this CTA's shared memory at
+// `dst` (16-byte aligned).  Completes `bytes` on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
 }
 
 // 16-byte cp.async (L2 only); `src_bytes` < 16 zero-fills the rest (0: all zeros).

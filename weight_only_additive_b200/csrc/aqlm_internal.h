@@ -39,6 +39,12 @@ struct Problem {
   const void* bias;  // may be null
   void* y;
   int M, B, g, K, N, batch;
+  // the tensor-core kernel's stream-K schedule: its counters (kStreamKCounterBytes,
+  // zero between calls) and partial slots, or null
+  uint32_t* sk_count = nullptr;
+  float* sk_part = nullptr;
+  size_t sk_part_bytes = 0;
+  int schedule = 0;  // aqlm_schedule: 0 auto, 1 tiles, 2 stream-K (forced)
 };
 
 // Each launcher enqueues its kernel(s) on `stream` and returns the launch error.
@@ -65,8 +71,15 @@ EncodeTiledFn encode_tiled();
 uint64_t current_context_id();
 
 // Pipelined decode -> tcgen05 kernel; cudaErrorNotSupported when the shape is
-// outside what it handles (the caller then uses the single-stage kernel).
+// outside what it handles (the caller then uses the single-stage kernel).  With a
+// workspace of tc_pipe_workspace_bytes (> 0) it may run the stream-K schedule.
 cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t stream);
+// Stream-K counters: one uint32 per (CTA, TMEM lane quadrant), at most 160 CTAs;
+// the first bytes of every workspace that can carry the schedule.
+constexpr size_t kStreamKCounterBytes = 160 * 4 * sizeof(uint32_t);
+// fp32 partial-slot bytes the stream-K schedule of the pipelined kernel needs on any
+// device; 0 when the shape never uses it.
+size_t tc_pipe_partial_bytes(int M, int B, int g, int K, int N, int batch);
 // Shape test of the pipelined kernel: K % 64 == 0 and code rows a multiple of 16 bytes.
 inline bool tc_pipelined_shape(int M, int B, int g, int K) {
   const long long row_bytes = static_cast<long long>(K / g) * M * (B <= 8 ? 1 : 2);
@@ -82,8 +95,13 @@ struct GradProblem {
   const void* scales;
   void* dx;
   int M, B, g, K, N, batch;
+  uint32_t* sk_count = nullptr;  // as in Problem
+  float* sk_part = nullptr;
+  size_t sk_part_bytes = 0;
+  int schedule = 0;
 };
 cudaError_t launch_input_grad(const GradProblem& p, uint32_t* status, cudaStream_t stream);
+size_t input_grad_partial_bytes(int M, int B, int g, int K, int N, int batch);
 // Shape test of the gradient kernel: dy rows and code rows are TMA tensors, so
 // N % 8 == 0 (16-byte dy rows) and code rows a multiple of 16 bytes.
 inline bool grad_shape_supported(int M, int B, int g, int K, int N) {

@@ -51,11 +51,12 @@ constexpr int kMaxDecoderGroups = 2;
 // codeword-gather decoders of the B = 16 layer kernels already keep L1TEX busy with
 // one group (a second made them 2-7 % slower), and 4x8 g8 ran faster with one.
 // Block: the decoder warps, then the x producer, the MMA issuer and the code producer.
-template <int M, int B, int G, bool kGrad>
+// Stream-K kernels (kStreamK) add four epilogue warps, one per TMEM lane quadrant.
+template <int M, int B, int G, bool kGrad, bool kStreamK = false>
 struct PipeShape {
   static constexpr int kGroups = (!kGrad && (B == 16 || (M == 4 && G == 8))) ? 1 : kMaxDecoderGroups;
   static constexpr int kDecoders = kGroups * kGroupThreads;
-  static constexpr int kThreads = kDecoders + 96;
+  static constexpr int kThreads = kDecoders + 96 + (kStreamK ? 128 : 0);
 };
 constexpr uint32_t kABytes = kRows * 128u;   // 16 KB per A stage (in shared memory)
 // A stages kept in tensor memory: the accumulator takes columns [0, 256) of a 512-column
@@ -83,6 +84,31 @@ struct PipeParams {
   int cb_sh;       // 2x8 g8 codebook copies in shared memory: 8 >> cb_sh of them (cb_layout_offset)
   int cs_log;      // code-tile ring of 1 << cs_log slots (2 or 4)
   uint32_t* status;
+  // Stream-K schedule (kStreamK kernels).  The work is the tiles x nk stages of
+  // (row tile, batch tile, K stage), tile t being row tile t / batch_tiles and batch
+  // tile t mod batch_tiles, cut into sk_units units of sk_unit stages; CTA c takes
+  // units [c U / C, (c + 1) U / C) with C = sk_ctas (SkRange).  A tile cut between
+  // CTAs is finished by whichever of its pieces ends last (see the epilogue).
+  int sk_ctas, sk_units, sk_unit, batch_tiles;
+  int acc_cols;         // TMEM columns of one accumulator (two, alternating by piece)
+  float* sk_part;       // 2 sk_ctas slots of 128 x BN fp32 partials ([4][BN / 4][32][4])
+  // per (CTA holding a cut tile's first piece, lane quadrant): pieces stored so far;
+  // zero between launches.  A CTA's range holds the first piece of at most one cut
+  // tile (only the last tile it reaches can continue past it), so the counters have
+  // a fixed size whatever the shape, and callers can share one workspace between shapes.
+  uint32_t* sk_count;
+};
+
+// Stream-K partition of a CTA range, in stages.
+struct SkRange {
+  int C, U, unit;
+  __host__ __device__ int begin(int c) const {
+    return static_cast<int>(static_cast<long long>(c) * U / C) * unit;
+  }
+  // the CTA whose range holds stage w: the largest c with begin(c) <= w
+  __host__ __device__ int cta_of(int w) const {
+    return static_cast<int>(((static_cast<long long>(w / unit) + 1) * C - 1) / U);
+  }
 };
 
 // Per-scheme constants.  A stage is 64 weights of a row: kStageCodeBytes of codes.
@@ -153,17 +179,19 @@ struct PipeLayout {
   uint32_t a, b, codes, cb, bars, total;
 };
 
-// a_stage_bytes: kABytes, or 0 when the A stages live in tensor memory.
+// a_stage_bytes: kABytes, or 0 when the A stages live in tensor memory.  acc_bars: 1,
+// or 8 for stream-K (accumulator full / empty for two accumulators, and one bulk-copy
+// barrier per epilogue warp).
 __host__ __device__ inline PipeLayout pipe_layout(int S, int BN, uint32_t code_tile_bytes, uint32_t cb_bytes,
-                                                  int code_slots, uint32_t a_stage_bytes) {
+                                                  int code_slots, uint32_t a_stage_bytes, int acc_bars = 1) {
   PipeLayout L;
   L.a = 0;                                                          // 1024-aligned stages
   L.b = L.a + static_cast<uint32_t>(S) * a_stage_bytes;
   L.codes = L.b + static_cast<uint32_t>(S) * static_cast<uint32_t>(BN) * 128u;
   L.cb = L.codes + static_cast<uint32_t>(code_slots) * code_tile_bytes;
   L.bars = L.cb + cb_bytes;
-  // full[S], empty[S], code_full[kCodeSlots], code_empty[kCodeSlots], acc, tmem slot, abort flag
-  L.total = L.bars + 8u * static_cast<uint32_t>(2 * S + 2 * kCodeSlots + 1) + 16u;
+  // full[S], empty[S], code_full[kCodeSlots], code_empty[kCodeSlots], acc bars, tmem slot, abort flag
+  L.total = L.bars + 8u * static_cast<uint32_t>(2 * S + 2 * kCodeSlots + acc_bars) + 16u;
   return L;
 }
 
@@ -227,6 +255,25 @@ __device__ __forceinline__ uint32_t code_tile_offset(int row, int off) {
     return static_cast<uint32_t>(row * 64 + ((((off >> 4) ^ (row >> 1)) & 3) << 4) + (off & 15));
   else
     return static_cast<uint32_t>(row * kTileRowBytes + off);
+}
+
+// pipe_wait for warps with nothing else to do (the stream-K epilogue): they sleep
+// between polls, so their waiting takes no issue slots or shared-memory bandwidth
+// from the decoders.
+__device__ __forceinline__ bool pipe_wait_sleepy(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                                 uint32_t* status, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    __nanosleep(256);
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      record_failure(status, site);
+      *abort_flag = 1u;
+      return false;
+    }
+  }
+  return true;
 }
 
 // Bounded wait that also gives up at once when another role has aborted.
@@ -488,19 +535,25 @@ __device__ __forceinline__ void cluster_barrier() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+
 // kGrad = false: y = x . W16^T . diag(s) + bias (rows = N, reduction over K).
 // kGrad = true:  dx = dy . W16 (rows = K input features, reduction over the N
 //                output rows; x_map then describes dy [batch, N]).
 // kATmem: the decoded A stages live in tensor memory (schemes with kATmemOk); a separate
 // instantiation, since the same loops with a runtime switch compiled measurably slower.
-template <int M, int B, int G, bool kGrad, bool kATmem>
-__global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
+// kStreamK: the CTA takes a range of the (tile, K stage) space that may cross tiles
+// (PipeParams), and four epilogue warps finish each tile piece while the decoders
+// go on with the next (see the epilogue below).
+template <int M, int B, int G, bool kGrad, bool kATmem, bool kStreamK>
+__global__ void __launch_bounds__(PipeShape<M, B, G, kGrad, kStreamK>::kThreads, 1)
     tc_pipe_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap code_map,
                    const PipeParams p) {
   constexpr int kDecoderGroups = PipeShape<M, B, G, kGrad>::kGroups;
   constexpr int kDecoders = PipeShape<M, B, G, kGrad>::kDecoders;
-  constexpr int kThreads = PipeShape<M, B, G, kGrad>::kThreads;
+  constexpr int kThreads = PipeShape<M, B, G, kGrad, kStreamK>::kThreads;
   constexpr int kWarpX = kDecoders / 32, kWarpMma = kWarpX + 1, kWarpCodes = kWarpX + 2;
+  constexpr int kWarpEpi = kWarpX + 3;  // stream-K: warps kWarpEpi .. + 3, lane quadrants 3, 0, 1, 2
+  static_assert(!(kATmem && kStreamK), "stream-K keeps A in shared memory");
   extern __shared__ uint8_t smem_raw[];
   // stages must be 1024-byte aligned for the 128-byte swizzle
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -511,8 +564,8 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
   const int S = p.S;
   static_assert(!kATmem || SC::kATmemOk, "A in tensor memory needs a register-decoded scheme");
   constexpr bool a_in_tmem = kATmem;
-  const PipeLayout L =
-      pipe_layout(S, p.BN, kCodeTileBytes, SC::kCbBytes * (8u >> p.cb_sh), 1 << p.cs_log, a_in_tmem ? 0u : kABytes);
+  const PipeLayout L = pipe_layout(S, p.BN, kCodeTileBytes, SC::kCbBytes * (8u >> p.cb_sh), 1 << p.cs_log,
+                                   a_in_tmem ? 0u : kABytes, kStreamK ? 8 : 1);
   const int cs_log = p.cs_log;          // code-tile slots: 1 << cs_log
   const int cs_mask = (1 << cs_log) - 1;
   const uint32_t sbase = smem_addr(smem);
@@ -521,21 +574,41 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
   uint64_t* cfull = empty + S;                                    // code tile landed
   uint64_t* cempty = cfull + kCodeSlots;                          // code tile read by the 8 decoder warps
   uint64_t* acc_bar = cempty + kCodeSlots;                        // accumulator complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+  // stream-K: acc_bar[a] = accumulator a complete, acc_bar[2 + a] = accumulator a
+  // drained, acc_bar[4 + q] = epilogue warp q's bulk copies landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + (kStreamK ? 8 : 1));
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int n0 = blockIdx.x * kRows;
-  const int b0 = blockIdx.y * p.BN;
+  const int n0 = kStreamK ? 0 : blockIdx.x * kRows;
+  const int b0 = kStreamK ? 0 : blockIdx.y * p.BN;
   const int split = blockIdx.z;  // == rank in the (1, 1, SK) cluster
   // this CTA's K range: stages [ks0, ks1), read as nct code tiles of kStagesPerTile
-  // stages starting at stage ks0 (the host keeps ks0's code offset 16-byte aligned)
-  const int ks0 = split * p.ks_per;
-  const int ks1 = min(p.nk, ks0 + p.ks_per);
-  const int nks = max(0, ks1 - ks0);  // host guarantees >= 1
+  // stages starting at stage ks0 (the host keeps ks0's code offset 16-byte aligned).
+  // Stream-K: stages [w0, w0 + nks) of the (tile, K stage) space; units are whole
+  // code tiles and nk a multiple of them, so no code tile straddles two tiles.
+  const SkRange skr{p.sk_ctas, p.sk_units, p.sk_unit};
+  const int w0 = kStreamK ? skr.begin(blockIdx.x) : 0;
+  const int ks0 = kStreamK ? 0 : split * p.ks_per;
+  const int ks1 = kStreamK ? 0 : min(p.nk, ks0 + p.ks_per);
+  const int nks = kStreamK ? skr.begin(blockIdx.x + 1) - w0 : max(0, ks1 - ks0);  // host guarantees >= 1
   const int nct = (nks + kStagesPerTile - 1) / kStagesPerTile;
+  // row-tile origin, batch-tile origin and K stage of the CTA's stage i
+  auto stage_at = [&](int i, int& n0_, int& b0_, int& k_) {
+    if constexpr (kStreamK) {
+      const int w = w0 + i;
+      const int t = w / p.nk;
+      k_ = w - t * p.nk;
+      n0_ = (t / p.batch_tiles) * kRows;
+      b0_ = (t % p.batch_tiles) * p.BN;
+    } else {
+      n0_ = n0;
+      b0_ = b0;
+      k_ = ks0 + i;
+    }
+  };
 
   // the next kernel on the stream may start its own set-up now; x is read (and
   // y written) only after this grid's dependency wait in the x producer below
@@ -552,6 +625,12 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
       mbar_init(&cempty[i], (kStagesPerTile >= kDecoderGroups ? kDecoders : kGroupThreads) / 32);
     }
     mbar_init(acc_bar, 1);
+    if constexpr (kStreamK) {
+      mbar_init(acc_bar + 1, 1);
+      mbar_init(acc_bar + 2, 4);  // the four epilogue warps
+      mbar_init(acc_bar + 3, 4);
+      for (int i = 4; i < 8; ++i) mbar_init(acc_bar + i, 1);
+    }
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -588,9 +667,10 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         const int s = i % S, u = i / S;
         if (u > 0 && !pipe_wait(&empty[s], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeEmpty))
           break;
+        int n0_, b0_, k_;
+        stage_at(i, n0_, b0_, k_);
         mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.BN) * 128u);
-        tma_load_2d(sbase + L.b + static_cast<uint32_t>(s * p.BN) * 128u, &x_map, (ks0 + i) * kStageK, b0, &full[s],
-                    pol);
+        tma_load_2d(sbase + L.b + static_cast<uint32_t>(s * p.BN) * 128u, &x_map, k_ * kStageK, b0_, &full[s], pol);
       }
     }
   } else if (warp == kWarpCodes) {
@@ -601,16 +681,18 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         const int c = t & cs_mask, u = t >> cs_log;
         if (u > 0 && !pipe_wait(&cempty[c], static_cast<uint32_t>((u - 1) & 1), abort_flag, p.status, kSitePipeCodes))
           break;
+        int n0_, b0_, k_;  // the tile's first stage
+        stage_at(t * kStagesPerTile, n0_, b0_, k_);
         mbar_arrive_expect_tx(&cfull[c], kCodeTileBytes);
         if constexpr (kGrad) {
-          // rows (ks0 + t) 64 .. + 63 of the CTA's feature columns; rows past N and
+          // rows k_ 64 .. + 63 of the feature columns of row tile n0_; rows past N and
           // bytes past the row end are zero-filled
           tma_load_2d(sbase + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes, &code_map,
-                      (n0 * SC::kTileCodeBytes / kRows) & ~15, (ks0 + t) * kStageK, &cfull[c], pol);
+                      (n0_ * SC::kTileCodeBytes / kRows) & ~15, k_ * kStageK, &cfull[c], pol);
         } else {
           // bytes past the row end (K edge) are zero-filled; stages past ks1 are not decoded
-          tma_load_2d(sbase + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes, &code_map,
-                      (ks0 + t * kStagesPerTile) * kStageCodeBytes, n0, &cfull[c], pol);
+          tma_load_2d(sbase + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes, &code_map, k_ * kStageCodeBytes,
+                      n0_, &cfull[c], pol);
         }
       }
     }
@@ -619,8 +701,24 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     if (lane == 0) {
       // the gradient's A stage is MN-major (bit 15 of the instruction descriptor)
       const uint32_t idesc = umma_idesc_f16_f32(kRows, static_cast<uint32_t>(p.BN)) | (kGrad ? (1u << 15) : 0u);
+      int piece = 0;  // stream-K: tile pieces begun so far; piece q accumulates into accumulator q mod 2
       for (int i = 0; i < nks; ++i) {
         const int s = i % S;
+        bool first = i == 0, last = i == nks - 1;  // the first / last stage of a tile piece
+        uint32_t d_tmem = tmem;
+        if constexpr (kStreamK) {
+          const int k_ = (w0 + i) % p.nk;
+          if (k_ == 0 && i > 0) ++piece;
+          first = first || k_ == 0;
+          last = last || k_ == p.nk - 1;
+          const int a = piece & 1;
+          d_tmem = tmem + static_cast<uint32_t>(a * p.acc_cols);
+          // the epilogue has drained what piece - 2 left in this accumulator
+          if (first && piece >= 2 &&
+              !pipe_wait(acc_bar + 2 + a, static_cast<uint32_t>(((piece - 2) >> 1) & 1), abort_flag, p.status,
+                         kSitePipeAcc))
+            break;
+        }
         if (!pipe_wait(&full[s], static_cast<uint32_t>((i / S) & 1), abort_flag, p.status, kSitePipeFull)) break;
         fence_proxy_async_smem();  // decoder writes (cp.async / st.shared) -> tensor-core reads
         tc_fence_after_sync();
@@ -630,7 +728,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
           const uint32_t a_tmem = tmem + kATmemCol + 32u * static_cast<uint32_t>(s);
 #pragma unroll
           for (int kk = 0; kk < kStageK / 16; ++kk)
-            umma_f16_ts(tmem, a_tmem + 8u * kk, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            umma_f16_ts(d_tmem, a_tmem + 8u * kk, bdesc + 2 * kk, idesc, (!first || kk > 0) ? 1u : 0u);
         } else {
           const uint32_t a_addr = sbase + L.a + static_cast<uint32_t>(s) * kABytes;
 #pragma unroll
@@ -638,12 +736,223 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
             // K = 16 per MMA: 32 bytes along a K-major row, or two 8-row atoms (2 x SBO) MN-major
             const uint64_t adesc = kGrad ? umma_desc_sw128_mnmajor(a_addr + 2u * kGradSbo * kk, kGradLbo, kGradSbo)
                                          : umma_desc_sw128_kmajor(a_addr) + 2 * kk;
-            umma_f16_ss(tmem, adesc, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            umma_f16_ss(d_tmem, adesc, bdesc + 2 * kk, idesc, (!first || kk > 0) ? 1u : 0u);
           }
         }
         umma_commit(&empty[s]);
+        if (kStreamK && last) umma_commit(acc_bar + (piece & 1));
       }
-      umma_commit(acc_bar);
+      if (!kStreamK) umma_commit(acc_bar);
+    }
+  } else if (kStreamK && warp >= kWarpEpi) {
+    if constexpr (kStreamK) {
+      // ---- stream-K epilogue.  Warp q = warp mod 4 owns TMEM lanes 32 q .. 32 q + 31,
+      // rows 32 q + lane of every tile piece of the CTA, taken in order as the MMAs
+      // complete them.  A tile done whole by this CTA goes straight to y.  A tile cut
+      // into P pieces (CTAs cf .. cf + P - 1, in K order) is finished by one of them:
+      // each piece stores its fp32 partial in its slot and counts itself in the
+      // counter of (cf, q); the piece that finds the other P - 1 counted (before
+      // storing, or from what its own increment returns) adds all P in K order (its own
+      // from TMEM), writes y and clears the counter.  No piece waits for another, the
+      // sum order does not depend on which piece finishes, and the warps of a CTA do
+      // not wait for each other.
+      //   A slot is [quadrant][BN / 4][32 rows][4] fp32, so the 32 rows of a warp form
+      // one contiguous run.  When the finishing piece is the CTA's last, every stage,
+      // code and codebook byte of shared memory is free (all MMAs are done), and each
+      // warp brings the other pieces' runs into its quarter of it with bulk copies
+      // before adding: the partial reads then cost one copy per piece instead of a
+      // chain of dependent L2 round trips per 16 columns.
+      const int q = warp & 3;
+      grid_dependency_wait();  // y and the workspace may be in use by the previous grid
+      const int cta = static_cast<int>(blockIdx.x);
+      const int w_end = w0 + nks;
+      const int BN = p.BN;
+      const uint32_t tq = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      const size_t slot_floats = static_cast<size_t>(kRows) * BN;
+      const size_t quad_float4s = static_cast<size_t>(BN / 4) * 32;  // this warp's run in a slot
+      const uint32_t quad_smem = ((L.bars - L.a) / 4u) & ~15u;        // this warp's share of the free memory
+      const uint32_t region = sbase + L.a + static_cast<uint32_t>(q) * quad_smem;
+      uint64_t* bulk_bar = acc_bar + 4 + q;
+      uint32_t bulk_phase = 0;
+      int piece = 0;
+      for (int w = w0; w < w_end; ++piece) {
+        const int t = w / p.nk;
+        const int w_next = min(w_end, (t + 1) * p.nk);
+        const int a = piece & 1;
+        if (!__all_sync(0xffffffffu,
+                        pipe_wait_sleepy(acc_bar + a, static_cast<uint32_t>((piece >> 1) & 1), abort_flag, p.status,
+                                         kSitePipeAcc) && !*abort_flag)) {
+          *abort_flag = 1u;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t acc = tq + static_cast<uint32_t>(a * p.acc_cols);
+        const int n0_ = (t / p.batch_tiles) * kRows, b0_ = (t % p.batch_tiles) * BN;
+        const int n = n0_ + 32 * q + lane;
+        const bool n_valid = n < p.rows;
+        // the gradient's scale is inside its A operand and it has no bias
+        const float sc = kGrad ? 1.f : (n_valid ? __half2float(p.scales[n]) : 0.f);
+        const float bi = (!kGrad && n_valid && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
+        const int cf = skr.cta_of(t * p.nk), cl = skr.cta_of((t + 1) * p.nk - 1);
+        const int P = cl - cf + 1;
+        // this warp's run of CTA cc's slot for tile t: slot 2 cc holds a CTA's first
+        // piece, 2 cc + 1 its last (middle pieces are whole tiles)
+        auto run_of = [&](int cc) {
+          return reinterpret_cast<float4*>(p.sk_part + static_cast<size_t>(2 * cc + (skr.begin(cc) < t * p.nk ? 1 : 0)) *
+                                                           slot_floats) +
+                 static_cast<size_t>(q) * quad_float4s;
+        };
+        auto store_y = [&](int c0, const float (&v)[16]) {
+          if (n_valid) {
+    #pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int b = b0_ + c0 + i;
+              if (b < p.batch) p.y[static_cast<size_t>(b) * p.rows + n] = __float2half_rn(v[i] * sc + bi);
+            }
+          }
+        };
+        uint32_t* cnt = p.sk_count + 4 * cf + q;
+        bool finish = P == 1;
+        if (!finish) {
+          uint32_t seen = lane == 0 ? ld_acquire_gpu_u32(cnt) : 0u;
+          seen = __shfl_sync(0xffffffffu, seen, 0);
+          if (seen == static_cast<uint32_t>(P - 1)) {
+            finish = true;  // every other piece is stored: no need to store this one
+          } else {
+            float4* mine = run_of(cta);
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+              float v[16];
+              tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c0), v);
+    #pragma unroll
+              for (int u = 0; u < 4; ++u)
+                __stcg(mine + (c0 / 4 + u) * 32 + lane, make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]));
+            }
+            __threadfence();
+            __syncwarp();
+            uint32_t old = lane == 0 ? atomicAdd(cnt, 1u) : 0u;
+            old = __shfl_sync(0xffffffffu, old, 0);
+            finish = old == static_cast<uint32_t>(P - 1);
+          }
+          if (finish) (void)ld_acquire_gpu_u32(cnt);  // every lane: the other pieces' stores are visible
+        }
+        if (finish && P == 1) {
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            float v[16];
+            tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c0), v);
+            store_y(c0, v);
+          }
+        } else if (finish && w_next == w_end && static_cast<uint32_t>(16 * ((P - 1) * 32 * 4 + 64)) <= quad_smem) {
+          // the CTA's last piece: the other pieces' runs come into shared memory by bulk
+          // copies, W columns of each per pass, and y leaves through a staged fp16 tile
+          // (32 rows x W columns, row index fastest) as 16-byte stores of 8 rows when
+          // the row count keeps them aligned
+          const int W = min(BN, static_cast<int>(quad_smem / static_cast<uint32_t>((P - 1) * 32 * 4 + 64)) / 16 * 16);
+          const bool vec_y = (p.rows & 7) == 0;
+          for (int c_lo = 0; c_lo < BN; c_lo += W) {
+            const int wcols = min(W, BN - c_lo);
+            const uint32_t run_bytes = static_cast<uint32_t>(wcols) * 32u * 4u;
+            __half* ystage = reinterpret_cast<__half*>(smem + (region - sbase) + static_cast<uint32_t>(P - 1) * run_bytes);
+            if (lane == 0) {
+              fence_proxy_async_global();  // the acquired partials, then the async-proxy copies
+              fence_proxy_async_smem();    // this warp's reads of the previous pass, then the copies
+              mbar_arrive_expect_tx(bulk_bar, static_cast<uint32_t>(P - 1) * run_bytes);
+              int k = 0;
+              for (int cc = cf; cc <= cl; ++cc) {
+                if (cc == cta) continue;
+                bulk_load(region + static_cast<uint32_t>(k) * run_bytes, run_of(cc) + (c_lo / 4) * 32, run_bytes,
+                          bulk_bar);
+                ++k;
+              }
+            }
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, pipe_wait(bulk_bar, bulk_phase, abort_flag, p.status, kSitePipeAcc))) {
+              *abort_flag = 1u;
+              break;
+            }
+            bulk_phase ^= 1u;
+            for (int c0 = c_lo; c0 < c_lo + wcols; c0 += 16) {
+              float v[16];
+              tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c0), v);
+              float sum[16];
+    #pragma unroll
+              for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+              int k = 0;
+              for (int cc = cf; cc <= cl; ++cc) {
+                if (cc == cta) {
+    #pragma unroll
+                  for (int i = 0; i < 16; ++i) sum[i] += v[i];
+                } else {
+                  const float4* src = reinterpret_cast<const float4*>(smem + (region - sbase)) +
+                                      static_cast<size_t>(k) * (run_bytes / 16u);
+    #pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    const float4 f = src[((c0 - c_lo) / 4 + u) * 32 + lane];
+                    sum[4 * u] += f.x;
+                    sum[4 * u + 1] += f.y;
+                    sum[4 * u + 2] += f.z;
+                    sum[4 * u + 3] += f.w;
+                  }
+                  ++k;
+                }
+              }
+              if (vec_y) {
+    #pragma unroll
+                for (int i = 0; i < 16; ++i) ystage[(c0 - c_lo + i) * 32 + lane] = __float2half_rn(sum[i] * sc + bi);
+              } else {
+                store_y(c0, sum);
+              }
+            }
+            if (vec_y) {
+              __syncwarp();  // the staged tile is complete
+              // lane l writes 8 rows of one column per step: 8 columns x 64 bytes per warp store
+              for (int u = lane; u < wcols * 4; u += 32) {
+                const int col = u >> 2, part = u & 3;
+                const int b = b0_ + c_lo + col;
+                const int nn = n0_ + 32 * q + 8 * part;
+                if (b < p.batch && nn < p.rows)
+                  *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(b) * p.rows + nn) =
+                      *reinterpret_cast<const uint4*>(ystage + col * 32 + 8 * part);
+              }
+            }
+            __syncwarp();  // every lane has read this pass before the next one's copies
+          }
+        } else if (finish) {
+          // a piece before the CTA's last: the pipeline still uses shared memory, so the
+          // partials are read from L2 directly
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            float v[16];
+            tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c0), v);
+            float sum[16];
+    #pragma unroll
+            for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+            for (int cc = cf; cc <= cl; ++cc) {
+              if (cc == cta) {
+    #pragma unroll
+                for (int i = 0; i < 16; ++i) sum[i] += v[i];
+              } else {
+                const float4* src = run_of(cc);
+    #pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const float4 f = __ldcg(src + (c0 / 4 + u) * 32 + lane);
+                  sum[4 * u] += f.x;
+                  sum[4 * u + 1] += f.y;
+                  sum[4 * u + 2] += f.z;
+                  sum[4 * u + 3] += f.w;
+                }
+              }
+            }
+            store_y(c0, sum);
+          }
+        }
+        if (finish && P > 1) {
+          __syncwarp();
+          if (lane == 0) *reinterpret_cast<volatile uint32_t*>(cnt) = 0u;  // ready for the next launch
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_bar + 2 + a);  // accumulator a may be overwritten
+        w = w_next;
+      }
     }
   } else {
     // the 65536-entry codebooks of the B = 16 schemes are gathered from L2 all kernel
@@ -657,8 +966,18 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     const int grp = warp / (kGroupThreads / 32);
     const int nl = 8 * (warp % (kGroupThreads / 32)) + (lane >> 2);
     const int qq = lane & 3;
-    const uint32_t code_off = static_cast<uint32_t>(nl * SC::kBoxBytes + ((n0 * SC::kTileCodeBytes / kRows) & 15) +
-                                                    qq * (SC::kTileCodeBytes / 4));
+    // this thread's codes in a code tile of row tile n0_ (whose first byte sits at
+    // offset (n0_ g-groups) mod 16 of the 16-byte-aligned box)
+    auto code_off_at = [&](int n0_) {
+      return static_cast<uint32_t>(nl * SC::kBoxBytes + ((n0_ * SC::kTileCodeBytes / kRows) & 15) +
+                                   qq * (SC::kTileCodeBytes / 4));
+    };
+    // output row n0_ and reduction row (over N) of stage i
+    auto grad_stage = [&](int i, int& n0_, int& n_) {
+      int b0_, k_;
+      stage_at(i, n0_, b0_, k_);
+      n_ = k_ * kStageK + nl;
+    };
     if constexpr (B == 16) {
       // codewords gathered from L2 into registers kLook stages ahead, as in the layer kernel
       constexpr int kLook = (M == 1) ? 3 : 1;
@@ -687,17 +1006,21 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
             break;
           }
           if (issue) {
-            const int n = (ks0 + i) * kStageK + nl;
+            int n0_, n;
+            grad_stage(i, n0_, n);
             const bool valid = n < p.N;
             sv[u] = valid ? __half2float(p.scales[n]) : 0.f;
-            gather_stage_b16<M, G>(st[u], smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, valid,
+            gather_stage_b16<M, G>(st[u], smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off_at(n0_),
+                                   valid,
                                    p.codebooks, p.cb32 != 0, cb_pol, 2 * (qq >> 1));
             __syncwarp();  // every lane has read its codes of this tile
             if (lane == 0) mbar_arrive(&cempty[c]);
           }
           if (store) {
             const int slot = (u + 1) % (kLook + 1);
-            const bool valid = (ks0 + j) * kStageK + nl < p.N;
+            int n0_, nj;
+            grad_stage(j, n0_, nj);
+            const bool valid = nj < p.N;
             const uint32_t a_off = L.a + static_cast<uint32_t>(sj) * kABytes;
 #pragma unroll
             for (int step = 0; step < 4; ++step) {
@@ -714,9 +1037,35 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
         }
       }
     } else {
-      // B = 8: codebooks in shared memory; the next stage's scale is loaded one stage ahead
-      const int n_first = (ks0 + grp) * kStageK + nl;
-      float s_next = (grp < nks && n_first < p.N) ? __half2float(p.scales[n_first]) : 0.f;
+      // B = 8: codebooks in shared memory; the next stage's scale is loaded one stage ahead.
+      // The (tile, K stage) of this group's stage is tracked by stepping, not divided out
+      // per stage (the decoders are issue-bound).
+      int ct = 0, ck = ks0 + grp;
+      if constexpr (kStreamK) {
+        const int w = w0 + grp;
+        ct = w / p.nk;
+        ck = w - ct * p.nk;
+      }
+      int cached_t = -1, cached_n0 = n0;
+      auto n0_of = [&](int t) {
+        if constexpr (kStreamK) {
+          if (t != cached_t) {
+            cached_t = t;
+            cached_n0 = (t / p.batch_tiles) * kRows;
+          }
+        }
+        return cached_n0;
+      };
+      auto step = [&](int& t, int& k) {
+        k += kDecoderGroups;
+        if constexpr (kStreamK) {
+          while (k >= p.nk) {
+            k -= p.nk;
+            ++t;
+          }
+        }
+      };
+      float s_next = (grp < nks && ck * kStageK + nl < p.N) ? __half2float(p.scales[ck * kStageK + nl]) : 0.f;
       for (int i = grp; i < nks; i += kDecoderGroups) {
         const int c = i & cs_mask;
         bool ready = pipe_wait(&cfull[c], static_cast<uint32_t>((i >> cs_log) & 1), abort_flag, p.status,
@@ -728,17 +1077,24 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
           *abort_flag = 1u;
           break;
         }
-        const int n = (ks0 + i) * kStageK + nl;
+        const int n = ck * kStageK + nl;
+        const int n0_ = n0_of(ct);
         const float sc = s_next;
-        const int n_next = n + kDecoderGroups * kStageK;
-        if (i + kDecoderGroups < nks) s_next = n_next < p.N ? __half2float(p.scales[n_next]) : 0.f;
+        int nt = ct, nkk = ck;
+        step(nt, nkk);
+        if (i + kDecoderGroups < nks) {
+          const int n_next = nkk * kStageK + nl;
+          s_next = n_next < p.N ? __half2float(p.scales[n_next]) : 0.f;
+        }
         decode_grad_b8<M, G>(smem, L.a + static_cast<uint32_t>(s) * kABytes, nl, qq, n < p.N,
-                             smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off, smem + L.cb, sc,
+                             smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes + code_off_at(n0_), smem + L.cb, sc,
                              p.cb_sh, lane);
         fence_proxy_async_smem();
         mbar_arrive(&full[s]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&cempty[c]);
+        ct = nt;
+        ck = nkk;
       }
     }
     } else {
@@ -750,6 +1106,18 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     const int hf = kDecoderGroups == 1 ? tid >> 7 : (tid >> 7) & 1;
     const int grp = kDecoderGroups == 1 ? 0 : tid / kGroupThreads;
     const bool row_valid = n0 + r < p.N;
+    // stream-K: whether row r of stage i's row tile exists
+    const bool all_rows = p.N % kRows == 0;  // every row tile full: no per-stage row test
+    auto row_valid_at = [&](int i) {
+      if constexpr (kStreamK) {
+        if (all_rows) return true;
+        int n0_, b0_, k_;
+        stage_at(i, n0_, b0_, k_);
+        return n0_ + r < p.N;
+      } else {
+        return row_valid;
+      }
+    };
     if constexpr (B == 16 && !PipeScheme<M, B, G>::kCpAsyncDecode) {
       // B = 16 except 1x16 g8: register-staged gathers, kLook stages ahead.  At step i
       // the thread issues the gathers of stage i (g = 16: one 256-bit load per 32-byte
@@ -786,7 +1154,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
             const uint8_t* cw = smem + L.codes + static_cast<uint32_t>(c) * kCodeTileBytes +
                                 code_tile_offset<SC::kTileRowBytes, SC::kSwizzle64>(
                                     r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
-            gather_stage_b16<M, G>(st[u], cw, row_valid, p.codebooks, p.cb32 != 0, cb_pol);
+            gather_stage_b16<M, G>(st[u], cw, row_valid_at(i), p.codebooks, p.cb32 != 0, cb_pol);
             if (within + kDecoderGroups >= kStagesPerTile || i + kDecoderGroups >= nks) {  // its last one
               __syncwarp();  // every lane has read its codes of this tile
               if (lane == 0) mbar_arrive(&cempty[c]);
@@ -836,7 +1204,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
                                 r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
         if (a_in_tmem) tc_fence_after_sync();  // the stage's release (MMA commit) -> these tcgen05.st
         decode_half_stage<M, B, G>(a_in_tmem, smem, sbase, L.a + static_cast<uint32_t>(s) * (a_in_tmem ? 0u : kABytes),
-                                           a_tmem_q + 32u * static_cast<uint32_t>(s), r, hf, row_valid, cw,
+                                           a_tmem_q + 32u * static_cast<uint32_t>(s), r, hf, row_valid_at(i), cw,
                                            p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
         if constexpr (B == 16) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
@@ -872,7 +1240,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
                                 r, within * kStageCodeBytes + hf * (kStageCodeBytes / 2));
         if (a_in_tmem) tc_fence_after_sync();  // the stage's release (MMA commit) -> these tcgen05.st
         decode_half_stage<M, B, G>(a_in_tmem, smem, sbase, L.a + static_cast<uint32_t>(s) * (a_in_tmem ? 0u : kABytes),
-                                           a_tmem_q + 32u * static_cast<uint32_t>(s), r, hf, row_valid, cw,
+                                           a_tmem_q + 32u * static_cast<uint32_t>(s), r, hf, row_valid_at(i), cw,
                                            p.codebooks, smem + L.cb, cb_pol, p.cb_sh);
         if constexpr (B == 16) {
           cp_async_arrive_noinc(&full[s]);  // 1x16 g8: the stage lands by cp.async
@@ -894,7 +1262,8 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
     asm volatile("cp.async.wait_all;" ::: "memory");
   }
 
-  // ---- epilogue ----------------------------------------------------------------------
+  // ---- epilogue (stream-K kernels finish their pieces above) ------------------------
+  if constexpr (!kStreamK) {
   // Decoder warp w reads TMEM lanes 32*(w % 4).. (weight rows) and, with the other
   // warps of its lane quadrant, every (kDecoders / 128)-th 16-column chunk of the batch tile.
   const bool decoder = warp < kDecoders / 32;
@@ -974,6 +1343,7 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
       }
     }
   }
+  }  // !kStreamK
 
   if (*abort_flag) {
     // a wait gave up: let copies already in flight land before the CTA leaves
@@ -1001,46 +1371,97 @@ __global__ void __launch_bounds__(PipeShape<M, B, G, kGrad>::kThreads, 1)
 struct TcPlan {
   int S = 0, SK = 1, ks_per = 0, red_rows = 128, cb_sh = 3, cs_log = 2;
   bool a_tmem = false;
+  bool streamk = false;  // stream-K schedule (needs the caller's workspace)
+  int sk_ctas = 0, sk_units = 0, sk_unit = 0;
 };
 
 constexpr int kPlanFixedStages = 3;     // set-up, pipeline fill and epilogue, in stage times
 constexpr int kPlanExchangePer16 = 2;   // split-K exchange, stage times per 16 batch columns
 constexpr int kMaxSplit = 16;
+// Stream-K: at most this many CTAs (one per SM; B200 has 148), so the workspace size is
+// known without a device.  Its overhead over a tile plan, in stage times: the fix-up of
+// cut tiles, the four-warp epilogue of every CTA's last piece, the spread of CTA
+// finish times that the next launch waits for, and a slower stage loop (measured: 0.85
+// to 0.9 us per stage against 0.57 to 0.75 for the same decode in tile plans, with 4x
+// the long-scoreboard stalls).  Measured on B200, one launch after another: about
+// 45-50 stage times at batch tile 256, about 5 at tile 16, so 8 + BN / 6.  Only the
+// input-gradient kernel gains, where its tile plan leaves a mostly empty last wave
+// (4096 x 14336 at batch 1024: 448 tiles on 148 SMs, 191-194 -> 177-184 us); the layer
+// kernel lost in every measured shape (2x8 11008 x 4096 at batch 256: 37.7 us as 86
+// tiles, 50.6 as stream-K; 14336 x 4096 at batch 1024: 147 against 163 us), so the
+// cost model offers stream-K to the gradient kernel only, and the layer kernel runs
+// it when a caller asks for it (AQLM_SCHEDULE_STREAMK).
+constexpr int kMaxSkCtas = 160;
+constexpr int kSkOverheadStages = 8;
+
+// Schemes with a stream-K kernel: all but the B = 16 gradient kernels, whose
+// register-staged gathers do not fit the 80 registers a thread has with the four
+// epilogue warps added (they spilled).
+template <int M, int B, int G, bool kGrad>
+constexpr bool kStreamKOk = !(kGrad && B == 16);
+
+// Stream-K work units: code tiles of the layer kernel (so no code tile straddles two
+// tiles), single stages for the gradient.  0 when the shape cannot use stream-K: the
+// A stages would live in tensor memory (its columns hold the second accumulator), or
+// nk is not a whole number of units.
+template <int M, int B, int G, bool kGrad>
+inline int streamk_unit(int nk, int BN) {
+  using SC = std::conditional_t<kGrad, GradScheme<M, B, G>, PipeScheme<M, B, G>>;
+  if (!kStreamKOk<M, B, G, kGrad>) return 0;
+  if (SC::kATmemOk && BN <= 128) return 0;
+  return nk % SC::kStagesPerTile == 0 ? SC::kStagesPerTile : 0;
+}
+
+// fp32 partial slots of the stream-K schedule with C CTAs: 2 C slots of 128 x BN.
+// (The counters live apart, in the kStreamKCounterBytes at the start of a workspace.)
+inline size_t streamk_partial_bytes(int C, int BN) {
+  return static_cast<size_t>(2 * C) * kRows * static_cast<size_t>(BN) * sizeof(float);
+}
+static_assert(kStreamKCounterBytes == static_cast<size_t>(kMaxSkCtas) * 4 * sizeof(uint32_t),
+              "one counter per (CTA, lane quadrant)");
 
 template <int M, int B, int G, bool kGrad>
 using PipeSchemeOf = std::conditional_t<kGrad, GradScheme<M, B, G>, PipeScheme<M, B, G>>;
 
 template <int M, int B, int G, bool kGrad>
-inline uint32_t pipe_smem_bytes(int S, int BN, int cb_sh, int cs_log, bool a_tmem) {
+inline uint32_t pipe_smem_bytes(int S, int BN, int cb_sh, int cs_log, bool a_tmem, bool streamk = false) {
   using SC = PipeSchemeOf<M, B, G, kGrad>;
-  const uint32_t bytes =
-      pipe_layout(S, BN, SC::kCodeTileBytes, SC::kCbBytes * (8u >> cb_sh), 1 << cs_log, a_tmem ? 0u : kABytes).total +
-      1024;
+  const uint32_t bytes = pipe_layout(S, BN, SC::kCodeTileBytes, SC::kCbBytes * (8u >> cb_sh), 1 << cs_log,
+                                     a_tmem ? 0u : kABytes, streamk ? 8 : 1)
+                             .total +
+                         1024;
   // With A in tensor memory a CTA allocates all 512 columns.  Two such CTAs on one SM
   // (from consecutive launches, or if the layout were small enough) would make the
   // second one's tcgen05.alloc wait for the first, and with split-K clusters two
   // clusters could then wait on each other.  Asking for more than half an SM's shared
-  // memory keeps every such CTA alone on its SM.
-  return a_tmem ? std::max(bytes, kSmemLimit / 2 + 1024u) : bytes;
+  // memory keeps every such CTA alone on its SM.  Stream-K CTAs stay alone too: the
+  // schedule spreads the work over one CTA per SM.
+  return (a_tmem || streamk) ? std::max(bytes, kSmemLimit / 2 + 1024u) : bytes;
 }
 
-// The instantiation a launch runs: A stages in tensor memory or in shared memory.
+// The instantiation a launch runs: A stages in tensor memory or in shared memory, or
+// the stream-K kernel.
 using PipeKernelFn = void (*)(CUtensorMap, CUtensorMap, PipeParams);
 template <int M, int B, int G, bool kGrad>
-PipeKernelFn pipe_kernel(bool a_tmem) {
-  if constexpr (PipeSchemeOf<M, B, G, kGrad>::kATmemOk) {
-    if (a_tmem) return tc_pipe_kernel<M, B, G, kGrad, true>;
+PipeKernelFn pipe_kernel(bool a_tmem, bool streamk = false) {
+  if constexpr (kStreamKOk<M, B, G, kGrad>) {
+    if (streamk) return tc_pipe_kernel<M, B, G, kGrad, false, true>;
   }
-  return tc_pipe_kernel<M, B, G, kGrad, false>;
+  if constexpr (PipeSchemeOf<M, B, G, kGrad>::kATmemOk) {
+    if (a_tmem) return tc_pipe_kernel<M, B, G, kGrad, true, false>;
+  }
+  return tc_pipe_kernel<M, B, G, kGrad, false, false>;
 }
 
 // rows: output rows (the MMA's M extent); nk: 64-wide reduction stages.
+// ws_ok: the caller gave a workspace for the stream-K schedule.  schedule: 0 = the cost
+// model picks, 1 = tile plan, 2 = stream-K (cudaErrorInvalidConfiguration if it cannot run).
 template <int M, int B, int G, bool kGrad>
-cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, TcPlan* out) {
+cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, bool ws_ok, int schedule, TcPlan* out) {
   constexpr int kSplitAlign = PipeSchemeOf<M, B, G, kGrad>::kSplitAlign;  // split starts keep 16-byte code offsets
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int>, TcPlan> cache;
-  const auto key = std::make_tuple(dev, rows, nk, batch);
+  static std::map<std::tuple<int, int, int, int, bool, int>, TcPlan> cache;
+  const auto key = std::make_tuple(dev, rows, nk, batch, ws_ok, schedule);
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -1127,6 +1548,45 @@ cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, TcPlan* out)
     }
   }
   if (best_cost < 0) return cudaErrorNotSupported;
+  // Stream-K: one CTA per SM over (tile, stage) units, so no SM idles when the tiles do
+  // not divide evenly over the SMs.  Taken when its estimate, overhead included
+  // (kSkOverheadStages), beats the tile plan's.
+  const int unit = streamk_unit<M, B, G, kGrad>(nk, BN);
+  if (ws_ok && unit > 0 && (schedule == 2 || (schedule == 0 && kGrad))) {
+    auto kern_sk = pipe_kernel<M, B, G, kGrad>(false, true);
+    int sms = 0;
+    if (cudaFuncSetAttribute(kern_sk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit)) ==
+            cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
+      const long long units = clusters * (nk / unit);
+      const int C = static_cast<int>(std::min<long long>({static_cast<long long>(sms), units, kMaxSkCtas}));
+      for (int S = 6; S >= 2 && C > 0; --S) {
+        const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(S, BN, cb_sh, cs_log, false, true);
+        if (smem > kSmemLimit) continue;
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern_sk, PipeShape<M, B, G, kGrad, true>::kThreads,
+                                                          smem) != cudaSuccess ||
+            per_sm < 1)
+          continue;
+        const long long per = (units + C - 1) / C * unit;
+        const long long cost = 16 * (per + kPlanFixedStages + kSkOverheadStages + BN / 6);
+        if (cost < best_cost || schedule == 2) {
+          best.streamk = true;
+          best.S = S;
+          best.SK = 1;
+          best.ks_per = 0;
+          best.red_rows = kRows;
+          best.a_tmem = false;
+          best.sk_ctas = C;
+          best.sk_units = static_cast<int>(units);
+          best.sk_unit = unit;
+        }
+        break;  // the deepest ring that fits
+      }
+    }
+    cudaGetLastError();
+  }
+  if (schedule == 2 && !best.streamk) return cudaErrorInvalidConfiguration;
   std::lock_guard<std::mutex> lock(mu);
   cache[key] = best;
   *out = best;
@@ -1139,7 +1599,7 @@ cudaError_t plan_pipe(int dev, int rows, int nk, int batch, int BN, TcPlan* out)
 template <int M, int B, int G, bool kGrad>
 cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, size_t row_bytes, int N,
                                uint32_t box_x, uint32_t box_rows, PipeParams p, const TcPlan& plan,
-                               cudaStream_t stream) {
+                               uint32_t* sk_count, float* sk_part, cudaStream_t stream) {
   EncodeTiledFn encode = encode_tiled();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap x_map, code_map;
@@ -1169,9 +1629,22 @@ cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, si
   }
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(p.BN)) cols <<= 1;
+  p.acc_cols = static_cast<int>(cols);
   // A stages in tensor memory: the accumulator's 256 columns, then 32 a stage
   if (plan.a_tmem) cols = 512;
+  // stream-K: two accumulators
+  if (plan.streamk) cols *= 2;
   p.tmem_cols = cols;
+  const int row_tiles = (p.rows + kRows - 1) / kRows;
+  const int batch_tiles = (p.batch + p.BN - 1) / p.BN;
+  p.batch_tiles = batch_tiles;
+  if (plan.streamk) {
+    p.sk_ctas = plan.sk_ctas;
+    p.sk_units = plan.sk_units;
+    p.sk_unit = plan.sk_unit;
+    p.sk_count = sk_count;
+    p.sk_part = sk_part;
+  }
   p.S = plan.S;
   p.SK = plan.SK;
   p.ks_per = plan.ks_per;
@@ -1179,16 +1652,15 @@ cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, si
   p.cb_sh = plan.cb_sh;
   p.cs_log = plan.cs_log;
   p.cb32 = (reinterpret_cast<uintptr_t>(p.codebooks) & 31u) == 0 ? 1 : 0;
-  const uint32_t smem = pipe_smem_bytes<M, B, G, kGrad>(plan.S, p.BN, plan.cb_sh, plan.cs_log, plan.a_tmem);
-  auto kern = pipe_kernel<M, B, G, kGrad>(plan.a_tmem);
+  const uint32_t smem =
+      pipe_smem_bytes<M, B, G, kGrad>(plan.S, p.BN, plan.cb_sh, plan.cs_log, plan.a_tmem, plan.streamk);
+  auto kern = pipe_kernel<M, B, G, kGrad>(plan.a_tmem, plan.streamk);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
   if (e != cudaSuccess) return e;
   if (plan.SK > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  const int row_tiles = (p.rows + kRows - 1) / kRows;
-  const int batch_tiles = (p.batch + p.BN - 1) / p.BN;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1197,9 +1669,11 @@ cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, si
   attr[0].val.clusterDim.z = static_cast<unsigned>(plan.SK);
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(row_tiles), static_cast<unsigned>(batch_tiles),
-                     static_cast<unsigned>(plan.SK));
-  cfg.blockDim = dim3(PipeShape<M, B, G, kGrad>::kThreads, 1, 1);
+  cfg.gridDim = plan.streamk ? dim3(static_cast<unsigned>(plan.sk_ctas), 1, 1)
+                             : dim3(static_cast<unsigned>(row_tiles), static_cast<unsigned>(batch_tiles),
+                                    static_cast<unsigned>(plan.SK));
+  cfg.blockDim = dim3(plan.streamk ? PipeShape<M, B, G, kGrad, true>::kThreads : PipeShape<M, B, G, kGrad>::kThreads,
+                      1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
@@ -1210,6 +1684,18 @@ cudaError_t launch_pipe_kernel(const void* x_src, int red, const void* codes, si
 // Batch tile: the batch rounded up to a multiple of 16, at most 256 (the MMA's N).
 inline int pipe_batch_tile(int batch) { return std::min(256, (batch + 15) / 16 * 16); }
 
+// Partial-slot bytes the stream-K schedule needs for (rows, nk, batch) on any device
+// (at most kMaxSkCtas CTAs); 0 when the shape cannot use it.
+template <int M, int B, int G, bool kGrad>
+size_t pipe_partial_bytes(int rows, int nk, int batch) {
+  const int BN = pipe_batch_tile(batch);
+  const int unit = streamk_unit<M, B, G, kGrad>(nk, BN);
+  if (unit == 0) return 0;
+  const long long tiles = static_cast<long long>((rows + kRows - 1) / kRows) * ((batch + BN - 1) / BN);
+  const long long units = tiles * (nk / unit);
+  return streamk_partial_bytes(static_cast<int>(std::min<long long>(units, kMaxSkCtas)), BN);
+}
+
 template <int M, int B, int G>
 cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream) {
   using SC = PipeScheme<M, B, G>;
@@ -1219,8 +1705,10 @@ cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const int BN = pipe_batch_tile(pr.batch);
+  const size_t part_need = pipe_partial_bytes<M, B, G, false>(pr.N, pr.K / kStageK, pr.batch);
+  const bool ws_ok = part_need > 0 && pr.sk_count != nullptr && pr.sk_part != nullptr && pr.sk_part_bytes >= part_need;
   TcPlan plan;
-  e = plan_pipe<M, B, G, false>(dev, pr.N, pr.K / kStageK, pr.batch, BN, &plan);
+  e = plan_pipe<M, B, G, false>(dev, pr.N, pr.K / kStageK, pr.batch, BN, ws_ok, pr.schedule, &plan);
   if (e != cudaSuccess) return e;
   PipeParams p{};
   p.codebooks = static_cast<const __half*>(pr.codebooks);
@@ -1237,7 +1725,7 @@ cudaError_t launch_pipe(const Problem& pr, uint32_t* status, cudaStream_t stream
   const size_t row_bytes = static_cast<size_t>(pr.K / G) * M * SC::kCodeBytes;
   return launch_pipe_kernel<M, B, G, false>(pr.x, pr.K, pr.codes, row_bytes, pr.N,
                                             static_cast<uint32_t>(SC::kTileRowBytes), static_cast<uint32_t>(kRows), p,
-                                            plan, stream);
+                                            plan, pr.sk_count, pr.sk_part, stream);
 }
 
 template <int M, int B, int G>
@@ -1250,8 +1738,10 @@ cudaError_t launch_grad(const GradProblem& pr, uint32_t* status, cudaStream_t st
   if (e != cudaSuccess) return e;
   const int BN = pipe_batch_tile(pr.batch);
   const int nk = (pr.N + kStageK - 1) / kStageK;
+  const size_t part_need = pipe_partial_bytes<M, B, G, true>(pr.K, nk, pr.batch);
+  const bool ws_ok = part_need > 0 && pr.sk_count != nullptr && pr.sk_part != nullptr && pr.sk_part_bytes >= part_need;
   TcPlan plan;
-  e = plan_pipe<M, B, G, true>(dev, pr.K, nk, pr.batch, BN, &plan);
+  e = plan_pipe<M, B, G, true>(dev, pr.K, nk, pr.batch, BN, ws_ok, pr.schedule, &plan);
   if (e != cudaSuccess) return e;
   PipeParams p{};
   p.codebooks = static_cast<const __half*>(pr.codebooks);
@@ -1268,7 +1758,7 @@ cudaError_t launch_grad(const GradProblem& pr, uint32_t* status, cudaStream_t st
   const size_t row_bytes = static_cast<size_t>(pr.K / G) * M * SC::kCodeBytes;
   return launch_pipe_kernel<M, B, G, true>(pr.dy, pr.N, pr.codes, row_bytes, pr.N,
                                            static_cast<uint32_t>(SC::kBoxBytes), static_cast<uint32_t>(kStageK), p,
-                                           plan, stream);
+                                           plan, pr.sk_count, pr.sk_part, stream);
 }
 
 struct PipeLauncher {
@@ -1285,6 +1775,22 @@ struct GradLauncher {
   }
 };
 
+struct PipeWorkspace {
+  template <int M, int B, int G>
+  static size_t run(int K, int N, int batch) {
+    if (!tc_pipelined_shape(M, B, G, K)) return 0;
+    return pipe_partial_bytes<M, B, G, false>(N, K / kStageK, batch);
+  }
+};
+
+struct GradWorkspace {
+  template <int M, int B, int G>
+  static size_t run(int K, int N, int batch) {
+    if (!grad_shape_supported(M, B, G, K, N)) return 0;
+    return pipe_partial_bytes<M, B, G, true>(K, (N + kStageK - 1) / kStageK, batch);
+  }
+};
+
 }  // namespace
 
 cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t stream) {
@@ -1293,6 +1799,14 @@ cudaError_t launch_tc_pipelined(const Problem& p, uint32_t* status, cudaStream_t
 
 cudaError_t launch_input_grad(const GradProblem& p, uint32_t* status, cudaStream_t stream) {
   return dispatch_scheme<GradLauncher>(p.M, p.B, p.g, cudaErrorNotSupported, p, status, stream);
+}
+
+size_t tc_pipe_partial_bytes(int M, int B, int g, int K, int N, int batch) {
+  return dispatch_scheme<PipeWorkspace>(M, B, g, size_t{0}, K, N, batch);
+}
+
+size_t input_grad_partial_bytes(int M, int B, int g, int K, int N, int batch) {
+  return dispatch_scheme<GradWorkspace>(M, B, g, size_t{0}, K, N, batch);
 }
 
 }  // namespace aqlm

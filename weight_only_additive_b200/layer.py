@@ -11,7 +11,7 @@ import numpy as np
 import torch
 
 from . import native
-from .native import Path
+from .native import Path, Schedule
 
 
 def _stream_handle(stream: Optional[torch.cuda.Stream], device) -> int:
@@ -21,6 +21,40 @@ def _stream_handle(stream: Optional[torch.cuda.Stream], device) -> int:
 
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
+
+
+# Workspaces of the tensor-core kernel's stream-K schedule, one per (device, stream):
+# calls on one stream may share one (the library leaves its counters zero), calls on
+# different streams must not.
+_workspaces: dict = {}
+
+
+def stream_workspace(nbytes: int, device, stream: Optional[torch.cuda.Stream] = None) -> Optional[torch.Tensor]:
+    """A zero-filled uint8 workspace of at least `nbytes` for calls on `stream` (the
+    device's current stream if None), kept and grown per (device, stream); None for 0."""
+    if nbytes <= 0:
+        return None
+    dev = torch.device(device)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    key = (dev.index, s.cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        # filled on the stream that uses it, so the fill is ordered before every call
+        with torch.cuda.stream(s):
+            ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
+        _workspaces[key] = ws
+    return ws
+
+
+def _resolve_workspace(workspace, nbytes: int, dev, stream):
+    """(pointer, bytes) for the C call: the caller's tensor, none (False), or the
+    per-stream workspace (None)."""
+    if workspace is False or nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = stream_workspace(nbytes, dev, stream)
+    _check_tensor(workspace, "workspace", torch.uint8, dev)
+    return workspace.data_ptr(), workspace.numel()
 
 
 @dataclass
@@ -64,8 +98,13 @@ def _check_tensor(t: torch.Tensor, name: str, dtype, device):
 
 
 def matmul(x: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = None,
-           path: Path = Path.AUTO, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """y = x . W^T . diag(s) + bias for x [batch, K] fp16 on the weights' device."""
+           path: Path = Path.AUTO, stream: Optional[torch.cuda.Stream] = None, workspace=None,
+           schedule: Schedule = Schedule.AUTO) -> torch.Tensor:
+    """y = x . W^T . diag(s) + bias for x [batch, K] fp16 on the weights' device.
+
+    workspace: None for this stream's cached workspace (stream_workspace), False for
+    none, or a zero-filled uint8 tensor of at least aqlm_matmul_workspace_size bytes.
+    schedule: the tensor-core kernel's work schedule (aqlm_schedule)."""
     dev = w.codes.device
     if dev.type != "cuda":
         raise ValueError("AQLM weights must live on a CUDA device")
@@ -76,16 +115,20 @@ def matmul(x: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = None,
     if out is None:
         out = torch.empty((batch, w.N), dtype=torch.float16, device=dev)
     _check_tensor(out, "out", torch.float16, dev)
-    native.aqlm_matmul_path(x.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(),
-                            w.scales.data_ptr(), _ptr(w.bias), out.data_ptr(),
-                            w.M, w.B, w.g, K, w.N, batch, path, _stream_handle(stream, dev))
+    ws, ws_bytes = _resolve_workspace(workspace, native.aqlm_matmul_workspace_size(w.M, w.B, w.g, K, w.N, batch),
+                                      dev, stream)
+    native.aqlm_matmul_ws(x.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(),
+                          w.scales.data_ptr(), _ptr(w.bias), out.data_ptr(),
+                          w.M, w.B, w.g, K, w.N, batch, path, schedule, ws, ws_bytes, _stream_handle(stream, dev))
     return out
 
 
 def input_grad(dy: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = None,
-               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+               stream: Optional[torch.cuda.Stream] = None, workspace=None,
+               schedule: Schedule = Schedule.AUTO) -> torch.Tensor:
     """dx = dy . diag(s) . W [batch, K] for dy [batch, N] fp16: the gradient of
-    matmul() with respect to its input (the weights are fixed)."""
+    matmul() with respect to its input (the weights are fixed).  workspace and
+    schedule as for matmul (aqlm_input_grad_workspace_size bytes)."""
     dev = w.codes.device
     if dev.type != "cuda":
         raise ValueError("AQLM weights must live on a CUDA device")
@@ -96,8 +139,11 @@ def input_grad(dy: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = N
     if out is None:
         out = torch.empty((batch, w.K), dtype=torch.float16, device=dev)
     _check_tensor(out, "out", torch.float16, dev)
-    native.aqlm_input_grad(dy.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(), w.scales.data_ptr(),
-                           out.data_ptr(), w.M, w.B, w.g, w.K, N, batch, _stream_handle(stream, dev))
+    ws, ws_bytes = _resolve_workspace(
+        workspace, native.aqlm_input_grad_workspace_size(w.M, w.B, w.g, w.K, N, batch), dev, stream)
+    native.aqlm_input_grad_ws(dy.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(), w.scales.data_ptr(),
+                              out.data_ptr(), w.M, w.B, w.g, w.K, N, batch, schedule, ws, ws_bytes,
+                              _stream_handle(stream, dev))
     return out
 
 
@@ -147,7 +193,8 @@ class LayerGroup:
         self.count = len(probs)
         self.workspace_bytes = native.aqlm_group_workspace_size(self.problems, self.count)
         # 256-byte aligned: torch's caching allocator hands out 512-byte aligned blocks
-        self.workspace = torch.empty((max(self.workspace_bytes, 1),), dtype=torch.uint8, device=dev)
+        # zero-filled once: the stream-K part keeps counters that every call leaves zero
+        self.workspace = torch.zeros((max(self.workspace_bytes, 1),), dtype=torch.uint8, device=dev)
 
     def run(self, stream: Optional[torch.cuda.Stream] = None):
         native.aqlm_matmul_group(self.problems, self.workspace.data_ptr(), self.workspace_bytes,

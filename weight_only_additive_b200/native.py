@@ -20,9 +20,10 @@ EXPORTS = ("aqlm_matmul", "aqlm_matmul_path", "aqlm_dequantize", "aqlm_select_pa
            "aqlm_last_cuda_error", "aqlm_abi_version", "aqlm_matmul_group",
            "aqlm_group_workspace_size", "aqlm_matmul_group_static", "aqlm_selftest_bounded_wait",
            "aqlm_input_grad", "aqlm_validate_input_grad", "aqlm_matmul_group_host",
-           "aqlm_static_group_scratch_bytes")
+           "aqlm_static_group_scratch_bytes", "aqlm_matmul_workspace_size", "aqlm_matmul_ws",
+           "aqlm_input_grad_workspace_size", "aqlm_input_grad_ws")
 
-ABI_VERSION = 7
+ABI_VERSION = 8
 
 # Site code aqlm_selftest_bounded_wait records in the device status word.
 SITE_SELFTEST = 0x501
@@ -31,6 +32,10 @@ SITE_SELFTEST = 0x501
 # (AQLM_STATIC_GROUP_SCRATCH_BYTES; the library reports its own value through
 # aqlm_static_group_scratch_bytes, which a CPU test compares with this one).
 STATIC_GROUP_SCRATCH_BYTES = 16 << 20
+
+# Counters at the start of a workspace that can carry the tensor-core kernel's
+# stream-K schedule (AQLM_WORKSPACE_COUNTER_BYTES; a CPU test compares the two).
+WORKSPACE_COUNTER_BYTES = 2560
 
 # Grouped problems one launch pair of aqlm_matmul_group computes together.
 MAX_GROUP_LAYERS = 32
@@ -43,6 +48,12 @@ class Status(enum.IntEnum):
     MISALIGNED = 3
     CUDA = 4
     TIMEOUT = 5
+
+
+class Schedule(enum.IntEnum):
+    AUTO = 0
+    TILES = 1
+    STREAMK = 2
 
 
 class Path(enum.IntEnum):
@@ -100,6 +111,16 @@ def lib() -> ctypes.CDLL:
                 L.aqlm_validate.restype = _i
                 L.aqlm_input_grad.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
                 L.aqlm_input_grad.restype = _i
+                L.aqlm_matmul_workspace_size.argtypes = [_i] * 6
+                L.aqlm_matmul_workspace_size.restype = ctypes.c_size_t
+                L.aqlm_matmul_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                             ctypes.c_size_t, _vp]
+                L.aqlm_matmul_ws.restype = _i
+                L.aqlm_input_grad_workspace_size.argtypes = [_i] * 6
+                L.aqlm_input_grad_workspace_size.restype = ctypes.c_size_t
+                L.aqlm_input_grad_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                                 ctypes.c_size_t, _vp]
+                L.aqlm_input_grad_ws.restype = _i
                 L.aqlm_validate_input_grad.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i]
                 L.aqlm_validate_input_grad.restype = _i
                 L.aqlm_status_string.argtypes = [_i]
@@ -147,6 +168,26 @@ def aqlm_matmul(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, stre
 def aqlm_matmul_path(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path, stream=None):
     _check(lib().aqlm_matmul_path(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch,
                                   int(path), stream), "aqlm_matmul_path")
+
+
+def aqlm_matmul_workspace_size(M, B, g, K, N, batch) -> int:
+    return lib().aqlm_matmul_workspace_size(M, B, g, K, N, batch)
+
+
+def aqlm_matmul_ws(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path, schedule, workspace,
+                   workspace_bytes, stream=None):
+    _check(lib().aqlm_matmul_ws(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, int(path),
+                                int(schedule), workspace, workspace_bytes, stream), "aqlm_matmul_ws")
+
+
+def aqlm_input_grad_workspace_size(M, B, g, K, N, batch) -> int:
+    return lib().aqlm_input_grad_workspace_size(M, B, g, K, N, batch)
+
+
+def aqlm_input_grad_ws(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch, schedule, workspace,
+                       workspace_bytes, stream=None):
+    _check(lib().aqlm_input_grad_ws(dy, codes, codebooks, scales, dx, M, B, g, K, N, batch, int(schedule),
+                                    workspace, workspace_bytes, stream), "aqlm_input_grad_ws")
 
 
 def aqlm_dequantize(codes, codebooks, scales, W_out, M, B, g, K, N, stream=None):
