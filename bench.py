@@ -94,6 +94,9 @@ def parse_args(argv=None):
                    help="replace every layer's codebook scheme (MxBgG, e.g. 4x8g8): the generic shapes")
     p.add_argument("--op", choices=("matmul", "input-grad"), default="matmul",
                    help="the layer (default) or its input gradient dx = dy . diag(s) . W")
+    p.add_argument("--schedule", choices=("auto", "tiles", "streamk"), default="auto",
+                   help="work schedule of the tensor-core kernel for --launch per-layer and --op input-grad "
+                        "(aqlm_schedule; the group call always uses auto)")
     p.add_argument("--pool", type=int, default=None,
                    help="rotating-pool copies (default: enough to exceed 3x L2); smaller for profiler captures")
     a = p.parse_args(argv)
@@ -134,6 +137,12 @@ KERNEL_SOURCES = {"gemv_gather_kernel": ("gemv.cu", "aqlm_device.cuh"),
                   "tc_decode_mma_kernel": ("tc_gemm.cu", "aqlm_device.cuh"),
                   "tc_pipe_kernel": ("tc_pipe.cu", "aqlm_device.cuh"),
                   "lut_group_kernel": ("lut_group.cu", "lut_table.cuh", "aqlm_device.cuh")}
+
+
+def schedule_of(a, native):
+    """The aqlm_schedule value of --schedule."""
+    return {"auto": native.Schedule.AUTO, "tiles": native.Schedule.TILES,
+            "streamk": native.Schedule.STREAMK}[getattr(a, "schedule", "auto")]
 
 
 def kernel_source_sha256(kernel):
@@ -471,6 +480,7 @@ class Bench:
         from weight_only_additive_b200 import native
 
         self.torch, self.L, self.native = torch, L, native
+        self.a = a
         self.rank, self.world, self.local = env_rank()
         if self.world > 1:
             import torch.distributed as dist
@@ -538,7 +548,7 @@ class Pool:
         ws = (self.ws.data_ptr(), ws_bytes) if ws_bytes else (None, 0)
         self.calls = [[(self.xs[c][li].data_ptr(), wt.codes.data_ptr(), wt.codebooks.data_ptr(), wt.scales.data_ptr(),
                         None, self.ys[li].data_ptr(), wt.M, wt.B, wt.g, lay.K, lay.N, batch, int(b.native.Path.AUTO),
-                        int(b.native.Schedule.AUTO), ws[0] if b.native.aqlm_matmul_workspace_size(wt.M, wt.B, wt.g, lay.K, lay.N, batch) else None,
+                        int(schedule_of(b.a, b.native)), ws[0] if b.native.aqlm_matmul_workspace_size(wt.M, wt.B, wt.g, lay.K, lay.N, batch) else None,
                         ws[1] if b.native.aqlm_matmul_workspace_size(wt.M, wt.B, wt.g, lay.K, lay.N, batch) else 0, h)
                        for li, (lay, wt) in enumerate(zip(w.layers, self.weights[c]))] for c in range(pool)]
         self.b = b
@@ -828,7 +838,8 @@ def run_ours(a):
                            "algorithmic_bytes_per_step": sbytes,
                            "l2": pool_desc,
                            "launch": ("one aqlm_matmul_group call per step (grouped lookup-table kernel + "
-                                      "reduction)" if mode == "group" else "one aqlm_matmul call per layer")
+                                      "reduction)" if mode == "group"
+                                      else f"one aqlm_matmul_ws call per layer, schedule {a.schedule}")
                                      + f"; CUDA graphs of {pool_size} consecutive steps (one pass over the pool)",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu, "cpu_kernel": cpu_kernel, "e2e": e2e,
@@ -929,7 +940,7 @@ def run_input_grad(a):
     ws = torch.zeros((max(max(ws_need), 1),), dtype=torch.uint8, device=dev)
     calls = [[(dys[c][li].data_ptr(), weights[c][li].codes.data_ptr(), weights[c][li].codebooks.data_ptr(),
                weights[c][li].scales.data_ptr(), dxs[li].data_ptr(), lay.scheme.M, lay.scheme.B, lay.scheme.g,
-               lay.K, lay.N, batch, int(native.Schedule.AUTO), ws.data_ptr() if ws_need[li] else None,
+               lay.K, lay.N, batch, int(schedule_of(a, native)), ws.data_ptr() if ws_need[li] else None,
                ws.numel() if ws_need[li] else 0, h)
               for li, lay in enumerate(w.layers)] for c in range(pool)]
 
@@ -1052,7 +1063,8 @@ def run_input_grad(a):
                            "flops_per_step": sflops,
                            "l2": f"inputs larger than L2: rotating pool of {pool} copies "
                                  f"({pool * sbytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
-                           "launch": f"one aqlm_input_grad call per layer; CUDA graphs of {pool} steps",
+                           "launch": f"one aqlm_input_grad_ws call per layer, schedule {a.schedule}; "
+                                     f"CUDA graphs of {pool} steps",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": len(w.layers) * steps, "clocks": clocks.summary(), "gpu": props.name}
