@@ -126,15 +126,20 @@ aqlm_status aqlm_matmul_path(const void* x, const void* codes, const void* codeb
                              aqlm_path path, aqlm_stream_t stream);
 
 /*
- * Bytes of workspace with which aqlm_matmul_ws may run the tensor-core kernel on a
- * stream-K schedule: every SM takes an equal share of the (weight-row tile, batch
- * tile, 64-wide K stage) space, and a tile cut between SMs is finished by the piece
- * that ends last, from fp32 partials in the workspace, summed in K order (so results
- * do not depend on timing).  The same y = x . W^T . diag(s) + bias as aqlm_matmul.
- * 0 when the shape never uses it (the schedule needs the decoded weight stages in
- * shared memory, i.e. a batch tile above 128 for schemes other than 1x16 g8, and K
- * a whole number of code tiles), or for invalid arguments.  Pure host logic, the
- * same for every device: needs no GPU.
+ * Bytes of workspace aqlm_matmul_ws can use for this shape, for either of:
+ *  - the tensor-core kernel's stream-K schedule: every SM takes an equal share of the
+ *    (weight-row tile, batch tile, 64-wide K stage) space, and a tile cut between SMs
+ *    is finished by the piece that ends last, from fp32 partials in the workspace,
+ *    summed in K order (so results do not depend on timing).  It needs the decoded
+ *    weight stages in shared memory (a batch tile above 128 for schemes other than
+ *    1x16 g8) and K a whole number of code tiles;
+ *  - batch 1 with 256-entry codebooks, at least 10 MiB of codes and code rows of at
+ *    least 1536 bytes: AUTO then runs the grouped lookup kernel of aqlm_matmul_group
+ *    on this one layer (faster there than the single-layer lookup kernel), its fp32
+ *    partial sums in the workspace.
+ * The same y = x . W^T . diag(s) + bias as aqlm_matmul either way.  0 when the shape
+ * uses neither, or for invalid arguments.  Pure host logic, the same for every
+ * device: needs no GPU.
  */
 size_t aqlm_matmul_workspace_size(int M, int B, int g, int K, int N, int batch);
 

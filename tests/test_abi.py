@@ -324,6 +324,22 @@ def test_matmul_workspace_size(lib):
     assert native.aqlm_matmul_workspace_size(5, 8, 8, 4096, 11008, 256) == 0
 
 
+def test_matmul_workspace_size_for_the_grouped_route(lib):
+    """Batch-1 B = 8 layers with >= 10 MiB of codes in code rows of >= 1536 bytes get
+    the counters plus the grouped kernel's partial sums (one fp32 per row and 128 code
+    bytes); the others, at batch 1 with A in tensor memory, none."""
+    def grouped(M, g, K, N):
+        slices = (K // g * M + 127) // 128
+        return COUNTERS + (slices * N * 4 + 255) // 256 * 256
+    assert native.aqlm_matmul_workspace_size(3, 8, 8, 4096, 11008, 1) == grouped(3, 8, 4096, 11008)
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 11008, 4096, 1) == grouped(2, 8, 11008, 4096)
+    assert native.aqlm_matmul_workspace_size(4, 8, 16, 11008, 4096, 1) == grouped(4, 16, 11008, 4096)
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 4096, 11008, 1) == 0   # 1024-byte rows
+    assert native.aqlm_matmul_workspace_size(4, 8, 8, 4096, 4096, 1) == 0    # 8 MiB of codes
+    assert native.aqlm_matmul_workspace_size(3, 8, 16, 11008, 4096, 1) == 0  # 8.1 MiB of codes
+    assert native.aqlm_matmul_workspace_size(2, 8, 8, 11008, 4096, 2) == 0   # batch 2
+
+
 def test_input_grad_workspace_size(lib):
     # Mixtral expert down-projection at batch 1024: 32 feature tiles x 4 batch tiles,
     # 224 single-stage units each

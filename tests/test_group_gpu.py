@@ -310,3 +310,28 @@ def test_group_llama_set_other_schemes_sampled_rows(dev, scheme):
         rows = np.unique(np.concatenate([rng.choice(lay.N, size=24, replace=False), [0, lay.N - 1]]))
         y_ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, M, 8, g, rows=rows)
         assert_close(item[2].cpu().numpy()[:, rows], y_ref, f"{scheme}/{lay.name}")
+
+
+@pytest.mark.parametrize("M,g,K,N", [(3, 8, 4096, 11008), (2, 8, 11008, 4096), (4, 8, 14336, 4096),
+                                     (4, 16, 11008, 4096)])
+def test_single_layer_call_takes_the_grouped_kernel_where_it_pays(dev, M, g, K, N):
+    """aqlm_matmul_ws at batch 1 (AUTO, with a workspace) runs the grouped lookup kernel
+    on long-row B = 8 layers with at least 10 MiB of codes: its result equals a
+    one-element group call's bit for bit (the same kernel and sum order), and the oracle
+    within the layer tolerance.  Without a workspace the single-layer kernel runs."""
+    assert native.aqlm_matmul_workspace_size(M, 8, g, K, N, 1) > 0
+    ld = synth.make_layer(M, 8, g, K, N, seed=77, with_bias=True)
+    x = synth.make_x(1, K, seed=78)
+    w = L.AqlmWeights.from_numpy(ld, dev)
+    xt = torch.from_numpy(x).to(dev)
+    out = torch.empty((1, N), dtype=torch.float16, device=dev)
+    L.LayerGroup([(w, xt, out)]).run()
+    y_route = L.matmul(xt, w)             # the per-stream workspace: routed
+    y_single = L.matmul(xt, w, workspace=False)
+    check_status()
+    assert np.array_equal(y_route.cpu().numpy().view(np.uint16), out.cpu().numpy().view(np.uint16))
+    rows = np.unique(np.concatenate([np.random.Generator(np.random.PCG64(N)).choice(N, 48, replace=False),
+                                     [0, 127, N - 1]]))
+    ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, 8, g, rows=rows)
+    assert_close(y_route.cpu().numpy()[:, rows], ref, f"routed {M}x8 g{g} {N}x{K}")
+    assert_close(y_single.cpu().numpy()[:, rows], ref, f"single-layer {M}x8 g{g} {N}x{K}")

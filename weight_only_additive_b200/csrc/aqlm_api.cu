@@ -86,6 +86,19 @@ bool path_accepts(aqlm_path path, int M, int B, int g, int K, int batch) {
 
 aqlm_status launch_matmul(const aqlm::Problem& p, aqlm_path path, cudaStream_t s);
 
+// Batch-1 layers that the grouped lookup kernel, as a one-problem group, runs faster
+// than the single-layer lookup kernel: measured on B200 for every B = 8 scheme at the
+// published shapes, the single-layer kernel's clusters fall behind once a layer has
+// at least 10 MiB of codes in code rows of at least 1536 bytes (3x8 g8 11008 x 4096:
+// 13.3 -> 11.1 us; 4x8 g8 4096 x 14336: 26.6 -> 15.6 us; 2x8 g8 4096 x 11008: 10.2 ->
+// 9.4 us), and is as fast or faster below (4x8 g8 4096 x 4096: 7.7 against 8.7 us;
+// 2x8 g8 11008 x 4096 with 1024-byte rows: 7.6 us).
+bool group_route_pays(const aqlm::Problem& p) {
+  if (p.batch != 1 || !aqlm::lut_group_supported(p)) return false;
+  const long long row_bytes = static_cast<long long>(p.K / p.g) * p.M * (p.B <= 8 ? 1 : 2);
+  return row_bytes >= 1536 && row_bytes * p.N >= (10ll << 20);
+}
+
 // A schedule request against the shape's workspace need (`need` 0: no stream-K).
 aqlm_status check_schedule(aqlm_schedule schedule, const void* workspace, size_t need) {
   if (schedule < AQLM_SCHEDULE_AUTO || schedule > AQLM_SCHEDULE_STREAMK) return AQLM_ERR_INVALID_ARG;
@@ -210,7 +223,9 @@ aqlm_status aqlm_validate(const void* x, const void* codes, const void* codebook
 
 size_t aqlm_matmul_workspace_size(int M, int B, int g, int K, int N, int batch) {
   if (validate_shape(M, B, g, K, N, batch) != AQLM_OK) return 0;
-  const size_t part = aqlm::tc_pipe_partial_bytes(M, B, g, K, N, batch);
+  size_t part = aqlm::tc_pipe_partial_bytes(M, B, g, K, N, batch);
+  const aqlm::Problem p{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, M, B, g, K, N, batch};
+  if (group_route_pays(p)) part = std::max(part, aqlm::lut_group_workspace_bytes(&p, 1));
   return part > 0 ? AQLM_WORKSPACE_COUNTER_BYTES + part : 0;
 }
 
@@ -242,6 +257,14 @@ aqlm_status aqlm_matmul_ws(const void* x, const void* codes, const void* codeboo
     p.sk_part_bytes = workspace_bytes - AQLM_WORKSPACE_COUNTER_BYTES;
   }
   p.schedule = static_cast<int>(schedule);
+  if (path == AQLM_PATH_AUTO && workspace && group_route_pays(p)) {
+    // a batch-1 layer the grouped lookup kernel runs faster than the single-layer one:
+    // a one-problem group, its partial sums after the workspace's counters
+    uint32_t* status = device_status_ptr();
+    if (!status) return from_cuda(cudaErrorInvalidDevice);
+    return from_cuda(aqlm::launch_lut_group(&p, 1, static_cast<uint8_t*>(workspace) + AQLM_WORKSPACE_COUNTER_BYTES,
+                                            status, reinterpret_cast<cudaStream_t>(stream)));
+  }
   return launch_matmul(p, path, reinterpret_cast<cudaStream_t>(stream));
 }
 
