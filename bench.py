@@ -644,54 +644,68 @@ class Pool:
     def e2e(self, mode, steps):
         """The same metric through the public API with host buffers: per step one pinned
         H2D copy of every layer's x (packed), the group call (aqlm_matmul_group_host, the
-        copies inside the call) or one aqlm_matmul per layer, one D2H copy of every y."""
+        copies inside the call) or one aqlm_matmul per layer, one D2H copy of every y.
+        Steps alternate between two streams, each with its own host and device buffers
+        (double buffering, as a serving loop would), so one step's copies overlap the
+        other stream's kernels; every step still moves its own inputs and result."""
         b, torch, w, batch = self.b, self.b.torch, self.w, self.batch
         L = b.L
         koff = np.cumsum([0] + [batch * lay.K for lay in w.layers])
         noff = np.cumsum([0] + [batch * lay.N for lay in w.layers])
-        hx_flat = torch.empty((int(koff[-1]),), dtype=torch.float16).pin_memory()
-        for li, lay in enumerate(w.layers):
-            hx_flat[koff[li]:koff[li + 1]] = torch.from_numpy(
-                synth.make_x(batch, lay.K, seed=7, layer=li)).reshape(-1)
-        hy_flat = torch.empty((int(noff[-1]),), dtype=torch.float16).pin_memory()
-        dx_flat = torch.empty_like(hx_flat, device=b.dev)
-        dy_flat = torch.empty_like(hy_flat, device=b.dev)
-        dx = [dx_flat[koff[li]:koff[li + 1]].view(batch, lay.K) for li, lay in enumerate(w.layers)]
-        dy = [dy_flat[noff[li]:noff[li + 1]].view(batch, lay.N) for li, lay in enumerate(w.layers)]
-        groups = [L.LayerGroup([(self.weights[c][li], dx[li], dy[li]) for li in range(len(w.layers))])
-                  for c in range(self.size)]
+        streams = [b.stream, torch.cuda.Stream(b.dev)]
+        sets = []
+        for si in range(2):
+            hx_flat = torch.empty((int(koff[-1]),), dtype=torch.float16).pin_memory()
+            for li, lay in enumerate(w.layers):
+                hx_flat[koff[li]:koff[li + 1]] = torch.from_numpy(
+                    synth.make_x(batch, lay.K, seed=7 + si, layer=li)).reshape(-1)
+            hy_flat = torch.empty((int(noff[-1]),), dtype=torch.float16).pin_memory()
+            dx_flat = torch.empty_like(hx_flat, device=b.dev)
+            dy_flat = torch.empty_like(hy_flat, device=b.dev)
+            dx = [dx_flat[koff[li]:koff[li + 1]].view(batch, lay.K) for li, lay in enumerate(w.layers)]
+            dy = [dy_flat[noff[li]:noff[li + 1]].view(batch, lay.N) for li, lay in enumerate(w.layers)]
+            groups = ([L.LayerGroup([(self.weights[c][li], dx[li], dy[li]) for li in range(len(w.layers))])
+                       for c in range(self.size)] if mode == "group" else None)
+            sets.append((hx_flat, hy_flat, dx_flat, dy_flat, dx, dy, groups))
 
-        def e2e_step(c):
+        def e2e_step(i):
+            si, c = i % 2, i % self.size
+            hx_flat, hy_flat, dx_flat, dy_flat, dx, dy, groups = sets[si]
+            st = streams[si]
             if mode == "group":
-                groups[c].run_host(hx_flat, hy_flat, stream=b.stream)
+                groups[c].run_host(hx_flat, hy_flat, stream=st)
             else:
-                dx_flat.copy_(hx_flat, non_blocking=True)
-                for li in range(len(w.layers)):
-                    L.matmul(dx[li], self.weights[c][li], out=dy[li], stream=b.stream)
-                hy_flat.copy_(dy_flat, non_blocking=True)
+                with torch.cuda.stream(st):
+                    dx_flat.copy_(hx_flat, non_blocking=True)
+                    for li in range(len(w.layers)):
+                        L.matmul(dx[li], self.weights[c][li], out=dy[li], stream=st)
+                    hy_flat.copy_(dy_flat, non_blocking=True)
 
-        with torch.cuda.stream(b.stream):
-            for i in range(3):
-                e2e_step(i % self.size)
+        for i in range(4):
+            e2e_step(i)
         torch.cuda.synchronize(b.dev)
         b.barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(b.stream):
-            e0.record(b.stream)
-            for i in range(steps):
-                e2e_step(i % self.size)
-            e1.record(b.stream)
+        e0.record(streams[0])
+        streams[1].wait_event(e0)
+        for i in range(steps):
+            e2e_step(i)
+        done1 = torch.cuda.Event()
+        done1.record(streams[1])
+        streams[0].wait_event(done1)
+        e1.record(streams[0])
         torch.cuda.synchronize(b.dev)
         ems = max_over_ranks(e0.elapsed_time(e1), b.dist, b.dev)
         api = ("weight_only_additive_b200.layer.LayerGroup.run_host -> aqlm_matmul_group_host (the copies "
                "inside the call)" if mode == "group"
-               else "weight_only_additive_b200.layer.matmul -> aqlm_matmul, per layer")
+               else "weight_only_additive_b200.layer.matmul -> aqlm_matmul_ws, per layer")
         return {"value": job_throughput_gbs(self.copy_bytes, steps, b.world, ems), "unit": "GB/s",
-                "h2d_bytes_per_step": hx_flat.numel() * 2, "d2h_bytes_per_step": hy_flat.numel() * 2,
+                "h2d_bytes_per_step": sets[0][0].numel() * 2, "d2h_bytes_per_step": sets[0][1].numel() * 2,
                 "steps": steps, "us_per_layer": ems * 1e3 / (steps * len(w.layers)),
                 "how": f"per step: one pinned H2D copy of every layer's x (packed), {api}, one D2H copy "
-                       f"of every y (packed); no CUDA graph"}
+                       f"of every y (packed); no CUDA graph; steps alternate between two streams with their "
+                       f"own host and device buffers, so one step's copies overlap the other's kernels"}
 
 
 def measure_config(b, w, batch, steps, warmup, with_e2e=True):
