@@ -1023,39 +1023,53 @@ def run_input_grad(a):
         e2e_steps = max(3, min(steps, 200))
         noff = np.cumsum([0] + [batch * lay.N for lay in w.layers])
         koff = np.cumsum([0] + [batch * lay.K for lay in w.layers])
-        hdy = torch.empty((int(noff[-1]),), dtype=torch.float16).pin_memory()
-        for li, lay in enumerate(w.layers):
-            hdy[noff[li]:noff[li + 1]] = torch.from_numpy(synth.make_x(batch, lay.N, seed=7, layer=li)).reshape(-1)
-        hdx = torch.empty((int(koff[-1]),), dtype=torch.float16).pin_memory()
-        ddy, ddx = torch.empty_like(hdy, device=dev), torch.empty_like(hdx, device=dev)
-        vdy = [ddy[noff[li]:noff[li + 1]].view(batch, lay.N) for li, lay in enumerate(w.layers)]
-        vdx = [ddx[koff[li]:koff[li + 1]].view(batch, lay.K) for li, lay in enumerate(w.layers)]
+        # two streams, each with its own host and device buffers (double buffering):
+        # one step's copies overlap the other stream's kernels
+        streams = [stream, torch.cuda.Stream(dev)]
+        sets = []
+        for si in range(2):
+            hdy = torch.empty((int(noff[-1]),), dtype=torch.float16).pin_memory()
+            for li, lay in enumerate(w.layers):
+                hdy[noff[li]:noff[li + 1]] = torch.from_numpy(
+                    synth.make_x(batch, lay.N, seed=7 + si, layer=li)).reshape(-1)
+            hdx = torch.empty((int(koff[-1]),), dtype=torch.float16).pin_memory()
+            ddy, ddx = torch.empty_like(hdy, device=dev), torch.empty_like(hdx, device=dev)
+            vdy = [ddy[noff[li]:noff[li + 1]].view(batch, lay.N) for li, lay in enumerate(w.layers)]
+            vdx = [ddx[koff[li]:koff[li + 1]].view(batch, lay.K) for li, lay in enumerate(w.layers)]
+            sets.append((hdy, hdx, ddy, ddx, vdy, vdx))
 
-        def e2e_step(c):
-            ddy.copy_(hdy, non_blocking=True)
-            for li in range(len(w.layers)):
-                L.input_grad(vdy[li], weights[c][li], out=vdx[li], stream=stream)
-            hdx.copy_(ddx, non_blocking=True)
+        def e2e_step(i):
+            hdy, hdx, ddy, ddx, vdy, vdx = sets[i % 2]
+            st = streams[i % 2]
+            with torch.cuda.stream(st):
+                ddy.copy_(hdy, non_blocking=True)
+                for li in range(len(w.layers)):
+                    L.input_grad(vdy[li], weights[i % pool][li], out=vdx[li], stream=st,
+                                 schedule=schedule_of(a, native))
+                hdx.copy_(ddx, non_blocking=True)
 
-        with torch.cuda.stream(stream):
-            for i in range(3):
-                e2e_step(i % pool)
+        for i in range(4):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for i in range(e2e_steps):
-                e2e_step(i % pool)
-            e1.record(stream)
+        e0.record(streams[0])
+        streams[1].wait_event(e0)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        done1 = torch.cuda.Event()
+        done1.record(streams[1])
+        streams[0].wait_event(done1)
+        e1.record(streams[0])
         torch.cuda.synchronize(dev)
         ems = max_over_ranks(e0.elapsed_time(e1), dist, dev)
         e2e = {"value": sflops * e2e_steps * world / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": hdy.numel() * 2, "d2h_bytes_per_step": hdx.numel() * 2,
+               "h2d_bytes_per_step": sets[0][0].numel() * 2, "d2h_bytes_per_step": sets[0][1].numel() * 2,
                "steps": e2e_steps, "us_per_layer": ems * 1e3 / (e2e_steps * len(w.layers)),
                "how": "per step: one pinned H2D copy of every layer's dy (packed), "
-                      "weight_only_additive_b200.layer.input_grad -> aqlm_input_grad per layer, one D2H copy "
-                      "of every dx (packed); no CUDA graph"}
+                      "weight_only_additive_b200.layer.input_grad -> aqlm_input_grad_ws per layer, one D2H "
+                      "copy of every dx (packed); no CUDA graph; steps alternate between two streams with "
+                      "their own host and device buffers, so one step's copies overlap the other's kernels"}
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
