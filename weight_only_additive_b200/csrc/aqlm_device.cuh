@@ -315,7 +315,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
 
-// 2D TMA tile load (never with multicast) into this CTA's shared memory; the
+// 2D TMA tile load into this CTA's own shared memory only (no cluster-wide copy); the
 // destination must be 128-byte aligned (1024 for a 128-byte-swizzled map) and
 // x * element size a multiple of 16 bytes.  Completes `bytes` on `bar`.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
@@ -326,9 +326,9 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(pol) : "memory");
 }
 
-// Bulk copy (no tensor map, never with multicast) of `bytes` (a multiple of 16) from
-// this GPU's global memory at `src` (16-byte aligned) into this CTA's shared memory at
-// `dst` (16-byte aligned).  Completes `bytes` on `bar`.
+// Bulk copy (no tensor map) of `bytes` (a multiple of 16) from this GPU's global
+// memory at `src` (16-byte aligned) into this CTA's own shared memory at `dst`
+// (16-byte aligned), and nowhere else.  Completes `bytes` on `bar`.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
