@@ -267,16 +267,13 @@ typedef struct {
  * reduction); the others are launched one after another as by aqlm_matmul.  Both kernels of a
  * pair keep the stream-ordering contract above.
  *
- * workspace: caller-owned DEVICE memory of aqlm_group_workspace_size(problems,
- * count) bytes, 256-byte aligned (NULL allowed when that size is 0), zero-filled
- * before its first use.  Layout: the AQLM_WORKSPACE_COUNTER_BYTES of stream-K
- * counters (as for aqlm_matmul_ws), then the fp32 partial sums between the two
- * kernels of a pair (required when any problem is grouped, else
- * AQLM_ERR_INVALID_ARG), then, after those rounded up to 256 bytes, the stream-K
- * partial slots that the problems launched one by one share (used only when the
- * whole size is given).  Every call whose kernels finish leaves it reusable, as for
- * aqlm_matmul_ws; calls that may run concurrently (different streams) must not
- * share a workspace.
+ * workspace: caller-owned DEVICE memory of at least
+ * aqlm_group_workspace_size(problems, count) bytes, 256-byte aligned (NULL allowed
+ * when that size is 0).  Layout: AQLM_WORKSPACE_COUNTER_BYTES left untouched (the
+ * counters of aqlm_matmul_ws sit there, so one buffer may serve both kinds of call on
+ * a stream), then the fp32 partial sums between the two kernels of a pair, which
+ * need no initialisation.  Calls that may run concurrently (different streams) must
+ * not share a workspace.
  * count == 0 is a no-op; count < 0 or problems == NULL (with count > 0) is
  * AQLM_ERR_INVALID_ARG.  Every problem is validated as aqlm_validate does before
  * anything is launched.
@@ -291,14 +288,11 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
  * AQLM_STATIC_GROUP_SCRATCH_BYTES inside the library (one per device; the address
  * is taken with cudaGetSymbolAddress on a device's first call and again whenever
  * the device's CUDA context has changed, e.g. after cudaDeviceReset); the call
- * allocates nothing.  Problems whose grouped part (the counters plus the grouped
- * partial sums of aqlm_group_workspace_size) exceeds that size are rejected with
- * AQLM_ERR_INVALID_ARG before anything is launched (16 MiB covers, for example, a
- * Llama-2-7B decoder layer set, 1.6 MB, or the 24 Mixtral-8x7B expert linears of
- * one layer, 11 MB).  The buffer needs no clearing: the reduction reads only
- * partials written by the same call.  Problems launched one by one use its
- * stream-K layout when the whole aqlm_group_workspace_size fits (the buffer starts
- * zero-filled and every call leaves the counters so).
+ * allocates nothing.  Problems whose aqlm_group_workspace_size exceeds that size
+ * are rejected with AQLM_ERR_INVALID_ARG before anything is launched (16 MiB
+ * covers, for example, a Llama-2-7B decoder layer set, 1.6 MB, or the 24
+ * Mixtral-8x7B expert linears of one layer, 11 MB).  The buffer needs no clearing:
+ * the reduction reads only partials written by the same call.
  * Calls that overlap in time (different streams or host threads on one device)
  * share the buffer and RACE: the caller must serialise them.  Calls on one
  * stream are ordered and safe.  Otherwise identical to aqlm_matmul_group.
@@ -328,13 +322,11 @@ aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aq
 aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, const void* x_host, void* y_host,
                                    void* workspace, size_t workspace_bytes, aqlm_stream_t stream);
 
-/* Workspace bytes aqlm_matmul_group takes for these problems: 0 if no problem is
- * grouped and none launched one by one has a nonzero aqlm_matmul_workspace_size;
- * else AQLM_WORKSPACE_COUNTER_BYTES, plus the grouped part (for every run of up to
- * 32 grouped problems, the sum over them of ceil(K / g * M / 128) * N * 4 bytes, one
- * fp32 partial per row and 128 code bytes, rounded up to 256; the maximum over
- * runs), plus the largest stream-K partial-slot size (aqlm_matmul_workspace_size
- * minus the counters) of the problems launched one by one.  Pure host logic. */
+/* Workspace bytes aqlm_matmul_group needs for these problems: 0 if no problem is
+ * grouped; else AQLM_WORKSPACE_COUNTER_BYTES plus, for every run of up to 32 grouped
+ * problems, the sum over them of ceil(K / g * M / 128) * N * 4 bytes (one fp32
+ * partial per row and 128 code bytes) rounded up to 256, the maximum over runs.  The
+ * problems launched one by one need none.  Pure host logic. */
 size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count);
 
 /* The kernel family AQLM_PATH_AUTO picks for this problem, or -1 if unsupported.

@@ -146,18 +146,17 @@ def _ws_bytes(K, N):
 
 
 def test_group_workspace_size(lib):
-    # layout: counters, grouped partial sums, the stream-K slots of the 1x16 layer
-    # launched on its own
+    # layout: the counters region, then the grouped partial sums; the 1x16 layer is
+    # launched on its own and needs nothing
     P = [_prob(1 << 32), _prob(1 << 33, K=11008, N=200), _prob(1 << 34, M=1, B=16)]
     grouped = _ws_bytes(4096, 4096) + _ws_bytes(11008, 200)
-    assert native.aqlm_group_workspace_size(P) == COUNTERS + grouped + _streamk_parts(32 * 16, 16)
+    assert native.aqlm_group_workspace_size(P) == COUNTERS + grouped
     assert native.aqlm_group_workspace_size(P[:2]) == COUNTERS + grouped
     assert native.aqlm_group_workspace_size([]) == 0
-    assert native.aqlm_group_workspace_size([_prob(1 << 32, M=1, B=16)]) == _streamk_bytes(32, 32 * 16, 16)
-    assert native.aqlm_group_workspace_size([_prob(1 << 32, M=1, B=16, K=4104)]) == 0  # nothing grouped, no stream-K
-    # batch 256: the largest stream-K slots of the layers launched one by one
+    assert native.aqlm_group_workspace_size([_prob(1 << 32, M=1, B=16)]) == 0       # nothing grouped
+    # batch 256: nothing grouped, the layers run the tile plans
     big = [_prob(1 << 32, batch=256, N=11008), _prob(1 << 33, batch=256, N=1000, K=2048)]
-    assert native.aqlm_group_workspace_size(big) == _streamk_bytes(86, 86 * 16, 256)
+    assert native.aqlm_group_workspace_size(big) == 0
     assert native.aqlm_group_workspace_size([_prob(1 << 32, batch=2)]) == 0         # batch 2: not grouped
     assert native.aqlm_group_workspace_size([_prob(1 << 32, K=4104)]) == 0          # K % 64 != 0
     assert native.aqlm_group_workspace_size([_prob(1 << 32, K=4095)]) == 0          # invalid shape

@@ -423,37 +423,15 @@ size_t group_workspace(const aqlm_problem* problems, int count) {
   return best;
 }
 
-// Stream-K partial slots of a group workspace: the largest need of the problems
-// launched one by one (they run in turn on the call's stream and share them).
-size_t group_streamk_partials(const aqlm_problem* problems, int count) {
-  size_t best = 0;
-  for (int i = 0; i < count; ++i) {
-    const aqlm_problem& q = problems[i];
-    if (aqlm::lut_group_supported(to_problem(q))) continue;
-    best = std::max(best, aqlm::tc_pipe_partial_bytes(q.M, q.B, q.g, q.K, q.N, q.batch));
-  }
-  return best;
-}
-
 size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 
-// Layout of a group workspace: [stream-K counters][grouped partial sums][stream-K
-// partial slots].  The counters come first in every workspace, so calls with other
-// problem sets (the static scratch serves them all) never write partials over them.
-struct GroupLayout {
-  size_t grouped = 0;   // bytes of grouped partial sums
-  size_t sk_part = 0;   // bytes of stream-K partial slots
-  size_t required() const { return grouped > 0 ? AQLM_WORKSPACE_COUNTER_BYTES + grouped : 0; }
-  size_t full() const {
-    return (grouped > 0 || sk_part > 0) ? AQLM_WORKSPACE_COUNTER_BYTES + round256(grouped) + sk_part : 0;
-  }
-};
-
-GroupLayout group_layout(const aqlm_problem* problems, int count) {
-  GroupLayout g;
-  g.grouped = group_workspace(problems, count);
-  g.sk_part = group_streamk_partials(problems, count);
-  return g;
+// Bytes a group workspace needs: the counters of the stream-K layout (kept first in
+// every workspace of this library, so a buffer shared with aqlm_matmul_ws calls never
+// has partials written over them), then the grouped partial sums; 0 when nothing is
+// grouped.  The problems launched one by one run the tile plans, which need none.
+size_t group_need(const aqlm_problem* problems, int count) {
+  const size_t grouped = group_workspace(problems, count);
+  return grouped > 0 ? AQLM_WORKSPACE_COUNTER_BYTES + round256(grouped) : 0;
 }
 
 }  // namespace
@@ -464,7 +442,7 @@ size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count) {
     const aqlm_problem& q = problems[i];
     if (validate_shape(q.M, q.B, q.g, q.K, q.N, q.batch) != AQLM_OK) return 0;
   }
-  return group_layout(problems, count).full();
+  return group_need(problems, count);
 }
 
 aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* workspace,
@@ -489,17 +467,12 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
         if (overlaps(ri[5], rj[k])) return AQLM_ERR_INVALID_ARG;
     }
   }
-  const GroupLayout lay = group_layout(problems, count);
-  const size_t need = lay.required();
+  const size_t need = group_need(problems, count);
   if (need > 0) {
     if (!workspace || workspace_bytes < need) return AQLM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return AQLM_ERR_MISALIGNED;
   }
   uint8_t* const ws = static_cast<uint8_t*>(workspace);
-  // the problems launched one by one run the tensor-core kernel's stream-K schedule
-  // when the workspace has room for its partial slots too
-  const bool sk_ok = lay.sk_part > 0 && ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 &&
-                     workspace_bytes >= lay.full();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   aqlm::Problem run[aqlm::kMaxGroupLayers];
   int n_run = 0;
@@ -521,13 +494,7 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
     if (aqlm::lut_group_supported(p)) {
       run[n_run++] = p;
     } else {
-      aqlm::Problem one = p;
-      if (sk_ok) {
-        one.sk_count = reinterpret_cast<uint32_t*>(ws);
-        one.sk_part = reinterpret_cast<float*>(ws + AQLM_WORKSPACE_COUNTER_BYTES + round256(lay.grouped));
-        one.sk_part_bytes = lay.sk_part;
-      }
-      const aqlm_status st = launch_matmul(one, AQLM_PATH_AUTO, s);
+      const aqlm_status st = launch_matmul(p, AQLM_PATH_AUTO, s);
       if (st != AQLM_OK) return st;
     }
   }
@@ -582,20 +549,10 @@ size_t aqlm_static_group_scratch_bytes(void) { return AQLM_STATIC_GROUP_SCRATCH_
 aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aqlm_stream_t stream) {
   if (count == 0) return AQLM_OK;
   if (count < 0 || !problems) return AQLM_ERR_INVALID_ARG;
-  bool shapes_ok = true;
-  for (int i = 0; i < count; ++i) {
-    const aqlm_problem& q = problems[i];
-    shapes_ok = shapes_ok && validate_shape(q.M, q.B, q.g, q.K, q.N, q.batch) == AQLM_OK;
-  }
-  // the grouped partial sums must fit; the stream-K slots of the others are used when
-  // they fit too (the buffer starts zero-filled and every call leaves its counters zero)
-  GroupLayout lay;
-  if (shapes_ok) lay = group_layout(problems, count);
-  const size_t need = lay.required();
+  const size_t need = aqlm_group_workspace_size(problems, count);
   if (need > AQLM_STATIC_GROUP_SCRATCH_BYTES) return AQLM_ERR_INVALID_ARG;
-  const bool use_sk = lay.sk_part > 0 && lay.full() <= AQLM_STATIC_GROUP_SCRATCH_BYTES;
   void* scratch = nullptr;
-  if (need > 0 || use_sk) {
+  if (need > 0) {
     // validate before touching the device, as every entry point does
     for (int i = 0; i < count; ++i) {
       const aqlm_problem& q = problems[i];

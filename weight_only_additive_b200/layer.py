@@ -192,8 +192,8 @@ class LayerGroup:
         self.problems = native.problem_array(probs)
         self.count = len(probs)
         self.workspace_bytes = native.aqlm_group_workspace_size(self.problems, self.count)
-        # 256-byte aligned: torch's caching allocator hands out 512-byte aligned blocks
-        # zero-filled once: the stream-K part keeps counters that every call leaves zero
+        # 256-byte aligned: torch's caching allocator hands out 512-byte aligned blocks;
+        # zero-filled once, so the buffer could also serve aqlm_matmul_ws calls
         self.workspace = torch.zeros((max(self.workspace_bytes, 1),), dtype=torch.uint8, device=dev)
 
     def run(self, stream: Optional[torch.cuda.Stream] = None):
