@@ -381,3 +381,17 @@ def test_workspace_validation_needs_no_gpu(lib):
     assert L_.aqlm_input_grad_ws(*gargs[:-1], Schedule.STREAMK, None, 0, None) == Status.INVALID_ARG
     g16 = gargs[:5] + (1, 16, 8, 4096, 4096, 1024, Schedule.STREAMK)  # B = 16 gradient: no stream-K
     assert L_.aqlm_input_grad_ws(*g16, W, 1 << 24, None) == Status.UNSUPPORTED
+
+
+def _header_enum(prefix):
+    """{NAME: value} of the enumerators of include/aqlm.h whose names start with prefix."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    return {m.group(1)[len(prefix):]: int(m.group(2))
+            for m in re.finditer(r"\b(" + prefix + r"[A-Z_]+)\s*=\s*(\d+)", text)}
+
+
+def test_binding_enums_agree_with_the_header():
+    """The ctypes enums carry the header's values (status codes, paths, schedules)."""
+    assert _header_enum("AQLM_ERR_") == {s.name: int(s) for s in Status if s.name != "OK"}
+    assert _header_enum("AQLM_PATH_") == {p.name: int(p) for p in Path}
+    assert _header_enum("AQLM_SCHEDULE_") == {s.name: int(s) for s in Schedule}
