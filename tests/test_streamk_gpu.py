@@ -205,3 +205,28 @@ def test_streamk_input_grad_matches_oracle(dev, M, B, g, K, N, batch, cut):
 def test_device_status_clean_after_streamk(dev):
     st, detail = L.check_device_status()
     assert st == Status.OK, hex(detail)
+
+
+def test_per_stream_workspaces_are_kept_apart_and_bounded(dev):
+    """layer.matmul's default workspace is one per (device, stream): calls on 20
+    streams at once (a layer whose call needs a workspace: the grouped-kernel route)
+    give one result bit for bit, meet the oracle, and the cache keeps at most 16."""
+    M, B, g, K, N = 2, 8, 8, 11008, 4096
+    assert native.aqlm_matmul_workspace_size(M, B, g, K, N, 1) > 0
+    ld = synth.make_layer(M, B, g, K, N, seed=170)
+    x = synth.make_x(1, K, seed=171)
+    w = L.AqlmWeights.from_numpy(ld, dev)
+    xt = torch.from_numpy(x).to(dev)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(dev) for _ in range(20)]
+    outs = [L.matmul(xt, w, stream=s) for s in streams]
+    torch.cuda.synchronize()
+    st, detail = L.check_device_status()
+    assert st == Status.OK, hex(detail)
+    first = outs[0].cpu().numpy()
+    for y in outs[1:]:
+        assert np.array_equal(y.cpu().numpy().view(np.uint16), first.view(np.uint16))
+    rows = np.array([0, 1, 127, 128, 2047, N - 1])
+    ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, None, M, B, g, rows=rows)
+    assert rel_err(first[:, rows], ref) <= TOL
+    assert len(L._workspaces) <= 16

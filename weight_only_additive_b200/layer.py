@@ -4,6 +4,7 @@ arithmetic happens in the library's kernels.
 """
 from __future__ import annotations
 
+from collections import OrderedDict
 from dataclasses import dataclass
 from typing import Optional
 
@@ -23,10 +24,12 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
-# Workspaces of the tensor-core kernel's stream-K schedule, one per (device, stream):
-# calls on one stream may share one (the library leaves its counters zero), calls on
-# different streams must not.
-_workspaces: dict = {}
+# Workspaces of aqlm_matmul_ws / aqlm_input_grad_ws, one per (device, stream): calls on
+# one stream may share one (the library leaves its counters zero), calls on different
+# streams must not.  The 16 most recently used are kept; a dropped one was allocated on
+# its own stream, so the caching allocator reuses its memory only in that stream's order.
+_workspaces: "OrderedDict" = OrderedDict()
+_MAX_WORKSPACES = 16
 
 
 def stream_workspace(nbytes: int, device, stream: Optional[torch.cuda.Stream] = None) -> Optional[torch.Tensor]:
@@ -43,6 +46,9 @@ def stream_workspace(nbytes: int, device, stream: Optional[torch.cuda.Stream] = 
         with torch.cuda.stream(s):
             ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
         _workspaces[key] = ws
+    _workspaces.move_to_end(key)
+    while len(_workspaces) > _MAX_WORKSPACES:
+        _workspaces.popitem(last=False)
     return ws
 
 
