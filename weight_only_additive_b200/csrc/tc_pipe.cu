@@ -10,7 +10,8 @@
 // whole batch tile, the same kernel also serves token generation (batch 1..8):
 // its decoders gather codewords faster than the GEMV's lanes do.
 //
-// Warp roles (352 threads):
+// Warp roles (352 threads with one decoder group; a second group of 8 decoder warps
+// takes every other stage in the 608-thread kernels):
 //   warps 0-7  decoders, then epilogue.  Threads r and r + 128 own weight row
 //              n0 + r (16-byte chunks 0-3 and 4-7 of each 64-wide K stage).  Per
 //              stage a thread reads its codes from the code tile and writes its
@@ -27,6 +28,9 @@
 // Split K: SK CTAs of a (1, 1, SK) cluster take consecutive K ranges of the same
 // weight rows and exchange fp32 partials through distributed shared memory.
 // Epilogue: tcgen05.ld of 16 columns at a time, y = s_n * D + bias_n -> fp16.
+// Stream-K (a separate instantiation, kStreamK): one CTA per SM over the (row tile,
+// batch tile, K stage) space, two TMEM accumulators, and four more warps that finish
+// each tile piece from fp32 partials in a caller workspace (see the epilogue).
 #include <cuda.h>
 
 #include <algorithm>
