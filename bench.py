@@ -372,6 +372,31 @@ def cpu_kernel_run(w, batch, seconds):
                       f"{elapsed:.1f} s"}
 
 
+def reference_config(a, w, batch, world):
+    """The `config` of the matching line of this library's arm (run_ours): the same
+    workload, batch, bytes per step, pool and launch description, so the two lines name
+    one configuration.  The pool size follows Pool's rule from the device's L2 size."""
+    copy_bytes = step_bytes(w, batch)
+    l2 = L2_FALLBACK
+    try:
+        import torch
+        if torch.cuda.is_available():
+            l2 = getattr(torch.cuda.get_device_properties(0), "L2_cache_size", 0) or L2_FALLBACK
+    except Exception:  # no usable device: the fallback size
+        pass
+    pool = max(8, math.ceil(3 * l2 / copy_bytes)) if a.pool is None else max(1, a.pool)
+    while pool > 2 and pool * copy_bytes > 60e9:
+        pool -= 1
+    launch = ("one aqlm_matmul_group call per step (grouped lookup-table kernel + reduction)" if a.launch == "group"
+              else f"one aqlm_matmul_ws call per layer, schedule {a.schedule}")
+    return {"workload": w.name, "layers": len(w.layers), "batch": batch, "scheme": w.layers[0].scheme.name,
+            "algorithmic_bytes_per_step": copy_bytes,
+            "l2": f"inputs larger than L2: rotating pool of {pool} copies ({pool * copy_bytes / 1e6:.0f} MB > "
+                  f"{l2 / 1e6:.0f} MB L2)",
+            "launch": launch + f"; CUDA graphs of {pool} consecutive steps (one pass over the pool)",
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(a):
     rank, world, _ = env_rank()
     w = select_workload(a)
@@ -395,8 +420,7 @@ def run_reference(a):
             "warmup": a.warmup, "ms_per_step": tot_s * 1e3 / a.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": w.name, "layers": len(w.layers), "batch": batch,
-                       "scheme": w.layers[0].scheme.name, "parallelism": "replicas"},
+            "config": reference_config(a, w, batch, world),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
