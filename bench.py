@@ -362,8 +362,10 @@ def cpu_kernel_run(w, batch, seconds):
         elapsed += time.perf_counter() - t0
         passes += 1
     sbytes = step_bytes(w, batch)
-    method = ("lookup tables per 16-group K slice" if w.layers[0].scheme.B == 8 and batch <= 8
-              else "decode to fp32 + dot products")
+    level, B = cpu_lib.simd_level(), w.layers[0].scheme.B
+    lut = B == 8 and (batch == 1 if level == 2 else batch <= 8)
+    method = ("lookup tables per 16-group K slice" if lut
+              else "fused decode + dot in registers" if level == 2 else "decode to fp32 + dot products")
     return {"value": sbytes * passes / elapsed / 1e9, "unit": "GB/s",
             "ms_per_step": elapsed * 1e3 / passes, "cores": os.cpu_count(),
             "simd": cpu_lib.SIMD_NAMES.get(cpu_lib.simd_level(), "?"),

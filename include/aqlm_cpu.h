@@ -1,6 +1,6 @@
 /*
  * aqlm_cpu.h -- C ABI of libaqlm_cpu.so: the AQLM weight-only linear layer on the
- * host CPU (multithreaded, AVX2/FMA/F16C where the CPU has them).
+ * host CPU (multithreaded; AVX2/FMA/F16C and AVX-512 where the CPU has them).
  *
  * The AQLM repo summary ("Additive quantization that actually survives one-bit
  * weights", section "Key highlights") lists CPU inference among the format's
@@ -28,11 +28,16 @@
  * even).  Tolerance against the fp64 reference of the decoded fp16 weights:
  * max|y - y_ref| / max|y_ref| <= 5e-3.
  *
- * Methods: B = 8 and batch <= 8 use the lookup tables, built per K slice of 16
- * groups and read for every output row (threads take slices and keep per-thread
- * partial sums, added in thread order at the end); otherwise each thread decodes its
- * output rows to fp32 one at a time and takes dot products with every batch row.
- * The result is deterministic for a given nthreads and SIMD level.
+ * Methods: lookup tables, built per K slice of 16 groups and read for every output
+ * row (threads take slices and keep per-thread partial sums, added in thread order
+ * at the end); decode + dot, where each thread decodes its output rows to fp32 one at
+ * a time and takes dot products with every batch row; and, with AVX-512, fused decode
+ * + dot, where 16 weights at a time are decoded in registers and multiplied into
+ * accumulators of up to 8 batch rows, nothing decoded being stored.  At SIMD level 2
+ * B = 8 at batch 1 uses the lookup tables and everything else the fused method; at
+ * levels 0 and 1 B = 8 at batch <= 8 uses the lookup tables and everything else
+ * decode + dot.  The result is deterministic for a given nthreads and SIMD level (the
+ * fused method's does not depend on nthreads).
  *
  * nthreads: 0 = the OpenMP default, else that many threads.  The call allocates
  * host scratch (tables, partial sums; released before it returns).
@@ -57,11 +62,13 @@ aqlm_status aqlm_cpu_matmul(const void* x, const void* codes, const void* codebo
                             int M, int B, int g, int K, int N, int batch, int nthreads);
 
 /* SIMD level the kernels run with on this CPU: 0 = portable scalar code,
- * 1 = AVX2 + FMA + F16C.  At most the cap set below. */
+ * 1 = AVX2 + FMA + F16C, 2 = AVX-512 F, BW and VL as well.  At most the cap set
+ * below. */
 int aqlm_cpu_simd_level(void);
 
-/* Caps the SIMD level (clamped to 0..1) for every later call in the process, so
- * that the scalar code can be run and tested on an AVX2 CPU; the default cap is 1.
+/* Caps the SIMD level (clamped to 0..2) for every later call in the process, so
+ * that the lower levels can be run and tested on a CPU that has the higher ones; the
+ * default cap is 2.
  * Returns the previous cap.  Not meant to be changed while another thread is inside
  * aqlm_cpu_matmul. */
 int aqlm_cpu_set_max_simd_level(int level);

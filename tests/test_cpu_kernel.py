@@ -3,10 +3,10 @@
 The same bar as the GPU path: max|y - y_ref| / max|y_ref| <= 5e-3 against the
 oracle's fp64 reference of the decoded fp16 weights, no NaN/Inf, for every
 supported scheme on both methods (lookup tables for B = 8 at batch <= 8, decode +
-dot otherwise); integer-valued layers bit for bit; the same bits run to run for a
-given thread count; argument errors before any work.  The numeric tests run at every
-SIMD level this CPU has (scalar, AVX2), selected with the library's process-wide
-cap.  No GPU is involved.
+dot otherwise, and the fused decode + dot with AVX-512); integer-valued layers bit
+for bit; the same bits run to run for a given thread count; argument errors before any
+work.  The numeric tests run at every SIMD level this CPU has (scalar, AVX2, AVX-512),
+selected with the library's process-wide cap.  No GPU is involved.
 """
 import ctypes
 import os
@@ -31,7 +31,7 @@ def built():
     cpu.lib()
 
 
-@pytest.fixture(params=[0, 1], ids=["scalar", "avx2"])
+@pytest.fixture(params=[0, 1, 2], ids=["scalar", "avx2", "avx512"])
 def simd(request):
     """Runs the test with the SIMD level capped at the parameter (skipped where the CPU
     lacks it); the previous cap is restored afterwards."""
@@ -56,7 +56,7 @@ def test_header_declares_the_binding_exports():
     assert declared == sorted(cpu.EXPORTS)
     for name in cpu.EXPORTS:
         assert isinstance(getattr(cpu.lib(), name), ctypes._CFuncPtr)
-    assert cpu.simd_level() in (0, 1)
+    assert cpu.simd_level() in (0, 1, 2)
 
 
 @pytest.mark.parametrize("M,B,g", SCHEMES)
@@ -86,6 +86,35 @@ def test_cpu_matmul_integer_layers_bit_exact(M, B, g, batch, simd):
     for nt in (1, 3):
         y = cpu.matmul(x, codes, cb, sc, bias, M, B, g, nthreads=nt).astype(np.float64)
         assert np.array_equal(y, ref), (nt, int((y != ref).sum()))
+
+
+@pytest.mark.parametrize("M,B,g", [(2, 8, 8), (3, 8, 8), (1, 16, 8), (2, 16, 8)])
+@pytest.mark.parametrize("batch", [1, 2, 5, 17])
+def test_cpu_matmul_odd_group_count_and_batch_chunks(M, B, g, batch, simd):
+    """K = 8 * 75 (an odd number of g = 8 groups: the last group has no partner in a
+    16-weight step), N = 101 (no multiple of any row block), and batches that leave a
+    partial chunk of 8."""
+    N, K = 101, 8 * 75
+    ld = synth.make_layer(M, B, g, K, N, seed=86, layer=batch, with_bias=True)
+    x = synth.make_x(batch, K, seed=87, layer=M)
+    ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+    for nt in (1, 5):
+        close(cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g, nthreads=nt), ref,
+              f"{M}x{B} g{g} b={batch} threads={nt} simd={simd}")
+
+
+def test_cpu_fused_method_independent_of_thread_count():
+    """At SIMD level 2 everything but B = 8 at batch 1 takes the fused decode + dot,
+    where each output row is summed by one thread in one order: any thread count gives
+    the same bits."""
+    if cpu.simd_level() < 2:
+        pytest.skip("this CPU has no AVX-512")
+    for M, B, g, batch in ((2, 8, 8, 4), (1, 16, 8, 1), (2, 16, 16, 9)):
+        ld = synth.make_layer(M, B, g, 1024, 300, seed=88)
+        x = synth.make_x(batch, 1024, seed=88)
+        ys = [cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, None, M, B, g, nthreads=nt).view(np.uint16)
+              for nt in (1, 2, 7)]
+        assert all(np.array_equal(ys[0], y) for y in ys[1:]), (M, B, g, batch)
 
 
 def test_cpu_matmul_full_size_layer_sampled_rows(simd):

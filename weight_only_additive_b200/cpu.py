@@ -23,7 +23,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIBRARY = os.path.join(PKG, "libaqlm_cpu.so")
 
 EXPORTS = ("aqlm_cpu_matmul", "aqlm_cpu_simd_level", "aqlm_cpu_set_max_simd_level", "aqlm_cpu_abi_version")
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 _lib = None
 _lock = threading.Lock()
@@ -52,7 +52,7 @@ def lib() -> ctypes.CDLL:
 
 
 def simd_level() -> int:
-    """0 = scalar, 1 = AVX2 + FMA + F16C."""
+    """0 = scalar, 1 = AVX2 + FMA + F16C, 2 = AVX-512 (F, BW, VL) as well."""
     return lib().aqlm_cpu_simd_level()
 
 
@@ -62,7 +62,7 @@ def set_max_simd_level(level: int) -> int:
     return lib().aqlm_cpu_set_max_simd_level(int(level))
 
 
-SIMD_NAMES = {0: "scalar", 1: "avx2+fma+f16c"}
+SIMD_NAMES = {0: "scalar", 1: "avx2+fma+f16c", 2: "avx512f+bw+vl"}
 
 
 def _arr(a, dtype):

@@ -3,23 +3,31 @@
 //
 //   y = x . W^T . diag(s) + bias,   W[n, j*g + t] = sum_m C_m[codes[n, j, m]][t]
 //
-// Two methods:
-//   * lookup tables (B = 8, batch <= 8): the route of the inference-research record
-//     "AQLM (additive / multi-codebook quantization)", section "Kernels".  For a K
-//     slice of kSlice groups, T[j][m][b][i] = x_b[j] . C_m[i] for all 256 entries i
-//     (g fused multiply-adds per 8 entries with AVX2); then every output row adds M
-//     table values per group.  Threads take slices (static schedule) and keep a
-//     partial sum per output; the partials are added in thread order at the end, so
-//     the table is built once per slice whatever N is.
-//   * decode + dot (B = 16, or batch > 8): each thread decodes blocks of 4 output rows
-//     to fp32 (codeword pieces converted with F16C and added in codebook order) and
-//     takes the dot products with every batch row (AVX2 FMA, 4 accumulators).
+// Three methods:
+//   * lookup tables (B = 8): the route of the inference-research record "AQLM
+//     (additive / multi-codebook quantization)", section "Kernels".  For a K slice of
+//     kSlice groups, T[j][m][b][i] = x_b[j] . C_m[i] for all 256 entries i (g fused
+//     multiply-adds per 8 or 16 entries); then every output row adds M table values
+//     per group (16 of them per gather instruction with AVX-512).  Threads take
+//     slices (static schedule) and keep a partial sum per output; the partials are
+//     added in thread order at the end, so the table is built once per slice
+//     whatever N is.
+//   * decode + dot: each thread decodes blocks of 4 output rows to fp32 (codeword
+//     pieces converted with F16C and added in codebook order) and takes the dot
+//     products with every batch row (AVX2 FMA, 4 accumulators).
+//   * fused decode + dot (AVX-512): 16 weights of a row are decoded in a register and
+//     multiplied into register accumulators for up to 8 batch rows and 2 to 8 output
+//     rows at once; nothing decoded is stored.
+// Which runs: with AVX-512, the lookup tables for B = 8 at batch 1 and the fused
+// method otherwise; without it, the lookup tables for B = 8 at batch <= 8 and decode
+// + dot otherwise.  (On a Xeon host with AVX-512 the lookups' gathers beat the fused
+// decode only at batch 1, where a table entry serves one product.)
 // fp32 accumulation everywhere; y = fp16_rne(s_n * acc + bias_n).
 //
-// The AVX2 functions carry target attributes and run only when the CPU reports
-// AVX2, FMA and F16C; otherwise portable scalar versions of the same loops run.  A
-// process-wide cap (aqlm_cpu_set_max_simd_level) selects the scalar code on such a
-// CPU too, for tests and comparisons.
+// The SIMD functions carry target attributes and run only when the CPU reports the
+// instruction sets they use; otherwise portable scalar versions of the lookup and
+// decode + dot loops run.  A process-wide cap (aqlm_cpu_set_max_simd_level) selects
+// a lower level on such a CPU too, for tests and comparisons.
 #include <immintrin.h>
 #include <omp.h>
 
@@ -27,6 +35,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 #include <vector>
 
 #include "aqlm_cpu.h"
@@ -36,6 +45,7 @@ namespace {
 constexpr int kSlice = 16;     // groups per lookup-table slice (tables of 16 KB per codebook fit L1)
 constexpr int kLutMaxBatch = 8;
 constexpr int kRowBlock = 4;    // rows decoded together in the decode + dot method
+constexpr int kPrefetchRows = 32;  // lookup rows: codes requested this many rows ahead
 
 // ---------------------------------------------------------------------------
 // binary16 <-> binary32 for the scalar code (IEEE 754: 1 sign, 5 exponent bits
@@ -95,12 +105,19 @@ bool cpu_has_avx2() {
   return ok;
 }
 
-std::atomic<int> g_max_simd{1};
+bool cpu_has_avx512() {
+  static const bool ok = cpu_has_avx2() && __builtin_cpu_supports("avx512f") &&
+                         __builtin_cpu_supports("avx512bw") && __builtin_cpu_supports("avx512vl");
+  return ok;
+}
 
-// 0 = scalar, 1 = AVX2 + FMA + F16C: what the CPU has, capped by
-// aqlm_cpu_set_max_simd_level.
+constexpr int kMaxSimd = 2;
+std::atomic<int> g_max_simd{kMaxSimd};
+
+// 0 = scalar, 1 = AVX2 + FMA + F16C, 2 = AVX-512 (F, BW, VL) as well: what the CPU
+// has, capped by aqlm_cpu_set_max_simd_level.
 int simd_level() {
-  const int hw = cpu_has_avx2() ? 1 : 0;
+  const int hw = cpu_has_avx512() ? 2 : cpu_has_avx2() ? 1 : 0;
   return std::min(hw, g_max_simd.load());
 }
 
@@ -173,8 +190,14 @@ template <int MM>
 void lookup_rows(const Layer& L, const float* T, int j0, int nj, float* partial) {
   const int M = MM > 0 ? MM : L.M;
   const int stride = M * nj;  // code bytes of the slice in a row
+  const int64_t row_bytes = static_cast<int64_t>(L.G) * M;
   for (int64_t n = 0; n < L.N; ++n) {
     const uint8_t* c = L.codes + (n * L.G + j0) * M;
+    if (n + kPrefetchRows < L.N) {  // the slice's codes kPrefetchRows rows ahead
+      const char* ahead = reinterpret_cast<const char*>(c + kPrefetchRows * row_bytes);
+      __builtin_prefetch(ahead);
+      __builtin_prefetch(ahead + stride - 1);
+    }
     for (int b = 0; b < L.batch; ++b) {
       const float* Tb = T + static_cast<size_t>(b) * 256;
       const size_t step = static_cast<size_t>(L.batch) * 256;  // next (group, codebook) table
@@ -189,6 +212,76 @@ void lookup_rows(const Layer& L, const float* T, int j0, int nj, float* partial)
       for (; k < stride; ++k) a0 += Tb[k * step + c[k]];
       partial[static_cast<size_t>(b) * L.N + n] += (a0 + a1) + (a2 + a3);
     }
+  }
+}
+
+// The same tables built 16 entries per instruction; per entry the same fused
+// multiply-adds in the same order as build_tables_avx2, so the values agree.
+__attribute__((target("avx512f,avx512bw,avx512vl,avx2,fma,f16c")))
+void build_tables_avx512(const Layer& L, const float* xf, const float* ct, int j0, int nj, float* T) {
+  for (int jj = 0; jj < nj; ++jj)
+    for (int m = 0; m < L.M; ++m)
+      for (int b = 0; b < L.batch; ++b) {
+        float* row = T + (static_cast<size_t>(jj * L.M + m) * L.batch + b) * 256;
+        const float* xv = xf + static_cast<size_t>(b) * L.K + static_cast<size_t>(j0 + jj) * L.g;
+        const float* cm = ct + static_cast<size_t>(m) * L.g * 256;
+        for (int i = 0; i < 256; i += 32) {
+          __m512 a0 = _mm512_setzero_ps(), a1 = _mm512_setzero_ps();
+          for (int t = 0; t < L.g; ++t) {
+            const __m512 xt = _mm512_set1_ps(xv[t]);
+            a0 = _mm512_fmadd_ps(xt, _mm512_loadu_ps(cm + t * 256 + i), a0);
+            a1 = _mm512_fmadd_ps(xt, _mm512_loadu_ps(cm + t * 256 + i + 16), a1);
+          }
+          _mm512_storeu_ps(row + i, a0);
+          _mm512_storeu_ps(row + i + 16, a1);
+        }
+      }
+}
+
+// lookup_rows with 16 table reads per gather instruction.  A row's codes of the
+// slice are M * nj consecutive bytes (at most 64, NV vectors of 16); lane l of vector
+// v reads table (16 v + l) at the entry its code names, so the index is
+// (16 v + l) * batch * 256 + code and the base pointer selects the batch row.
+template <int NV>
+__attribute__((target("avx512f,avx512bw,avx512vl,avx2,fma,f16c")))
+void lookup_rows_avx512(const Layer& L, const float* T, int j0, int nj, float* partial) {
+  const int stride = L.M * nj;
+  const int step = L.batch * 256;
+  const __m512i lane = _mm512_set_epi32(15, 14, 13, 12, 11, 10, 9, 8, 7, 6, 5, 4, 3, 2, 1, 0);
+  __m512i off[NV];
+  __mmask16 msk[NV];
+  for (int v = 0; v < NV; ++v) {
+    const int rem = stride - 16 * v;
+    msk[v] = static_cast<__mmask16>(rem >= 16 ? 0xFFFFu : (1u << rem) - 1u);
+    off[v] = _mm512_mullo_epi32(_mm512_add_epi32(lane, _mm512_set1_epi32(16 * v)), _mm512_set1_epi32(step));
+  }
+  const int64_t row_bytes = static_cast<int64_t>(L.G) * L.M;
+  for (int64_t n = 0; n < L.N; ++n) {
+    const uint8_t* c = L.codes + (n * L.G + j0) * L.M;
+    if (n + kPrefetchRows < L.N) {  // the slice's codes kPrefetchRows rows ahead
+      const char* ahead = reinterpret_cast<const char*>(c + kPrefetchRows * row_bytes);
+      _mm_prefetch(ahead, _MM_HINT_T0);
+      _mm_prefetch(ahead + stride - 1, _MM_HINT_T0);
+    }
+    __m512i idx[NV];
+    for (int v = 0; v < NV; ++v)
+      idx[v] = _mm512_add_epi32(_mm512_cvtepu8_epi32(_mm_maskz_loadu_epi8(msk[v], c + 16 * v)), off[v]);
+    for (int b = 0; b < L.batch; ++b) {
+      const float* Tb = T + static_cast<size_t>(b) * 256;
+      __m512 acc = _mm512_mask_i32gather_ps(_mm512_setzero_ps(), msk[0], idx[0], Tb, 4);
+      for (int v = 1; v < NV; ++v)
+        acc = _mm512_add_ps(acc, _mm512_mask_i32gather_ps(_mm512_setzero_ps(), msk[v], idx[v], Tb, 4));
+      partial[static_cast<size_t>(b) * L.N + n] += _mm512_reduce_add_ps(acc);
+    }
+  }
+}
+
+void lookup_rows_level2(const Layer& L, const float* T, int j0, int nj, float* partial) {
+  switch ((L.M * nj + 15) / 16) {
+    case 1: lookup_rows_avx512<1>(L, T, j0, nj, partial); break;
+    case 2: lookup_rows_avx512<2>(L, T, j0, nj, partial); break;
+    case 3: lookup_rows_avx512<3>(L, T, j0, nj, partial); break;
+    default: lookup_rows_avx512<4>(L, T, j0, nj, partial); break;
   }
 }
 
@@ -208,6 +301,11 @@ void run_lut(const Layer& L, const float* xf, int nt) {
     for (int s = 0; s < S; ++s) {
       if (part.empty()) part.assign(static_cast<size_t>(L.batch) * L.N, 0.f);
       const int j0 = s * kSlice, nj = std::min(kSlice, L.G - j0);
+      if (level == 2) {
+        build_tables_avx512(L, xf, ct.data(), j0, nj, T.data());
+        lookup_rows_level2(L, T.data(), j0, nj, part.data());
+        continue;
+      }
       if (level == 1)
         build_tables_avx2(L, xf, ct.data(), j0, nj, T.data());
       else
@@ -319,6 +417,158 @@ void run_decode_dot(const Layer& L, const float* xf, int nt) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// fused decode + dot (AVX-512): 16 weights of a row are decoded in a register and
+// multiplied into per-(row, batch row) accumulators at once, so no decoded row is
+// stored.  B = 8 codebooks are read from an fp32 copy ([M][256][g], 8 KB per codebook
+// at g = 8, so L1-resident); B = 16 codebooks stay fp16 and are converted as they are
+// read.  Per weight the pieces are added in codebook order in fp32 (as the decode
+// defines), the products accumulate in fp32 lanes, and the lanes are added at the end
+// of the row; every row is computed by one thread in one fixed order, so the result
+// does not depend on the thread count.
+// ---------------------------------------------------------------------------
+// rows per block for BB batch rows: R * BB accumulators (at most 16 of the 32 zmm)
+template <int BB>
+constexpr int fused_rows() { return BB <= 2 ? 8 : BB <= 4 ? 4 : BB == 5 ? 3 : 2; }
+
+// 16 decoded weights of one row from its codes at groups j (and j + 1 when g = 8):
+// cr points at the row's codes of group j, cb at the codebooks (fp32 for B = 8, fp16
+// for B = 16).  `two` = false decodes only group j (g = 8, last group of an odd G),
+// leaving the upper 8 lanes zero.
+template <int MM, int GG, bool kF32>
+__attribute__((target("avx512f,avx512bw,avx512vl,avx2,fma,f16c"), always_inline))
+inline __m512 decode16(const void* cr, const void* cb, int M, int g, bool two) {
+  const int nm = MM > 0 ? MM : M;
+  const int gg = GG > 0 ? GG : g;
+  __m512 w = _mm512_setzero_ps();
+  for (int m = 0; m < nm; ++m) {
+    __m512 piece;
+    if constexpr (kF32) {
+      const uint8_t* c = static_cast<const uint8_t*>(cr);
+      const float* cm = static_cast<const float*>(cb) + static_cast<size_t>(m) * 256 * gg;
+      if (gg == 16) {
+        piece = _mm512_loadu_ps(cm + static_cast<size_t>(c[m]) * 16);
+      } else {
+        const __m256 lo = _mm256_loadu_ps(cm + static_cast<size_t>(c[m]) * 8);
+        const __m256 hi = two ? _mm256_loadu_ps(cm + static_cast<size_t>(c[nm + m]) * 8) : _mm256_setzero_ps();
+        piece = _mm512_castpd_ps(_mm512_insertf64x4(_mm512_castps_pd(_mm512_castps256_ps512(lo)),
+                                                    _mm256_castps_pd(hi), 1));
+      }
+    } else {
+      const uint16_t* c = static_cast<const uint16_t*>(cr);
+      const uint16_t* cm = static_cast<const uint16_t*>(cb) + (static_cast<size_t>(m) << 16) * gg;
+      if (gg == 16) {
+        piece = _mm512_cvtph_ps(_mm256_loadu_si256(reinterpret_cast<const __m256i*>(cm + static_cast<size_t>(c[m]) * 16)));
+      } else {
+        const __m128i lo = _mm_loadu_si128(reinterpret_cast<const __m128i*>(cm + static_cast<size_t>(c[m]) * 8));
+        const __m128i hi = two ? _mm_loadu_si128(reinterpret_cast<const __m128i*>(cm + static_cast<size_t>(c[nm + m]) * 8))
+                               : _mm_setzero_si128();
+        piece = _mm512_cvtph_ps(_mm256_inserti128_si256(_mm256_castsi128_si256(lo), hi, 1));
+      }
+    }
+    w = m == 0 ? piece : _mm512_add_ps(w, piece);
+  }
+  return w;
+}
+
+// y[b0 .. b0 + BB) x rows [n0, n0 + R) (rows past N repeat row N - 1 and are not stored).
+template <int MM, int GG, bool kF32, int BB>
+__attribute__((target("avx512f,avx512bw,avx512vl,avx2,fma,f16c")))
+void fused_block_avx512(const Layer& L, const float* xf, const void* cb, int64_t n0, int b0) {
+  constexpr int R = fused_rows<BB>();
+  const int M = MM > 0 ? MM : L.M, g = GG > 0 ? GG : L.g;
+  const int cbytes = kF32 ? 1 : 2;
+  const int64_t rowc = static_cast<int64_t>(L.G) * M;  // codes per row
+  const uint8_t* crow[R];
+  for (int r = 0; r < R; ++r)
+    crow[r] = L.codes + std::min<int64_t>(n0 + r, L.N - 1) * rowc * cbytes;
+  const float* xb = xf + static_cast<size_t>(b0) * L.K;
+  __m512 acc[R][BB];
+  for (int r = 0; r < R; ++r)
+    for (int b = 0; b < BB; ++b) acc[r][b] = _mm512_setzero_ps();
+  const int K16 = L.K & ~15;
+  for (int k = 0; k < K16; k += 16) {
+    __m512 xk[BB];
+    for (int b = 0; b < BB; ++b) xk[b] = _mm512_loadu_ps(xb + static_cast<size_t>(b) * L.K + k);
+    const int64_t coff = static_cast<int64_t>(k / g) * M * cbytes;
+    for (int r = 0; r < R; ++r) {
+      const __m512 w = decode16<MM, GG, kF32>(crow[r] + coff, cb, M, g, true);
+      for (int b = 0; b < BB; ++b) acc[r][b] = _mm512_fmadd_ps(w, xk[b], acc[r][b]);
+    }
+  }
+  if (K16 < L.K) {  // g = 8 and G odd: the last group alone
+    __m512 xk[BB];
+    for (int b = 0; b < BB; ++b) xk[b] = _mm512_maskz_loadu_ps(0x00FF, xb + static_cast<size_t>(b) * L.K + K16);
+    const int64_t coff = static_cast<int64_t>(K16 / g) * M * cbytes;
+    for (int r = 0; r < R; ++r) {
+      const __m512 w = decode16<MM, GG, kF32>(crow[r] + coff, cb, M, g, false);
+      for (int b = 0; b < BB; ++b) acc[r][b] = _mm512_fmadd_ps(w, xk[b], acc[r][b]);
+    }
+  }
+  for (int r = 0; r < R; ++r) {
+    const int64_t n = n0 + r;
+    if (n >= L.N) break;
+    const float sc = half_to_float(L.scales[n]);
+    const float bi = L.bias ? half_to_float(L.bias[n]) : 0.f;
+    for (int b = 0; b < BB; ++b)
+      L.y[static_cast<size_t>(b0 + b) * L.N + n] = float_to_half(_mm512_reduce_add_ps(acc[r][b]) * sc + bi);
+  }
+}
+
+template <int MM, int GG, bool kF32>
+void fused_rows_avx512(const Layer& L, const float* xf, const void* cb, int64_t n0, int rows_per_task) {
+  // one task: rows [n0, n0 + rows_per_task) for every batch row, in chunks of 8
+  for (int b0 = 0; b0 < L.batch; b0 += 8) {
+    const int bb = std::min(8, L.batch - b0);
+    auto run = [&](auto tag) {
+      constexpr int BBc = decltype(tag)::value;
+      constexpr int R = fused_rows<BBc>();
+      for (int64_t n = n0; n < std::min<int64_t>(n0 + rows_per_task, L.N); n += R)
+        fused_block_avx512<MM, GG, kF32, BBc>(L, xf, cb, n, b0);
+    };
+    switch (bb) {
+      case 1: run(std::integral_constant<int, 1>()); break;
+      case 2: run(std::integral_constant<int, 2>()); break;
+      case 3: run(std::integral_constant<int, 3>()); break;
+      case 4: run(std::integral_constant<int, 4>()); break;
+      case 5: run(std::integral_constant<int, 5>()); break;
+      case 6: run(std::integral_constant<int, 6>()); break;
+      case 7: run(std::integral_constant<int, 7>()); break;
+      default: run(std::integral_constant<int, 8>()); break;
+    }
+  }
+}
+
+// rows per task: a multiple of every fused_rows value (8, 4, 3, 2)
+constexpr int kFusedTaskRows = 48;
+
+void run_fused(const Layer& L, const float* xf, int nt) {
+  std::vector<float> cbf;
+  const void* cb = L.cb;
+  if (L.B == 8) {  // fp32 copy, [M][256][g] as stored
+    cbf.resize(static_cast<size_t>(L.M) * 256 * L.g);
+    for (size_t i = 0; i < cbf.size(); ++i) cbf[i] = half_to_float(L.cb[i]);
+    cb = cbf.data();
+  }
+  using Fn = void (*)(const Layer&, const float*, const void*, int64_t, int);
+  Fn fn;
+  if (L.B == 8) {
+    static constexpr Fn g8[4] = {fused_rows_avx512<1, 8, true>, fused_rows_avx512<2, 8, true>,
+                                 fused_rows_avx512<3, 8, true>, fused_rows_avx512<4, 8, true>};
+    static constexpr Fn g16[4] = {fused_rows_avx512<1, 16, true>, fused_rows_avx512<2, 16, true>,
+                                  fused_rows_avx512<3, 16, true>, fused_rows_avx512<4, 16, true>};
+    fn = (L.g == 8 ? g8 : g16)[L.M - 1];
+  } else {
+    if (L.g == 8)
+      fn = L.M == 1 ? fused_rows_avx512<1, 8, false> : fused_rows_avx512<2, 8, false>;
+    else
+      fn = L.M == 1 ? fused_rows_avx512<1, 16, false> : fused_rows_avx512<2, 16, false>;
+  }
+  const int64_t tasks = (L.N + kFusedTaskRows - 1) / kFusedTaskRows;
+#pragma omp parallel for schedule(static) num_threads(nt)
+  for (int64_t t = 0; t < tasks; ++t) fn(L, xf, cb, t * kFusedTaskRows, kFusedTaskRows);
+}
+
 bool scheme_ok(int M, int B, int g) {
   if (g != 8 && g != 16) return false;
   if (B == 8) return M >= 1 && M <= 4;
@@ -335,12 +585,12 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 extern "C" {
 
-int aqlm_cpu_abi_version(void) { return 2; }
+int aqlm_cpu_abi_version(void) { return 3; }
 
 int aqlm_cpu_simd_level(void) { return simd_level(); }
 
 int aqlm_cpu_set_max_simd_level(int level) {
-  return g_max_simd.exchange(std::max(0, std::min(1, level)));
+  return g_max_simd.exchange(std::max(0, std::min(kMaxSimd, level)));
 }
 
 aqlm_status aqlm_cpu_matmul(const void* x, const void* codes, const void* codebooks,
@@ -368,7 +618,9 @@ aqlm_status aqlm_cpu_matmul(const void* x, const void* codes, const void* codebo
   const int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
   std::vector<float> xf(static_cast<size_t>(batch) * K);
   for (size_t i = 0; i < xf.size(); ++i) xf[i] = half_to_float(L.x[i]);
-  if (B == 8 && batch <= kLutMaxBatch)
+  if (simd_level() == 2 && !(B == 8 && batch == 1))
+    run_fused(L, xf.data(), nt);
+  else if (B == 8 && batch <= kLutMaxBatch)
     run_lut(L, xf.data(), nt);
   else
     run_decode_dot(L, xf.data(), nt);
