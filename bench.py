@@ -374,39 +374,66 @@ def cpu_kernel_run(w, batch, seconds):
                       f"{elapsed:.1f} s"}
 
 
-def reference_config(a, w, batch, world):
-    """The `config` of the matching line of this library's arm (run_ours): the same
-    workload, batch, bytes per step, pool and launch description, so the two lines name
-    one configuration.  The pool size follows Pool's rule from the device's L2 size."""
-    copy_bytes = step_bytes(w, batch)
-    l2 = L2_FALLBACK
-    try:
-        import torch
-        if torch.cuda.is_available():
-            l2 = getattr(torch.cuda.get_device_properties(0), "L2_cache_size", 0) or L2_FALLBACK
-    except Exception:  # no usable device: the fallback size
-        pass
-    pool = max(8, math.ceil(3 * l2 / copy_bytes)) if a.pool is None else max(1, a.pool)
+def pool_copies(copy_bytes, l2, copies=None):
+    """How many seeded copies of a workload's layers the timing pool holds: at least 3x
+    L2 so no step finds its weights in L2, and at least 8 copies so a CUDA graph holds
+    8 steps (consecutive launches overlap through programmatic dependent launch inside a
+    graph, not across graph launches); at most 60 GB.  `copies` overrides the rule."""
+    pool = max(8, math.ceil(3 * l2 / copy_bytes)) if copies is None else max(1, copies)
     while pool > 2 and pool * copy_bytes > 60e9:
         pool -= 1
-    launch = ("one aqlm_matmul_group call per step (grouped lookup-table kernel + reduction)" if a.launch == "group"
-              else f"one aqlm_matmul_ws call per layer, schedule {a.schedule}")
+    return pool
+
+
+def line_config(w, batch, world, launch, schedule, pool, l2):
+    """The `config` object of a bench line: the workload, batch, bytes per step, the
+    pool that keeps inputs out of L2 and the launch form.  Both arms print it, so the
+    two lines name one configuration."""
+    copy_bytes = step_bytes(w, batch)
+    desc = ("one aqlm_matmul_group call per step (grouped lookup-table kernel + reduction)" if launch == "group"
+            else f"one aqlm_matmul_ws call per layer, schedule {schedule}")
     return {"workload": w.name, "layers": len(w.layers), "batch": batch, "scheme": w.layers[0].scheme.name,
             "algorithmic_bytes_per_step": copy_bytes,
             "l2": f"inputs larger than L2: rotating pool of {pool} copies ({pool * copy_bytes / 1e6:.0f} MB > "
                   f"{l2 / 1e6:.0f} MB L2)",
-            "launch": launch + f"; CUDA graphs of {pool} consecutive steps (one pass over the pool)",
+            "launch": desc + f"; CUDA graphs of {pool} consecutive steps (one pass over the pool)",
             "parallelism": f"replicas x{world}"}
+
+
+def device_l2_bytes():
+    """L2 size of device 0, or the fallback size without a usable GPU."""
+    try:
+        import torch
+        if torch.cuda.is_available():
+            return getattr(torch.cuda.get_device_properties(0), "L2_cache_size", 0) or L2_FALLBACK
+    except Exception:  # no usable device: the fallback size
+        pass
+    return L2_FALLBACK
+
+
+def reference_config(a, w, batch, world):
+    """The `config` of the matching line of this library's arm (run_ours or
+    run_input_grad), with the pool sized by the same rule from the device's L2 size."""
+    l2 = device_l2_bytes()
+    if a.op == "input-grad":
+        return grad_line_config(w, batch, world, a.schedule, grad_pool_copies(grad_step_bytes(w, batch), l2, a.pool),
+                                l2)
+    return line_config(w, batch, world, a.launch, a.schedule, pool_copies(step_bytes(w, batch), l2, a.pool), l2)
 
 
 def run_reference(a):
     rank, world, _ = env_rank()
     w = select_workload(a)
-    batch = workload_batch(w, a.batch)
+    if a.op == "input-grad":
+        batch = a.batch if a.batch is not None else GRAD_DEFAULT_BATCH
+    else:
+        batch = workload_batch(w, a.batch)
     if rank != 0:
         return 0
     # each step is a bounded sample sized so that warmup + steps fit ~2 minutes
     per_step = max(0.002, min(5.0, 120.0 / (a.steps + a.warmup)))
+    if a.op == "input-grad":
+        return run_reference_grad(a, w, batch, world, per_step)
     for i in range(a.warmup):
         oracle_sample_run(w, batch, per_step, copy=i)
     tot_b, tot_s = 0.0, 0.0
@@ -426,6 +453,31 @@ def run_reference(a):
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_grad(a, w, batch, world, per_step):
+    """The reference arm of `--op input-grad`: the oracle's input gradient on column
+    samples of every layer, per_step seconds of it per step (at least one layer)."""
+    for i in range(a.warmup):
+        oracle_grad_sample_run(w, batch, per_step, seed=100 + i)
+    tot_f, tot_s, cols, threads = 0.0, 0.0, 0, 1
+    for i in range(a.steps):
+        f, s, cols, threads = oracle_grad_sample_run(w, batch, per_step, seed=1000 + i)
+        tot_f += f
+        tot_s += s
+    value = tot_f / tot_s / 1e12
+    sample = (f"{cols} sampled columns of dx per layer and step (the oracle decodes the whole W16 each call, "
+              f"then fp64 dy . W16 for those columns), batch {batch}")
+    line = {"metric": GRAD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": tot_s * 1e3 / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": reference_config(a, w, batch, world),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -543,12 +595,7 @@ class Pool:
         torch, L = b.torch, b.L
         self.w, self.batch = w, batch
         copy_bytes = step_bytes(w, batch)
-        # at least 3x L2 so no step finds its weights in L2, and at least 8 copies so a
-        # CUDA graph holds 8 steps: consecutive launches overlap through programmatic
-        # dependent launch inside a graph, not across graph launches
-        pool = max(8, math.ceil(3 * b.l2 / copy_bytes)) if copies is None else max(1, copies)
-        while pool > 2 and pool * copy_bytes > 60e9:
-            pool -= 1
+        pool = pool_copies(copy_bytes, b.l2, copies)
         self.size, self.copy_bytes = pool, copy_bytes
         self.weights, self.xs = [], []
         off = w.extra.get("layer_offset", 0)
@@ -845,9 +892,7 @@ def run_ours(a):
         cpu["single_thread"] = {"value": b1 / s1 / 1e9, "unit": "GB/s", "cores": 1,
                                 "sample": f"{rows1} rows of each layer, {s1:.1f} s on one thread"}
         cpu_kernel = cpu_kernel_run(w, batch, min(a.cpu_seconds, 5.0))
-    pool_desc = (f"inputs larger than L2: rotating pool of {pool.size} copies "
-                 f"({pool.size * pool.copy_bytes / 1e6:.0f} MB > {b.l2 / 1e6:.0f} MB L2)")
-    pool_size = pool.size
+    config = line_config(w, batch, world, mode, a.schedule, pool.size, b.l2)
     del pool
     torch.cuda.empty_cache()
 
@@ -873,15 +918,7 @@ def run_ours(a):
                 "us_per_layer": ms_step * 1e3 / len(w.layers),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
                 "data": "synthetic",
-                "config": {"workload": w.name, "layers": len(w.layers), "batch": batch,
-                           "scheme": w.layers[0].scheme.name,
-                           "algorithmic_bytes_per_step": sbytes,
-                           "l2": pool_desc,
-                           "launch": ("one aqlm_matmul_group call per step (grouped lookup-table kernel + "
-                                      "reduction)" if mode == "group"
-                                      else f"one aqlm_matmul_ws call per layer, schedule {a.schedule}")
-                                     + f"; CUDA graphs of {pool_size} consecutive steps (one pass over the pool)",
-                           "parallelism": f"replicas x{world}"},
+                "config": config,
                 "roofline": roofline, "cpu_baseline": cpu, "cpu_kernel": cpu_kernel, "e2e": e2e,
                 "other_launch": other, "no_graph": direct, "context": context,
                 "per_config": per_config,
@@ -908,19 +945,31 @@ def grad_step_bytes(w, batch):
     return out
 
 
-def oracle_grad_sample_run(w, batch, seconds):
+_GRAD_HOST = {}
+
+
+def grad_host_layers(w, batch):
+    """The workload's layers and dy [batch, N] as host arrays (generated once per process)."""
+    key = (w.name, batch)
+    if key not in _GRAD_HOST:
+        host = []
+        for li, lay in enumerate(w.layers):
+            s = lay.scheme
+            host.append((synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index, layer=li),
+                         synth.make_x(batch, lay.N, seed=1, workload=w.index, layer=li)))
+        _GRAD_HOST[key] = host
+    return _GRAD_HOST[key]
+
+
+def oracle_grad_sample_run(w, batch, seconds, seed=5):
     """Times oracle.input_grad (decode to fp16 + fp64 dy . W16) on column samples of
-    every layer until about `seconds` have been spent.  Returns (flops credited, seconds,
-    columns per layer, threads)."""
+    every layer until about `seconds` have been spent (at least one layer).  Returns
+    (flops credited, seconds, columns per layer, threads)."""
     import oracle
 
-    rng = np.random.Generator(np.random.PCG64(5))
+    rng = np.random.Generator(np.random.PCG64(seed))
     flops, elapsed, cols = 0.0, 0.0, 16
-    host = []
-    for li, lay in enumerate(w.layers):
-        s = lay.scheme
-        host.append((synth.make_layer(s.M, s.B, s.g, lay.K, lay.N, seed=0, workload=w.index, layer=li),
-                     synth.make_x(batch, lay.N, seed=1, workload=w.index, layer=li)))
+    host = grad_host_layers(w, batch)
     while elapsed < 0.9 * seconds:
         for lay, (ld, dy) in zip(w.layers, host):
             s = lay.scheme
@@ -932,6 +981,24 @@ def oracle_grad_sample_run(w, batch, seconds):
             if elapsed >= 0.9 * seconds:
                 break
     return flops, elapsed, cols, oracle.max_threads()
+
+
+def grad_pool_copies(step_bytes_, l2, copies=None):
+    """Copies of the workload in the input-gradient timing pool: at least 3x L2 and at
+    least 2 (`copies` overrides)."""
+    return max(2, math.ceil(3 * l2 / step_bytes_)) if copies is None else max(1, copies)
+
+
+def grad_line_config(w, batch, world, schedule, pool, l2):
+    """The `config` object of an input-gradient line; both arms print it."""
+    sbytes = grad_step_bytes(w, batch)
+    return {"workload": w.name, "op": "input-grad", "layers": len(w.layers), "batch": batch,
+            "scheme": w.layers[0].scheme.name, "algorithmic_bytes_per_step": sbytes,
+            "flops_per_step": sum(2.0 * batch * l.N * l.K for l in w.layers),
+            "l2": f"inputs larger than L2: rotating pool of {pool} copies "
+                  f"({pool * sbytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
+            "launch": f"one aqlm_input_grad_ws call per layer, schedule {schedule}; CUDA graphs of {pool} steps",
+            "parallelism": f"replicas x{world}"}
 
 
 def run_input_grad(a):
@@ -957,7 +1024,7 @@ def run_input_grad(a):
     sflops = sum(2.0 * batch * l.N * l.K for l in w.layers)
     props = torch.cuda.get_device_properties(dev)
     l2 = getattr(props, "L2_cache_size", 0) or L2_FALLBACK
-    pool = max(2, math.ceil(3 * l2 / sbytes)) if a.pool is None else max(1, a.pool)
+    pool = grad_pool_copies(sbytes, l2, a.pool)
 
     weights, dys = [], []
     for c in range(pool):
@@ -1112,14 +1179,7 @@ def run_input_grad(a):
                 "warmup": a.warmup, "ms_per_step": ms_step, "us_per_layer": ms_step * 1e3 / len(w.layers),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
                 "data": "synthetic",
-                "config": {"workload": w.name, "op": "input-grad", "layers": len(w.layers), "batch": batch,
-                           "scheme": w.layers[0].scheme.name, "algorithmic_bytes_per_step": sbytes,
-                           "flops_per_step": sflops,
-                           "l2": f"inputs larger than L2: rotating pool of {pool} copies "
-                                 f"({pool * sbytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
-                           "launch": f"one aqlm_input_grad_ws call per layer, schedule {a.schedule}; "
-                                     f"CUDA graphs of {pool} steps",
-                           "parallelism": f"replicas x{world}"},
+                "config": grad_line_config(w, batch, world, a.schedule, pool, l2),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": len(w.layers) * steps, "clocks": clocks.summary(), "gpu": props.name}
         print(json.dumps(line), flush=True)

@@ -57,3 +57,35 @@ def test_bench_scheme_override_parses():
     import pytest
     with pytest.raises(SystemExit):
         bench.parse_scheme("3x8")
+
+
+def test_reference_arm_names_the_same_config():
+    """Both arms' lines carry line_config's object: for a given L2 size the reference
+    arm's config equals what the library's arm prints for the same arguments."""
+    for argv in ([], ["--launch", "per-layer", "--schedule", "streamk"], ["--pool", "3"],
+                 ["--workload", "llama2_7b_layer_set_2x8g8", "--batch", "4"]):
+        a = bench.parse_args(argv)
+        w = bench.select_workload(a)
+        batch = bench.workload_batch(w, a.batch)
+        ref = bench.reference_config(a, w, batch, 2)
+        pool = bench.pool_copies(bench.step_bytes(w, batch), bench.L2_FALLBACK, a.pool)
+        assert ref == bench.line_config(w, batch, 2, a.launch, a.schedule, pool, bench.L2_FALLBACK)
+        assert ref["workload"] == w.name and ref["batch"] == batch and ref["parallelism"] == "replicas x2"
+        assert f"pool of {pool} copies" in ref["l2"] and f"graphs of {pool} consecutive" in ref["launch"]
+
+
+def test_pool_rule():
+    l2 = 126 << 20
+    assert bench.pool_copies(354e6, l2) == 8            # 8 copies already exceed 3x L2
+    assert bench.pool_copies(5e6, l2) == 80            # ceil(3 L2 / 5 MB)
+    assert bench.pool_copies(20e9, l2) == 3            # capped at 60 GB
+    assert bench.pool_copies(5e6, l2, copies=3) == 3
+
+
+def test_reference_arm_names_the_same_config_for_the_input_gradient():
+    a = bench.parse_args(["--op", "input-grad", "--workload", "llama2_7b_layer_set_2x8g8", "--batch", "64"])
+    w = bench.select_workload(a)
+    ref = bench.reference_config(a, w, 64, 1)
+    pool = bench.grad_pool_copies(bench.grad_step_bytes(w, 64), bench.L2_FALLBACK, a.pool)
+    assert ref == bench.grad_line_config(w, 64, 1, a.schedule, pool, bench.L2_FALLBACK)
+    assert ref["op"] == "input-grad" and ref["flops_per_step"] == sum(2.0 * 64 * l.N * l.K for l in w.layers)
