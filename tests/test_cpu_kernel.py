@@ -177,3 +177,16 @@ def test_cpu_matmul_argument_errors(kwargs, want):
                                y.ctypes.data, 2, 8, 8, 64, 4, 1, 0) == Status.MISALIGNED
     assert lib.aqlm_cpu_matmul(None, codes.ctypes.data, cb.ctypes.data, sc.ctypes.data, None,
                                y.ctypes.data, 2, 8, 8, 64, 4, 1, 0) == Status.INVALID_ARG
+
+
+@pytest.mark.parametrize("M,B,g", SCHEMES)
+def test_cpu_matmul_degenerate_shapes(M, B, g, simd):
+    """One output row, one or two groups of K (for g = 8 a single group is the fused
+    method's odd-group tail alone), batch 1 and 9, more threads than rows or slices."""
+    for N, K, batch in ((1, g, 1), (1, g, 9), (3, 2 * g, 1), (2, g, 2)):
+        ld = synth.make_layer(M, B, g, K, N, seed=89, layer=N + K, with_bias=True)
+        x = synth.make_x(batch, K, seed=90, layer=M)
+        ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+        for nt in (1, 8):
+            close(cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g, nthreads=nt), ref,
+                  f"{M}x{B} g{g} N={N} K={K} b={batch} threads={nt} simd={simd}")
