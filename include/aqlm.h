@@ -167,7 +167,9 @@ size_t aqlm_matmul_workspace_size(int M, int B, int g, int K, int N, int batch);
  * (different streams) must not share a workspace; calls on one stream may.
  * The library may also ignore the workspace (another path, or a faster plan).
  * AQLM_SCHEDULE_STREAMK without a workspace is AQLM_ERR_INVALID_ARG; an unknown
- * schedule is AQLM_ERR_INVALID_ARG.
+ * schedule is AQLM_ERR_INVALID_ARG.  AQLM_SCHEDULE_STREAMK on another kernel family,
+ * or on a shape the stream-K schedule cannot take (including one whose workspace
+ * serves only the grouped lookup route), is AQLM_ERR_UNSUPPORTED, before any launch.
  */
 aqlm_status aqlm_matmul_ws(const void* x, const void* codes, const void* codebooks,
                            const void* scales, const void* bias, void* y,

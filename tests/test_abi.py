@@ -372,6 +372,12 @@ def test_workspace_validation_needs_no_gpu(lib):
     assert L_.aqlm_matmul_ws(*small, W, 1 << 20, None) == Status.UNSUPPORTED
     gemv = args[:6] + (1, 16, 8, 4096, 4096, 1, Path.GEMV, Schedule.STREAMK)
     assert L_.aqlm_matmul_ws(*gemv, W, 1 << 24, None) == Status.UNSUPPORTED
+    # a shape whose workspace serves only the grouped lookup route: stream-K stays
+    # unsupported there, before any CUDA call
+    routed = args[:6] + (2, 8, 8, 14336, 4096, 1, Path.AUTO, Schedule.STREAMK)
+    rneed = native.aqlm_matmul_workspace_size(2, 8, 8, 14336, 4096, 1)
+    assert rneed > 0
+    assert L_.aqlm_matmul_ws(*routed, W, rneed, None) == Status.UNSUPPORTED
     gneed = native.aqlm_input_grad_workspace_size(2, 8, 8, 4096, 14336, 1024)
     gargs = (x, x + (1 << 31), x + (1 << 31) + (1 << 28), x + (1 << 31) + (1 << 29), y, 2, 8, 8, 4096, 14336, 1024,
              Schedule.AUTO)

@@ -236,7 +236,9 @@ aqlm_status aqlm_matmul_ws(const void* x, const void* codes, const void* codeboo
                            aqlm_stream_t stream) {
   aqlm_status st = aqlm_validate(x, codes, codebooks, scales, bias, y, M, B, g, K, N, batch, path);
   if (st != AQLM_OK) return st;
-  st = check_schedule(schedule, workspace, aqlm_matmul_workspace_size(M, B, g, K, N, batch));
+  // stream-K is possible only where the tensor-core kernel has partial slots for it
+  // (the workspace may be sized for the grouped route alone)
+  st = check_schedule(schedule, workspace, aqlm::tc_pipe_partial_bytes(M, B, g, K, N, batch));
   if (st != AQLM_OK) return st;
   if (schedule == AQLM_SCHEDULE_STREAMK) {
     // a forced stream-K schedule is the tensor-core kernel's
