@@ -106,7 +106,8 @@ typedef enum {
  *   codebooks  fp16 [M, 2^B, g], read         scales     fp16 [N], read
  *   bias       fp16 [N] or NULL, read         y          fp16 [batch, N], written
  * All are caller-owned device memory (layout, alignment and ownership as in the file
- * header); y must not overlap an input.  Accumulation is fp32 (or better); y is
+ * header); y must not overlap an input (AQLM_ERR_INVALID_ARG).  Accumulation is
+ * fp32 (or better); y is
  * rounded to fp16 (RNE).  Result tolerance against the fp64 reference of the
  * decoded fp16 weights: max|y - y_ref| / max|y_ref| <= 5e-3.
  * Returns AQLM_OK after enqueueing the work on `stream`; AQLM_ERR_INVALID_ARG,

@@ -49,10 +49,37 @@ A = 1 << 20  # a 16-byte aligned fake address: validation never dereferences it
 SUPPORTED = [(m, 8, g) for m in (1, 2, 3, 4) for g in (8, 16)] + [(m, 16, g) for m in (1, 2) for g in (8, 16)]
 
 
+# disjoint 16-byte aligned fake buffers (x, codes, codebooks, scales, bias, y), 64 MiB apart
+D = tuple(A + i * (1 << 26) for i in range(6))
+
+
 @pytest.mark.parametrize("M,B,g", SUPPORTED)
 def test_supported_schemes_validate(lib, M, B, g):
-    assert native.aqlm_validate(A, A, A, A, None, A, M, B, g, 4096, 4096, 1) == Status.OK
-    assert native.aqlm_validate(A, A, A, A, A, A, M, B, g, 4096, 11008, 256) == Status.OK
+    x, codes, cb, sc, bias, y = D
+    assert native.aqlm_validate(x, codes, cb, sc, None, y, M, B, g, 4096, 4096, 1) == Status.OK
+    assert native.aqlm_validate(x, codes, cb, sc, bias, y, M, B, g, 4096, 11008, 256) == Status.OK
+
+
+def test_output_overlapping_an_input_is_rejected(lib):
+    x, codes, cb, sc, bias, y = D
+    K, N, batch = 4096, 4096, 4
+    ok = (x, codes, cb, sc, bias, y, 2, 8, 8, K, N, batch)
+    assert native.aqlm_validate(*ok) == Status.OK
+    for i, name in enumerate(("x", "codes", "codebooks", "scales", "bias")):
+        args = list(ok)
+        args[5] = ok[i] + 16  # y starts inside that input
+        assert native.aqlm_validate(*args) == Status.INVALID_ARG, name
+    # y ending exactly where x starts touches nothing
+    args = list(ok)
+    args[5] = x - batch * N * 2
+    assert native.aqlm_validate(*args) == Status.OK
+    # an absent bias overlaps nothing
+    args = list(ok)
+    args[4], args[5] = None, bias
+    assert native.aqlm_validate(*args) == Status.OK
+    with pytest.raises(native.AqlmError) as e:
+        native.aqlm_matmul(x, codes, cb, sc, None, x, 2, 8, 8, K, N, batch)  # in place: rejected before launch
+    assert e.value.status == Status.INVALID_ARG
 
 
 @pytest.mark.parametrize("args,want", [

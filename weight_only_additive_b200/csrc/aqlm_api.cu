@@ -218,6 +218,19 @@ aqlm_status aqlm_validate(const void* x, const void* codes, const void* codebook
     if (path < AQLM_PATH_AUTO || path > AQLM_PATH_TENSOR_CORE) return AQLM_ERR_INVALID_ARG;
     return AQLM_ERR_UNSUPPORTED;
   }
+  // y is written while x, the weights and the bias are read
+  const auto at = [](const void* p, size_t n) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return std::make_pair(a, a + n);
+  };
+  const auto yr = at(y, static_cast<size_t>(batch) * N * 2);
+  const size_t code_bytes = static_cast<size_t>(N) * (K / g) * M * (B <= 8 ? 1 : 2);
+  const std::pair<uintptr_t, uintptr_t> inputs[5] = {
+      at(x, static_cast<size_t>(batch) * K * 2), at(codes, code_bytes),
+      at(codebooks, static_cast<size_t>(M) * (size_t(1) << B) * g * 2), at(scales, static_cast<size_t>(N) * 2),
+      at(bias, bias ? static_cast<size_t>(N) * 2 : 0)};
+  for (const auto& r : inputs)
+    if (r.first != r.second && yr.first < r.second && r.first < yr.second) return AQLM_ERR_INVALID_ARG;
   return AQLM_OK;
 }
 
