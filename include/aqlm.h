@@ -191,7 +191,8 @@ aqlm_status aqlm_matmul_ws(const void* x, const void* codes, const void* codeboo
  * starting from C_0 itself, then one fp32 multiply by the channel scale and
  * one round-to-nearest-even to fp16.  Bit-exact by definition.
  *   codes, codebooks, scales  as for aqlm_matmul, read
- *   W_out                     fp16 [N, K], caller-owned device memory, written
+ *   W_out                     fp16 [N, K], caller-owned device memory, written;
+ *                             must not overlap an input (AQLM_ERR_INVALID_ARG)
  * Errors as for aqlm_matmul (no bias, no batch); returns after enqueueing.
  */
 aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void* scales,

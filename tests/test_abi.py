@@ -80,6 +80,11 @@ def test_output_overlapping_an_input_is_rejected(lib):
     with pytest.raises(native.AqlmError) as e:
         native.aqlm_matmul(x, codes, cb, sc, None, x, 2, 8, 8, K, N, batch)  # in place: rejected before launch
     assert e.value.status == Status.INVALID_ARG
+    # the dequantised weight must not land on the codes, codebooks or scales either
+    for target in (codes + 16, cb, sc - 16):
+        with pytest.raises(native.AqlmError) as e:
+            native.aqlm_dequantize(codes, cb, sc, target, 2, 8, 8, K, N)
+        assert e.value.status == Status.INVALID_ARG
 
 
 @pytest.mark.parametrize("args,want", [

@@ -597,6 +597,15 @@ aqlm_status aqlm_dequantize(const void* codes, const void* codebooks, const void
   if (st != AQLM_OK) return st;
   if (!aligned16(codes) || !aligned16(codebooks) || !aligned16(scales) || !aligned16(W_out))
     return AQLM_ERR_MISALIGNED;
+  // W_out is written while the codes, codebooks and scales are read
+  const uintptr_t w0 = reinterpret_cast<uintptr_t>(W_out), w1 = w0 + static_cast<size_t>(N) * K * 2;
+  const size_t code_bytes = static_cast<size_t>(N) * (K / g) * M * (B <= 8 ? 1 : 2);
+  const std::pair<const void*, size_t> inputs[3] = {
+      {codes, code_bytes}, {codebooks, static_cast<size_t>(M) * (size_t(1) << B) * g * 2}, {scales, size_t(N) * 2}};
+  for (const auto& in : inputs) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(in.first);
+    if (w0 < a + in.second && a < w1) return AQLM_ERR_INVALID_ARG;
+  }
   return from_cuda(aqlm::launch_dequantize(codes, codebooks, scales, W_out, M, B, g, K, N,
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
