@@ -301,6 +301,23 @@ def test_group_host_rejects_missing_host_buffers_without_a_gpu(lib):
     assert L_.aqlm_matmul_group_host(probs, 1, None, A, A, 1 << 20, None) == Status.INVALID_ARG
     assert L_.aqlm_matmul_group_host(probs, 1, A, None, A, 1 << 20, None) == Status.INVALID_ARG
     assert L_.aqlm_matmul_group_host(probs, 0, None, None, None, 0, None) == Status.OK
+    # every check of the group call comes before the first host-to-device copy: a
+    # missing, short or misaligned workspace is reported as such, not as a failed copy
+    need = native.aqlm_group_workspace_size(native.problem_array([_prob(1 << 32)]), 1)
+    hx, hy = 1 << 45, 1 << 46
+    assert L_.aqlm_matmul_group_host(probs, 1, hx, hy, None, 0, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_group_host(probs, 1, hx, hy, 1 << 40, need - 256, None) == Status.INVALID_ARG
+    assert L_.aqlm_matmul_group_host(probs, 1, hx, hy, (1 << 40) + 16, need, None) == Status.MISALIGNED
+
+
+def test_group_workspace_must_not_overlap_a_problem(lib):
+    L_ = native.lib()
+    P = [_prob(1 << 32), _prob(1 << 33, K=11008, N=200)]
+    arr = native.problem_array(P)
+    need = native.aqlm_group_workspace_size(arr, 2)
+    for i, k in ((0, 0), (0, 5), (1, 1), (1, 3)):  # x / y of problem 0, codes / scales of problem 1
+        assert L_.aqlm_matmul_group(arr, 2, P[i][k], need, None) == Status.INVALID_ARG, (i, k)
+        assert L_.aqlm_matmul_group_host(arr, 2, 1 << 45, 1 << 46, P[i][k], need, None) == Status.INVALID_ARG
 
 
 @pytest.mark.parametrize("M,g,K", [(1, 8, 4096), (3, 8, 1024), (4, 16, 4096), (1, 16, 4096)])

@@ -449,21 +449,11 @@ size_t group_need(const aqlm_problem* problems, int count) {
   return grouped > 0 ? AQLM_WORKSPACE_COUNTER_BYTES + round256(grouped) : 0;
 }
 
-}  // namespace
-
-size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count) {
-  if (!problems || count <= 0) return 0;
-  for (int i = 0; i < count; ++i) {
-    const aqlm_problem& q = problems[i];
-    if (validate_shape(q.M, q.B, q.g, q.K, q.N, q.batch) != AQLM_OK) return 0;
-  }
-  return group_need(problems, count);
-}
-
-aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* workspace,
-                              size_t workspace_bytes, aqlm_stream_t stream) {
-  if (count == 0) return AQLM_OK;
-  if (count < 0 || !problems) return AQLM_ERR_INVALID_ARG;
+// The argument checks of a group call, made before any copy or launch: every problem
+// valid, no output overlapping another problem's buffers, and (when anything is
+// grouped) a workspace of the needed size and alignment that overlaps none of them.
+aqlm_status validate_group(const aqlm_problem* problems, int count, const void* workspace,
+                           size_t workspace_bytes, size_t* need_out) {
   for (int i = 0; i < count; ++i) {
     const aqlm_problem& q = problems[i];
     const aqlm_status st = aqlm_validate(q.x, q.codes, q.codebooks, q.scales, q.bias, q.y, q.M, q.B, q.g, q.K,
@@ -486,9 +476,22 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
   if (need > 0) {
     if (!workspace || workspace_bytes < need) return AQLM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return AQLM_ERR_MISALIGNED;
+    const ByteRange wr = range_of(workspace, need);
+    for (int i = 0; i < count; ++i) {
+      ByteRange ri[6];
+      problem_ranges(problems[i], ri);
+      for (int k = 0; k < 6; ++k)
+        if (overlaps(wr, ri[k])) return AQLM_ERR_INVALID_ARG;
+    }
   }
+  *need_out = need;
+  return AQLM_OK;
+}
+
+// Launches a validated group (`need` from validate_group): runs of up to
+// kMaxGroupLayers grouped problems in the grouped kernel, the others one by one.
+aqlm_status run_group(const aqlm_problem* problems, int count, void* workspace, size_t need, cudaStream_t s) {
   uint8_t* const ws = static_cast<uint8_t*>(workspace);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   aqlm::Problem run[aqlm::kMaxGroupLayers];
   int n_run = 0;
   uint32_t* status = nullptr;
@@ -516,16 +519,35 @@ aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* wor
   return AQLM_OK;
 }
 
+}  // namespace
+
+size_t aqlm_group_workspace_size(const aqlm_problem* problems, int count) {
+  if (!problems || count <= 0) return 0;
+  for (int i = 0; i < count; ++i) {
+    const aqlm_problem& q = problems[i];
+    if (validate_shape(q.M, q.B, q.g, q.K, q.N, q.batch) != AQLM_OK) return 0;
+  }
+  return group_need(problems, count);
+}
+
+aqlm_status aqlm_matmul_group(const aqlm_problem* problems, int count, void* workspace,
+                              size_t workspace_bytes, aqlm_stream_t stream) {
+  if (count == 0) return AQLM_OK;
+  if (count < 0 || !problems) return AQLM_ERR_INVALID_ARG;
+  size_t need = 0;
+  const aqlm_status vst = validate_group(problems, count, workspace, workspace_bytes, &need);
+  if (vst != AQLM_OK) return vst;
+  return run_group(problems, count, workspace, need, reinterpret_cast<cudaStream_t>(stream));
+}
+
 aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, const void* x_host, void* y_host,
                                    void* workspace, size_t workspace_bytes, aqlm_stream_t stream) {
   if (count == 0) return AQLM_OK;
   if (count < 0 || !problems || !x_host || !y_host) return AQLM_ERR_INVALID_ARG;
-  for (int i = 0; i < count; ++i) {
-    const aqlm_problem& q = problems[i];
-    const aqlm_status st = aqlm_validate(q.x, q.codes, q.codebooks, q.scales, q.bias, q.y, q.M, q.B, q.g, q.K,
-                                         q.N, q.batch, AQLM_PATH_AUTO);
-    if (st != AQLM_OK) return st;
-  }
+  // every argument check of the group call before the first copy
+  size_t need = 0;
+  const aqlm_status vst = validate_group(problems, count, workspace, workspace_bytes, &need);
+  if (vst != AQLM_OK) return vst;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const auto xbytes = [&](int i) { return static_cast<size_t>(problems[i].batch) * problems[i].K * 2; };
   const auto ybytes = [&](int i) { return static_cast<size_t>(problems[i].batch) * problems[i].N * 2; };
@@ -554,7 +576,7 @@ aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, cons
   };
   aqlm_status st = copy_runs(true);
   if (st != AQLM_OK) return st;
-  st = aqlm_matmul_group(problems, count, workspace, workspace_bytes, stream);
+  st = run_group(problems, count, workspace, need, s);
   if (st != AQLM_OK) return st;
   return copy_runs(false);
 }
