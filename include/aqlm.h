@@ -276,7 +276,8 @@ typedef struct {
  * when that size is 0).  Layout: AQLM_WORKSPACE_COUNTER_BYTES left untouched (the
  * counters of aqlm_matmul_ws sit there, so one buffer may serve both kinds of call on
  * a stream), then the fp32 partial sums between the two kernels of a pair, which
- * need no initialisation.  Calls that may run concurrently (different streams) must
+ * need no initialisation.  It must not overlap any problem's buffers
+ * (AQLM_ERR_INVALID_ARG).  Calls that may run concurrently (different streams) must
  * not share a workspace.
  * count == 0 is a no-op; count < 0 or problems == NULL (with count > 0) is
  * AQLM_ERR_INVALID_ARG.  Every problem is validated as aqlm_validate does before
@@ -321,7 +322,8 @@ aqlm_status aqlm_matmul_group_static(const aqlm_problem* problems, int count, aq
  * x_host may be modified, once `stream` has passed the call (synchronise before).  The pages have
  * no counterpart: this is the token-generation step of a serving loop, from host
  * activations to host outputs.  Validation, workspace and errors as for
- * aqlm_matmul_group; NULL x_host or y_host (with count > 0) is AQLM_ERR_INVALID_ARG.
+ * aqlm_matmul_group, all checked before the first copy (a rejected call changes no
+ * device buffer); NULL x_host or y_host (with count > 0) is AQLM_ERR_INVALID_ARG.
  */
 aqlm_status aqlm_matmul_group_host(const aqlm_problem* problems, int count, const void* x_host, void* y_host,
                                    void* workspace, size_t workspace_bytes, aqlm_stream_t stream);
