@@ -74,6 +74,20 @@ class AqlmWeights:
     B: int
     g: int
 
+    def __post_init__(self):
+        # the kernels read exactly the sizes (M, B, g, K, N) imply: check them once here
+        code_dtypes = (torch.uint8,) if self.B <= 8 else (torch.int16, torch.uint16)
+        if self.codes.dtype not in code_dtypes:
+            raise TypeError(f"codes must be {' or '.join(map(str, code_dtypes))} for B={self.B}, "
+                            f"got {self.codes.dtype}")
+        if self.codes.dim() != 3 or self.codes.shape[2] != self.M or not self.codes.is_contiguous():
+            raise ValueError(f"codes must be a contiguous [N, K/g, {self.M}] tensor, got shape {tuple(self.codes.shape)}")
+        dev = self.codes.device
+        _check_tensor(self.codebooks, "codebooks", torch.float16, dev, (self.M, 1 << self.B, self.g))
+        _check_tensor(self.scales, "scales", torch.float16, dev, (self.N,))
+        if self.bias is not None:
+            _check_tensor(self.bias, "bias", torch.float16, dev, (self.N,))
+
     @property
     def N(self) -> int:
         return self.codes.shape[0]
@@ -94,13 +108,16 @@ class AqlmWeights:
                    M=layer.M, B=layer.B, g=layer.g)
 
 
-def _check_tensor(t: torch.Tensor, name: str, dtype, device):
+def _check_tensor(t: torch.Tensor, name: str, dtype, device, shape=None):
     if t.device != device:
         raise ValueError(f"{name} must be on {device}, got {t.device}")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        # the kernels write exactly this many values: a smaller buffer would be overrun
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
 def matmul(x: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = None,
@@ -115,12 +132,14 @@ def matmul(x: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = None,
     if dev.type != "cuda":
         raise ValueError("AQLM weights must live on a CUDA device")
     _check_tensor(x, "x", torch.float16, dev)
+    if x.dim() != 2:
+        raise ValueError(f"x must be [batch, K], got shape {tuple(x.shape)}")
     batch, K = x.shape
     if K != w.K:
         raise ValueError(f"x has K={K}, weights have K={w.K}")
     if out is None:
         out = torch.empty((batch, w.N), dtype=torch.float16, device=dev)
-    _check_tensor(out, "out", torch.float16, dev)
+    _check_tensor(out, "out", torch.float16, dev, (batch, w.N))
     ws, ws_bytes = _resolve_workspace(workspace, native.aqlm_matmul_workspace_size(w.M, w.B, w.g, K, w.N, batch),
                                       dev, stream)
     native.aqlm_matmul_ws(x.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(),
@@ -139,12 +158,14 @@ def input_grad(dy: torch.Tensor, w: AqlmWeights, out: Optional[torch.Tensor] = N
     if dev.type != "cuda":
         raise ValueError("AQLM weights must live on a CUDA device")
     _check_tensor(dy, "dy", torch.float16, dev)
+    if dy.dim() != 2:
+        raise ValueError(f"dy must be [batch, N], got shape {tuple(dy.shape)}")
     batch, N = dy.shape
     if N != w.N:
         raise ValueError(f"dy has N={N}, weights have N={w.N}")
     if out is None:
         out = torch.empty((batch, w.K), dtype=torch.float16, device=dev)
-    _check_tensor(out, "out", torch.float16, dev)
+    _check_tensor(out, "out", torch.float16, dev, (batch, w.K))
     ws, ws_bytes = _resolve_workspace(
         workspace, native.aqlm_input_grad_workspace_size(w.M, w.B, w.g, w.K, N, batch), dev, stream)
     native.aqlm_input_grad_ws(dy.data_ptr(), w.codes.data_ptr(), w.codebooks.data_ptr(), w.scales.data_ptr(),
@@ -159,7 +180,7 @@ def dequantize(w: AqlmWeights, out: Optional[torch.Tensor] = None,
     dev = w.codes.device
     if out is None:
         out = torch.empty((w.N, w.K), dtype=torch.float16, device=dev)
-    _check_tensor(out, "out", torch.float16, dev)
+    _check_tensor(out, "out", torch.float16, dev, (w.N, w.K))
     native.aqlm_dequantize(w.codes.data_ptr(), w.codebooks.data_ptr(), w.scales.data_ptr(),
                            out.data_ptr(), w.M, w.B, w.g, w.K, w.N, _stream_handle(stream, dev))
     return out
