@@ -190,3 +190,18 @@ def test_cpu_matmul_degenerate_shapes(M, B, g, simd):
         for nt in (1, 8):
             close(cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g, nthreads=nt), ref,
                   f"{M}x{B} g{g} N={N} K={K} b={batch} threads={nt} simd={simd}")
+
+
+def test_binding_rejects_mis_sized_bias_and_output():
+    """The kernel reads N bias values and writes batch x N outputs: the binding checks
+    both sizes before the call."""
+    ld = synth.make_layer(2, 8, 8, 64, 16, seed=91, with_bias=True)
+    x = synth.make_x(2, 64, seed=91)
+    with pytest.raises(ValueError):
+        cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias[:8].copy(), 2, 8, 8)
+    with pytest.raises(ValueError):
+        cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, 2, 8, 8, out=np.empty((1, 16), np.float16))
+    with pytest.raises(ValueError):
+        cpu.matmul(x[0], ld.codes, ld.codebooks, ld.scales, ld.bias, 2, 8, 8)
+    out = np.empty((2, 16), np.float16)
+    assert cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, 2, 8, 8, out=out) is out

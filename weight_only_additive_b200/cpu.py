@@ -82,11 +82,17 @@ def matmul(x, codes, codebooks, scales, bias, M: int, B: int, g: int, nthreads: 
     cb = _arr(codebooks, np.float16)
     sc = _arr(scales, np.float16)
     bi = _arr(bias, np.float16) if bias is not None else None
+    if x.ndim != 2 or codes.ndim != 3:
+        raise ValueError("expected x [batch, K] and codes [N, K/g, M]")
     batch, K = x.shape
     N = codes.shape[0]
     if codes.shape != (N, K // g, M) or cb.shape != (M, 1 << B, g) or sc.shape != (N,):
         raise ValueError("expected codes [N, K/g, M], codebooks [M, 2^B, g], scales [N]")
+    if bi is not None and bi.shape != (N,):
+        raise ValueError(f"expected bias [N] = [{N}], got {bi.shape}")
     y = np.empty((batch, N), np.float16) if out is None else _arr(out, np.float16)
+    if y.shape != (batch, N):  # the kernel writes batch x N values
+        raise ValueError(f"expected out [batch, N] = [{batch}, {N}], got {y.shape}")
     st = lib().aqlm_cpu_matmul(x.ctypes.data, codes.ctypes.data, cb.ctypes.data, sc.ctypes.data,
                                bi.ctypes.data if bi is not None else None, y.ctypes.data,
                                M, B, g, K, N, batch, nthreads)
