@@ -205,3 +205,32 @@ def test_binding_rejects_mis_sized_bias_and_output():
         cpu.matmul(x[0], ld.codes, ld.codebooks, ld.scales, ld.bias, 2, 8, 8)
     out = np.empty((2, 16), np.float16)
     assert cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, 2, 8, 8, out=out) is out
+
+
+try:
+    import hypothesis.strategies as hst
+    from hypothesis import HealthCheck, given, settings
+except ImportError:  # pragma: no cover
+    hst = None
+
+
+if hst is not None:
+    @settings(max_examples=300, deadline=None, derandomize=True, suppress_health_check=list(HealthCheck))
+    @given(scheme=hst.sampled_from(SCHEMES), N=hst.integers(1, 300), G=hst.integers(1, 40),
+           batch=hst.integers(1, 20), nt=hst.integers(1, 8), level=hst.integers(0, 2),
+           bias=hst.booleans(), seed=hst.integers(0, 1000))
+    def test_cpu_matmul_random_shapes(scheme, N, G, batch, nt, level, bias, seed):
+        """Random shapes against the oracle at a random SIMD level (capped to what the
+        CPU has): partial slices, groups that straddle them, batch chunk remainders."""
+        M, B, g = scheme
+        K = G * g
+        ld = synth.make_layer(M, B, g, K, N, seed=seed, layer=N, with_bias=bias)
+        x = synth.make_x(batch, K, seed=seed + 1, layer=G)
+        ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
+        prev = cpu.set_max_simd_level(level)
+        try:
+            y = cpu.matmul(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g, nthreads=nt)
+        finally:
+            cpu.set_max_simd_level(prev)
+        if np.abs(ref).max() > 0:
+            close(y, ref, f"{M}x{B} g{g} N={N} K={K} b={batch} threads={nt} level={level}")
