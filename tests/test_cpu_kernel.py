@@ -221,9 +221,17 @@ if hst is not None:
            bias=hst.booleans(), seed=hst.integers(0, 1000))
     def test_cpu_matmul_random_shapes(scheme, N, G, batch, nt, level, bias, seed):
         """Random shapes against the oracle at a random SIMD level (capped to what the
-        CPU has): partial slices, groups that straddle them, batch chunk remainders."""
+        CPU has): partial slices, groups that straddle them, batch chunk remainders.
+
+        At least 64 outputs per case: the bar is relative to the layer's largest output,
+        and with a handful of outputs that maximum can cancel to near zero, where the
+        accepted difference between weights decoded in fp32 (scale on the accumulator)
+        and the reference's fp16-rounded W, about 2^-11 of sum |x w| / sqrt(K), is no
+        longer small beside it (N = 1 cases with fixed seeds are in
+        test_cpu_matmul_degenerate_shapes)."""
         M, B, g = scheme
         K = G * g
+        N = max(N, -(-64 // batch))
         ld = synth.make_layer(M, B, g, K, N, seed=seed, layer=N, with_bias=bias)
         x = synth.make_x(batch, K, seed=seed + 1, layer=G)
         ref = oracle.linear(x, ld.codes, ld.codebooks, ld.scales, ld.bias, M, B, g)
