@@ -545,7 +545,23 @@ def roofline_record(w, batch, step_s, peaks, sms, sm_mhz):
     rec["peak_source"] = {"hbm": f"{src} hbm_gbs", "tensor": f"{src} bf16_tflops (burst)",
                           "l1tex_gather": f"{GATHERS_PER_SM_CLOCK:g} request per SM per clock x {sms} SMs x "
                                           f"{sm_mhz:.0f} MHz"}[bound]
+    l2 = l2_gather_traffic(w, batch)
+    if l2 is not None:
+        rec["l2_gather_sectors"] = l2
     return rec
+
+
+def l2_gather_traffic(w, batch):
+    """The L2 sector traffic of the B = 16 schemes' codeword gathers, next to the HBM
+    bytes: one 32-byte L2 sector per codeword piece, once per decode of a weight tile
+    (one decode per 256-wide batch tile).  None for a workload without B = 16 layers."""
+    sectors = sum(l.N * l.G * l.scheme.M * -(-batch // 256) for l in w.layers if l.scheme.B == 16)
+    if not sectors:
+        return None
+    return {"sectors": sectors, "bytes": 32 * sectors, "per_hbm_byte": 32 * sectors / step_bytes(w, batch),
+            "basis": "one 32-byte sector per codeword gather; ncu counted 2,337,475 L2 sectors read by the SMs "
+                     "for the 2,097,152 gathers plus 5.3 MB of codes of 4096x4096 1x16 g8 at batch 1 "
+                     "(profiles/tc_pipe_1x16g8_4096x4096_b1.md)"}
 
 
 class Bench:

@@ -89,3 +89,21 @@ def test_reference_arm_names_the_same_config_for_the_input_gradient():
     pool = bench.grad_pool_copies(bench.grad_step_bytes(w, 64), bench.L2_FALLBACK, a.pool)
     assert ref == bench.grad_line_config(w, 64, 1, a.schedule, pool, bench.L2_FALLBACK)
     assert ref["op"] == "input-grad" and ref["flops_per_step"] == sum(2.0 * 64 * l.N * l.K for l in w.layers)
+
+
+def test_roofline_record_names_the_bound_and_the_gather_traffic():
+    from weight_only_additive_b200 import workloads
+    peaks = {"hbm_gbs": 6451.2, "tc_tflops": 1650.0, "source": "measured"}
+    w = workloads.get("single_4096x4096_1x16g8")
+    rec = bench.roofline_record(w, 1, 14.6e-6, peaks, 148, 1965.0)
+    assert rec["bound"] == "l1tex_gather" and set(rec["roofs"]) >= {"hbm", "l1tex_gather"}
+    gathers = 4096 * 512  # one codeword per 8 weights of 4096 x 4096
+    assert rec["roofs"]["l1tex_gather"]["achieved"] == pytest.approx(gathers / 1e9 / 14.6e-6)
+    l2 = rec["l2_gather_sectors"]
+    assert l2["sectors"] == gathers and l2["bytes"] == 32 * gathers
+    assert l2["per_hbm_byte"] == pytest.approx(32 * gathers / bench.step_bytes(w, 1))
+    # a 2x8 workload: HBM-bound at batch 1, no gathers from L2
+    w2 = workloads.get("llama2_7b_layer_set_2x8g8")
+    rec2 = bench.roofline_record(w2, 1, 18e-6, peaks, 148, 1965.0)
+    assert rec2["bound"] == "hbm" and "l2_gather_sectors" not in rec2
+    assert rec2["frac"] == pytest.approx(bench.step_bytes(w2, 1) / 18e-6 / 1e9 / 6451.2)
