@@ -166,8 +166,6 @@ struct GradScheme {
   static constexpr int kBoxBytes = kTileCodeBytes % 16 == 0 ? kTileCodeBytes : (kTileCodeBytes + 8 + 15) / 16 * 16;
   static constexpr int kStagesPerTile = 1;
   static constexpr int kStageCodeBytes = kTileCodeBytes;   // one code tile per stage
-  static constexpr int kTileRowBytes = kBoxBytes;
-  static constexpr bool kSwizzle64 = false;
   static constexpr uint32_t kCodeTileBytes = static_cast<uint32_t>(kStageK * kBoxBytes);
   static constexpr bool kSmemCb = B == 8;
   static constexpr bool kATmemOk = false;  // the MN-major A stage stays in shared memory
