@@ -107,3 +107,42 @@ def test_roofline_record_names_the_bound_and_the_gather_traffic():
     rec2 = bench.roofline_record(w2, 1, 18e-6, peaks, 148, 1965.0)
     assert rec2["bound"] == "hbm" and "l2_gather_sectors" not in rec2
     assert rec2["frac"] == pytest.approx(bench.step_bytes(w2, 1) / 18e-6 / 1e9 / 6451.2)
+
+
+def test_reference_arm_prints_one_complete_line(monkeypatch, capsys):
+    """`bench.py --impl reference` end to end on the CPU, with the oracle's timing
+    replaced by fixed numbers: one JSON line with the contract's keys, its config
+    equal to the library arm's for the same arguments."""
+    import json
+
+    calls = []
+
+    def fake_sample(w, batch, seconds, copy=0, nthreads=0):
+        calls.append(seconds)
+        return 2e6, 0.5, 7, 4          # bytes credited, seconds, rows per layer, threads
+
+    def fake_grad(w, batch, seconds, seed=5):
+        calls.append(seconds)
+        return 3e9, 0.25, 16, 4        # flops credited, seconds, columns per layer, threads
+
+    monkeypatch.setattr(bench, "oracle_sample_run", fake_sample)
+    monkeypatch.setattr(bench, "oracle_grad_sample_run", fake_grad)
+    for argv, unit, value in ((["--impl", "reference", "--steps", "4", "--warmup", "3"], "GB/s", 2e6 / 0.5 / 1e9),
+                              (["--impl", "reference", "--op", "input-grad", "--workload",
+                                "llama2_7b_layer_set_2x8g8", "--steps", "4", "--warmup", "3"],
+                               "TFLOP/s", 3e9 / 0.25 / 1e12)):
+        calls.clear()
+        assert bench.main(argv) == 0
+        line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+        assert len(calls) == 7                                   # warm-up + timed steps
+        assert line["impl"] == "reference" and line["unit"] == unit and line["steps"] == 4
+        assert line["value"] == pytest.approx(value) and line["e2e"]["value"] == line["value"]
+        assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+        assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 4
+        a = bench.parse_args(argv)
+        w = bench.select_workload(a)
+        batch = line["config"]["batch"]
+        assert line["config"] == bench.reference_config(a, w, batch, 1)
+        for key in ("metric", "n_gpus", "warmup", "ms_per_step", "higher_is_better", "scaling", "vs_baseline",
+                    "dtype", "data"):
+            assert key in line, key
