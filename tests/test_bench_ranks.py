@@ -146,3 +146,18 @@ def test_reference_arm_prints_one_complete_line(monkeypatch, capsys):
         for key in ("metric", "n_gpus", "warmup", "ms_per_step", "higher_is_better", "scaling", "vs_baseline",
                     "dtype", "data"):
             assert key in line, key
+
+
+def test_cpu_kernel_leg_reports_its_method():
+    """The `cpu_kernel` record of the library's arm, on a short budget: positive
+    throughput over whole layers, and the method the CPU library runs at its level."""
+    from weight_only_additive_b200 import cpu, workloads
+    for name, batch in (("single_4096x4096_1x16g8", 1), ("llama2_7b_layer_set_2x8g8", 1)):
+        w = workloads.BY_NAME[name]
+        rec = bench.cpu_kernel_run(w, batch, 0.2)
+        assert rec["value"] > 0 and rec["unit"] == "GB/s" and rec["simd"] == cpu.SIMD_NAMES[cpu.simd_level()]
+        level, B = cpu.simd_level(), w.layers[0].scheme.B
+        if B == 8:
+            assert "lookup tables" in rec["sample"]
+        else:
+            assert ("fused decode" if level == 2 else "decode to fp32") in rec["sample"]
